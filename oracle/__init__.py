@@ -1,0 +1,192 @@
+"""CPU oracle for the fused non-GEMM layer ops -- TEST INFRASTRUCTURE.
+
+Thin numpy/ctypes wrapper over ``frt_oracle.cpp`` (plain fp64 C++).  Only the
+tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
+import this package; the CUDA library never does, and the two share no code.
+
+16-bit tensors are passed as ``np.uint16`` bit patterns; ``dt`` is ``"f16"``
+or ``"bf16"``.  Every function returns freshly allocated numpy arrays.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_DT = {"f16": 0, "bf16": 1}
+_QM = {"static": 0, "block128": 1}
+_ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
+
+_lib = None
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        c = ctypes
+        L.oracle_f16_decode.argtypes = [c.c_uint16]
+        L.oracle_f16_decode.restype = c.c_double
+        L.oracle_bf16_decode.argtypes = [c.c_uint16]
+        L.oracle_bf16_decode.restype = c.c_double
+        L.oracle_f16_round.argtypes = [c.c_double, c.c_double]
+        L.oracle_f16_round.restype = c.c_uint16
+        L.oracle_bf16_round.argtypes = [c.c_double, c.c_double]
+        L.oracle_bf16_round.restype = c.c_uint16
+        L.oracle_e4m3_encode.argtypes = [c.c_double]
+        L.oracle_e4m3_encode.restype = c.c_uint8
+        L.oracle_e4m3_decode.argtypes = [c.c_uint8]
+        L.oracle_e4m3_decode.restype = c.c_double
+        L.oracle_act.argtypes = [c.c_int, c.c_double]
+        L.oracle_act.restype = c.c_double
+        L.oracle_add16.argtypes = [c.c_uint16, c.c_uint16, c.c_int]
+        L.oracle_add16.restype = c.c_uint16
+        L.oracle_quant_static.argtypes = [c.c_void_p, c.c_int64, c.c_double, c.c_void_p]
+        L.oracle_quant_static.restype = None
+        L.oracle_quant_block128.argtypes = [c.c_void_p, c.c_int64, c.c_void_p, c.c_void_p]
+        L.oracle_quant_block128.restype = None
+        L.oracle_rmsnorm.argtypes = [c.c_void_p, c.c_int64, c.c_void_p, c.c_double, c.c_void_p]
+        L.oracle_rmsnorm.restype = None
+        L.oracle_rope_rotate_half.argtypes = [c.c_void_p, c.c_int, c.c_void_p, c.c_void_p]
+        L.oracle_rope_rotate_half.restype = None
+        L.oracle_residual_rmsnorm_fp8.argtypes = [c.c_void_p] * 5 + [c.c_double, c.c_void_p, c.c_void_p,
+                                                                     c.c_int64, c.c_int64, c.c_double,
+                                                                     c.c_int, c.c_int]
+        L.oracle_residual_rmsnorm_fp8.restype = c.c_int
+        L.oracle_qkv_norm_rope_kvcache.argtypes = [c.c_void_p] * 11 + [c.c_int64] * 6 + [c.c_double, c.c_int]
+        L.oracle_qkv_norm_rope_kvcache.restype = c.c_int
+        L.oracle_gate_act_fp8.argtypes = [c.c_void_p, c.c_void_p, c.c_double, c.c_void_p, c.c_void_p,
+                                          c.c_int64, c.c_int64, c.c_int, c.c_int, c.c_int]
+        L.oracle_gate_act_fp8.restype = c.c_int
+        _lib = L
+    return _lib
+
+
+# ----------------------------------------------------------------- scalars --
+def decode16(bits, dt):
+    f = lib().oracle_bf16_decode if dt == "bf16" else lib().oracle_f16_decode
+    b = np.asarray(bits, dtype=np.uint16)
+    return np.array([f(int(v)) for v in b.ravel()], dtype=np.float64).reshape(b.shape)
+
+
+def round16(hi, lo, dt):
+    f = lib().oracle_bf16_round if dt == "bf16" else lib().oracle_f16_round
+    return int(f(float(hi), float(lo)))
+
+
+def add16(x_bits, r_bits, dt):
+    return int(lib().oracle_add16(int(x_bits), int(r_bits), _DT[dt]))
+
+
+def e4m3_encode(v):
+    return int(lib().oracle_e4m3_encode(float(v)))
+
+
+def e4m3_decode(c):
+    return float(lib().oracle_e4m3_decode(int(c)))
+
+
+def act(name, g):
+    return float(lib().oracle_act(_ACT[name], float(g)))
+
+
+# ------------------------------------------------------------- components --
+def quant_static(y, s):
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    q = np.empty(y.size, dtype=np.uint8)
+    lib().oracle_quant_static(_p(y), y.size, float(s), _p(q))
+    return q.reshape(y.shape)
+
+
+def quant_block128(y):
+    y = np.ascontiguousarray(y, dtype=np.float64).ravel()
+    q = np.empty(y.size, dtype=np.uint8)
+    sc = np.empty((y.size + 127) // 128, dtype=np.float64)
+    lib().oracle_quant_block128(_p(y), y.size, _p(q), _p(sc))
+    return q, sc
+
+
+def rmsnorm(h, w, eps):
+    h = np.ascontiguousarray(h, dtype=np.float64)
+    w = None if w is None else np.ascontiguousarray(w, dtype=np.float64)
+    y = np.empty_like(h)
+    lib().oracle_rmsnorm(_p(h), h.size, _p(w), float(eps), _p(y))
+    return y
+
+
+def rope_rotate_half(v, c, s):
+    v = np.array(v, dtype=np.float64, copy=True)
+    c = np.ascontiguousarray(c, dtype=np.float32)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    lib().oracle_rope_rotate_half(_p(v), v.size, _p(c), _p(s))
+    return v
+
+
+# -------------------------------------------------------------------- ops --
+def residual_rmsnorm_fp8(x, residual_in, weight, eps, dt, quant, static_scale=None, want_y=False):
+    """Op (a). x, residual_in: uint16 [M, D]; weight: uint16 [D] or None."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    r = np.ascontiguousarray(residual_in, dtype=np.uint16)
+    M, D = x.shape
+    w = None if weight is None else np.ascontiguousarray(weight, dtype=np.uint16)
+    r_out = np.empty_like(r)
+    q = np.empty((M, D), dtype=np.uint8)
+    nb = (D + 127) // 128
+    sc = np.empty((M, nb), dtype=np.float64) if quant == "block128" else None
+    y = np.empty((M, D), dtype=np.float64) if want_y else None
+    s = float(static_scale) if quant == "static" else 0.0
+    rc = lib().oracle_residual_rmsnorm_fp8(_p(x), _p(r), _p(r_out), _p(w), _p(q), s, _p(sc), _p(y),
+                                           M, D, float(eps), _DT[dt], _QM[quant])
+    if rc != 0:
+        raise ValueError("oracle_residual_rmsnorm_fp8: bad argument")
+    return {"residual_out": r_out, "out_fp8": q, "block_scales": sc, "y": y}
+
+
+def qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, Hq, Hkv, hd, capacity,
+                          eps, dt, slots=None, k_cache=None, v_cache=None):
+    """Op (b). Returns q_out (fp64 [M,Hq,hd]), k_cache (fp64 [cap,Hkv,hd]),
+    v_cache (uint16 [cap,Hkv,hd]) and the status word.  Cache rows that are
+    not written keep their initial contents (NaN / the given arrays)."""
+    qkv = np.ascontiguousarray(qkv, dtype=np.uint16)
+    M = qkv.shape[0]
+    cos_tab = np.ascontiguousarray(cos_tab, dtype=np.float32)
+    sin_tab = np.ascontiguousarray(sin_tab, dtype=np.float32)
+    max_pos = cos_tab.shape[0]
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    sl = None if slots is None else np.ascontiguousarray(slots, dtype=np.int64)
+    qw = None if q_norm_w is None else np.ascontiguousarray(q_norm_w, dtype=np.uint16)
+    kw = None if k_norm_w is None else np.ascontiguousarray(k_norm_w, dtype=np.uint16)
+    q_out = np.full((M, Hq, hd), np.nan, dtype=np.float64)
+    kc = (np.full((capacity, Hkv, hd), np.nan, dtype=np.float64) if k_cache is None
+          else np.array(k_cache, dtype=np.float64, copy=True))
+    vc = (np.zeros((capacity, Hkv, hd), dtype=np.uint16) if v_cache is None
+          else np.array(v_cache, dtype=np.uint16, copy=True))
+    status = np.zeros(1, dtype=np.int32)
+    rc = lib().oracle_qkv_norm_rope_kvcache(_p(qkv), _p(qw), _p(kw), _p(cos_tab), _p(sin_tab), _p(pos), _p(sl),
+                                            _p(q_out), _p(kc), _p(vc), _p(status), M, Hq, Hkv, hd, max_pos,
+                                            capacity, float(eps), _DT[dt])
+    if rc != 0:
+        raise ValueError("oracle_qkv_norm_rope_kvcache: bad argument")
+    return {"q_out": q_out, "k_cache": kc, "v_cache": vc, "status": int(status[0])}
+
+
+def gate_act_fp8(gate_up, act_name, dt, quant, static_scale=None, want_a=False):
+    """Op (c). gate_up: uint16 [M, 2I] interleaved (g0,u0,g1,u1,...)."""
+    gu = np.ascontiguousarray(gate_up, dtype=np.uint16)
+    M, two_i = gu.shape
+    I = two_i // 2
+    q = np.empty((M, I), dtype=np.uint8)
+    nb = (I + 127) // 128
+    sc = np.empty((M, nb), dtype=np.float64) if quant == "block128" else None
+    a = np.empty((M, I), dtype=np.float64) if want_a else None
+    s = float(static_scale) if quant == "static" else 0.0
+    rc = lib().oracle_gate_act_fp8(_p(gu), _p(q), s, _p(sc), _p(a), M, I, _ACT[act_name], _DT[dt], _QM[quant])
+    if rc != 0:
+        raise ValueError("oracle_gate_act_fp8: bad argument")
+    return {"out_fp8": q, "block_scales": sc, "a": a}

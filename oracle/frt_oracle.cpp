@@ -1,0 +1,384 @@
+// Oracle for the fused non-GEMM layer chain -- TEST INFRASTRUCTURE ONLY.
+//
+// A plain, slow, obviously-correct CPU restatement of what the three fused
+// ops compute, in fp64, one element at a time, in the order the sources state
+// the steps.  It shares no code, header, table or constant with the CUDA
+// library; only tests, the smoke check and the bench's CPU-baseline leg may
+// load it.  The product path never calls it.
+//
+// Sources (web pages; cited by title and section):
+//   [FR]  "FlashRT kernel fusion: RMSNorm / residual / FP8 / QKV post-processing"
+//         (xdnf.cn/news/367260), sections 一..六 and the per-layer table in §二.
+//   [FR4] "sm89 prefill FFN megakernel" (FlashRT issue #1), Phase 1/Phase 2 and
+//         the correctness paragraph (per-token block-128 FP8 scales, out_scale).
+//   [FP]  "Falcon-Perception inference optimisation" (nxmr.cn/news/154322),
+//         third technique: interleaved [g0,u0,g1,u1,...] gate/up, relu(g)^2*u,
+//         sqrt(2) pre-baked into the gate weights.
+//
+// Readings taken where the pages are silent are listed in the design notes;
+// each function below states the one it relies on.
+//
+// Parity pins: every exported function is pinned by -m "not gpu" tests
+// (closed forms, invariants, library special cases, exhaustive round trips and
+// an independent brute-force restatement on tiny inputs).
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+namespace {
+
+// Own enumerations (numerically equal to the library's ABI values because
+// they are the interface the tests speak, not shared code).
+enum { DT_F16 = 0, DT_BF16 = 1 };
+enum { Q_STATIC = 0, Q_BLOCK128 = 1 };
+enum { ACT_GELU_TANH = 0, ACT_SILU = 1, ACT_RELU2 = 2 };
+
+// ---------------------------------------------------------------- formats --
+// IEEE-style binary16 (1/5/10) and bfloat16 (1/8/7) described by their field
+// widths; decoding is exact in double.
+struct Fmt16 {
+  int exp_bits;
+  int mant_bits;
+};
+const Fmt16 kF16 = {5, 10};
+const Fmt16 kBF16 = {8, 7};
+
+double decode16(uint16_t b, Fmt16 f) {
+  const int bias = (1 << (f.exp_bits - 1)) - 1;
+  const int emask = (1 << f.exp_bits) - 1;
+  const int sign = (b >> 15) & 1;
+  const int e = (b >> f.mant_bits) & emask;
+  const int m = b & ((1 << f.mant_bits) - 1);
+  double v;
+  if (e == 0) {
+    v = std::ldexp((double)m, 1 - bias - f.mant_bits);  // subnormal / zero
+  } else if (e == emask) {
+    v = (m == 0) ? INFINITY : NAN;
+  } else {
+    v = std::ldexp((double)((1 << f.mant_bits) | m), e - bias - f.mant_bits);
+  }
+  return sign ? -v : v;
+}
+
+// Round the exact real number hi + lo (|lo| at most half an ulp of hi in
+// double, as produced by an error-free sum) to the 16-bit format, round to
+// nearest, ties to even.  lo only decides exact 16-bit midpoints of hi.
+uint16_t round16(double hi, double lo, Fmt16 f) {
+  const int bias = (1 << (f.exp_bits - 1)) - 1;
+  const int emask = (1 << f.exp_bits) - 1;
+  const int emin = 1 - bias, emax = bias;
+  const uint16_t sign = std::signbit(hi) ? 0x8000 : 0;
+  if (std::isnan(hi)) return (uint16_t)(sign | (emask << f.mant_bits) | (1 << (f.mant_bits - 1)));
+  const double a = std::fabs(hi);
+  const double l = std::signbit(hi) ? -lo : lo;  // error term, same orientation as a
+  if (std::isinf(a)) return (uint16_t)(sign | (emask << f.mant_bits));
+  if (a == 0.0) return sign;
+  int e2;
+  std::frexp(a, &e2);           // a = fr * 2^e2, fr in [0.5, 1)
+  int E = e2 - 1;               // floor(log2 a)
+  if (E < emin) E = emin;       // subnormal range shares the emin quantum
+  const double quantum = std::ldexp(1.0, E - f.mant_bits);
+  const double n = a / quantum;  // exact: scaling by a power of two
+  const double fl = std::floor(n);
+  const double frac = n - fl;
+  double m;
+  if (frac > 0.5) {
+    m = fl + 1.0;
+  } else if (frac < 0.5) {
+    m = fl;
+  } else if (l > 0.0) {
+    m = fl + 1.0;               // exact value lies above the midpoint
+  } else if (l < 0.0) {
+    m = fl;                     // exact value lies below the midpoint
+  } else {
+    m = (std::fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;  // true tie: to even
+  }
+  if (m == std::ldexp(1.0, f.mant_bits + 1)) {  // carried into the next binade
+    E += 1;
+    m = std::ldexp(1.0, f.mant_bits);
+  }
+  if (E > emax) return (uint16_t)(sign | (emask << f.mant_bits));  // overflow: inf
+  const uint32_t mi = (uint32_t)m;
+  if (mi < (1u << f.mant_bits)) return (uint16_t)(sign | mi);      // subnormal
+  return (uint16_t)(sign | ((uint32_t)(E + bias) << f.mant_bits) | (mi - (1u << f.mant_bits)));
+}
+
+Fmt16 fmt_of(int dt) { return dt == DT_BF16 ? kBF16 : kF16; }
+
+// Error-free transformation: a + b == s + err exactly (Knuth's TwoSum).
+void two_sum(double a, double b, double* s, double* err) {
+  const double sum = a + b;
+  const double bb = sum - a;
+  *err = (a - (sum - bb)) + (b - bb);
+  *s = sum;
+}
+
+// OCP FP8 E4M3 ("e4m3fn"): bias 7, 3 mantissa bits, no infinities, one NaN
+// code per sign (0x7F / 0xFF), largest finite 448, smallest normal 2^-6,
+// subnormal step 2^-9.  Round to nearest, ties to even, saturating at +-448.
+uint8_t e4m3_encode(double v) {
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t s = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(v);
+  if (a >= 448.0) return (uint8_t)(s | 0x7E);
+  if (a == 0.0) return s;
+  int e2;
+  std::frexp(a, &e2);
+  int e = e2 - 1;
+  if (e < -6) e = -6;
+  const double quantum = std::ldexp(1.0, e - 3);
+  const double n = a / quantum;
+  const double fl = std::floor(n);
+  const double frac = n - fl;
+  double m;
+  if (frac > 0.5) {
+    m = fl + 1.0;
+  } else if (frac < 0.5) {
+    m = fl;
+  } else {
+    m = (std::fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+  }
+  if (m == 16.0) {
+    e += 1;
+    m = 8.0;
+  }
+  const int mi = (int)m;
+  if (mi < 8) return (uint8_t)(s | mi);  // subnormal (e == -6)
+  return (uint8_t)(s | ((e + 7) << 3) | (mi - 8));
+}
+
+double e4m3_decode(uint8_t c) {
+  const int sign = c >> 7;
+  const int e = (c >> 3) & 0xF;
+  const int m = c & 7;
+  double v;
+  if (e == 0xF && m == 7) {
+    v = NAN;
+  } else if (e == 0) {
+    v = std::ldexp((double)m, -9);
+  } else {
+    v = std::ldexp((double)(8 + m), e - 7 - 3);
+  }
+  return sign ? -v : v;
+}
+
+// ------------------------------------------------------------ quantisers --
+// Static per-tensor FP8 ([FR] §六: `_static` = the activation scale is a
+// constant).  s is a dequantisation scale: q = e4m3(y / s), y ~ q * s.
+void quant_static(const double* y, int64_t n, double s, uint8_t* q) {
+  for (int64_t j = 0; j < n; ++j) q[j] = e4m3_encode(y[j] / s);
+}
+
+// Per-token block-128 FP8 ([FR4] Phase 2: per-token block-128 quantisation
+// with an out_scale per row and block).  Block b covers columns
+// [128b, min(128b+128, n)); s_b = amax_b / 448, or 1 when the block is all
+// zero; q = e4m3(y / s_b).
+void quant_block128(const double* y, int64_t n, uint8_t* q, double* scales) {
+  const int64_t nb = (n + 127) / 128;
+  for (int64_t b = 0; b < nb; ++b) {
+    const int64_t lo = 128 * b;
+    const int64_t hi = (lo + 128 < n) ? lo + 128 : n;
+    double amax = 0.0;
+    for (int64_t j = lo; j < hi; ++j) amax = std::fmax(amax, std::fabs(y[j]));
+    const double s = (amax > 0.0) ? amax / 448.0 : 1.0;
+    scales[b] = s;
+    for (int64_t j = lo; j < hi; ++j) q[j] = e4m3_encode(y[j] / s);
+  }
+}
+
+// --------------------------------------------------------------- RMSNorm --
+// y_j = h_j * rstd * w_j with rstd = 1 / sqrt(mean(h^2) + eps); w == nullptr
+// is the `_noweight` form whose (1 + w) lives in the next GEMM's weights
+// ([FR] §三 and the §二.1 naming table).
+void rmsnorm(const double* h, int64_t n, const double* w, double eps, double* y) {
+  double ss = 0.0;
+  for (int64_t j = 0; j < n; ++j) ss += h[j] * h[j];
+  const double rstd = 1.0 / std::sqrt(ss / (double)n + eps);
+  for (int64_t j = 0; j < n; ++j) y[j] = h[j] * rstd * (w ? w[j] : 1.0);
+}
+
+// Rotate-half RoPE ([FR] §2.2, second bullet): for j < n/2 the pair
+// (v_j, v_{j+n/2}) is rotated by the angle whose cosine and sine are c_j, s_j.
+void rope_rotate_half(double* v, int n, const float* c, const float* s) {
+  const int half = n / 2;
+  for (int j = 0; j < half; ++j) {
+    const double a = v[j], b = v[j + half];
+    const double cj = (double)c[j], sj = (double)s[j];
+    v[j] = a * cj - b * sj;
+    v[j + half] = b * cj + a * sj;
+  }
+}
+
+// Gated activations ([FR] §二 steps 8-10: GELU(gate) * up; [FP] third
+// technique: relu(gate)^2 * up; SiLU * up for the SwiGLU FFNs).
+double act_fn(int act, double g) {
+  switch (act) {
+    case ACT_GELU_TANH: {
+      const double k = std::sqrt(2.0 / M_PI);
+      return 0.5 * g * (1.0 + std::tanh(k * (g + 0.044715 * g * g * g)));
+    }
+    case ACT_SILU:
+      return g / (1.0 + std::exp(-g));
+    case ACT_RELU2:
+      return g > 0.0 ? g * g : 0.0;
+    default:
+      return NAN;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+// ---------------------------------------------------------------- exports --
+double oracle_f16_decode(uint16_t b) { return decode16(b, kF16); }
+double oracle_bf16_decode(uint16_t b) { return decode16(b, kBF16); }
+uint16_t oracle_f16_round(double hi, double lo) { return round16(hi, lo, kF16); }
+uint16_t oracle_bf16_round(double hi, double lo) { return round16(hi, lo, kBF16); }
+uint8_t oracle_e4m3_encode(double v) { return e4m3_encode(v); }
+double oracle_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
+double oracle_act(int act, double g) { return act_fn(act, g); }
+
+// 16-bit rounding of the exact sum of two 16-bit values (the residual add).
+uint16_t oracle_add16(uint16_t x, uint16_t r, int dt) {
+  const Fmt16 f = fmt_of(dt);
+  double s, err;
+  two_sum(decode16(x, f), decode16(r, f), &s, &err);
+  return round16(s, err, f);
+}
+
+void oracle_quant_static(const double* y, int64_t n, double s, uint8_t* q) { quant_static(y, n, s, q); }
+void oracle_quant_block128(const double* y, int64_t n, uint8_t* q, double* scales) {
+  quant_block128(y, n, q, scales);
+}
+void oracle_rmsnorm(const double* h, int64_t n, const double* w, double eps, double* y) {
+  rmsnorm(h, n, w, eps, y);
+}
+void oracle_rope_rotate_half(double* v, int n, const float* c, const float* s) { rope_rotate_half(v, n, c, s); }
+
+// Op (a): residual add + RMSNorm + FP8 ([FR] §二 steps 1 and 7; §2.1 says
+// the three element-wise steps share one read of the same input).
+//   h = rn16(x + r) exactly rounded; residual_out = h; y = RMSNorm(h) in
+//   fp64 (the norm reads the rounded h, as the unfused add -> norm pipeline
+//   does); q = FP8(y) with the static scale or per-row block-128 scales.
+//   residual_out may alias residual_in.  y_out (optional, [M, D]) receives
+//   the fp64 y.  block_scales is [M, ceil(D/128)].  Returns 0, or -1 on a
+//   bad argument.
+int oracle_residual_rmsnorm_fp8(const uint16_t* x, const uint16_t* residual_in, uint16_t* residual_out,
+                                const uint16_t* weight, uint8_t* out_fp8, double static_scale,
+                                double* block_scales, double* y_out, int64_t M, int64_t D, double eps,
+                                int dt, int qm) {
+  if (M < 0 || D <= 0 || !x || !residual_in || !residual_out || !out_fp8) return -1;
+  if (qm == Q_BLOCK128 && !block_scales) return -1;
+  const Fmt16 f = fmt_of(dt);
+  const int64_t nb = (D + 127) / 128;
+  std::vector<double> h(D), w(D), y(D);
+  if (weight)
+    for (int64_t j = 0; j < D; ++j) w[j] = decode16(weight[j], f);
+  for (int64_t i = 0; i < M; ++i) {
+    for (int64_t j = 0; j < D; ++j) {
+      double s, err;
+      two_sum(decode16(x[i * D + j], f), decode16(residual_in[i * D + j], f), &s, &err);
+      const uint16_t hb = round16(s, err, f);
+      residual_out[i * D + j] = hb;
+      h[j] = decode16(hb, f);
+    }
+    rmsnorm(h.data(), D, weight ? w.data() : nullptr, eps, y.data());
+    if (y_out) std::memcpy(y_out + i * D, y.data(), sizeof(double) * D);
+    if (qm == Q_STATIC)
+      quant_static(y.data(), D, static_scale, out_fp8 + i * D);
+    else
+      quant_block128(y.data(), D, out_fp8 + i * D, block_scales + i * nb);
+  }
+  return 0;
+}
+
+// Op (b): packed QKV split + per-head q/k RMSNorm + rotate-half RoPE + Q
+// staging write + KV-cache write ([FR] §2.2 first bullet: q_norm -> RoPE ->
+// Q staging, k_norm -> RoPE -> KV cache; V passes through; [FR] §二 step 3).
+//   qkv row i = [Q heads (Hq*hd) | K heads (Hkv*hd) | V heads (Hkv*hd)].
+//   q_norm_w / k_norm_w ([hd], 16-bit) may each be null (no norm on that side).
+//   cos/sin tables are [max_pos, hd/2] fp32; position p = positions[i].
+//   q_out  [M, Hq, hd] receives the unrounded fp64 result.
+//   k_cache [capacity, Hkv, hd] fp64, v_cache [capacity, Hkv, hd] 16-bit bits.
+//   slots (optional, test convenience) stores row i at slots[i] instead of
+//   at positions[i]; the rotation always uses positions[i].
+//   A row whose position is outside [0, max_pos) or whose slot is outside
+//   [0, capacity) is skipped and bit 0 of *status is set.
+int oracle_qkv_norm_rope_kvcache(const uint16_t* qkv, const uint16_t* q_norm_w, const uint16_t* k_norm_w,
+                                 const float* cos_tab, const float* sin_tab, const int32_t* positions,
+                                 const int64_t* slots, double* q_out, double* k_cache, uint16_t* v_cache,
+                                 int32_t* status, int64_t M, int64_t Hq, int64_t Hkv, int64_t hd,
+                                 int64_t max_pos, int64_t capacity, double eps, int dt) {
+  if (M < 0 || Hq <= 0 || Hkv <= 0 || hd <= 0 || hd % 2 != 0) return -1;
+  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return -1;
+  const Fmt16 f = fmt_of(dt);
+  const int64_t width = (Hq + 2 * Hkv) * hd;
+  const int64_t half = hd / 2;
+  std::vector<double> v(hd), wq(hd), wk(hd), y(hd);
+  for (int64_t j = 0; j < hd; ++j) {
+    if (q_norm_w) wq[j] = decode16(q_norm_w[j], f);
+    if (k_norm_w) wk[j] = decode16(k_norm_w[j], f);
+  }
+  for (int64_t i = 0; i < M; ++i) {
+    const int64_t p = positions[i];
+    const int64_t slot = slots ? slots[i] : p;
+    if (p < 0 || p >= max_pos || slot < 0 || slot >= capacity) {
+      if (status) *status |= 1;
+      continue;
+    }
+    const float* c = cos_tab + p * half;
+    const float* s = sin_tab + p * half;
+    const uint16_t* row = qkv + i * width;
+    for (int64_t h = 0; h < Hq + Hkv; ++h) {
+      const bool is_q = h < Hq;
+      for (int64_t j = 0; j < hd; ++j) v[j] = decode16(row[h * hd + j], f);
+      const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
+      if (nw) {
+        rmsnorm(v.data(), hd, is_q ? wq.data() : wk.data(), eps, y.data());
+        v = y;
+      }
+      rope_rotate_half(v.data(), (int)hd, c, s);
+      double* dst = is_q ? q_out + (i * Hq + h) * hd : k_cache + (slot * Hkv + (h - Hq)) * hd;
+      std::memcpy(dst, v.data(), sizeof(double) * hd);
+    }
+    for (int64_t g = 0; g < Hkv; ++g)
+      std::memcpy(v_cache + (slot * Hkv + g) * hd, row + (Hq + Hkv + g) * hd, sizeof(uint16_t) * hd);
+  }
+  return 0;
+}
+
+// Op (c): gated activation on the interleaved gate/up buffer + FP8
+// ([FP] third technique: adjacent (gate, up) pairs, even index = gate;
+// [FR] §二 steps 8-10 GELU*up + quant; [FR4] Phase 2 block-128 FP8).
+//   a_j = act(g_j) * u_j with g_j = gate_up[i, 2j], u_j = gate_up[i, 2j+1].
+//   relu^2 takes g as given (sqrt(2) is already in the gate weights).
+//   a_out (optional, [M, I]) receives the fp64 a.  block_scales is
+//   [M, ceil(I/128)].
+int oracle_gate_act_fp8(const uint16_t* gate_up, uint8_t* out_fp8, double static_scale, double* block_scales,
+                        double* a_out, int64_t M, int64_t I, int act, int dt, int qm) {
+  if (M < 0 || I <= 0 || !gate_up || !out_fp8) return -1;
+  if (act < ACT_GELU_TANH || act > ACT_RELU2) return -1;
+  if (qm == Q_BLOCK128 && !block_scales) return -1;
+  const Fmt16 f = fmt_of(dt);
+  const int64_t nb = (I + 127) / 128;
+  std::vector<double> a(I);
+  for (int64_t i = 0; i < M; ++i) {
+    const uint16_t* row = gate_up + i * 2 * I;
+    for (int64_t j = 0; j < I; ++j) {
+      const double g = decode16(row[2 * j], f);
+      const double u = decode16(row[2 * j + 1], f);
+      a[j] = act_fn(act, g) * u;
+    }
+    if (a_out) std::memcpy(a_out + i * I, a.data(), sizeof(double) * I);
+    if (qm == Q_STATIC)
+      quant_static(a.data(), I, static_scale, out_fp8 + i * I);
+    else
+      quant_block128(a.data(), I, out_fp8 + i * I, block_scales + i * nb);
+  }
+  return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,447 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Closed forms, invariants, library special cases (numpy / torch float
+conversions, torch's rms_norm, transformers' rotate_half RoPE, torch's GELU
+and SiLU), exhaustive round trips, and an independent brute-force restatement
+on tiny inputs.  Runs without a GPU.
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import np_restatement as npr
+from memory_bound_non_b200 import workloads as W
+
+# ------------------------------------------------------------------ e4m3 --
+# OCP 8-bit floating point, E4M3 "fn" variant: bias 7, no infinities.
+E4M3_POINTS = {
+    0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x30: 0.5, 0x38: 1.0, 0x3F: 1.875,
+    0x40: 2.0, 0x48: 4.0, 0x70: 128.0, 0x77: 240.0, 0x78: 256.0, 0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0,
+}
+
+
+def test_e4m3_decode_points():
+    for c, v in E4M3_POINTS.items():
+        assert oracle.e4m3_decode(c) == v, hex(c)
+    assert math.isnan(oracle.e4m3_decode(0x7F)) and math.isnan(oracle.e4m3_decode(0xFF))
+    assert math.copysign(1.0, oracle.e4m3_decode(0x80)) < 0
+
+
+def test_e4m3_decode_monotonic():
+    vals = [oracle.e4m3_decode(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))
+    assert len(set(vals)) == 127
+
+
+def test_e4m3_roundtrip_all_finite_codes():
+    for c in range(256):
+        if c in (0x7F, 0xFF):
+            continue
+        assert oracle.e4m3_encode(oracle.e4m3_decode(c)) == c, hex(c)
+
+
+def test_e4m3_midpoints_round_to_even():
+    for c in range(0x7E):
+        lo, hi = oracle.e4m3_decode(c), oracle.e4m3_decode(c + 1)
+        mid = (lo + hi) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert oracle.e4m3_encode(mid) == even, hex(c)
+        assert oracle.e4m3_encode(-mid) == 0x80 | even
+        eps = (hi - lo) * 1e-6
+        assert oracle.e4m3_encode(mid - eps) == c
+        assert oracle.e4m3_encode(mid + eps) == c + 1
+
+
+def test_e4m3_saturation_and_specials():
+    for v in (448.0 * (1 + 2.0 ** -5), 464.0, 479.9, 500.0, 1e6, float("inf")):
+        assert oracle.e4m3_encode(v) == 0x7E
+        assert oracle.e4m3_encode(-v) == 0xFE
+    assert oracle.e4m3_encode(2.0 ** -10) == 0x00          # half the smallest subnormal: tie to even (0)
+    assert oracle.e4m3_encode(2.0 ** -10 * 1.01) == 0x01
+    assert oracle.e4m3_encode(3 * 2.0 ** -10) == 0x02       # tie between codes 1 and 2
+    assert oracle.e4m3_encode(-0.0) == 0x80
+    assert oracle.e4m3_encode(0.0) == 0x00
+    assert oracle.e4m3_encode(float("nan")) == 0x7F
+
+
+def test_e4m3_matches_torch_float8_in_range():
+    # torch's float32 -> float8_e4m3fn cast rounds to nearest-even; inside the
+    # finite range it is the same function.
+    g = torch.Generator().manual_seed(7)
+    v = torch.cat([torch.randn(4000, generator=g) * 40, torch.randn(2000, generator=g) * 0.01,
+                   (torch.rand(2000, generator=g) - 0.5) * 890]).float()
+    v = v[v.abs() < 448]
+    ref = v.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = np.array([oracle.e4m3_encode(float(t)) for t in v])
+    np.testing.assert_array_equal(ours, ref)
+
+
+# ------------------------------------------------------------ 16-bit fmts --
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_16bit_roundtrip_exhaustive(dt):
+    codes = np.arange(65536, dtype=np.uint16)
+    vals = oracle.decode16(codes, dt)
+    for b, v in zip(codes, vals):
+        if math.isnan(v):
+            continue
+        assert oracle.round16(v, 0.0, dt) == int(b), hex(int(b))
+
+
+def test_f16_decode_matches_numpy():
+    codes = np.arange(65536, dtype=np.uint16)
+    ref = codes.view(np.float16).astype(np.float64)
+    ours = oracle.decode16(codes, "f16")
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(ours[ok], ref[ok])
+    assert np.all(np.isnan(ours[~ok]))
+
+
+def test_bf16_decode_matches_torch():
+    codes = np.arange(65536, dtype=np.uint16)
+    ref = torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).double().numpy()
+    ours = oracle.decode16(codes, "bf16")
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(ours[ok], ref[ok])
+
+
+def test_f16_rounding_matches_numpy():
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.standard_normal(3000) * 100, rng.standard_normal(1000) * 1e-6,
+                        rng.standard_normal(500) * 7e4, rng.standard_normal(500) * 1e-8])
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16).view(np.uint16)
+    ours = np.array([oracle.round16(t, 0.0, "f16") for t in v], dtype=np.uint16)
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_bf16_rounding_matches_torch():
+    g = torch.Generator().manual_seed(4)
+    v = torch.cat([torch.randn(3000, generator=g) * 100, torch.randn(1000, generator=g) * 1e-30,
+                   torch.randn(500, generator=g) * 1e38]).float()
+    ref = v.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    ours = np.array([oracle.round16(float(t), 0.0, "bf16") for t in v], dtype=np.uint16)
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_16bit_midpoint_ties():
+    # 1 + 2^-8 lies halfway between bf16 1 and 1 + 2^-7: even -> 1.0 (0x3F80)
+    assert oracle.round16(1 + 2.0 ** -8, 0.0, "bf16") == 0x3F80
+    # halfway between 1 + 2^-7 (odd) and 1 + 2^-6: even is 1 + 2^-6 (0x3F82)
+    assert oracle.round16(1 + 3 * 2.0 ** -8, 0.0, "bf16") == 0x3F82
+    # the error term decides an exact midpoint of hi
+    assert oracle.round16(1 + 2.0 ** -8, 1e-30, "bf16") == 0x3F81
+    assert oracle.round16(1 + 3 * 2.0 ** -8, -1e-30, "bf16") == 0x3F81
+    # fp16: 1 + 2^-11 is the midpoint of 1 and 1 + 2^-10
+    assert oracle.round16(1 + 2.0 ** -11, 0.0, "f16") == 0x3C00
+    assert oracle.round16(1 + 2.0 ** -11, 1e-30, "f16") == 0x3C01
+    # overflow: fp16 max 65504, midpoint to 65536 rounds to inf
+    assert oracle.round16(65519.0, 0.0, "f16") == 0x7BFF
+    assert oracle.round16(65520.0, 0.0, "f16") == 0x7C00
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_add16_is_exactly_rounded_sum(dt):
+    """Residual sum: the 16-bit rounding of the exact sum (rational brute force),
+    including pairs whose exponents are far apart."""
+    rng = np.random.default_rng(11)
+    bits = rng.integers(0, 65536, size=(4000, 2)).astype(np.uint16)
+    near = rng.integers(0x3C00 if dt == "f16" else 0x3F00, 0x4400 if dt == "f16" else 0x4100,
+                        size=(2000, 2)).astype(np.uint16)
+    near[:, 1] ^= 0x8000 * (rng.integers(0, 2, size=2000)).astype(np.uint16)
+    bits = np.concatenate([bits, near])
+    dec = npr.DECODE[dt]
+    n_checked = 0
+    for xb, rb in bits:
+        a, b = dec(int(xb)), dec(int(rb))
+        if not (math.isfinite(a) and math.isfinite(b)):
+            continue
+        if a == 0.0 and b == 0.0:
+            continue
+        s = Fraction(a) + Fraction(b)
+        ref = npr.round16_exact(s, dt)
+        assert oracle.add16(xb, rb, dt) == ref, (hex(int(xb)), hex(int(rb)))
+        n_checked += 1
+    assert n_checked > 4000
+
+
+# ---------------------------------------------------------------- RMSNorm --
+def test_rmsnorm_constant_row_gives_weight():
+    rng = np.random.default_rng(0)
+    w = 1 + 0.1 * rng.standard_normal(64)
+    for c in (0.25, -3.0, 1024.0, 2.0 ** -20):
+        y = oracle.rmsnorm(np.full(64, c), w, 0.0)
+        np.testing.assert_allclose(y, math.copysign(1.0, c) * w, rtol=4e-16, atol=0)
+    for c in (0.3, -7.0):
+        eps = 1e-2
+        y = oracle.rmsnorm(np.full(64, c), w, eps)
+        np.testing.assert_allclose(y, w * c / math.sqrt(c * c + eps), rtol=1e-15)
+
+
+def test_rmsnorm_scale_invariance():
+    rng = np.random.default_rng(1)
+    h = rng.standard_normal(4096)
+    w = 1 + 0.1 * rng.standard_normal(4096)
+    y = oracle.rmsnorm(h, w, 0.0)
+    for alpha in (2.0 ** 10, 3.7, -0.001):
+        np.testing.assert_allclose(oracle.rmsnorm(alpha * h, w, 0.0), math.copysign(1, alpha) * y,
+                                   rtol=1e-13, atol=1e-15)
+
+
+def test_rmsnorm_matches_torch_rms_norm():
+    rng = np.random.default_rng(2)
+    for n, eps in ((1024, 1e-6), (72, 1e-5), (7, 0.5)):
+        h = rng.standard_normal(n) * 3
+        w = 1 + 0.1 * rng.standard_normal(n)
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(h), (n,), torch.from_numpy(w), eps).numpy()
+        np.testing.assert_allclose(oracle.rmsnorm(h, w, eps), ref, rtol=1e-14, atol=1e-15)
+        ref0 = torch.nn.functional.rms_norm(torch.from_numpy(h), (n,), None, eps).numpy()
+        np.testing.assert_allclose(oracle.rmsnorm(h, None, eps), ref0, rtol=1e-14, atol=1e-15)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_op_a_unit_weight_equals_noweight(dt):
+    wl = W.get("tiny", dt=dt, M=4, D=256)
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False)
+    x, r = W.bits16(inp.layers[0].x_attn), W.bits16(inp.residual)
+    ones = W.bits16(torch.ones(256, dtype=W.DTYPES[dt]))
+    for quant in ("static", "block128"):
+        a = oracle.residual_rmsnorm_fp8(x, r, ones, 1e-6, dt, quant, static_scale=0.01, want_y=True)
+        b = oracle.residual_rmsnorm_fp8(x, r, None, 1e-6, dt, quant, static_scale=0.01, want_y=True)
+        np.testing.assert_array_equal(a["y"], b["y"])
+        np.testing.assert_array_equal(a["out_fp8"], b["out_fp8"])
+
+
+def test_op_a_composition_of_pinned_steps():
+    """The op is the pinned steps in order: exact residual add -> RMSNorm of the
+    rounded h -> FP8 of y."""
+    wl = W.get("tiny", M=3, D=384, dt="bf16")
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False)
+    L = inp.layers[0]
+    x, r, w = W.bits16(L.x_attn), W.bits16(inp.residual), W.bits16(L.w_attn)
+    out = oracle.residual_rmsnorm_fp8(x, r, w, 1e-6, "bf16", "block128", want_y=True)
+    for i in range(3):
+        h_bits = np.array([oracle.add16(a, b, "bf16") for a, b in zip(x[i], r[i])], dtype=np.uint16)
+        np.testing.assert_array_equal(out["residual_out"][i], h_bits)
+        h = oracle.decode16(h_bits, "bf16")
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(h), (384,),
+                                           torch.from_numpy(oracle.decode16(w, "bf16")), 1e-6).numpy()
+        np.testing.assert_allclose(out["y"][i], ref, rtol=1e-14, atol=1e-15)
+        q, sc = oracle.quant_block128(out["y"][i])
+        np.testing.assert_array_equal(out["out_fp8"][i], q)
+        np.testing.assert_array_equal(out["block_scales"][i], sc)
+
+
+# ------------------------------------------------------------------ RoPE --
+def test_rope_position_zero_is_identity():
+    cos, sin = W.rope_tables(8, 128, 1e4)
+    v = np.random.default_rng(0).standard_normal(128)
+    np.testing.assert_array_equal(oracle.rope_rotate_half(v, cos[0].numpy(), sin[0].numpy()), v)
+
+
+def test_rope_quarter_turn_exact():
+    v = np.arange(1.0, 9.0)
+    c = np.zeros(4, dtype=np.float32)
+    s = np.ones(4, dtype=np.float32)
+    # rotating (a, b) by +90 degrees gives (-b, a)
+    np.testing.assert_array_equal(oracle.rope_rotate_half(v, c, s), np.concatenate([-v[4:], v[:4]]))
+
+
+def test_rope_preserves_pair_norm():
+    rng = np.random.default_rng(5)
+    cos, sin = W.rope_tables(4096, 128, 1e6)
+    for p in (1, 17, 4095):
+        v = rng.standard_normal(128)
+        c, s = cos[p].double().numpy(), sin[p].double().numpy()
+        o = oracle.rope_rotate_half(v, cos[p].numpy(), sin[p].numpy())
+        n_in = (v[:64] ** 2 + v[64:] ** 2) * (c * c + s * s)
+        n_out = o[:64] ** 2 + o[64:] ** 2
+        np.testing.assert_allclose(n_out, n_in, rtol=1e-12)
+
+
+def test_rope_matches_complex_multiplication():
+    rng = np.random.default_rng(6)
+    cos, sin = W.rope_tables(64, 72, 1e4)
+    v = rng.standard_normal(72)
+    p = 37
+    z = (v[:36] + 1j * v[36:]) * (cos[p].double().numpy() + 1j * sin[p].double().numpy())
+    o = oracle.rope_rotate_half(v, cos[p].numpy(), sin[p].numpy())
+    np.testing.assert_allclose(o, np.concatenate([z.real, z.imag]), rtol=1e-14, atol=1e-15)
+
+
+def test_rope_matches_transformers_rotate_half():
+    from transformers.models.llama.modeling_llama import apply_rotary_pos_emb
+    rng = np.random.default_rng(8)
+    hd = 128
+    cos, sin = W.rope_tables(100, hd, 1e4)
+    p = torch.tensor([0, 5, 99])
+    cos_full = torch.cat([cos[p], cos[p]], dim=-1).double()[None, None]   # [1,1,3,hd]
+    sin_full = torch.cat([sin[p], sin[p]], dim=-1).double()[None, None]
+    q = torch.from_numpy(rng.standard_normal((1, 1, 3, hd)))
+    k = torch.from_numpy(rng.standard_normal((1, 1, 3, hd)))
+    q_ref, k_ref = apply_rotary_pos_emb(q, k, cos_full[0, 0], sin_full[0, 0], unsqueeze_dim=0)
+    for t in range(3):
+        qo = oracle.rope_rotate_half(q[0, 0, t].numpy(), cos[p[t]].numpy(), sin[p[t]].numpy())
+        ko = oracle.rope_rotate_half(k[0, 0, t].numpy(), cos[p[t]].numpy(), sin[p[t]].numpy())
+        np.testing.assert_allclose(qo, q_ref[0, 0, t].numpy(), rtol=1e-14, atol=1e-14)
+        np.testing.assert_allclose(ko, k_ref[0, 0, t].numpy(), rtol=1e-14, atol=1e-14)
+
+
+def test_rope_composition():
+    # rotating by p then by q equals rotating by p + q (tables rounded to fp32)
+    cos, sin = W.rope_tables(256, 64, 1e4)
+    v = np.random.default_rng(9).standard_normal(64)
+    for p, q in ((3, 5), (100, 155), (1, 1)):
+        two = oracle.rope_rotate_half(oracle.rope_rotate_half(v, cos[p].numpy(), sin[p].numpy()),
+                                      cos[q].numpy(), sin[q].numpy())
+        one = oracle.rope_rotate_half(v, cos[p + q].numpy(), sin[p + q].numpy())
+        np.testing.assert_allclose(two, one, rtol=0, atol=3e-6 * np.abs(v).max())
+
+
+# ----------------------------------------------------------- activations --
+def test_activation_closed_forms():
+    assert oracle.act("relu2", 2.0) * 3.0 == 12.0
+    assert oracle.act("relu2", -1.0) == 0.0
+    assert oracle.act("silu", 0.0) == 0.0
+    assert oracle.act("silu", 1.0) == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
+    assert oracle.act("gelu_tanh", 0.0) == 0.0
+    assert oracle.act("gelu_tanh", 1.0) == pytest.approx(0.5 * (1 + math.tanh(0.7978845608028654 * 1.044715)),
+                                                        rel=1e-15)
+    assert oracle.act("gelu_tanh", 10.0) == pytest.approx(10.0, rel=1e-15)
+    assert abs(oracle.act("gelu_tanh", -10.0)) < 1e-20
+    assert oracle.act("silu", 40.0) == pytest.approx(40.0, rel=1e-15)
+    assert abs(oracle.act("silu", -40.0)) < 1e-15
+
+
+def test_activations_match_torch():
+    g = torch.linspace(-12, 12, 2001, dtype=torch.float64)
+    gel = torch.nn.functional.gelu(g, approximate="tanh").numpy()
+    sil = torch.nn.functional.silu(g).numpy()
+    rel = torch.relu(g).pow(2).numpy()
+    for i, t in enumerate(g.tolist()):
+        # 1 + tanh(z) cancels for g << 0: both sides carry ~|g| * 1e-16 absolute error there
+        assert oracle.act("gelu_tanh", t) == pytest.approx(gel[i], rel=1e-13, abs=1e-14)
+        assert oracle.act("silu", t) == pytest.approx(sil[i], rel=1e-13, abs=1e-300)
+        assert oracle.act("relu2", t) == rel[i]
+
+
+def test_relu2_sqrt2_prebaked_identity():
+    for g in (0.3, 1.7, 5.0, -2.0):
+        assert oracle.act("relu2", math.sqrt(2) * g) == pytest.approx(2 * oracle.act("relu2", g), rel=1e-15)
+
+
+def test_op_c_reads_even_as_gate_odd_as_up():
+    # gate_up row = [g0,u0,g1,u1,...]; a_j = act(g_j) * u_j
+    g = torch.tensor([[2.0, 3.0, -1.0, 5.0, 0.5, -4.0, 1.0, 1.0]], dtype=torch.bfloat16)
+    out = oracle.gate_act_fp8(W.bits16(g), "relu2", "bf16", "static", static_scale=1.0, want_a=True)
+    np.testing.assert_array_equal(out["a"][0], [12.0, 0.0, -1.0, 1.0])
+    np.testing.assert_array_equal(out["out_fp8"][0], [oracle.e4m3_encode(v) for v in (12.0, 0.0, -1.0, 1.0)])
+
+
+# ---------------------------------------------------------------- quant --
+def test_quant_static_reproduces_exact_codes():
+    rng = np.random.default_rng(12)
+    codes = rng.integers(0, 256, size=2000).astype(np.uint8)
+    codes = codes[(codes != 0x7F) & (codes != 0xFF)]
+    s = 0.0371337890625  # exactly representable, so q * s is exact in fp64
+    y = np.array([oracle.e4m3_decode(c) for c in codes]) * s
+    q = oracle.quant_static(y, s)
+    np.testing.assert_array_equal(q, codes)
+
+
+def test_quant_block128_scales_and_edges():
+    rng = np.random.default_rng(13)
+    n = 128 * 3 + 80  # partial last block of 80 columns
+    y = rng.standard_normal(n)
+    y[128:256] = 0.0                # all-zero block -> scale 1, codes 0
+    q, sc = oracle.quant_block128(y)
+    assert sc.size == 4
+    assert sc[1] == 1.0 and np.all(q[128:256] == 0)
+    for b in (0, 2, 3):
+        blk = y[128 * b:min(n, 128 * b + 128)]
+        assert sc[b] == np.abs(blk).max() / 448.0
+        jmax = 128 * b + int(np.argmax(np.abs(blk)))
+        assert q[jmax] & 0x7F == 0x7E   # the block's largest element maps to +-448
+    # exact values: y = code * s with a known amax element reproduce the codes
+    codes = np.array([0x7E] + list(rng.integers(0, 0x7E, size=127)), dtype=np.uint8)
+    s = 0.5
+    yy = np.array([oracle.e4m3_decode(c) for c in codes]) * s * 448 / 448
+    q2, sc2 = oracle.quant_block128(yy * 1.0)
+    assert sc2[0] == 448 * s / 448
+    np.testing.assert_array_equal(q2, codes)
+
+
+# -------------------------------------------------------- brute force 4x8 --
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("weighted", [True, False])
+@pytest.mark.parametrize("quant", ["static", "block128"])
+def test_bruteforce_op_a(dt, weighted, quant):
+    g = W.generator(21)
+    x = W.normal16((4, 8), dt, g)
+    r = W.normal16((4, 8), dt, g, scale=3.0)
+    w = W.norm_weight(8, dt, g) if weighted else None
+    xb, rb = W.bits16(x), W.bits16(r)
+    wb = None if w is None else W.bits16(w)
+    s = 0.0078125
+    o = oracle.residual_rmsnorm_fp8(xb, rb, wb, 1e-6, dt, quant, static_scale=s)
+    h_ref, q_ref, sc_ref = npr.residual_rmsnorm_fp8(xb, rb, wb, 1e-6, dt, quant, static_scale=s)
+    np.testing.assert_array_equal(o["residual_out"], h_ref)
+    np.testing.assert_array_equal(o["out_fp8"], q_ref)
+    if quant == "block128":
+        np.testing.assert_allclose(o["block_scales"], sc_ref, rtol=1e-14)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("qk_norm", [True, False])
+def test_bruteforce_op_b(dt, qk_norm):
+    g = W.generator(22)
+    Hq, Hkv, hd, M = 2, 1, 8, 4
+    qkv = W.bits16(W.normal16((M, (Hq + 2 * Hkv) * hd), dt, g))
+    qw = W.bits16(W.norm_weight(hd, dt, g)) if qk_norm else None
+    kw = W.bits16(W.norm_weight(hd, dt, g)) if qk_norm else None
+    cos, sin = W.rope_tables(16, hd, 1e4)
+    pos = np.array([3, 0, 15, 7], dtype=np.int32)
+    o = oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos.numpy(), sin.numpy(), pos, Hq, Hkv, hd, 16, 1e-6, dt)
+    q_ref, k_ref, v_ref = npr.qkv_norm_rope(qkv, qw, kw, cos.numpy(), sin.numpy(), pos, Hq, Hkv, hd, 1e-6, dt)
+    np.testing.assert_allclose(o["q_out"], q_ref, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(o["k_cache"][pos], k_ref, rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(o["v_cache"][pos], v_ref)
+    assert o["status"] == 0
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("act", ["gelu_tanh", "silu", "relu2"])
+@pytest.mark.parametrize("quant", ["static", "block128"])
+def test_bruteforce_op_c(dt, act, quant):
+    g = W.generator(23)
+    gu = W.bits16(W.normal16((4, 16), dt, g, scale=2.0))
+    s = 0.00390625
+    o = oracle.gate_act_fp8(gu, act, dt, quant, static_scale=s, want_a=True)
+    q_ref, sc_ref, a_ref = npr.gate_act_fp8(gu, act, dt, quant, static_scale=s)
+    np.testing.assert_allclose(o["a"], a_ref, rtol=1e-13, atol=1e-300)
+    np.testing.assert_array_equal(o["out_fp8"], q_ref)
+    if quant == "block128":
+        np.testing.assert_allclose(o["block_scales"], sc_ref, rtol=1e-13)
+
+
+# ---------------------------------------------------------- KV placement --
+def test_kv_placement_and_bad_positions():
+    g = W.generator(24)
+    Hq, Hkv, hd, M, cap = 4, 2, 16, 6, 32
+    qkv = W.bits16(W.normal16((M, (Hq + 2 * Hkv) * hd), "bf16", g))
+    cos, sin = W.rope_tables(cap, hd, 1e4)
+    pos = np.array([5, 31, 0, 40, -1, 12], dtype=np.int32)   # 40 and -1 are out of range
+    v0 = np.full((cap, Hkv, hd), 0x7E7E, dtype=np.uint16)
+    o = oracle.qkv_norm_rope_kvcache(qkv, None, None, cos.numpy(), sin.numpy(), pos, Hq, Hkv, hd, cap, 1e-6,
+                                     "bf16", v_cache=v0)
+    assert o["status"] == 1
+    written = {5, 31, 0, 12}
+    for slot in range(cap):
+        k_nan = np.isnan(o["k_cache"][slot]).all()
+        v_sent = (o["v_cache"][slot] == 0x7E7E).all()
+        assert k_nan == (slot not in written) and v_sent == (slot not in written), slot
+    assert np.isnan(o["q_out"][3]).all() and np.isnan(o["q_out"][4]).all()
+    assert not np.isnan(o["q_out"][[0, 1, 2, 5]]).any()
