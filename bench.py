@@ -1,0 +1,572 @@
+#!/usr/bin/env python
+"""Benchmark of the fused non-GEMM layer chain on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload large_m_M65536] [--no-chain] [--no-e2e] [--no-cpu]
+
+One step = one pass of the whole hot path over one batch: the four fused-op
+launches of a layer (attention-input residual+RMSNorm+FP8, QKV
+norm+RoPE+KV-cache write, FFN-input residual+RMSNorm+FP8, gated activation +
+FP8) on the large-M workload (M=65536 tokens, D=4096, 32/8 heads of 128,
+squared-ReLU FFN with I=16384, 131072-slot KV cache): about 10.8 GB of
+algorithmic HBM traffic per step, far larger than L2.  `value` is the
+achieved HBM bandwidth of the step (algorithmic bytes / device time, summed
+over ranks / max over ranks).
+
+Also reported on the same JSON line:
+  per_op        each op's CUDA-event time inside the timed steps, GB/s and
+                fraction of the measured HBM copy peak and of 8 TB/s;
+  roofline      the dominant kernel (gated activation) against the HBM peak;
+  chain         microseconds per graphed layer chain: the Pi0.5-like decoder
+                (18 layers x 10 steps = 720 nodes) and the VLA denoise loop
+                (32 x 10 = 1280 nodes), each one CUDA graph, L2 flushed
+                between replays; per-node cost against the launch floor;
+  launch_floor  an empty kernel per stream launch and per graph node;
+  small_m       per-op microseconds at M <= 41 against the launch floor;
+  e2e           the same step through the public API with pinned host
+                buffers: host->device copy of the step's inputs, the four ops,
+                device->host copy of the step's outputs;
+  clocks        nvidia-smi SM clock and throttle reasons sampled while timing;
+  cpu_baseline  the CPU oracle (single thread) on a bounded row sample.
+
+Multi-GPU (torchrun): each rank runs its own row shard (weak scaling, no
+collective on the data path); timing is max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "achieved HBM GB/s (% of roofline) per fused op; µs per graphed layer chain"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ---------------------------------------------------------------- helpers --
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="large_m_M65536")
+    p.add_argument("--no-chain", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--chain-reps", type=int, default=30)
+    p.add_argument("--json-out", default=None)
+    return p.parse_args(argv)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def op_bytes(wl):
+    """Algorithmic HBM bytes of one call of each op (what it must move).
+    a: x, residual in, residual out (2 B each), FP8 out (1 B), + weight,
+       + scales; b: qkv read + Q/K/V written (2 B each), the token's cos and
+       sin rows (4 B x hd/2 x 2), its position, + q/k norm weights;
+    c: gate/up read (2 x 2 B per output), FP8 out (1 B), + scales."""
+    M, D, I, hd = wl.M, wl.D, wl.I, wl.hd
+    nbd, nbi = (D + 127) // 128, (I + 127) // 128
+    width = (wl.Hq + 2 * wl.Hkv) * hd
+    a = M * D * 7 + (2 * D if wl.weighted else 0) + (4 * M * nbd if wl.quant == "block128" else 4)
+    b = M * width * 4 + M * hd * 4 + 4 * M + (4 * hd if wl.qk_norm else 0)
+    c = M * I * 5 + (4 * M * nbi if wl.quant == "block128" else 4)
+    return {"attn_norm": a, "qkv": b, "ffn_norm": a, "gate": c}
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling in the background."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device=0):
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                if self.uuid and self.uuid not in parts[0] and parts[0] not in self.uuid:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        busy = [r for r in rows if (num(r[4]) or 0) >= 50] or rows
+        sm = [num(r[1]) for r in busy if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
+                "reasons": reasons, "samples": len(rows), "samples_busy": len(busy),
+                "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def time_graph(graph, reps, flush_buf, stream):
+    """Median and mean device time of one replay, L2 flushed before each."""
+    times = []
+    for _ in range(reps):
+        flush_l2(flush_buf)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.median(times), times
+
+
+# ------------------------------------------------------------- GPU legs --
+def launch_floor(reps=2000):
+    import memory_bound_non_b200 as frt
+    s = torch.cuda.current_stream()
+    for _ in range(50):
+        frt.frt_noop(1, 32)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        frt.frt_noop(1, 32)
+    e1.record(s)
+    e1.synchronize()
+    per_launch = e0.elapsed_time(e1) * 1e3 / reps
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(s)
+    with torch.cuda.stream(side):
+        frt.frt_noop(1, 32)
+    s.wait_stream(side)
+    with torch.cuda.graph(g):
+        for _ in range(1000):
+            frt.frt_noop(1, 32)
+    g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(20):
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3 / 1000)
+    del g
+    return {"stream_launch_us": per_launch, "graph_node_us": statistics.median(ts),
+            "kernel": "frt_noop <<<1, 32>>>"}
+
+
+def small_m_ops(floor, reps=400):
+    """Per-op us at M <= 41: back-to-back stream launches and graph nodes."""
+    from memory_bound_non_b200 import workloads as W
+    from memory_bound_non_b200.chain import LayerChain
+    out = {}
+    s = torch.cuda.current_stream()
+    for name in ("tiny", "pi05", "vla_denoise"):
+        wl = W.get(name, layers=1, steps=1)
+        ch = LayerChain(wl, W.make_inputs(wl, n_layers=1))
+        ch.calibrate_static_scales()
+        res = {}
+        for op in ("attn_norm", "qkv", "gate"):
+            fn = getattr(ch, op)
+            for _ in range(20):
+                fn(0)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(reps):
+                fn(0)
+            e1.record(s)
+            e1.synchronize()
+            stream_us = e0.elapsed_time(e1) * 1e3 / reps
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(200):
+                    fn(0)
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(10):
+                e0.record(s)
+                g.replay()
+                e1.record(s)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3 / 200)
+            del g
+            node_us = statistics.median(ts)
+            res[op] = {"stream_us": round(stream_us, 3), "graph_node_us": round(node_us, 3),
+                       "x_stream_floor": round(stream_us / floor["stream_launch_us"], 3),
+                       "x_graph_floor": round(node_us / floor["graph_node_us"], 3)}
+        out[name] = res
+    return out
+
+
+def chain_leg(reps, floor):
+    from memory_bound_non_b200 import workloads as W
+    from memory_bound_non_b200.chain import LayerChain
+    out = {}
+    s = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for name in ("pi05", "vla_denoise"):
+        wl = W.get(name)
+        ch = LayerChain(wl, W.make_inputs(wl))
+        ch.calibrate_static_scales()
+        ch.capture()
+        for _ in range(3):
+            ch.replay()
+        torch.cuda.synchronize()
+        med, ts = time_graph(ch.graph, reps, flush, s)
+        # back-to-back replays (warm L2), for reference
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(reps):
+            ch.replay()
+        e1.record(s)
+        e1.synchronize()
+        warm = e0.elapsed_time(e1) * 1e3 / reps
+        nodes = ch.launches_per_chain
+        b = op_bytes(wl)
+        chain_bytes = sum(b.values()) * wl.layers * wl.steps
+        out[name] = {"layers": wl.layers, "steps": wl.steps, "nodes": nodes, "us_per_chain": round(med, 2),
+                     "us_per_chain_warm_l2": round(warm, 2), "us_per_layer": round(med / (wl.layers * wl.steps), 3),
+                     "us_per_node": round(med / nodes, 3),
+                     "x_graph_node_floor": round(med / nodes / floor["graph_node_us"], 3),
+                     "hbm_bytes_per_chain": chain_bytes,
+                     "hbm_us_at_8TBps": round(chain_bytes / NOMINAL_HBM_GBS / 1e3, 2),
+                     "l2": "flushed before each replay (512 MiB write)"}
+        del ch
+    return out
+
+
+# ------------------------------------------------------------ large-M step --
+class Step:
+    """Device buffers of one layer at the bench workload, and its four ops."""
+
+    def __init__(self, wl, rank):
+        from memory_bound_non_b200 import workloads as W
+        from memory_bound_non_b200.chain import LayerChain
+        import dataclasses
+        wl_r = dataclasses.replace(wl, seed=wl.seed + 1000 * rank, layers=1, steps=1)
+        self.wl = wl_r
+        t0 = time.time()
+        self.host = W.make_inputs(wl_r, n_layers=1, device="cuda")  # seeded device generator
+        self.gen_s = time.time() - t0
+        self.chain = LayerChain(wl_r, self.host)
+        self.chain.calibrate_static_scales()
+        self.ops = [("attn_norm", self.chain.attn_norm), ("qkv", self.chain.qkv),
+                    ("ffn_norm", self.chain.ffn_norm), ("gate", self.chain.gate)]
+
+    def run(self):
+        for _, fn in self.ops:
+            fn(0)
+
+
+def timed_step_leg(step, K, W_, barrier):
+    s = torch.cuda.current_stream()
+    for _ in range(W_):
+        step.run()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    nops = len(step.ops)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s)
+    for k in range(K):
+        ev[k][0].record(s)
+        for i, (_, fn) in enumerate(step.ops):
+            fn(0)
+            ev[k][i + 1].record(s)
+    end.record(s)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    total_ms = start.elapsed_time(end)
+    per_op = {}
+    for i, (name, _) in enumerate(step.ops):
+        per_op[name] = [ev[k][i].elapsed_time(ev[k][i + 1]) * 1e3 for k in range(K)]
+    return total_ms, per_op
+
+
+def e2e_leg(step, K, W_):
+    """Public-API step with host buffers: H2D of the step's inputs from pinned
+    memory, the four ops, D2H of the step's outputs, on one stream."""
+    ch = step.chain
+    L, H = ch.layers[0], step.host
+    hl = H.layers[0]
+    ins = [(hl.x_attn, L.x_attn), (H.residual, ch.residual), (hl.qkv, L.qkv), (H.positions, ch.positions),
+           (hl.x_ffn, L.x_ffn), (hl.gate_up, L.gate_up)]
+    ins = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t), d) for t, d in ins]
+    outs = [(d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True))
+            for d in (L.q8_attn, L.q_out, ch.residual, L.q8_ffn, L.act8)]
+    h2d = sum(h.numel() * h.element_size() for h, _ in ins)
+    d2h = sum(h.numel() * h.element_size() for _, h in outs)
+    s = torch.cuda.current_stream()
+
+    def one():
+        for h, d in ins:
+            d.copy_(h, non_blocking=True)
+        step.run()
+        for d, h in outs:
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(W_):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(K):
+        one()
+    e1.record(s)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / K, h2d, d2h
+
+
+# -------------------------------------------------------------- CPU legs --
+def oracle_sample(wl, host, rows):
+    """Run the oracle on the first `rows` rows of every op of the step.
+    Returns seconds."""
+    import oracle
+    from memory_bound_non_b200 import workloads as W
+    hl = host.layers[0]
+    x_a, x_f = W.bits16(hl.x_attn[:rows]), W.bits16(hl.x_ffn[:rows])
+    r = W.bits16(host.residual[:rows])
+    wa = None if hl.w_attn is None else W.bits16(hl.w_attn)
+    wf = None if hl.w_ffn is None else W.bits16(hl.w_ffn)
+    qkv = W.bits16(hl.qkv[:rows])
+    qw = None if hl.q_norm_w is None else W.bits16(hl.q_norm_w)
+    kw = None if hl.k_norm_w is None else W.bits16(hl.k_norm_w)
+    gu = W.bits16(hl.gate_up[:rows])
+    pos = host.positions[:rows].cpu().numpy()
+    cos, sin = host.cos.cpu().numpy(), host.sin.cpu().numpy()
+    t0 = time.perf_counter()
+    o = oracle.residual_rmsnorm_fp8(x_a, r, wa, wl.eps, wl.dt, wl.quant, static_scale=0.01)
+    oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, wl.Hq, wl.Hkv, wl.hd, rows, wl.eps, wl.dt,
+                                 slots=np.arange(rows))
+    oracle.residual_rmsnorm_fp8(x_f, o["residual_out"], wf, wl.eps, wl.dt, wl.quant, static_scale=0.01)
+    oracle.gate_act_fp8(gu, wl.act, wl.dt, wl.quant, static_scale=0.01)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, host, budget_s=12.0):
+    import dataclasses
+    rows = 16
+    secs = oracle_sample(wl, host, rows)
+    rows = int(max(16, min(wl.M, rows * budget_s / max(secs, 1e-6))))
+    secs = oracle_sample(wl, host, rows)
+    b = sum(op_bytes(dataclasses.replace(wl, M=rows)).values())
+    return {"value": round(b / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d of %d token rows of every op of the step (%.1f s, single thread)"
+                      % (rows, wl.M, secs)}
+
+
+def host_inputs_only(wl):
+    from memory_bound_non_b200 import workloads as W
+    return W.make_inputs(wl, n_layers=1)
+
+
+def reference_arm(args):
+    """The oracle, as it stands, timed on host cores on the same workload."""
+    import dataclasses
+    from memory_bound_non_b200 import workloads as W
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = W.get(args.workload)
+    # inputs for a row sample only (the oracle runs on the first rows)
+    probe_rows = 16
+    host = W.make_inputs(dataclasses.replace(wl, M=4096), n_layers=1)
+    t = oracle_sample(wl, host, probe_rows) / probe_rows
+    budget = 150.0
+    rows = int(max(1, min(4096, budget / max(1, args.steps + args.warmup) / max(t, 1e-9))))
+    for _ in range(args.warmup):
+        oracle_sample(wl, host, rows)
+    secs = 0.0
+    for _ in range(args.steps):
+        secs += oracle_sample(wl, host, rows)
+    per_step = secs / args.steps
+    b = sum(op_bytes(dataclasses.replace(wl, M=rows)).values())
+    val = b / per_step / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded torch.Generator('cpu'))",
+            "config": {"workload": wl.name, "M": wl.M, "D": wl.D, "Hq": wl.Hq, "Hkv": wl.Hkv, "hd": wl.hd,
+                       "I": wl.I, "act": wl.act, "quant": wl.quant, "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": "first %d token rows of every op per step" % rows},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main --
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return reference_arm(args)
+    import memory_bound_non_b200 as frt
+    from memory_bound_non_b200 import workloads as W
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    frt.load()
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(x):
+        if pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = W.get(args.workload)
+    peak, peak_kind = measured_peak()
+    step = Step(wl, rank)
+    bytes_op = op_bytes(step.wl)
+    step_bytes = sum(bytes_op.values())
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    total_ms, per_op_us = timed_step_leg(step, args.steps, args.warmup, barrier)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(total_ms)
+    ms_per_step = total_ms / args.steps
+    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+
+    per_op = {}
+    for name, ts in per_op_us.items():
+        mean_us = sum(ts) / len(ts)
+        gbs = bytes_op[name] / (mean_us * 1e-6) / 1e9
+        per_op[name] = {"us_mean": round(mean_us, 2), "us_median": round(statistics.median(ts), 2),
+                        "bytes": bytes_op[name], "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                        "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4)}
+    dom = max(per_op, key=lambda k: per_op[k]["us_mean"])
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr_path):
+        with open(tr_path) as f:
+            traffic = json.load(f).get(wl.name, {}).get(dom)
+    roofline = {"bound": "hbm", "kernel": {"gate": "frt_gate_act_fp8", "qkv": "frt_qkv_norm_rope_kvcache",
+                                          "attn_norm": "frt_residual_rmsnorm_fp8",
+                                          "ffn_norm": "frt_residual_rmsnorm_fp8"}[dom],
+                "achieved": per_op[dom]["GBps"], "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": round(per_op[dom]["GBps"] / peak, 4), "traffic": traffic,
+                "algorithmic_bytes_per_launch": bytes_op[dom]}
+
+    extra = {}
+    if rank == 0 and not args.no_chain:
+        floor = launch_floor()
+        extra["launch_floor"] = {k: (round(v, 3) if isinstance(v, float) else v) for k, v in floor.items()}
+        extra["chain"] = chain_leg(args.chain_reps, floor)
+        extra["small_m"] = small_m_ops(floor)
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_leg(step, args.e2e_steps, 1)
+        e2e_ms = max_over_ranks(e2e_ms)
+        e2e = {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(step.wl, step.host)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic: seeded torch.Generator('cpu'), N(0,1) activations, 1+0.1N norm weights",
+                "config": {"workload": wl.name, "M": wl.M, "D": wl.D, "Hq": wl.Hq, "Hkv": wl.Hkv, "hd": wl.hd,
+                           "I": wl.I, "act": wl.act, "quant": wl.quant, "io": "bf16 in, e4m3 out",
+                           "capacity": wl.capacity, "bytes_per_step_per_gpu": step_bytes,
+                           "l2": "inputs larger than L2 (%.1f GB per step)" % (step_bytes / 1e9),
+                           "parallelism": "row shards, no collective" if world > 1 else "single GPU"},
+                "roofline": roofline, "per_op": per_op, "gpu_launches": 4 * args.steps, "clocks": clk,
+                "e2e": e2e, "cpu_baseline": cpu, "input_gen_s": round(step.gen_s, 1)}
+        line.update(extra)
+        s = json.dumps(line)
+        print(s, flush=True)
+        if args.json_out:
+            with open(args.json_out, "w") as f:
+                f.write(s + "\n")
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,187 @@
+/*
+ * frt.h -- fused non-GEMM layer ops for B200 (sm_100a), C ABI of libfrt.so.
+ *
+ * Three fused ops cover the memory- and launch-bound chain that sits between
+ * the GEMMs of a small-batch transformer layer ("FlashRT kernel fusion",
+ * §二 per-layer table: steps 1/7, 3 and 8-10):
+ *
+ *   frt_residual_rmsnorm_fp8   residual add + RMSNorm + FP8 e4m3 quantisation
+ *   frt_qkv_norm_rope_kvcache  packed-QKV split + per-head q/k RMSNorm +
+ *                              rotate-half RoPE + Q staging + KV-cache write
+ *   frt_gate_act_fp8           gated activation on interleaved gate/up + FP8
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers marked "device" are caller-owned device memory; the library
+ *    allocates nothing and keeps no pointer after the call returns.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream), never
+ *    synchronises, holds no state between calls and may be captured into a
+ *    CUDA graph.
+ *  - Host-detectable errors return a status before anything is launched:
+ *      FRT_ERR_INVALID_ARG  negative sizes, a size that breaks the layout rule
+ *                           stated per op, a required pointer that is NULL,
+ *                           a pointer below its stated alignment, a missing
+ *                           scale pointer for the chosen quant mode, an unknown
+ *                           enum value;
+ *      FRT_ERR_UNSUPPORTED  a valid shape this build does not cover (stated per
+ *                           op);
+ *      FRT_ERR_CUDA         the launch itself failed (cudaGetLastError after
+ *                           the launch).
+ *  - M == 0 is an empty batch: the call returns FRT_OK and launches nothing.
+ *  - Device-side data errors never trap: see the status word of op (b).
+ *  - 16-bit tensors are fp16 or bf16 as selected by `dt`; all layouts are
+ *    row-major and contiguous.  e4m3 is OCP FP8 E4M3 ("fn": max 448, no inf).
+ *  - FP8 conversion rounds to nearest-even and saturates to +-448; NaN input
+ *    gives the NaN code.
+ *  - Aliasing: only residual_out == residual_in (op a) is allowed; any other
+ *    overlap between outputs, or between an output and an input, is undefined.
+ */
+#ifndef FRT_H_
+#define FRT_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FRT_OK = 0,
+  FRT_ERR_INVALID_ARG = 1,
+  FRT_ERR_UNSUPPORTED = 2,
+  FRT_ERR_CUDA = 3
+} frt_status;
+
+typedef enum { FRT_F16 = 0, FRT_BF16 = 1 } frt_dtype;
+
+/* FP8 scaling.  A scale s is a dequantisation scale: code = e4m3(y / s), so
+ * y ~ code * s.
+ *  STATIC   one fp32 scale for the whole tensor, read from device memory
+ *           ("FlashRT kernel fusion", §六: `_static` = constant activation
+ *           scale).
+ *  BLOCK128 per row and per 128-column block b = [128b, min(128b+128, N)):
+ *           s = amax/448 over the block's valid columns (s = 1 for an all-zero
+ *           block), written as fp32 to block_scales[row * ceil(N/128) + b]
+ *           ("sm89 prefill FFN megakernel", Phase 2: per-token block-128 FP8
+ *           and its out_scale).  Every scale of every row is written. */
+typedef enum { FRT_QUANT_STATIC = 0, FRT_QUANT_BLOCK128 = 1 } frt_quant;
+
+/* Gate activations, applied to the even element g of each (g, u) pair:
+ *  GELU_TANH  0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3)))  (GeGLU)
+ *  SILU       g / (1 + exp(-g))                                (SwiGLU)
+ *  RELU2      max(g, 0)^2; any sqrt(2) factor is already in the gate weights
+ *             ("Falcon-Perception inference optimisation", third technique). */
+typedef enum { FRT_ACT_GELU_TANH = 0, FRT_ACT_SILU = 1, FRT_ACT_RELU2 = 2 } frt_act;
+
+/*
+ * (a) Residual add + RMSNorm + FP8 quantisation.
+ * "FlashRT kernel fusion", §二 steps 1 and 7 (residual_add_rms_norm_fp8_noweight)
+ * and §2.1 (the three element-wise steps share one pass over the row); §三 for
+ * the `_noweight` form whose (1 + w) is folded into the next GEMM's weights.
+ *
+ * For each row i (M rows of D columns):
+ *   h[i,j]   = x[i,j] + residual_in[i,j], the exact sum rounded once to the
+ *              16-bit type (RNE); written to residual_out (the new residual
+ *              stream).
+ *   rstd_i   = 1 / sqrt(mean_j(h[i,j]^2) + eps), computed from the rounded h
+ *              with fp32 accumulation in a fixed order.
+ *   y[i,j]   = h[i,j] * rstd_i * weight[j]   (weight == NULL: no weight).
+ *   out_fp8  = e4m3 of y / s (quant mode as above; block scales over D).
+ *
+ *   x, residual_in, residual_out  device, [M, D] 16-bit, 16-byte aligned;
+ *                                 residual_out may equal residual_in.
+ *   weight        device [D] 16-bit, 16-byte aligned, or NULL.
+ *   out_fp8       device [M, D] uint8, 8-byte aligned.
+ *   static_scale  STATIC: device fp32[1], 4-byte aligned; else ignored.
+ *   block_scales  BLOCK128: device fp32 [M, ceil(D/128)]; else ignored.
+ *   Layout rule: D > 0 and D % 8 == 0.  Unsupported: D > 32768.
+ */
+frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residual_in, void* residual_out,
+                                    const void* weight, uint8_t* out_fp8, const float* static_scale,
+                                    float* block_scales, int M, int D, float eps, frt_dtype dt,
+                                    frt_quant qm, cudaStream_t stream);
+
+/*
+ * (b) Packed QKV split + per-head q/k RMSNorm + rotate-half RoPE + Q staging
+ *     + KV-cache write.
+ * "FlashRT kernel fusion", §2.2 first bullet (q_norm -> RoPE -> Q staging and
+ * k_norm -> RoPE -> KV cache in one kernel; V passes straight through) and
+ * second bullet (rotate_half RoPE with each rotation pair kept in one lane);
+ * §二 step 3 (QKV split + RoPE + KV-cache write, no q/k norm); §四 (RoPE table
+ * precomputed).
+ *
+ * Row i of qkv is [Q heads (Hq*hd) | K heads (Hkv*hd) | V heads (Hkv*hd)],
+ * each head contiguous.  With p = positions[i] and half = hd/2:
+ *   v      = one Q or K head, in fp32;
+ *   norm   v = v * (1/sqrt(mean(v^2) + eps)) * w   with w = q_norm_w for Q
+ *            heads, k_norm_w for K heads; skipped for a side whose weight is
+ *            NULL;
+ *   rope   for j < half, c = cos_tab[p, j], s = sin_tab[p, j]:
+ *            o[j] = v[j] c - v[j+half] s,  o[j+half] = v[j+half] c + v[j] s;
+ *   q_out[i, h, :]          = o (Q head h), rounded once to 16 bits;
+ *   k_cache[p, g, :]        = o (K head g), rounded once to 16 bits;
+ *   v_cache[p, g, :]        = V head g, bit copy.
+ * The RoPE position is also the cache slot.  Duplicate positions within one
+ * call leave the slot with one of the rows (which one is unspecified).
+ *
+ *   qkv                 device [M, (Hq+2Hkv)*hd] 16-bit.
+ *   q_norm_w, k_norm_w  device [hd] 16-bit each, or NULL.
+ *   cos_tab, sin_tab    device [max_pos, hd/2] fp32, 16-byte aligned.
+ *   positions           device int32 [M].
+ *   q_out               device [M, Hq, hd] 16-bit.
+ *   k_cache, v_cache    device [capacity, Hkv, hd] 16-bit; rows other than the
+ *                       M written slots are left untouched.
+ *   status              device int32[1] or NULL.  A row whose position is
+ *                       < 0, >= max_pos or >= capacity is skipped entirely
+ *                       (no Q, K or V write) and bit 0 of *status is set with
+ *                       an atomic OR; the word is never cleared by the call.
+ *   16-bit pointers must be 16-byte aligned when hd % 16 == 0 and 8-byte
+ *   aligned otherwise.
+ *   Layout rule: Hq, Hkv > 0, Hq % Hkv == 0, hd > 0 and even, max_pos > 0,
+ *   capacity > 0.  Unsupported: hd % 8 != 0 or hd > 256.
+ */
+frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_norm_w, const void* k_norm_w,
+                                     const float* cos_tab, const float* sin_tab, const int32_t* positions,
+                                     void* q_out, void* k_cache, void* v_cache, int32_t* status, int M,
+                                     int Hq, int Hkv, int hd, int max_pos, int capacity, float eps,
+                                     frt_dtype dt, cudaStream_t stream);
+
+/*
+ * (c) Gated activation on an interleaved gate/up buffer + FP8 quantisation.
+ * "Falcon-Perception inference optimisation", third technique (the gate and
+ * up weights are stored interleaved so one GEMM yields [g0,u0,g1,u1,...]; one
+ * kernel reads each adjacent pair, computes relu(g)^2 * u and writes once);
+ * "FlashRT kernel fusion", §二 steps 8-10 (GELU * up + quant, 3 -> 1);
+ * "sm89 prefill FFN megakernel", Phase 2 (silu * mul + per-token block-128 FP8).
+ *
+ *   a[i,j]   = act(g) * u with g = gate_up[i, 2j], u = gate_up[i, 2j+1],
+ *              in fp32, one rounding at the FP8 store.
+ *   out_fp8  = e4m3 of a / s (quant mode as above; block scales over I).
+ *
+ *   gate_up       device [M, 2I] 16-bit, 16-byte aligned.
+ *   out_fp8       device [M, I] uint8, 4-byte aligned.
+ *   static_scale  STATIC: device fp32[1]; else ignored.
+ *   block_scales  BLOCK128: device fp32 [M, ceil(I/128)]; else ignored.
+ *   Layout rule: I > 0 and I % 4 == 0.
+ */
+frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* static_scale,
+                            float* block_scales, int M, int I, frt_act act, frt_dtype dt, frt_quant qm,
+                            cudaStream_t stream);
+
+/*
+ * Empty kernel used to measure the launch floor that the ops above are graded
+ * against (the roofline of a launch-bound op is the larger of its HBM time and
+ * this floor).  Launches `grid` blocks of `block` threads that do nothing.
+ * Returns FRT_ERR_INVALID_ARG for grid < 1 or block outside [1, 1024].
+ */
+frt_status frt_noop(int grid, int block, cudaStream_t stream);
+
+/* Static, NUL-terminated description of a status value; never NULL. */
+const char* frt_status_string(frt_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FRT_H_ */

@@ -1,0 +1,128 @@
+"""Fused non-GEMM transformer-layer ops for B200: Python binding of libfrt.so.
+
+Argument marshalling only.  Every op runs in the CUDA kernels of libfrt.so;
+there is no CPU or PyTorch fallback: if the library is missing or a call
+fails, a ``FrtError`` is raised.  PyTorch supplies device memory and streams.
+
+Functions carry the C names of ``include/frt.h``:
+
+    frt_residual_rmsnorm_fp8(x, residual_in, residual_out, weight, out_fp8, ...)
+    frt_qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos, sin, positions, ...)
+    frt_gate_act_fp8(gate_up, out_fp8, ...)
+    frt_noop(grid, block)
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfrt.so")
+
+FRT_OK, FRT_ERR_INVALID_ARG, FRT_ERR_UNSUPPORTED, FRT_ERR_CUDA = 0, 1, 2, 3
+DTYPE = {torch.float16: 0, torch.bfloat16: 1}
+QUANT = {"static": 0, "block128": 1}
+ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
+
+# C entry points declared in include/frt.h
+EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8", "frt_noop",
+           "frt_status_string")
+
+
+class FrtError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__("%s failed: %s" % (fn, msg))
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfrt.so (once) and declare its C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FrtError("load", -1, "%s is missing; build it with `python -m memory_bound_non_b200.build`" % path)
+    L = ctypes.CDLL(path)
+    c = ctypes
+    vp, i32, f32 = c.c_void_p, c.c_int, c.c_float
+    L.frt_residual_rmsnorm_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, i32, i32, vp]
+    L.frt_residual_rmsnorm_fp8.restype = i32
+    L.frt_qkv_norm_rope_kvcache.argtypes = [vp] * 10 + [i32] * 6 + [f32, i32, vp]
+    L.frt_qkv_norm_rope_kvcache.restype = i32
+    L.frt_gate_act_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
+    L.frt_gate_act_fp8.restype = i32
+    L.frt_noop.argtypes = [i32, i32, vp]
+    L.frt_noop.restype = i32
+    L.frt_status_string.argtypes = [i32]
+    L.frt_status_string.restype = c.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().frt_status_string(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != FRT_OK:
+        raise FrtError(fn, status, status_string(status))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise FrtError("marshal", FRT_ERR_INVALID_ARG, "tensor is not on a CUDA device")
+    if not t.is_contiguous():
+        raise FrtError("marshal", FRT_ERR_INVALID_ARG, "tensor is not contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def frt_residual_rmsnorm_fp8(x, residual_in, residual_out, weight, out_fp8, static_scale=None,
+                             block_scales=None, eps=1e-6, quant="static", stream=None):
+    """Op (a): residual add + RMSNorm (+ weight) + FP8 e4m3.  x, residual_*: [M, D]
+    fp16/bf16; weight [D] or None; out_fp8 [M, D] uint8; static_scale fp32[1]
+    (static) or block_scales fp32 [M, ceil(D/128)] (block128)."""
+    M, D = x.shape
+    st = load().frt_residual_rmsnorm_fp8(
+        _ptr(x), _ptr(residual_in), _ptr(residual_out), _ptr(weight), _ptr(out_fp8), _ptr(static_scale),
+        _ptr(block_scales), M, D, float(eps), DTYPE[x.dtype], QUANT[quant], _stream(stream))
+    _check("frt_residual_rmsnorm_fp8", st)
+
+
+def frt_qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache,
+                              Hq, Hkv, hd, status=None, eps=1e-6, stream=None):
+    """Op (b): QKV split + q/k RMSNorm + rotate-half RoPE + Q staging + KV write.
+    qkv [M, (Hq+2Hkv)*hd]; cos/sin fp32 [max_pos, hd/2]; positions int32 [M];
+    q_out [M, Hq, hd]; caches [capacity, Hkv, hd]; status int32[1] or None."""
+    M = qkv.shape[0]
+    max_pos = cos_tab.shape[0]
+    capacity = k_cache.shape[0]
+    st = load().frt_qkv_norm_rope_kvcache(
+        _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(cos_tab), _ptr(sin_tab), _ptr(positions), _ptr(q_out),
+        _ptr(k_cache), _ptr(v_cache), _ptr(status), M, Hq, Hkv, hd, max_pos, capacity, float(eps),
+        DTYPE[qkv.dtype], _stream(stream))
+    _check("frt_qkv_norm_rope_kvcache", st)
+
+
+def frt_gate_act_fp8(gate_up, out_fp8, static_scale=None, block_scales=None, act="gelu_tanh", quant="static",
+                     stream=None):
+    """Op (c): act(g) * u on interleaved [M, 2I] gate/up + FP8 e4m3 -> [M, I]."""
+    M, two_i = gate_up.shape
+    st = load().frt_gate_act_fp8(_ptr(gate_up), _ptr(out_fp8), _ptr(static_scale), _ptr(block_scales), M,
+                                 two_i // 2, ACT[act], DTYPE[gate_up.dtype], QUANT[quant], _stream(stream))
+    _check("frt_gate_act_fp8", st)
+
+
+def frt_noop(grid=1, block=32, stream=None):
+    """Empty kernel: the launch floor."""
+    _check("frt_noop", load().frt_noop(int(grid), int(block), _stream(stream)))

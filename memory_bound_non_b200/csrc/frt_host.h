@@ -1,0 +1,26 @@
+// Host-side helpers for argument validation and launch status.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime_api.h>
+
+#include "frt.h"
+
+namespace frt {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline bool valid_dtype(frt_dtype dt) { return dt == FRT_F16 || dt == FRT_BF16; }
+inline bool valid_quant(frt_quant q) { return q == FRT_QUANT_STATIC || q == FRT_QUANT_BLOCK128; }
+
+// Status of the launch just issued on this thread.
+inline frt_status launch_status() { return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA; }
+
+// Checks shared by the two FP8-producing ops: the pointer the quant mode needs.
+inline bool quant_args_ok(frt_quant qm, const float* static_scale, const float* block_scales) {
+  if (qm == FRT_QUANT_STATIC) return static_scale != nullptr && aligned(static_scale, 4);
+  return block_scales != nullptr && aligned(block_scales, 4);
+}
+
+}  // namespace frt

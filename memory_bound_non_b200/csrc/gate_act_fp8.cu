@@ -1,0 +1,172 @@
+// Op (c): gated activation on an interleaved gate/up buffer + FP8 e4m3.
+//
+// "Falcon-Perception inference optimisation", third technique: gate and up
+// come out of one GEMM interleaved as [g0,u0,g1,u1,...]; one kernel reads each
+// adjacent pair, forms act(g) * u and writes once, so the [M, 2I] transient is
+// read once and the output is half its width.  "FlashRT kernel fusion", §二
+// steps 8-10 and "sm89 prefill FFN megakernel", Phase 2 add the FP8 quant
+// (static, or per-token block-128 scales) to the same pass.
+//
+// Mapping (B200): a 16-byte load holds 4 (g, u) pairs -> 4 outputs -> one
+// 32-bit store of 4 codes, so one warp-wide load covers exactly one 128-column
+// scale block (512 contiguous input bytes, 128 output bytes) and the block's
+// amax is a 5-step xor shuffle.  Each warp owns U consecutive blocks of the
+// flattened (row, block) index space and issues all U loads before computing,
+// which keeps enough bytes in flight per SM to saturate HBM.
+#include <cmath>
+
+#include "frt_device.cuh"
+#include "frt_host.h"
+
+namespace frt {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kU = 4;  // scale blocks per warp
+
+constexpr float kSqrt2OverPi = 0.7978845608028654f;
+constexpr float kGeluCubic = 0.044715f;
+
+// act(g) in fp32.  GELU-tanh uses 0.5 (1 + tanh(z)) = 1 / (1 + exp(-2 z)) and
+// SiLU is g / (1 + exp(-g)); the exponent is capped at 80 so the denominator
+// stays finite (the result is ~0 there either way).
+template <int ACT>
+__device__ __forceinline__ float act_fn(float g) {
+  if (ACT == FRT_ACT_RELU2) {
+    const float r = fmaxf(g, 0.0f);
+    return r * r;
+  } else if (ACT == FRT_ACT_SILU) {
+    const float e = expf(fminf(-g, 80.0f));
+    return __fdividef(g, 1.0f + e);
+  } else {
+    const float z = g * fmaf(kSqrt2OverPi * kGeluCubic, g * g, kSqrt2OverPi);
+    const float e = expf(fminf(-2.0f * z, 80.0f));
+    return __fdividef(g, 1.0f + e);
+  }
+}
+
+template <int DT, int ACT, int QM>
+__global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __restrict__ gu,
+                                                                 uint32_t* __restrict__ q,
+                                                                 const float* __restrict__ static_scale,
+                                                                 float* __restrict__ block_scales,
+                                                                 int64_t total_blocks, int NB, int C4) {
+  using P16 = Pack16<DT>;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int64_t gb0 = warp * kU;
+
+  // Load phase: chunk `lane` of each of the U blocks (4 outputs = 16 bytes).
+  uint4 v[kU];
+  int64_t idx[kU];
+  bool valid[kU];
+  int64_t row = gb0 / NB;
+  int b = (int)(gb0 - row * NB);
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int chunk = b * 32 + lane;  // chunk index within the row (4 outputs each)
+    valid[u] = gb0 + u < total_blocks && chunk < C4;
+    idx[u] = row * C4 + chunk;       // same index for the input (uint4) and output (uint32) views
+    if (valid[u]) v[u] = ld_stream(gu + idx[u]);
+    if (++b == NB) {
+      b = 0;
+      ++row;
+    }
+  }
+
+  float inv_static = 0.0f, s_static = 0.0f;
+  bool div_static = false;
+  if (QM == FRT_QUANT_STATIC) {
+    s_static = __ldg(static_scale);
+    inv_static = 1.0f / s_static;
+    div_static = !(fabsf(inv_static) < INFINITY);
+  }
+
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (valid[u]) {
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 p = P16::to_float2(w[e]);  // (gate, up)
+        a[e] = act_fn<ACT>(p.x) * p.y;
+      }
+    }
+    float s, inv;
+    bool div;
+    if (QM == FRT_QUANT_BLOCK128) {
+      const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
+      if (am == 0.0f) {
+        s = 1.0f;
+        inv = 1.0f;
+        div = false;
+      } else {
+        s = am / 448.0f;
+        div = am < 0x1p-100f;
+        inv = div ? 0.0f : 448.0f / am;
+      }
+      const int64_t gb = gb0 + u;
+      if (lane == 0 && gb < total_blocks) block_scales[gb] = s;  // [M, NB] row-major == flat block index
+    } else {
+      s = s_static;
+      inv = inv_static;
+      div = div_static;
+    }
+    if (valid[u]) {
+      float o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = div ? __fdiv_rn(a[e], s) : a[e] * inv;
+      q[idx[u]] = e4m3x4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+template <int DT, int ACT>
+void launch_act(frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total, int NB,
+                int C4, cudaStream_t st) {
+  const int64_t warps = (total + kU - 1) / kU;
+  const unsigned grid = (unsigned)((warps + kWarps - 1) / kWarps);
+  if (qm == FRT_QUANT_STATIC)
+    gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC><<<grid, kThreads, 0, st>>>(
+        static_cast<const uint4*>(gu), reinterpret_cast<uint32_t*>(q), ss, bs, total, NB, C4);
+  else
+    gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128><<<grid, kThreads, 0, st>>>(
+        static_cast<const uint4*>(gu), reinterpret_cast<uint32_t*>(q), ss, bs, total, NB, C4);
+}
+
+template <int DT>
+void launch_dt(frt_act act, frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total,
+               int NB, int C4, cudaStream_t st) {
+  switch (act) {
+    case FRT_ACT_GELU_TANH: launch_act<DT, FRT_ACT_GELU_TANH>(qm, gu, q, ss, bs, total, NB, C4, st); break;
+    case FRT_ACT_SILU: launch_act<DT, FRT_ACT_SILU>(qm, gu, q, ss, bs, total, NB, C4, st); break;
+    default: launch_act<DT, FRT_ACT_RELU2>(qm, gu, q, ss, bs, total, NB, C4, st); break;
+  }
+}
+
+}  // namespace
+}  // namespace frt
+
+extern "C" frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* static_scale,
+                                       float* block_scales, int M, int I, frt_act act, frt_dtype dt, frt_quant qm,
+                                       cudaStream_t stream) {
+  using namespace frt;
+  if (M < 0 || I <= 0 || I % 4 != 0) return FRT_ERR_INVALID_ARG;
+  if (!valid_dtype(dt) || !valid_quant(qm)) return FRT_ERR_INVALID_ARG;
+  if (act != FRT_ACT_GELU_TANH && act != FRT_ACT_SILU && act != FRT_ACT_RELU2) return FRT_ERR_INVALID_ARG;
+  if (!gate_up || !out_fp8 || !aligned(gate_up, 16) || !aligned(out_fp8, 4)) return FRT_ERR_INVALID_ARG;
+  if (!quant_args_ok(qm, static_scale, block_scales)) return FRT_ERR_INVALID_ARG;
+  if (M == 0) return FRT_OK;
+  const int NB = (I + 127) / 128;
+  const int C4 = I / 4;
+  const int64_t total = (int64_t)M * NB;
+  const int64_t grid = (total + (int64_t)kU * kWarps - 1) / ((int64_t)kU * kWarps);
+  if (grid > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
+  if (dt == FRT_F16)
+    launch_dt<FRT_F16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
+  else
+    launch_dt<FRT_BF16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
+  return launch_status();
+}

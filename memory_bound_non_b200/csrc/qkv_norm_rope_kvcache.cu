@@ -1,0 +1,240 @@
+// Op (b): packed-QKV split + per-head q/k RMSNorm + rotate-half RoPE + Q staging
+// write + KV-cache write, one pass over the QKV GEMM output.
+//
+// "FlashRT kernel fusion", §2.2 first bullet: q_norm -> RoPE -> write Q staging
+// and k_norm -> RoPE -> write KV cache in one kernel, V passing straight
+// through (replacing ~16 small ops per layer); second bullet: the rotate_half
+// pair (j, j + hd/2) is kept in one lane, so RoPE needs no warp shuffle; §二
+// step 3: split + RoPE + KV write with no q/k norm.
+//
+// Mapping (B200): a group of GP lanes (power of two) owns one (token, head)
+// unit; lane l holds elements [lP, lP+P) and their RoPE partners
+// [hd/2 + lP, ...), P = 8 (16-byte vectors) when hd % 16 == 0, else P = 4
+// (8-byte vectors; e.g. the unpadded head_dim 72 of the ViT).  The per-head
+// sum of squares is an xor shuffle inside the group; cos/sin rows are shared
+// by all heads of a token and come from L1.  Every unit is independent, so the
+// grid is simply (tokens x heads x GP) threads.
+#include <cmath>
+
+#include "frt_device.cuh"
+#include "frt_host.h"
+
+namespace frt {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <int P>
+struct Vec16;
+template <>
+struct Vec16<8> {
+  using T = uint4;
+};
+template <>
+struct Vec16<4> {
+  using T = uint2;
+};
+
+template <int P>
+__device__ __forceinline__ typename Vec16<P>::T ld_vec(const uint16_t* p) {
+  return *reinterpret_cast<const typename Vec16<P>::T*>(p);
+}
+
+template <int DT, int P>
+__device__ __forceinline__ void unpack(const typename Vec16<P>::T& v, float* f) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+  for (int e = 0; e < P / 2; ++e) {
+    const float2 t = Pack16<DT>::to_float2(w[e]);
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+
+template <int DT, int P>
+__device__ __forceinline__ void store_packed(uint16_t* dst, const float* f) {
+  typename Vec16<P>::T v;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+  for (int e = 0; e < P / 2; ++e) w[e] = Pack16<DT>::from_float2(f[2 * e], f[2 * e + 1]);
+  *reinterpret_cast<typename Vec16<P>::T*>(dst) = v;
+}
+
+template <int P>
+__device__ __forceinline__ void ld_f32(const float* p, float* f) {
+#pragma unroll
+  for (int e = 0; e < P; e += 4) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(p + e));
+    f[e] = t.x;
+    f[e + 1] = t.y;
+    f[e + 2] = t.z;
+    f[e + 3] = t.w;
+  }
+}
+
+template <int DT, int P, int GP>
+__global__ void __launch_bounds__(kThreads) qkv_norm_rope_kvcache_kernel(
+    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
+    const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
+    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, uint16_t* __restrict__ k_cache,
+    uint16_t* __restrict__ v_cache, int32_t* status, int64_t units, int H, int Hq, int Hkv, int hd, int G,
+    int max_pos, int capacity, float eps) {
+  const int64_t gt = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  const int64_t unit = gt / GP;
+  const int li = threadIdx.x & (GP - 1);
+  const bool in_range = unit < units;
+  const int64_t tok = in_range ? unit / H : 0;
+  const int h = in_range ? (int)(unit - tok * H) : 0;
+
+  int p = 0;
+  bool row_ok = false;
+  if (in_range) {
+    p = __ldg(positions + tok);
+    row_ok = p >= 0 && p < max_pos && p < capacity;
+    if (!row_ok && h == 0 && li == 0 && status != nullptr) atomicOr(status, 1);
+  }
+  const bool active = row_ok && li < G;
+  const int half = hd >> 1;
+  const int j0 = li * P;
+  const bool is_q = h < Hq;
+  const bool is_v = h >= Hq + Hkv;
+  const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
+  const bool do_norm = !is_v && nw != nullptr;
+
+  const uint16_t* src = qkv + tok * (int64_t)H * hd + (int64_t)h * hd;
+  typename Vec16<P>::T va, vb;
+  if (active) {
+    va = *reinterpret_cast<const typename Vec16<P>::T*>(src + j0);
+    vb = *reinterpret_cast<const typename Vec16<P>::T*>(src + half + j0);
+  }
+
+  if (is_v) {  // V: bit copy into the cache slot
+    if (active) {
+      uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
+      *reinterpret_cast<typename Vec16<P>::T*>(dst + j0) = va;
+      *reinterpret_cast<typename Vec16<P>::T*>(dst + half + j0) = vb;
+    }
+  }
+
+  float a[P], b[P];
+  float ss = 0.0f;
+  if (active && !is_v) {
+    unpack<DT, P>(va, a);
+    unpack<DT, P>(vb, b);
+    if (do_norm) {
+#pragma unroll
+      for (int e = 0; e < P; ++e) ss = fmaf(b[e], b[e], fmaf(a[e], a[e], ss));
+    }
+  }
+  ss = group_sum<GP>(ss);  // every lane of the warp takes part
+
+  if (active && !is_v) {
+    if (do_norm) {
+      const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
+      float wa[P], wb[P];
+      unpack<DT, P>(ld_vec<P>(nw + j0), wa);
+      unpack<DT, P>(ld_vec<P>(nw + half + j0), wb);
+#pragma unroll
+      for (int e = 0; e < P; ++e) {
+        a[e] = a[e] * rstd * wa[e];
+        b[e] = b[e] * rstd * wb[e];
+      }
+    }
+    float c[P], s[P];
+    ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
+    ld_f32<P>(sin_tab + (int64_t)p * half + j0, s);
+    float o1[P], o2[P];
+#pragma unroll
+    for (int e = 0; e < P; ++e) {
+      o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
+      o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
+    }
+    uint16_t* dst = is_q ? q_out + (tok * Hq + h) * (int64_t)hd
+                         : k_cache + ((int64_t)p * Hkv + (h - Hq)) * hd;
+    store_packed<DT, P>(dst + j0, o1);
+    store_packed<DT, P>(dst + half + j0, o2);
+  }
+}
+
+struct Args {
+  const void* qkv;
+  const void* qw;
+  const void* kw;
+  const float* cos_tab;
+  const float* sin_tab;
+  const int32_t* pos;
+  void* q_out;
+  void* kc;
+  void* vc;
+  int32_t* status;
+  int64_t units;
+  int H, Hq, Hkv, hd, G, max_pos, capacity;
+  float eps;
+};
+
+template <int DT, int P, int GP>
+void launch_gp(const Args& a, cudaStream_t st) {
+  const int64_t threads = a.units * GP;
+  const unsigned grid = (unsigned)((threads + kThreads - 1) / kThreads);
+  qkv_norm_rope_kvcache_kernel<DT, P, GP><<<grid, kThreads, 0, st>>>(
+      static_cast<const uint16_t*>(a.qkv), static_cast<const uint16_t*>(a.qw), static_cast<const uint16_t*>(a.kw),
+      a.cos_tab, a.sin_tab, a.pos, static_cast<uint16_t*>(a.q_out), static_cast<uint16_t*>(a.kc),
+      static_cast<uint16_t*>(a.vc), a.status, a.units, a.H, a.Hq, a.Hkv, a.hd, a.G, a.max_pos, a.capacity,
+      a.eps);
+}
+
+template <int DT, int P>
+void launch_p(int GP, const Args& a, cudaStream_t st) {
+  switch (GP) {
+    case 1: launch_gp<DT, P, 1>(a, st); break;
+    case 2: launch_gp<DT, P, 2>(a, st); break;
+    case 4: launch_gp<DT, P, 4>(a, st); break;
+    case 8: launch_gp<DT, P, 8>(a, st); break;
+    case 16: launch_gp<DT, P, 16>(a, st); break;
+    default: launch_gp<DT, P, 32>(a, st); break;
+  }
+}
+
+template <int DT>
+void launch_dt(int P, int GP, const Args& a, cudaStream_t st) {
+  if (P == 8)
+    launch_p<DT, 8>(GP, a, st);
+  else
+    launch_p<DT, 4>(GP, a, st);
+}
+
+}  // namespace
+}  // namespace frt
+
+extern "C" frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_norm_w, const void* k_norm_w,
+                                                const float* cos_tab, const float* sin_tab,
+                                                const int32_t* positions, void* q_out, void* k_cache,
+                                                void* v_cache, int32_t* status, int M, int Hq, int Hkv, int hd,
+                                                int max_pos, int capacity, float eps, frt_dtype dt,
+                                                cudaStream_t stream) {
+  using namespace frt;
+  if (M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || hd <= 0 || hd % 2 != 0) return FRT_ERR_INVALID_ARG;
+  if (max_pos <= 0 || capacity <= 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
+  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
+  if (hd % 8 != 0 || hd > 256) return FRT_ERR_UNSUPPORTED;
+  const int P = (hd % 16 == 0) ? 8 : 4;
+  const uintptr_t al = (P == 8) ? 16 : 8;
+  if (!aligned(qkv, al) || !aligned(q_out, al) || !aligned(k_cache, al) || !aligned(v_cache, al))
+    return FRT_ERR_INVALID_ARG;
+  if ((q_norm_w && !aligned(q_norm_w, al)) || (k_norm_w && !aligned(k_norm_w, al))) return FRT_ERR_INVALID_ARG;
+  if (!aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(positions, 4)) return FRT_ERR_INVALID_ARG;
+  if (status && !aligned(status, 4)) return FRT_ERR_INVALID_ARG;
+  if (M == 0) return FRT_OK;
+  const int H = Hq + 2 * Hkv;
+  const int G = (hd / 2) / P;  // active lanes per head, <= 31
+  int GP = 1;
+  while (GP < G) GP *= 2;
+  Args a{qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status,
+         (int64_t)M * H, H, Hq, Hkv, hd, G, max_pos, capacity, eps};
+  if ((a.units * GP + kThreads - 1) / kThreads > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
+  if (dt == FRT_F16)
+    launch_dt<FRT_F16>(P, GP, a, stream);
+  else
+    launch_dt<FRT_BF16>(P, GP, a, stream);
+  return launch_status();
+}

@@ -5,8 +5,11 @@ sets and the precomputed RoPE cos/sin table that a caller hands to the op.  It
 holds none of the ops' arithmetic, so the CUDA path and the CPU oracle can
 both consume exactly the same host buffers.
 
-Every tensor is drawn on the host from ``torch.Generator('cpu')`` with a
-stated seed.  The shapes follow the workloads of the source pages:
+Every tensor is drawn from a seeded ``torch.Generator``: on the host
+(``device="cpu"``, the default, used for every case the oracle checks in
+full) or, for the multi-GB large-M workloads, on the GPU (``device="cuda"``;
+the same recipe and seed, a different stream of numbers), with host copies
+taken for the oracle.  The shapes follow the workloads of the source pages:
   * a Pi0.5-like action decoder (M=10 tokens; 18 layers x 10 flow steps),
   * a Qwen3-style text prefill (S = 128..1024, q/k norm, block-128 FP8),
   * a VLA denoise step (M=41, 32 layers x 10 steps) and its ViT (M=1176,
@@ -99,8 +102,8 @@ def get(name: str, **overrides) -> Workload:
 
 
 # ------------------------------------------------------------ primitives --
-def generator(seed: int) -> torch.Generator:
-    g = torch.Generator("cpu")
+def generator(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device)
     g.manual_seed(int(seed))
     return g
 
@@ -111,13 +114,13 @@ def normal16(shape: Tuple[int, ...], dt: str, g: torch.Generator, scale: float =
 
     col_mult (float32 [shape[-1]]) multiplies columns before the rounding (used
     for the outlier channels)."""
-    out = torch.empty(shape, dtype=DTYPES[dt])
+    out = torch.empty(shape, dtype=DTYPES[dt], device=g.device)
     flat = out.view(-1, shape[-1]) if len(shape) > 1 else out.view(1, -1)
     rows = flat.shape[0]
     step = max(1, _CHUNK_ELEMS // max(1, flat.shape[1]))
     for r0 in range(0, rows, step):
         r1 = min(rows, r0 + step)
-        t = torch.randn((r1 - r0, flat.shape[1]), generator=g, dtype=torch.float32)
+        t = torch.randn((r1 - r0, flat.shape[1]), generator=g, dtype=torch.float32, device=g.device)
         if scale != 1.0:
             t.mul_(scale)
         if col_mult is not None:
@@ -128,7 +131,7 @@ def normal16(shape: Tuple[int, ...], dt: str, g: torch.Generator, scale: float =
 
 def norm_weight(n: int, dt: str, g: torch.Generator) -> torch.Tensor:
     """A norm weight ~ 1 + 0.1 N(0, 1) (any +1 of the model already included)."""
-    t = torch.randn((n,), generator=g, dtype=torch.float32).mul_(0.1).add_(1.0)
+    t = torch.randn((n,), generator=g, dtype=torch.float32, device=g.device).mul_(0.1).add_(1.0)
     return t.to(DTYPES[dt])
 
 
@@ -137,8 +140,8 @@ def outlier_multipliers(n: int, frac: float, mult: float, g: torch.Generator) ->
     if frac <= 0.0:
         return None
     k = max(1, math.ceil(frac * n))
-    idx = torch.randperm(n, generator=g)[:k]
-    m = torch.ones(n, dtype=torch.float32)
+    idx = torch.randperm(n, generator=g, device=g.device)[:k]
+    m = torch.ones(n, dtype=torch.float32, device=g.device)
     m[idx] = mult
     return m
 
@@ -157,9 +160,9 @@ def rope_tables(max_pos: int, hd: int, theta: float) -> Tuple[torch.Tensor, torc
 
 def positions(wl: Workload, g: torch.Generator) -> torch.Tensor:
     if wl.positions == "range":
-        return torch.arange(wl.pos_start, wl.pos_start + wl.M, dtype=torch.int32)
+        return torch.arange(wl.pos_start, wl.pos_start + wl.M, dtype=torch.int32, device=g.device)
     # unique slots sampled without replacement from the whole cache
-    return torch.randperm(wl.capacity, generator=g)[: wl.M].to(torch.int32)
+    return torch.randperm(wl.capacity, generator=g, device=g.device)[: wl.M].to(torch.int32)
 
 
 # ---------------------------------------------------------------- inputs --
@@ -188,16 +191,18 @@ class Inputs:
     layers: list = field(default_factory=list)
 
 
-def make_inputs(wl: Workload, n_layers: Optional[int] = None, with_caches: bool = True) -> Inputs:
-    """All host inputs for ``n_layers`` (default wl.layers) distinct layers."""
-    g = generator(wl.seed)
+def make_inputs(wl: Workload, n_layers: Optional[int] = None, with_caches: bool = True,
+                device="cpu") -> Inputs:
+    """All inputs for ``n_layers`` (default wl.layers) distinct layers, drawn
+    on ``device``."""
+    g = generator(wl.seed, device)
     L = wl.layers if n_layers is None else n_layers
     col_d = outlier_multipliers(wl.D, wl.outlier_frac, wl.outlier_mult, g)
     col_i = outlier_multipliers(wl.I, wl.outlier_frac, wl.outlier_mult, g)
     col_gu = None if col_i is None else col_i.repeat_interleave(2)  # scale g and u of a channel
     residual = normal16((wl.M, wl.D), wl.dt, g, col_mult=col_d)
     pos = positions(wl, g)
-    cos, sin = rope_tables(wl.max_pos, wl.hd, wl.theta)
+    cos, sin = (t.to(g.device) for t in rope_tables(wl.max_pos, wl.hd, wl.theta))
     inp = Inputs(wl=wl, residual=residual, positions=pos, cos=cos, sin=sin)
     for _ in range(L):
         x_attn = normal16((wl.M, wl.D), wl.dt, g, col_mult=col_d)
@@ -209,8 +214,8 @@ def make_inputs(wl: Workload, n_layers: Optional[int] = None, with_caches: bool 
         kw = norm_weight(wl.hd, wl.dt, g) if wl.qk_norm else None
         gate_up = normal16((wl.M, 2 * wl.I), wl.dt, g, col_mult=col_gu)
         if with_caches:
-            kc = torch.empty((wl.capacity, wl.Hkv, wl.hd), dtype=DTYPES[wl.dt])
-            vc = torch.empty((wl.capacity, wl.Hkv, wl.hd), dtype=DTYPES[wl.dt])
+            kc = torch.empty((wl.capacity, wl.Hkv, wl.hd), dtype=DTYPES[wl.dt], device=g.device)
+            vc = torch.empty((wl.capacity, wl.Hkv, wl.hd), dtype=DTYPES[wl.dt], device=g.device)
             if wl.prefill > 0:  # earlier tokens already in the cache
                 kc[: wl.prefill] = normal16((wl.prefill, wl.Hkv, wl.hd), wl.dt, g)
                 vc[: wl.prefill] = normal16((wl.prefill, wl.Hkv, wl.hd), wl.dt, g)
@@ -224,6 +229,6 @@ def make_inputs(wl: Workload, n_layers: Optional[int] = None, with_caches: bool 
 
 
 def bits16(t: torch.Tensor):
-    """uint16 numpy view of a 16-bit CPU tensor (for the oracle)."""
+    """uint16 numpy bits of a 16-bit tensor, copied to the host (for the oracle)."""
     import numpy as np
-    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)

@@ -1,0 +1,94 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/frt.h declares, and rejects bad arguments on the host before any CUDA
+call (fake, never-dereferenced pointers)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import memory_bound_non_b200 as frt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+A = 0x100000          # a 256-byte aligned fake device address (never dereferenced)
+INV, UNSUP, OK = frt.FRT_ERR_INVALID_ARG, frt.FRT_ERR_UNSUPPORTED, frt.FRT_OK
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "frt.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(frt_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = frt.load()
+    names = declared_functions()
+    assert set(names) == set(frt.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for s in (OK, INV, UNSUP, frt.FRT_ERR_CUDA, 99):
+        assert isinstance(frt.status_string(s), str) and frt.status_string(s)
+
+
+def a_call(M=4, D=256, x=A, r=A, ro=A, w=None, q=A, ss=A, bs=None, dt=1, qm=0):
+    return frt.load().frt_residual_rmsnorm_fp8(x, r, ro, w, q, ss, bs, M, D, 1e-6, dt, qm, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=-1), INV), (dict(D=0), INV), (dict(D=12), INV), (dict(x=None), INV), (dict(ro=None), INV),
+    (dict(q=None), INV), (dict(x=A + 8), INV), (dict(r=A + 4), INV), (dict(q=A + 4), INV),
+    (dict(w=A + 2), INV), (dict(ss=None), INV), (dict(qm=1, bs=None), INV), (dict(dt=2), INV),
+    (dict(qm=5), INV), (dict(D=32776), UNSUP), (dict(M=0), OK), (dict(M=0, qm=1, bs=A), OK),
+])
+def test_residual_rmsnorm_host_validation(kw, want):
+    assert a_call(**kw) == want
+
+
+def b_call(M=4, Hq=8, Hkv=2, hd=128, qkv=A, cos=A, sin=A, pos=A, qo=A, kc=A, vc=A, qw=None, kw=None,
+           status=None, max_pos=64, cap=64, dt=1):
+    return frt.load().frt_qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, qo, kc, vc, status, M, Hq, Hkv, hd,
+                                                max_pos, cap, 1e-6, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=-3), INV), (dict(Hq=0), INV), (dict(Hkv=0), INV), (dict(Hq=6, Hkv=4), INV), (dict(hd=7), INV),
+    (dict(hd=0), INV), (dict(hd=6), UNSUP), (dict(hd=12), UNSUP), (dict(hd=264), UNSUP),
+    (dict(max_pos=0), INV), (dict(cap=0), INV), (dict(qkv=None), INV), (dict(cos=None), INV),
+    (dict(pos=None), INV), (dict(kc=None), INV), (dict(qkv=A + 8), INV), (dict(hd=72, qkv=A + 8, M=0), OK),
+    (dict(hd=72, qkv=A + 4), INV), (dict(cos=A + 8), INV), (dict(pos=A + 2), INV), (dict(status=A + 1), INV),
+    (dict(qw=A + 8), INV), (dict(dt=9), INV), (dict(M=0), OK),
+])
+def test_qkv_host_validation(kw, want):
+    assert b_call(**kw) == want
+
+
+def c_call(M=4, I=256, gu=A, q=A, ss=A, bs=None, act=0, dt=1, qm=0):
+    return frt.load().frt_gate_act_fp8(gu, q, ss, bs, M, I, act, dt, qm, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=-1), INV), (dict(I=0), INV), (dict(I=6), INV), (dict(act=3), INV), (dict(act=-1), INV),
+    (dict(gu=None), INV), (dict(gu=A + 8), INV), (dict(q=A + 2), INV), (dict(ss=None), INV),
+    (dict(qm=1, bs=None), INV), (dict(qm=1, bs=A + 2), INV), (dict(dt=3), INV), (dict(M=0), OK),
+    (dict(M=0, I=4, qm=1, bs=A), OK),
+])
+def test_gate_act_host_validation(kw, want):
+    assert c_call(**kw) == want
+
+
+def test_noop_host_validation():
+    L = frt.load()
+    assert L.frt_noop(0, 32, None) == INV
+    assert L.frt_noop(1, 0, None) == INV
+    assert L.frt_noop(1, 1025, None) == INV
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    x = torch.zeros(2, 8, dtype=torch.bfloat16)
+    with pytest.raises(frt.FrtError):
+        frt.frt_residual_rmsnorm_fp8(x, x, x, None, torch.zeros(2, 8, dtype=torch.uint8),
+                                     static_scale=torch.ones(1))

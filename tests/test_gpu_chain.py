@@ -1,0 +1,73 @@
+"""GPU parity of the graphed layer chain: layers x steps invocations of
+a -> b -> a -> c captured in one CUDA graph, against the oracle replaying the
+same sequence (residual carried in place from one invocation to the next)."""
+import numpy as np
+import pytest
+import torch
+
+import parity as P
+from memory_bound_non_b200 import workloads as W
+from memory_bound_non_b200.chain import LayerChain
+
+pytestmark = pytest.mark.gpu
+
+
+def compare_chain(wl, inp, chain, r_ref, outs):
+    np.testing.assert_array_equal(P.np16(chain.residual), r_ref)
+    assert int(chain.status.item()) == 0
+    for l, (L, o) in enumerate(zip(chain.layers, outs)):
+        P.assert_fp8_codes(L.q8_attn.cpu().numpy(), o["a1"]["out_fp8"], what="layer %d attn fp8" % l)
+        P.assert_fp8_codes(L.q8_ffn.cpu().numpy(), o["a2"]["out_fp8"], what="layer %d ffn fp8" % l)
+        P.assert_fp8_codes(L.act8.cpu().numpy(), o["c"]["out_fp8"], what="layer %d act fp8" % l)
+        if wl.quant == "block128":
+            P.assert_scales_close(L.bs_attn.cpu().numpy(), o["a1"]["block_scales"])
+            P.assert_scales_close(L.bs_act.cpu().numpy(), o["c"]["block_scales"])
+        P.assert_16bit_close(P.decode16(L.q_out), o["b"]["q_out"], what="layer %d Q" % l)
+        written = ~np.isnan(o["b"]["k_cache"]).all(axis=(1, 2))
+        P.assert_16bit_close(P.decode16(L.k_cache)[written], o["b"]["k_cache"][written], what="layer %d K" % l)
+        np.testing.assert_array_equal(P.np16(L.v_cache), o["b"]["v_cache"])
+        k0 = W.bits16(inp.layers[l].k_cache)
+        np.testing.assert_array_equal(P.np16(L.k_cache)[~written], k0[~written])
+
+
+@pytest.mark.parametrize("name,steps", [("pi05", 10), ("vla_denoise", 10), ("tiny", 3),
+                                        ("qwen3_prefill_S128", 2)])
+def test_graphed_chain_matches_oracle(name, steps):
+    wl = W.get(name, steps=steps, layers=max(W.get(name).layers, 2))
+    inp = W.make_inputs(wl)
+    scales = P.chain_scales(wl, inp)
+    chain = LayerChain(wl, inp, scales=scales)
+    chain.capture()
+    chain.reset()
+    chain.replay()
+    torch.cuda.synchronize()
+    r_ref, outs = P.oracle_chain(wl, inp, scales, steps)
+    compare_chain(wl, inp, chain, r_ref, outs)
+
+
+def test_graph_replay_equals_stream_launches_and_is_bitwise_repeatable():
+    wl = W.get("pi05", steps=3)
+    inp = W.make_inputs(wl)
+    chain = LayerChain(wl, inp, scales=P.chain_scales(wl, inp))
+    chain.reset()
+    chain.run()
+    torch.cuda.synchronize()
+    eager = [t.clone() for L in chain.layers for t in (L.q8_attn, L.q8_ffn, L.act8, L.q_out, L.k_cache)]
+    r_eager = chain.residual.clone()
+    chain.capture()
+    for _ in range(5):  # five replays from the same start: bit-identical
+        chain.reset()
+        chain.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(chain.residual, r_eager)
+        got = [t for L in chain.layers for t in (L.q8_attn, L.q8_ffn, L.act8, L.q_out, L.k_cache)]
+        assert all(torch.equal(a, b) for a, b in zip(eager, got))
+
+
+def test_calibrated_static_scales_match_oracle_calibration():
+    wl = W.get("pi05")
+    inp = W.make_inputs(wl, n_layers=1)
+    chain = LayerChain(wl, inp)
+    got = chain.calibrate_static_scales().cpu().numpy()
+    want = np.array(P.chain_scales(wl, inp))
+    np.testing.assert_allclose(got, want, rtol=1e-6)
