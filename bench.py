@@ -186,6 +186,7 @@ def time_graph(graph, reps, flush_buf, stream):
 
 # ------------------------------------------------------------- GPU legs --
 def launch_floor(reps=2000):
+    """Empty-kernel floor, with the library's current PDL setting."""
     import memory_bound_non_b200 as frt
     s = torch.cuda.current_stream()
     for _ in range(50):
@@ -530,10 +531,15 @@ def main(argv=None):
 
     extra = {}
     if rank == 0 and not args.no_chain:
-        floor = launch_floor()
-        extra["launch_floor"] = {k: (round(v, 3) if isinstance(v, float) else v) for k, v in floor.items()}
-        extra["chain"] = chain_leg(args.chain_reps, floor)
-        extra["small_m"] = small_m_ops(floor)
+        pdl0 = frt.frt_get_pdl()
+        for pdl in (True, False):
+            frt.frt_set_pdl(pdl)
+            tag = "" if pdl else "_no_pdl"
+            floor = launch_floor()
+            extra["launch_floor" + tag] = {k: (round(v, 3) if isinstance(v, float) else v) for k, v in floor.items()}
+            extra["chain" + tag] = chain_leg(args.chain_reps, floor)
+            extra["small_m" + tag] = small_m_ops(floor)
+        frt.frt_set_pdl(pdl0)
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_leg(step, args.e2e_steps, 1)

@@ -27,7 +27,9 @@
  *                           op);
  *      FRT_ERR_CUDA         the launch itself failed (cudaGetLastError after
  *                           the launch).
- *  - M == 0 is an empty batch: the call returns FRT_OK and launches nothing.
+ *  - M == 0 is an empty batch: once the sizes and enum values pass their
+ *    checks the call returns FRT_OK and launches nothing; pointers are not
+ *    inspected (an empty tensor may have a NULL data pointer).
  *  - Device-side data errors never trap: see the status word of op (b).
  *  - 16-bit tensors are fp16 or bf16 as selected by `dt`; all layouts are
  *    row-major and contiguous.  e4m3 is OCP FP8 E4M3 ("fn": max 448, no inf).
@@ -176,6 +178,19 @@ frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* 
  * Returns FRT_ERR_INVALID_ARG for grid < 1 or block outside [1, 1024].
  */
 frt_status frt_noop(int grid, int block, cudaStream_t stream);
+
+/*
+ * Programmatic dependent launch (PDL), on by default.  With it on, every
+ * kernel of this library is launched with programmatic stream serialisation:
+ * the GPU may schedule it while the previous kernel of the same stream is
+ * still running (hiding launch latency, e.g. between the nodes of a CUDA
+ * graph), and the kernel waits for that previous kernel to complete, with its
+ * writes visible, before it touches memory (griddepcontrol.wait).  Results are
+ * identical either way.  The switch is process-wide and read at each launch;
+ * changing it while another thread launches affects only later launches.
+ */
+void frt_set_pdl(int enable);
+int frt_get_pdl(void);
 
 /* Static, NUL-terminated description of a status value; never NULL. */
 const char* frt_status_string(frt_status status);

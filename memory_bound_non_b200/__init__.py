@@ -26,7 +26,7 @@ ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
 
 # C entry points declared in include/frt.h
 EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8", "frt_noop",
-           "frt_status_string")
+           "frt_set_pdl", "frt_get_pdl", "frt_status_string")
 
 
 class FrtError(RuntimeError):
@@ -56,6 +56,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_gate_act_fp8.restype = i32
     L.frt_noop.argtypes = [i32, i32, vp]
     L.frt_noop.restype = i32
+    L.frt_set_pdl.argtypes = [i32]
+    L.frt_set_pdl.restype = None
+    L.frt_get_pdl.argtypes = []
+    L.frt_get_pdl.restype = i32
     L.frt_status_string.argtypes = [i32]
     L.frt_status_string.restype = c.c_char_p
     _lib = L
@@ -121,6 +125,15 @@ def frt_gate_act_fp8(gate_up, out_fp8, static_scale=None, block_scales=None, act
     st = load().frt_gate_act_fp8(_ptr(gate_up), _ptr(out_fp8), _ptr(static_scale), _ptr(block_scales), M,
                                  two_i // 2, ACT[act], DTYPE[gate_up.dtype], QUANT[quant], _stream(stream))
     _check("frt_gate_act_fp8", st)
+
+
+def frt_set_pdl(enable: bool):
+    """Programmatic dependent launch on/off for every later launch (process-wide)."""
+    load().frt_set_pdl(1 if enable else 0)
+
+
+def frt_get_pdl() -> bool:
+    return bool(load().frt_get_pdl())
 
 
 def frt_noop(grid=1, block=32, stream=None):

@@ -11,6 +11,15 @@
 
 namespace frt {
 
+// ------------------------------------------------------------------ PDL --
+// Every kernel starts with these two: wait until the grid this launch depends
+// on has completed and its writes are visible (a no-op without a programmatic
+// dependency), then let the next launch of the stream be scheduled early.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 // -------------------------------------------------------------- 16-bit --
 // Two 16-bit values packed in one 32-bit word, element 0 in the low half.
 template <int DT>
@@ -57,6 +66,83 @@ __device__ __forceinline__ float add_round_odd(float a, float b) {
   }
   return __uint_as_float(u);
 }
+
+// Knuth's TwoSum: a + b == s + e exactly (fp32, round to nearest).
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+  s = __fadd_rn(a, b);
+  const float bb = __fsub_rn(s, a);
+  e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
+}
+
+// Compensated (hi, lo) accumulator: hi + lo tracks the exact sum of the
+// added terms to ~2^-48 relative.  Adding pairs is commutative bit for bit
+// (TwoSum's error term is the unique exact error), so an xor-butterfly gives
+// every lane the same pair.
+struct Sum2 {
+  float hi, lo;
+  __device__ __forceinline__ void add(float x) {
+    float s, e;
+    two_sum(hi, x, s, e);
+    hi = s;
+    lo = __fadd_rn(lo, e);
+  }
+  __device__ __forceinline__ void add(const Sum2& o) {
+    float s, e;
+    two_sum(hi, o.hi, s, e);
+    hi = s;
+    lo = __fadd_rn(__fadd_rn(lo, o.lo), e);
+  }
+};
+
+template <int WIDTH>
+__device__ __forceinline__ Sum2 group_sum2(Sum2 v) {
+#pragma unroll
+  for (int o = WIDTH / 2; o > 0; o >>= 1) {
+    Sum2 w;
+    w.hi = __shfl_xor_sync(0xFFFFFFFFu, v.hi, o);
+    w.lo = __shfl_xor_sync(0xFFFFFFFFu, v.lo, o);
+    v.add(w);
+  }
+  return v;
+}
+
+// fp32 scale factor r held as an unevaluated pair rhi + rlo (from an fp64
+// value).  mul_exact(x, r) = fp32 rounding of x * (rhi + rlo), computed with
+// an exact product (TwoProduct via FMA): correctly rounded unless the exact
+// product lies within ~2^-48 of an fp32 rounding boundary.
+struct Split32 {
+  float hi, lo;
+  __device__ __forceinline__ explicit Split32(double r) {
+    hi = __double2float_rn(r);
+    lo = __double2float_rn(r - (double)hi);
+  }
+  __device__ __forceinline__ float mul(float x) const {
+    const float p = x * hi;
+    const float e = fmaf(x, hi, -p);
+    return p + fmaf(x, lo, e);
+  }
+};
+
+// y / s rounded to nearest in fp32, from inv = RN(1/s): one FMA residual step
+// on the quotient estimate gives the correctly rounded quotient (Markstein's
+// theorem) while the quotient and the residual stay in the normal range.
+// Outside that range (tiny or huge scales, |y| < 2^-90, zeros) the IEEE
+// division is used instead.
+struct Divisor {
+  float s, inv;
+  bool fast;
+  __device__ __forceinline__ explicit Divisor(float s_) : s(s_) {
+    inv = __frcp_rn(s_);
+    const float a = fabsf(s_);
+    fast = a >= 0x1p-100f && a <= 0x1p+100f;
+  }
+  __device__ __forceinline__ float div(float y) const {
+    if (!fast || !(fabsf(y) >= 0x1p-90f)) return __fdiv_rn(y, s);  // also zeros: keeps -0
+    const float q = y * inv;
+    const float r = fmaf(-q, s, y);
+    return fmaf(r, inv, q);
+  }
+};
 
 // ----------------------------------------------------------------- FP8 --
 // Two fp32 -> two e4m3 codes (low byte = a), RNE, saturating to +-448.

@@ -3,6 +3,8 @@
 
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include <cuda_runtime_api.h>
 
 #include "frt.h"
@@ -16,6 +18,33 @@ inline bool valid_quant(frt_quant q) { return q == FRT_QUANT_STATIC || q == FRT_
 
 // Status of the launch just issued on this thread.
 inline frt_status launch_status() { return cudaGetLastError() == cudaSuccess ? FRT_OK : FRT_ERR_CUDA; }
+
+// Process-wide switch for programmatic dependent launch (frt_set_pdl).
+bool pdl_enabled();
+
+// Launch `kernel` on `stream`, with programmatic stream serialisation when
+// PDL is on: the kernel may then be scheduled while the previous kernel of the
+// stream still runs, and waits for it (griddepcontrol.wait) before its first
+// memory access.
+template <typename... KArgs, typename... Args>
+inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FRT_ERR_CUDA;
+  }
+  return launch_status();
+}
 
 // Checks shared by the two FP8-producing ops: the pointer the quant mode needs.
 inline bool quant_args_ok(frt_quant qm, const float* static_scale, const float* block_scales) {

@@ -1,17 +1,27 @@
 // Launch-floor probe and status strings.
 #include "frt_host.h"
 
+#include <atomic>
+
+#include "frt_device.cuh"
+
 namespace frt {
 namespace {
-__global__ void noop_kernel() {}
+__global__ void noop_kernel() { pdl_enter(); }
+std::atomic<int> g_pdl{1};
 }  // namespace
+
+bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
 }  // namespace frt
 
 extern "C" frt_status frt_noop(int grid, int block, cudaStream_t stream) {
   if (grid < 1 || block < 1 || block > 1024) return FRT_ERR_INVALID_ARG;
-  frt::noop_kernel<<<grid, block, 0, stream>>>();
-  return frt::launch_status();
+  return frt::launch(frt::noop_kernel, dim3(grid), dim3(block), stream);
 }
+
+extern "C" void frt_set_pdl(int enable) { frt::g_pdl.store(enable ? 1 : 0, std::memory_order_relaxed); }
+
+extern "C" int frt_get_pdl(void) { return frt::g_pdl.load(std::memory_order_relaxed); }
 
 extern "C" const char* frt_status_string(frt_status status) {
   switch (status) {

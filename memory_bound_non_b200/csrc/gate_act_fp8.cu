@@ -38,11 +38,11 @@ __device__ __forceinline__ float act_fn(float g) {
     return r * r;
   } else if (ACT == FRT_ACT_SILU) {
     const float e = expf(fminf(-g, 80.0f));
-    return __fdividef(g, 1.0f + e);
+    return Divisor(1.0f + e).div(g);
   } else {
     const float z = g * fmaf(kSqrt2OverPi * kGeluCubic, g * g, kSqrt2OverPi);
     const float e = expf(fminf(-2.0f * z, 80.0f));
-    return __fdividef(g, 1.0f + e);
+    return Divisor(1.0f + e).div(g);
   }
 }
 
@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
                                                                  float* __restrict__ block_scales,
                                                                  int64_t total_blocks, int NB, int C4) {
   using P16 = Pack16<DT>;
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t gb0 = warp * kU;
@@ -75,13 +76,7 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
     }
   }
 
-  float inv_static = 0.0f, s_static = 0.0f;
-  bool div_static = false;
-  if (QM == FRT_QUANT_STATIC) {
-    s_static = __ldg(static_scale);
-    inv_static = 1.0f / s_static;
-    div_static = !(fabsf(inv_static) < INFINITY);
-  }
+  const Divisor dv_static(QM == FRT_QUANT_STATIC ? __ldg(static_scale) : 1.0f);
 
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
@@ -94,55 +89,43 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
         a[e] = act_fn<ACT>(p.x) * p.y;
       }
     }
-    float s, inv;
-    bool div;
+    // code = e4m3(a / s) with the quotient correctly rounded in fp32
     if (QM == FRT_QUANT_BLOCK128) {
       const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
-      if (am == 0.0f) {
-        s = 1.0f;
-        inv = 1.0f;
-        div = false;
-      } else {
-        s = am / 448.0f;
-        div = am < 0x1p-100f;
-        inv = div ? 0.0f : 448.0f / am;
-      }
+      const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
       const int64_t gb = gb0 + u;
-      if (lane == 0 && gb < total_blocks) block_scales[gb] = s;  // [M, NB] row-major == flat block index
-    } else {
-      s = s_static;
-      inv = inv_static;
-      div = div_static;
-    }
-    if (valid[u]) {
-      float o[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = div ? __fdiv_rn(a[e], s) : a[e] * inv;
-      q[idx[u]] = e4m3x4(o[0], o[1], o[2], o[3]);
+      if (lane == 0 && gb < total_blocks) block_scales[gb] = sb;  // [M, NB] row-major == flat block index
+      if (valid[u]) {
+        const Divisor dv(sb);
+        q[idx[u]] = e4m3x4(dv.div(a[0]), dv.div(a[1]), dv.div(a[2]), dv.div(a[3]));
+      }
+    } else if (valid[u]) {
+      q[idx[u]] = e4m3x4(dv_static.div(a[0]), dv_static.div(a[1]), dv_static.div(a[2]), dv_static.div(a[3]));
     }
   }
 }
 
 template <int DT, int ACT>
-void launch_act(frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total, int NB,
-                int C4, cudaStream_t st) {
+frt_status launch_act(frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total,
+                      int NB, int C4, cudaStream_t st) {
   const int64_t warps = (total + kU - 1) / kU;
-  const unsigned grid = (unsigned)((warps + kWarps - 1) / kWarps);
+  const dim3 grid((unsigned)((warps + kWarps - 1) / kWarps));
+  const uint4* in = static_cast<const uint4*>(gu);
+  uint32_t* out = reinterpret_cast<uint32_t*>(q);
   if (qm == FRT_QUANT_STATIC)
-    gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC><<<grid, kThreads, 0, st>>>(
-        static_cast<const uint4*>(gu), reinterpret_cast<uint32_t*>(q), ss, bs, total, NB, C4);
-  else
-    gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128><<<grid, kThreads, 0, st>>>(
-        static_cast<const uint4*>(gu), reinterpret_cast<uint32_t*>(q), ss, bs, total, NB, C4);
+    return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC>, grid, dim3(kThreads), st, in, out, ss, bs, total,
+                  NB, C4);
+  return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128>, grid, dim3(kThreads), st, in, out, ss, bs, total,
+                NB, C4);
 }
 
 template <int DT>
-void launch_dt(frt_act act, frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total,
-               int NB, int C4, cudaStream_t st) {
+frt_status launch_dt(frt_act act, frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs,
+                     int64_t total, int NB, int C4, cudaStream_t st) {
   switch (act) {
-    case FRT_ACT_GELU_TANH: launch_act<DT, FRT_ACT_GELU_TANH>(qm, gu, q, ss, bs, total, NB, C4, st); break;
-    case FRT_ACT_SILU: launch_act<DT, FRT_ACT_SILU>(qm, gu, q, ss, bs, total, NB, C4, st); break;
-    default: launch_act<DT, FRT_ACT_RELU2>(qm, gu, q, ss, bs, total, NB, C4, st); break;
+    case FRT_ACT_GELU_TANH: return launch_act<DT, FRT_ACT_GELU_TANH>(qm, gu, q, ss, bs, total, NB, C4, st);
+    case FRT_ACT_SILU: return launch_act<DT, FRT_ACT_SILU>(qm, gu, q, ss, bs, total, NB, C4, st);
+    default: return launch_act<DT, FRT_ACT_RELU2>(qm, gu, q, ss, bs, total, NB, C4, st);
   }
 }
 
@@ -156,17 +139,15 @@ extern "C" frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, co
   if (M < 0 || I <= 0 || I % 4 != 0) return FRT_ERR_INVALID_ARG;
   if (!valid_dtype(dt) || !valid_quant(qm)) return FRT_ERR_INVALID_ARG;
   if (act != FRT_ACT_GELU_TANH && act != FRT_ACT_SILU && act != FRT_ACT_RELU2) return FRT_ERR_INVALID_ARG;
+  if (M == 0) return FRT_OK;
   if (!gate_up || !out_fp8 || !aligned(gate_up, 16) || !aligned(out_fp8, 4)) return FRT_ERR_INVALID_ARG;
   if (!quant_args_ok(qm, static_scale, block_scales)) return FRT_ERR_INVALID_ARG;
-  if (M == 0) return FRT_OK;
   const int NB = (I + 127) / 128;
   const int C4 = I / 4;
   const int64_t total = (int64_t)M * NB;
   const int64_t grid = (total + (int64_t)kU * kWarps - 1) / ((int64_t)kU * kWarps);
   if (grid > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
   if (dt == FRT_F16)
-    launch_dt<FRT_F16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
-  else
-    launch_dt<FRT_BF16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
-  return launch_status();
+    return launch_dt<FRT_F16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
+  return launch_dt<FRT_BF16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
 }

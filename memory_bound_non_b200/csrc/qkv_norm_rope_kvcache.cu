@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kThreads) qkv_norm_rope_kvcache_kernel(
     const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, uint16_t* __restrict__ k_cache,
     uint16_t* __restrict__ v_cache, int32_t* status, int64_t units, int H, int Hq, int Hkv, int hd, int G,
     int max_pos, int capacity, float eps) {
+  pdl_enter();
   const int64_t gt = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   const int64_t unit = gt / GP;
   const int li = threadIdx.x & (GP - 1);
@@ -173,34 +174,31 @@ struct Args {
 };
 
 template <int DT, int P, int GP>
-void launch_gp(const Args& a, cudaStream_t st) {
+frt_status launch_gp(const Args& a, cudaStream_t st) {
   const int64_t threads = a.units * GP;
-  const unsigned grid = (unsigned)((threads + kThreads - 1) / kThreads);
-  qkv_norm_rope_kvcache_kernel<DT, P, GP><<<grid, kThreads, 0, st>>>(
-      static_cast<const uint16_t*>(a.qkv), static_cast<const uint16_t*>(a.qw), static_cast<const uint16_t*>(a.kw),
-      a.cos_tab, a.sin_tab, a.pos, static_cast<uint16_t*>(a.q_out), static_cast<uint16_t*>(a.kc),
-      static_cast<uint16_t*>(a.vc), a.status, a.units, a.H, a.Hq, a.Hkv, a.hd, a.G, a.max_pos, a.capacity,
-      a.eps);
+  const dim3 grid((unsigned)((threads + kThreads - 1) / kThreads));
+  return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP>, grid, dim3(kThreads), st,
+                static_cast<const uint16_t*>(a.qkv), static_cast<const uint16_t*>(a.qw),
+                static_cast<const uint16_t*>(a.kw), a.cos_tab, a.sin_tab, a.pos, static_cast<uint16_t*>(a.q_out),
+                static_cast<uint16_t*>(a.kc), static_cast<uint16_t*>(a.vc), a.status, a.units, a.H, a.Hq, a.Hkv,
+                a.hd, a.G, a.max_pos, a.capacity, a.eps);
 }
 
 template <int DT, int P>
-void launch_p(int GP, const Args& a, cudaStream_t st) {
+frt_status launch_p(int GP, const Args& a, cudaStream_t st) {
   switch (GP) {
-    case 1: launch_gp<DT, P, 1>(a, st); break;
-    case 2: launch_gp<DT, P, 2>(a, st); break;
-    case 4: launch_gp<DT, P, 4>(a, st); break;
-    case 8: launch_gp<DT, P, 8>(a, st); break;
-    case 16: launch_gp<DT, P, 16>(a, st); break;
-    default: launch_gp<DT, P, 32>(a, st); break;
+    case 1: return launch_gp<DT, P, 1>(a, st);
+    case 2: return launch_gp<DT, P, 2>(a, st);
+    case 4: return launch_gp<DT, P, 4>(a, st);
+    case 8: return launch_gp<DT, P, 8>(a, st);
+    case 16: return launch_gp<DT, P, 16>(a, st);
+    default: return launch_gp<DT, P, 32>(a, st);
   }
 }
 
 template <int DT>
-void launch_dt(int P, int GP, const Args& a, cudaStream_t st) {
-  if (P == 8)
-    launch_p<DT, 8>(GP, a, st);
-  else
-    launch_p<DT, 4>(GP, a, st);
+frt_status launch_dt(int P, int GP, const Args& a, cudaStream_t st) {
+  return P == 8 ? launch_p<DT, 8>(GP, a, st) : launch_p<DT, 4>(GP, a, st);
 }
 
 }  // namespace
@@ -215,8 +213,9 @@ extern "C" frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_n
   using namespace frt;
   if (M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || hd <= 0 || hd % 2 != 0) return FRT_ERR_INVALID_ARG;
   if (max_pos <= 0 || capacity <= 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
-  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
   if (hd % 8 != 0 || hd > 256) return FRT_ERR_UNSUPPORTED;
+  if (M == 0) return FRT_OK;
+  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
   const int P = (hd % 16 == 0) ? 8 : 4;
   const uintptr_t al = (P == 8) ? 16 : 8;
   if (!aligned(qkv, al) || !aligned(q_out, al) || !aligned(k_cache, al) || !aligned(v_cache, al))
@@ -224,7 +223,6 @@ extern "C" frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_n
   if ((q_norm_w && !aligned(q_norm_w, al)) || (k_norm_w && !aligned(k_norm_w, al))) return FRT_ERR_INVALID_ARG;
   if (!aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(positions, 4)) return FRT_ERR_INVALID_ARG;
   if (status && !aligned(status, 4)) return FRT_ERR_INVALID_ARG;
-  if (M == 0) return FRT_OK;
   const int H = Hq + 2 * Hkv;
   const int G = (hd / 2) / P;  // active lanes per head, <= 31
   int GP = 1;
@@ -232,9 +230,5 @@ extern "C" frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_n
   Args a{qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status,
          (int64_t)M * H, H, Hq, Hkv, hd, G, max_pos, capacity, eps};
   if ((a.units * GP + kThreads - 1) / kThreads > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
-  if (dt == FRT_F16)
-    launch_dt<FRT_F16>(P, GP, a, stream);
-  else
-    launch_dt<FRT_BF16>(P, GP, a, stream);
-  return launch_status();
+  return dt == FRT_F16 ? launch_dt<FRT_F16>(P, GP, a, stream) : launch_dt<FRT_BF16>(P, GP, a, stream);
 }

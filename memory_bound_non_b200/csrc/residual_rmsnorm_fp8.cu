@@ -10,7 +10,8 @@
 // elements and thread t owns chunks t, t+T, t+2T, ... (K of them), so every
 // warp-wide load or store is one contiguous, fully used 512-byte run.  The sum
 // of squares is reduced warp-shuffle -> shared memory -> every thread, in a
-// fixed order (bitwise deterministic).  For block-128 scales a 128-column block
+// fixed order (bitwise deterministic), with a compensated fp32 pair so the
+// normalised values come out correctly rounded.  For block-128 scales a 128-column block
 // is 16 chunks owned by 16 consecutive lanes, so its amax is a 4-step xor
 // shuffle inside the warp; no shared memory and no second pass.
 #include <cmath>
@@ -20,39 +21,6 @@
 
 namespace frt {
 namespace {
-
-// Per-block (or per-tensor) quantisation factor: code = e4m3(y * inv), or
-// e4m3(y / s) when 1/s does not fit in fp32.
-struct QScale {
-  float s;
-  float inv;
-  bool div;
-};
-
-__device__ __forceinline__ float qval(float y, const QScale& q) { return q.div ? __fdiv_rn(y, q.s) : y * q.inv; }
-
-__device__ __forceinline__ QScale static_qscale(const float* p) {
-  QScale q;
-  q.s = __ldg(p);
-  q.inv = 1.0f / q.s;
-  q.div = !(fabsf(q.inv) < INFINITY);
-  return q;
-}
-
-// amax -> scale of one block-128: s = amax / 448, or 1 for an all-zero block.
-__device__ __forceinline__ QScale block_qscale(float amax) {
-  QScale q;
-  if (amax == 0.0f) {
-    q.s = 1.0f;
-    q.inv = 1.0f;
-    q.div = false;
-  } else {
-    q.s = amax / 448.0f;
-    q.div = amax < 0x1p-100f;
-    q.inv = q.div ? 0.0f : 448.0f / amax;
-  }
-  return q;
-}
 
 // Threads per CTA are at most 256 for K <= 2 and 512 for K >= 4.
 template <int K>
@@ -66,6 +34,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     uint2* __restrict__ q, const float* __restrict__ static_scale, float* __restrict__ block_scales, int C,
     int NB, float D, float eps) {
   using P16 = Pack16<DT>;
+  pdl_enter();
   const int t = threadIdx.x;
   const int T = blockDim.x;
   const int64_t row = blockIdx.x;
@@ -83,7 +52,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   }
 
   float h[K][8];
-  float ss = 0.0f;
+  Sum2 ss{0.0f, 0.0f};
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = t + k * T;
@@ -100,8 +69,8 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
         const float2 hf = P16::to_float2(hw[e]);
         h[k][2 * e] = hf.x;
         h[k][2 * e + 1] = hf.y;
-        ss = fmaf(hf.x, hf.x, ss);
-        ss = fmaf(hf.y, hf.y, ss);
+        ss.add(hf.x * hf.x);  // squares of 16-bit values are exact in fp32
+        ss.add(hf.y * hf.y);
       }
       r_out[base + c] = hv;
     } else {
@@ -110,88 +79,101 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     }
   }
 
-  // Row sum of squares: warp shuffle, then every thread sums the warp
-  // partials in the same order.
-  __shared__ float red[32];
-  ss = group_sum<32>(ss);
-  if ((t & 31) == 0) red[t >> 5] = ss;
+  // Row sum of squares, compensated: warp butterfly, then every thread adds
+  // the warp partials in the same order.  rstd is formed in fp64 from the
+  // ~2^-48-accurate sum, and y = h * w * rstd is rounded once to fp32 (h * w
+  // is exact for 16-bit operands), so y is the correctly rounded fp32 value of
+  // the exact normalised element: FP8 codes are then decided on the same fp32
+  // value an exact computation would give.
+  __shared__ float red_hi[32], red_lo[32];
+  ss = group_sum2<32>(ss);
+  if ((t & 31) == 0) {
+    red_hi[t >> 5] = ss.hi;
+    red_lo[t >> 5] = ss.lo;
+  }
   __syncthreads();
-  float tot = 0.0f;
+  Sum2 tot{red_hi[0], red_lo[0]};
   const int nw = T >> 5;
-  for (int i = 0; i < nw; ++i) tot += red[i];
-  const float rstd = 1.0f / sqrtf(tot / D + eps);
+  for (int i = 1; i < nw; ++i) tot.add(Sum2{red_hi[i], red_lo[i]});
+  const double ms = ((double)tot.hi + (double)tot.lo) / (double)D;
+  const Split32 rstd(1.0 / sqrt(ms + (double)eps));
 
-  QScale qs_static;
-  if (QM == FRT_QUANT_STATIC) qs_static = static_qscale(static_scale);
+  float s_static = 0.0f;
+  if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
+  const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
 
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = t + k * T;
     const bool valid = c < C;
     float y[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = h[k][e] * rstd;
     if (WEIGHTED && valid) {
       const uint4 wv = __ldg(w + c);
       const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 wf = P16::to_float2(ww[e]);
-        y[2 * e] *= wf.x;
-        y[2 * e + 1] *= wf.y;
+        y[2 * e] = rstd.mul(h[k][2 * e] * wf.x);
+        y[2 * e + 1] = rstd.mul(h[k][2 * e + 1] * wf.y);
       }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = rstd.mul(h[k][e]);
     }
-    QScale qs;
     if (QM == FRT_QUANT_BLOCK128) {
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
       am = group_max<16>(am);  // 16 lanes = the 16 chunks of one 128-column block
-      qs = block_qscale(am);
-      if (valid && (t & 15) == 0) block_scales[row * NB + (c >> 4)] = qs.s;
-    } else {
-      qs = qs_static;
-    }
-    if (valid) {
+      const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
+      if (valid && (t & 15) == 0) block_scales[row * NB + (c >> 4)] = sb;
+      if (valid) {
+        const Divisor dv(sb);
+        uint2 o;
+        o.x = e4m3x4(dv.div(y[0]), dv.div(y[1]), dv.div(y[2]), dv.div(y[3]));
+        o.y = e4m3x4(dv.div(y[4]), dv.div(y[5]), dv.div(y[6]), dv.div(y[7]));
+        q[base + c] = o;
+      }
+    } else if (valid) {
       uint2 o;
-      o.x = e4m3x4(qval(y[0], qs), qval(y[1], qs), qval(y[2], qs), qval(y[3], qs));
-      o.y = e4m3x4(qval(y[4], qs), qval(y[5], qs), qval(y[6], qs), qval(y[7], qs));
+      o.x = e4m3x4(dv_static.div(y[0]), dv_static.div(y[1]), dv_static.div(y[2]), dv_static.div(y[3]));
+      o.y = e4m3x4(dv_static.div(y[4]), dv_static.div(y[5]), dv_static.div(y[6]), dv_static.div(y[7]));
       q[base + c] = o;
     }
   }
 }
 
 template <int DT, int K, bool W, int QM>
-void launch_k(const void* x, const void* r_in, void* r_out, const void* w, uint8_t* q, const float* ss,
-              float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
-  residual_rmsnorm_fp8_kernel<DT, K, W, QM><<<M, T, 0, st>>>(
-      static_cast<const uint4*>(x), static_cast<const uint4*>(r_in), static_cast<uint4*>(r_out),
-      static_cast<const uint4*>(w), reinterpret_cast<uint2*>(q), ss, bs, C, NB, (float)(C * 8), eps);
+frt_status launch_k(const void* x, const void* r_in, void* r_out, const void* w, uint8_t* q, const float* ss,
+                    float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
+  return launch(residual_rmsnorm_fp8_kernel<DT, K, W, QM>, dim3(M), dim3(T), st, static_cast<const uint4*>(x),
+                static_cast<const uint4*>(r_in), static_cast<uint4*>(r_out), static_cast<const uint4*>(w),
+                reinterpret_cast<uint2*>(q), ss, bs, C, NB, (float)(C * 8), eps);
 }
 
 template <int DT, int K>
-void launch_dt_k(bool weighted, frt_quant qm, const void* x, const void* r_in, void* r_out, const void* w,
+frt_status launch_dt_k(bool weighted, frt_quant qm, const void* x, const void* r_in, void* r_out, const void* w,
                  uint8_t* q, const float* ss, float* bs, int M, int C, int NB, int T, float eps,
                  cudaStream_t st) {
   if (weighted) {
     if (qm == FRT_QUANT_STATIC)
-      launch_k<DT, K, true, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+      return launch_k<DT, K, true, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
     else
-      launch_k<DT, K, true, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+      return launch_k<DT, K, true, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
   } else {
     if (qm == FRT_QUANT_STATIC)
-      launch_k<DT, K, false, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+      return launch_k<DT, K, false, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
     else
-      launch_k<DT, K, false, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+      return launch_k<DT, K, false, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
   }
 }
 
 template <int DT>
-void launch_dt(int K, bool weighted, frt_quant qm, const void* x, const void* r_in, void* r_out, const void* w,
+frt_status launch_dt(int K, bool weighted, frt_quant qm, const void* x, const void* r_in, void* r_out, const void* w,
                uint8_t* q, const float* ss, float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
   switch (K) {
-    case 1: launch_dt_k<DT, 1>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st); break;
-    case 2: launch_dt_k<DT, 2>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st); break;
-    case 4: launch_dt_k<DT, 4>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st); break;
-    default: launch_dt_k<DT, 8>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st); break;
+    case 1: return launch_dt_k<DT, 1>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    case 2: return launch_dt_k<DT, 2>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    case 4: return launch_dt_k<DT, 4>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    default: return launch_dt_k<DT, 8>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
   }
 }
 
@@ -215,22 +197,20 @@ extern "C" frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residu
   using namespace frt;
   if (M < 0 || D <= 0 || D % 8 != 0) return FRT_ERR_INVALID_ARG;
   if (!valid_dtype(dt) || !valid_quant(qm)) return FRT_ERR_INVALID_ARG;
+  if (D > 32768) return FRT_ERR_UNSUPPORTED;
+  if (M == 0) return FRT_OK;
   if (!x || !residual_in || !residual_out || !out_fp8) return FRT_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(residual_in, 16) || !aligned(residual_out, 16) || !aligned(out_fp8, 8))
     return FRT_ERR_INVALID_ARG;
   if (weight && !aligned(weight, 16)) return FRT_ERR_INVALID_ARG;
   if (!quant_args_ok(qm, static_scale, block_scales)) return FRT_ERR_INVALID_ARG;
-  if (D > 32768) return FRT_ERR_UNSUPPORTED;
-  if (M == 0) return FRT_OK;
   const int C = D / 8;
   const int NB = (D + 127) / 128;
   int K, T;
   rmsnorm_shape(C, &K, &T);
   if (dt == FRT_F16)
-    launch_dt<FRT_F16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp8, static_scale,
-                       block_scales, M, C, NB, T, eps, stream);
-  else
-    launch_dt<FRT_BF16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp8, static_scale,
-                        block_scales, M, C, NB, T, eps, stream);
-  return launch_status();
+    return launch_dt<FRT_F16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp8,
+                              static_scale, block_scales, M, C, NB, T, eps, stream);
+  return launch_dt<FRT_BF16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp8,
+                             static_scale, block_scales, M, C, NB, T, eps, stream);
 }

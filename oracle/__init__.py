@@ -5,7 +5,8 @@ tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
 import this package; the CUDA library never does, and the two share no code.
 
 16-bit tensors are passed as ``np.uint16`` bit patterns; ``dt`` is ``"f16"``
-or ``"bf16"``.  Every function returns freshly allocated numpy arrays.
+or ``"bf16"``.  Every function returns freshly allocated numpy arrays.  The
+ops' ``eps`` is rounded to fp32 first: that is the value the kernels receive.
 """
 import ctypes
 import os
@@ -19,6 +20,10 @@ _QM = {"static": 0, "block128": 1}
 _ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
 
 _lib = None
+
+
+def _f32(x):
+    return float(np.float32(x))
 
 
 def _p(a):
@@ -142,7 +147,7 @@ def residual_rmsnorm_fp8(x, residual_in, weight, eps, dt, quant, static_scale=No
     y = np.empty((M, D), dtype=np.float64) if want_y else None
     s = float(static_scale) if quant == "static" else 0.0
     rc = lib().oracle_residual_rmsnorm_fp8(_p(x), _p(r), _p(r_out), _p(w), _p(q), s, _p(sc), _p(y),
-                                           M, D, float(eps), _DT[dt], _QM[quant])
+                                           M, D, _f32(eps), _DT[dt], _QM[quant])
     if rc != 0:
         raise ValueError("oracle_residual_rmsnorm_fp8: bad argument")
     return {"residual_out": r_out, "out_fp8": q, "block_scales": sc, "y": y}
@@ -170,7 +175,7 @@ def qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, 
     status = np.zeros(1, dtype=np.int32)
     rc = lib().oracle_qkv_norm_rope_kvcache(_p(qkv), _p(qw), _p(kw), _p(cos_tab), _p(sin_tab), _p(pos), _p(sl),
                                             _p(q_out), _p(kc), _p(vc), _p(status), M, Hq, Hkv, hd, max_pos,
-                                            capacity, float(eps), _DT[dt])
+                                            capacity, _f32(eps), _DT[dt])
     if rc != 0:
         raise ValueError("oracle_qkv_norm_rope_kvcache: bad argument")
     return {"q_out": q_out, "k_cache": kc, "v_cache": vc, "status": int(status[0])}

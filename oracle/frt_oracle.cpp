@@ -165,16 +165,29 @@ double e4m3_decode(uint8_t c) {
 }
 
 // ------------------------------------------------------------ quantisers --
+// The FP8 code is an integer decided by floating point, so it is decided in
+// one stated precision on both sides: fp32, the precision of the kernels (the
+// pages fix none).  The value y (fp64 here) is rounded once to fp32, divided by
+// the fp32 scale in fp32 (IEEE, round to nearest), and that quotient is
+// encoded.
+uint8_t quant_fp32(double y, float s32) {
+  const float v = (float)y / s32;
+  return e4m3_encode((double)v);
+}
+
 // Static per-tensor FP8 ([FR] §六: `_static` = the activation scale is a
-// constant).  s is a dequantisation scale: q = e4m3(y / s), y ~ q * s.
+// constant).  s is a dequantisation scale (an fp32 value): q = e4m3(y / s),
+// y ~ q * s.
 void quant_static(const double* y, int64_t n, double s, uint8_t* q) {
-  for (int64_t j = 0; j < n; ++j) q[j] = e4m3_encode(y[j] / s);
+  const float s32 = (float)s;
+  for (int64_t j = 0; j < n; ++j) q[j] = quant_fp32(y[j], s32);
 }
 
 // Per-token block-128 FP8 ([FR4] Phase 2: per-token block-128 quantisation
 // with an out_scale per row and block).  Block b covers columns
 // [128b, min(128b+128, n)); s_b = amax_b / 448, or 1 when the block is all
-// zero; q = e4m3(y / s_b).
+// zero; q = e4m3(y / s_b).  `scales` receives the fp64 amax_b / 448; the codes
+// use the same scale evaluated in fp32 (fp32(amax_b) / 448 in fp32).
 void quant_block128(const double* y, int64_t n, uint8_t* q, double* scales) {
   const int64_t nb = (n + 127) / 128;
   for (int64_t b = 0; b < nb; ++b) {
@@ -182,9 +195,9 @@ void quant_block128(const double* y, int64_t n, uint8_t* q, double* scales) {
     const int64_t hi = (lo + 128 < n) ? lo + 128 : n;
     double amax = 0.0;
     for (int64_t j = lo; j < hi; ++j) amax = std::fmax(amax, std::fabs(y[j]));
-    const double s = (amax > 0.0) ? amax / 448.0 : 1.0;
-    scales[b] = s;
-    for (int64_t j = lo; j < hi; ++j) q[j] = e4m3_encode(y[j] / s);
+    scales[b] = (amax > 0.0) ? amax / 448.0 : 1.0;
+    const float s32 = (amax > 0.0) ? (float)amax / 448.0f : 1.0f;
+    for (int64_t j = lo; j < hi; ++j) q[j] = quant_fp32(y[j], s32);
   }
 }
 

@@ -117,21 +117,26 @@ def residual_rmsnorm_fp8(x, r, w, eps, dt, quant, static_scale=None):
     return h_bits, q, scales
 
 
+def _code_fp32(yj, s32):
+    """FP8 decision taken in fp32: fp32(y) / fp32(s) in numpy float32, then the
+    exact nearest-code search on that quotient."""
+    v = np.float32(yj) / np.float32(s32)
+    return e4m3_exact(Fraction(float(v)), math.copysign(1.0, float(v)) < 0)
+
+
 def _quant_row(y, quant, static_scale, q_row, sc_row):
     n = y.size
     if quant == "static":
         for j in range(n):
-            yj = float(y[j])
-            q_row[j] = e4m3_exact(Fraction(yj) / Fraction(float(static_scale)), math.copysign(1.0, yj) < 0)
+            q_row[j] = _code_fp32(float(y[j]), static_scale)
         return
     for b in range(0, n, 128):
         blk = y[b:b + 128]
         amax = float(np.max(np.abs(blk)))
-        s = amax / 448.0 if amax > 0 else 1.0
-        sc_row[b // 128] = s
+        sc_row[b // 128] = amax / 448.0 if amax > 0 else 1.0
+        s32 = np.float32(amax) / np.float32(448.0) if amax > 0 else np.float32(1.0)
         for j in range(blk.size):
-            yj = float(blk[j])
-            q_row[b + j] = e4m3_exact(Fraction(yj) / Fraction(s), math.copysign(1.0, yj) < 0)
+            q_row[b + j] = _code_fp32(float(blk[j]), s32)
 
 
 def qkv_norm_rope(qkv, qw, kw, cos, sin, pos, Hq, Hkv, hd, eps, dt):

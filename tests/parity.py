@@ -3,9 +3,12 @@ helpers the GPU tests share (static-scale calibration, the chain replay).
 
 Tolerances (element by element):
   * residual h, V cache, slot placement, untouched slots: bit-exact;
-  * 16-bit outputs (Q staging, K cache): |g - o| / max(|o|, 2^-6) <= 2e-3,
-    o the unrounded fp64 oracle value (a correctly rounded bf16 is within
-    2^-9 ~ 1.95e-3 of it);
+  * 16-bit outputs (Q staging, K cache), against the unrounded fp64 oracle
+    value o: |g - o| <= 2e-3 * max(|o|, 2^-6) + ulp16(o) / 2, i.e. a relative
+    error of 2e-3 for the arithmetic on top of the final rounding to 16 bits
+    (a correctly rounded bf16 alone is up to 2^-8 ~ 3.9e-3 from o, so a bare
+    2e-3 bound cannot hold for any bf16 output); and at least 99% of the
+    elements must be the correctly rounded value itself (|g - o| <= ulp/2);
   * FP8 codes: equal (+0 == -0), else one code step apart with the same sign,
     on at most 0.1% of the elements;
   * block scales: relative error <= 1e-6 against the fp64 amax / 448.
@@ -51,14 +54,35 @@ def assert_fp8_codes(gpu, ref, max_frac=FP8_MAX_FRAC, what="fp8"):
     return n
 
 
-def assert_16bit_close(gpu_vals, ref, what="16-bit"):
+# significand bits and smallest normal exponent of the 16-bit formats
+_FMT16 = {"bf16": (8, -126), "f16": (11, -14)}
+MAX_OFF_ROUNDING = 0.01
+
+
+def ulp16(o, dt):
+    """Spacing of the 16-bit format at |o| (the binade of o; subnormal spacing
+    below the smallest normal)."""
+    p, emin = _FMT16[dt]
+    a = np.abs(o)
+    e = np.floor(np.log2(np.where(a > 0, a, 2.0 ** emin)))
+    e = np.maximum(e, emin)
+    return np.ldexp(1.0, (e - (p - 1)).astype(np.int64))
+
+
+def assert_16bit_close(gpu_vals, ref, what="16-bit", dt="bf16"):
     g = np.asarray(gpu_vals, dtype=np.float64).ravel()
     o = np.asarray(ref, dtype=np.float64).ravel()
     assert g.shape == o.shape
     assert np.isfinite(o).all(), what + ": oracle has non-finite values"
-    err = np.abs(g - o) / np.maximum(np.abs(o), FLOOR_16)
-    k = int(np.argmax(err))
-    assert err[k] <= REL_16, "%s: rel err %.3g at %d (gpu %r oracle %r)" % (what, err[k], k, g[k], o[k])
+    half = ulp16(o, dt) / 2
+    bar = REL_16 * np.maximum(np.abs(o), FLOOR_16) + half
+    err = np.abs(g - o)
+    k = int(np.argmax(err / bar))
+    assert err[k] <= bar[k], "%s: |g-o| %.3g > bar %.3g at %d (gpu %r oracle %r)" % (what, err[k], bar[k], k,
+                                                                                      g[k], o[k])
+    off = int((err > half * (1 + 1e-12)).sum())
+    assert off <= MAX_OFF_ROUNDING * g.size, "%s: %d of %d not the correctly rounded value" % (what, off, g.size)
+    return off
 
 
 def assert_scales_close(gpu, ref, what="block scales"):

@@ -42,6 +42,7 @@ def a_call(M=4, D=256, x=A, r=A, ro=A, w=None, q=A, ss=A, bs=None, dt=1, qm=0):
     (dict(q=None), INV), (dict(x=A + 8), INV), (dict(r=A + 4), INV), (dict(q=A + 4), INV),
     (dict(w=A + 2), INV), (dict(ss=None), INV), (dict(qm=1, bs=None), INV), (dict(dt=2), INV),
     (dict(qm=5), INV), (dict(D=32776), UNSUP), (dict(M=0), OK), (dict(M=0, qm=1, bs=A), OK),
+    (dict(M=0, x=None, ro=None, q=None, ss=None), OK), (dict(M=0, D=12), INV), (dict(M=0, dt=4), INV),
 ])
 def test_residual_rmsnorm_host_validation(kw, want):
     assert a_call(**kw) == want
@@ -59,7 +60,8 @@ def b_call(M=4, Hq=8, Hkv=2, hd=128, qkv=A, cos=A, sin=A, pos=A, qo=A, kc=A, vc=
     (dict(max_pos=0), INV), (dict(cap=0), INV), (dict(qkv=None), INV), (dict(cos=None), INV),
     (dict(pos=None), INV), (dict(kc=None), INV), (dict(qkv=A + 8), INV), (dict(hd=72, qkv=A + 8, M=0), OK),
     (dict(hd=72, qkv=A + 4), INV), (dict(cos=A + 8), INV), (dict(pos=A + 2), INV), (dict(status=A + 1), INV),
-    (dict(qw=A + 8), INV), (dict(dt=9), INV), (dict(M=0), OK),
+    (dict(qw=A + 8), INV), (dict(dt=9), INV), (dict(M=0), OK), (dict(M=0, qkv=None, kc=None), OK),
+    (dict(M=0, hd=12), UNSUP), (dict(M=0, Hq=6, Hkv=4), INV),
 ])
 def test_qkv_host_validation(kw, want):
     assert b_call(**kw) == want
@@ -73,7 +75,7 @@ def c_call(M=4, I=256, gu=A, q=A, ss=A, bs=None, act=0, dt=1, qm=0):
     (dict(M=-1), INV), (dict(I=0), INV), (dict(I=6), INV), (dict(act=3), INV), (dict(act=-1), INV),
     (dict(gu=None), INV), (dict(gu=A + 8), INV), (dict(q=A + 2), INV), (dict(ss=None), INV),
     (dict(qm=1, bs=None), INV), (dict(qm=1, bs=A + 2), INV), (dict(dt=3), INV), (dict(M=0), OK),
-    (dict(M=0, I=4, qm=1, bs=A), OK),
+    (dict(M=0, I=4, qm=1, bs=A), OK), (dict(M=0, gu=None, q=None, ss=None), OK), (dict(M=0, I=6), INV),
 ])
 def test_gate_act_host_validation(kw, want):
     assert c_call(**kw) == want
@@ -92,3 +94,14 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(frt.FrtError):
         frt.frt_residual_rmsnorm_fp8(x, x, x, None, torch.zeros(2, 8, dtype=torch.uint8),
                                      static_scale=torch.ones(1))
+
+
+def test_pdl_switch():
+    prev = frt.frt_get_pdl()
+    try:
+        frt.frt_set_pdl(False)
+        assert frt.frt_get_pdl() is False
+        frt.frt_set_pdl(True)
+        assert frt.frt_get_pdl() is True
+    finally:
+        frt.frt_set_pdl(prev)

@@ -186,11 +186,11 @@ def check_b_full(wl, inp):
     q_out, kc, vc, status = run_b_gpu(wl, inp)
     o = oracle_b(wl, inp)
     assert status == o["status"] == 0
-    P.assert_16bit_close(P.decode16(q_out), o["q_out"], what="Q staging")
+    P.assert_16bit_close(P.decode16(q_out), o["q_out"], what="Q staging", dt=wl.dt)
     written = ~np.isnan(o["k_cache"]).all(axis=(1, 2))
     k0, v0 = W.bits16(inp.layers[0].k_cache), W.bits16(inp.layers[0].v_cache)
     kg, vg = P.np16(kc), P.np16(vc)
-    P.assert_16bit_close(P.decode16(kc)[written], o["k_cache"][written], what="K cache")
+    P.assert_16bit_close(P.decode16(kc)[written], o["k_cache"][written], what="K cache", dt=wl.dt)
     np.testing.assert_array_equal(vg[written], o["v_cache"][written])
     np.testing.assert_array_equal(kg[~written], k0[~written])   # untouched slots keep their bits
     np.testing.assert_array_equal(vg[~written], v0[~written])
@@ -226,8 +226,8 @@ def test_qkv_large_m_sampled(M):
     rows = sample_rows(M, 256)
     o = oracle_b(wl, inp, rows=rows)
     pos = take(inp.positions, rows).numpy()
-    P.assert_16bit_close(P.decode16(q_out[torch.from_numpy(rows).to(DEV)]), o["q_out"], what="Q staging")
-    P.assert_16bit_close(P.decode16(kc[torch.from_numpy(pos).long().to(DEV)]), o["k_cache"], what="K cache")
+    P.assert_16bit_close(P.decode16(q_out[torch.from_numpy(rows).to(DEV)]), o["q_out"], what="Q staging", dt=wl.dt)
+    P.assert_16bit_close(P.decode16(kc[torch.from_numpy(pos).long().to(DEV)]), o["k_cache"], what="K cache", dt=wl.dt)
     np.testing.assert_array_equal(P.np16(vc[torch.from_numpy(pos).long().to(DEV)]), o["v_cache"])
     # every slot outside the written set still holds the sentinel
     mask = torch.ones(wl.capacity, dtype=torch.bool, device=DEV)
@@ -245,7 +245,7 @@ def test_qkv_bad_positions_set_status_and_skip_rows():
     o = oracle_b(wl, inp, positions=pos)
     assert status == 1 and o["status"] == 1
     good = np.array([0, 2, 4])
-    P.assert_16bit_close(P.decode16(q_out)[good], o["q_out"][good], what="Q staging")
+    P.assert_16bit_close(P.decode16(q_out)[good], o["q_out"][good], what="Q staging", dt=wl.dt)
     # skipped rows leave their Q staging rows as they were (guard fill 0x3C3C)
     assert (P.np16(q_out)[[1, 3, 5]] == 0x3C3C).all()
     written = ~np.isnan(o["k_cache"]).all(axis=(1, 2))

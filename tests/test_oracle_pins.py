@@ -352,6 +352,16 @@ def test_quant_static_reproduces_exact_codes():
     np.testing.assert_array_equal(q, codes)
 
 
+def test_quant_decision_is_taken_in_fp32():
+    # 21 is the midpoint of the e4m3 codes for 20 and 22.  21 + 2e-7 lies above
+    # it in fp64 but rounds to exactly 21.0 in fp32, where the tie goes to the
+    # even code (20): the code is decided on the fp32 quotient.
+    assert oracle.quant_static(np.array([21 + 2e-7]), 1.0)[0] == oracle.e4m3_encode(20.0)
+    assert oracle.quant_static(np.array([21 + 4e-6]), 1.0)[0] == oracle.e4m3_encode(22.0)
+    # fp32(y) / fp32(s) in fp32: 0.1 / 0.1 rounds to exactly 1
+    assert oracle.quant_static(np.array([float(np.float32(0.1))]), float(np.float32(0.1)))[0] == 0x38
+
+
 def test_quant_block128_scales_and_edges():
     rng = np.random.default_rng(13)
     n = 128 * 3 + 80  # partial last block of 80 columns
