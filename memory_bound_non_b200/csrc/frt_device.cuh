@@ -48,70 +48,32 @@ struct Pack16<FRT_BF16> {
   }
 };
 
-// Sum of two floats rounded to odd: the nearest of the two fp32 neighbours of
-// the exact sum whose last significand bit is 1 (or the exact sum when it is
-// representable).  Rounding this value once more to a format with at least two
-// fewer significand bits gives the correctly rounded (RNE) exact sum, so
-// RN16(add_round_odd(x, r)) == RN16(x + r) with no double-rounding error.
-// The error term comes from Knuth's TwoSum.
-__device__ __forceinline__ float add_round_odd(float a, float b) {
-  const float s = __fadd_rn(a, b);
-  const float bb = __fsub_rn(s, a);
-  const float err = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
-  uint32_t u = __float_as_uint(s);
-  if (err != 0.0f && (u & 1u) == 0u) {
-    // step one ulp towards the exact value: away from zero when err has the
-    // sign of s, towards zero otherwise
-    u += ((__float_as_uint(err) ^ u) & 0x80000000u) ? 0xFFFFFFFFu : 1u;
-  }
-  return __uint_as_float(u);
-}
+// Residual add of two 16-bit values: the fp32 sum rounded to the 16-bit type
+// is the correctly rounded exact sum.  Rounding an exact sum first to q = 24
+// bits and then to p bits equals rounding it once to p bits whenever
+// q >= 2p + 1 (S. A. Figueroa, "When is double rounding innocuous?", 1995);
+// p = 8 (bf16) and p = 11 (fp16) both satisfy it.
+__device__ __forceinline__ float add_for_16(float a, float b) { return __fadd_rn(a, b); }
 
-// Knuth's TwoSum: a + b == s + e exactly (fp32, round to nearest).
-__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
-  s = __fadd_rn(a, b);
-  const float bb = __fsub_rn(s, a);
-  e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
-}
-
-// Compensated (hi, lo) accumulator: hi + lo tracks the exact sum of the
-// added terms to ~2^-48 relative.  Adding pairs is commutative bit for bit
-// (TwoSum's error term is the unique exact error), so an xor-butterfly gives
-// every lane the same pair.
-struct Sum2 {
-  float hi, lo;
-  __device__ __forceinline__ void add(float x) {
-    float s, e;
-    two_sum(hi, x, s, e);
-    hi = s;
-    lo = __fadd_rn(lo, e);
-  }
-  __device__ __forceinline__ void add(const Sum2& o) {
-    float s, e;
-    two_sum(hi, o.hi, s, e);
-    hi = s;
-    lo = __fadd_rn(__fadd_rn(lo, o.lo), e);
-  }
-};
-
-template <int WIDTH>
-__device__ __forceinline__ Sum2 group_sum2(Sum2 v) {
-#pragma unroll
-  for (int o = WIDTH / 2; o > 0; o >>= 1) {
-    Sum2 w;
-    w.hi = __shfl_xor_sync(0xFFFFFFFFu, v.hi, o);
-    w.lo = __shfl_xor_sync(0xFFFFFFFFu, v.lo, o);
-    v.add(w);
-  }
-  return v;
+// 1 / sqrt(x) in fp64, to ~1e-16 relative (not correctly rounded): an fp32
+// estimate refined by two Newton steps in fp64.  Every lane can afford it
+// (about a dozen instructions), unlike a correctly rounded sqrt + divide.
+// Arguments outside the fp32 range of the estimate take the IEEE path.
+__device__ __forceinline__ double rsqrt_f64(double x) {
+  if (!(x >= 0x1p-120 && x <= 0x1p+120)) return 1.0 / sqrt(x);
+  double r = (double)rsqrtf((float)x);
+  r = r * fma(-0.5 * x * r, r, 1.5);
+  r = r * fma(-0.5 * x * r, r, 1.5);
+  return r;
 }
 
 // fp32 scale factor r held as an unevaluated pair rhi + rlo (from an fp64
-// value).  mul_exact(x, r) = fp32 rounding of x * (rhi + rlo), computed with
+// value).  mul(x) = fp32 rounding of x * (rhi + rlo), computed with
 // an exact product (TwoProduct via FMA): correctly rounded unless the exact
 // product lies within ~2^-48 of an fp32 rounding boundary.
 struct Split32 {
   float hi, lo;
+  __device__ __forceinline__ Split32() : hi(0.0f), lo(0.0f) {}
   __device__ __forceinline__ explicit Split32(double r) {
     hi = __double2float_rn(r);
     lo = __double2float_rn(r - (double)hi);
@@ -125,24 +87,32 @@ struct Split32 {
 
 // y / s rounded to nearest in fp32, from inv = RN(1/s): one FMA residual step
 // on the quotient estimate gives the correctly rounded quotient (Markstein's
-// theorem) while the quotient and the residual stay in the normal range.
-// Outside that range (tiny or huge scales, |y| < 2^-90, zeros) the IEEE
-// division is used instead.
+// theorem) while the residual y - q*s is exactly representable, which holds
+// for positive scales in [2^-100, 2^100] and |y| >= 2^-100 (for smaller |y|
+// the result can be one ulp off; zeros keep their sign).  Scales outside that
+// range (`fast` false) use the IEEE division for every element; callers
+// branch on `fast` once, outside their element loops.
 struct Divisor {
   float s, inv;
   bool fast;
   __device__ __forceinline__ explicit Divisor(float s_) : s(s_) {
     inv = __frcp_rn(s_);
-    const float a = fabsf(s_);
-    fast = a >= 0x1p-100f && a <= 0x1p+100f;
+    fast = s_ >= 0x1p-100f && s_ <= 0x1p+100f;
   }
   __device__ __forceinline__ float div(float y) const {
-    if (!fast || !(fabsf(y) >= 0x1p-90f)) return __fdiv_rn(y, s);  // also zeros: keeps -0
     const float q = y * inv;
     const float r = fmaf(-q, s, y);
-    return fmaf(r, inv, q);
+    const float v = fmaf(r, inv, q);
+    // s > 0, so the quotient has the sign of y (this also keeps -0)
+    return __uint_as_float((__float_as_uint(v) & 0x7FFFFFFFu) | (__float_as_uint(y) & 0x80000000u));
   }
+  __device__ __forceinline__ float div_slow(float y) const { return __fdiv_rn(y, s); }
 };
+
+// Eight values -> eight e4m3 codes of y / s (low byte first).
+__device__ __forceinline__ uint2 quant8(const float* y, const Divisor& dv);
+// Four values -> four e4m3 codes of y / s.
+__device__ __forceinline__ uint32_t quant4(const float* y, const Divisor& dv);
 
 // ----------------------------------------------------------------- FP8 --
 // Two fp32 -> two e4m3 codes (low byte = a), RNE, saturating to +-448.
@@ -151,6 +121,15 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 }
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return e4m3x2(a, b) | (e4m3x2(c, d) << 16);
+}
+
+__device__ __forceinline__ uint32_t quant4(const float* y, const Divisor& dv) {
+  if (dv.fast) return e4m3x4(dv.div(y[0]), dv.div(y[1]), dv.div(y[2]), dv.div(y[3]));
+  return e4m3x4(dv.div_slow(y[0]), dv.div_slow(y[1]), dv.div_slow(y[2]), dv.div_slow(y[3]));
+}
+
+__device__ __forceinline__ uint2 quant8(const float* y, const Divisor& dv) {
+  return make_uint2(quant4(y, dv), quant4(y + 4, dv));
 }
 
 // ------------------------------------------------------------ memory ops --
@@ -176,6 +155,18 @@ __device__ __forceinline__ uint4 ld_plain(const uint4* p) {
                : "l"(p)
                : "memory");
   return v;
+}
+
+// Per-thread asynchronous 16-byte global -> shared copy (L2 only), with
+// commit/wait on this thread's own copy groups.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // --------------------------------------------------------- reductions --

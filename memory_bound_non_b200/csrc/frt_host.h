@@ -27,11 +27,12 @@ bool pdl_enabled();
 // stream still runs, and waits for it (griddepcontrol.wait) before its first
 // memory access.
 template <typename... KArgs, typename... Args>
-inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream, Args... args) {
+inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                         Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -45,6 +46,11 @@ inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaSt
   }
   return launch_status();
 }
+
+// Resident CTAs per SM x SMs for `kernel` at `threads` threads and `smem`
+// bytes of dynamic shared memory (cached per kernel, block size and device):
+// the grid size of a persistent launch.
+int persistent_grid(const void* kernel, int threads, size_t smem = 0);
 
 // Checks shared by the two FP8-producing ops: the pointer the quant mode needs.
 inline bool quant_args_ok(frt_quant qm, const float* static_scale, const float* block_scales) {

@@ -38,11 +38,11 @@ __device__ __forceinline__ float act_fn(float g) {
     return r * r;
   } else if (ACT == FRT_ACT_SILU) {
     const float e = expf(fminf(-g, 80.0f));
-    return Divisor(1.0f + e).div(g);
+    return __fdividef(g, 1.0f + e);
   } else {
     const float z = g * fmaf(kSqrt2OverPi * kGeluCubic, g * g, kSqrt2OverPi);
     const float e = expf(fminf(-2.0f * z, 80.0f));
-    return Divisor(1.0f + e).div(g);
+    return __fdividef(g, 1.0f + e);
   }
 }
 
@@ -95,12 +95,9 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
       const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
       const int64_t gb = gb0 + u;
       if (lane == 0 && gb < total_blocks) block_scales[gb] = sb;  // [M, NB] row-major == flat block index
-      if (valid[u]) {
-        const Divisor dv(sb);
-        q[idx[u]] = e4m3x4(dv.div(a[0]), dv.div(a[1]), dv.div(a[2]), dv.div(a[3]));
-      }
+      if (valid[u]) q[idx[u]] = quant4(a, Divisor(sb));
     } else if (valid[u]) {
-      q[idx[u]] = e4m3x4(dv_static.div(a[0]), dv_static.div(a[1]), dv_static.div(a[2]), dv_static.div(a[3]));
+      q[idx[u]] = quant4(a, dv_static);
     }
   }
 }
@@ -113,9 +110,9 @@ frt_status launch_act(frt_quant qm, const void* gu, uint8_t* q, const float* ss,
   const uint4* in = static_cast<const uint4*>(gu);
   uint32_t* out = reinterpret_cast<uint32_t*>(q);
   if (qm == FRT_QUANT_STATIC)
-    return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC>, grid, dim3(kThreads), st, in, out, ss, bs, total,
+    return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
                   NB, C4);
-  return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128>, grid, dim3(kThreads), st, in, out, ss, bs, total,
+  return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
                 NB, C4);
 }
 

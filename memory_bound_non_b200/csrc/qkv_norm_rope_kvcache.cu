@@ -11,9 +11,10 @@
 // unit; lane l holds elements [lP, lP+P) and their RoPE partners
 // [hd/2 + lP, ...), P = 8 (16-byte vectors) when hd % 16 == 0, else P = 4
 // (8-byte vectors; e.g. the unpadded head_dim 72 of the ViT).  The per-head
-// sum of squares is an xor shuffle inside the group; cos/sin rows are shared
-// by all heads of a token and come from L1.  Every unit is independent, so the
-// grid is simply (tokens x heads x GP) threads.
+// sum of squares is an xor shuffle inside the group.  A CTA holds one token's
+// heads (all of them when heads x GP <= 1024), so the token's position and
+// cos/sin row are read once into L1 and shared by every head, and no thread
+// divides by the head count.
 #include <cmath>
 
 #include "frt_device.cuh"
@@ -21,8 +22,6 @@
 
 namespace frt {
 namespace {
-
-constexpr int kThreads = 256;
 
 template <int P>
 struct Vec16;
@@ -73,28 +72,23 @@ __device__ __forceinline__ void ld_f32(const float* p, float* f) {
 }
 
 template <int DT, int P, int GP>
-__global__ void __launch_bounds__(kThreads) qkv_norm_rope_kvcache_kernel(
+__global__ void __launch_bounds__(1024) qkv_norm_rope_kvcache_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
     const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
     const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, uint16_t* __restrict__ k_cache,
-    uint16_t* __restrict__ v_cache, int32_t* status, int64_t units, int H, int Hq, int Hkv, int hd, int G,
+    uint16_t* __restrict__ v_cache, int32_t* status, int H, int HB, int nhb, int Hq, int Hkv, int hd, int G,
     int max_pos, int capacity, float eps) {
   pdl_enter();
-  const int64_t gt = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  const int64_t unit = gt / GP;
+  // CTA = (token, group of HB heads); GP lanes per head.
+  const int tok = blockIdx.x / nhb;
+  const int h = (blockIdx.x - tok * nhb) * HB + (int)(threadIdx.x / GP);
   const int li = threadIdx.x & (GP - 1);
-  const bool in_range = unit < units;
-  const int64_t tok = in_range ? unit / H : 0;
-  const int h = in_range ? (int)(unit - tok * H) : 0;
+  const bool in_range = threadIdx.x < (unsigned)(HB * GP) && h < H;
 
-  int p = 0;
-  bool row_ok = false;
-  if (in_range) {
-    p = __ldg(positions + tok);
-    row_ok = p >= 0 && p < max_pos && p < capacity;
-    if (!row_ok && h == 0 && li == 0 && status != nullptr) atomicOr(status, 1);
-  }
-  const bool active = row_ok && li < G;
+  const int p = __ldg(positions + tok);
+  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
+  if (!row_ok && threadIdx.x == 0 && blockIdx.x == tok * nhb && status != nullptr) atomicOr(status, 1);
+  const bool active = in_range && row_ok && li < G;
   const int half = hd >> 1;
   const int j0 = li * P;
   const bool is_q = h < Hq;
@@ -102,11 +96,20 @@ __global__ void __launch_bounds__(kThreads) qkv_norm_rope_kvcache_kernel(
   const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
   const bool do_norm = !is_v && nw != nullptr;
 
-  const uint16_t* src = qkv + tok * (int64_t)H * hd + (int64_t)h * hd;
+  // Issue the QKV loads first and prefetch the token's cos/sin slice into L1
+  // (no registers held), so the table's latency overlaps the QKV loads and
+  // the per-head reduction; the table is read after the reduction.
+  const uint16_t* src = qkv + ((int64_t)tok * H + h) * hd;
+  const float* crow = cos_tab + (int64_t)p * half + j0;
+  const float* srow = sin_tab + (int64_t)p * half + j0;
   typename Vec16<P>::T va, vb;
   if (active) {
     va = *reinterpret_cast<const typename Vec16<P>::T*>(src + j0);
     vb = *reinterpret_cast<const typename Vec16<P>::T*>(src + half + j0);
+    if (!is_v) {
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(crow));
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(srow));
+    }
   }
 
   if (is_v) {  // V: bit copy into the cache slot
@@ -132,25 +135,25 @@ __global__ void __launch_bounds__(kThreads) qkv_norm_rope_kvcache_kernel(
   if (active && !is_v) {
     if (do_norm) {
       const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
-      float wa[P], wb[P];
-      unpack<DT, P>(ld_vec<P>(nw + j0), wa);
-      unpack<DT, P>(ld_vec<P>(nw + half + j0), wb);
+      float fa[P], fb[P];
+      unpack<DT, P>(ld_vec<P>(nw + j0), fa);
+      unpack<DT, P>(ld_vec<P>(nw + half + j0), fb);
 #pragma unroll
       for (int e = 0; e < P; ++e) {
-        a[e] = a[e] * rstd * wa[e];
-        b[e] = b[e] * rstd * wb[e];
+        a[e] = a[e] * rstd * fa[e];
+        b[e] = b[e] * rstd * fb[e];
       }
     }
     float c[P], s[P];
-    ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
-    ld_f32<P>(sin_tab + (int64_t)p * half + j0, s);
+    ld_f32<P>(crow, c);
+    ld_f32<P>(srow, s);
     float o1[P], o2[P];
 #pragma unroll
     for (int e = 0; e < P; ++e) {
       o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
       o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
     }
-    uint16_t* dst = is_q ? q_out + (tok * Hq + h) * (int64_t)hd
+    uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd
                          : k_cache + ((int64_t)p * Hkv + (h - Hq)) * hd;
     store_packed<DT, P>(dst + j0, o1);
     store_packed<DT, P>(dst + half + j0, o2);
@@ -168,19 +171,21 @@ struct Args {
   void* kc;
   void* vc;
   int32_t* status;
-  int64_t units;
-  int H, Hq, Hkv, hd, G, max_pos, capacity;
+  int M, H, Hq, Hkv, hd, G, max_pos, capacity;
   float eps;
 };
 
+// One CTA per (token, group of HB heads): HB = all heads when H * GP <= 1024.
 template <int DT, int P, int GP>
 frt_status launch_gp(const Args& a, cudaStream_t st) {
-  const int64_t threads = a.units * GP;
-  const dim3 grid((unsigned)((threads + kThreads - 1) / kThreads));
-  return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP>, grid, dim3(kThreads), st,
+  const int HB = a.H * GP <= 1024 ? a.H : 1024 / GP;
+  const int nhb = (a.H + HB - 1) / HB;
+  const int threads = ((HB * GP + 31) / 32) * 32;
+  const dim3 grid((unsigned)((int64_t)a.M * nhb));
+  return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP>, grid, dim3(threads), 0, st,
                 static_cast<const uint16_t*>(a.qkv), static_cast<const uint16_t*>(a.qw),
                 static_cast<const uint16_t*>(a.kw), a.cos_tab, a.sin_tab, a.pos, static_cast<uint16_t*>(a.q_out),
-                static_cast<uint16_t*>(a.kc), static_cast<uint16_t*>(a.vc), a.status, a.units, a.H, a.Hq, a.Hkv,
+                static_cast<uint16_t*>(a.kc), static_cast<uint16_t*>(a.vc), a.status, a.H, HB, nhb, a.Hq, a.Hkv,
                 a.hd, a.G, a.max_pos, a.capacity, a.eps);
 }
 
@@ -228,7 +233,8 @@ extern "C" frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_n
   int GP = 1;
   while (GP < G) GP *= 2;
   Args a{qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status,
-         (int64_t)M * H, H, Hq, Hkv, hd, G, max_pos, capacity, eps};
-  if ((a.units * GP + kThreads - 1) / kThreads > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
+         M, H, Hq, Hkv, hd, G, max_pos, capacity, eps};
+  const int64_t HB = (int64_t)H * GP <= 1024 ? H : 1024 / GP;
+  if ((int64_t)M * ((H + HB - 1) / HB) > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
   return dt == FRT_F16 ? launch_dt<FRT_F16>(P, GP, a, stream) : launch_dt<FRT_BF16>(P, GP, a, stream);
 }

@@ -6,12 +6,13 @@
 // (new residual + FP8 codes).  §三: the `_noweight` variant drops the weight
 // multiply because (1 + w) already lives in the next GEMM's weights.
 //
-// Mapping (B200): one CTA per row; the row is split into 16-byte chunks of 8
+// Mapping (B200): one small CTA per row (128 threads for D <= 16384, so up to
+// 16 rows are in flight per SM); the row is split into 16-byte chunks of 8
 // elements and thread t owns chunks t, t+T, t+2T, ... (K of them), so every
 // warp-wide load or store is one contiguous, fully used 512-byte run.  The sum
 // of squares is reduced warp-shuffle -> shared memory -> every thread, in a
-// fixed order (bitwise deterministic), with a compensated fp32 pair so the
-// normalised values come out correctly rounded.  For block-128 scales a 128-column block
+// fixed order (bitwise deterministic), in fp64 so the normalised values come
+// out correctly rounded in fp32.  For block-128 scales a 128-column block
 // is 16 chunks owned by 16 consecutive lanes, so its amax is a 4-step xor
 // shuffle inside the warp; no shared memory and no second pass.
 #include <cmath>
@@ -22,10 +23,12 @@
 namespace frt {
 namespace {
 
-// Threads per CTA are at most 256 for K <= 2 and 512 for K >= 4.
+// Threads per CTA: at most 128 for K <= 2, 512 for K >= 4 (128 at D = 4096).
+// Small CTAs keep many rows in flight per SM, which is what hides each row's
+// load -> reduce -> quantise latency.
 template <int K>
 constexpr int max_threads() {
-  return K >= 4 ? 512 : 256;
+  return K >= 4 ? 512 : 128;
 }
 
 template <int DT, int K, bool WEIGHTED, int QM>
@@ -39,6 +42,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   const int T = blockDim.x;
   const int64_t row = blockIdx.x;
   const int64_t base = row * (int64_t)C;
+  __shared__ double red[32];
 
   // Issue every load of the row before any store (r_out may alias r_in).
   uint4 xv[K], rv[K];
@@ -50,93 +54,91 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       rv[k] = ld_plain(r_in + base + c);
     }
   }
+  float s_static = 0.0f;
+  if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
 
-  float h[K][8];
-  Sum2 ss{0.0f, 0.0f};
+  // Pass 1: h = x + r rounded once to 16 bits (exactly the rounded exact sum,
+  // see add_for_16), kept packed; fp64 sum of squares (squares of 16-bit
+  // values are exact, so the sum is exact to ~2^-40), one accumulator per chunk.
+  uint4 hv[K];
+  double ss[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
+    ss[k] = 0.0;
     const int c = t + k * T;
     if (c < C) {
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv[k]);
       const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rv[k]);
-      uint4 hv;
-      uint32_t* hw = reinterpret_cast<uint32_t*>(&hv);
+      uint32_t* hw = reinterpret_cast<uint32_t*>(&hv[k]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 xf = P16::to_float2(xw[e]);
         const float2 rf = P16::to_float2(rw[e]);
-        hw[e] = P16::from_float2(add_round_odd(xf.x, rf.x), add_round_odd(xf.y, rf.y));
-        const float2 hf = P16::to_float2(hw[e]);
-        h[k][2 * e] = hf.x;
-        h[k][2 * e + 1] = hf.y;
-        ss.add(hf.x * hf.x);  // squares of 16-bit values are exact in fp32
-        ss.add(hf.y * hf.y);
+        hw[e] = P16::from_float2(add_for_16(xf.x, rf.x), add_for_16(xf.y, rf.y));
       }
-      r_out[base + c] = hv;
-    } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) h[k][e] = 0.0f;
+      for (int e = 0; e < 4; ++e) {
+        const float2 hf = P16::to_float2(hw[e]);
+        ss[k] = fma((double)hf.x, (double)hf.x, ss[k]);
+        ss[k] = fma((double)hf.y, (double)hf.y, ss[k]);
+      }
+      r_out[base + c] = hv[k];
+    } else {
+      hv[k] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  double sst = ss[0];
+#pragma unroll
+  for (int k = 1; k < K; ++k) sst += ss[k];
 
-  // Row sum of squares, compensated: warp butterfly, then every thread adds
-  // the warp partials in the same order.  rstd is formed in fp64 from the
-  // ~2^-48-accurate sum, and y = h * w * rstd is rounded once to fp32 (h * w
-  // is exact for 16-bit operands), so y is the correctly rounded fp32 value of
-  // the exact normalised element: FP8 codes are then decided on the same fp32
-  // value an exact computation would give.
-  __shared__ float red_hi[32], red_lo[32];
-  ss = group_sum2<32>(ss);
-  if ((t & 31) == 0) {
-    red_hi[t >> 5] = ss.hi;
-    red_lo[t >> 5] = ss.lo;
-  }
+  // Row total: warp butterfly, then every thread adds the warp partials in
+  // the same order and forms rstd in fp64.  y = h * w * rstd is rounded once
+  // to fp32 (h * w is exact for 16-bit operands), so y is the correctly
+  // rounded fp32 value of the exact normalised element and the FP8 codes are
+  // decided on the value an exact computation would give.
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sst += __shfl_xor_sync(0xFFFFFFFFu, sst, o);
+  if ((t & 31) == 0) red[t >> 5] = sst;
   __syncthreads();
-  Sum2 tot{red_hi[0], red_lo[0]};
+  double tot = 0.0;
   const int nw = T >> 5;
-  for (int i = 1; i < nw; ++i) tot.add(Sum2{red_hi[i], red_lo[i]});
-  const double ms = ((double)tot.hi + (double)tot.lo) / (double)D;
-  const Split32 rstd(1.0 / sqrt(ms + (double)eps));
-
-  float s_static = 0.0f;
-  if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
+  for (int i = 0; i < nw; ++i) tot += red[i];
+  const Split32 rstd(rsqrt_f64(tot / (double)D + (double)eps));
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
 
+  // Pass 2: y and its FP8 codes.
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = t + k * T;
     const bool valid = c < C;
+    const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv[k]);
     float y[8];
     if (WEIGHTED && valid) {
       const uint4 wv = __ldg(w + c);
       const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
+        const float2 hf = P16::to_float2(hw[e]);
         const float2 wf = P16::to_float2(ww[e]);
-        y[2 * e] = rstd.mul(h[k][2 * e] * wf.x);
-        y[2 * e + 1] = rstd.mul(h[k][2 * e + 1] * wf.y);
+        y[2 * e] = rstd.mul(hf.x * wf.x);
+        y[2 * e + 1] = rstd.mul(hf.y * wf.y);
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = rstd.mul(h[k][e]);
+      for (int e = 0; e < 4; ++e) {
+        const float2 hf = P16::to_float2(hw[e]);
+        y[2 * e] = rstd.mul(hf.x);
+        y[2 * e + 1] = rstd.mul(hf.y);
+      }
     }
     if (QM == FRT_QUANT_BLOCK128) {
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
       am = group_max<16>(am);  // 16 lanes = the 16 chunks of one 128-column block
       const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
       if (valid && (t & 15) == 0) block_scales[row * NB + (c >> 4)] = sb;
-      if (valid) {
-        const Divisor dv(sb);
-        uint2 o;
-        o.x = e4m3x4(dv.div(y[0]), dv.div(y[1]), dv.div(y[2]), dv.div(y[3]));
-        o.y = e4m3x4(dv.div(y[4]), dv.div(y[5]), dv.div(y[6]), dv.div(y[7]));
-        q[base + c] = o;
-      }
+      if (valid) q[base + c] = quant8(y, Divisor(sb));
     } else if (valid) {
-      uint2 o;
-      o.x = e4m3x4(dv_static.div(y[0]), dv_static.div(y[1]), dv_static.div(y[2]), dv_static.div(y[3]));
-      o.y = e4m3x4(dv_static.div(y[4]), dv_static.div(y[5]), dv_static.div(y[6]), dv_static.div(y[7]));
-      q[base + c] = o;
+      q[base + c] = quant8(y, dv_static);
     }
   }
 }
@@ -144,9 +146,10 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
 template <int DT, int K, bool W, int QM>
 frt_status launch_k(const void* x, const void* r_in, void* r_out, const void* w, uint8_t* q, const float* ss,
                     float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
-  return launch(residual_rmsnorm_fp8_kernel<DT, K, W, QM>, dim3(M), dim3(T), st, static_cast<const uint4*>(x),
-                static_cast<const uint4*>(r_in), static_cast<uint4*>(r_out), static_cast<const uint4*>(w),
-                reinterpret_cast<uint2*>(q), ss, bs, C, NB, (float)(C * 8), eps);
+  auto kern = residual_rmsnorm_fp8_kernel<DT, K, W, QM>;
+  return launch(kern, dim3(M), dim3(T), 0, st, static_cast<const uint4*>(x), static_cast<const uint4*>(r_in),
+                static_cast<uint4*>(r_out), static_cast<const uint4*>(w), reinterpret_cast<uint2*>(q), ss, bs, C, NB,
+                (float)(C * 8), eps);
 }
 
 template <int DT, int K>
@@ -180,9 +183,10 @@ frt_status launch_dt(int K, bool weighted, frt_quant qm, const void* x, const vo
 }  // namespace
 
 // Chunks per thread (K) and threads per row (T) for a row of C 16-byte
-// chunks: K = 1 up to D = 2048, 2 up to 4096, 4 up to 16384, 8 up to 32768.
+// chunks (D = 8C): K = 1 up to D = 1024, 2 up to 2048, 4 up to 16384 (128 to
+// 512 threads), 8 up to 32768.
 static void rmsnorm_shape(int C, int* K, int* T) {
-  const int k = C <= 256 ? 1 : C <= 512 ? 2 : C <= 2048 ? 4 : 8;
+  const int k = C <= 128 ? 1 : C <= 256 ? 2 : C <= 2048 ? 4 : 8;
   const int per = (C + k - 1) / k;
   *K = k;
   *T = ((per + 31) / 32) * 32;
