@@ -12,9 +12,10 @@
 // [hd/2 + lP, ...), P = 8 (16-byte vectors) when hd % 16 == 0, else P = 4
 // (8-byte vectors; e.g. the unpadded head_dim 72 of the ViT).  The per-head
 // sum of squares is an xor shuffle inside the group.  A CTA holds one token's
-// heads (all of them when heads x GP <= 1024), so the token's position and
-// cos/sin row are read once into L1 and shared by every head, and no thread
-// divides by the head count.
+// heads (or a block of them), so the token's position and cos/sin row are
+// read once per lane and shared by every head the lane handles; on large
+// batches each lane group takes up to four heads to keep more bytes in flight.
+#include <atomic>
 #include <cmath>
 
 #include "frt_device.cuh"
@@ -71,92 +72,225 @@ __device__ __forceinline__ void ld_f32(const float* p, float* f) {
   }
 }
 
-template <int DT, int P, int GP>
-__global__ void __launch_bounds__(1024) qkv_norm_rope_kvcache_kernel(
+// Register kernel (small batches, or pointers below 16-byte alignment).  One
+// CTA per (token, block of heads).  The CTA's NG lane groups take up to HPG
+// heads each: slot i of group g is head (hb * hpg + i) * NG + g, so for every
+// slot consecutive groups read consecutive heads.  All slots' loads are issued
+// first and a lane's cos/sin slice is loaded once for all its heads.
+template <int DT, int P, int GP, int HPG>
+__global__ void __launch_bounds__(HPG == 1 ? 1024 : 256) qkv_norm_rope_kvcache_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
     const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
     const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, uint16_t* __restrict__ k_cache,
-    uint16_t* __restrict__ v_cache, int32_t* status, int H, int HB, int nhb, int Hq, int Hkv, int hd, int G,
-    int max_pos, int capacity, float eps) {
+    uint16_t* __restrict__ v_cache, int32_t* status, int H, int NG, int hpg, int nhb, int Hq, int Hkv, int hd,
+    int G, int max_pos, int capacity, float eps) {
+  using V = typename Vec16<P>::T;
   pdl_enter();
-  // CTA = (token, group of HB heads); GP lanes per head.
   const int tok = blockIdx.x / nhb;
-  const int h = (blockIdx.x - tok * nhb) * HB + (int)(threadIdx.x / GP);
+  const int hb = blockIdx.x - tok * nhb;
+  const int grp = (int)(threadIdx.x / GP);
   const int li = threadIdx.x & (GP - 1);
-  const bool in_range = threadIdx.x < (unsigned)(HB * GP) && h < H;
-
+  const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G;
   const int p = __ldg(positions + tok);
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
-  if (!row_ok && threadIdx.x == 0 && blockIdx.x == tok * nhb && status != nullptr) atomicOr(status, 1);
-  const bool active = in_range && row_ok && li < G;
+  if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
+  const bool active = lane_ok && row_ok;
   const int half = hd >> 1;
   const int j0 = li * P;
-  const bool is_q = h < Hq;
-  const bool is_v = h >= Hq + Hkv;
-  const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
-  const bool do_norm = !is_v && nw != nullptr;
-
-  // Issue the QKV loads first and prefetch the token's cos/sin slice into L1
-  // (no registers held), so the table's latency overlaps the QKV loads and
-  // the per-head reduction; the table is read after the reduction.
-  const uint16_t* src = qkv + ((int64_t)tok * H + h) * hd;
-  const float* crow = cos_tab + (int64_t)p * half + j0;
-  const float* srow = sin_tab + (int64_t)p * half + j0;
-  typename Vec16<P>::T va, vb;
+  const uint16_t* row = qkv + (int64_t)tok * H * hd;
+  V va[HPG], vb[HPG];
+#pragma unroll
+  for (int i = 0; i < HPG; ++i) {
+    const int h = (hb * hpg + i) * NG + grp;
+    if (active && i < hpg && h < H) {
+      va[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + j0);
+      vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
+    }
+  }
+  float c[P], s[P];
   if (active) {
-    va = *reinterpret_cast<const typename Vec16<P>::T*>(src + j0);
-    vb = *reinterpret_cast<const typename Vec16<P>::T*>(src + half + j0);
-    if (!is_v) {
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(crow));
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(srow));
-    }
+    ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
+    ld_f32<P>(sin_tab + (int64_t)p * half + j0, s);
   }
-
-  if (is_v) {  // V: bit copy into the cache slot
-    if (active) {
+#pragma unroll
+  for (int i = 0; i < HPG; ++i) {
+    if (i >= hpg) break;  // uniform across the CTA
+    const int h = (hb * hpg + i) * NG + grp;
+    const bool on = active && h < H;
+    const bool is_q = h < Hq;
+    const bool is_v = h >= Hq + Hkv;
+    const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
+    const bool do_norm = !is_v && nw != nullptr;
+    if (on && is_v) {  // V: bit copy into the cache slot
       uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
-      *reinterpret_cast<typename Vec16<P>::T*>(dst + j0) = va;
-      *reinterpret_cast<typename Vec16<P>::T*>(dst + half + j0) = vb;
+      *reinterpret_cast<V*>(dst + j0) = va[i];
+      *reinterpret_cast<V*>(dst + half + j0) = vb[i];
     }
-  }
-
-  float a[P], b[P];
-  float ss = 0.0f;
-  if (active && !is_v) {
-    unpack<DT, P>(va, a);
-    unpack<DT, P>(vb, b);
-    if (do_norm) {
+    float a[P], b[P];
+    float ss = 0.0f;
+    if (on && !is_v) {
+      unpack<DT, P>(va[i], a);
+      unpack<DT, P>(vb[i], b);
+      if (do_norm) {
 #pragma unroll
-      for (int e = 0; e < P; ++e) ss = fmaf(b[e], b[e], fmaf(a[e], a[e], ss));
-    }
-  }
-  ss = group_sum<GP>(ss);  // every lane of the warp takes part
-
-  if (active && !is_v) {
-    if (do_norm) {
-      const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
-      float fa[P], fb[P];
-      unpack<DT, P>(ld_vec<P>(nw + j0), fa);
-      unpack<DT, P>(ld_vec<P>(nw + half + j0), fb);
-#pragma unroll
-      for (int e = 0; e < P; ++e) {
-        a[e] = a[e] * rstd * fa[e];
-        b[e] = b[e] * rstd * fb[e];
+        for (int e = 0; e < P; ++e) ss = fmaf(b[e], b[e], fmaf(a[e], a[e], ss));
       }
     }
-    float c[P], s[P];
-    ld_f32<P>(crow, c);
-    ld_f32<P>(srow, s);
-    float o1[P], o2[P];
+    ss = group_sum<GP>(ss);  // every lane of the warp takes part
+    if (on && !is_v) {
+      if (do_norm) {
+        const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
+        float fa[P], fb[P];
+        unpack<DT, P>(ld_vec<P>(nw + j0), fa);
+        unpack<DT, P>(ld_vec<P>(nw + half + j0), fb);
+#pragma unroll
+        for (int e = 0; e < P; ++e) {
+          a[e] = a[e] * rstd * fa[e];
+          b[e] = b[e] * rstd * fb[e];
+        }
+      }
+      float o1[P], o2[P];
+#pragma unroll
+      for (int e = 0; e < P; ++e) {
+        o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
+        o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
+      }
+      uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + (h - Hq)) * hd;
+      store_packed<DT, P>(dst + j0, o1);
+      store_packed<DT, P>(dst + half + j0, o2);
+    }
+  }
+}
+
+// Polls of a bulk-copy barrier before the kernel gives up (each poll may
+// suspend the thread for a while; the bound is far beyond any real copy).
+constexpr int kMaxPolls = 1 << 22;
+
+// Bulk-copy kernel (large batches).  One CTA per token.  One thread moves the
+// token's whole QKV row, its cos/sin rows and both norm weights into shared
+// memory with 1-D bulk copies (TMA) completed on an mbarrier, so no register
+// holds in-flight data and a small CTA keeps 12+ KB per token in flight.  Lane
+// groups (GP lanes per head) normalise and rotate the Q and K heads in place;
+// then the Q row, the K row and the untouched V row leave as three bulk
+// stores.  A barrier wait that runs out of polls sets bit 1 of *status and the
+// CTA returns without writing.
+template <int DT, int P, int GP>
+__global__ void __launch_bounds__(256) qkv_norm_rope_kvcache_tma_kernel(
+    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
+    const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
+    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, uint16_t* __restrict__ k_cache,
+    uint16_t* __restrict__ v_cache, int32_t* status, int H, int NG, int Hq, int Hkv, int hd, int G, int max_pos,
+    int capacity, float eps) {
+  using V = typename Vec16<P>::T;
+  pdl_enter();
+  extern __shared__ __align__(128) uint8_t dsmem[];  // [QKV row][cos][sin][q weight][k weight]
+  __shared__ uint64_t bar;
+  __shared__ int s_pos;
+  const int tok = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int half = hd >> 1;
+  const unsigned row_bytes = (unsigned)(H * hd * 2);
+  const unsigned tab_bytes = (unsigned)(half * 4);
+  const unsigned w_bytes = (unsigned)(hd * 2);
+  uint16_t* rowbuf = reinterpret_cast<uint16_t*>(dsmem);
+  float* cbuf = reinterpret_cast<float*>(dsmem + row_bytes);
+  float* sbuf = cbuf + half;
+  uint16_t* qwbuf = reinterpret_cast<uint16_t*>(sbuf + half);
+  uint16_t* kwbuf = qwbuf + hd;
+
+  if (tid == 0) {
+    mbar_init(&bar, 2);  // two arrivals: the row (+ weights), then the table rows
+    mbar_init_fence();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned first = row_bytes + (q_norm_w ? w_bytes : 0u) + (k_norm_w ? w_bytes : 0u);
+    mbar_arrive_expect_tx(&bar, first);
+    bulk_load(rowbuf, qkv + (int64_t)tok * H * hd, row_bytes, &bar);
+    if (q_norm_w) bulk_load(qwbuf, q_norm_w, w_bytes, &bar);
+    if (k_norm_w) bulk_load(kwbuf, k_norm_w, w_bytes, &bar);
+    const int p = __ldg(positions + tok);
+    const bool ok = p >= 0 && p < max_pos && p < capacity;
+    s_pos = ok ? p : -1;
+    if (ok) {
+      mbar_arrive_expect_tx(&bar, 2 * tab_bytes);
+      bulk_load(cbuf, cos_tab + (int64_t)p * half, tab_bytes, &bar);
+      bulk_load(sbuf, sin_tab + (int64_t)p * half, tab_bytes, &bar);
+    } else {
+      if (status != nullptr) atomicOr(status, 1);
+      mbar_arrive_expect_tx(&bar, 0u);
+    }
+  }
+  const bool landed = mbar_wait_bounded(&bar, 0, kMaxPolls);
+  if (!__syncthreads_and(landed)) {
+    if (tid == 0 && status != nullptr) atomicOr(status, 2);
+    mbar_wait_bounded(&bar, 0, kMaxPolls);  // give copies still in flight a last chance to land
+    return;
+  }
+  const int p = s_pos;
+  if (p < 0) return;  // position out of range: nothing is written
+
+  const int grp = tid / GP;
+  const int li = tid & (GP - 1);
+  const bool lane_ok = grp < NG && li < G;
+  const int j0 = li * P;
+  float c[P], s[P];
+  if (lane_ok) {
 #pragma unroll
     for (int e = 0; e < P; ++e) {
-      o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
-      o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
+      c[e] = cbuf[j0 + e];
+      s[e] = sbuf[j0 + e];
     }
-    uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd
-                         : k_cache + ((int64_t)p * Hkv + (h - Hq)) * hd;
-    store_packed<DT, P>(dst + j0, o1);
-    store_packed<DT, P>(dst + half + j0, o2);
+  }
+  const int nslots = (Hq + Hkv + NG - 1) / NG;  // Q and K heads only; V leaves untouched
+  for (int i = 0; i < nslots; ++i) {
+    const int h = i * NG + grp;
+    const bool on = lane_ok && h < Hq + Hkv;
+    const bool is_q = h < Hq;
+    const uint16_t* nwg = is_q ? q_norm_w : k_norm_w;
+    const uint16_t* nws = is_q ? qwbuf : kwbuf;
+    uint16_t* vec = rowbuf + h * hd;
+    float a[P], b[P];
+    float ss = 0.0f;
+    if (on) {
+      unpack<DT, P>(*reinterpret_cast<const V*>(vec + j0), a);
+      unpack<DT, P>(*reinterpret_cast<const V*>(vec + half + j0), b);
+      if (nwg != nullptr) {
+#pragma unroll
+        for (int e = 0; e < P; ++e) ss = fmaf(b[e], b[e], fmaf(a[e], a[e], ss));
+      }
+    }
+    ss = group_sum<GP>(ss);  // every lane of the warp takes part
+    if (on) {
+      if (nwg != nullptr) {
+        const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
+        float fa[P], fb[P];
+        unpack<DT, P>(*reinterpret_cast<const V*>(nws + j0), fa);
+        unpack<DT, P>(*reinterpret_cast<const V*>(nws + half + j0), fb);
+#pragma unroll
+        for (int e = 0; e < P; ++e) {
+          a[e] = a[e] * rstd * fa[e];
+          b[e] = b[e] * rstd * fb[e];
+        }
+      }
+      float o1[P], o2[P];
+#pragma unroll
+      for (int e = 0; e < P; ++e) {
+        o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
+        o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
+      }
+      store_packed<DT, P>(vec + j0, o1);
+      store_packed<DT, P>(vec + half + j0, o2);
+    }
+  }
+  fence_proxy_async_smem();  // this thread's writes -> the bulk stores below
+  __syncthreads();
+  if (tid == 0) {
+    bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
+    bulk_store(k_cache + (int64_t)p * Hkv * hd, rowbuf + Hq * hd, (unsigned)(Hkv * hd * 2));
+    bulk_store(v_cache + (int64_t)p * Hkv * hd, rowbuf + (Hq + Hkv) * hd, (unsigned)(Hkv * hd * 2));
+    bulk_commit();
+    bulk_wait_all();  // shared memory must outlive the stores; writes done before exit
   }
 }
 
@@ -175,35 +309,97 @@ struct Args {
   float eps;
 };
 
-// One CTA per (token, group of HB heads): HB = all heads when H * GP <= 1024.
+// CTA shape for GP lanes per head.  Small batches (launch/latency-bound):
+// one head per group and up to 1024 threads per token.  Large batches: up to
+// four heads per group, NG = ceil(H / 4) groups (at most 256 threads), so each
+// thread keeps four heads' loads in flight.
+struct Shape {
+  int NG, hpg, nhb, threads;
+};
+
+inline Shape qkv_shape(int M, int H, int GP) {
+  Shape sh;
+  const bool large = M >= 4 * 148;
+  if (large && H >= 2) {
+    sh.NG = (H + 3) / 4;
+    if (sh.NG * GP > 256) sh.NG = 256 / GP;
+    sh.hpg = (H + sh.NG - 1) / sh.NG;
+    if (sh.hpg > 4) sh.hpg = 4;
+  } else {
+    sh.NG = H * GP <= 1024 ? H : 1024 / GP;
+    sh.hpg = 1;
+  }
+  sh.nhb = (H + sh.NG * sh.hpg - 1) / (sh.NG * sh.hpg);
+  sh.threads = ((sh.NG * GP + 31) / 32) * 32;
+  return sh;
+}
+
+template <typename Kern>
+frt_status opt_in_smem(Kern kern, size_t bytes, std::atomic<int>& opted) {
+  if ((int)bytes > opted.load(std::memory_order_relaxed)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return FRT_ERR_CUDA;
+    }
+    int cur = opted.load(std::memory_order_relaxed);
+    while ((int)bytes > cur && !opted.compare_exchange_weak(cur, (int)bytes)) {
+    }
+  }
+  return FRT_OK;
+}
+
+// Shared memory of the bulk-copy kernel: the QKV row, cos and sin rows, two
+// norm weights.
+inline size_t tma_smem(int H, int hd) { return (size_t)H * hd * 2 + (size_t)hd * 4 + (size_t)hd * 4; }
+constexpr size_t kTmaSmemMax = 200 * 1024;
+
 template <int DT, int P, int GP>
-frt_status launch_gp(const Args& a, cudaStream_t st) {
-  const int HB = a.H * GP <= 1024 ? a.H : 1024 / GP;
-  const int nhb = (a.H + HB - 1) / HB;
-  const int threads = ((HB * GP + 31) / 32) * 32;
-  const dim3 grid((unsigned)((int64_t)a.M * nhb));
-  return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP>, grid, dim3(threads), 0, st,
-                static_cast<const uint16_t*>(a.qkv), static_cast<const uint16_t*>(a.qw),
-                static_cast<const uint16_t*>(a.kw), a.cos_tab, a.sin_tab, a.pos, static_cast<uint16_t*>(a.q_out),
-                static_cast<uint16_t*>(a.kc), static_cast<uint16_t*>(a.vc), a.status, a.H, HB, nhb, a.Hq, a.Hkv,
-                a.hd, a.G, a.max_pos, a.capacity, a.eps);
+frt_status launch_gp(const Args& a, bool tma, cudaStream_t st) {
+  const uint16_t* qkv = static_cast<const uint16_t*>(a.qkv);
+  const uint16_t* qw = static_cast<const uint16_t*>(a.qw);
+  const uint16_t* kw = static_cast<const uint16_t*>(a.kw);
+  uint16_t* qo = static_cast<uint16_t*>(a.q_out);
+  uint16_t* kc = static_cast<uint16_t*>(a.kc);
+  uint16_t* vc = static_cast<uint16_t*>(a.vc);
+  if (tma) {
+    static std::atomic<int> opted{0};
+    auto kt = qkv_norm_rope_kvcache_tma_kernel<DT, P, GP>;
+    const size_t smem = tma_smem(a.H, a.hd);
+    const frt_status os = opt_in_smem(kt, smem, opted);
+    if (os != FRT_OK) return os;
+    const int per = a.Hq + a.Hkv;  // lane groups needed for one slot of every Q/K head
+    int NG = (per * GP <= 128) ? per : 128 / GP;
+    if (NG < 1) NG = 1;
+    const int threads = ((NG * GP + 31) / 32) * 32;
+    return launch(kt, dim3((unsigned)a.M), dim3(threads), smem, st, qkv, qw, kw, a.cos_tab, a.sin_tab, a.pos, qo,
+                  kc, vc, a.status, a.H, NG, a.Hq, a.Hkv, a.hd, a.G, a.max_pos, a.capacity, a.eps);
+  }
+  const Shape sh = qkv_shape(a.M, a.H, GP);
+  const dim3 grid((unsigned)((int64_t)a.M * sh.nhb));
+  if (sh.hpg == 1)
+    return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP, 1>, grid, dim3(sh.threads), 0, st, qkv, qw, kw,
+                  a.cos_tab, a.sin_tab, a.pos, qo, kc, vc, a.status, a.H, sh.NG, sh.hpg, sh.nhb, a.Hq, a.Hkv, a.hd,
+                  a.G, a.max_pos, a.capacity, a.eps);
+  return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP, 4>, grid, dim3(sh.threads), 0, st, qkv, qw, kw, a.cos_tab,
+                a.sin_tab, a.pos, qo, kc, vc, a.status, a.H, sh.NG, sh.hpg, sh.nhb, a.Hq, a.Hkv, a.hd, a.G,
+                a.max_pos, a.capacity, a.eps);
 }
 
 template <int DT, int P>
-frt_status launch_p(int GP, const Args& a, cudaStream_t st) {
+frt_status launch_p(int GP, const Args& a, bool tma, cudaStream_t st) {
   switch (GP) {
-    case 1: return launch_gp<DT, P, 1>(a, st);
-    case 2: return launch_gp<DT, P, 2>(a, st);
-    case 4: return launch_gp<DT, P, 4>(a, st);
-    case 8: return launch_gp<DT, P, 8>(a, st);
-    case 16: return launch_gp<DT, P, 16>(a, st);
-    default: return launch_gp<DT, P, 32>(a, st);
+    case 1: return launch_gp<DT, P, 1>(a, tma, st);
+    case 2: return launch_gp<DT, P, 2>(a, tma, st);
+    case 4: return launch_gp<DT, P, 4>(a, tma, st);
+    case 8: return launch_gp<DT, P, 8>(a, tma, st);
+    case 16: return launch_gp<DT, P, 16>(a, tma, st);
+    default: return launch_gp<DT, P, 32>(a, tma, st);
   }
 }
 
 template <int DT>
-frt_status launch_dt(int P, int GP, const Args& a, cudaStream_t st) {
-  return P == 8 ? launch_p<DT, 8>(GP, a, st) : launch_p<DT, 4>(GP, a, st);
+frt_status launch_dt(int P, int GP, const Args& a, bool tma, cudaStream_t st) {
+  return P == 8 ? launch_p<DT, 8>(GP, a, tma, st) : launch_p<DT, 4>(GP, a, tma, st);
 }
 
 }  // namespace
@@ -234,7 +430,12 @@ extern "C" frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_n
   while (GP < G) GP *= 2;
   Args a{qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status,
          M, H, Hq, Hkv, hd, G, max_pos, capacity, eps};
-  const int64_t HB = (int64_t)H * GP <= 1024 ? H : 1024 / GP;
-  if ((int64_t)M * ((H + HB - 1) / HB) > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
-  return dt == FRT_F16 ? launch_dt<FRT_F16>(P, GP, a, stream) : launch_dt<FRT_BF16>(P, GP, a, stream);
+  if ((int64_t)M * qkv_shape(M, H, GP).nhb > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
+  // Bulk-copy path for large batches when every row it moves is 16-byte
+  // aligned (bulk copies need 16-byte addresses and sizes) and fits in
+  // shared memory; the register kernel otherwise.
+  const bool tma = M >= 4 * 148 && aligned(qkv, 16) && aligned(q_out, 16) && aligned(k_cache, 16) &&
+                   aligned(v_cache, 16) && (!q_norm_w || aligned(q_norm_w, 16)) &&
+                   (!k_norm_w || aligned(k_norm_w, 16)) && tma_smem(H, hd) <= kTmaSmemMax;
+  return dt == FRT_F16 ? launch_dt<FRT_F16>(P, GP, a, tma, stream) : launch_dt<FRT_BF16>(P, GP, a, tma, stream);
 }
