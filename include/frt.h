@@ -134,10 +134,15 @@ frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residual_in, void
  *   q_out               device [M, Hq, hd] 16-bit.
  *   k_cache, v_cache    device [capacity, Hkv, hd] 16-bit; rows other than the
  *                       M written slots are left untouched.
- *   status              device int32[1] or NULL.  A row whose position is
- *                       < 0, >= max_pos or >= capacity is skipped entirely
- *                       (no Q, K or V write) and bit 0 of *status is set with
- *                       an atomic OR; the word is never cleared by the call.
+ *   status              device int32[1] or NULL.  Bits are set with an atomic
+ *                       OR and never cleared by the call:
+ *                       bit 0  a row's position is < 0, >= max_pos or
+ *                              >= capacity; that row is skipped entirely (no
+ *                              Q, K or V write);
+ *                       bit 1  a kernel gave up waiting for its own bulk copy
+ *                              (a bounded wait ran out; only a failing device
+ *                              can cause it); that token's outputs are not
+ *                              written.
  *   16-bit pointers must be 16-byte aligned when hd % 16 == 0 and 8-byte
  *   aligned otherwise.
  *   Layout rule: Hq, Hkv > 0, Hq % Hkv == 0, hd > 0 and even, max_pos > 0,

@@ -157,22 +157,6 @@ __device__ __forceinline__ uint4 ld_plain(const uint4* p) {
   return v;
 }
 
-// Per-thread asynchronous 16-byte global -> shared copy (L2 only), with
-// commit/wait on this thread's own copy groups.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // ------------------------------------------------------ bulk copies (TMA) --
 // 1-D bulk copies between global and shared memory (cp.async.bulk), completed
 // through an mbarrier.  Addresses must be 16-byte aligned and sizes multiples

@@ -47,11 +47,6 @@ inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
   return launch_status();
 }
 
-// Resident CTAs per SM x SMs for `kernel` at `threads` threads and `smem`
-// bytes of dynamic shared memory (cached per kernel, block size and device):
-// the grid size of a persistent launch.
-int persistent_grid(const void* kernel, int threads, size_t smem = 0);
-
 // Checks shared by the two FP8-producing ops: the pointer the quant mode needs.
 inline bool quant_args_ok(frt_quant qm, const float* static_scale, const float* block_scales) {
   if (qm == FRT_QUANT_STATIC) return static_scale != nullptr && aligned(static_scale, 4);

@@ -2,8 +2,6 @@
 #include "frt_host.h"
 
 #include <atomic>
-#include <mutex>
-#include <unordered_map>
 
 #include "frt_device.cuh"
 
@@ -15,28 +13,6 @@ std::atomic<int> g_pdl{1};
 
 bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
 
-int persistent_grid(const void* kernel, int threads, size_t smem) {
-  static std::mutex mu;
-  static std::unordered_map<uint64_t, int> cache;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  const uint64_t key = reinterpret_cast<uintptr_t>(kernel) ^ ((uint64_t)threads << 40) ^ ((uint64_t)dev << 56);
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
-  }
-  int sms = 0, per_sm = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return 0;
-  }
-  const int g = sms * (per_sm > 0 ? per_sm : 1);
-  std::lock_guard<std::mutex> lk(mu);
-  cache[key] = g;
-  return g;
-}
 }  // namespace frt
 
 extern "C" frt_status frt_noop(int grid, int block, cudaStream_t stream) {
