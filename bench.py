@@ -39,7 +39,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import numpy as np
@@ -59,7 +58,7 @@ L2_FLUSH_BYTES = 512 << 20
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=500)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="large_m_M65536")
@@ -77,6 +76,53 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+class Dist:
+    """Process-group plumbing of a multi-rank run (one process per GPU): a
+    barrier and a max over ranks.  Single-process runs need no group."""
+
+    def __init__(self, world, backend="nccl", device=None, timeout_s=120):
+        self.world = world
+        self.pg = None
+        self.device = device
+        if world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"timeout": datetime.timedelta(seconds=timeout_s)}
+            if backend == "nccl" and device is not None:
+                kw["device_id"] = device
+            dist.init_process_group(backend, **kw)
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max_over_ranks(self, x):
+        if self.pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=self.device if self.device is not None else "cpu")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.barrier()
+            self.pg.destroy_process_group()
+            self.pg = None
+
+
+def rank_workload(wl, rank):
+    """Each rank draws its own row shard: same shapes, seed offset by rank
+    (weak scaling: per-rank work is fixed as ranks are added)."""
+    import dataclasses
+    return dataclasses.replace(wl, seed=wl.seed + 1000 * rank, layers=1, steps=1)
+
+
+def job_throughput(bytes_per_rank, world, ms_per_step_max):
+    """Whole-job GB/s: bytes all ranks moved / the slowest rank's time."""
+    return bytes_per_rank * world / (ms_per_step_max * 1e-3) / 1e9
 
 
 def measured_peak():
@@ -164,6 +210,35 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
                 "reasons": reasons, "samples": len(rows), "samples_busy": len(busy),
                 "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+def kernel_source_hash():
+    """sha256 over the CUDA sources: ties a recorded ncu traffic figure to the
+    kernels it was measured on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "memory_bound_non_b200", "csrc")
+    for path in sorted(glob.glob(os.path.join(csrc, "*"))):
+        if path.endswith((".cu", ".cuh", ".h")):
+            with open(path, "rb") as f:
+                h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload, op):
+    """DRAM bytes per launch (read + write) of `op` on `workload` from the
+    committed ncu record, or None when the kernels changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    v = rec.get("per_launch_bytes", {}).get(workload, {}).get(op)
+    return int(v) if v is not None else None
 
 
 def flush_l2(buf):
@@ -311,8 +386,7 @@ class Step:
     def __init__(self, wl, rank):
         from memory_bound_non_b200 import workloads as W
         from memory_bound_non_b200.chain import LayerChain
-        import dataclasses
-        wl_r = dataclasses.replace(wl, seed=wl.seed + 1000 * rank, layers=1, steps=1)
+        wl_r = rank_workload(wl, rank)
         self.wl = wl_r
         t0 = time.time()
         self.host = W.make_inputs(wl_r, n_layers=1, device="cuda")  # seeded device generator
@@ -476,24 +550,8 @@ def main(argv=None):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     frt.load()
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-        pg = dist
-
-    def barrier():
-        if pg is not None:
-            pg.barrier()
-
-    def max_over_ranks(x):
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    dist = Dist(world, "nccl", torch.device("cuda", local))
+    barrier, max_over_ranks = dist.barrier, dist.max_over_ranks
 
     wl = W.get(args.workload)
     peak, peak_kind = measured_peak()
@@ -507,7 +565,7 @@ def main(argv=None):
     clk = clocks.stop()
     total_ms = max_over_ranks(total_ms)
     ms_per_step = total_ms / args.steps
-    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+    value = job_throughput(step_bytes, world, ms_per_step)
 
     per_op = {}
     for name, ts in per_op_us.items():
@@ -517,11 +575,7 @@ def main(argv=None):
                         "bytes": bytes_op[name], "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
                         "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4)}
     dom = max(per_op, key=lambda k: per_op[k]["us_mean"])
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tr_path):
-        with open(tr_path) as f:
-            traffic = json.load(f).get(wl.name, {}).get(dom)
+    traffic = measured_traffic(wl.name, dom)
     roofline = {"bound": "hbm", "kernel": {"gate": "frt_gate_act_fp8", "qkv": "frt_qkv_norm_rope_kvcache",
                                           "attn_norm": "frt_residual_rmsnorm_fp8",
                                           "ffn_norm": "frt_residual_rmsnorm_fp8"}[dom],
@@ -544,7 +598,7 @@ def main(argv=None):
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_leg(step, args.e2e_steps, 1)
         e2e_ms = max_over_ranks(e2e_ms)
-        e2e = {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        e2e = {"value": round(job_throughput(step_bytes, world, e2e_ms), 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -568,9 +622,7 @@ def main(argv=None):
         if args.json_out:
             with open(args.json_out, "w") as f:
                 f.write(s + "\n")
-    if pg is not None:
-        pg.barrier()
-        pg.destroy_process_group()
+    dist.close()
     return 0
 
 

@@ -1,0 +1,72 @@
+"""Multi-rank host logic of the bench on CPU: two gloo ranks on 127.0.0.1.
+
+The data path shards by rows with no collective; what the ranks share is the
+barrier and the max-over-ranks timing that turns per-rank times into one
+whole-job number.  Also: every rank draws its own shard of the workload.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from memory_bound_non_b200 import workloads as W
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    d = bench.Dist(world, backend="gloo", timeout_s=60)
+    d.barrier()
+    local_ms = 10.0 + 5.0 * rank                 # rank 1 is the slow one
+    worst = d.max_over_ranks(local_ms)
+    wl = bench.rank_workload(W.get("tiny"), rank)
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False)
+    out[rank] = (worst, float(inp.residual.float().sum()), tuple(inp.residual.shape))
+    d.close()
+
+
+def test_two_gloo_ranks_agree_on_the_slowest_time_and_shard_inputs():
+    world = 2
+    port = _free_port()
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    assert out[0][0] == out[1][0] == 15.0
+    assert out[0][2] == out[1][2]            # same shapes on every rank
+    assert out[0][1] != out[1][1]            # different rows on every rank
+    # whole-job throughput: both ranks' bytes over the slowest rank's time
+    assert bench.job_throughput(1e9, world, 15.0) == pytest.approx(2e9 / 15e-3 / 1e9)
+
+
+def test_single_rank_needs_no_group():
+    d = bench.Dist(1)
+    d.barrier()
+    assert d.max_over_ranks(3.5) == 3.5
+    d.close()
+
+
+def test_reference_arm_prints_only_on_rank_zero(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_op_bytes_are_the_algorithmic_bytes():
+    wl = W.get("large_m_M65536")
+    b = bench.op_bytes(wl)
+    # a: x, r_in, r_out (2 B) + fp8 (1 B) per element, weight, static scale
+    assert b["attn_norm"] == 65536 * 4096 * 7 + 2 * 4096 + 4
+    # b: QKV read + Q/K/V written (2 B each), cos+sin rows, position, two norm weights
+    assert b["qkv"] == 65536 * 6144 * 4 + 65536 * 128 * 4 + 4 * 65536 + 4 * 128
+    # c: gate/up read (4 B per output) + fp8 out, static scale
+    assert b["gate"] == 65536 * 16384 * 5 + 4
