@@ -254,6 +254,72 @@ def test_qkv_bad_positions_set_status_and_skip_rows():
     np.testing.assert_array_equal(P.np16(vc)[written], o["v_cache"][written])
 
 
+# --------------------------------------------- large batches (bulk-copy path)
+@pytest.mark.parametrize("ov", [
+    {"M": 600, "dt": "f16"},                                   # smallest batch on the bulk-copy path
+    {"M": 700, "hd": 256, "Hq": 8, "Hkv": 2, "capacity": 1024},  # 16 lanes per head, 4 KB+ rows
+    {"M": 640, "hd": 64, "Hq": 12, "Hkv": 4, "capacity": 1024},
+    {"M": 1200, "hd": 72, "Hq": 16, "Hkv": 16, "qk_norm": True, "capacity": 2048},  # P = 4
+])
+def test_qkv_bulk_copy_path_parity(ov):
+    wl = W.get("large_m_M4096", **ov)
+    check_b_full(wl, b_inputs(wl))
+
+
+def test_qkv_bulk_copy_path_bad_positions():
+    wl = W.get("large_m_M4096", M=640, capacity=2048)
+    inp = b_inputs(wl)
+    pos = inp.positions.clone()
+    bad = torch.tensor([3, 100, 639])
+    pos[bad] = torch.tensor([-5, 2048, 1 << 29], dtype=torch.int32)
+    q_out, kc, vc, status = run_b_gpu(wl, inp, positions=pos)
+    o = oracle_b(wl, inp, positions=pos)
+    assert status == 1 and o["status"] == 1
+    good = np.setdiff1d(np.arange(wl.M), bad.numpy())
+    P.assert_16bit_close(P.decode16(q_out)[good], o["q_out"][good], what="Q staging", dt=wl.dt)
+    assert (P.np16(q_out)[bad.numpy()] == 0x3C3C).all()          # skipped rows untouched
+    written = ~np.isnan(o["k_cache"]).all(axis=(1, 2))
+    assert written.sum() == wl.M - 3
+    np.testing.assert_array_equal(P.np16(kc)[~written], W.bits16(inp.layers[0].k_cache)[~written])
+    np.testing.assert_array_equal(P.np16(vc), o["v_cache"])
+
+
+@pytest.mark.parametrize("qn,kn", [(True, False), (False, True), (False, False)])
+def test_qkv_bulk_copy_path_one_sided_norm(qn, kn):
+    wl = W.get("large_m_M4096", M=600)
+    inp = b_inputs(wl)
+    L = inp.layers[0]
+    L.q_norm_w = L.q_norm_w if qn else None
+    L.k_norm_w = L.k_norm_w if kn else None
+    check_b_full(wl, inp)
+
+
+def test_qkv_large_batch_with_8_byte_aligned_rows_uses_the_register_kernel():
+    # hd = 72 needs only 8-byte alignment; views offset by 8 bytes rule out the
+    # bulk-copy path, so the register kernel runs the large batch
+    wl = W.get("vit", M=800, qk_norm=True)
+    inp = b_inputs(wl)
+    L = inp.layers[0]
+    o = oracle_b(wl, inp)
+
+    def off8(t):
+        raw = torch.empty(t.numel() + 4, dtype=t.dtype, device=DEV)
+        v = raw[4:].view(t.shape)                                   # +8 bytes
+        v.copy_(t.to(DEV))
+        return v
+    qkv = off8(L.qkv)
+    kc, vc = off8(L.k_cache), off8(L.v_cache)
+    q_out = off8(torch.zeros((wl.M, wl.Hq, wl.hd), dtype=L.qkv.dtype))
+    frt.frt_qkv_norm_rope_kvcache(qkv, off8(L.q_norm_w), off8(L.k_norm_w), inp.cos.to(DEV), inp.sin.to(DEV),
+                                  inp.positions.to(DEV), q_out, kc, vc, wl.Hq, wl.Hkv, wl.hd, eps=wl.eps)
+    torch.cuda.synchronize()
+    assert qkv.data_ptr() % 16 == 8
+    P.assert_16bit_close(P.decode16(q_out), o["q_out"], what="Q staging", dt=wl.dt)
+    written = ~np.isnan(o["k_cache"]).all(axis=(1, 2))
+    P.assert_16bit_close(P.decode16(kc)[written], o["k_cache"][written], what="K cache", dt=wl.dt)
+    np.testing.assert_array_equal(P.np16(vc), o["v_cache"])
+
+
 # ================================================================ op (c) ===
 C_CASES = [
     ("tiny", {}), ("pi05", {}), ("vla_denoise", {}), ("vit", {}), ("vit", {"quant": "block128"}),
