@@ -91,22 +91,35 @@ __global__ void __launch_bounds__(HPG == 1 ? 1024 : 256) qkv_norm_rope_kvcache_k
   const int grp = (int)(threadIdx.x / GP);
   const int li = threadIdx.x & (GP - 1);
   const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G;
-  const int p = __ldg(positions + tok);
-  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
-  if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
-  const bool active = lane_ok && row_ok;
   const int half = hd >> 1;
   const int j0 = li * P;
   const uint16_t* row = qkv + (int64_t)tok * H * hd;
+  // The QKV vectors and the norm weights do not depend on the position: load
+  // them alongside it, so only the cos/sin rows wait for the position.
   V va[HPG], vb[HPG];
 #pragma unroll
   for (int i = 0; i < HPG; ++i) {
     const int h = (hb * hpg + i) * NG + grp;
-    if (active && i < hpg && h < H) {
+    if (lane_ok && i < hpg && h < H) {
       va[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + j0);
       vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
     }
   }
+  V qwa, qwb, kwa, kwb;
+  if (HPG == 1 && lane_ok) {
+    if (q_norm_w != nullptr) {
+      qwa = ld_vec<P>(q_norm_w + j0);
+      qwb = ld_vec<P>(q_norm_w + half + j0);
+    }
+    if (k_norm_w != nullptr) {
+      kwa = ld_vec<P>(k_norm_w + j0);
+      kwb = ld_vec<P>(k_norm_w + half + j0);
+    }
+  }
+  const int p = __ldg(positions + tok);
+  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
+  if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
+  const bool active = lane_ok && row_ok;
   float c[P], s[P];
   if (active) {
     ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
@@ -141,8 +154,13 @@ __global__ void __launch_bounds__(HPG == 1 ? 1024 : 256) qkv_norm_rope_kvcache_k
       if (do_norm) {
         const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
         float fa[P], fb[P];
-        unpack<DT, P>(ld_vec<P>(nw + j0), fa);
-        unpack<DT, P>(ld_vec<P>(nw + half + j0), fb);
+        if (HPG == 1) {  // weights already in registers
+          unpack<DT, P>(is_q ? qwa : kwa, fa);
+          unpack<DT, P>(is_q ? qwb : kwb, fb);
+        } else {
+          unpack<DT, P>(ld_vec<P>(nw + j0), fa);
+          unpack<DT, P>(ld_vec<P>(nw + half + j0), fb);
+        }
 #pragma unroll
         for (int e = 0; e < P; ++e) {
           a[e] = a[e] * rstd * fa[e];

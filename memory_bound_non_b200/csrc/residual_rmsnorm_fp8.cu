@@ -56,6 +56,16 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   }
   float s_static = 0.0f;
   if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
+  // Narrow rows (small-batch, latency-bound calls) load the weight with the
+  // row instead of after the reduction: one memory round trip less on the
+  // critical path.  Wide rows keep the registers for occupancy.
+  constexpr bool kEarlyWeight = WEIGHTED && K <= 2;
+  uint4 wv_early[kEarlyWeight ? K : 1];
+  if (kEarlyWeight) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (t + k * T < C) wv_early[k] = __ldg(w + t + k * T);
+  }
 
   // Pass 1: h = x + r rounded once to 16 bits (exactly the rounded exact sum,
   // see add_for_16), kept packed; fp64 sum of squares (squares of 16-bit
@@ -114,7 +124,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv[k]);
     float y[8];
     if (WEIGHTED && valid) {
-      const uint4 wv = __ldg(w + c);
+      const uint4 wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : __ldg(w + c);
       const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
