@@ -428,9 +428,28 @@ def timed_step_leg(step, K, W_, barrier):
     return total_ms, per_op
 
 
-def e2e_leg(step, K, W_):
-    """Public-API step with host buffers: H2D of the step's inputs from pinned
-    memory, the four ops, D2H of the step's outputs, on one stream."""
+def run_rows(ch, r0, r1, stream):
+    """The step's four ops on token rows [r0, r1) (every op is row-independent)."""
+    import memory_bound_non_b200 as frt
+    wl, L = ch.wl, ch.layers[0]
+    frt.frt_residual_rmsnorm_fp8(L.x_attn[r0:r1], ch.residual[r0:r1], ch.residual[r0:r1], L.w_attn,
+                                 L.q8_attn[r0:r1], static_scale=ch.scales[0:1], eps=wl.eps, quant=wl.quant,
+                                 stream=stream)
+    frt.frt_qkv_norm_rope_kvcache(L.qkv[r0:r1], L.q_norm_w, L.k_norm_w, ch.cos, ch.sin, ch.positions[r0:r1],
+                                  L.q_out[r0:r1], L.k_cache, L.v_cache, wl.Hq, wl.Hkv, wl.hd, status=ch.status,
+                                  eps=wl.eps, stream=stream)
+    frt.frt_residual_rmsnorm_fp8(L.x_ffn[r0:r1], ch.residual[r0:r1], ch.residual[r0:r1], L.w_ffn,
+                                 L.q8_ffn[r0:r1], static_scale=ch.scales[1:2], eps=wl.eps, quant=wl.quant,
+                                 stream=stream)
+    frt.frt_gate_act_fp8(L.gate_up[r0:r1], L.act8[r0:r1], static_scale=ch.scales[2:3], act=wl.act,
+                         quant=wl.quant, stream=stream)
+
+
+def e2e_leg(step, K, W_, chunks=8):
+    """Public-API step with host buffers: the step's inputs are copied from
+    pinned host memory and its outputs copied back inside the timed region.
+    Rows are cut into `chunks` pieces pipelined over three streams (copy in,
+    compute, copy out), so the transfers overlap each other and the kernels."""
     ch = step.chain
     L, H = ch.layers[0], step.host
     hl = H.layers[0]
@@ -441,23 +460,40 @@ def e2e_leg(step, K, W_):
             for d in (L.q8_attn, L.q_out, ch.residual, L.q8_ffn, L.act8)]
     h2d = sum(h.numel() * h.element_size() for h, _ in ins)
     d2h = sum(h.numel() * h.element_size() for _, h in outs)
-    s = torch.cuda.current_stream()
+    M = ch.wl.M
+    bounds = [(M * i // chunks, M * (i + 1) // chunks) for i in range(chunks)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    main = torch.cuda.current_stream()
 
     def one():
-        for h, d in ins:
-            d.copy_(h, non_blocking=True)
-        step.run()
-        for d, h in outs:
-            h.copy_(d, non_blocking=True)
+        for s in (s_in, s_comp, s_out):
+            s.wait_stream(main)
+        done = []
+        for r0, r1 in bounds:
+            with torch.cuda.stream(s_in):
+                for h, d in ins:
+                    d[r0:r1].copy_(h[r0:r1], non_blocking=True)
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            s_comp.wait_event(e_in)
+            run_rows(ch, r0, r1, s_comp)
+            e_c = torch.cuda.Event()
+            e_c.record(s_comp)
+            s_out.wait_event(e_c)
+            with torch.cuda.stream(s_out):
+                for d, h in outs:
+                    h[r0:r1].copy_(d[r0:r1], non_blocking=True)
+        for s in (s_in, s_comp, s_out):
+            main.wait_stream(s)
 
     for _ in range(W_):
         one()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
+    e0.record(main)
     for _ in range(K):
         one()
-    e1.record(s)
+    e1.record(main)
     e1.synchronize()
     return e0.elapsed_time(e1) / K, h2d, d2h
 
