@@ -205,9 +205,9 @@ __device__ __forceinline__ void bulk_store(void* gmem_dst, const void* smem_src,
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Blocks until the committed bulk stores are complete (shared memory read and
-// global memory written).
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Blocks until the committed bulk stores have finished reading shared memory
+// (the stores themselves complete before the grid does).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Orders this thread's generic-proxy shared-memory writes before later
 // bulk-copy (async-proxy) reads of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(256) qkv_norm_rope_kvcache_tma_kernel(
     bulk_store(k_cache + (int64_t)p * Hkv * hd, rowbuf + Hq * hd, (unsigned)(Hkv * hd * 2));
     bulk_store(v_cache + (int64_t)p * Hkv * hd, rowbuf + (Hq + Hkv) * hd, (unsigned)(Hkv * hd * 2));
     bulk_commit();
-    bulk_wait_all();  // shared memory must outlive the stores; writes done before exit
+    bulk_wait_read();  // shared memory must outlive the stores' reads
   }
 }
 
