@@ -69,6 +69,10 @@ def lib():
         L.oracle_gate_act_fp8.argtypes = [c.c_void_p, c.c_void_p, c.c_double, c.c_void_p, c.c_void_p,
                                           c.c_int64, c.c_int64, c.c_int, c.c_int, c.c_int]
         L.oracle_gate_act_fp8.restype = c.c_int
+        L.oracle_gate_residual_adarms_fp8.argtypes = [c.c_void_p] * 7 + [c.c_double, c.c_void_p, c.c_void_p,
+                                                                          c.c_int64, c.c_int64, c.c_int64,
+                                                                          c.c_double, c.c_int, c.c_int]
+        L.oracle_gate_residual_adarms_fp8.restype = c.c_int
         _lib = L
     return _lib
 
@@ -195,3 +199,24 @@ def gate_act_fp8(gate_up, act_name, dt, quant, static_scale=None, want_a=False):
     if rc != 0:
         raise ValueError("oracle_gate_act_fp8: bad argument")
     return {"out_fp8": q, "block_scales": sc, "a": a}
+
+
+def gate_residual_adarms_fp8(x, gate, residual_in, scale, shift, eps, dt, quant, rows_per_cond, static_scale=None,
+                             want_y=False):
+    """NEXT-1 op.  x, residual_in: uint16 [M, D]; gate / scale / shift: uint16
+    [ceil(M / rows_per_cond), D] or None."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    r = np.ascontiguousarray(residual_in, dtype=np.uint16)
+    M, D = x.shape
+    g, sc, sh = (None if a is None else np.ascontiguousarray(a, dtype=np.uint16) for a in (gate, scale, shift))
+    r_out = np.empty_like(r)
+    q = np.empty((M, D), dtype=np.uint8)
+    nb = (D + 127) // 128
+    bs = np.empty((M, nb), dtype=np.float64) if quant == "block128" else None
+    y = np.empty((M, D), dtype=np.float64) if want_y else None
+    s = float(static_scale) if quant == "static" else 0.0
+    rc = lib().oracle_gate_residual_adarms_fp8(_p(x), _p(g), _p(r), _p(r_out), _p(sc), _p(sh), _p(q), s, _p(bs),
+                                               _p(y), M, D, int(rows_per_cond), _f32(eps), _DT[dt], _QM[quant])
+    if rc != 0:
+        raise ValueError("oracle_gate_residual_adarms_fp8: bad argument")
+    return {"residual_out": r_out, "out_fp8": q, "block_scales": bs, "y": y}

@@ -394,4 +394,50 @@ int oracle_gate_act_fp8(const uint16_t* gate_up, uint8_t* out_fp8, double static
   return 0;
 }
 
+// NEXT-1: gated residual + AdaRMSNorm modulation + FP8 ([FR] §三: the Pi0.5
+// decoder's cross-layer kernel fuses gate multiply, residual add, AdaRMSNorm
+// modulation, FP8 quantisation and descale, 6 ops -> 1, run 180 times per
+// decode).  Reading (the pages give no formula; the adaptive RMSNorm of
+// diffusion/flow-matching transformers):
+//   c        = row / rows_per_cond (one condition per group of rows)
+//   h        = rn16(r + g_c * x), the exact value rounded once
+//   y        = h * rstd * (1 + scale_c) + shift_c, rstd = 1/sqrt(mean(h^2)+eps)
+//   out_fp8  = FP8(y) as in op (a) (static or block-128)
+// gate / scale / shift are [ceil(M / rows_per_cond), D] 16-bit; NULL gate
+// means 1, NULL scale or shift means 0.  residual_out may alias residual_in.
+int oracle_gate_residual_adarms_fp8(const uint16_t* x, const uint16_t* gate, const uint16_t* residual_in,
+                                    uint16_t* residual_out, const uint16_t* scale, const uint16_t* shift,
+                                    uint8_t* out_fp8, double static_scale, double* block_scales, double* y_out,
+                                    int64_t M, int64_t D, int64_t rows_per_cond, double eps, int dt, int qm) {
+  if (M < 0 || D <= 0 || rows_per_cond <= 0 || !x || !residual_in || !residual_out || !out_fp8) return -1;
+  if (qm == Q_BLOCK128 && !block_scales) return -1;
+  const Fmt16 f = fmt_of(dt);
+  const int64_t nb = (D + 127) / 128;
+  std::vector<double> h(D), y(D);
+  for (int64_t i = 0; i < M; ++i) {
+    const int64_t c = i / rows_per_cond;
+    for (int64_t j = 0; j < D; ++j) {
+      const double g = gate ? decode16(gate[c * D + j], f) : 1.0;
+      const double gx = g * decode16(x[i * D + j], f);  // exact: two 16-bit significands
+      double s, err;
+      two_sum(decode16(residual_in[i * D + j], f), gx, &s, &err);
+      const uint16_t hb = round16(s, err, f);
+      residual_out[i * D + j] = hb;
+      h[j] = decode16(hb, f);
+    }
+    rmsnorm(h.data(), D, nullptr, eps, y.data());
+    for (int64_t j = 0; j < D; ++j) {
+      const double sc = scale ? decode16(scale[c * D + j], f) : 0.0;
+      const double sh = shift ? decode16(shift[c * D + j], f) : 0.0;
+      y[j] = y[j] * (1.0 + sc) + sh;
+    }
+    if (y_out) std::memcpy(y_out + i * D, y.data(), sizeof(double) * D);
+    if (qm == Q_STATIC)
+      quant_static(y.data(), D, static_scale, out_fp8 + i * D);
+    else
+      quant_block128(y.data(), D, out_fp8 + i * D, block_scales + i * nb);
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -191,3 +191,26 @@ def gate_act_fp8(gu, act_name, dt, quant, static_scale=None):
         a[i] = np.array([act(act_name, float(gg)) for gg in g]) * u
         _quant_row(a[i], quant, static_scale, q[i], scales[i])
     return q, scales, a
+
+
+def gate_residual_adarms_fp8(x, gate, r, scale, shift, eps, dt, quant, rows_per_cond, static_scale=None):
+    """NEXT-1 restated: exact rational residual r + g * x rounded by search,
+    numpy fp64 RMS and modulation, fp32 FP8 decisions."""
+    M, D = x.shape
+    dec = DECODE[dt]
+    h_bits = np.zeros((M, D), dtype=np.uint16)
+    q = np.zeros((M, D), dtype=np.uint8)
+    scales = np.zeros((M, (D + 127) // 128))
+    for i in range(M):
+        c = i // rows_per_cond
+        for j in range(D):
+            g = Fraction(dec(gate[c, j])) if gate is not None else Fraction(1)
+            v = Fraction(dec(r[i, j])) + g * Fraction(dec(x[i, j]))
+            h_bits[i, j] = round16_exact(v, dt) if v != 0 else (h_bits[i, j] & 0)
+        h = np.array([dec(b) for b in h_bits[i]])
+        y = h / np.sqrt(np.mean(h * h) + eps)
+        sc = np.array([dec(b) for b in scale[c]]) if scale is not None else np.zeros(D)
+        sh = np.array([dec(b) for b in shift[c]]) if shift is not None else np.zeros(D)
+        y = y * (1.0 + sc) + sh
+        _quant_row(y, quant, static_scale, q[i], scales[i])
+    return h_bits, q, scales
