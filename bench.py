@@ -23,6 +23,8 @@ Also reported on the same JSON line:
                 between replays; per-node cost against the launch floor;
   launch_floor  an empty kernel per stream launch and per graph node;
   small_m       per-op microseconds at M <= 41 against the launch floor;
+  next_ops      the widened ops timed alone (gated residual + AdaRMSNorm +
+                FP8 at 65536 x 4096 and at the Pi0.5 action-expert shape);
   e2e           the same step through the public API with pinned host
                 buffers: host->device copy of the step's inputs, the four ops,
                 device->host copy of the step's outputs;
@@ -342,6 +344,68 @@ def small_m_ops(floor, reps=400):
     return out
 
 
+def next_ops_leg(peak, floor, reps=50):
+    """The widened ops, timed alone: NEXT-1 (gated residual + AdaRMSNorm + FP8)
+    at 65536 x 4096 bf16 with one condition row per 1024 rows (inputs larger
+    than L2), and at the Pi0.5 action-expert shape (10 x 1024) as a graph node."""
+    import memory_bound_non_b200 as frt
+    from memory_bound_non_b200 import workloads as W
+    out = {}
+    s = torch.cuda.current_stream()
+    for M, D, rpc in ((65536, 4096, 1024), (10, 1024, 10)):
+        g = W.generator(61, "cuda")
+        nc = (M + rpc - 1) // rpc
+        x = W.normal16((M, D), "bf16", g)
+        r = W.normal16((M, D), "bf16", g, scale=2.0)
+        gate = W.normal16((nc, D), "bf16", g, scale=0.5)
+        sc = W.normal16((nc, D), "bf16", g, scale=0.2)
+        sh = W.normal16((nc, D), "bf16", g, scale=0.2)
+        q = torch.empty((M, D), dtype=torch.uint8, device="cuda")
+        ss = torch.tensor([0.02], dtype=torch.float32, device="cuda")
+
+        def op():
+            frt.frt_gate_residual_adarms_fp8(x, gate, r, r, sc, sh, q, static_scale=ss, rows_per_cond=rpc)
+        nbytes = M * D * 7 + nc * D * 6
+        for _ in range(5):
+            op()
+        torch.cuda.synchronize()
+        if M > 1024:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+            for i in range(reps):
+                ev[2 * i].record(s)
+                op()
+                ev[2 * i + 1].record(s)
+            torch.cuda.synchronize()
+            ts = [ev[2 * i].elapsed_time(ev[2 * i + 1]) * 1e3 for i in range(reps)]
+            us = sum(ts) / len(ts)
+            gbs = nbytes / (us * 1e-6) / 1e9
+            out["gate_residual_adarms_M%d_D%d" % (M, D)] = {
+                "us_mean": round(us, 2), "us_median": round(statistics.median(ts), 2), "bytes": nbytes,
+                "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4), "l2": "inputs larger than L2"}
+        else:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                for _ in range(200):
+                    op()
+            gr.replay()
+            torch.cuda.synchronize()
+            ts = []
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for _ in range(10):
+                e0.record(s)
+                gr.replay()
+                e1.record(s)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3 / 200)
+            del gr
+            node = statistics.median(ts)
+            out["gate_residual_adarms_M%d_D%d" % (M, D)] = {
+                "graph_node_us": round(node, 3), "x_graph_floor": round(node / floor["graph_node_us"], 3)}
+        del x, r, gate, sc, sh, q
+    return out
+
+
 def chain_leg(reps, floor):
     from memory_bound_non_b200 import workloads as W
     from memory_bound_non_b200.chain import LayerChain
@@ -629,6 +693,8 @@ def main(argv=None):
             extra["launch_floor" + tag] = {k: (round(v, 3) if isinstance(v, float) else v) for k, v in floor.items()}
             extra["chain" + tag] = chain_leg(args.chain_reps, floor)
             extra["small_m" + tag] = small_m_ops(floor)
+            if pdl:
+                extra["next_ops"] = next_ops_leg(peak, floor)
         frt.frt_set_pdl(pdl0)
     e2e = None
     if not args.no_e2e:

@@ -177,6 +177,36 @@ frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* 
                             cudaStream_t stream);
 
 /*
+ * NEXT-1: gated residual + AdaRMSNorm modulation + FP8 quantisation.
+ * "FlashRT kernel fusion", §三: the Pi0.5 decoder's cross-layer kernel
+ * (gate_res_adarms_fp8_static) fuses gate multiply, residual add, AdaRMSNorm
+ * modulation, FP8 quantisation and descale (6 ops -> 1) and runs once per
+ * sub-layer per flow step.  The pages give no formula; the reading is the
+ * adaptive RMSNorm of flow-matching / diffusion transformers:
+ *
+ * For row i with condition row c = i / rows_per_cond:
+ *   h[i,j]  = residual_in[i,j] + gate[c,j] * x[i,j], the exact value rounded
+ *             once to the 16-bit type; written to residual_out.
+ *   y[i,j]  = h[i,j] * rstd_i * (1 + scale[c,j]) + shift[c,j],
+ *             rstd_i = 1 / sqrt(mean_j(h[i,j]^2) + eps).
+ *   out_fp8 = e4m3 of y / s (quant mode as in op (a); block scales over D).
+ *
+ *   x, residual_in, residual_out  device [M, D] 16-bit, 16-byte aligned;
+ *                                 residual_out may equal residual_in.
+ *   gate, scale, shift            device [ceil(M / rows_per_cond), D] 16-bit,
+ *                                 16-byte aligned, or NULL (gate NULL = 1,
+ *                                 scale / shift NULL = 0).
+ *   out_fp8, static_scale, block_scales  as op (a).
+ *   Layout rule: D > 0, D % 8 == 0, rows_per_cond > 0.  Unsupported:
+ *   D > 32768.
+ */
+frt_status frt_gate_residual_adarms_fp8(const void* x, const void* gate, const void* residual_in,
+                                        void* residual_out, const void* scale, const void* shift,
+                                        uint8_t* out_fp8, const float* static_scale, float* block_scales,
+                                        int M, int D, int rows_per_cond, float eps, frt_dtype dt, frt_quant qm,
+                                        cudaStream_t stream);
+
+/*
  * Empty kernel used to measure the launch floor that the ops above are graded
  * against (the roofline of a launch-bound op is the larger of its HBM time and
  * this floor).  Launches `grid` blocks of `block` threads that do nothing.

@@ -25,8 +25,8 @@ QUANT = {"static": 0, "block128": 1}
 ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
 
 # C entry points declared in include/frt.h
-EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8", "frt_noop",
-           "frt_set_pdl", "frt_get_pdl", "frt_status_string")
+EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8",
+           "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_status_string")
 
 
 class FrtError(RuntimeError):
@@ -54,6 +54,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_qkv_norm_rope_kvcache.restype = i32
     L.frt_gate_act_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     L.frt_gate_act_fp8.restype = i32
+    L.frt_gate_residual_adarms_fp8.argtypes = [vp] * 9 + [i32, i32, i32, f32, i32, i32, vp]
+    L.frt_gate_residual_adarms_fp8.restype = i32
     L.frt_noop.argtypes = [i32, i32, vp]
     L.frt_noop.restype = i32
     L.frt_set_pdl.argtypes = [i32]
@@ -125,6 +127,20 @@ def frt_gate_act_fp8(gate_up, out_fp8, static_scale=None, block_scales=None, act
     st = load().frt_gate_act_fp8(_ptr(gate_up), _ptr(out_fp8), _ptr(static_scale), _ptr(block_scales), M,
                                  two_i // 2, ACT[act], DTYPE[gate_up.dtype], QUANT[quant], _stream(stream))
     _check("frt_gate_act_fp8", st)
+
+
+def frt_gate_residual_adarms_fp8(x, gate, residual_in, residual_out, scale, shift, out_fp8, static_scale=None,
+                                 block_scales=None, rows_per_cond=None, eps=1e-6, quant="static", stream=None):
+    """NEXT-1: h = residual + gate * x (rounded once), y = RMSNorm(h) * (1 + scale)
+    + shift, FP8 e4m3.  gate / scale / shift: [ceil(M / rows_per_cond), D] or
+    None; rows_per_cond defaults to M (one condition for all rows)."""
+    M, D = x.shape
+    rpc = M if rows_per_cond is None else int(rows_per_cond)
+    st = load().frt_gate_residual_adarms_fp8(
+        _ptr(x), _ptr(gate), _ptr(residual_in), _ptr(residual_out), _ptr(scale), _ptr(shift), _ptr(out_fp8),
+        _ptr(static_scale), _ptr(block_scales), M, D, max(rpc, 1), float(eps), DTYPE[x.dtype], QUANT[quant],
+        _stream(stream))
+    _check("frt_gate_residual_adarms_fp8", st)
 
 
 def frt_set_pdl(enable: bool):

@@ -105,3 +105,19 @@ def test_pdl_switch():
         assert frt.frt_get_pdl() is True
     finally:
         frt.frt_set_pdl(prev)
+
+
+def ada_call(M=4, D=256, x=A, g=A, r=A, ro=A, sc=A, sh=A, q=A, ss=A, bs=None, rpc=4, dt=1, qm=0):
+    return frt.load().frt_gate_residual_adarms_fp8(x, g, r, ro, sc, sh, q, ss, bs, M, D, rpc, 1e-6, dt, qm, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=-1), INV), (dict(D=12), INV), (dict(rpc=0), INV), (dict(x=None), INV), (dict(g=A + 8), INV),
+    (dict(sc=A + 4), INV), (dict(sh=A + 2), INV), (dict(q=A + 4), INV), (dict(ss=None), INV),
+    (dict(qm=1), INV), (dict(D=32776), UNSUP), (dict(M=0), OK), (dict(g=None, sc=None, sh=None), None),
+])
+def test_gate_residual_adarms_host_validation(kw, want):
+    if want is None:   # NULL gate / scale / shift are valid: validation passes (no launch here at M = 0)
+        assert ada_call(M=0, **kw) == OK
+    else:
+        assert ada_call(**kw) == want

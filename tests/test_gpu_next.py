@@ -1,0 +1,197 @@
+"""GPU parity for the NEXT ops through the C ABI against the fp64 oracle.
+
+NEXT-1, gated residual + AdaRMSNorm modulation + FP8 ("FlashRT kernel
+fusion", §三, gate_res_adarms_fp8_static): the Pi0.5 decoder shape, every
+mode (16-bit type, quantisation, gate present or not, modulation present or
+not), condition-row groups, edge widths, in-place and guarded out-of-place
+outputs, sums that land on a 16-bit rounding midpoint in fp32, and the
+full-size large-M workload on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import memory_bound_non_b200 as frt
+import oracle
+import parity as P
+from memory_bound_non_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+GUARD = 256
+
+
+def guarded(shape, dtype, fill):
+    n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+    raw = torch.full((n + GUARD,), fill, dtype=torch.uint8, device=DEV)
+    return raw, raw[:n].view(dtype).view(shape)
+
+
+def assert_guard(raw, n_bytes, fill):
+    assert (raw[n_bytes:].cpu().numpy() == fill).all(), "write past the end of an output"
+
+
+def ada_inputs(M, D, dt, seed, rpc, gated=True, modulated=True, device="cpu"):
+    """x ~ N(0, 1), residual ~ N(0, 4), gate ~ N(0, 0.25), scale / shift ~
+    N(0, 0.04), the last three one row per condition (ceil(M / rpc) rows)."""
+    g = W.generator(seed, device)
+    nc = (M + rpc - 1) // rpc
+    x = W.normal16((M, D), dt, g)
+    r = W.normal16((M, D), dt, g, scale=2.0)
+    gate = W.normal16((nc, D), dt, g, scale=0.5) if gated else None
+    sc = W.normal16((nc, D), dt, g, scale=0.2) if modulated else None
+    sh = W.normal16((nc, D), dt, g, scale=0.2) if modulated else None
+    return x, r, gate, sc, sh
+
+
+def host_bits(t):
+    return None if t is None else W.bits16(t.cpu())
+
+
+def calibrate(x, r, gate, sc, sh, dt, rpc):
+    o = oracle.gate_residual_adarms_fp8(x, gate, r, sc, sh, 1e-6, dt, "block128", rpc, want_y=True)
+    return P.f32(np.abs(o["y"]).max() / 448.0)
+
+
+def run_gpu(x, r, gate, sc, sh, quant, scale, rpc, inplace=True):
+    M, D = x.shape
+    dev = [None if t is None else t.to(DEV) for t in (x, r, gate, sc, sh)]
+    xd, rd, gd, scd, shd = dev
+    rd = rd.clone()
+    if inplace:
+        ro_raw, ro = None, rd
+    else:
+        ro_raw, ro = guarded((M, D), rd.dtype, 0x5A)
+    q_raw, q = guarded((M, D), torch.uint8, 0xA5)
+    nb = (D + 127) // 128
+    bs_raw = bs = ss = None
+    if quant == "block128":
+        bs_raw, bs = guarded((M, nb), torch.float32, 0xFF)
+    else:
+        ss = torch.tensor([scale], dtype=torch.float32, device=DEV)
+    frt.frt_gate_residual_adarms_fp8(xd, gd, rd, ro, scd, shd, q, static_scale=ss, block_scales=bs,
+                                     rows_per_cond=rpc, eps=1e-6, quant=quant)
+    torch.cuda.synchronize()
+    assert_guard(q_raw, M * D, 0xA5)
+    if bs_raw is not None:
+        assert_guard(bs_raw, M * nb * 4, 0xFF)
+    if ro_raw is not None:
+        assert_guard(ro_raw, M * D * 2, 0x5A)
+    return ro, q, bs
+
+
+def check(M, D, dt, quant, rpc, gated=True, modulated=True, seed=11, inplace=True):
+    x, r, gate, sc, sh = ada_inputs(M, D, dt, seed, rpc, gated, modulated)
+    hx, hr, hg, hsc, hsh = (host_bits(t) for t in (x, r, gate, sc, sh))
+    scale = calibrate(hx, hr, hg, hsc, hsh, dt, rpc) if quant == "static" else None
+    ro, q, bs = run_gpu(x, r, gate, sc, sh, quant, scale, rpc, inplace=inplace)
+    o = oracle.gate_residual_adarms_fp8(hx, hg, hr, hsc, hsh, 1e-6, dt, quant, rpc, static_scale=scale)
+    np.testing.assert_array_equal(W.bits16(ro.cpu()), o["residual_out"])
+    P.assert_fp8_codes(q.cpu().numpy(), o["out_fp8"], what="adarms codes")
+    if quant == "block128":
+        P.assert_scales_close(bs.cpu().numpy(), o["block_scales"])
+
+
+@pytest.mark.parametrize("quant", ["static", "block128"])
+def test_adarms_pi05_decoder_shape(quant):
+    # Pi0.5 action expert: 10 action tokens, width 1024, one condition (the flow time step)
+    check(10, 1024, "bf16", quant, rpc=10)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("quant", ["static", "block128"])
+@pytest.mark.parametrize("gated,modulated", [(True, True), (True, False), (False, True), (False, False)])
+def test_adarms_modes_out_of_place(dt, quant, gated, modulated):
+    check(33, 1280, dt, quant, rpc=11, gated=gated, modulated=modulated, inplace=False)
+
+
+@pytest.mark.parametrize("M,D,quant,rpc", [
+    (1, 8, "static", 1), (3, 136, "block128", 2), (5, 1032, "block128", 1), (7, 2056, "static", 3),
+    (4, 8192, "block128", 4), (3, 16384, "static", 1), (2, 16392, "block128", 1), (2, 32768, "block128", 2),
+])
+def test_adarms_edge_widths(M, D, quant, rpc):
+    check(M, D, "bf16", quant, rpc=rpc, seed=M * 7 + D)
+
+
+def test_adarms_fp16_wide_and_in_place():
+    check(6, 4096, "f16", "block128", rpc=1, seed=21, inplace=True)
+
+
+def test_adarms_sums_on_a_16bit_midpoint():
+    """Triples whose fp32 sum r + g x lies on a bf16 rounding midpoint while the
+    exact sum does not: rounding the fp32 sum again would give the wrong h."""
+    rng = np.random.default_rng(7)
+    n = 1 << 18
+    # |r| << |g x|: r's bits fall below the fp32 ulp of the sum, and when g x
+    # sits on a bf16 midpoint the sign of r alone decides the rounding
+    r = rng.integers(0x3000, 0x3800, n).astype(np.uint16) | (rng.integers(0, 2, n).astype(np.uint16) << 15)
+    g = rng.integers(0x3C00, 0x3F80, n).astype(np.uint16)          # gate in [2^-7, 1)
+    x = rng.integers(0x3F80, 0x4100, n).astype(np.uint16) | (rng.integers(0, 2, n).astype(np.uint16) << 15)
+    tr, tg, tx = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) for a in (r, g, x))
+    naive = W.bits16((tr.float() + tg.float() * tx.float()).to(torch.bfloat16))
+    D = 1024
+    o = oracle.gate_residual_adarms_fp8(x.reshape(-1, D), g.reshape(-1, D), r.reshape(-1, D), None, None, 1e-6,
+                                        "bf16", "block128", 1)
+    hard = naive.reshape(-1, D) != o["residual_out"]
+    assert hard.sum() > 50, "the inputs do not exercise the midpoint case"
+    rows = np.flatnonzero(hard.any(axis=1))[:64]
+    M = len(rows)
+    xs, gs, rs = (torch.from_numpy(a.reshape(-1, D)[rows].copy().view(np.int16)).view(torch.bfloat16)
+                  for a in (x, g, r))
+    ro, q, bs = run_gpu(xs, rs, gs, None, None, "block128", None, 1)
+    want = o["residual_out"][rows]
+    np.testing.assert_array_equal(W.bits16(ro.cpu()), want)
+    om = oracle.gate_residual_adarms_fp8(W.bits16(xs), W.bits16(gs), W.bits16(rs), None, None, 1e-6, "bf16",
+                                         "block128", 1)
+    P.assert_fp8_codes(q.cpu().numpy(), om["out_fp8"], what="midpoint rows codes")
+
+
+def test_adarms_without_gate_or_modulation_equals_op_a():
+    """No gate, no modulation: the op is op (a) with `_noweight`, bit for bit."""
+    x, r, _, _, _ = ada_inputs(64, 2048, "bf16", 31, 64, gated=False, modulated=False)
+    xd, rd = x.to(DEV), r.to(DEV)
+    r1, r2 = rd.clone(), rd.clone()
+    q1 = torch.empty((64, 2048), dtype=torch.uint8, device=DEV)
+    q2 = torch.empty_like(q1)
+    ss = torch.tensor([0.01], dtype=torch.float32, device=DEV)
+    frt.frt_gate_residual_adarms_fp8(xd, None, r1, r1, None, None, q1, static_scale=ss)
+    frt.frt_residual_rmsnorm_fp8(xd, r2, r2, None, q2, static_scale=ss)
+    torch.cuda.synchronize()
+    assert torch.equal(r1, r2)
+    assert torch.equal(q1, q2)
+
+
+@pytest.mark.parametrize("M", [16384, 65536])
+def test_adarms_large_m_sampled(M):
+    """Full-size launch (D = 4096, one condition per 1024 rows), sampled rows
+    against the oracle (each sampled row with its own condition row)."""
+    D, rpc, dt = 4096, 1024, "bf16"
+    x, r, gate, sc, sh = ada_inputs(M, D, dt, 41, rpc, device=DEV)
+    rng = np.random.default_rng(M)
+    rows = np.unique(np.concatenate([rng.choice(M, 256, replace=False), [0, M - 1]]))
+    ti = torch.as_tensor(rows, device=DEV)
+    ci = torch.as_tensor(rows // rpc, device=DEV)
+    hx, hr = W.bits16(x[ti].cpu()), W.bits16(r[ti].cpu())
+    hg, hsc, hsh = (W.bits16(t[ci].cpu()) for t in (gate, sc, sh))
+    scale = calibrate(hx, hr, hg, hsc, hsh, dt, 1)
+    q = torch.empty((M, D), dtype=torch.uint8, device=DEV)
+    ss = torch.tensor([scale], dtype=torch.float32, device=DEV)
+    frt.frt_gate_residual_adarms_fp8(x, gate, r, r, sc, sh, q, static_scale=ss, rows_per_cond=rpc)
+    torch.cuda.synchronize()
+    o = oracle.gate_residual_adarms_fp8(hx, hg, hr, hsc, hsh, 1e-6, dt, "static", 1, static_scale=scale)
+    np.testing.assert_array_equal(W.bits16(r[ti].cpu()), o["residual_out"])
+    P.assert_fp8_codes(q[ti].cpu().numpy(), o["out_fp8"], what="large-M adarms codes")
+
+
+def test_adarms_deterministic():
+    x, r, gate, sc, sh = ada_inputs(40, 3072, "bf16", 51, 8, device=DEV)
+    outs = []
+    for _ in range(2):
+        rr = r.clone()
+        q = torch.empty((40, 3072), dtype=torch.uint8, device=DEV)
+        bs = torch.empty((40, 24), dtype=torch.float32, device=DEV)
+        frt.frt_gate_residual_adarms_fp8(x, gate, rr, rr, sc, sh, q, block_scales=bs, rows_per_cond=8,
+                                         quant="block128")
+        outs.append((rr, q, bs))
+    torch.cuda.synchronize()
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
