@@ -70,6 +70,10 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--chain-reps", type=int, default=30)
     p.add_argument("--json-out", default=None)
+    p.add_argument("--next-only", action="store_true",
+                   help="time only the widened ops (gated residual + AdaRMSNorm + FP8) and print their JSON")
+    p.add_argument("--next-m", type=int, default=65536, help="rows of the large widened-op case")
+    p.add_argument("--next-reps", type=int, default=50)
     return p.parse_args(argv)
 
 
@@ -344,15 +348,17 @@ def small_m_ops(floor, reps=400):
     return out
 
 
-def next_ops_leg(peak, floor, reps=50):
+def next_ops_leg(peak, floor, reps=50, big_m=65536):
     """The widened ops, timed alone: NEXT-1 (gated residual + AdaRMSNorm + FP8)
-    at 65536 x 4096 bf16 with one condition row per 1024 rows (inputs larger
-    than L2), and at the Pi0.5 action-expert shape (10 x 1024) as a graph node."""
+    at big_m x 4096 bf16 with one condition row per 1024 rows (inputs larger
+    than L2 at the default 65536), static and block-128 scales, and at the
+    Pi0.5 action-expert shape (10 x 1024) as a graph node."""
     import memory_bound_non_b200 as frt
     from memory_bound_non_b200 import workloads as W
     out = {}
     s = torch.cuda.current_stream()
-    for M, D, rpc in ((65536, 4096, 1024), (10, 1024, 10)):
+    for M, D, rpc, quant in ((big_m, 4096, 1024, "static"), (big_m, 4096, 1024, "block128"),
+                             (10, 1024, 10, "static")):
         g = W.generator(61, "cuda")
         nc = (M + rpc - 1) // rpc
         x = W.normal16((M, D), "bf16", g)
@@ -362,13 +368,19 @@ def next_ops_leg(peak, floor, reps=50):
         sh = W.normal16((nc, D), "bf16", g, scale=0.2)
         q = torch.empty((M, D), dtype=torch.uint8, device="cuda")
         ss = torch.tensor([0.02], dtype=torch.float32, device="cuda")
+        bs = torch.empty((M, (D + 127) // 128), dtype=torch.float32, device="cuda")
 
         def op():
-            frt.frt_gate_residual_adarms_fp8(x, gate, r, r, sc, sh, q, static_scale=ss, rows_per_cond=rpc)
-        nbytes = M * D * 7 + nc * D * 6
+            if quant == "static":
+                frt.frt_gate_residual_adarms_fp8(x, gate, r, r, sc, sh, q, static_scale=ss, rows_per_cond=rpc)
+            else:
+                frt.frt_gate_residual_adarms_fp8(x, gate, r, r, sc, sh, q, block_scales=bs, rows_per_cond=rpc,
+                                                 quant="block128")
+        nbytes = M * D * 7 + nc * D * 6 + (bs.numel() * 4 if quant == "block128" else 0)
         for _ in range(5):
             op()
         torch.cuda.synchronize()
+        key = "gate_residual_adarms_M%d_D%d_%s" % (M, D, quant)
         if M > 1024:
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
             for i in range(reps):
@@ -379,10 +391,10 @@ def next_ops_leg(peak, floor, reps=50):
             ts = [ev[2 * i].elapsed_time(ev[2 * i + 1]) * 1e3 for i in range(reps)]
             us = sum(ts) / len(ts)
             gbs = nbytes / (us * 1e-6) / 1e9
-            out["gate_residual_adarms_M%d_D%d" % (M, D)] = {
-                "us_mean": round(us, 2), "us_median": round(statistics.median(ts), 2), "bytes": nbytes,
-                "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
-                "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4), "l2": "inputs larger than L2"}
+            out[key] = {"us_mean": round(us, 2), "us_median": round(statistics.median(ts), 2), "bytes": nbytes,
+                        "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                        "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4),
+                        "l2": "inputs larger than L2" if nbytes > (252 << 20) else "fits in L2"}
         else:
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr):
@@ -400,9 +412,8 @@ def next_ops_leg(peak, floor, reps=50):
                 ts.append(e0.elapsed_time(e1) * 1e3 / 200)
             del gr
             node = statistics.median(ts)
-            out["gate_residual_adarms_M%d_D%d" % (M, D)] = {
-                "graph_node_us": round(node, 3), "x_graph_floor": round(node / floor["graph_node_us"], 3)}
-        del x, r, gate, sc, sh, q
+            out[key] = {"graph_node_us": round(node, 3), "x_graph_floor": round(node / floor["graph_node_us"], 3)}
+        del x, r, gate, sc, sh, q, bs
     return out
 
 
@@ -655,6 +666,17 @@ def main(argv=None):
 
     wl = W.get(args.workload)
     peak, peak_kind = measured_peak()
+    if args.next_only:
+        if rank == 0:
+            floor = launch_floor()
+            s = json.dumps({"next_ops": next_ops_leg(peak, floor, args.next_reps, args.next_m),
+                            "launch_floor": floor, "peak": peak, "peak_kind": peak_kind})
+            print(s, flush=True)
+            if args.json_out:
+                with open(args.json_out, "w") as f:
+                    f.write(s + "\n")
+        dist.close()
+        return 0
     step = Step(wl, rank)
     bytes_op = op_bytes(step.wl)
     step_bytes = sum(bytes_op.values())
@@ -694,7 +716,7 @@ def main(argv=None):
             extra["chain" + tag] = chain_leg(args.chain_reps, floor)
             extra["small_m" + tag] = small_m_ops(floor)
             if pdl:
-                extra["next_ops"] = next_ops_leg(peak, floor)
+                extra["next_ops"] = next_ops_leg(peak, floor, args.next_reps, args.next_m)
         frt.frt_set_pdl(pdl0)
     e2e = None
     if not args.no_e2e:

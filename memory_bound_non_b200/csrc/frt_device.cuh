@@ -35,6 +35,14 @@ struct Pack16<FRT_F16> {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
   }
+  // a * b + c on both halves, the exact value rounded once (round to nearest
+  // even, subnormals kept): IEEE fusedMultiplyAdd in binary16.
+  static __device__ __forceinline__ uint32_t fma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+  }
+  static constexpr uint32_t kOnes = 0x3C003C00u;  // (1.0, 1.0)
 };
 
 template <>
@@ -46,6 +54,14 @@ struct Pack16<FRT_BF16> {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
   }
+  // a * b + c on both halves, the exact value rounded once to bfloat16
+  // (round to nearest even).
+  static __device__ __forceinline__ uint32_t fma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+  }
+  static constexpr uint32_t kOnes = 0x3F803F80u;  // (1.0, 1.0)
 };
 
 // Residual add of two 16-bit values: the fp32 sum rounded to the 16-bit type

@@ -3,6 +3,7 @@
 
 #include <cstdint>
 
+#include <atomic>
 #include <cuda_runtime.h>
 
 #include <cuda_runtime_api.h>
@@ -51,6 +52,22 @@ inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
 inline bool quant_args_ok(frt_quant qm, const float* static_scale, const float* block_scales) {
   if (qm == FRT_QUANT_STATIC) return static_scale != nullptr && aligned(static_scale, 4);
   return block_scales != nullptr && aligned(block_scales, 4);
+}
+
+// Raises a kernel's dynamic shared memory limit to `bytes` once (the largest
+// size seen so far is kept in `opted`); needed above the 48 KB default.
+template <typename Kern>
+frt_status opt_in_smem(Kern kern, size_t bytes, std::atomic<int>& opted) {
+  if ((int)bytes > opted.load(std::memory_order_relaxed)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return FRT_ERR_CUDA;
+    }
+    int cur = opted.load(std::memory_order_relaxed);
+    while ((int)bytes > cur && !opted.compare_exchange_weak(cur, (int)bytes)) {
+    }
+  }
+  return FRT_OK;
 }
 
 }  // namespace frt

@@ -1,4 +1,4 @@
-// NEXT-1: gated residual + AdaRMSNorm modulation + FP8 e4m3, one pass per row.
+// NEXT-1: gated residual + AdaRMSNorm modulation + FP8 e4m3.
 //
 // "FlashRT kernel fusion", §三: the Pi0.5 decoder's cross-layer kernel
 // gate_res_adarms_fp8_static does gate multiply + residual add + AdaRMSNorm
@@ -9,10 +9,23 @@
 //   y = h * rstd * (1 + scale_c) + shift_c,  rstd = 1 / sqrt(mean(h^2) + eps);
 //   FP8 of y (static scale or per-token block-128 scales), as op (a).
 //
-// Same mapping as op (a): one small CTA per row, 16-byte vectors, fp64 sum of
-// squares, h * rstd formed as a correctly rounded fp32 value, FP8 codes of the
-// correctly rounded quotient.
+// Mapping (B200): op (a)'s layout -- one small CTA per row, thread t owns the
+// 16-byte chunks t, t+T, ... of the row, sum of squares warp shuffle ->
+// shared memory -> every thread.  Every load is issued at entry: x and the
+// residual (HBM) and the gate (L2) into registers, scale and shift by
+// asynchronous copies into shared memory, which holds them without registers
+// until pass 2 needs them (each thread copies and reads back only its own
+// chunks, so the staging needs no barrier).
+//
+// Arithmetic.  h is one packed 16-bit FMA per pair (fma.rn.{bf16x2,f16x2}:
+// the exact g * x + r rounded once, subnormals kept), which is the oracle's
+// definition itself.  Without modulation the sum of squares is fp64 and
+// y = h * rstd is the correctly rounded fp32 value, as in op (a); with
+// modulation y carries three fp32 roundings anyway and an fp32 sum of squares
+// suffices.  FP8 codes are those of the correctly rounded quotient y / s.
+#include <atomic>
 #include <cmath>
+#include <type_traits>
 
 #include "frt_device.cuh"
 #include "frt_host.h"
@@ -25,127 +38,151 @@ constexpr int max_threads() {
   return K >= 4 ? 512 : 128;
 }
 
-// True when s is a rounding midpoint of the 16-bit type DT.
-template <int DT>
-__device__ __forceinline__ bool midpoint16(float s) {
-  const uint32_t u = __float_as_uint(s);
-  if (DT == FRT_BF16) return (u & 0xFFFFu) == 0x8000u;
-  const float a = fabsf(s);
-  if (a >= 0x1p-14f) return (u & 0x1FFFu) == 0x1000u;
-  const float t = a * 0x1p25f;  // fp16 subnormal midpoints: odd multiples of 2^-25
-  return t == rintf(t) && (((int)t) & 1);
+// 16-byte asynchronous global -> shared copy (cached in L2 only), and its
+// group bookkeeping.
+__device__ __forceinline__ void cp_async16(uint4* smem, const uint4* gmem) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// r + p (p = g * x, exact in fp32) rounded so that one more rounding to the
-// 16-bit type is the correctly rounded exact sum: the fp32 sum from TwoSum,
-// moved one ulp towards the exact value only when it sits exactly on a 16-bit
-// midpoint while the sum was inexact (the one case where rounding it again
-// would differ).  Branch-free.
-template <int DT>
-__device__ __forceinline__ float gated_sum(float r, float p) {
-  const float s = __fadd_rn(r, p);
-  const float bb = __fsub_rn(s, r);
-  const float e = __fadd_rn(__fsub_rn(r, __fsub_rn(s, bb)), __fsub_rn(p, bb));
-  const uint32_t u = __float_as_uint(s);
-  const uint32_t toward = ((__float_as_uint(e) ^ u) & 0x80000000u) ? u - 1u : u + 1u;
-  return (e != 0.0f && midpoint16<DT>(s)) ? __uint_as_float(toward) : s;
-}
-
-template <int DT, int K, bool GATED, int QM>
+template <int DT, int K, bool GATED, bool MOD, int QM>
 __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_kernel(
     const uint4* __restrict__ x, const uint4* __restrict__ gate, const uint4* r_in, uint4* r_out,
     const uint4* __restrict__ scale, const uint4* __restrict__ shift, uint2* __restrict__ q,
     const float* __restrict__ static_scale, float* __restrict__ block_scales, int C, int NB, int rows_per_cond,
     float D, float eps) {
   using P16 = Pack16<DT>;
+  using Acc = typename std::conditional<MOD, float, double>::type;
+  // The gate rides in registers with x and the residual; at the widest rows
+  // (K = 8) registers run out and it is staged in shared memory instead.
+  constexpr bool kGateSmem = K >= 8;
   pdl_enter();
   const int t = threadIdx.x;
   const int T = blockDim.x;
   const int64_t row = blockIdx.x;
   const int64_t base = row * (int64_t)C;
-  const int64_t cbase = (row / rows_per_cond) * (int64_t)C;
+  const int64_t cbase = (int64_t)((int)blockIdx.x / rows_per_cond) * C;
   __shared__ double red[32];
+  extern __shared__ uint4 cond[];
+  uint4* s_gate = cond;
+  uint4* s_scale = cond + (GATED && kGateSmem ? C : 0);
+  uint4* s_shift = s_scale + C;
 
-  uint4 xv[K], rv[K], gv[GATED ? K : 1];
+  uint4 xv[K], rv[K], gv[GATED && !kGateSmem ? K : 1];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = t + k * T;
     if (c < C) {
       xv[k] = ld_stream(x + base + c);
       rv[k] = ld_plain(r_in + base + c);
-      if (GATED) gv[k] = __ldg(gate + cbase + c);
+      if (GATED && !kGateSmem) gv[k] = __ldg(gate + cbase + c);
     }
+  }
+  if (GATED && kGateSmem) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (t + k * T < C) cp_async16(s_gate + t + k * T, gate + cbase + t + k * T);
+    cp_async_commit();
+  }
+  if (MOD) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = t + k * T;
+      if (c < C) {
+        if (scale != nullptr) cp_async16(s_scale + c, scale + cbase + c);
+        else s_scale[c] = make_uint4(0u, 0u, 0u, 0u);  // 16-bit zeros
+        if (shift != nullptr) cp_async16(s_shift + c, shift + cbase + c);
+        else s_shift[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    cp_async_commit();
   }
   float s_static = 0.0f;
   if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
+  if (GATED && kGateSmem) {
+    if (MOD) cp_async_wait<1>();  // the gate group; scale / shift may still be in flight
+    else cp_async_wait<0>();
+  }
 
-  // Pass 1: h = gate * x + r rounded once to 16 bits (packed), fp64 sum of squares.
+  // Pass 1: h = gate * x + r rounded once to 16 bits (packed), written back;
+  // sum of squares (squares of 16-bit values are exact in fp32).
   uint4 hv[K];
-  double ss[K];
+  Acc ss = 0;
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    ss[k] = 0.0;
     const int c = t + k * T;
+    hv[k] = make_uint4(0u, 0u, 0u, 0u);
     if (c < C) {
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv[k]);
       const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rv[k]);
-      const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv[GATED ? k : 0]);
+      uint4 g = make_uint4(0u, 0u, 0u, 0u);
+      if (GATED) g = kGateSmem ? s_gate[c] : gv[kGateSmem ? 0 : k];
+      const uint32_t* gw = reinterpret_cast<const uint32_t*>(&g);
       uint32_t* hw = reinterpret_cast<uint32_t*>(&hv[k]);
+      Acc sk = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 xf = P16::to_float2(xw[e]);
-        const float2 rf = P16::to_float2(rw[e]);
-        float s0, s1;
-        if (GATED) {
-          const float2 gf = P16::to_float2(gw[e]);
-          s0 = gated_sum<DT>(rf.x, gf.x * xf.x);  // 16-bit x 16-bit: exact in fp32
-          s1 = gated_sum<DT>(rf.y, gf.y * xf.y);
-        } else {
-          s0 = add_for_16(xf.x, rf.x);
-          s1 = add_for_16(xf.y, rf.y);
-        }
-        hw[e] = P16::from_float2(s0, s1);
+        // h = g * x + r with one rounding of the exact value: the packed
+        // 16-bit FMA (without a gate, 1 * x + r).
+        hw[e] = P16::fma2(GATED ? gw[e] : P16::kOnes, xw[e], rw[e]);
         const float2 hf = P16::to_float2(hw[e]);
-        ss[k] = fma((double)hf.x, (double)hf.x, ss[k]);
-        ss[k] = fma((double)hf.y, (double)hf.y, ss[k]);
+        sk = fma((Acc)hf.x, (Acc)hf.x, sk);
+        sk = fma((Acc)hf.y, (Acc)hf.y, sk);
       }
+      ss += sk;
       r_out[base + c] = hv[k];
-    } else {
-      hv[k] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  double sst = ss[0];
+
+  // Row total: warp butterfly, then every thread adds the warp partials in
+  // the same order (bitwise deterministic).
 #pragma unroll
-  for (int k = 1; k < K; ++k) sst += ss[k];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sst += __shfl_xor_sync(0xFFFFFFFFu, sst, o);
-  if ((t & 31) == 0) red[t >> 5] = sst;
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+  if ((t & 31) == 0) red[t >> 5] = (double)ss;
   __syncthreads();
   double tot = 0.0;
   const int nw = T >> 5;
   for (int i = 0; i < nw; ++i) tot += red[i];
-  const Split32 rstd(rsqrt_f64(tot / (double)D + (double)eps));
+  const Split32 rstd(MOD ? 0.0 : rsqrt_f64(tot / (double)D + (double)eps));
+  const float rstd32 = MOD ? rsqrtf((float)tot / D + eps) : 0.0f;
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
+  if (MOD) cp_async_wait<0>();
 
-  // Pass 2: y = h * rstd * (1 + scale) + shift, then FP8.
+  // Pass 2: y and its FP8 codes.
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = t + k * T;
     const bool valid = c < C;
     const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv[k]);
-    uint4 scv = make_uint4(0u, 0u, 0u, 0u), shv = make_uint4(0u, 0u, 0u, 0u);  // 16-bit zeros
-    if (valid && scale != nullptr) scv = __ldg(scale + cbase + c);
-    if (valid && shift != nullptr) shv = __ldg(shift + cbase + c);
-    const uint32_t* scw = reinterpret_cast<const uint32_t*>(&scv);
-    const uint32_t* shw = reinterpret_cast<const uint32_t*>(&shv);
     float y[8];
+    if (MOD) {
+      uint4 scv = make_uint4(0u, 0u, 0u, 0u), shv = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) {
+        scv = s_scale[c];
+        shv = s_shift[c];
+      }
+      const uint32_t* scw = reinterpret_cast<const uint32_t*>(&scv);
+      const uint32_t* shw = reinterpret_cast<const uint32_t*>(&shv);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 hf = P16::to_float2(hw[e]);
-      const float2 sc = P16::to_float2(scw[e]);
-      const float2 sh = P16::to_float2(shw[e]);
-      y[2 * e] = fmaf(rstd.mul(hf.x), 1.0f + sc.x, sh.x);
-      y[2 * e + 1] = fmaf(rstd.mul(hf.y), 1.0f + sc.y, sh.y);
+      for (int e = 0; e < 4; ++e) {
+        const float2 hf = P16::to_float2(hw[e]);
+        const float2 sc = P16::to_float2(scw[e]);
+        const float2 sh = P16::to_float2(shw[e]);
+        y[2 * e] = fmaf(hf.x * rstd32, 1.0f + sc.x, sh.x);
+        y[2 * e + 1] = fmaf(hf.y * rstd32, 1.0f + sc.y, sh.y);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 hf = P16::to_float2(hw[e]);
+        y[2 * e] = rstd.mul(hf.x);
+        y[2 * e + 1] = rstd.mul(hf.y);
+      }
     }
     if (QM == FRT_QUANT_BLOCK128) {
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
@@ -170,30 +207,40 @@ struct Args {
   float eps;
 };
 
-template <int DT, int K, bool G, int QM>
+template <int DT, int K, bool G, bool MOD, int QM>
 frt_status launch_k(const Args& a, cudaStream_t st) {
-  return launch(gate_residual_adarms_fp8_kernel<DT, K, G, QM>, dim3(a.M), dim3(a.T), 0, st,
-                static_cast<const uint4*>(a.x), static_cast<const uint4*>(a.gate), static_cast<const uint4*>(a.r_in),
-                static_cast<uint4*>(a.r_out), static_cast<const uint4*>(a.scale), static_cast<const uint4*>(a.shift),
-                reinterpret_cast<uint2*>(a.q), a.ss, a.bs, a.C, a.NB, a.rows_per_cond, (float)(a.C * 8), a.eps);
+  static std::atomic<int> opted{0};
+  auto kern = gate_residual_adarms_fp8_kernel<DT, K, G, MOD, QM>;
+  const size_t smem = (size_t)((G && K >= 8 ? 1 : 0) + (MOD ? 2 : 0)) * a.C * sizeof(uint4);
+  const frt_status os = opt_in_smem(kern, smem, opted);
+  if (os != FRT_OK) return os;
+  return launch(kern, dim3(a.M), dim3(a.T), smem, st, static_cast<const uint4*>(a.x),
+                static_cast<const uint4*>(a.gate), static_cast<const uint4*>(a.r_in), static_cast<uint4*>(a.r_out),
+                static_cast<const uint4*>(a.scale), static_cast<const uint4*>(a.shift), reinterpret_cast<uint2*>(a.q),
+                a.ss, a.bs, a.C, a.NB, a.rows_per_cond, (float)(a.C * 8), a.eps);
+}
+
+template <int DT, int K, bool G>
+frt_status launch_gk(bool mod, frt_quant qm, const Args& a, cudaStream_t st) {
+  if (mod)
+    return qm == FRT_QUANT_STATIC ? launch_k<DT, K, G, true, FRT_QUANT_STATIC>(a, st)
+                                  : launch_k<DT, K, G, true, FRT_QUANT_BLOCK128>(a, st);
+  return qm == FRT_QUANT_STATIC ? launch_k<DT, K, G, false, FRT_QUANT_STATIC>(a, st)
+                                : launch_k<DT, K, G, false, FRT_QUANT_BLOCK128>(a, st);
 }
 
 template <int DT, int K>
-frt_status launch_dk(bool gated, frt_quant qm, const Args& a, cudaStream_t st) {
-  if (gated)
-    return qm == FRT_QUANT_STATIC ? launch_k<DT, K, true, FRT_QUANT_STATIC>(a, st)
-                                  : launch_k<DT, K, true, FRT_QUANT_BLOCK128>(a, st);
-  return qm == FRT_QUANT_STATIC ? launch_k<DT, K, false, FRT_QUANT_STATIC>(a, st)
-                                : launch_k<DT, K, false, FRT_QUANT_BLOCK128>(a, st);
+frt_status launch_dk(bool gated, bool mod, frt_quant qm, const Args& a, cudaStream_t st) {
+  return gated ? launch_gk<DT, K, true>(mod, qm, a, st) : launch_gk<DT, K, false>(mod, qm, a, st);
 }
 
 template <int DT>
-frt_status launch_dt(int K, bool gated, frt_quant qm, const Args& a, cudaStream_t st) {
+frt_status launch_dt(int K, bool gated, bool mod, frt_quant qm, const Args& a, cudaStream_t st) {
   switch (K) {
-    case 1: return launch_dk<DT, 1>(gated, qm, a, st);
-    case 2: return launch_dk<DT, 2>(gated, qm, a, st);
-    case 4: return launch_dk<DT, 4>(gated, qm, a, st);
-    default: return launch_dk<DT, 8>(gated, qm, a, st);
+    case 1: return launch_dk<DT, 1>(gated, mod, qm, a, st);
+    case 2: return launch_dk<DT, 2>(gated, mod, qm, a, st);
+    case 4: return launch_dk<DT, 4>(gated, mod, qm, a, st);
+    default: return launch_dk<DT, 8>(gated, mod, qm, a, st);
   }
 }
 
@@ -221,6 +268,7 @@ extern "C" frt_status frt_gate_residual_adarms_fp8(const void* x, const void* ga
   const int per = (C + K - 1) / K;
   Args a{x, gate, residual_in, residual_out, scale, shift, out_fp8, static_scale, block_scales, M, C,
          (D + 127) / 128, rows_per_cond, ((per + 31) / 32) * 32, eps};
-  return dt == FRT_F16 ? launch_dt<FRT_F16>(K, gate != nullptr, qm, a, stream)
-                       : launch_dt<FRT_BF16>(K, gate != nullptr, qm, a, stream);
+  const bool mod = scale != nullptr || shift != nullptr;
+  return dt == FRT_F16 ? launch_dt<FRT_F16>(K, gate != nullptr, mod, qm, a, stream)
+                       : launch_dt<FRT_BF16>(K, gate != nullptr, mod, qm, a, stream);
 }

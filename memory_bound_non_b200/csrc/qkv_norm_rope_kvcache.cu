@@ -352,20 +352,6 @@ inline Shape qkv_shape(int M, int H, int GP) {
   return sh;
 }
 
-template <typename Kern>
-frt_status opt_in_smem(Kern kern, size_t bytes, std::atomic<int>& opted) {
-  if ((int)bytes > opted.load(std::memory_order_relaxed)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) {
-      (void)cudaGetLastError();
-      return FRT_ERR_CUDA;
-    }
-    int cur = opted.load(std::memory_order_relaxed);
-    while ((int)bytes > cur && !opted.compare_exchange_weak(cur, (int)bytes)) {
-    }
-  }
-  return FRT_OK;
-}
-
 // Shared memory of the bulk-copy kernel: the QKV row, cos and sin rows, two
 // norm weights.
 inline size_t tma_smem(int H, int hd) { return (size_t)H * hd * 2 + (size_t)hd * 4 + (size_t)hd * 4; }

@@ -65,3 +65,4 @@ def test_products_of_16bit_values_are_exact_in_fp32():
         p64 = x.astype(np.float64) * y.astype(np.float64)
         ok = np.isfinite(p64) & (np.abs(p64) > 2.0 ** -126) & (np.abs(p64) < 3e38)
         np.testing.assert_array_equal(p32[ok].astype(np.float64), p64[ok])
+

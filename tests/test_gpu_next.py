@@ -116,33 +116,81 @@ def test_adarms_fp16_wide_and_in_place():
     check(6, 4096, "f16", "block128", rpc=1, seed=21, inplace=True)
 
 
-def test_adarms_sums_on_a_16bit_midpoint():
-    """Triples whose fp32 sum r + g x lies on a bf16 rounding midpoint while the
-    exact sum does not: rounding the fp32 sum again would give the wrong h."""
+def _midpoint_triples(dt, n, rng):
+    """r, g, x bit patterns where |r| is far below |g x| half of the time, so
+    that r's bits fall below the fp32 ulp of the sum and, when g x sits on a
+    16-bit midpoint, the sign of r alone decides the rounding."""
+    sgn = lambda: rng.integers(0, 2, n) << 15
+    coin = lambda: rng.integers(0, 2, n) == 1
+    if dt == "bf16":
+        r = np.where(coin(), rng.integers(0x3000, 0x3800, n), rng.integers(0x3800, 0x4800, n)) | sgn()
+        g = rng.integers(0x3C00, 0x3F80, n)
+        x = rng.integers(0x3F80, 0x4100, n) | sgn()
+    else:
+        r = np.where(coin(), rng.integers(0x0001, 0x0040, n), rng.integers(0x0400, 0x5000, n)) | sgn()
+        g = np.where(coin(), rng.choice([0x3E00, 0x3D00, 0x3F00, 0x3A00, 0x3500], n), rng.integers(0x3000, 0x3C00, n))
+        x = rng.integers(0x3C00, 0x4800, n) | sgn()
+    return tuple(a.astype(np.uint16) for a in (r, g, x))
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_adarms_sums_on_a_16bit_midpoint(dt):
+    """Rows holding triples whose plain fp32 sum r + g x lies on a 16-bit
+    rounding midpoint while the exact sum does not (rounding the fp32 sum again
+    would give the wrong h): h must still be the oracle's, bit for bit."""
     rng = np.random.default_rng(7)
-    n = 1 << 18
-    # |r| << |g x|: r's bits fall below the fp32 ulp of the sum, and when g x
-    # sits on a bf16 midpoint the sign of r alone decides the rounding
-    r = rng.integers(0x3000, 0x3800, n).astype(np.uint16) | (rng.integers(0, 2, n).astype(np.uint16) << 15)
-    g = rng.integers(0x3C00, 0x3F80, n).astype(np.uint16)          # gate in [2^-7, 1)
-    x = rng.integers(0x3F80, 0x4100, n).astype(np.uint16) | (rng.integers(0, 2, n).astype(np.uint16) << 15)
-    tr, tg, tx = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) for a in (r, g, x))
-    naive = W.bits16((tr.float() + tg.float() * tx.float()).to(torch.bfloat16))
     D = 1024
+    r, g, x = _midpoint_triples(dt, 1 << 18, rng)
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float16
+    tr, tg, tx = (torch.from_numpy(a.view(np.int16)).view(tdt) for a in (r, g, x))
+    naive = W.bits16((tr.float() + tg.float() * tx.float()).to(tdt))
     o = oracle.gate_residual_adarms_fp8(x.reshape(-1, D), g.reshape(-1, D), r.reshape(-1, D), None, None, 1e-6,
-                                        "bf16", "block128", 1)
+                                        dt, "block128", 1)
     hard = naive.reshape(-1, D) != o["residual_out"]
-    assert hard.sum() > 50, "the inputs do not exercise the midpoint case"
+    assert hard.sum() > 20, "the inputs do not exercise the midpoint case"
     rows = np.flatnonzero(hard.any(axis=1))[:64]
-    M = len(rows)
-    xs, gs, rs = (torch.from_numpy(a.reshape(-1, D)[rows].copy().view(np.int16)).view(torch.bfloat16)
-                  for a in (x, g, r))
+    xs, gs, rs = (torch.from_numpy(a.reshape(-1, D)[rows].copy().view(np.int16)).view(tdt) for a in (x, g, r))
     ro, q, bs = run_gpu(xs, rs, gs, None, None, "block128", None, 1)
-    want = o["residual_out"][rows]
-    np.testing.assert_array_equal(W.bits16(ro.cpu()), want)
-    om = oracle.gate_residual_adarms_fp8(W.bits16(xs), W.bits16(gs), W.bits16(rs), None, None, 1e-6, "bf16",
+    np.testing.assert_array_equal(W.bits16(ro.cpu()), o["residual_out"][rows])
+    om = oracle.gate_residual_adarms_fp8(W.bits16(xs), W.bits16(gs), W.bits16(rs), None, None, 1e-6, dt,
                                          "block128", 1)
     P.assert_fp8_codes(q.cpu().numpy(), om["out_fp8"], what="midpoint rows codes")
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("gated", [True, False])
+def test_adarms_subnormal_and_signed_zero_sums(dt, gated):
+    """Subnormal residuals and products, exact cancellations (+0) and -0 + -0
+    (-0): h is still the oracle's value bit for bit."""
+    rng = np.random.default_rng(9)
+    M, D = 4, 1024
+    n = M * D
+    sub_hi = 0x0080 if dt == "bf16" else 0x0400            # exponent field zero
+    one = 0x3F80 if dt == "bf16" else 0x3C00
+    sgn = lambda: (rng.integers(0, 2, n) << 15).astype(np.uint16)
+    r = (rng.integers(1, sub_hi, n).astype(np.uint16) | sgn())
+    x = (rng.integers(1, sub_hi, n).astype(np.uint16) | sgn())
+    lo_g, hi_g = (0x3E80, 0x4000) if dt == "bf16" else (0x3400, 0x4000)   # gate in [0.25, 2)
+    g = rng.integers(lo_g, hi_g, n).astype(np.uint16)
+    k = np.arange(n)
+    cancel, negzero = k % 16 == 3, k % 16 == 7
+    g[cancel] = one
+    x[cancel] = r[cancel] ^ 0x8000                          # 1 * (-r) + r = +0
+    r[negzero] = 0x8000
+    x[negzero] = 0x8000                                     # g * (-0) + (-0) = -0
+    gate = g.reshape(M, D) if gated else None
+    if not gated:
+        x[cancel] = r[cancel] ^ 0x8000
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float16
+    to_t = lambda a: torch.from_numpy(a.reshape(M, D).copy().view(np.int16)).view(tdt)
+    o = oracle.gate_residual_adarms_fp8(x.reshape(M, D), None if gate is None else gate.reshape(M, D),
+                                        r.reshape(M, D), None, None, 1e-6, dt, "block128", 1)
+    want = o["residual_out"]
+    assert (want.ravel()[cancel] == 0x0000).all() and (want.ravel()[negzero] == 0x8000).all()
+    assert ((want & 0x7FFF) < sub_hi).sum() > n // 4, "few subnormal results"
+    ro, q, bs = run_gpu(to_t(x), to_t(r), None if gate is None else to_t(g), None, None, "block128", None, 1)
+    np.testing.assert_array_equal(W.bits16(ro.cpu()), want)
+    P.assert_fp8_codes(q.cpu().numpy(), o["out_fp8"], what="subnormal rows codes")
 
 
 def test_adarms_without_gate_or_modulation_equals_op_a():
