@@ -394,7 +394,8 @@ def next_ops_leg(peak, floor, reps=50, big_m=65536):
             out[key] = {"us_mean": round(us, 2), "us_median": round(statistics.median(ts), 2), "bytes": nbytes,
                         "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
                         "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4),
-                        "l2": "inputs larger than L2" if nbytes > (252 << 20) else "fits in L2"}
+                        "l2": "inputs larger than L2" if nbytes > (252 << 20) else "fits in L2",
+                        "traffic": measured_traffic(key, "gate_residual_adarms")}
         else:
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr):
