@@ -64,13 +64,6 @@ struct Pack16<FRT_BF16> {
   static constexpr uint32_t kOnes = 0x3F803F80u;  // (1.0, 1.0)
 };
 
-// Residual add of two 16-bit values: the fp32 sum rounded to the 16-bit type
-// is the correctly rounded exact sum.  Rounding an exact sum first to q = 24
-// bits and then to p bits equals rounding it once to p bits whenever
-// q >= 2p + 1 (S. A. Figueroa, "When is double rounding innocuous?", 1995);
-// p = 8 (bf16) and p = 11 (fp16) both satisfy it.
-__device__ __forceinline__ float add_for_16(float a, float b) { return __fadd_rn(a, b); }
-
 // 1 / sqrt(x) in fp64, to ~1e-16 relative (not correctly rounded): an fp32
 // estimate refined by two Newton steps in fp64.  Every lane can afford it
 // (about a dozen instructions), unlike a correctly rounded sqrt + divide.

@@ -46,7 +46,7 @@ __device__ __forceinline__ float act_fn(float g) {
   }
 }
 
-template <int DT, int ACT, int QM>
+template <int DT, int ACT, int QM, bool FULL>
 __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __restrict__ gu,
                                                                  uint32_t* __restrict__ q,
                                                                  const float* __restrict__ static_scale,
@@ -59,20 +59,33 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
   const int64_t gb0 = warp * kU;
 
   // Load phase: chunk `lane` of each of the U blocks (4 outputs = 16 bytes).
+  // FULL (I % 128 == 0): every block is 32 whole chunks, so the flat chunk
+  // index is just 32 * block + lane; otherwise rows end in a partial block
+  // and the (row, block) position is tracked.
   uint4 v[kU];
   int64_t idx[kU];
   bool valid[kU];
-  int64_t row = gb0 / NB;
-  int b = (int)(gb0 - row * NB);
+  if (FULL) {
+    const int64_t i0 = gb0 * 32 + lane;
 #pragma unroll
-  for (int u = 0; u < kU; ++u) {
-    const int chunk = b * 32 + lane;  // chunk index within the row (4 outputs each)
-    valid[u] = gb0 + u < total_blocks && chunk < C4;
-    idx[u] = row * C4 + chunk;       // same index for the input (uint4) and output (uint32) views
-    if (valid[u]) v[u] = ld_stream(gu + idx[u]);
-    if (++b == NB) {
-      b = 0;
-      ++row;
+    for (int u = 0; u < kU; ++u) {
+      valid[u] = gb0 + u < total_blocks;
+      idx[u] = i0 + 32 * u;  // same index for the input (uint4) and output (uint32) views
+      if (valid[u]) v[u] = ld_stream(gu + idx[u]);
+    }
+  } else {
+    int64_t row = gb0 / NB;
+    int b = (int)(gb0 - row * NB);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int chunk = b * 32 + lane;  // chunk index within the row (4 outputs each)
+      valid[u] = gb0 + u < total_blocks && chunk < C4;
+      idx[u] = row * C4 + chunk;
+      if (valid[u]) v[u] = ld_stream(gu + idx[u]);
+      if (++b == NB) {
+        b = 0;
+        ++row;
+      }
     }
   }
 
@@ -109,11 +122,16 @@ frt_status launch_act(frt_quant qm, const void* gu, uint8_t* q, const float* ss,
   const dim3 grid((unsigned)((warps + kWarps - 1) / kWarps));
   const uint4* in = static_cast<const uint4*>(gu);
   uint32_t* out = reinterpret_cast<uint32_t*>(q);
+  const bool full = C4 == NB * 32;
   if (qm == FRT_QUANT_STATIC)
-    return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
-                  NB, C4);
-  return launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
-                NB, C4);
+    return full ? launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC, true>, grid, dim3(kThreads), 0, st, in, out,
+                         ss, bs, total, NB, C4)
+                : launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC, false>, grid, dim3(kThreads), 0, st, in, out,
+                         ss, bs, total, NB, C4);
+  return full ? launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128, true>, grid, dim3(kThreads), 0, st, in, out,
+                       ss, bs, total, NB, C4)
+              : launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128, false>, grid, dim3(kThreads), 0, st, in, out,
+                       ss, bs, total, NB, C4);
 }
 
 template <int DT>

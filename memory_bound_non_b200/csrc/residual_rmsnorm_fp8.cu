@@ -67,9 +67,9 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       if (t + k * T < C) wv_early[k] = __ldg(w + t + k * T);
   }
 
-  // Pass 1: h = x + r rounded once to 16 bits (exactly the rounded exact sum,
-  // see add_for_16), kept packed; fp64 sum of squares (squares of 16-bit
-  // values are exact, so the sum is exact to ~2^-40), one accumulator per chunk.
+  // Pass 1: h = x + r rounded once to 16 bits (the correctly rounded exact
+  // sum), kept packed; fp64 sum of squares (squares of 16-bit values are
+  // exact, so the sum is exact to ~2^-40), one accumulator per chunk.
   uint4 hv[K];
   double ss[K];
 #pragma unroll
@@ -80,12 +80,10 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv[k]);
       const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rv[k]);
       uint32_t* hw = reinterpret_cast<uint32_t*>(&hv[k]);
+      // h = 1 * x + r by the packed 16-bit FMA: the exact sum rounded once,
+      // half an instruction per element.
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 xf = P16::to_float2(xw[e]);
-        const float2 rf = P16::to_float2(rw[e]);
-        hw[e] = P16::from_float2(add_for_16(xf.x, rf.x), add_for_16(xf.y, rf.y));
-      }
+      for (int e = 0; e < 4; ++e) hw[e] = P16::fma2(P16::kOnes, xw[e], rw[e]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 hf = P16::to_float2(hw[e]);

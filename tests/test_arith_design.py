@@ -1,11 +1,13 @@
-"""CPU checks of the arithmetic identities the kernels rely on (no GPU).
+"""CPU checks of arithmetic identities behind the kernels and the oracle (no GPU).
 
-The residual add is computed in fp32 and rounded once to the 16-bit type; that
-equals the correctly rounded exact sum because fp32 carries at least 2p + 1
-significand bits for p = 8 (bf16) and p = 11 (fp16) -- the double-rounding
-condition of Figueroa ("When is double rounding innocuous?").  Here IEEE fp32
-addition (numpy) followed by a library RNE conversion is compared with the
-oracle's exact sum on pairs that cover every exponent gap.
+The oracle rounds the exact sum of two 16-bit values once (add16).  An
+independent route to the same value: the IEEE fp32 sum (numpy) followed by a
+library RNE conversion, which equals the correctly rounded exact sum because
+fp32 carries at least 2p + 1 significand bits for p = 8 (bf16) and p = 11
+(fp16) -- the double-rounding condition of Figueroa ("When is double rounding
+innocuous?").  Compared on pairs that cover every exponent gap.  The kernels
+form the same sum with the packed 16-bit FMA (one rounding of the exact
+value), checked against the oracle on the GPU.
 """
 import numpy as np
 import pytest
