@@ -440,4 +440,78 @@ int oracle_gate_residual_adarms_fp8(const uint16_t* x, const uint16_t* gate, con
   return 0;
 }
 
+// NEXT-2: op (b) with the attention's Q preparation folded in and an
+// optional FP8 KV cache ([FR] §2.2 first bullet for op (b); the "sm89 / 5060
+// Ti" port's step 10, FA2 prepare_q fused into RoPE).  Reading (the pages
+// name the fusion only): prepare_q multiplies Q by the attention's softmax
+// scale q_scale and may lay Q out head-major for the attention kernel; the
+// FP8 cache holds e4m3 codes with one static dequantisation scale per tensor.
+//   q        = rope(norm(q_head)) * q_scale (fp64, unrounded), stored at
+//              q_out[i, h, :] (q_head_major == 0) or q_out[h, i, :] (== 1);
+//   kv_fp8 == 0: k_cache (fp64) and v_cache (16-bit) exactly as op (b);
+//   kv_fp8 == 1: k_cache8[slot, g, :] = e4m3(fp32(k) / fp32(k_scale)),
+//                v_cache8[slot, g, :] = e4m3(fp32(v) / fp32(v_scale)), the
+//                FP8 decision taken in fp32 as for the other FP8 outputs.
+// Positions outside [0, max_pos) or slots outside [0, capacity) skip the row
+// and set status bit 0, as op (b).
+int oracle_qkv_norm_rope_prepq_kvcache(const uint16_t* qkv, const uint16_t* q_norm_w, const uint16_t* k_norm_w,
+                                       const float* cos_tab, const float* sin_tab, const int32_t* positions,
+                                       double* q_out, double* k_cache, uint16_t* v_cache, uint8_t* k_cache8,
+                                       uint8_t* v_cache8, int32_t* status, int64_t M, int64_t Hq, int64_t Hkv,
+                                       int64_t hd, int64_t max_pos, int64_t capacity, double eps, int dt,
+                                       double q_scale, int q_head_major, int kv_fp8, double k_scale,
+                                       double v_scale) {
+  if (M < 0 || Hq <= 0 || Hkv <= 0 || hd <= 0 || hd % 2 != 0) return -1;
+  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out) return -1;
+  if (kv_fp8 ? (!k_cache8 || !v_cache8) : (!k_cache || !v_cache)) return -1;
+  const Fmt16 f = fmt_of(dt);
+  const int64_t width = (Hq + 2 * Hkv) * hd;
+  const int64_t half = hd / 2;
+  const float ks32 = (float)k_scale, vs32 = (float)v_scale;
+  std::vector<double> v(hd), wq(hd), wk(hd), y(hd);
+  for (int64_t j = 0; j < hd; ++j) {
+    if (q_norm_w) wq[j] = decode16(q_norm_w[j], f);
+    if (k_norm_w) wk[j] = decode16(k_norm_w[j], f);
+  }
+  for (int64_t i = 0; i < M; ++i) {
+    const int64_t p = positions[i];
+    if (p < 0 || p >= max_pos || p >= capacity) {
+      if (status) *status |= 1;
+      continue;
+    }
+    const float* c = cos_tab + p * half;
+    const float* s = sin_tab + p * half;
+    const uint16_t* row = qkv + i * width;
+    for (int64_t h = 0; h < Hq + Hkv; ++h) {
+      const bool is_q = h < Hq;
+      for (int64_t j = 0; j < hd; ++j) v[j] = decode16(row[h * hd + j], f);
+      const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
+      if (nw) {
+        rmsnorm(v.data(), hd, is_q ? wq.data() : wk.data(), eps, y.data());
+        v = y;
+      }
+      rope_rotate_half(v.data(), (int)hd, c, s);
+      if (is_q) {
+        double* dst = q_head_major ? q_out + (h * M + i) * hd : q_out + (i * Hq + h) * hd;
+        for (int64_t j = 0; j < hd; ++j) dst[j] = v[j] * q_scale;
+      } else if (kv_fp8) {
+        uint8_t* dst = k_cache8 + (p * Hkv + (h - Hq)) * hd;
+        for (int64_t j = 0; j < hd; ++j) dst[j] = quant_fp32(v[j], ks32);
+      } else {
+        std::memcpy(k_cache + (p * Hkv + (h - Hq)) * hd, v.data(), sizeof(double) * hd);
+      }
+    }
+    for (int64_t g = 0; g < Hkv; ++g) {
+      const uint16_t* src = row + (Hq + Hkv + g) * hd;
+      if (kv_fp8) {
+        uint8_t* dst = v_cache8 + (p * Hkv + g) * hd;
+        for (int64_t j = 0; j < hd; ++j) dst[j] = quant_fp32(decode16(src[j], f), vs32);
+      } else {
+        std::memcpy(v_cache + (p * Hkv + g) * hd, src, sizeof(uint16_t) * hd);
+      }
+    }
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -95,3 +95,104 @@ def test_adarms_residual_is_the_exactly_rounded_gated_sum():
         h, _, _ = npr.gate_residual_adarms_fp8(x, gate, r, None, None, 1e-6, dt, "block128", 1)
         ok = np.isfinite(oracle.decode16(o["residual_out"], dt))
         np.testing.assert_array_equal(o["residual_out"][ok], h[ok])
+
+
+# ------------------------------------------------------------------ NEXT-2 --
+# Op (b) with the attention's Q preparation (softmax-scale pre-multiply,
+# head-major layout) and an optional e4m3 KV cache with static scales (the
+# "5060 Ti" port's step 10, FA2 prepare_q fused into RoPE; "FlashRT kernel
+# fusion", §2.2).
+
+def _qkv_inputs(M=5, Hq=4, Hkv=2, hd=16, dt="bf16", seed=7, qk_norm=True):
+    g = W.generator(seed)
+    H = Hq + 2 * Hkv
+    qkv = W.bits16(W.normal16((M, H * hd), dt, g))
+    qw = W.bits16(W.norm_weight(hd, dt, g)) if qk_norm else None
+    kw = W.bits16(W.norm_weight(hd, dt, g)) if qk_norm else None
+    cos, sin = W.rope_tables(64, hd, 1e4)
+    pos = np.arange(3, 3 + M, dtype=np.int32)
+    return qkv, qw, kw, cos.numpy(), sin.numpy(), pos
+
+
+def _nearest_e4m3(y):
+    """Brute force: the finite e4m3 code nearest to y (ties to the even code,
+    |y| beyond 448 saturating), by scanning the whole code table."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = np.array([oracle.e4m3_decode(int(c)) for c in codes])
+    out = np.empty(y.shape, dtype=np.uint8)
+    for idx, v in np.ndenumerate(y):
+        v = float(np.clip(v, -448.0, 448.0))
+        d = np.abs(vals - v)
+        best = np.flatnonzero(d == d.min())
+        best = [c for c in codes[best] if not (v >= 0) ^ (c < 0x80)] or list(codes[best])
+        even = [c for c in best if (c & 1) == 0]
+        out[idx] = (even or best)[0]
+    return out
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("qk_norm", [True, False])
+def test_prepq_defaults_reduce_to_op_b(dt, qk_norm):
+    qkv, qw, kw, cos, sin, pos = _qkv_inputs(dt=dt, qk_norm=qk_norm)
+    a = oracle.qkv_norm_rope_prepq_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, dt)
+    b = oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, dt)
+    np.testing.assert_array_equal(a["q_out"], b["q_out"])
+    np.testing.assert_array_equal(a["k_cache"], b["k_cache"])
+    np.testing.assert_array_equal(a["v_cache"], b["v_cache"])
+
+
+def test_prepq_head_major_is_the_transpose_and_power_of_two_scale_is_exact():
+    qkv, qw, kw, cos, sin, pos = _qkv_inputs()
+    base = oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, "bf16")["q_out"]
+    o = oracle.qkv_norm_rope_prepq_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, "bf16", q_scale=0.125,
+                                           q_layout="head")
+    assert o["q_out"].shape == (4, 5, 16)
+    np.testing.assert_array_equal(o["q_out"], 0.125 * base.transpose(1, 0, 2))
+
+
+def test_prepq_softmax_scale():
+    qkv, qw, kw, cos, sin, pos = _qkv_inputs(hd=16)
+    base = oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, "bf16")["q_out"]
+    sc = float(np.float32(1.0 / math.sqrt(16.0) * 1.4426950408889634))   # 1/sqrt(hd) * log2(e), as fp32
+    o = oracle.qkv_norm_rope_prepq_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, "bf16", q_scale=sc)
+    np.testing.assert_allclose(o["q_out"], base * sc, rtol=1e-15, atol=0)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_prepq_fp8_cache_codes_are_the_nearest_codes(dt):
+    qkv, qw, kw, cos, sin, pos = _qkv_inputs(dt=dt)
+    base = oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, dt)
+    ks, vs = 0.0078125, 0.00390625 * 3      # K: power of two; V: 3/256 (an inexact quotient)
+    o = oracle.qkv_norm_rope_prepq_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 16, 1e-6, dt, kv="e4m3",
+                                           k_scale=ks, v_scale=vs)
+    rows = pos
+    k = base["k_cache"][rows].astype(np.float32).astype(np.float64)       # the fp32 value the decision uses
+    np.testing.assert_array_equal(o["k_cache"][rows], _nearest_e4m3(k / ks))
+    v = oracle.decode16(base["v_cache"][rows], dt)
+    vq = (v.astype(np.float32) / np.float32(vs)).astype(np.float64)       # fp32 quotient, as the reading says
+    np.testing.assert_array_equal(o["v_cache"][rows], _nearest_e4m3(vq))
+    untouched = np.setdiff1d(np.arange(16), rows)
+    assert (o["k_cache"][untouched] == 0x7E).all() and (o["v_cache"][untouched] == 0x7E).all()
+
+
+def test_prepq_fp8_cache_saturates_and_keeps_sign():
+    qkv, qw, kw, cos, sin, pos = _qkv_inputs(qk_norm=False)
+    o = oracle.qkv_norm_rope_prepq_kvcache(qkv, None, None, cos, sin, pos, 4, 2, 16, 16, 1e-6, "bf16", kv="e4m3",
+                                           k_scale=1e-4, v_scale=1e-4)
+    v = oracle.decode16(qkv[:, 6 * 16:].reshape(5, 2, 16), "bf16")
+    codes = o["v_cache"][pos]
+    big = np.abs(v) / 1e-4 > 464                       # beyond the last rounding boundary of 448
+    assert big.any()
+    assert (codes[big & (v > 0)] == 0x7E).all() and (codes[big & (v < 0)] == 0xFE).all()
+
+
+def test_prepq_bad_positions_skip_rows():
+    qkv, qw, kw, cos, sin, pos = _qkv_inputs()
+    pos = pos.copy()
+    pos[1] = -1
+    pos[3] = 64                                         # == max_pos
+    o = oracle.qkv_norm_rope_prepq_kvcache(qkv, qw, kw, cos, sin, pos, 4, 2, 16, 80, 1e-6, "bf16", kv="e4m3",
+                                           k_scale=0.01, v_scale=0.01, q_layout="head")
+    assert o["status"] & 1
+    assert np.isnan(o["q_out"][:, [1, 3]]).all() and np.isfinite(o["q_out"][:, [0, 2, 4]]).all()
+    assert (o["k_cache"][64] == 0x7E).all()
