@@ -415,6 +415,44 @@ def next_ops_leg(peak, floor, reps=50, big_m=65536):
             node = statistics.median(ts)
             out[key] = {"graph_node_us": round(node, 3), "x_graph_floor": round(node / floor["graph_node_us"], 3)}
         del x, r, gate, sc, sh, q, bs
+    # NEXT-2: the QKV op with the Q epilogue (softmax scale, head-major Q) and
+    # an e4m3 KV cache, on the large-M QKV shape (32 q / 8 kv heads of 128).
+    wl = W.get("large_m_M65536", M=big_m)
+    g = W.generator(62, "cuda")
+    H, hd = wl.Hq + 2 * wl.Hkv, wl.hd
+    qkv = W.normal16((big_m, H * hd), "bf16", g)
+    qw, kw = W.norm_weight(hd, "bf16", g), W.norm_weight(hd, "bf16", g)
+    cos, sin = W.rope_tables(wl.capacity, hd, wl.theta)
+    cos, sin = cos.cuda(), sin.cuda()
+    pos = W.positions(wl, g)
+    q_out = torch.empty((wl.Hq, big_m, hd), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((wl.capacity, wl.Hkv, hd), dtype=torch.uint8, device="cuda")
+    vc = torch.zeros_like(kc)
+    kvs = torch.tensor([0.02, 0.015], dtype=torch.float32, device="cuda")
+    qs = float(1.0 / np.sqrt(hd))
+
+    def qop():
+        frt.frt_qkv_norm_rope_prepq_kvcache(qkv, qw, kw, cos, sin, pos, q_out, kc, vc, wl.Hq, wl.Hkv, hd,
+                                            q_scale=qs, q_layout="head", kv="e4m3", kv_scales=kvs, eps=wl.eps)
+    nbytes = big_m * (H * hd * 2 + wl.Hq * hd * 2 + 2 * wl.Hkv * hd + hd * 4 + 4) + 2 * hd * 2
+    for _ in range(5):
+        qop()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+    for i in range(reps):
+        ev[2 * i].record(s)
+        qop()
+        ev[2 * i + 1].record(s)
+    torch.cuda.synchronize()
+    ts = [ev[2 * i].elapsed_time(ev[2 * i + 1]) * 1e3 for i in range(reps)]
+    us = sum(ts) / len(ts)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    key = "qkv_prepq_e4m3_M%d" % big_m
+    out[key] = {"us_mean": round(us, 2), "us_median": round(statistics.median(ts), 2), "bytes": nbytes,
+                "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4), "q_layout": "head-major", "kv": "e4m3",
+                "traffic": measured_traffic(key, "qkv_prepq")}
+    del qkv, q_out, kc, vc
     return out
 
 

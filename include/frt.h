@@ -76,6 +76,17 @@ typedef enum { FRT_QUANT_STATIC = 0, FRT_QUANT_BLOCK128 = 1 } frt_quant;
  *             ("Falcon-Perception inference optimisation", third technique). */
 typedef enum { FRT_ACT_GELU_TANH = 0, FRT_ACT_SILU = 1, FRT_ACT_RELU2 = 2 } frt_act;
 
+/* Q staging layout of the QKV op with the Q epilogue (NEXT-2):
+ *  TOKEN_MAJOR  q_out[M, Hq, hd]  (op (b)'s layout)
+ *  HEAD_MAJOR   q_out[Hq, M, hd]  (one contiguous [M, hd] slab per head) */
+typedef enum { FRT_Q_TOKEN_MAJOR = 0, FRT_Q_HEAD_MAJOR = 1 } frt_q_layout;
+
+/* KV-cache element format of the QKV op with the Q epilogue (NEXT-2):
+ *  16BIT  the op's 16-bit type (op (b))
+ *  E4M3   FP8 e4m3 codes, one static dequantisation scale per tensor:
+ *         code = e4m3(k / k_scale), e4m3(v / v_scale) */
+typedef enum { FRT_KV_16BIT = 0, FRT_KV_E4M3 = 1 } frt_kv_format;
+
 /*
  * (a) Residual add + RMSNorm + FP8 quantisation.
  * "FlashRT kernel fusion", §二 steps 1 and 7 (residual_add_rms_norm_fp8_noweight)
@@ -175,6 +186,41 @@ frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_norm_w, cons
 frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* static_scale,
                             float* block_scales, int M, int I, frt_act act, frt_dtype dt, frt_quant qm,
                             cudaStream_t stream);
+
+/*
+ * NEXT-2: op (b) with the attention's Q preparation and an optional FP8 KV
+ * cache.  The "5060 Ti" FlashRT port's optimisation log, step 10: FA2's
+ * prepare_q folded into the RoPE kernel (removing 320 launches); "FlashRT
+ * kernel fusion", §2.2 for the rest of the op.  The pages name the fusion
+ * only; the reading: prepare_q multiplies Q by the attention's softmax scale
+ * and may lay Q out head-major, and the KV cache may hold e4m3 codes with a
+ * static scale per tensor.
+ *
+ * Everything as frt_qkv_norm_rope_kvcache, except:
+ *   q_out[i, h, :] (token-major) or q_out[h, i, :] (head-major)
+ *          = o * q_scale, the product in fp32, rounded once to 16 bits;
+ *   kv_format E4M3:
+ *     k_cache[p, g, :] = e4m3(o / k_scale)  (uint8; o the K head after norm
+ *                                           and RoPE, in fp32),
+ *     v_cache[p, g, :] = e4m3(v / v_scale)  (uint8),
+ *     each quotient correctly rounded in fp32, RNE, saturating to +-448.
+ *
+ *   q_scale      host fp32, finite (1 = no scaling).
+ *   q_layout     FRT_Q_TOKEN_MAJOR or FRT_Q_HEAD_MAJOR.
+ *   kv_format    FRT_KV_16BIT (caches as op (b)) or FRT_KV_E4M3 (caches
+ *                [capacity, Hkv, hd] uint8, 8-byte aligned when hd % 16 == 0,
+ *                4-byte aligned otherwise).
+ *   kv_scales    device fp32[2] = {k_scale, v_scale}, read with E4M3 only
+ *                (may be NULL with 16BIT).
+ *   Errors: as op (b); also FRT_ERR_INVALID_ARG for an unknown layout or
+ *   format, a non-finite q_scale, or E4M3 without kv_scales.
+ */
+frt_status frt_qkv_norm_rope_prepq_kvcache(const void* qkv, const void* q_norm_w, const void* k_norm_w,
+                                           const float* cos_tab, const float* sin_tab, const int32_t* positions,
+                                           void* q_out, void* k_cache, void* v_cache, int32_t* status, int M,
+                                           int Hq, int Hkv, int hd, int max_pos, int capacity, float eps,
+                                           float q_scale, frt_q_layout q_layout, frt_kv_format kv_format,
+                                           const float* kv_scales, frt_dtype dt, cudaStream_t stream);
 
 /*
  * NEXT-1: gated residual + AdaRMSNorm modulation + FP8 quantisation.

@@ -9,6 +9,8 @@ Functions carry the C names of ``include/frt.h``:
     frt_residual_rmsnorm_fp8(x, residual_in, residual_out, weight, out_fp8, ...)
     frt_qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos, sin, positions, ...)
     frt_gate_act_fp8(gate_up, out_fp8, ...)
+    frt_qkv_norm_rope_prepq_kvcache(...)   (NEXT-2)
+    frt_gate_residual_adarms_fp8(...)      (NEXT-1)
     frt_noop(grid, block)
 """
 import ctypes
@@ -26,7 +28,8 @@ ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
 
 # C entry points declared in include/frt.h
 EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8",
-           "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_status_string")
+           "frt_qkv_norm_rope_prepq_kvcache", "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl",
+           "frt_get_pdl", "frt_status_string")
 
 
 class FrtError(RuntimeError):
@@ -52,6 +55,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_residual_rmsnorm_fp8.restype = i32
     L.frt_qkv_norm_rope_kvcache.argtypes = [vp] * 10 + [i32] * 6 + [f32, i32, vp]
     L.frt_qkv_norm_rope_kvcache.restype = i32
+    L.frt_qkv_norm_rope_prepq_kvcache.argtypes = [vp] * 10 + [i32] * 6 + [f32, f32, i32, i32, vp, i32, vp]
+    L.frt_qkv_norm_rope_prepq_kvcache.restype = i32
     L.frt_gate_act_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     L.frt_gate_act_fp8.restype = i32
     L.frt_gate_residual_adarms_fp8.argtypes = [vp] * 9 + [i32, i32, i32, f32, i32, i32, vp]
@@ -118,6 +123,26 @@ def frt_qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positio
         _ptr(k_cache), _ptr(v_cache), _ptr(status), M, Hq, Hkv, hd, max_pos, capacity, float(eps),
         DTYPE[qkv.dtype], _stream(stream))
     _check("frt_qkv_norm_rope_kvcache", st)
+
+
+Q_LAYOUT = {"token": 0, "head": 1}
+KV_FORMAT = {"16": 0, "e4m3": 1}
+
+
+def frt_qkv_norm_rope_prepq_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache,
+                                    Hq, Hkv, hd, q_scale=1.0, q_layout="token", kv="16", kv_scales=None,
+                                    status=None, eps=1e-6, stream=None):
+    """NEXT-2: op (b) + Q softmax-scale pre-multiply / head-major Q layout
+    (q_out [Hq, M, hd]) + optional e4m3 KV cache (uint8 caches; kv_scales
+    fp32[2] = (k_scale, v_scale) on the device)."""
+    M = qkv.shape[0]
+    max_pos = cos_tab.shape[0]
+    capacity = k_cache.shape[0]
+    st = load().frt_qkv_norm_rope_prepq_kvcache(
+        _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(cos_tab), _ptr(sin_tab), _ptr(positions), _ptr(q_out),
+        _ptr(k_cache), _ptr(v_cache), _ptr(status), M, Hq, Hkv, hd, max_pos, capacity, float(eps), float(q_scale),
+        Q_LAYOUT[q_layout], KV_FORMAT[kv], _ptr(kv_scales), DTYPE[qkv.dtype], _stream(stream))
+    _check("frt_qkv_norm_rope_prepq_kvcache", st)
 
 
 def frt_gate_act_fp8(gate_up, out_fp8, static_scale=None, block_scales=None, act="gelu_tanh", quant="static",

@@ -72,19 +72,53 @@ __device__ __forceinline__ void ld_f32(const float* p, float* f) {
   }
 }
 
+// Epilogue of the op (NEXT-2, the attention's Q preparation folded in): Q is
+// multiplied by q_scale in fp32 before its one rounding and written
+// token-major [M, Hq, hd] or head-major [Hq, M, hd]; with KV8 the K and V
+// cache rows are e4m3 codes of k / k_scale and v / v_scale (kv_scales[0..1],
+// device), the quotient correctly rounded in fp32.
+struct Epilogue {
+  float q_scale;
+  int q_head_major;
+  int M;
+  const float* kv_scales;
+};
+
+__device__ __forceinline__ int64_t q_row(const Epilogue& ep, int tok, int h, int Hq) {
+  return ep.q_head_major ? (int64_t)h * ep.M + tok : (int64_t)tok * Hq + h;
+}
+
+// P fp32 values -> P e4m3 codes of v / s stored at dst (P bytes, P-aligned).
+template <int P>
+__device__ __forceinline__ void store_codes(uint8_t* dst, const float* v, const Divisor& dv) {
+  if (P == 8)
+    *reinterpret_cast<uint2*>(dst) = quant8(v, dv);
+  else
+    *reinterpret_cast<uint32_t*>(dst) = quant4(v, dv);
+}
+
 // Register kernel (small batches, or pointers below 16-byte alignment).  One
 // CTA per (token, block of heads).  The CTA's NG lane groups take up to HPG
 // heads each: slot i of group g is head (hb * hpg + i) * NG + g, so for every
 // slot consecutive groups read consecutive heads.  All slots' loads are issued
 // first and a lane's cos/sin slice is loaded once for all its heads.
-template <int DT, int P, int GP, int HPG>
-__global__ void __launch_bounds__(HPG == 1 ? 1024 : 256) qkv_norm_rope_kvcache_kernel(
+// Threads per CTA of the register kernel: up to 1024 with one head per lane
+// group, 512 when the e4m3 epilogue needs the registers, 256 with four heads.
+template <int HPG, int EPI>
+constexpr int reg_kernel_threads() {
+  return HPG == 1 ? (EPI == 2 ? 512 : 1024) : 256;
+}
+
+template <int DT, int P, int GP, int HPG, int EPI>
+__global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_kvcache_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
     const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
-    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, uint16_t* __restrict__ k_cache,
-    uint16_t* __restrict__ v_cache, int32_t* status, int H, int NG, int hpg, int nhb, int Hq, int Hkv, int hd,
-    int G, int max_pos, int capacity, float eps) {
+    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, void* __restrict__ k_cache,
+    void* __restrict__ v_cache, int32_t* status, int H, int NG, int hpg, int nhb, int Hq, int Hkv, int hd,
+    int G, int max_pos, int capacity, float eps, Epilogue ep) {
   using V = typename Vec16<P>::T;
+  constexpr bool QEPI = EPI >= 1;
+  constexpr bool KV8 = EPI == 2;
   pdl_enter();
   const int tok = blockIdx.x / nhb;
   const int hb = blockIdx.x - tok * nhb;
@@ -125,6 +159,8 @@ __global__ void __launch_bounds__(HPG == 1 ? 1024 : 256) qkv_norm_rope_kvcache_k
     ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
     ld_f32<P>(sin_tab + (int64_t)p * half + j0, s);
   }
+  const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
+  const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
 #pragma unroll
   for (int i = 0; i < HPG; ++i) {
     if (i >= hpg) break;  // uniform across the CTA
@@ -134,10 +170,21 @@ __global__ void __launch_bounds__(HPG == 1 ? 1024 : 256) qkv_norm_rope_kvcache_k
     const bool is_v = h >= Hq + Hkv;
     const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
     const bool do_norm = !is_v && nw != nullptr;
-    if (on && is_v) {  // V: bit copy into the cache slot
-      uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
-      *reinterpret_cast<V*>(dst + j0) = va[i];
-      *reinterpret_cast<V*>(dst + half + j0) = vb[i];
+    if (on && is_v) {  // V: bit copy into the cache slot (or its e4m3 codes)
+      const int64_t off = ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
+      if (KV8) {
+        float a[P], b[P];
+        unpack<DT, P>(va[i], a);
+        unpack<DT, P>(vb[i], b);
+        uint8_t* dst = static_cast<uint8_t*>(v_cache) + off;
+        const Divisor dvs(v_scale);
+        store_codes<P>(dst + j0, a, dvs);
+        store_codes<P>(dst + half + j0, b, dvs);
+      } else {
+        uint16_t* dst = static_cast<uint16_t*>(v_cache) + off;
+        *reinterpret_cast<V*>(dst + j0) = va[i];
+        *reinterpret_cast<V*>(dst + half + j0) = vb[i];
+      }
     }
     float a[P], b[P];
     float ss = 0.0f;
@@ -173,9 +220,30 @@ __global__ void __launch_bounds__(HPG == 1 ? 1024 : 256) qkv_norm_rope_kvcache_k
         o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
         o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
       }
-      uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + (h - Hq)) * hd;
-      store_packed<DT, P>(dst + j0, o1);
-      store_packed<DT, P>(dst + half + j0, o2);
+      if (is_q) {
+        if (QEPI) {
+#pragma unroll
+          for (int e = 0; e < P; ++e) {
+            o1[e] *= ep.q_scale;
+            o2[e] *= ep.q_scale;
+          }
+        }
+        uint16_t* dst = q_out + (QEPI ? q_row(ep, tok, h, Hq) : (int64_t)tok * Hq + h) * hd;
+        store_packed<DT, P>(dst + j0, o1);
+        store_packed<DT, P>(dst + half + j0, o2);
+      } else {
+        const int64_t off = ((int64_t)p * Hkv + (h - Hq)) * hd;
+        if (KV8) {
+          uint8_t* dst = static_cast<uint8_t*>(k_cache) + off;
+          const Divisor dk(k_scale);
+          store_codes<P>(dst + j0, o1, dk);
+          store_codes<P>(dst + half + j0, o2, dk);
+        } else {
+          uint16_t* dst = static_cast<uint16_t*>(k_cache) + off;
+          store_packed<DT, P>(dst + j0, o1);
+          store_packed<DT, P>(dst + half + j0, o2);
+        }
+      }
     }
   }
 }
@@ -192,16 +260,29 @@ constexpr int kMaxPolls = 1 << 22;
 // then the Q row, the K row and the untouched V row leave as three bulk
 // stores.  A barrier wait that runs out of polls sets bit 1 of *status and the
 // CTA returns without writing.
-template <int DT, int P, int GP>
-__global__ void __launch_bounds__(256) qkv_norm_rope_kvcache_tma_kernel(
+// EPI: 0 = op (b) as is (Q token-major, unscaled; 16-bit caches), 1 = Q
+// epilogue (scale, layout), 2 = Q epilogue + e4m3 caches.  At most 128
+// threads; the register budget keeps 10 CTAs (tokens) resident per SM (8 for
+// the 16-bit Q epilogue, which would spill at 10): the kernel waits on memory,
+// so resident tokens, not instruction count, set its rate.
+template <int EPI>
+constexpr int tma_min_blocks() {
+  return EPI == 1 ? 8 : 10;
+}
+
+template <int DT, int P, int GP, int EPI>
+__global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvcache_tma_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
     const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
-    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, uint16_t* __restrict__ k_cache,
-    uint16_t* __restrict__ v_cache, int32_t* status, int H, int NG, int Hq, int Hkv, int hd, int G, int max_pos,
-    int capacity, float eps) {
+    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, void* __restrict__ k_cache,
+    void* __restrict__ v_cache, int32_t* status, int H, int NG, int Hq, int Hkv, int hd, int G, int max_pos,
+    int capacity, float eps, Epilogue ep) {
   using V = typename Vec16<P>::T;
+  constexpr bool QEPI = EPI >= 1;
+  constexpr bool KV8 = EPI == 2;
   pdl_enter();
-  extern __shared__ __align__(128) uint8_t dsmem[];  // [QKV row][cos][sin][q weight][k weight]
+  // [QKV row][cos][sin][q weight][k weight] (+ [K codes][V codes] with KV8)
+  extern __shared__ __align__(128) uint8_t dsmem[];
   __shared__ uint64_t bar;
   __shared__ int s_pos;
   const int tok = blockIdx.x;
@@ -215,6 +296,8 @@ __global__ void __launch_bounds__(256) qkv_norm_rope_kvcache_tma_kernel(
   float* sbuf = cbuf + half;
   uint16_t* qwbuf = reinterpret_cast<uint16_t*>(sbuf + half);
   uint16_t* kwbuf = qwbuf + hd;
+  uint8_t* k8buf = reinterpret_cast<uint8_t*>(kwbuf + hd);
+  uint8_t* v8buf = k8buf + Hkv * hd;
 
   if (tid == 0) {
     mbar_init(&bar, 2);  // two arrivals: the row (+ weights), then the table rows
@@ -260,12 +343,18 @@ __global__ void __launch_bounds__(256) qkv_norm_rope_kvcache_tma_kernel(
       s[e] = sbuf[j0 + e];
     }
   }
-  const int nslots = (Hq + Hkv + NG - 1) / NG;  // Q and K heads only; V leaves untouched
+  const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
+  const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
+  const bool q_direct = QEPI && ep.q_head_major;  // head-major Q leaves from registers
+  // Q and K heads; V heads too with KV8 (their codes), else V leaves untouched.
+  const int nheads = KV8 ? H : Hq + Hkv;
+  const int nslots = (nheads + NG - 1) / NG;
   for (int i = 0; i < nslots; ++i) {
     const int h = i * NG + grp;
-    const bool on = lane_ok && h < Hq + Hkv;
+    const bool on = lane_ok && h < nheads;
     const bool is_q = h < Hq;
-    const uint16_t* nwg = is_q ? q_norm_w : k_norm_w;
+    const bool is_v = h >= Hq + Hkv;
+    const uint16_t* nwg = is_v ? nullptr : is_q ? q_norm_w : k_norm_w;
     const uint16_t* nws = is_q ? qwbuf : kwbuf;
     uint16_t* vec = rowbuf + h * hd;
     float a[P], b[P];
@@ -279,7 +368,12 @@ __global__ void __launch_bounds__(256) qkv_norm_rope_kvcache_tma_kernel(
       }
     }
     ss = group_sum<GP>(ss);  // every lane of the warp takes part
-    if (on) {
+    if (on && KV8 && is_v) {
+      uint8_t* dst = v8buf + (h - Hq - Hkv) * hd;
+      const Divisor dvs(v_scale);
+      store_codes<P>(dst + j0, a, dvs);
+      store_codes<P>(dst + half + j0, b, dvs);
+    } else if (on) {
       if (nwg != nullptr) {
         const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
         float fa[P], fb[P];
@@ -297,16 +391,43 @@ __global__ void __launch_bounds__(256) qkv_norm_rope_kvcache_tma_kernel(
         o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
         o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
       }
-      store_packed<DT, P>(vec + j0, o1);
-      store_packed<DT, P>(vec + half + j0, o2);
+      if (QEPI && is_q) {
+#pragma unroll
+        for (int e = 0; e < P; ++e) {
+          o1[e] *= ep.q_scale;
+          o2[e] *= ep.q_scale;
+        }
+      }
+      if (KV8 && !is_q) {
+        uint8_t* dst = k8buf + (h - Hq) * hd;
+        const Divisor dk(k_scale);
+        store_codes<P>(dst + j0, o1, dk);
+        store_codes<P>(dst + half + j0, o2, dk);
+      } else if (q_direct && is_q) {
+        uint16_t* dst = q_out + ((int64_t)h * ep.M + tok) * hd;
+        store_packed<DT, P>(dst + j0, o1);
+        store_packed<DT, P>(dst + half + j0, o2);
+      } else {
+        store_packed<DT, P>(vec + j0, o1);
+        store_packed<DT, P>(vec + half + j0, o2);
+      }
     }
   }
   fence_proxy_async_smem();  // this thread's writes -> the bulk stores below
   __syncthreads();
+  // Token-major Q leaves as one bulk store with the K and V rows (head-major
+  // Q went straight from registers above).
   if (tid == 0) {
-    bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
-    bulk_store(k_cache + (int64_t)p * Hkv * hd, rowbuf + Hq * hd, (unsigned)(Hkv * hd * 2));
-    bulk_store(v_cache + (int64_t)p * Hkv * hd, rowbuf + (Hq + Hkv) * hd, (unsigned)(Hkv * hd * 2));
+    if (!q_direct) bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
+    if (KV8) {
+      bulk_store(static_cast<uint8_t*>(k_cache) + (int64_t)p * Hkv * hd, k8buf, (unsigned)(Hkv * hd));
+      bulk_store(static_cast<uint8_t*>(v_cache) + (int64_t)p * Hkv * hd, v8buf, (unsigned)(Hkv * hd));
+    } else {
+      bulk_store(static_cast<uint16_t*>(k_cache) + (int64_t)p * Hkv * hd, rowbuf + Hq * hd,
+                 (unsigned)(Hkv * hd * 2));
+      bulk_store(static_cast<uint16_t*>(v_cache) + (int64_t)p * Hkv * hd, rowbuf + (Hq + Hkv) * hd,
+                 (unsigned)(Hkv * hd * 2));
+    }
     bulk_commit();
     bulk_wait_read();  // shared memory must outlive the stores' reads
   }
@@ -325,6 +446,7 @@ struct Args {
   int32_t* status;
   int M, H, Hq, Hkv, hd, G, max_pos, capacity;
   float eps;
+  Epilogue ep;
 };
 
 // CTA shape for GP lanes per head.  Small batches (launch/latency-bound):
@@ -335,16 +457,17 @@ struct Shape {
   int NG, hpg, nhb, threads;
 };
 
-inline Shape qkv_shape(int M, int H, int GP) {
+inline Shape qkv_shape(int M, int H, int GP, bool kv8) {
   Shape sh;
   const bool large = M >= 4 * 148;
+  const int max_threads = kv8 ? 512 : 1024;
   if (large && H >= 2) {
     sh.NG = (H + 3) / 4;
     if (sh.NG * GP > 256) sh.NG = 256 / GP;
     sh.hpg = (H + sh.NG - 1) / sh.NG;
     if (sh.hpg > 4) sh.hpg = 4;
   } else {
-    sh.NG = H * GP <= 1024 ? H : 1024 / GP;
+    sh.NG = H * GP <= max_threads ? H : max_threads / GP;
     sh.hpg = 1;
   }
   sh.nhb = (H + sh.NG * sh.hpg - 1) / (sh.NG * sh.hpg);
@@ -353,57 +476,111 @@ inline Shape qkv_shape(int M, int H, int GP) {
 }
 
 // Shared memory of the bulk-copy kernel: the QKV row, cos and sin rows, two
-// norm weights.
-inline size_t tma_smem(int H, int hd) { return (size_t)H * hd * 2 + (size_t)hd * 4 + (size_t)hd * 4; }
+// norm weights, and with an e4m3 cache the K and V code rows.
+inline size_t tma_smem(int H, int Hkv, int hd, bool kv8) {
+  return (size_t)H * hd * 2 + (size_t)hd * 4 + (size_t)hd * 4 + (kv8 ? (size_t)2 * Hkv * hd : 0);
+}
 constexpr size_t kTmaSmemMax = 200 * 1024;
 
-template <int DT, int P, int GP>
+template <int DT, int P, int GP, int EPI>
 frt_status launch_gp(const Args& a, bool tma, cudaStream_t st) {
+  constexpr bool KV8 = EPI == 2;
   const uint16_t* qkv = static_cast<const uint16_t*>(a.qkv);
   const uint16_t* qw = static_cast<const uint16_t*>(a.qw);
   const uint16_t* kw = static_cast<const uint16_t*>(a.kw);
   uint16_t* qo = static_cast<uint16_t*>(a.q_out);
-  uint16_t* kc = static_cast<uint16_t*>(a.kc);
-  uint16_t* vc = static_cast<uint16_t*>(a.vc);
   if (tma) {
     static std::atomic<int> opted{0};
-    auto kt = qkv_norm_rope_kvcache_tma_kernel<DT, P, GP>;
-    const size_t smem = tma_smem(a.H, a.hd);
+    auto kt = qkv_norm_rope_kvcache_tma_kernel<DT, P, GP, EPI>;
+    const size_t smem = tma_smem(a.H, a.Hkv, a.hd, KV8);
     const frt_status os = opt_in_smem(kt, smem, opted);
     if (os != FRT_OK) return os;
-    const int per = a.Hq + a.Hkv;  // lane groups needed for one slot of every Q/K head
+    const int per = KV8 ? a.H : a.Hq + a.Hkv;  // lane groups needed for one slot of every processed head
     int NG = (per * GP <= 128) ? per : 128 / GP;
     if (NG < 1) NG = 1;
     const int threads = ((NG * GP + 31) / 32) * 32;
     return launch(kt, dim3((unsigned)a.M), dim3(threads), smem, st, qkv, qw, kw, a.cos_tab, a.sin_tab, a.pos, qo,
-                  kc, vc, a.status, a.H, NG, a.Hq, a.Hkv, a.hd, a.G, a.max_pos, a.capacity, a.eps);
+                  a.kc, a.vc, a.status, a.H, NG, a.Hq, a.Hkv, a.hd, a.G, a.max_pos, a.capacity, a.eps, a.ep);
   }
-  const Shape sh = qkv_shape(a.M, a.H, GP);
+  const Shape sh = qkv_shape(a.M, a.H, GP, KV8);
   const dim3 grid((unsigned)((int64_t)a.M * sh.nhb));
   if (sh.hpg == 1)
-    return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP, 1>, grid, dim3(sh.threads), 0, st, qkv, qw, kw,
-                  a.cos_tab, a.sin_tab, a.pos, qo, kc, vc, a.status, a.H, sh.NG, sh.hpg, sh.nhb, a.Hq, a.Hkv, a.hd,
-                  a.G, a.max_pos, a.capacity, a.eps);
-  return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP, 4>, grid, dim3(sh.threads), 0, st, qkv, qw, kw, a.cos_tab,
-                a.sin_tab, a.pos, qo, kc, vc, a.status, a.H, sh.NG, sh.hpg, sh.nhb, a.Hq, a.Hkv, a.hd, a.G,
-                a.max_pos, a.capacity, a.eps);
+    return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP, 1, EPI>, grid, dim3(sh.threads), 0, st, qkv, qw, kw,
+                  a.cos_tab, a.sin_tab, a.pos, qo, a.kc, a.vc, a.status, a.H, sh.NG, sh.hpg, sh.nhb, a.Hq, a.Hkv,
+                  a.hd, a.G, a.max_pos, a.capacity, a.eps, a.ep);
+  return launch(qkv_norm_rope_kvcache_kernel<DT, P, GP, 4, EPI>, grid, dim3(sh.threads), 0, st, qkv, qw, kw,
+                a.cos_tab, a.sin_tab, a.pos, qo, a.kc, a.vc, a.status, a.H, sh.NG, sh.hpg, sh.nhb, a.Hq, a.Hkv, a.hd,
+                a.G, a.max_pos, a.capacity, a.eps, a.ep);
+}
+
+template <int DT, int P, int GP>
+frt_status launch_kv(int epi, const Args& a, bool tma, cudaStream_t st) {
+  switch (epi) {
+    case 0: return launch_gp<DT, P, GP, 0>(a, tma, st);
+    case 1: return launch_gp<DT, P, GP, 1>(a, tma, st);
+    default: return launch_gp<DT, P, GP, 2>(a, tma, st);
+  }
 }
 
 template <int DT, int P>
-frt_status launch_p(int GP, const Args& a, bool tma, cudaStream_t st) {
+frt_status launch_p(int GP, int epi, const Args& a, bool tma, cudaStream_t st) {
   switch (GP) {
-    case 1: return launch_gp<DT, P, 1>(a, tma, st);
-    case 2: return launch_gp<DT, P, 2>(a, tma, st);
-    case 4: return launch_gp<DT, P, 4>(a, tma, st);
-    case 8: return launch_gp<DT, P, 8>(a, tma, st);
-    case 16: return launch_gp<DT, P, 16>(a, tma, st);
-    default: return launch_gp<DT, P, 32>(a, tma, st);
+    case 1: return launch_kv<DT, P, 1>(epi, a, tma, st);
+    case 2: return launch_kv<DT, P, 2>(epi, a, tma, st);
+    case 4: return launch_kv<DT, P, 4>(epi, a, tma, st);
+    case 8: return launch_kv<DT, P, 8>(epi, a, tma, st);
+    case 16: return launch_kv<DT, P, 16>(epi, a, tma, st);
+    default: return launch_kv<DT, P, 32>(epi, a, tma, st);
   }
 }
 
 template <int DT>
-frt_status launch_dt(int P, int GP, const Args& a, bool tma, cudaStream_t st) {
-  return P == 8 ? launch_p<DT, 8>(GP, a, tma, st) : launch_p<DT, 4>(GP, a, tma, st);
+frt_status launch_dt(int P, int GP, int epi, const Args& a, bool tma, cudaStream_t st) {
+  return P == 8 ? launch_p<DT, 8>(GP, epi, a, tma, st) : launch_p<DT, 4>(GP, epi, a, tma, st);
+}
+
+// Shared validation and dispatch of both entry points.
+frt_status qkv_op(const void* qkv, const void* q_norm_w, const void* k_norm_w, const float* cos_tab,
+                  const float* sin_tab, const int32_t* positions, void* q_out, void* k_cache, void* v_cache,
+                  int32_t* status, int M, int Hq, int Hkv, int hd, int max_pos, int capacity, float eps,
+                  float q_scale, frt_q_layout q_layout, frt_kv_format kv_format, const float* kv_scales,
+                  frt_dtype dt, cudaStream_t stream) {
+  if (M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || hd <= 0 || hd % 2 != 0) return FRT_ERR_INVALID_ARG;
+  if (max_pos <= 0 || capacity <= 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
+  if (q_layout != FRT_Q_TOKEN_MAJOR && q_layout != FRT_Q_HEAD_MAJOR) return FRT_ERR_INVALID_ARG;
+  if (kv_format != FRT_KV_16BIT && kv_format != FRT_KV_E4M3) return FRT_ERR_INVALID_ARG;
+  if (!std::isfinite(q_scale)) return FRT_ERR_INVALID_ARG;
+  if (hd % 8 != 0 || hd > 256) return FRT_ERR_UNSUPPORTED;
+  if (M == 0) return FRT_OK;
+  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
+  const bool kv8 = kv_format == FRT_KV_E4M3;
+  if (kv8 && (!kv_scales || !aligned(kv_scales, 4))) return FRT_ERR_INVALID_ARG;
+  const int P = (hd % 16 == 0) ? 8 : 4;
+  const uintptr_t al = (P == 8) ? 16 : 8;
+  const uintptr_t al_kv = kv8 ? (uintptr_t)P : al;  // e4m3 rows: P codes per lane store
+  if (!aligned(qkv, al) || !aligned(q_out, al) || !aligned(k_cache, al_kv) || !aligned(v_cache, al_kv))
+    return FRT_ERR_INVALID_ARG;
+  if ((q_norm_w && !aligned(q_norm_w, al)) || (k_norm_w && !aligned(k_norm_w, al))) return FRT_ERR_INVALID_ARG;
+  if (!aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(positions, 4)) return FRT_ERR_INVALID_ARG;
+  if (status && !aligned(status, 4)) return FRT_ERR_INVALID_ARG;
+  const int H = Hq + 2 * Hkv;
+  const int G = (hd / 2) / P;  // active lanes per head, <= 31
+  int GP = 1;
+  while (GP < G) GP *= 2;
+  Args a{qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status,
+         M, H, Hq, Hkv, hd, G, max_pos, capacity, eps,
+         Epilogue{q_scale, q_layout == FRT_Q_HEAD_MAJOR ? 1 : 0, M, kv_scales}};
+  if ((int64_t)M * qkv_shape(M, H, GP, kv8).nhb > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
+  // Bulk-copy path for large batches when every row it moves is 16-byte
+  // aligned (bulk copies need 16-byte addresses and sizes) and fits in
+  // shared memory; the register kernel otherwise.
+  const bool tma = M >= 4 * 148 && aligned(qkv, 16) && aligned(q_out, 16) && aligned(k_cache, 16) &&
+                   aligned(v_cache, 16) && (!q_norm_w || aligned(q_norm_w, 16)) &&
+                   (!k_norm_w || aligned(k_norm_w, 16)) && (!kv8 || (Hkv * hd) % 16 == 0) &&
+                   tma_smem(H, Hkv, hd, kv8) <= kTmaSmemMax;
+  const int epi = kv8 ? 2 : (q_scale != 1.0f || q_layout != FRT_Q_TOKEN_MAJOR) ? 1 : 0;
+  return dt == FRT_F16 ? launch_dt<FRT_F16>(P, GP, epi, a, tma, stream)
+                       : launch_dt<FRT_BF16>(P, GP, epi, a, tma, stream);
 }
 
 }  // namespace
@@ -415,31 +592,17 @@ extern "C" frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_n
                                                 void* v_cache, int32_t* status, int M, int Hq, int Hkv, int hd,
                                                 int max_pos, int capacity, float eps, frt_dtype dt,
                                                 cudaStream_t stream) {
-  using namespace frt;
-  if (M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || hd <= 0 || hd % 2 != 0) return FRT_ERR_INVALID_ARG;
-  if (max_pos <= 0 || capacity <= 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
-  if (hd % 8 != 0 || hd > 256) return FRT_ERR_UNSUPPORTED;
-  if (M == 0) return FRT_OK;
-  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
-  const int P = (hd % 16 == 0) ? 8 : 4;
-  const uintptr_t al = (P == 8) ? 16 : 8;
-  if (!aligned(qkv, al) || !aligned(q_out, al) || !aligned(k_cache, al) || !aligned(v_cache, al))
-    return FRT_ERR_INVALID_ARG;
-  if ((q_norm_w && !aligned(q_norm_w, al)) || (k_norm_w && !aligned(k_norm_w, al))) return FRT_ERR_INVALID_ARG;
-  if (!aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(positions, 4)) return FRT_ERR_INVALID_ARG;
-  if (status && !aligned(status, 4)) return FRT_ERR_INVALID_ARG;
-  const int H = Hq + 2 * Hkv;
-  const int G = (hd / 2) / P;  // active lanes per head, <= 31
-  int GP = 1;
-  while (GP < G) GP *= 2;
-  Args a{qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status,
-         M, H, Hq, Hkv, hd, G, max_pos, capacity, eps};
-  if ((int64_t)M * qkv_shape(M, H, GP).nhb > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
-  // Bulk-copy path for large batches when every row it moves is 16-byte
-  // aligned (bulk copies need 16-byte addresses and sizes) and fits in
-  // shared memory; the register kernel otherwise.
-  const bool tma = M >= 4 * 148 && aligned(qkv, 16) && aligned(q_out, 16) && aligned(k_cache, 16) &&
-                   aligned(v_cache, 16) && (!q_norm_w || aligned(q_norm_w, 16)) &&
-                   (!k_norm_w || aligned(k_norm_w, 16)) && tma_smem(H, hd) <= kTmaSmemMax;
-  return dt == FRT_F16 ? launch_dt<FRT_F16>(P, GP, a, tma, stream) : launch_dt<FRT_BF16>(P, GP, a, tma, stream);
+  return frt::qkv_op(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status, M, Hq,
+                     Hkv, hd, max_pos, capacity, eps, 1.0f, FRT_Q_TOKEN_MAJOR, FRT_KV_16BIT, nullptr, dt, stream);
+}
+
+extern "C" frt_status frt_qkv_norm_rope_prepq_kvcache(const void* qkv, const void* q_norm_w, const void* k_norm_w,
+                                                      const float* cos_tab, const float* sin_tab,
+                                                      const int32_t* positions, void* q_out, void* k_cache,
+                                                      void* v_cache, int32_t* status, int M, int Hq, int Hkv,
+                                                      int hd, int max_pos, int capacity, float eps, float q_scale,
+                                                      frt_q_layout q_layout, frt_kv_format kv_format,
+                                                      const float* kv_scales, frt_dtype dt, cudaStream_t stream) {
+  return frt::qkv_op(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status, M, Hq,
+                     Hkv, hd, max_pos, capacity, eps, q_scale, q_layout, kv_format, kv_scales, dt, stream);
 }

@@ -73,7 +73,7 @@ def lib():
                                                                           c.c_int64, c.c_int64, c.c_int64,
                                                                           c.c_double, c.c_int, c.c_int]
         L.oracle_gate_residual_adarms_fp8.restype = c.c_int
-        L.oracle_qkv_norm_rope_prepq_kvcache.argtypes = ([c.c_void_p] * 12 + [c.c_int64] * 6 +
+        L.oracle_qkv_norm_rope_prepq_kvcache.argtypes = ([c.c_void_p] * 13 + [c.c_int64] * 6 +
                                                          [c.c_double, c.c_int, c.c_double, c.c_int, c.c_int,
                                                           c.c_double, c.c_double])
         L.oracle_qkv_norm_rope_prepq_kvcache.restype = c.c_int
@@ -191,7 +191,7 @@ def qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, 
 
 def qkv_norm_rope_prepq_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, Hq, Hkv, hd, capacity,
                                 eps, dt, q_scale=1.0, q_layout="token", kv="16", k_scale=None, v_scale=None,
-                                k_cache=None, v_cache=None):
+                                k_cache=None, v_cache=None, slots=None):
     """NEXT-2 op.  q_out is fp64 [M, Hq, hd] (q_layout "token") or [Hq, M, hd]
     ("head"); with kv "16" the caches are as op (b) (fp64 K, uint16 V), with
     kv "e4m3" both are uint8 codes (initial contents: the given arrays or
@@ -204,6 +204,7 @@ def qkv_norm_rope_prepq_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, posit
     pos = np.ascontiguousarray(positions, dtype=np.int32)
     qw = None if q_norm_w is None else np.ascontiguousarray(q_norm_w, dtype=np.uint16)
     kw = None if k_norm_w is None else np.ascontiguousarray(k_norm_w, dtype=np.uint16)
+    sl = None if slots is None else np.ascontiguousarray(slots, dtype=np.int64)
     head = {"token": 0, "head": 1}[q_layout]
     fp8 = {"16": 0, "e4m3": 1}[kv]
     q_out = np.full((Hq, M, hd) if head else (M, Hq, hd), np.nan, dtype=np.float64)
@@ -220,7 +221,7 @@ def qkv_norm_rope_prepq_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, posit
               else np.array(v_cache, dtype=np.uint16, copy=True))
     status = np.zeros(1, dtype=np.int32)
     rc = lib().oracle_qkv_norm_rope_prepq_kvcache(
-        _p(qkv), _p(qw), _p(kw), _p(cos_tab), _p(sin_tab), _p(pos), _p(q_out), _p(kc), _p(vc), _p(kc8), _p(vc8),
+        _p(qkv), _p(qw), _p(kw), _p(cos_tab), _p(sin_tab), _p(pos), _p(sl), _p(q_out), _p(kc), _p(vc), _p(kc8), _p(vc8),
         _p(status), M, Hq, Hkv, hd, max_pos, capacity, _f32(eps), _DT[dt], float(q_scale), head, fp8,
         float(k_scale or 0.0), float(v_scale or 0.0))
     if rc != 0:

@@ -456,7 +456,7 @@ int oracle_gate_residual_adarms_fp8(const uint16_t* x, const uint16_t* gate, con
 // and set status bit 0, as op (b).
 int oracle_qkv_norm_rope_prepq_kvcache(const uint16_t* qkv, const uint16_t* q_norm_w, const uint16_t* k_norm_w,
                                        const float* cos_tab, const float* sin_tab, const int32_t* positions,
-                                       double* q_out, double* k_cache, uint16_t* v_cache, uint8_t* k_cache8,
+                                       const int64_t* slots, double* q_out, double* k_cache, uint16_t* v_cache, uint8_t* k_cache8,
                                        uint8_t* v_cache8, int32_t* status, int64_t M, int64_t Hq, int64_t Hkv,
                                        int64_t hd, int64_t max_pos, int64_t capacity, double eps, int dt,
                                        double q_scale, int q_head_major, int kv_fp8, double k_scale,
@@ -475,7 +475,10 @@ int oracle_qkv_norm_rope_prepq_kvcache(const uint16_t* qkv, const uint16_t* q_no
   }
   for (int64_t i = 0; i < M; ++i) {
     const int64_t p = positions[i];
-    if (p < 0 || p >= max_pos || p >= capacity) {
+    // slots (test use only) stores row i's cache rows at slots[i] instead of
+    // at p, so a sample of a large batch can use a compact cache.
+    const int64_t slot = slots ? slots[i] : p;
+    if (p < 0 || p >= max_pos || slot < 0 || slot >= capacity) {
       if (status) *status |= 1;
       continue;
     }
@@ -495,19 +498,19 @@ int oracle_qkv_norm_rope_prepq_kvcache(const uint16_t* qkv, const uint16_t* q_no
         double* dst = q_head_major ? q_out + (h * M + i) * hd : q_out + (i * Hq + h) * hd;
         for (int64_t j = 0; j < hd; ++j) dst[j] = v[j] * q_scale;
       } else if (kv_fp8) {
-        uint8_t* dst = k_cache8 + (p * Hkv + (h - Hq)) * hd;
+        uint8_t* dst = k_cache8 + (slot * Hkv + (h - Hq)) * hd;
         for (int64_t j = 0; j < hd; ++j) dst[j] = quant_fp32(v[j], ks32);
       } else {
-        std::memcpy(k_cache + (p * Hkv + (h - Hq)) * hd, v.data(), sizeof(double) * hd);
+        std::memcpy(k_cache + (slot * Hkv + (h - Hq)) * hd, v.data(), sizeof(double) * hd);
       }
     }
     for (int64_t g = 0; g < Hkv; ++g) {
       const uint16_t* src = row + (Hq + Hkv + g) * hd;
       if (kv_fp8) {
-        uint8_t* dst = v_cache8 + (p * Hkv + g) * hd;
+        uint8_t* dst = v_cache8 + (slot * Hkv + g) * hd;
         for (int64_t j = 0; j < hd; ++j) dst[j] = quant_fp32(decode16(src[j], f), vs32);
       } else {
-        std::memcpy(v_cache + (p * Hkv + g) * hd, src, sizeof(uint16_t) * hd);
+        std::memcpy(v_cache + (slot * Hkv + g) * hd, src, sizeof(uint16_t) * hd);
       }
     }
   }

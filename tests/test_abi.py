@@ -121,3 +121,18 @@ def test_gate_residual_adarms_host_validation(kw, want):
         assert ada_call(M=0, **kw) == OK
     else:
         assert ada_call(**kw) == want
+
+
+def b8_call(M=4, Hq=8, Hkv=2, hd=128, kc=A, vc=A, qs=0.125, layout=1, kv=1, scales=A, dt=1):
+    return frt.load().frt_qkv_norm_rope_prepq_kvcache(A, None, None, A, A, A, A, kc, vc, None, M, Hq, Hkv, hd, 64,
+                                                      64, 1e-6, qs, layout, kv, scales, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(layout=2), INV), (dict(layout=-1), INV), (dict(kv=2), INV), (dict(qs=float("inf")), INV),
+    (dict(qs=float("nan")), INV), (dict(scales=None), INV), (dict(scales=A + 2), INV), (dict(kc=A + 4), INV),
+    (dict(hd=72, vc=A + 2), INV), (dict(kc=None), INV), (dict(hd=12), UNSUP), (dict(M=-1), INV),
+    (dict(M=0), OK), (dict(M=0, scales=None), OK), (dict(M=0, layout=3), INV), (dict(M=0, kv=0, scales=None), OK),
+])
+def test_qkv_prepq_host_validation(kw, want):
+    assert b8_call(**kw) == want
