@@ -248,89 +248,20 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
   }
 }
 
-// Polls of a bulk-copy barrier before the kernel gives up (each poll may
-// suspend the thread for a while; the bound is far beyond any real copy).
-constexpr int kMaxPolls = 1 << 22;
-
-// Bulk-copy kernel (large batches).  One CTA per token.  One thread moves the
-// token's whole QKV row, its cos/sin rows and both norm weights into shared
-// memory with 1-D bulk copies (TMA) completed on an mbarrier, so no register
-// holds in-flight data and a small CTA keeps 12+ KB per token in flight.  Lane
-// groups (GP lanes per head) normalise and rotate the Q and K heads in place;
-// then the Q row, the K row and the untouched V row leave as three bulk
-// stores.  A barrier wait that runs out of polls sets bit 1 of *status and the
-// CTA returns without writing.
-// EPI: 0 = op (b) as is (Q token-major, unscaled; 16-bit caches), 1 = Q
-// epilogue (scale, layout), 2 = Q epilogue + e4m3 caches.  At most 128
-// threads; the register budget keeps 10 CTAs (tokens) resident per SM (8 for
-// the 16-bit Q epilogue, which would spill at 10): the kernel waits on memory,
-// so resident tokens, not instruction count, set its rate.
-template <int EPI>
-constexpr int tma_min_blocks() {
-  return EPI == 1 ? 8 : 10;
-}
-
+// One token's heads, in shared memory, for the bulk-copy kernels: lane groups
+// normalise and rotate the Q and K heads in place (Q scaled, head-major Q
+// straight to global memory; e4m3 codes of K and V into their own rows with
+// EPI 2).  The caller orders these writes before its bulk stores.
 template <int DT, int P, int GP, int EPI>
-__global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvcache_tma_kernel(
-    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
-    const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
-    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, void* __restrict__ k_cache,
-    void* __restrict__ v_cache, int32_t* status, int H, int NG, int Hq, int Hkv, int hd, int G, int max_pos,
-    int capacity, float eps, Epilogue ep) {
+__device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbuf, const float* sbuf,
+                                              const uint16_t* qwbuf, const uint16_t* kwbuf, uint8_t* k8buf,
+                                              uint8_t* v8buf, const uint16_t* q_norm_w, const uint16_t* k_norm_w,
+                                              uint16_t* q_out, int tok, int tid, int H, int NG, int Hq, int Hkv,
+                                              int hd, int G, float eps, const Epilogue& ep) {
   using V = typename Vec16<P>::T;
   constexpr bool QEPI = EPI >= 1;
   constexpr bool KV8 = EPI == 2;
-  pdl_enter();
-  // [QKV row][cos][sin][q weight][k weight] (+ [K codes][V codes] with KV8)
-  extern __shared__ __align__(128) uint8_t dsmem[];
-  __shared__ uint64_t bar;
-  __shared__ int s_pos;
-  const int tok = blockIdx.x;
-  const int tid = threadIdx.x;
   const int half = hd >> 1;
-  const unsigned row_bytes = (unsigned)(H * hd * 2);
-  const unsigned tab_bytes = (unsigned)(half * 4);
-  const unsigned w_bytes = (unsigned)(hd * 2);
-  uint16_t* rowbuf = reinterpret_cast<uint16_t*>(dsmem);
-  float* cbuf = reinterpret_cast<float*>(dsmem + row_bytes);
-  float* sbuf = cbuf + half;
-  uint16_t* qwbuf = reinterpret_cast<uint16_t*>(sbuf + half);
-  uint16_t* kwbuf = qwbuf + hd;
-  uint8_t* k8buf = reinterpret_cast<uint8_t*>(kwbuf + hd);
-  uint8_t* v8buf = k8buf + Hkv * hd;
-
-  if (tid == 0) {
-    mbar_init(&bar, 2);  // two arrivals: the row (+ weights), then the table rows
-    mbar_init_fence();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned first = row_bytes + (q_norm_w ? w_bytes : 0u) + (k_norm_w ? w_bytes : 0u);
-    mbar_arrive_expect_tx(&bar, first);
-    bulk_load(rowbuf, qkv + (int64_t)tok * H * hd, row_bytes, &bar);
-    if (q_norm_w) bulk_load(qwbuf, q_norm_w, w_bytes, &bar);
-    if (k_norm_w) bulk_load(kwbuf, k_norm_w, w_bytes, &bar);
-    const int p = __ldg(positions + tok);
-    const bool ok = p >= 0 && p < max_pos && p < capacity;
-    s_pos = ok ? p : -1;
-    if (ok) {
-      mbar_arrive_expect_tx(&bar, 2 * tab_bytes);
-      bulk_load(cbuf, cos_tab + (int64_t)p * half, tab_bytes, &bar);
-      bulk_load(sbuf, sin_tab + (int64_t)p * half, tab_bytes, &bar);
-    } else {
-      if (status != nullptr) atomicOr(status, 1);
-      mbar_arrive_expect_tx(&bar, 0u);
-    }
-  }
-  const bool landed = mbar_wait_bounded(&bar, 0, kMaxPolls);
-  if (!__syncthreads_and(landed)) {
-    if (tid == 0 && status != nullptr) atomicOr(status, 2);
-    mbar_wait_bounded(&bar, 0, kMaxPolls);  // give copies still in flight a last chance to land
-    return;
-  }
-  const int p = s_pos;
-  if (p < 0) return;  // position out of range: nothing is written
-
   const int grp = tid / GP;
   const int li = tid & (GP - 1);
   const bool lane_ok = grp < NG && li < G;
@@ -413,21 +344,111 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
       }
     }
   }
+}
+
+// One token's outputs leave shared memory as bulk stores (issued by one
+// thread; the caller commits and waits): token-major Q as one row (head-major
+// Q went straight from registers), the K and V cache rows at slot p.
+template <int EPI>
+__device__ __forceinline__ void store_token(const uint16_t* rowbuf, const uint8_t* k8buf, const uint8_t* v8buf,
+                                            uint16_t* q_out, void* k_cache, void* v_cache, int tok, int p, int Hq,
+                                            int Hkv, int hd, const Epilogue& ep) {
+  if (!(EPI >= 1 && ep.q_head_major)) bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
+  if (EPI == 2) {
+    bulk_store(static_cast<uint8_t*>(k_cache) + (int64_t)p * Hkv * hd, k8buf, (unsigned)(Hkv * hd));
+    bulk_store(static_cast<uint8_t*>(v_cache) + (int64_t)p * Hkv * hd, v8buf, (unsigned)(Hkv * hd));
+  } else {
+    bulk_store(static_cast<uint16_t*>(k_cache) + (int64_t)p * Hkv * hd, rowbuf + Hq * hd, (unsigned)(Hkv * hd * 2));
+    bulk_store(static_cast<uint16_t*>(v_cache) + (int64_t)p * Hkv * hd, rowbuf + (Hq + Hkv) * hd,
+               (unsigned)(Hkv * hd * 2));
+  }
+}
+
+// Polls of a bulk-copy barrier before the kernel gives up (each poll may
+// suspend the thread for a while; the bound is far beyond any real copy).
+constexpr int kMaxPolls = 1 << 22;
+
+// Bulk-copy kernel (large batches).  One CTA per token.  One thread moves the
+// token's whole QKV row, its cos/sin rows and both norm weights into shared
+// memory with 1-D bulk copies (TMA) completed on an mbarrier, so no register
+// holds in-flight data and a small CTA keeps 12+ KB per token in flight.  Lane
+// groups (GP lanes per head) normalise and rotate the Q and K heads in place;
+// then the Q row, the K row and the untouched V row leave as three bulk
+// stores.  A barrier wait that runs out of polls sets bit 1 of *status and the
+// CTA returns without writing.
+// EPI: 0 = op (b) as is (Q token-major, unscaled; 16-bit caches), 1 = Q
+// epilogue (scale, layout), 2 = Q epilogue + e4m3 caches.  At most 128
+// threads; the register budget keeps 10 CTAs (tokens) resident per SM (8 for
+// the 16-bit Q epilogue, which would spill at 10): the kernel waits on memory,
+// so resident tokens, not instruction count, set its rate.
+template <int EPI>
+constexpr int tma_min_blocks() {
+  return EPI == 1 ? 8 : 10;
+}
+
+template <int DT, int P, int GP, int EPI>
+__global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvcache_tma_kernel(
+    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_norm_w,
+    const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
+    const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, void* __restrict__ k_cache,
+    void* __restrict__ v_cache, int32_t* status, int H, int NG, int Hq, int Hkv, int hd, int G, int max_pos,
+    int capacity, float eps, Epilogue ep) {
+  pdl_enter();
+  // [QKV row][cos][sin][q weight][k weight] (+ [K codes][V codes] with EPI 2)
+  extern __shared__ __align__(128) uint8_t dsmem[];
+  __shared__ uint64_t bar;
+  __shared__ int s_pos;
+  const int tok = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int half = hd >> 1;
+  const unsigned row_bytes = (unsigned)(H * hd * 2);
+  const unsigned tab_bytes = (unsigned)(half * 4);
+  const unsigned w_bytes = (unsigned)(hd * 2);
+  uint16_t* rowbuf = reinterpret_cast<uint16_t*>(dsmem);
+  float* cbuf = reinterpret_cast<float*>(dsmem + row_bytes);
+  float* sbuf = cbuf + half;
+  uint16_t* qwbuf = reinterpret_cast<uint16_t*>(sbuf + half);
+  uint16_t* kwbuf = qwbuf + hd;
+  uint8_t* k8buf = reinterpret_cast<uint8_t*>(kwbuf + hd);
+  uint8_t* v8buf = k8buf + Hkv * hd;
+
+  if (tid == 0) {
+    mbar_init(&bar, 2);  // two arrivals: the row (+ weights), then the table rows
+    mbar_init_fence();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned first = row_bytes + (q_norm_w ? w_bytes : 0u) + (k_norm_w ? w_bytes : 0u);
+    mbar_arrive_expect_tx(&bar, first);
+    bulk_load(rowbuf, qkv + (int64_t)tok * H * hd, row_bytes, &bar);
+    if (q_norm_w) bulk_load(qwbuf, q_norm_w, w_bytes, &bar);
+    if (k_norm_w) bulk_load(kwbuf, k_norm_w, w_bytes, &bar);
+    const int p = __ldg(positions + tok);
+    const bool ok = p >= 0 && p < max_pos && p < capacity;
+    s_pos = ok ? p : -1;
+    if (ok) {
+      mbar_arrive_expect_tx(&bar, 2 * tab_bytes);
+      bulk_load(cbuf, cos_tab + (int64_t)p * half, tab_bytes, &bar);
+      bulk_load(sbuf, sin_tab + (int64_t)p * half, tab_bytes, &bar);
+    } else {
+      if (status != nullptr) atomicOr(status, 1);
+      mbar_arrive_expect_tx(&bar, 0u);
+    }
+  }
+  const bool landed = mbar_wait_bounded(&bar, 0, kMaxPolls);
+  if (!__syncthreads_and(landed)) {
+    if (tid == 0 && status != nullptr) atomicOr(status, 2);
+    mbar_wait_bounded(&bar, 0, kMaxPolls);  // give copies still in flight a last chance to land
+    return;
+  }
+  const int p = s_pos;
+  if (p < 0) return;  // position out of range: nothing is written
+  process_token<DT, P, GP, EPI>(rowbuf, cbuf, sbuf, qwbuf, kwbuf, k8buf, v8buf, q_norm_w, k_norm_w, q_out, tok, tid,
+                                H, NG, Hq, Hkv, hd, G, eps, ep);
   fence_proxy_async_smem();  // this thread's writes -> the bulk stores below
   __syncthreads();
-  // Token-major Q leaves as one bulk store with the K and V rows (head-major
-  // Q went straight from registers above).
   if (tid == 0) {
-    if (!q_direct) bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
-    if (KV8) {
-      bulk_store(static_cast<uint8_t*>(k_cache) + (int64_t)p * Hkv * hd, k8buf, (unsigned)(Hkv * hd));
-      bulk_store(static_cast<uint8_t*>(v_cache) + (int64_t)p * Hkv * hd, v8buf, (unsigned)(Hkv * hd));
-    } else {
-      bulk_store(static_cast<uint16_t*>(k_cache) + (int64_t)p * Hkv * hd, rowbuf + Hq * hd,
-                 (unsigned)(Hkv * hd * 2));
-      bulk_store(static_cast<uint16_t*>(v_cache) + (int64_t)p * Hkv * hd, rowbuf + (Hq + Hkv) * hd,
-                 (unsigned)(Hkv * hd * 2));
-    }
+    store_token<EPI>(rowbuf, k8buf, v8buf, q_out, k_cache, v_cache, tok, p, Hq, Hkv, hd, ep);
     bulk_commit();
     bulk_wait_read();  // shared memory must outlive the stores' reads
   }
