@@ -77,6 +77,20 @@ def lib():
                                                          [c.c_double, c.c_int, c.c_double, c.c_int, c.c_int,
                                                           c.c_double, c.c_double])
         L.oracle_qkv_norm_rope_prepq_kvcache.restype = c.c_int
+        L.oracle_e2m1_encode.argtypes = [c.c_double]
+        L.oracle_e2m1_encode.restype = c.c_uint8
+        L.oracle_e2m1_decode.argtypes = [c.c_uint8]
+        L.oracle_e2m1_decode.restype = c.c_double
+        L.oracle_sf_swizzle_offset.argtypes = [c.c_int64, c.c_int64, c.c_int64]
+        L.oracle_sf_swizzle_offset.restype = c.c_int64
+        L.oracle_quant_nvfp4_row.argtypes = [c.c_void_p, c.c_int64, c.c_float, c.c_void_p, c.c_void_p]
+        L.oracle_quant_nvfp4_row.restype = None
+        L.oracle_residual_rmsnorm_nvfp4.argtypes = [c.c_void_p] * 6 + [c.c_double, c.c_void_p, c.c_int64,
+                                                                       c.c_int64, c.c_double, c.c_int]
+        L.oracle_residual_rmsnorm_nvfp4.restype = c.c_int
+        L.oracle_gate_act_nvfp4.argtypes = [c.c_void_p] * 3 + [c.c_double, c.c_void_p, c.c_int64, c.c_int64,
+                                                               c.c_int, c.c_int]
+        L.oracle_gate_act_nvfp4.restype = c.c_int
         _lib = L
     return _lib
 
@@ -265,3 +279,69 @@ def gate_residual_adarms_fp8(x, gate, residual_in, scale, shift, eps, dt, quant,
     if rc != 0:
         raise ValueError("oracle_gate_residual_adarms_fp8: bad argument")
     return {"residual_out": r_out, "out_fp8": q, "block_scales": bs, "y": y}
+
+
+# ------------------------------------------------------------------ NEXT-3 --
+def e2m1_encode(v):
+    return int(lib().oracle_e2m1_encode(float(v)))
+
+
+def e2m1_decode(c):
+    return float(lib().oracle_e2m1_decode(int(c)))
+
+
+def sf_swizzle_offset(r, c, n_cols):
+    return int(lib().oracle_sf_swizzle_offset(int(r), int(c), int(n_cols)))
+
+
+def quant_nvfp4_row(y, global_scale):
+    """One row (length a multiple of 16) -> (packed uint8 [n/2], sf uint8 [n/16])."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    n = y.shape[0]
+    packed = np.empty(n // 2, dtype=np.uint8)
+    sf = np.empty(n // 16, dtype=np.uint8)
+    lib().oracle_quant_nvfp4_row(_p(y), n, float(global_scale), _p(packed), _p(sf))
+    return packed, sf
+
+
+def residual_rmsnorm_nvfp4(x, residual_in, weight, eps, dt, global_scale, want_y=False):
+    """Op (a) with an NVFP4 output: residual_out, out_fp4 [M, D/2], sf [M, D/16]."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    r = np.ascontiguousarray(residual_in, dtype=np.uint16)
+    M, D = x.shape
+    w = None if weight is None else np.ascontiguousarray(weight, dtype=np.uint16)
+    r_out = np.empty_like(r)
+    q = np.empty((M, D // 2), dtype=np.uint8)
+    sf = np.empty((M, D // 16), dtype=np.uint8)
+    y = np.empty((M, D), dtype=np.float64) if want_y else None
+    rc = lib().oracle_residual_rmsnorm_nvfp4(_p(x), _p(r), _p(r_out), _p(w), _p(q), _p(sf), float(global_scale),
+                                             _p(y), M, D, _f32(eps), _DT[dt])
+    if rc != 0:
+        raise ValueError("oracle_residual_rmsnorm_nvfp4: bad argument")
+    return {"residual_out": r_out, "out_fp4": q, "sf": sf, "y": y}
+
+
+def gate_act_nvfp4(gate_up, act_name, dt, global_scale, want_a=False):
+    """Op (c) with an NVFP4 output: out_fp4 [M, I/2], sf [M, I/16]."""
+    gu = np.ascontiguousarray(gate_up, dtype=np.uint16)
+    M, two_i = gu.shape
+    I = two_i // 2
+    q = np.empty((M, I // 2), dtype=np.uint8)
+    sf = np.empty((M, I // 16), dtype=np.uint8)
+    a = np.empty((M, I), dtype=np.float64) if want_a else None
+    rc = lib().oracle_gate_act_nvfp4(_p(gu), _p(q), _p(sf), float(global_scale), _p(a), M, I, _ACT[act_name],
+                                     _DT[dt])
+    if rc != 0:
+        raise ValueError("oracle_gate_act_nvfp4: bad argument")
+    return {"out_fp4": q, "sf": sf, "a": a}
+
+
+def sf_swizzle(sf_rowmajor):
+    """Row-major scale factors [M, C] -> the 128x4-swizzled byte array
+    (padded to 128-row / 4-column atoms; padding bytes 0)."""
+    M, C = sf_rowmajor.shape
+    out = np.zeros(((M + 127) // 128) * 128 * ((C + 3) // 4) * 4, dtype=np.uint8)
+    for r in range(M):
+        for c in range(C):
+            out[sf_swizzle_offset(r, c, C)] = sf_rowmajor[r, c]
+    return out

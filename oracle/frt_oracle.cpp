@@ -201,6 +201,74 @@ void quant_block128(const double* y, int64_t n, uint8_t* q, double* scales) {
   }
 }
 
+// ---------------------------------------------------------------- NVFP4 --
+// NVFP4 (NEXT-3; the pages' W4A4 path: "residual_add_rms_norm_to_nvfp4",
+// "silu_mul_merged_grouped32", NVFP4 producers feeding FP4 GEMMs).  The pages
+// name the format only; the reading is NVIDIA's NVFP4:
+//   element  e2m1 (1 sign, 2 exponent, 1 mantissa bit): magnitudes
+//            0, 0.5, 1, 1.5, 2, 3, 4, 6; round to nearest, ties to even
+//            mantissa, saturating at 6; two per byte, element 2j in the low
+//            nibble of byte j.
+//   block    16 consecutive elements of a row share one unsigned e4m3 scale
+//            factor sf; with the per-tensor fp32 global scale gs,
+//            y ~ e2m1 * decode(sf) * gs.
+//   decision in fp32 (as every FP8 decision here): with y32 the fp32 values,
+//            amax32 = max |y32| over the block, den = fp32(6 * gs),
+//            sf = e4m3(amax32 / den) (IEEE fp32 quotient, RNE, saturating to
+//            448), eff = fp32(decode(sf) * gs), code = e2m1(y32 / eff) (IEEE
+//            fp32 quotient); sf == 0 (an all-zero or negligible block) gives
+//            all-zero codes.
+uint8_t e2m1_encode(double v) {
+  const uint8_t s = std::signbit(v) ? 0x8 : 0x0;
+  const double a = std::fabs(v);
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  if (!(a < 6.0)) return (uint8_t)(s | 7);  // saturate (NaN inputs are not defined here)
+  int best = 0;
+  for (int c = 1; c < 8; ++c) {
+    const double d = std::fabs(mag[c] - a), db = std::fabs(mag[best] - a);
+    if (d < db || (d == db && (c & 1) == 0)) best = c;  // ties to the even mantissa bit
+  }
+  return (uint8_t)(s | best);
+}
+
+double e2m1_decode(uint8_t c) {
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  const double v = mag[c & 7];
+  return (c & 0x8) ? -v : v;
+}
+
+// One row of n (a multiple of 16) values -> n/2 packed bytes and n/16 scale
+// factors (row-major).
+void quant_nvfp4_row(const double* y, int64_t n, float gs, uint8_t* packed, uint8_t* sf) {
+  const float den = 6.0f * gs;
+  for (int64_t b = 0; b < n / 16; ++b) {
+    float y32[16];
+    float amax = 0.0f;
+    for (int j = 0; j < 16; ++j) {
+      y32[j] = (float)y[16 * b + j];
+      amax = std::fmax(amax, std::fabs(y32[j]));
+    }
+    const uint8_t code_sf = e4m3_encode((double)(amax / den));
+    sf[b] = code_sf;
+    const float eff = (float)e4m3_decode(code_sf) * gs;
+    uint8_t q[16];
+    for (int j = 0; j < 16; ++j) q[j] = (eff > 0.0f) ? e2m1_encode((double)(y32[j] / eff)) : 0;
+    for (int j = 0; j < 8; ++j) packed[8 * b + j] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+  }
+}
+
+// Byte offset of scale factor (row r, column c) in the 128x4-swizzled layout
+// that block-scaled tensor-core GEMMs read: atoms of 128 rows x 4 scale
+// columns (512 bytes), atoms laid out row-major over (row / 128, c / 4) with
+// ceil(n_cols / 4) atoms per atom-row; inside an atom, row r % 128 = 32 i + k
+// and column c % 4 = l sit at byte 16 k + 4 i + l.
+int64_t sf_swizzle_offset(int64_t r, int64_t c, int64_t n_cols) {
+  const int64_t atoms_per_row = (n_cols + 3) / 4;
+  const int64_t atom = (r / 128) * atoms_per_row + c / 4;
+  const int64_t rr = r % 128;
+  return atom * 512 + (rr % 32) * 16 + (rr / 32) * 4 + (c % 4);
+}
+
 // --------------------------------------------------------------- RMSNorm --
 // y_j = h_j * rstd * w_j with rstd = 1 / sqrt(mean(h^2) + eps); w == nullptr
 // is the `_noweight` form whose (1 + w) lives in the next GEMM's weights
@@ -513,6 +581,56 @@ int oracle_qkv_norm_rope_prepq_kvcache(const uint16_t* qkv, const uint16_t* q_no
         std::memcpy(v_cache + (slot * Hkv + g) * hd, src, sizeof(uint16_t) * hd);
       }
     }
+  }
+  return 0;
+}
+
+// ------------------------------------------------------------- NEXT-3 --
+uint8_t oracle_e2m1_encode(double v) { return e2m1_encode(v); }
+double oracle_e2m1_decode(uint8_t c) { return e2m1_decode(c); }
+int64_t oracle_sf_swizzle_offset(int64_t r, int64_t c, int64_t n_cols) { return sf_swizzle_offset(r, c, n_cols); }
+void oracle_quant_nvfp4_row(const double* y, int64_t n, float gs, uint8_t* packed, uint8_t* sf) {
+  quant_nvfp4_row(y, n, gs, packed, sf);
+}
+
+// Op (a) with an NVFP4 output ("residual_add_rms_norm_to_nvfp4"): h and y as
+// op (a); out_fp4 [M, D/2] packed e2m1, sf [M, D/16] row-major e4m3.
+int oracle_residual_rmsnorm_nvfp4(const uint16_t* x, const uint16_t* residual_in, uint16_t* residual_out,
+                                  const uint16_t* weight, uint8_t* out_fp4, uint8_t* sf, double global_scale,
+                                  double* y_out, int64_t M, int64_t D, double eps, int dt) {
+  if (M < 0 || D <= 0 || D % 16 != 0 || !x || !residual_in || !residual_out || !out_fp4 || !sf) return -1;
+  const Fmt16 f = fmt_of(dt);
+  std::vector<double> h(D), w(D), y(D);
+  if (weight)
+    for (int64_t j = 0; j < D; ++j) w[j] = decode16(weight[j], f);
+  for (int64_t i = 0; i < M; ++i) {
+    for (int64_t j = 0; j < D; ++j) {
+      double s, err;
+      two_sum(decode16(x[i * D + j], f), decode16(residual_in[i * D + j], f), &s, &err);
+      const uint16_t hb = round16(s, err, f);
+      residual_out[i * D + j] = hb;
+      h[j] = decode16(hb, f);
+    }
+    rmsnorm(h.data(), D, weight ? w.data() : nullptr, eps, y.data());
+    if (y_out) std::memcpy(y_out + i * D, y.data(), sizeof(double) * D);
+    quant_nvfp4_row(y.data(), D, (float)global_scale, out_fp4 + i * D / 2, sf + i * D / 16);
+  }
+  return 0;
+}
+
+// Op (c) with an NVFP4 output ("silu_mul_merged_grouped32"): a as op (c);
+// out_fp4 [M, I/2] packed e2m1, sf [M, I/16] row-major e4m3.
+int oracle_gate_act_nvfp4(const uint16_t* gate_up, uint8_t* out_fp4, uint8_t* sf, double global_scale,
+                          double* a_out, int64_t M, int64_t I, int act, int dt) {
+  if (M < 0 || I <= 0 || I % 16 != 0 || !gate_up || !out_fp4 || !sf) return -1;
+  if (act < ACT_GELU_TANH || act > ACT_RELU2) return -1;
+  const Fmt16 f = fmt_of(dt);
+  std::vector<double> a(I);
+  for (int64_t i = 0; i < M; ++i) {
+    const uint16_t* row = gate_up + i * 2 * I;
+    for (int64_t j = 0; j < I; ++j) a[j] = act_fn(act, decode16(row[2 * j], f)) * decode16(row[2 * j + 1], f);
+    if (a_out) std::memcpy(a_out + i * I, a.data(), sizeof(double) * I);
+    quant_nvfp4_row(a.data(), I, (float)global_scale, out_fp4 + i * I / 2, sf + i * I / 16);
   }
   return 0;
 }

@@ -196,3 +196,138 @@ def test_prepq_bad_positions_skip_rows():
     assert o["status"] & 1
     assert np.isnan(o["q_out"][:, [1, 3]]).all() and np.isfinite(o["q_out"][:, [0, 2, 4]]).all()
     assert (o["k_cache"][64] == 0x7E).all()
+
+
+# ------------------------------------------------------------------ NEXT-3 --
+# NVFP4 outputs of ops (a) and (c) (the pages' "residual_add_rms_norm_to_nvfp4"
+# and "silu_mul_merged_grouped32" NVFP4 producers): e2m1 codes, 16-element
+# blocks with e4m3 scale factors and a per-tensor fp32 global scale.
+
+E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # the format's magnitudes, code = index (+8 for negative)
+
+
+def test_e2m1_codes_and_round_trip():
+    for c in range(16):
+        v = E2M1[c & 7] * (-1 if c & 8 else 1)
+        assert oracle.e2m1_decode(c) == v
+        assert oracle.e2m1_encode(oracle.e2m1_decode(c)) == c, c
+    assert math.copysign(1.0, oracle.e2m1_decode(8)) < 0
+
+
+def test_e2m1_ties_to_even_and_saturation():
+    for lo, hi in zip(E2M1[:-1], E2M1[1:]):
+        mid = (lo + hi) / 2
+        want = E2M1.index(lo) if E2M1.index(lo) % 2 == 0 else E2M1.index(hi)
+        assert oracle.e2m1_encode(mid) == want, mid
+        assert oracle.e2m1_encode(-mid) == want | 8
+        assert oracle.e2m1_encode(np.nextafter(mid, 0)) == E2M1.index(lo)
+        assert oracle.e2m1_encode(np.nextafter(mid, 10)) == E2M1.index(hi)
+    assert oracle.e2m1_encode(6.0) == 7 and oracle.e2m1_encode(1e30) == 7 and oracle.e2m1_encode(-7.5) == 15
+
+
+def _nvfp4_brute(y, gs):
+    """The NVFP4 reading restated with numpy fp32 scalars and brute-force
+    nearest-code searches (e4m3 via the whole code table, e2m1 over its 8
+    magnitudes, ties to the even code)."""
+    y32 = np.asarray(y, dtype=np.float32)
+    packed, sfs = [], []
+    for b in range(len(y32) // 16):
+        blk = y32[16 * b:16 * b + 16]
+        amax = np.float32(np.max(np.abs(blk)))
+        den = np.float32(6.0) * np.float32(gs)
+        sf = int(_nearest_e4m3(np.array([float(np.float32(amax / den))]))[0])
+        eff = np.float32(np.float32(oracle.e4m3_decode(sf)) * np.float32(gs))
+        codes = []
+        for v in blk:
+            if eff == 0:
+                codes.append(0)
+                continue
+            t = float(np.float32(v / eff))
+            a = min(abs(t), 6.0)
+            d = [abs(m - a) for m in E2M1]
+            best = [k for k in range(8) if d[k] == min(d)]
+            k = [k for k in best if k % 2 == 0][0] if len(best) > 1 else best[0]
+            codes.append(k | (8 if math.copysign(1.0, t) < 0 else 0))
+        sfs.append(sf)
+        packed += [codes[2 * j] | (codes[2 * j + 1] << 4) for j in range(8)]
+    return np.array(packed, dtype=np.uint8), np.array(sfs, dtype=np.uint8)
+
+
+@pytest.mark.parametrize("gs", [1.0, 0.0123, 3.7e-4])
+def test_nvfp4_row_matches_brute_force(gs):
+    g = W.generator(11)
+    y = torch.randn(96, generator=g, dtype=torch.float64).numpy() * 2.5
+    y[16:32] *= 1e-3                          # a small block
+    y[32:48] = 0.0                            # an all-zero block
+    packed, sf = oracle.quant_nvfp4_row(y, gs)
+    bp, bsf = _nvfp4_brute(y, gs)
+    np.testing.assert_array_equal(sf, bsf)
+    np.testing.assert_array_equal(packed, bp)
+    assert sf[2] == 0 and (packed[16:24] == 0).all()
+
+
+def test_nvfp4_exact_block_closed_form_and_nibble_order():
+    # gs = 1: den = 6; a block whose amax is 6 * 2^k has sf = 2^k exactly and
+    # every value k-scaled e2m1 magnitude quantises to its own code
+    k = -3
+    vals = np.array([E2M1[j % 8] * (-1 if j >= 8 else 1) for j in range(16)]) * 2.0 ** k
+    vals[0] = 6.0 * 2.0 ** k                  # amax (code 7) in element 0
+    packed, sf = oracle.quant_nvfp4_row(vals, 1.0)
+    assert oracle.e4m3_decode(int(sf[0])) == 2.0 ** k
+    codes = [int(packed[j // 2] >> (4 * (j % 2))) & 0xF for j in range(16)]
+    want = [oracle.e2m1_encode(v / 2.0 ** k) for v in vals]
+    assert codes == want and codes[0] == 7   # element 0 in the low nibble of byte 0
+
+
+def test_nvfp4_dequantisation_error_bound():
+    g = W.generator(12)
+    y = torch.randn(16 * 64, generator=g, dtype=torch.float64).numpy()
+    gs = 0.002
+    packed, sf = oracle.quant_nvfp4_row(y, gs)
+    codes = np.stack([packed & 0xF, packed >> 4], axis=1).ravel()
+    for b in range(64):
+        eff = oracle.e4m3_decode(int(sf[b])) * np.float32(gs)
+        amax = np.max(np.abs(y[16 * b:16 * b + 16]))
+        assert abs(eff * 6 - amax) <= amax * 2.0 ** -3                 # e4m3 scale: within half a step (2^-4) + fp32
+        for j in range(16):
+            v = y[16 * b + j]
+            dq = oracle.e2m1_decode(int(codes[16 * b + j])) * eff
+            t = min(abs(v) / eff, 6.0)
+            spacing = 0.5 if t < 2 else (1.0 if t < 4 else 2.0)
+            assert abs(abs(dq) - min(abs(v), 6 * eff)) <= spacing / 2 * eff * (1 + 1e-6) + 1e-12
+
+
+def test_nvfp4_ops_reuse_op_a_and_op_c():
+    x, r, _, _, _ = _inputs(3, 256, "bf16", 13, 1)
+    g = W.generator(13)
+    w = W.bits16(W.norm_weight(256, "bf16", g))
+    a = oracle.residual_rmsnorm_nvfp4(x, r, w, 1e-6, "bf16", 0.004, want_y=True)
+    b = oracle.residual_rmsnorm_fp8(x, r, w, 1e-6, "bf16", "static", static_scale=0.01, want_y=True)
+    np.testing.assert_array_equal(a["residual_out"], b["residual_out"])
+    np.testing.assert_array_equal(a["y"], b["y"])
+    for i in range(3):
+        p, s = oracle.quant_nvfp4_row(a["y"][i], 0.004)
+        np.testing.assert_array_equal(a["out_fp4"][i], p)
+        np.testing.assert_array_equal(a["sf"][i], s)
+    gu = W.bits16(W.normal16((2, 2 * 128), "bf16", g))
+    c = oracle.gate_act_nvfp4(gu, "silu", "bf16", 0.003, want_a=True)
+    d = oracle.gate_act_fp8(gu, "silu", "bf16", "static", static_scale=0.01, want_a=True)
+    np.testing.assert_array_equal(c["a"], d["a"])
+    for i in range(2):
+        p, s = oracle.quant_nvfp4_row(c["a"][i], 0.003)
+        np.testing.assert_array_equal(c["out_fp4"][i], p)
+
+
+def test_sf_swizzle_layout():
+    C = 10
+    atoms = (C + 3) // 4
+    assert oracle.sf_swizzle_offset(0, 0, C) == 0
+    assert oracle.sf_swizzle_offset(1, 0, C) == 16
+    assert oracle.sf_swizzle_offset(31, 0, C) == 496
+    assert oracle.sf_swizzle_offset(32, 0, C) == 4
+    assert oracle.sf_swizzle_offset(97, 3, C) == 16 * 1 + 4 * 3 + 3
+    assert oracle.sf_swizzle_offset(0, 4, C) == 512
+    assert oracle.sf_swizzle_offset(128, 0, C) == atoms * 512
+    M = 300
+    offs = {oracle.sf_swizzle_offset(r, c, C) for r in range(((M + 127) // 128) * 128) for c in range(atoms * 4)}
+    assert offs == set(range(((M + 127) // 128) * 128 * atoms * 4))   # a bijection onto the padded array
