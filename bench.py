@@ -453,6 +453,41 @@ def next_ops_leg(peak, floor, reps=50, big_m=65536):
                 "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4), "q_layout": "head-major", "kv": "e4m3",
                 "traffic": measured_traffic(key, "qkv_prepq")}
     del qkv, q_out, kc, vc
+    # NEXT-3: the NVFP4 producers on the large-M shapes (norm 65536 x 4096,
+    # gated activation 65536 x 16384 squared ReLU), row-major scale factors.
+    g = W.generator(63, "cuda")
+    D, I = wl.D, wl.I
+    x = W.normal16((big_m, D), "bf16", g)
+    r = W.normal16((big_m, D), "bf16", g)
+    w = W.norm_weight(D, "bf16", g)
+    q = torch.empty((big_m, D // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((big_m * D // 16,), dtype=torch.uint8, device="cuda")
+    gsd = torch.tensor([0.0015], dtype=torch.float32, device="cuda")
+    cases = [("residual_rmsnorm_nvfp4_M%d_D%d" % (big_m, D), big_m * D * 6.5 + big_m * D // 16 + 2 * D,
+              lambda: frt.frt_residual_rmsnorm_nvfp4(x, r, r, w, q, sf, gsd))]
+    gu = W.normal16((big_m, 2 * I), "bf16", g)
+    qc = torch.empty((big_m, I // 2), dtype=torch.uint8, device="cuda")
+    sfc = torch.empty((big_m * I // 16,), dtype=torch.uint8, device="cuda")
+    cases.append(("gate_act_nvfp4_relu2_M%d_I%d" % (big_m, I), big_m * I * 4.5 + big_m * I // 16,
+                  lambda: frt.frt_gate_act_nvfp4(gu, qc, sfc, gsd, act="relu2")))
+    for key, nbytes, fn in cases:
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+        for i in range(reps):
+            ev[2 * i].record(s)
+            fn()
+            ev[2 * i + 1].record(s)
+        torch.cuda.synchronize()
+        ts = [ev[2 * i].elapsed_time(ev[2 * i + 1]) * 1e3 for i in range(reps)]
+        us = sum(ts) / len(ts)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[key] = {"us_mean": round(us, 2), "us_median": round(statistics.median(ts), 2), "bytes": int(nbytes),
+                    "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                    "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4), "sf_layout": "rows",
+                    "traffic": measured_traffic(key, "nvfp4")}
+    del x, r, q, sf, gu, qc, sfc
     return out
 
 

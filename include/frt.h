@@ -76,6 +76,16 @@ typedef enum { FRT_QUANT_STATIC = 0, FRT_QUANT_BLOCK128 = 1 } frt_quant;
  *             ("Falcon-Perception inference optimisation", third technique). */
 typedef enum { FRT_ACT_GELU_TANH = 0, FRT_ACT_SILU = 1, FRT_ACT_RELU2 = 2 } frt_act;
 
+/* Scale-factor layout of the NVFP4 producers (NEXT-3):
+ *  ROW_MAJOR       sf[M, N/16] row-major bytes
+ *  SWIZZLED_128X4  the layout block-scaled tensor-core GEMMs read: 512-byte
+ *                  atoms of 128 rows x 4 scale columns, laid out row-major over
+ *                  (row / 128, column / 4) with ceil(N/64) atoms per atom row;
+ *                  inside an atom, row 32 i + k and column l sit at byte
+ *                  16 k + 4 i + l.  The array holds ceil(M/128) * 128 *
+ *                  ceil(N/64) * 4 bytes; padding bytes are not written. */
+typedef enum { FRT_SF_ROW_MAJOR = 0, FRT_SF_SWIZZLED_128X4 = 1 } frt_sf_layout;
+
 /* Q staging layout of the QKV op with the Q epilogue (NEXT-2):
  *  TOKEN_MAJOR  q_out[M, Hq, hd]  (op (b)'s layout)
  *  HEAD_MAJOR   q_out[Hq, M, hd]  (one contiguous [M, hd] slab per head) */
@@ -186,6 +196,36 @@ frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_norm_w, cons
 frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* static_scale,
                             float* block_scales, int M, int I, frt_act act, frt_dtype dt, frt_quant qm,
                             cudaStream_t stream);
+
+/*
+ * NEXT-3: NVFP4 outputs of ops (a) and (c).  The FlashRT port's NVFP4
+ * producers "residual_add_rms_norm_to_nvfp4" and "silu_mul_merged_grouped32"
+ * (the "5060 Ti" report's per-kernel census and its W4A4 NVFP4 GEMM path).
+ * The pages name the format only; the reading is NVFP4:
+ *   e2m1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte with
+ *   element 2j in the low nibble of byte j; blocks of 16 consecutive elements
+ *   of a row share an unsigned e4m3 scale factor sf; with the per-tensor
+ *   global scale gs, y ~ e2m1 * sf * gs.  Decisions in fp32, scaling by
+ *   correctly rounded reciprocals (RN = fp32 round to nearest even):
+ *     sf   = e4m3(RN(amax_block * RN(1 / RN(6 gs))))  (RNE, saturating to 448)
+ *     eff  = RN(sf * gs)
+ *     code = e2m1(RN(y * RN(1 / eff)))     (RNE, saturating to 6; 0 when sf = 0)
+ *   global_scale must lie in [2^-100, 2^100].
+ *
+ * frt_residual_rmsnorm_nvfp4: h and y exactly as frt_residual_rmsnorm_fp8
+ *   (residual written back); out_fp4 [M, D/2] bytes, 4-byte aligned.
+ * frt_gate_act_nvfp4: a exactly as frt_gate_act_fp8; out_fp4 [M, I/2] bytes,
+ *   2-byte aligned.
+ *   out_sf        device bytes in `sf_layout` (see frt_sf_layout).
+ *   global_scale  device fp32[1].
+ *   Layout rule: D (I) > 0 and D % 16 == 0 (I % 16 == 0); other arguments
+ *   as the FP8 ops.  Unsupported: D > 32768.
+ */
+frt_status frt_residual_rmsnorm_nvfp4(const void* x, const void* residual_in, void* residual_out, const void* weight,
+                                      uint8_t* out_fp4, uint8_t* out_sf, const float* global_scale, int M, int D,
+                                      float eps, frt_dtype dt, frt_sf_layout sf_layout, cudaStream_t stream);
+frt_status frt_gate_act_nvfp4(const void* gate_up, uint8_t* out_fp4, uint8_t* out_sf, const float* global_scale,
+                              int M, int I, frt_act act, frt_dtype dt, frt_sf_layout sf_layout, cudaStream_t stream);
 
 /*
  * NEXT-2: op (b) with the attention's Q preparation and an optional FP8 KV

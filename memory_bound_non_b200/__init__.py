@@ -28,8 +28,8 @@ ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
 
 # C entry points declared in include/frt.h
 EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8",
-           "frt_qkv_norm_rope_prepq_kvcache", "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl",
-           "frt_get_pdl", "frt_status_string")
+           "frt_residual_rmsnorm_nvfp4", "frt_gate_act_nvfp4", "frt_qkv_norm_rope_prepq_kvcache",
+           "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_status_string")
 
 
 class FrtError(RuntimeError):
@@ -57,6 +57,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_qkv_norm_rope_kvcache.restype = i32
     L.frt_qkv_norm_rope_prepq_kvcache.argtypes = [vp] * 10 + [i32] * 6 + [f32, f32, i32, i32, vp, i32, vp]
     L.frt_qkv_norm_rope_prepq_kvcache.restype = i32
+    L.frt_residual_rmsnorm_nvfp4.argtypes = [vp] * 7 + [i32, i32, f32, i32, i32, vp]
+    L.frt_residual_rmsnorm_nvfp4.restype = i32
+    L.frt_gate_act_nvfp4.argtypes = [vp] * 4 + [i32, i32, i32, i32, i32, vp]
+    L.frt_gate_act_nvfp4.restype = i32
     L.frt_gate_act_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     L.frt_gate_act_fp8.restype = i32
     L.frt_gate_residual_adarms_fp8.argtypes = [vp] * 9 + [i32, i32, i32, f32, i32, i32, vp]
@@ -123,6 +127,36 @@ def frt_qkv_norm_rope_kvcache(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positio
         _ptr(k_cache), _ptr(v_cache), _ptr(status), M, Hq, Hkv, hd, max_pos, capacity, float(eps),
         DTYPE[qkv.dtype], _stream(stream))
     _check("frt_qkv_norm_rope_kvcache", st)
+
+
+SF_LAYOUT = {"rows": 0, "swizzled": 1}
+
+
+def nvfp4_sf_bytes(rows, n, layout="rows"):
+    """Bytes of the scale-factor array of an [rows, n] NVFP4 output."""
+    if layout == "rows":
+        return rows * (n // 16)
+    return ((rows + 127) // 128) * 128 * ((n // 16 + 3) // 4) * 4
+
+
+def frt_residual_rmsnorm_nvfp4(x, residual_in, residual_out, weight, out_fp4, out_sf, global_scale, eps=1e-6,
+                               sf_layout="rows", stream=None):
+    """NEXT-3: op (a) with an NVFP4 output: out_fp4 uint8 [M, D/2] (two e2m1
+    per byte), out_sf uint8 scale factors (see nvfp4_sf_bytes), global_scale
+    fp32[1] on the device."""
+    M, D = x.shape
+    st = load().frt_residual_rmsnorm_nvfp4(
+        _ptr(x), _ptr(residual_in), _ptr(residual_out), _ptr(weight), _ptr(out_fp4), _ptr(out_sf),
+        _ptr(global_scale), M, D, float(eps), DTYPE[x.dtype], SF_LAYOUT[sf_layout], _stream(stream))
+    _check("frt_residual_rmsnorm_nvfp4", st)
+
+
+def frt_gate_act_nvfp4(gate_up, out_fp4, out_sf, global_scale, act="gelu_tanh", sf_layout="rows", stream=None):
+    """NEXT-3: op (c) with an NVFP4 output: out_fp4 uint8 [M, I/2]."""
+    M, two_i = gate_up.shape
+    st = load().frt_gate_act_nvfp4(_ptr(gate_up), _ptr(out_fp4), _ptr(out_sf), _ptr(global_scale), M, two_i // 2,
+                                   ACT[act], DTYPE[gate_up.dtype], SF_LAYOUT[sf_layout], _stream(stream))
+    _check("frt_gate_act_nvfp4", st)
 
 
 Q_LAYOUT = {"token": 0, "head": 1}

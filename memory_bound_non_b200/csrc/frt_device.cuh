@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "frt.h"
@@ -139,6 +140,49 @@ __device__ __forceinline__ uint32_t quant4(const float* y, const Divisor& dv) {
 
 __device__ __forceinline__ uint2 quant8(const float* y, const Divisor& dv) {
   return make_uint2(quant4(y, dv), quant4(y + 4, dv));
+}
+
+// ----------------------------------------------------------------- NVFP4 --
+// e2m1 elements in 16-element blocks, each block scaled by an unsigned e4m3
+// factor sf and the per-tensor fp32 global scale gs (y ~ e2m1 * sf * gs).
+// Decisions in fp32, scaling by correctly rounded reciprocals:
+//   rden = RN(1 / RN(6 gs)), sf = e4m3(RN(amax * rden)),
+//   eff = RN(sf * gs), reff = RN(1 / eff), code = e2m1(RN(y * reff));
+// sf == 0 gives zero codes.  gs must lie in [2^-100, 2^100].
+
+// Two fp32 -> two e2m1 codes in one byte (a in the low nibble), RNE, saturating.
+__device__ __forceinline__ uint32_t e2m1x2(float a, float b) {
+  return (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(a, b), __NV_E2M1, cudaRoundNearest);
+}
+// Exact value of an e4m3 code (e4m3 is a subset of binary16).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+  return __half2float(__half(h));
+}
+// Block scale: returns the sf code and the reciprocal of eff = RN(sf * gs)
+// (0 when sf is 0).
+__device__ __forceinline__ uint32_t nvfp4_scale(float amax, float rden, float gs, float* reff) {
+  const uint32_t sf = e4m3x2(amax * rden, 0.0f) & 0xFFu;
+  const float eff = e4m3_value(sf) * gs;
+  *reff = eff > 0.0f ? __frcp_rn(eff) : 0.0f;
+  return sf;
+}
+// N (4 or 8) values -> N e2m1 codes of y * reff, element 0 in the low nibble.
+template <int N>
+__device__ __forceinline__ uint32_t nvfp4_codes(const float* y, float reff) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int e = 0; e < N; e += 2) w |= e2m1x2(y[e] * reff, y[e + 1] * reff) << (4 * e);
+  return w;
+}
+// Byte offset of scale factor (row r, column c) of an [M, n_cols] scale
+// matrix in the 128x4-swizzled layout read by block-scaled tensor-core GEMMs:
+// 512-byte atoms of 128 rows x 4 columns, row-major over (r / 128, c / 4);
+// inside an atom, row 32 i + k and column l sit at byte 16 k + 4 i + l.
+__device__ __forceinline__ int64_t sf_offset_swizzled(int64_t r, int c, int n_cols) {
+  const int64_t atom = (r >> 7) * (int64_t)((n_cols + 3) >> 2) + (c >> 2);
+  const int rr = (int)(r & 127);
+  return atom * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (c & 3);
 }
 
 // ------------------------------------------------------------ memory ops --

@@ -48,6 +48,11 @@ inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
   return launch_status();
 }
 
+// Output modes of the quantising kernels beyond the ABI's FP8 modes: NVFP4
+// with row-major or 128x4-swizzled scale factors (internal template values).
+constexpr int kQuantNvfp4Rows = 2;
+constexpr int kQuantNvfp4Swizzled = 3;
+
 // Checks shared by the two FP8-producing ops: the pointer the quant mode needs.
 inline bool quant_args_ok(frt_quant qm, const float* static_scale, const float* block_scales) {
   if (qm == FRT_QUANT_STATIC) return static_scale != nullptr && aligned(static_scale, 4);
@@ -68,6 +73,15 @@ frt_status opt_in_smem(Kern kern, size_t bytes, std::atomic<int>& opted) {
     }
   }
   return FRT_OK;
+}
+
+// Validation shared by the NVFP4 producers: scale-factor layout, the global
+// scale pointer, and the packed-code and scale-factor outputs.
+inline bool nvfp4_args_ok(frt_sf_layout layout, const float* global_scale, const void* out_fp4, const void* out_sf,
+                          uintptr_t code_align) {
+  if (layout != FRT_SF_ROW_MAJOR && layout != FRT_SF_SWIZZLED_128X4) return false;
+  return global_scale != nullptr && aligned(global_scale, 4) && out_fp4 != nullptr && out_sf != nullptr &&
+         aligned(out_fp4, code_align);
 }
 
 }  // namespace frt

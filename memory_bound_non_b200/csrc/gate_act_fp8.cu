@@ -89,6 +89,9 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
     }
   }
 
+  // static FP8: the scale; NVFP4: the global scale gs and RN(1 / RN(6 gs))
+  const float gs = QM >= kQuantNvfp4Rows ? __ldg(static_scale) : 0.0f;
+  const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * gs) : 0.0f;
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? __ldg(static_scale) : 1.0f);
 
 #pragma unroll
@@ -109,33 +112,61 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
       const int64_t gb = gb0 + u;
       if (lane == 0 && gb < total_blocks) block_scales[gb] = sb;  // [M, NB] row-major == flat block index
       if (valid[u]) q[idx[u]] = quant4(a, Divisor(sb));
+    } else if (QM >= kQuantNvfp4Rows) {
+      // NVFP4: a 16-output block is 4 consecutive lanes; codes leave as 16 bits
+      // per lane, the scale factor from the block's first lane.  q /
+      // block_scales carry the code and sf pointers.
+      float am = absmax4(a[0], a[1], a[2], a[3]);
+      am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+      float reff;
+      const uint32_t sf = nvfp4_scale(am, rden, gs, &reff);
+      if (valid[u]) {
+        reinterpret_cast<uint16_t*>(q)[idx[u]] = (uint16_t)nvfp4_codes<4>(a, reff);
+        if ((lane & 3) == 0) {
+          uint8_t* sfo = reinterpret_cast<uint8_t*>(block_scales);
+          if (QM == kQuantNvfp4Rows) {
+            sfo[idx[u] >> 2] = (uint8_t)sf;  // flat output index / 16 == row * (I/16) + column block
+          } else {
+            const int64_t row = idx[u] / C4;
+            sfo[sf_offset_swizzled(row, (int)((idx[u] - row * C4) >> 2), C4 >> 2)] = (uint8_t)sf;
+          }
+        }
+      }
     } else if (valid[u]) {
       q[idx[u]] = quant4(a, dv_static);
     }
   }
 }
 
+template <int DT, int ACT, int QM>
+frt_status launch_q(bool full, dim3 grid, const uint4* in, uint32_t* out, const float* ss, float* bs, int64_t total,
+                    int NB, int C4, cudaStream_t st) {
+  return full ? launch(gate_act_fp8_kernel<DT, ACT, QM, true>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
+                       NB, C4)
+              : launch(gate_act_fp8_kernel<DT, ACT, QM, false>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
+                       NB, C4);
+}
+
 template <int DT, int ACT>
-frt_status launch_act(frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total,
-                      int NB, int C4, cudaStream_t st) {
+frt_status launch_act(int qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total, int NB, int C4,
+                      cudaStream_t st) {
   const int64_t warps = (total + kU - 1) / kU;
   const dim3 grid((unsigned)((warps + kWarps - 1) / kWarps));
   const uint4* in = static_cast<const uint4*>(gu);
   uint32_t* out = reinterpret_cast<uint32_t*>(q);
   const bool full = C4 == NB * 32;
-  if (qm == FRT_QUANT_STATIC)
-    return full ? launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC, true>, grid, dim3(kThreads), 0, st, in, out,
-                         ss, bs, total, NB, C4)
-                : launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_STATIC, false>, grid, dim3(kThreads), 0, st, in, out,
-                         ss, bs, total, NB, C4);
-  return full ? launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128, true>, grid, dim3(kThreads), 0, st, in, out,
-                       ss, bs, total, NB, C4)
-              : launch(gate_act_fp8_kernel<DT, ACT, FRT_QUANT_BLOCK128, false>, grid, dim3(kThreads), 0, st, in, out,
-                       ss, bs, total, NB, C4);
+  switch (qm) {
+    case FRT_QUANT_STATIC: return launch_q<DT, ACT, FRT_QUANT_STATIC>(full, grid, in, out, ss, bs, total, NB, C4, st);
+    case FRT_QUANT_BLOCK128:
+      return launch_q<DT, ACT, FRT_QUANT_BLOCK128>(full, grid, in, out, ss, bs, total, NB, C4, st);
+    case kQuantNvfp4Rows: return launch_q<DT, ACT, kQuantNvfp4Rows>(full, grid, in, out, ss, bs, total, NB, C4, st);
+    default: return launch_q<DT, ACT, kQuantNvfp4Swizzled>(full, grid, in, out, ss, bs, total, NB, C4, st);
+  }
 }
 
 template <int DT>
-frt_status launch_dt(frt_act act, frt_quant qm, const void* gu, uint8_t* q, const float* ss, float* bs,
+frt_status launch_dt(frt_act act, int qm, const void* gu, uint8_t* q, const float* ss, float* bs,
                      int64_t total, int NB, int C4, cudaStream_t st) {
   switch (act) {
     case FRT_ACT_GELU_TANH: return launch_act<DT, FRT_ACT_GELU_TANH>(qm, gu, q, ss, bs, total, NB, C4, st);
@@ -165,4 +196,26 @@ extern "C" frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, co
   if (dt == FRT_F16)
     return launch_dt<FRT_F16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
   return launch_dt<FRT_BF16>(act, qm, gate_up, out_fp8, static_scale, block_scales, total, NB, C4, stream);
+}
+
+extern "C" frt_status frt_gate_act_nvfp4(const void* gate_up, uint8_t* out_fp4, uint8_t* out_sf,
+                                         const float* global_scale, int M, int I, frt_act act, frt_dtype dt,
+                                         frt_sf_layout sf_layout, cudaStream_t stream) {
+  using namespace frt;
+  if (M < 0 || I <= 0 || I % 16 != 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
+  if (act != FRT_ACT_GELU_TANH && act != FRT_ACT_SILU && act != FRT_ACT_RELU2) return FRT_ERR_INVALID_ARG;
+  if (sf_layout != FRT_SF_ROW_MAJOR && sf_layout != FRT_SF_SWIZZLED_128X4) return FRT_ERR_INVALID_ARG;
+  if (M == 0) return FRT_OK;
+  if (!gate_up || !aligned(gate_up, 16)) return FRT_ERR_INVALID_ARG;
+  if (!nvfp4_args_ok(sf_layout, global_scale, out_fp4, out_sf, 2)) return FRT_ERR_INVALID_ARG;
+  const int NB = (I + 127) / 128;
+  const int C4 = I / 4;
+  const int64_t total = (int64_t)M * NB;
+  const int64_t grid = (total + (int64_t)kU * kWarps - 1) / ((int64_t)kU * kWarps);
+  if (grid > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
+  const int qm = sf_layout == FRT_SF_ROW_MAJOR ? kQuantNvfp4Rows : kQuantNvfp4Swizzled;
+  float* sf = reinterpret_cast<float*>(out_sf);  // the kernel's scale pointer carries the sf bytes
+  if (dt == FRT_F16)
+    return launch_dt<FRT_F16>(act, qm, gate_up, out_fp4, global_scale, sf, total, NB, C4, stream);
+  return launch_dt<FRT_BF16>(act, qm, gate_up, out_fp4, global_scale, sf, total, NB, C4, stream);
 }

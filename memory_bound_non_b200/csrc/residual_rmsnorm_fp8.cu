@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     }
   }
   float s_static = 0.0f;
-  if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
+  if (QM == FRT_QUANT_STATIC || QM >= kQuantNvfp4Rows) s_static = __ldg(static_scale);
   // Narrow rows (small-batch, latency-bound calls) load the weight with the
   // row instead of after the reduction: one memory round trip less on the
   // critical path.  Wide rows keep the registers for occupancy.
@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   for (int i = 0; i < nw; ++i) tot += red[i];
   const Split32 rstd(rsqrt_f64(tot / (double)D + (double)eps));
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
+  const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * s_static) : 0.0f;  // NVFP4: RN(1 / RN(6 gs))
 
   // Pass 2: y and its FP8 codes.
 #pragma unroll
@@ -145,6 +146,22 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
       if (valid && (t & 15) == 0) block_scales[row * NB + (c >> 4)] = sb;
       if (valid) q[base + c] = quant8(y, Divisor(sb));
+    } else if (QM >= kQuantNvfp4Rows) {
+      // NVFP4: a 16-element block is chunks 2b and 2b+1, held by lanes t and
+      // t ^ 1; codes leave as one 32-bit word per chunk, the scale factor from
+      // the even lane.  q / block_scales carry the code and sf pointers.
+      float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
+      am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+      float reff;
+      const uint32_t sf = nvfp4_scale(am, rden, s_static, &reff);
+      if (valid) {
+        reinterpret_cast<uint32_t*>(q)[base + c] = nvfp4_codes<8>(y, reff);
+        if ((c & 1) == 0) {
+          uint8_t* sfo = reinterpret_cast<uint8_t*>(block_scales);
+          const int nsf = C >> 1;
+          sfo[QM == kQuantNvfp4Rows ? row * nsf + (c >> 1) : sf_offset_swizzled(row, c >> 1, nsf)] = (uint8_t)sf;
+        }
+      }
     } else if (valid) {
       q[base + c] = quant8(y, dv_static);
     }
@@ -160,25 +177,28 @@ frt_status launch_k(const void* x, const void* r_in, void* r_out, const void* w,
                 (float)(C * 8), eps);
 }
 
-template <int DT, int K>
-frt_status launch_dt_k(bool weighted, frt_quant qm, const void* x, const void* r_in, void* r_out, const void* w,
-                 uint8_t* q, const float* ss, float* bs, int M, int C, int NB, int T, float eps,
-                 cudaStream_t st) {
-  if (weighted) {
-    if (qm == FRT_QUANT_STATIC)
-      return launch_k<DT, K, true, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    else
-      return launch_k<DT, K, true, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-  } else {
-    if (qm == FRT_QUANT_STATIC)
-      return launch_k<DT, K, false, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    else
-      return launch_k<DT, K, false, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+template <int DT, int K, bool W>
+frt_status launch_w(int qm, const void* x, const void* r_in, void* r_out, const void* w, uint8_t* q,
+                    const float* ss, float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
+  switch (qm) {
+    case FRT_QUANT_STATIC: return launch_k<DT, K, W, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    case FRT_QUANT_BLOCK128:
+      return launch_k<DT, K, W, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    case kQuantNvfp4Rows: return launch_k<DT, K, W, kQuantNvfp4Rows>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    default: return launch_k<DT, K, W, kQuantNvfp4Swizzled>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
   }
 }
 
+template <int DT, int K>
+frt_status launch_dt_k(bool weighted, int qm, const void* x, const void* r_in, void* r_out, const void* w,
+                       uint8_t* q, const float* ss, float* bs, int M, int C, int NB, int T, float eps,
+                       cudaStream_t st) {
+  return weighted ? launch_w<DT, K, true>(qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st)
+                  : launch_w<DT, K, false>(qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+}
+
 template <int DT>
-frt_status launch_dt(int K, bool weighted, frt_quant qm, const void* x, const void* r_in, void* r_out, const void* w,
+frt_status launch_dt(int K, bool weighted, int qm, const void* x, const void* r_in, void* r_out, const void* w,
                uint8_t* q, const float* ss, float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
   switch (K) {
     case 1: return launch_dt_k<DT, 1>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
@@ -225,4 +245,29 @@ extern "C" frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residu
                               static_scale, block_scales, M, C, NB, T, eps, stream);
   return launch_dt<FRT_BF16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp8,
                              static_scale, block_scales, M, C, NB, T, eps, stream);
+}
+
+extern "C" frt_status frt_residual_rmsnorm_nvfp4(const void* x, const void* residual_in, void* residual_out,
+                                                 const void* weight, uint8_t* out_fp4, uint8_t* out_sf,
+                                                 const float* global_scale, int M, int D, float eps, frt_dtype dt,
+                                                 frt_sf_layout sf_layout, cudaStream_t stream) {
+  using namespace frt;
+  if (M < 0 || D <= 0 || D % 16 != 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
+  if (sf_layout != FRT_SF_ROW_MAJOR && sf_layout != FRT_SF_SWIZZLED_128X4) return FRT_ERR_INVALID_ARG;
+  if (D > 32768) return FRT_ERR_UNSUPPORTED;
+  if (M == 0) return FRT_OK;
+  if (!x || !residual_in || !residual_out) return FRT_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(residual_in, 16) || !aligned(residual_out, 16)) return FRT_ERR_INVALID_ARG;
+  if (weight && !aligned(weight, 16)) return FRT_ERR_INVALID_ARG;
+  if (!nvfp4_args_ok(sf_layout, global_scale, out_fp4, out_sf, 4)) return FRT_ERR_INVALID_ARG;
+  const int C = D / 8;
+  int K, T;
+  rmsnorm_shape(C, &K, &T);
+  const int qm = sf_layout == FRT_SF_ROW_MAJOR ? kQuantNvfp4Rows : kQuantNvfp4Swizzled;
+  float* sf = reinterpret_cast<float*>(out_sf);  // the kernel's scale pointer carries the sf bytes
+  if (dt == FRT_F16)
+    return launch_dt<FRT_F16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp4, global_scale,
+                              sf, M, C, 0, T, eps, stream);
+  return launch_dt<FRT_BF16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp4, global_scale,
+                             sf, M, C, 0, T, eps, stream);
 }

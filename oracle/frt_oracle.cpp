@@ -212,12 +212,14 @@ void quant_block128(const double* y, int64_t n, uint8_t* q, double* scales) {
 //   block    16 consecutive elements of a row share one unsigned e4m3 scale
 //            factor sf; with the per-tensor fp32 global scale gs,
 //            y ~ e2m1 * decode(sf) * gs.
-//   decision in fp32 (as every FP8 decision here): with y32 the fp32 values,
-//            amax32 = max |y32| over the block, den = fp32(6 * gs),
-//            sf = e4m3(amax32 / den) (IEEE fp32 quotient, RNE, saturating to
-//            448), eff = fp32(decode(sf) * gs), code = e2m1(y32 / eff) (IEEE
-//            fp32 quotient); sf == 0 (an all-zero or negligible block) gives
-//            all-zero codes.
+//   decision in fp32 (as every FP8 decision here), scaling by correctly
+//            rounded reciprocals as NVFP4 quantisers do: with y32 the fp32
+//            values and amax32 = max |y32| over the block,
+//              rden = fp32(1 / fp32(6 * gs)),
+//              sf   = e4m3(fp32(amax32 * rden))   (RNE, saturating to 448),
+//              eff  = fp32(decode(sf) * gs),  reff = fp32(1 / eff),
+//              code = e2m1(fp32(y32 * reff));
+//            sf == 0 (an all-zero or negligible block) gives all-zero codes.
 uint8_t e2m1_encode(double v) {
   const uint8_t s = std::signbit(v) ? 0x8 : 0x0;
   const double a = std::fabs(v);
@@ -240,7 +242,7 @@ double e2m1_decode(uint8_t c) {
 // One row of n (a multiple of 16) values -> n/2 packed bytes and n/16 scale
 // factors (row-major).
 void quant_nvfp4_row(const double* y, int64_t n, float gs, uint8_t* packed, uint8_t* sf) {
-  const float den = 6.0f * gs;
+  const float rden = 1.0f / (6.0f * gs);
   for (int64_t b = 0; b < n / 16; ++b) {
     float y32[16];
     float amax = 0.0f;
@@ -248,11 +250,12 @@ void quant_nvfp4_row(const double* y, int64_t n, float gs, uint8_t* packed, uint
       y32[j] = (float)y[16 * b + j];
       amax = std::fmax(amax, std::fabs(y32[j]));
     }
-    const uint8_t code_sf = e4m3_encode((double)(amax / den));
+    const uint8_t code_sf = e4m3_encode((double)(amax * rden));
     sf[b] = code_sf;
     const float eff = (float)e4m3_decode(code_sf) * gs;
+    const float reff = (eff > 0.0f) ? 1.0f / eff : 0.0f;
     uint8_t q[16];
-    for (int j = 0; j < 16; ++j) q[j] = (eff > 0.0f) ? e2m1_encode((double)(y32[j] / eff)) : 0;
+    for (int j = 0; j < 16; ++j) q[j] = (eff > 0.0f) ? e2m1_encode((double)(y32[j] * reff)) : 0;
     for (int j = 0; j < 8; ++j) packed[8 * b + j] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
   }
 }

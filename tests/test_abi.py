@@ -136,3 +136,28 @@ def b8_call(M=4, Hq=8, Hkv=2, hd=128, kc=A, vc=A, qs=0.125, layout=1, kv=1, scal
 ])
 def test_qkv_prepq_host_validation(kw, want):
     assert b8_call(**kw) == want
+
+
+def a4_call(M=4, D=256, x=A, r=A, ro=A, w=None, q=A, sf=A, gs=A, dt=1, lay=0):
+    return frt.load().frt_residual_rmsnorm_nvfp4(x, r, ro, w, q, sf, gs, M, D, 1e-6, dt, lay, None)
+
+
+def c4_call(M=4, I=256, gu=A, q=A, sf=A, gs=A, act=0, dt=1, lay=0):
+    return frt.load().frt_gate_act_nvfp4(gu, q, sf, gs, M, I, act, dt, lay, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(D=8), INV), (dict(D=24), INV), (dict(lay=2), INV), (dict(gs=None), INV), (dict(gs=A + 2), INV),
+    (dict(sf=None), INV), (dict(q=A + 2), INV), (dict(x=A + 8), INV), (dict(D=32784), UNSUP), (dict(M=0), OK),
+    (dict(M=0, lay=5), INV), (dict(M=-1), INV), (dict(dt=3), INV),
+])
+def test_residual_rmsnorm_nvfp4_host_validation(kw, want):
+    assert a4_call(**kw) == want
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(I=8), INV), (dict(I=20), INV), (dict(lay=-1), INV), (dict(gs=None), INV), (dict(sf=None), INV),
+    (dict(q=A + 1), INV), (dict(gu=A + 4), INV), (dict(act=7), INV), (dict(M=0), OK), (dict(M=0, I=20), INV),
+])
+def test_gate_act_nvfp4_host_validation(kw, want):
+    assert c4_call(**kw) == want

@@ -376,3 +376,162 @@ def test_prepq_large_m_sampled(M):
     mask = torch.ones(wl.capacity, dtype=torch.bool, device=DEV)
     mask[inp.positions.long()] = False
     assert bool((kc[mask] == 0x7E).all()) and bool((vc[mask] == 0x7E).all())
+
+
+# ================================================================== NEXT-3 ===
+# NVFP4 outputs of ops (a) and (c): e2m1 codes in 16-element blocks with e4m3
+# scale factors and a global fp32 scale, scale factors row-major or in the
+# 128x4-swizzled layout of block-scaled GEMMs.
+
+def unpack_e2m1(packed):
+    p = np.asarray(packed, dtype=np.uint8)
+    return np.stack([p & 0xF, p >> 4], axis=-1).reshape(*p.shape[:-1], p.shape[-1] * 2)
+
+
+def assert_e2m1_codes(gpu, ref, max_frac=0.0, what="e2m1"):
+    g, o = unpack_e2m1(gpu).ravel().astype(np.int32), unpack_e2m1(ref).ravel().astype(np.int32)
+    gm, om = g & 7, o & 7
+    same = (g == o) | ((gm == 0) & (om == 0))
+    diff = ~same
+    n = int(diff.sum())
+    if n:
+        bad = (np.abs(gm[diff] - om[diff]) != 1) | (((g[diff] ^ o[diff]) & 8) != 0) & (gm[diff] != 0) & (om[diff] != 0)
+        assert not bad.any(), "%s: %d codes differ by more than one step" % (what, int(bad.sum()))
+    assert n <= max_frac * g.size, "%s: %d of %d codes one step off" % (what, n, g.size)
+    return n
+
+
+def global_scale_for(vals):
+    """gs so the largest block scale lands near the top of e4m3: amax / (6 * 448)."""
+    return float(np.float32(np.abs(vals).max() / (6.0 * 448.0)))
+
+
+def run_a_nvfp4(x, r, w, gs, sf_layout="rows", inplace=True):
+    M, D = x.shape
+    xd, rd = x.to(DEV), r.to(DEV).clone()
+    ro = rd if inplace else torch.empty_like(rd)
+    q_raw, q = guarded((M, D // 2), torch.uint8, 0xA5)
+    nsf = frt.nvfp4_sf_bytes(M, D, sf_layout)
+    sf_raw, sf = guarded((nsf,), torch.uint8, 0)
+    gsd = torch.tensor([gs], dtype=torch.float32, device=DEV)
+    frt.frt_residual_rmsnorm_nvfp4(xd, rd, ro, None if w is None else w.to(DEV), q, sf, gsd, sf_layout=sf_layout)
+    torch.cuda.synchronize()
+    assert_guard(q_raw, M * D // 2, 0xA5)
+    assert_guard(sf_raw, nsf, 0)
+    return ro, q, sf
+
+
+A4_CASES = [("pi05", {}), ("vla_denoise", {}), ("vit", {}), ("tiny", {"M": 3, "D": 16}),
+            ("tiny", {"M": 5, "D": 1040}), ("large_m_M4096", {"M": 300}), ("vit", {"M": 2, "D": 32768}),
+            ("tiny", {"M": 130, "D": 2048, "dt": "bf16"})]
+
+
+@pytest.mark.parametrize("name,ov", A4_CASES, ids=["%s%s" % (n, "".join("-%s%s" % kv for kv in o.items()))
+                                                   for n, o in A4_CASES])
+@pytest.mark.parametrize("sf_layout", ["rows", "swizzled"])
+def test_residual_rmsnorm_nvfp4_parity(name, ov, sf_layout):
+    wl = W.get(name, **ov)
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False)
+    L = inp.layers[0]
+    x, r = W.bits16(L.x_attn), W.bits16(inp.residual)
+    w = None if L.w_attn is None else W.bits16(L.w_attn)
+    y = oracle.residual_rmsnorm_fp8(x, r, w, wl.eps, wl.dt, "block128", want_y=True)["y"]
+    gs = global_scale_for(y)
+    ro, q, sf = run_a_nvfp4(L.x_attn, inp.residual, L.w_attn, gs, sf_layout)
+    o = oracle.residual_rmsnorm_nvfp4(x, r, w, wl.eps, wl.dt, gs)
+    np.testing.assert_array_equal(W.bits16(ro.cpu()), o["residual_out"])
+    assert_e2m1_codes(q.cpu().numpy(), o["out_fp4"], what="op a e2m1")
+    want_sf = o["sf"].ravel() if sf_layout == "rows" else oracle.sf_swizzle(o["sf"])
+    np.testing.assert_array_equal(sf.cpu().numpy(), want_sf)
+
+
+@pytest.mark.parametrize("gs", [1e-6, 1e4])
+def test_residual_rmsnorm_nvfp4_scale_saturation_and_underflow(gs):
+    """A tiny global scale saturates every block scale at 448 (codes saturate
+    at 6); a huge one rounds small blocks' scales to 0 (all-zero codes)."""
+    wl = W.get("vla_denoise", M=9)
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False)
+    L = inp.layers[0]
+    x, r, w = W.bits16(L.x_attn), W.bits16(inp.residual), W.bits16(L.w_attn)
+    ro, q, sf = run_a_nvfp4(L.x_attn, inp.residual, L.w_attn, gs)
+    o = oracle.residual_rmsnorm_nvfp4(x, r, w, wl.eps, wl.dt, gs)
+    np.testing.assert_array_equal(sf.cpu().numpy(), o["sf"].ravel())
+    assert_e2m1_codes(q.cpu().numpy(), o["out_fp4"], what="op a e2m1")
+    assert (o["sf"] == 0x7E).all() if gs < 1 else (o["sf"] == 0).all()
+
+
+def run_c_nvfp4(gu, gs, act, sf_layout="rows"):
+    M, two_i = gu.shape
+    I = two_i // 2
+    q_raw, q = guarded((M, I // 2), torch.uint8, 0xA5)
+    nsf = frt.nvfp4_sf_bytes(M, I, sf_layout)
+    sf_raw, sf = guarded((nsf,), torch.uint8, 0)
+    gsd = torch.tensor([gs], dtype=torch.float32, device=DEV)
+    frt.frt_gate_act_nvfp4(gu.to(DEV), q, sf, gsd, act=act, sf_layout=sf_layout)
+    torch.cuda.synchronize()
+    assert_guard(q_raw, M * I // 2, 0xA5)
+    assert_guard(sf_raw, nsf, 0)
+    return q, sf
+
+
+C4_CASES = [("pi05", {}), ("vla_denoise", {}), ("vit", {}), ("tiny", {"M": 1, "I": 16}),
+            ("tiny", {"M": 3, "I": 48, "act": "relu2"}), ("large_m_M4096", {"M": 160})]
+
+
+@pytest.mark.parametrize("name,ov", C4_CASES, ids=["%s%s" % (n, "".join("-%s%s" % kv for kv in o.items()))
+                                                   for n, o in C4_CASES])
+@pytest.mark.parametrize("sf_layout", ["rows", "swizzled"])
+def test_gate_act_nvfp4_parity(name, ov, sf_layout):
+    wl = W.get(name, **ov)
+    gu = W.make_inputs(wl, n_layers=1, with_caches=False).layers[0].gate_up
+    hb = W.bits16(gu)
+    a = oracle.gate_act_fp8(hb, wl.act, wl.dt, "block128", want_a=True)["a"]
+    gs = global_scale_for(a)
+    q, sf = run_c_nvfp4(gu, gs, wl.act, sf_layout)
+    o = oracle.gate_act_nvfp4(hb, wl.act, wl.dt, gs)
+    exact = wl.act == "relu2"
+    assert_e2m1_codes(q.cpu().numpy(), o["out_fp4"], max_frac=0.0 if exact else 1e-3, what="op c e2m1")
+    want_sf = o["sf"].ravel() if sf_layout == "rows" else oracle.sf_swizzle(o["sf"])
+    got_sf = sf.cpu().numpy()
+    if exact:
+        np.testing.assert_array_equal(got_sf, want_sf)
+    else:
+        step = np.abs(got_sf.astype(int) - want_sf.astype(int))   # positive e4m3 codes: adjacent = 1 apart
+        assert (step <= 1).all() and (step > 0).mean() <= 1e-3
+
+
+def test_nvfp4_large_m_sampled():
+    """Full-size launches (65536 x 4096 norm, 16384 x 16384 gate), sampled rows
+    against the oracle."""
+    M, D = 65536, 4096
+    wl = W.get("large_m_M65536")
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False, device=DEV)
+    L = inp.layers[0]
+    rows = np.unique(np.concatenate([np.random.default_rng(3).choice(M, 192, replace=False), [0, M - 1]]))
+    ti = torch.as_tensor(rows, device=DEV)
+    x, r, w = W.bits16(L.x_attn[ti].cpu()), W.bits16(inp.residual[ti].cpu()), W.bits16(L.w_attn.cpu())
+    gs = global_scale_for(oracle.residual_rmsnorm_fp8(x, r, w, wl.eps, wl.dt, "block128", want_y=True)["y"])
+    q = torch.empty((M, D // 2), dtype=torch.uint8, device=DEV)
+    sf = torch.empty((M * D // 16,), dtype=torch.uint8, device=DEV)
+    rr = inp.residual.clone()
+    frt.frt_residual_rmsnorm_nvfp4(L.x_attn, rr, rr, L.w_attn, q, sf,
+                                   torch.tensor([gs], dtype=torch.float32, device=DEV))
+    torch.cuda.synchronize()
+    o = oracle.residual_rmsnorm_nvfp4(x, r, w, wl.eps, wl.dt, gs)
+    np.testing.assert_array_equal(W.bits16(rr[ti].cpu()), o["residual_out"])
+    assert_e2m1_codes(q[ti].cpu().numpy(), o["out_fp4"], what="large-M op a e2m1")
+    np.testing.assert_array_equal(sf.view(M, D // 16)[ti].cpu().numpy(), o["sf"])
+    # op c on the first 16384 rows of the large-M gate/up buffer
+    Mc, I = 16384, wl.I
+    gu = L.gate_up[:Mc]
+    rows = rows[rows < Mc]
+    tc = torch.as_tensor(rows, device=DEV)
+    hb = W.bits16(gu[tc].cpu())
+    gs = global_scale_for(oracle.gate_act_fp8(hb, wl.act, wl.dt, "block128", want_a=True)["a"])
+    q = torch.empty((Mc, I // 2), dtype=torch.uint8, device=DEV)
+    sf = torch.empty((Mc * I // 16,), dtype=torch.uint8, device=DEV)
+    frt.frt_gate_act_nvfp4(gu, q, sf, torch.tensor([gs], dtype=torch.float32, device=DEV), act=wl.act)
+    torch.cuda.synchronize()
+    o = oracle.gate_act_nvfp4(hb, wl.act, wl.dt, gs)
+    assert_e2m1_codes(q[tc].cpu().numpy(), o["out_fp4"], what="large-M op c e2m1")
+    np.testing.assert_array_equal(sf.view(Mc, I // 16)[tc].cpu().numpy(), o["sf"])

@@ -226,23 +226,23 @@ def test_e2m1_ties_to_even_and_saturation():
 
 
 def _nvfp4_brute(y, gs):
-    """The NVFP4 reading restated with numpy fp32 scalars and brute-force
-    nearest-code searches (e4m3 via the whole code table, e2m1 over its 8
-    magnitudes, ties to the even code)."""
+    """The NVFP4 reading restated with numpy fp32 scalars (scaling by correctly
+    rounded reciprocals) and brute-force nearest-code searches (e4m3 via the
+    whole code table, e2m1 over its 8 magnitudes, ties to the even code)."""
     y32 = np.asarray(y, dtype=np.float32)
     packed, sfs = [], []
     for b in range(len(y32) // 16):
         blk = y32[16 * b:16 * b + 16]
         amax = np.float32(np.max(np.abs(blk)))
-        den = np.float32(6.0) * np.float32(gs)
-        sf = int(_nearest_e4m3(np.array([float(np.float32(amax / den))]))[0])
+        rden = np.float32(np.float32(1.0) / (np.float32(6.0) * np.float32(gs)))
+        sf = int(_nearest_e4m3(np.array([float(np.float32(amax * rden))]))[0])
         eff = np.float32(np.float32(oracle.e4m3_decode(sf)) * np.float32(gs))
         codes = []
         for v in blk:
             if eff == 0:
                 codes.append(0)
                 continue
-            t = float(np.float32(v / eff))
+            t = float(np.float32(v * np.float32(np.float32(1.0) / eff)))
             a = min(abs(t), 6.0)
             d = [abs(m - a) for m in E2M1]
             best = [k for k in range(8) if d[k] == min(d)]
