@@ -91,6 +91,14 @@ def lib():
         L.oracle_gate_act_nvfp4.argtypes = [c.c_void_p] * 3 + [c.c_double, c.c_void_p, c.c_int64, c.c_int64,
                                                                c.c_int, c.c_int]
         L.oracle_gate_act_nvfp4.restype = c.c_int
+        L.oracle_layernorm.argtypes = [c.c_void_p, c.c_int64, c.c_void_p, c.c_void_p, c.c_double, c.c_void_p]
+        L.oracle_layernorm.restype = None
+        L.oracle_residual_layernorm_quant.argtypes = ([c.c_void_p] * 6 + [c.c_double, c.c_void_p, c.c_void_p,
+                                                       c.c_double, c.c_void_p, c.c_int64, c.c_int64, c.c_double,
+                                                       c.c_int, c.c_int])
+        L.oracle_residual_layernorm_quant.restype = c.c_int
+        L.oracle_qkv_layernorm_rope_kvcache.argtypes = [c.c_void_p] * 13 + [c.c_int64] * 6 + [c.c_double, c.c_int]
+        L.oracle_qkv_layernorm_rope_kvcache.restype = c.c_int
         _lib = L
     return _lib
 
@@ -345,3 +353,60 @@ def sf_swizzle(sf_rowmajor):
         for c in range(C):
             out[sf_swizzle_offset(r, c, C)] = sf_rowmajor[r, c]
     return out
+
+
+# ------------------------------------------------------------------ NEXT-4 --
+def layernorm(h, w=None, b=None, eps=1e-6):
+    h = np.ascontiguousarray(h, dtype=np.float64)
+    y = np.empty_like(h)
+    wv = None if w is None else np.ascontiguousarray(w, dtype=np.float64)
+    bv = None if b is None else np.ascontiguousarray(b, dtype=np.float64)
+    lib().oracle_layernorm(_p(h), h.shape[0], _p(wv), _p(bv), float(eps), _p(y))
+    return y
+
+
+def residual_layernorm(x, residual_in, weight, bias, eps, dt, quant, static_scale=None, global_scale=None,
+                       want_y=False):
+    """Op (a) with LayerNorm.  quant: "static" / "block128" (FP8, out [M, D])
+    or "nvfp4" (out [M, D/2] + sf [M, D/16])."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    r = np.ascontiguousarray(residual_in, dtype=np.uint16)
+    M, D = x.shape
+    w = None if weight is None else np.ascontiguousarray(weight, dtype=np.uint16)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+    mode = {"static": 0, "block128": 1, "nvfp4": 2}[quant]
+    r_out = np.empty_like(r)
+    q = np.empty((M, D // 2) if mode == 2 else (M, D), dtype=np.uint8)
+    bs = np.empty((M, (D + 127) // 128), dtype=np.float64) if mode == 1 else None
+    sf = np.empty((M, D // 16), dtype=np.uint8) if mode == 2 else None
+    y = np.empty((M, D), dtype=np.float64) if want_y else None
+    rc = lib().oracle_residual_layernorm_quant(_p(x), _p(r), _p(r_out), _p(w), _p(b), _p(q),
+                                               float(static_scale or 0.0), _p(bs), _p(sf), float(global_scale or 0.0),
+                                               _p(y), M, D, _f32(eps), _DT[dt], mode)
+    if rc != 0:
+        raise ValueError("oracle_residual_layernorm_quant: bad argument")
+    return {"residual_out": r_out, "out": q, "block_scales": bs, "sf": sf, "y": y}
+
+
+def qkv_layernorm_rope_kvcache(qkv, q_w, q_b, k_w, k_b, cos_tab, sin_tab, positions, Hq, Hkv, hd, capacity, eps, dt,
+                               slots=None, v_cache=None):
+    """Op (b) with per-head LayerNorm ([Hq, hd] / [Hkv, hd] affine, each
+    optional).  Returns q_out (fp64), k_cache (fp64), v_cache (uint16), status."""
+    qkv = np.ascontiguousarray(qkv, dtype=np.uint16)
+    M = qkv.shape[0]
+    cos_tab = np.ascontiguousarray(cos_tab, dtype=np.float32)
+    sin_tab = np.ascontiguousarray(sin_tab, dtype=np.float32)
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    sl = None if slots is None else np.ascontiguousarray(slots, dtype=np.int64)
+    prm = [None if a is None else np.ascontiguousarray(a, dtype=np.uint16) for a in (q_w, q_b, k_w, k_b)]
+    q_out = np.full((M, Hq, hd), np.nan, dtype=np.float64)
+    kc = np.full((capacity, Hkv, hd), np.nan, dtype=np.float64)
+    vc = (np.zeros((capacity, Hkv, hd), dtype=np.uint16) if v_cache is None
+          else np.array(v_cache, dtype=np.uint16, copy=True))
+    status = np.zeros(1, dtype=np.int32)
+    rc = lib().oracle_qkv_layernorm_rope_kvcache(_p(qkv), *[_p(a) for a in prm], _p(cos_tab), _p(sin_tab), _p(pos),
+                                                 _p(sl), _p(q_out), _p(kc), _p(vc), _p(status), M, Hq, Hkv, hd,
+                                                 cos_tab.shape[0], capacity, _f32(eps), _DT[dt])
+    if rc != 0:
+        raise ValueError("oracle_qkv_layernorm_rope_kvcache: bad argument")
+    return {"q_out": q_out, "k_cache": kc, "v_cache": vc, "status": int(status[0])}

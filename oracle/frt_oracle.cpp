@@ -283,6 +283,19 @@ void rmsnorm(const double* h, int64_t n, const double* w, double eps, double* y)
   for (int64_t j = 0; j < n; ++j) y[j] = h[j] * rstd * (w ? w[j] : 1.0);
 }
 
+// LayerNorm (NEXT-4): y_j = (h_j - mean) / sqrt(var + eps) * w_j + b_j with
+// mean and var (biased) over the n values, in two passes; w or b null means
+// 1 or 0.
+void layernorm(const double* h, int64_t n, const double* w, const double* b, double eps, double* y) {
+  double sum = 0.0;
+  for (int64_t j = 0; j < n; ++j) sum += h[j];
+  const double mean = sum / (double)n;
+  double ss = 0.0;
+  for (int64_t j = 0; j < n; ++j) ss += (h[j] - mean) * (h[j] - mean);
+  const double rstd = 1.0 / std::sqrt(ss / (double)n + eps);
+  for (int64_t j = 0; j < n; ++j) y[j] = (h[j] - mean) * rstd * (w ? w[j] : 1.0) + (b ? b[j] : 0.0);
+}
+
 // Rotate-half RoPE ([FR] §2.2, second bullet): for j < n/2 the pair
 // (v_j, v_{j+n/2}) is rotated by the angle whose cosine and sine are c_j, s_j.
 void rope_rotate_half(double* v, int n, const float* c, const float* s) {
@@ -634,6 +647,95 @@ int oracle_gate_act_nvfp4(const uint16_t* gate_up, uint8_t* out_fp4, uint8_t* sf
     for (int64_t j = 0; j < I; ++j) a[j] = act_fn(act, decode16(row[2 * j], f)) * decode16(row[2 * j + 1], f);
     if (a_out) std::memcpy(a_out + i * I, a.data(), sizeof(double) * I);
     quant_nvfp4_row(a.data(), I, (float)global_scale, out_fp4 + i * I / 2, sf + i * I / 16);
+  }
+  return 0;
+}
+
+// ------------------------------------------------------------- NEXT-4 --
+void oracle_layernorm(const double* h, int64_t n, const double* w, const double* b, double eps, double* y) {
+  layernorm(h, n, w, b, eps, y);
+}
+
+// Op (a) with LayerNorm (the ViT "add_layer_norm" producer): h as op (a);
+// y = LayerNorm(h) with weight / bias ([D] 16-bit, each optional); output
+// FP8 (qm 0 / 1 as op (a)) or NVFP4 (out_fp4 [M, D/2], sf [M, D/16], gs).
+int oracle_residual_layernorm_quant(const uint16_t* x, const uint16_t* residual_in, uint16_t* residual_out,
+                                    const uint16_t* weight, const uint16_t* bias, uint8_t* out_q, double static_scale,
+                                    double* block_scales, uint8_t* sf, double global_scale, double* y_out, int64_t M,
+                                    int64_t D, double eps, int dt, int mode) {
+  // mode 0: FP8 static, 1: FP8 block-128, 2: NVFP4
+  if (M < 0 || D <= 0 || !x || !residual_in || !residual_out || !out_q) return -1;
+  if ((mode == 1 && !block_scales) || (mode == 2 && (!sf || D % 16 != 0))) return -1;
+  const Fmt16 f = fmt_of(dt);
+  const int64_t nb = (D + 127) / 128;
+  std::vector<double> h(D), w(D), b(D), y(D);
+  for (int64_t j = 0; j < D; ++j) {
+    if (weight) w[j] = decode16(weight[j], f);
+    if (bias) b[j] = decode16(bias[j], f);
+  }
+  for (int64_t i = 0; i < M; ++i) {
+    for (int64_t j = 0; j < D; ++j) {
+      double s, err;
+      two_sum(decode16(x[i * D + j], f), decode16(residual_in[i * D + j], f), &s, &err);
+      const uint16_t hb = round16(s, err, f);
+      residual_out[i * D + j] = hb;
+      h[j] = decode16(hb, f);
+    }
+    layernorm(h.data(), D, weight ? w.data() : nullptr, bias ? b.data() : nullptr, eps, y.data());
+    if (y_out) std::memcpy(y_out + i * D, y.data(), sizeof(double) * D);
+    if (mode == 0)
+      quant_static(y.data(), D, static_scale, out_q + i * D);
+    else if (mode == 1)
+      quant_block128(y.data(), D, out_q + i * D, block_scales + i * nb);
+    else
+      quant_nvfp4_row(y.data(), D, (float)global_scale, out_q + i * D / 2, sf + i * D / 16);
+  }
+  return 0;
+}
+
+// Op (b) with per-head LayerNorm on Q and K (the Chameleon prefill kernel:
+// LayerNorm(Q) + LayerNorm(K) + rotate-half RoPE, [FR] §2.2 second bullet).
+// q_w / q_b are [Hq, hd], k_w / k_b [Hkv, hd] (per-head affine), each
+// optional; everything else as op (b).
+int oracle_qkv_layernorm_rope_kvcache(const uint16_t* qkv, const uint16_t* q_w, const uint16_t* q_b,
+                                      const uint16_t* k_w, const uint16_t* k_b, const float* cos_tab,
+                                      const float* sin_tab, const int32_t* positions, const int64_t* slots,
+                                      double* q_out, double* k_cache, uint16_t* v_cache, int32_t* status, int64_t M,
+                                      int64_t Hq, int64_t Hkv, int64_t hd, int64_t max_pos, int64_t capacity,
+                                      double eps, int dt) {
+  if (M < 0 || Hq <= 0 || Hkv <= 0 || hd <= 0 || hd % 2 != 0) return -1;
+  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return -1;
+  const Fmt16 f = fmt_of(dt);
+  const int64_t width = (Hq + 2 * Hkv) * hd;
+  const int64_t half = hd / 2;
+  std::vector<double> v(hd), w(hd), b(hd), y(hd);
+  for (int64_t i = 0; i < M; ++i) {
+    const int64_t p = positions[i];
+    const int64_t slot = slots ? slots[i] : p;
+    if (p < 0 || p >= max_pos || slot < 0 || slot >= capacity) {
+      if (status) *status |= 1;
+      continue;
+    }
+    const float* c = cos_tab + p * half;
+    const float* s = sin_tab + p * half;
+    const uint16_t* row = qkv + i * width;
+    for (int64_t h = 0; h < Hq + Hkv; ++h) {
+      const bool is_q = h < Hq;
+      const int64_t hh = is_q ? h : h - Hq;
+      const uint16_t* pw = is_q ? q_w : k_w;
+      const uint16_t* pb = is_q ? q_b : k_b;
+      for (int64_t j = 0; j < hd; ++j) {
+        v[j] = decode16(row[h * hd + j], f);
+        if (pw) w[j] = decode16(pw[hh * hd + j], f);
+        if (pb) b[j] = decode16(pb[hh * hd + j], f);
+      }
+      layernorm(v.data(), hd, pw ? w.data() : nullptr, pb ? b.data() : nullptr, eps, y.data());
+      rope_rotate_half(y.data(), (int)hd, c, s);
+      double* dst = is_q ? q_out + (i * Hq + h) * hd : k_cache + (slot * Hkv + hh) * hd;
+      std::memcpy(dst, y.data(), sizeof(double) * hd);
+    }
+    for (int64_t g = 0; g < Hkv; ++g)
+      std::memcpy(v_cache + (slot * Hkv + g) * hd, row + (Hq + Hkv + g) * hd, sizeof(uint16_t) * hd);
   }
   return 0;
 }

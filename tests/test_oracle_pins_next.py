@@ -331,3 +331,80 @@ def test_sf_swizzle_layout():
     M = 300
     offs = {oracle.sf_swizzle_offset(r, c, C) for r in range(((M + 127) // 128) * 128) for c in range(atoms * 4)}
     assert offs == set(range(((M + 127) // 128) * 128 * atoms * 4))   # a bijection onto the padded array
+
+
+# ------------------------------------------------------------------ NEXT-4 --
+# LayerNorm variants: the ViT add + LayerNorm producer (op (a) with LayerNorm)
+# and the Chameleon LayerNorm(Q) + LayerNorm(K) + RoPE kernel ("FlashRT kernel
+# fusion", §2.2 second bullet).
+
+def test_layernorm_closed_form_and_invariants():
+    np.testing.assert_allclose(oracle.layernorm(np.array([1.0, 2.0, 3.0, 4.0]), eps=0.0),
+                               np.array([-3, -1, 1, 3]) / math.sqrt(5.0), rtol=1e-15)
+    g = W.generator(21)
+    h = torch.randn(512, generator=g, dtype=torch.float64).numpy() * 3 + 7
+    y = oracle.layernorm(h, eps=0.0)
+    assert abs(y.mean()) < 1e-14 and abs((y * y).mean() - 1.0) < 1e-13
+    np.testing.assert_allclose(oracle.layernorm(h + 1000.0, eps=0.0), y, atol=1e-10)     # shift invariance
+    np.testing.assert_allclose(oracle.layernorm(h * 0.25, eps=0.0), y, rtol=1e-13, atol=1e-14)
+
+
+def test_layernorm_matches_torch():
+    g = W.generator(22)
+    h = torch.randn(4, 384, generator=g, dtype=torch.float64)
+    w = torch.randn(384, generator=g, dtype=torch.float64)
+    b = torch.randn(384, generator=g, dtype=torch.float64)
+    ref = torch.nn.functional.layer_norm(h, (384,), w, b, eps=1e-5).numpy()
+    for i in range(4):
+        np.testing.assert_allclose(oracle.layernorm(h[i].numpy(), w.numpy(), b.numpy(), 1e-5), ref[i], rtol=1e-12,
+                                   atol=1e-12)
+    ref = torch.nn.functional.layer_norm(h, (384,), None, None, eps=1e-5).numpy()
+    np.testing.assert_allclose(oracle.layernorm(h[0].numpy(), eps=1e-5), ref[0], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("quant", ["static", "block128", "nvfp4"])
+def test_residual_layernorm_composes_op_a_pieces(quant):
+    x, r, _, _, _ = _inputs(3, 256, "bf16", 23, 1)
+    g = W.generator(23)
+    w = W.bits16(W.norm_weight(256, "bf16", g))
+    b = W.bits16(W.normal16((256,), "bf16", g, scale=0.1))
+    o = oracle.residual_layernorm(x, r, w, b, 1e-6, "bf16", quant, static_scale=0.01, global_scale=0.002,
+                                  want_y=True)
+    a = oracle.residual_rmsnorm_fp8(x, r, None, 1e-6, "bf16", "static", static_scale=0.01)
+    np.testing.assert_array_equal(o["residual_out"], a["residual_out"])
+    h = oracle.decode16(o["residual_out"], "bf16")
+    for i in range(3):
+        y = torch.nn.functional.layer_norm(torch.from_numpy(h[i]), (256,),
+                                           torch.from_numpy(oracle.decode16(w, "bf16")),
+                                           torch.from_numpy(oracle.decode16(b, "bf16")),
+                                           eps=float(np.float32(1e-6))).numpy()
+        np.testing.assert_allclose(o["y"][i], y, rtol=1e-12, atol=1e-12)
+        if quant == "nvfp4":
+            p, s = oracle.quant_nvfp4_row(o["y"][i], 0.002)
+            np.testing.assert_array_equal(o["out"][i], p)
+            np.testing.assert_array_equal(o["sf"][i], s)
+        elif quant == "static":
+            np.testing.assert_array_equal(o["out"][i], oracle.quant_static(o["y"][i], 0.01))
+
+
+def test_qkv_layernorm_per_head_affine_and_rope():
+    M, Hq, Hkv, hd = 3, 4, 2, 16
+    qkv, _, _, cos, sin, pos = _qkv_inputs(M=M, Hq=Hq, Hkv=Hkv, hd=hd, qk_norm=False)
+    g = W.generator(24)
+    qw = W.bits16(W.normal16((Hq, hd), "bf16", g))
+    qb = W.bits16(W.normal16((Hq, hd), "bf16", g, scale=0.1))
+    kw = W.bits16(W.normal16((Hkv, hd), "bf16", g))
+    o = oracle.qkv_layernorm_rope_kvcache(qkv, qw, qb, kw, None, cos, sin, pos, Hq, Hkv, hd, 16, 1e-6, "bf16")
+    v = oracle.decode16(qkv, "bf16").reshape(M, Hq + 2 * Hkv, hd)
+    for i in range(M):
+        for h in range(Hq + Hkv):
+            is_q = h < Hq
+            w = oracle.decode16((qw if is_q else kw)[h if is_q else h - Hq], "bf16")
+            bb = oracle.decode16(qb[h], "bf16") if is_q else None
+            y = torch.nn.functional.layer_norm(torch.from_numpy(v[i, h]), (hd,), torch.from_numpy(w),
+                                               None if bb is None else torch.from_numpy(bb),
+                                               eps=float(np.float32(1e-6))).numpy()
+            y = oracle.rope_rotate_half(y, cos[pos[i]], sin[pos[i]])
+            got = o["q_out"][i, h] if is_q else o["k_cache"][pos[i], h - Hq]
+            np.testing.assert_allclose(got, y, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(o["v_cache"][pos], qkv.reshape(M, Hq + 2 * Hkv, hd)[:, Hq + Hkv:])
