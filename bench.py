@@ -487,7 +487,44 @@ def next_ops_leg(peak, floor, reps=50, big_m=65536):
                     "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
                     "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4), "sf_layout": "rows",
                     "traffic": measured_traffic(key, "nvfp4")}
-    del x, r, q, sf, gu, qc, sfc
+    del q, sf, gu, qc, sfc
+    # NEXT-4: the LayerNorm producer (weight + bias, static FP8) on the norm
+    # shape, and the per-head LayerNorm(Q/K) + RoPE op on the QKV shape.
+    bvec = W.normal16((D,), "bf16", g, scale=0.2)
+    q8 = torch.empty((big_m, D), dtype=torch.uint8, device="cuda")
+    ss8 = torch.tensor([0.02], dtype=torch.float32, device="cuda")
+    H, hd = wl.Hq + 2 * wl.Hkv, wl.hd
+    qkv = W.normal16((big_m, H * hd), "bf16", g)
+    qlw, qlb = W.normal16((wl.Hq, hd), "bf16", g), W.normal16((wl.Hq, hd), "bf16", g, scale=0.1)
+    klw, klb = W.normal16((wl.Hkv, hd), "bf16", g), W.normal16((wl.Hkv, hd), "bf16", g, scale=0.1)
+    cos, sin = W.rope_tables(wl.capacity, hd, wl.theta)
+    cos, sin = cos.cuda(), sin.cuda()
+    pos = W.positions(wl, g)
+    q_out = torch.empty((big_m, wl.Hq, hd), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((wl.capacity, wl.Hkv, hd), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    cases = [("residual_layernorm_fp8_M%d_D%d" % (big_m, D), big_m * D * 7 + 4 * D,
+              lambda: frt.frt_residual_layernorm_fp8(x, r, r, w, bvec, q8, static_scale=ss8)),
+             ("qkv_layernorm_rope_M%d" % big_m, big_m * (H * hd * 4 + hd * 4 + 4) + 4 * (wl.Hq + wl.Hkv) * hd,
+              lambda: frt.frt_qkv_layernorm_rope_kvcache(qkv, qlw, qlb, klw, klb, cos, sin, pos, q_out, kc, vc,
+                                                         wl.Hq, wl.Hkv, hd))]
+    for key, nbytes, fn in cases:
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+        for i in range(reps):
+            ev[2 * i].record(s)
+            fn()
+            ev[2 * i + 1].record(s)
+        torch.cuda.synchronize()
+        ts = [ev[2 * i].elapsed_time(ev[2 * i + 1]) * 1e3 for i in range(reps)]
+        us = sum(ts) / len(ts)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[key] = {"us_mean": round(us, 2), "us_median": round(statistics.median(ts), 2), "bytes": int(nbytes),
+                    "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                    "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4), "traffic": measured_traffic(key, "layernorm")}
+    del x, r, q8, qkv, q_out, kc, vc
     return out
 
 

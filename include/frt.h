@@ -198,6 +198,42 @@ frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* 
                             cudaStream_t stream);
 
 /*
+ * NEXT-4: LayerNorm variants.
+ *
+ * frt_residual_layernorm_fp8 / _nvfp4: the ViT "add_layer_norm" producer (the
+ * FlashRT port's census: add_layer_norm_to_nvfp4).  Op (a) / its NVFP4 form
+ * with LayerNorm in place of RMSNorm:
+ *   h = x + residual (rounded once, written back);
+ *   y = (h - mean) / sqrt(var + eps) * weight + bias, mean and (biased) var
+ *       over the row, y rounded once to fp32;
+ *   then FP8 (static / block-128) or NVFP4 exactly as the RMSNorm ops.
+ *   weight, bias: device [D] 16-bit, 16-byte aligned, each optional (NULL:
+ *   1 / 0).  Other arguments and rules as frt_residual_rmsnorm_fp8 /
+ *   frt_residual_rmsnorm_nvfp4.
+ *
+ * frt_qkv_layernorm_rope_kvcache: "FlashRT kernel fusion", §2.2 second bullet
+ * (the Chameleon prefill kernel: LayerNorm(Q) + LayerNorm(K) + rotate-half
+ * RoPE in one kernel).  Op (b) with a per-head LayerNorm over hd in place of
+ * the RMSNorm:  v' = (v - mean) / sqrt(var + eps) * w[h] + b[h], with
+ * per-head affine rows q_w, q_b [Hq, hd] and k_w, k_b [Hkv, hd] (device
+ * 16-bit, each optional).  Other arguments, layouts and status bit 0 as
+ * frt_qkv_norm_rope_kvcache.
+ */
+frt_status frt_residual_layernorm_fp8(const void* x, const void* residual_in, void* residual_out, const void* weight,
+                                      const void* bias, uint8_t* out_fp8, const float* static_scale,
+                                      float* block_scales, int M, int D, float eps, frt_dtype dt, frt_quant qm,
+                                      cudaStream_t stream);
+frt_status frt_residual_layernorm_nvfp4(const void* x, const void* residual_in, void* residual_out,
+                                        const void* weight, const void* bias, uint8_t* out_fp4, uint8_t* out_sf,
+                                        const float* global_scale, int M, int D, float eps, frt_dtype dt,
+                                        frt_sf_layout sf_layout, cudaStream_t stream);
+frt_status frt_qkv_layernorm_rope_kvcache(const void* qkv, const void* q_w, const void* q_b, const void* k_w,
+                                          const void* k_b, const float* cos_tab, const float* sin_tab,
+                                          const int32_t* positions, void* q_out, void* k_cache, void* v_cache,
+                                          int32_t* status, int M, int Hq, int Hkv, int hd, int max_pos,
+                                          int capacity, float eps, frt_dtype dt, cudaStream_t stream);
+
+/*
  * NEXT-3: NVFP4 outputs of ops (a) and (c).  The FlashRT port's NVFP4
  * producers "residual_add_rms_norm_to_nvfp4" and "silu_mul_merged_grouped32"
  * (the "5060 Ti" report's per-kernel census and its W4A4 NVFP4 GEMM path).

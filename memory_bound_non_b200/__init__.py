@@ -28,6 +28,7 @@ ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
 
 # C entry points declared in include/frt.h
 EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8",
+           "frt_residual_layernorm_fp8", "frt_residual_layernorm_nvfp4", "frt_qkv_layernorm_rope_kvcache",
            "frt_residual_rmsnorm_nvfp4", "frt_gate_act_nvfp4", "frt_qkv_norm_rope_prepq_kvcache",
            "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_status_string")
 
@@ -57,6 +58,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_qkv_norm_rope_kvcache.restype = i32
     L.frt_qkv_norm_rope_prepq_kvcache.argtypes = [vp] * 10 + [i32] * 6 + [f32, f32, i32, i32, vp, i32, vp]
     L.frt_qkv_norm_rope_prepq_kvcache.restype = i32
+    L.frt_residual_layernorm_fp8.argtypes = [vp] * 8 + [i32, i32, f32, i32, i32, vp]
+    L.frt_residual_layernorm_fp8.restype = i32
+    L.frt_residual_layernorm_nvfp4.argtypes = [vp] * 8 + [i32, i32, f32, i32, i32, vp]
+    L.frt_residual_layernorm_nvfp4.restype = i32
+    L.frt_qkv_layernorm_rope_kvcache.argtypes = [vp] * 12 + [i32] * 6 + [f32, i32, vp]
+    L.frt_qkv_layernorm_rope_kvcache.restype = i32
     L.frt_residual_rmsnorm_nvfp4.argtypes = [vp] * 7 + [i32, i32, f32, i32, i32, vp]
     L.frt_residual_rmsnorm_nvfp4.restype = i32
     L.frt_gate_act_nvfp4.argtypes = [vp] * 4 + [i32, i32, i32, i32, i32, vp]
@@ -157,6 +164,38 @@ def frt_gate_act_nvfp4(gate_up, out_fp4, out_sf, global_scale, act="gelu_tanh", 
     st = load().frt_gate_act_nvfp4(_ptr(gate_up), _ptr(out_fp4), _ptr(out_sf), _ptr(global_scale), M, two_i // 2,
                                    ACT[act], DTYPE[gate_up.dtype], SF_LAYOUT[sf_layout], _stream(stream))
     _check("frt_gate_act_nvfp4", st)
+
+
+def frt_residual_layernorm_fp8(x, residual_in, residual_out, weight, bias, out_fp8, static_scale=None,
+                              block_scales=None, eps=1e-6, quant="static", stream=None):
+    """NEXT-4: op (a) with LayerNorm (weight / bias [D] or None) + FP8."""
+    M, D = x.shape
+    st = load().frt_residual_layernorm_fp8(
+        _ptr(x), _ptr(residual_in), _ptr(residual_out), _ptr(weight), _ptr(bias), _ptr(out_fp8), _ptr(static_scale),
+        _ptr(block_scales), M, D, float(eps), DTYPE[x.dtype], QUANT[quant], _stream(stream))
+    _check("frt_residual_layernorm_fp8", st)
+
+
+def frt_residual_layernorm_nvfp4(x, residual_in, residual_out, weight, bias, out_fp4, out_sf, global_scale, eps=1e-6,
+                                 sf_layout="rows", stream=None):
+    """NEXT-4: op (a) with LayerNorm + NVFP4 (the ViT add_layer_norm producer)."""
+    M, D = x.shape
+    st = load().frt_residual_layernorm_nvfp4(
+        _ptr(x), _ptr(residual_in), _ptr(residual_out), _ptr(weight), _ptr(bias), _ptr(out_fp4), _ptr(out_sf),
+        _ptr(global_scale), M, D, float(eps), DTYPE[x.dtype], SF_LAYOUT[sf_layout], _stream(stream))
+    _check("frt_residual_layernorm_nvfp4", st)
+
+
+def frt_qkv_layernorm_rope_kvcache(qkv, q_w, q_b, k_w, k_b, cos_tab, sin_tab, positions, q_out, k_cache, v_cache,
+                                   Hq, Hkv, hd, status=None, eps=1e-6, stream=None):
+    """NEXT-4: op (b) with per-head LayerNorm on Q and K (affine rows
+    [Hq, hd] / [Hkv, hd], each optional)."""
+    M = qkv.shape[0]
+    st = load().frt_qkv_layernorm_rope_kvcache(
+        _ptr(qkv), _ptr(q_w), _ptr(q_b), _ptr(k_w), _ptr(k_b), _ptr(cos_tab), _ptr(sin_tab), _ptr(positions),
+        _ptr(q_out), _ptr(k_cache), _ptr(v_cache), _ptr(status), M, Hq, Hkv, hd, cos_tab.shape[0], k_cache.shape[0],
+        float(eps), DTYPE[qkv.dtype], _stream(stream))
+    _check("frt_qkv_layernorm_rope_kvcache", st)
 
 
 Q_LAYOUT = {"token": 0, "head": 1}

@@ -364,6 +364,99 @@ __device__ __forceinline__ void store_token(const uint16_t* rowbuf, const uint8_
   }
 }
 
+// NEXT-4: per-head LayerNorm on Q and K + rotate-half RoPE + Q staging + KV
+// write ("FlashRT kernel fusion", §2.2 second bullet: the Chameleon prefill
+// kernel, LayerNorm(Q) + LayerNorm(K) + two rotate_half RoPE in one kernel
+// with each rotation pair kept in one lane).  One lane group per head, the
+// token's heads spread over nhb CTAs; per head the mean and the centred sum
+// of squares are two xor-shuffle reductions inside the group, then
+// y = (v - mean) * rstd * w_h + b_h with per-head affine rows (each optional).
+template <int DT, int P, int GP>
+__global__ void __launch_bounds__(512) qkv_layernorm_rope_kvcache_kernel(
+    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_w, const uint16_t* __restrict__ q_b,
+    const uint16_t* __restrict__ k_w, const uint16_t* __restrict__ k_b, const float* __restrict__ cos_tab,
+    const float* __restrict__ sin_tab, const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out,
+    uint16_t* __restrict__ k_cache, uint16_t* __restrict__ v_cache, int32_t* status, int H, int NG, int nhb, int Hq,
+    int Hkv, int hd, int G, int max_pos, int capacity, float eps) {
+  using V = typename Vec16<P>::T;
+  pdl_enter();
+  const int tok = blockIdx.x / nhb;
+  const int h = (blockIdx.x - tok * nhb) * NG + (int)(threadIdx.x / GP);
+  const int li = threadIdx.x & (GP - 1);
+  const int half = hd >> 1;
+  const int j0 = li * P;
+  const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G && h < H;
+  V va, vb;
+  if (lane_ok) {
+    const uint16_t* row = qkv + ((int64_t)tok * H + h) * hd;
+    va = *reinterpret_cast<const V*>(row + j0);
+    vb = *reinterpret_cast<const V*>(row + half + j0);
+  }
+  const int p = __ldg(positions + tok);
+  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
+  if (!row_ok && threadIdx.x == 0 && blockIdx.x % nhb == 0 && status != nullptr) atomicOr(status, 1);
+  const bool on = lane_ok && row_ok;
+  const bool is_q = h < Hq;
+  const bool is_v = h >= Hq + Hkv;
+  if (on && is_v) {  // V: bit copy into the cache slot
+    uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
+    *reinterpret_cast<V*>(dst + j0) = va;
+    *reinterpret_cast<V*>(dst + half + j0) = vb;
+  }
+  float a[P], b[P];
+  float s1 = 0.0f;
+  if (on && !is_v) {
+    unpack<DT, P>(va, a);
+    unpack<DT, P>(vb, b);
+#pragma unroll
+    for (int e = 0; e < P; ++e) s1 += a[e] + b[e];
+  }
+  const float mean = group_sum<GP>(s1) / (float)hd;  // every lane of the warp takes part
+  float s2 = 0.0f;
+  if (on && !is_v) {
+#pragma unroll
+    for (int e = 0; e < P; ++e) {
+      a[e] -= mean;
+      b[e] -= mean;
+      s2 = fmaf(a[e], a[e], fmaf(b[e], b[e], s2));
+    }
+  }
+  s2 = group_sum<GP>(s2);
+  if (!(on && !is_v)) return;
+  const float rstd = 1.0f / sqrtf(s2 / (float)hd + eps);
+  const int hh = is_q ? h : h - Hq;
+  const uint16_t* pw = is_q ? q_w : k_w;
+  const uint16_t* pb = is_q ? q_b : k_b;
+  float fw[2 * P], fb[2 * P];
+#pragma unroll
+  for (int e = 0; e < 2 * P; ++e) {
+    fw[e] = 1.0f;
+    fb[e] = 0.0f;
+  }
+  if (pw != nullptr) {
+    unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + j0), fw);
+    unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + half + j0), fw + P);
+  }
+  if (pb != nullptr) {
+    unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + j0), fb);
+    unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + half + j0), fb + P);
+  }
+  float c[P], sn[P];
+  ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
+  ld_f32<P>(sin_tab + (int64_t)p * half + j0, sn);
+  float o1[P], o2[P];
+#pragma unroll
+  for (int e = 0; e < P; ++e) {
+    const float x1 = fmaf(a[e] * rstd, fw[e], fb[e]);
+    const float x2 = fmaf(b[e] * rstd, fw[P + e], fb[P + e]);
+    o1[e] = fmaf(x1, c[e], -(x2 * sn[e]));
+    o2[e] = fmaf(x2, c[e], x1 * sn[e]);
+  }
+  uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + hh) * hd;
+  store_packed<DT, P>(dst + j0, o1);
+  store_packed<DT, P>(dst + half + j0, o2);
+}
+
 // Polls of a bulk-copy barrier before the kernel gives up (each poll may
 // suspend the thread for a while; the bound is far beyond any real copy).
 constexpr int kMaxPolls = 1 << 22;
@@ -626,4 +719,67 @@ extern "C" frt_status frt_qkv_norm_rope_prepq_kvcache(const void* qkv, const voi
                                                       const float* kv_scales, frt_dtype dt, cudaStream_t stream) {
   return frt::qkv_op(qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status, M, Hq,
                      Hkv, hd, max_pos, capacity, eps, q_scale, q_layout, kv_format, kv_scales, dt, stream);
+}
+
+extern "C" frt_status frt_qkv_layernorm_rope_kvcache(const void* qkv, const void* q_w, const void* q_b, const void* k_w,
+                                                    const void* k_b, const float* cos_tab, const float* sin_tab,
+                                                    const int32_t* positions, void* q_out, void* k_cache,
+                                                    void* v_cache, int32_t* status, int M, int Hq, int Hkv, int hd,
+                                                    int max_pos, int capacity, float eps, frt_dtype dt,
+                                                    cudaStream_t stream) {
+  using namespace frt;
+  if (M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || hd <= 0 || hd % 2 != 0) return FRT_ERR_INVALID_ARG;
+  if (max_pos <= 0 || capacity <= 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
+  if (hd % 8 != 0 || hd > 256) return FRT_ERR_UNSUPPORTED;
+  if (M == 0) return FRT_OK;
+  if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
+  const int P = (hd % 16 == 0) ? 8 : 4;
+  const uintptr_t al = (P == 8) ? 16 : 8;
+  if (!aligned(qkv, al) || !aligned(q_out, al) || !aligned(k_cache, al) || !aligned(v_cache, al))
+    return FRT_ERR_INVALID_ARG;
+  for (const void* w : {q_w, q_b, k_w, k_b})
+    if (w && !aligned(w, al)) return FRT_ERR_INVALID_ARG;
+  if (!aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(positions, 4)) return FRT_ERR_INVALID_ARG;
+  if (status && !aligned(status, 4)) return FRT_ERR_INVALID_ARG;
+  const int H = Hq + 2 * Hkv;
+  const int G = (hd / 2) / P;
+  int GP = 1;
+  while (GP < G) GP *= 2;
+  const int NG = H * GP <= 512 ? H : 512 / GP;  // up to 512 threads: the affine rows need the registers
+  const int nhb = (H + NG - 1) / NG;
+  if ((int64_t)M * nhb > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
+  const int threads = ((NG * GP + 31) / 32) * 32;
+  const dim3 grid((unsigned)((int64_t)M * nhb));
+  const uint16_t* qk = static_cast<const uint16_t*>(qkv);
+  const uint16_t* w16[4] = {static_cast<const uint16_t*>(q_w), static_cast<const uint16_t*>(q_b),
+                            static_cast<const uint16_t*>(k_w), static_cast<const uint16_t*>(k_b)};
+  uint16_t* qo = static_cast<uint16_t*>(q_out);
+  uint16_t* kc = static_cast<uint16_t*>(k_cache);
+  uint16_t* vc = static_cast<uint16_t*>(v_cache);
+#define FRT_LN_LAUNCH(DT_, P_, GP_)                                                                                 \
+  return launch(qkv_layernorm_rope_kvcache_kernel<DT_, P_, GP_>, grid, dim3(threads), 0, stream, qk, w16[0], w16[1], \
+                w16[2], w16[3], cos_tab, sin_tab, positions, qo, kc, vc, status, H, NG, nhb, Hq, Hkv, hd, G, max_pos, \
+                capacity, eps)
+#define FRT_LN_GP(DT_, P_)          \
+  switch (GP) {                     \
+    case 1: FRT_LN_LAUNCH(DT_, P_, 1);  \
+    case 2: FRT_LN_LAUNCH(DT_, P_, 2);  \
+    case 4: FRT_LN_LAUNCH(DT_, P_, 4);  \
+    case 8: FRT_LN_LAUNCH(DT_, P_, 8);  \
+    case 16: FRT_LN_LAUNCH(DT_, P_, 16); \
+    default: FRT_LN_LAUNCH(DT_, P_, 32); \
+  }
+  if (dt == FRT_F16) {
+    if (P == 8) {
+      FRT_LN_GP(FRT_F16, 8)
+    } else {
+      FRT_LN_GP(FRT_F16, 4)
+    }
+  }
+  if (P == 8) {
+    FRT_LN_GP(FRT_BF16, 8)
+  }
+  FRT_LN_GP(FRT_BF16, 4)
+#undef FRT_LN_GP
+#undef FRT_LN_LAUNCH
 }

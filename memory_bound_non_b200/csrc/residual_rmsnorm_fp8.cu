@@ -31,11 +31,15 @@ constexpr int max_threads() {
   return K >= 4 ? 512 : 128;
 }
 
-template <int DT, int K, bool WEIGHTED, int QM>
+// LN (NEXT-4, the ViT "add_layer_norm" producer): LayerNorm instead of
+// RMSNorm, y = (h - mean) * rstd * w + b with mean and the centred sum of
+// squares from two fp64 reductions over the register-held row, and y formed
+// in fp64 and rounded once to fp32 (bias may be null).
+template <int DT, int K, bool WEIGHTED, int QM, bool LN>
 __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     const uint4* __restrict__ x, const uint4* r_in, uint4* r_out, const uint4* __restrict__ w,
-    uint2* __restrict__ q, const float* __restrict__ static_scale, float* __restrict__ block_scales, int C,
-    int NB, float D, float eps) {
+    const uint4* __restrict__ bias, uint2* __restrict__ q, const float* __restrict__ static_scale,
+    float* __restrict__ block_scales, int C, int NB, float D, float eps) {
   using P16 = Pack16<DT>;
   pdl_enter();
   const int t = threadIdx.x;
@@ -87,8 +91,12 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 hf = P16::to_float2(hw[e]);
-        ss[k] = fma((double)hf.x, (double)hf.x, ss[k]);
-        ss[k] = fma((double)hf.y, (double)hf.y, ss[k]);
+        if (LN) {  // the row sum first (the centred squares need the mean)
+          ss[k] += (double)hf.x + (double)hf.y;
+        } else {
+          ss[k] = fma((double)hf.x, (double)hf.x, ss[k]);
+          ss[k] = fma((double)hf.y, (double)hf.y, ss[k]);
+        }
       }
       r_out[base + c] = hv[k];
     } else {
@@ -111,7 +119,33 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   double tot = 0.0;
   const int nw = T >> 5;
   for (int i = 0; i < nw; ++i) tot += red[i];
-  const Split32 rstd(rsqrt_f64(tot / (double)D + (double)eps));
+  double mean = 0.0;
+  if (LN) {
+    // second reduction: the centred sum of squares of the held row
+    mean = tot / (double)D;
+    double sc = 0.0;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      if (t + k * T < C) {
+        const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv[k]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 hf = P16::to_float2(hw[e]);
+          const double d0 = (double)hf.x - mean, d1 = (double)hf.y - mean;
+          sc = fma(d0, d0, fma(d1, d1, sc));
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, o);
+    __syncthreads();  // every thread has read the first partials
+    if ((t & 31) == 0) red[t >> 5] = sc;
+    __syncthreads();
+    tot = 0.0;
+    for (int i = 0; i < nw; ++i) tot += red[i];
+  }
+  const double rstd64 = rsqrt_f64(tot / (double)D + (double)eps);
+  const Split32 rstd(rstd64);
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
   const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * s_static) : 0.0f;  // NVFP4: RN(1 / RN(6 gs))
 
@@ -122,7 +156,30 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     const bool valid = c < C;
     const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv[k]);
     float y[8];
-    if (WEIGHTED && valid) {
+    if (LN) {
+      uint4 wv = make_uint4(0u, 0u, 0u, 0u), bv = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) {
+        if (WEIGHTED) wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : __ldg(w + c);
+        if (bias != nullptr) bv = __ldg(bias + c);
+      }
+      const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv);
+      const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 hf = P16::to_float2(hw[e]);
+        const float2 wf = P16::to_float2(ww[e]);
+        const float2 bf = P16::to_float2(bw[e]);
+        double y0 = ((double)hf.x - mean) * rstd64, y1 = ((double)hf.y - mean) * rstd64;
+        if (WEIGHTED) {
+          y0 *= (double)wf.x;
+          y1 *= (double)wf.y;
+        }
+        // bias zeros when absent; lanes past the row end hold 0 (they take
+        // part in the block amax)
+        y[2 * e] = valid ? (float)(y0 + (double)bf.x) : 0.0f;
+        y[2 * e + 1] = valid ? (float)(y1 + (double)bf.y) : 0.0f;
+      }
+    } else if (WEIGHTED && valid) {
       const uint4 wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : __ldg(w + c);
       const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv);
 #pragma unroll
@@ -168,43 +225,49 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   }
 }
 
-template <int DT, int K, bool W, int QM>
-frt_status launch_k(const void* x, const void* r_in, void* r_out, const void* w, uint8_t* q, const float* ss,
-                    float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
-  auto kern = residual_rmsnorm_fp8_kernel<DT, K, W, QM>;
-  return launch(kern, dim3(M), dim3(T), 0, st, static_cast<const uint4*>(x), static_cast<const uint4*>(r_in),
-                static_cast<uint4*>(r_out), static_cast<const uint4*>(w), reinterpret_cast<uint2*>(q), ss, bs, C, NB,
-                (float)(C * 8), eps);
+// Row-norm launch arguments (bias only with LN).
+struct NormArgs {
+  const void *x, *r_in;
+  void* r_out;
+  const void *w, *bias;
+  uint8_t* q;
+  const float* ss;
+  float* bs;
+  int M, C, NB, T;
+  float eps;
+};
+
+template <int DT, int K, bool W, int QM, bool LN>
+frt_status launch_k(const NormArgs& a, cudaStream_t st) {
+  auto kern = residual_rmsnorm_fp8_kernel<DT, K, W, QM, LN>;
+  return launch(kern, dim3(a.M), dim3(a.T), 0, st, static_cast<const uint4*>(a.x), static_cast<const uint4*>(a.r_in),
+                static_cast<uint4*>(a.r_out), static_cast<const uint4*>(a.w), static_cast<const uint4*>(a.bias),
+                reinterpret_cast<uint2*>(a.q), a.ss, a.bs, a.C, a.NB, (float)(a.C * 8), a.eps);
 }
 
-template <int DT, int K, bool W>
-frt_status launch_w(int qm, const void* x, const void* r_in, void* r_out, const void* w, uint8_t* q,
-                    const float* ss, float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
+template <int DT, int K, bool W, bool LN>
+frt_status launch_w(int qm, const NormArgs& a, cudaStream_t st) {
   switch (qm) {
-    case FRT_QUANT_STATIC: return launch_k<DT, K, W, FRT_QUANT_STATIC>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    case FRT_QUANT_BLOCK128:
-      return launch_k<DT, K, W, FRT_QUANT_BLOCK128>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    case kQuantNvfp4Rows: return launch_k<DT, K, W, kQuantNvfp4Rows>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    default: return launch_k<DT, K, W, kQuantNvfp4Swizzled>(x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    case FRT_QUANT_STATIC: return launch_k<DT, K, W, FRT_QUANT_STATIC, LN>(a, st);
+    case FRT_QUANT_BLOCK128: return launch_k<DT, K, W, FRT_QUANT_BLOCK128, LN>(a, st);
+    case kQuantNvfp4Rows: return launch_k<DT, K, W, kQuantNvfp4Rows, LN>(a, st);
+    default: return launch_k<DT, K, W, kQuantNvfp4Swizzled, LN>(a, st);
   }
 }
 
 template <int DT, int K>
-frt_status launch_dt_k(bool weighted, int qm, const void* x, const void* r_in, void* r_out, const void* w,
-                       uint8_t* q, const float* ss, float* bs, int M, int C, int NB, int T, float eps,
-                       cudaStream_t st) {
-  return weighted ? launch_w<DT, K, true>(qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st)
-                  : launch_w<DT, K, false>(qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+frt_status launch_dt_k(bool weighted, bool ln, int qm, const NormArgs& a, cudaStream_t st) {
+  if (ln) return weighted ? launch_w<DT, K, true, true>(qm, a, st) : launch_w<DT, K, false, true>(qm, a, st);
+  return weighted ? launch_w<DT, K, true, false>(qm, a, st) : launch_w<DT, K, false, false>(qm, a, st);
 }
 
 template <int DT>
-frt_status launch_dt(int K, bool weighted, int qm, const void* x, const void* r_in, void* r_out, const void* w,
-               uint8_t* q, const float* ss, float* bs, int M, int C, int NB, int T, float eps, cudaStream_t st) {
+frt_status launch_dt(int K, bool weighted, bool ln, int qm, const NormArgs& a, cudaStream_t st) {
   switch (K) {
-    case 1: return launch_dt_k<DT, 1>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    case 2: return launch_dt_k<DT, 2>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    case 4: return launch_dt_k<DT, 4>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
-    default: return launch_dt_k<DT, 8>(weighted, qm, x, r_in, r_out, w, q, ss, bs, M, C, NB, T, eps, st);
+    case 1: return launch_dt_k<DT, 1>(weighted, ln, qm, a, st);
+    case 2: return launch_dt_k<DT, 2>(weighted, ln, qm, a, st);
+    case 4: return launch_dt_k<DT, 4>(weighted, ln, qm, a, st);
+    default: return launch_dt_k<DT, 8>(weighted, ln, qm, a, st);
   }
 }
 
@@ -240,11 +303,10 @@ extern "C" frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residu
   const int NB = (D + 127) / 128;
   int K, T;
   rmsnorm_shape(C, &K, &T);
-  if (dt == FRT_F16)
-    return launch_dt<FRT_F16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp8,
-                              static_scale, block_scales, M, C, NB, T, eps, stream);
-  return launch_dt<FRT_BF16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp8,
-                             static_scale, block_scales, M, C, NB, T, eps, stream);
+  const NormArgs a{x, residual_in, residual_out, weight, nullptr, out_fp8, static_scale, block_scales, M, C, NB, T,
+                   eps};
+  return dt == FRT_F16 ? launch_dt<FRT_F16>(K, weight != nullptr, false, qm, a, stream)
+                       : launch_dt<FRT_BF16>(K, weight != nullptr, false, qm, a, stream);
 }
 
 extern "C" frt_status frt_residual_rmsnorm_nvfp4(const void* x, const void* residual_in, void* residual_out,
@@ -265,9 +327,56 @@ extern "C" frt_status frt_residual_rmsnorm_nvfp4(const void* x, const void* resi
   rmsnorm_shape(C, &K, &T);
   const int qm = sf_layout == FRT_SF_ROW_MAJOR ? kQuantNvfp4Rows : kQuantNvfp4Swizzled;
   float* sf = reinterpret_cast<float*>(out_sf);  // the kernel's scale pointer carries the sf bytes
-  if (dt == FRT_F16)
-    return launch_dt<FRT_F16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp4, global_scale,
-                              sf, M, C, 0, T, eps, stream);
-  return launch_dt<FRT_BF16>(K, weight != nullptr, qm, x, residual_in, residual_out, weight, out_fp4, global_scale,
-                             sf, M, C, 0, T, eps, stream);
+  const NormArgs a{x, residual_in, residual_out, weight, nullptr, out_fp4, global_scale, sf, M, C, 0, T, eps};
+  return dt == FRT_F16 ? launch_dt<FRT_F16>(K, weight != nullptr, false, qm, a, stream)
+                       : launch_dt<FRT_BF16>(K, weight != nullptr, false, qm, a, stream);
+}
+
+// NEXT-4: residual add + LayerNorm producers (the ViT "add_layer_norm").
+namespace frt {
+namespace {
+frt_status layernorm_op(const void* x, const void* residual_in, void* residual_out, const void* weight,
+                        const void* bias, uint8_t* out, const float* scale, float* scales_out, int M, int D,
+                        float eps, frt_dtype dt, int qm, cudaStream_t stream) {
+  if (M == 0) return FRT_OK;
+  if (!x || !residual_in || !residual_out) return FRT_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(residual_in, 16) || !aligned(residual_out, 16)) return FRT_ERR_INVALID_ARG;
+  if ((weight && !aligned(weight, 16)) || (bias && !aligned(bias, 16))) return FRT_ERR_INVALID_ARG;
+  const int C = D / 8;
+  int K, T;
+  rmsnorm_shape(C, &K, &T);
+  const NormArgs a{x, residual_in, residual_out, weight, bias, out, scale, scales_out, M, C, (D + 127) / 128, T,
+                   eps};
+  return dt == FRT_F16 ? launch_dt<FRT_F16>(K, weight != nullptr, true, qm, a, stream)
+                       : launch_dt<FRT_BF16>(K, weight != nullptr, true, qm, a, stream);
+}
+}  // namespace
+}  // namespace frt
+
+extern "C" frt_status frt_residual_layernorm_fp8(const void* x, const void* residual_in, void* residual_out,
+                                                 const void* weight, const void* bias, uint8_t* out_fp8,
+                                                 const float* static_scale, float* block_scales, int M, int D,
+                                                 float eps, frt_dtype dt, frt_quant qm, cudaStream_t stream) {
+  using namespace frt;
+  if (M < 0 || D <= 0 || D % 8 != 0 || !valid_dtype(dt) || !valid_quant(qm)) return FRT_ERR_INVALID_ARG;
+  if (D > 32768) return FRT_ERR_UNSUPPORTED;
+  if (M > 0 && (!out_fp8 || !aligned(out_fp8, 8) || !quant_args_ok(qm, static_scale, block_scales)))
+    return FRT_ERR_INVALID_ARG;
+  return layernorm_op(x, residual_in, residual_out, weight, bias, out_fp8, static_scale, block_scales, M, D, eps, dt,
+                      qm, stream);
+}
+
+extern "C" frt_status frt_residual_layernorm_nvfp4(const void* x, const void* residual_in, void* residual_out,
+                                                   const void* weight, const void* bias, uint8_t* out_fp4,
+                                                   uint8_t* out_sf, const float* global_scale, int M, int D,
+                                                   float eps, frt_dtype dt, frt_sf_layout sf_layout,
+                                                   cudaStream_t stream) {
+  using namespace frt;
+  if (M < 0 || D <= 0 || D % 16 != 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
+  if (sf_layout != FRT_SF_ROW_MAJOR && sf_layout != FRT_SF_SWIZZLED_128X4) return FRT_ERR_INVALID_ARG;
+  if (D > 32768) return FRT_ERR_UNSUPPORTED;
+  if (M > 0 && !nvfp4_args_ok(sf_layout, global_scale, out_fp4, out_sf, 4)) return FRT_ERR_INVALID_ARG;
+  const int qm = sf_layout == FRT_SF_ROW_MAJOR ? kQuantNvfp4Rows : kQuantNvfp4Swizzled;
+  return layernorm_op(x, residual_in, residual_out, weight, bias, out_fp4, global_scale,
+                      reinterpret_cast<float*>(out_sf), M, D, eps, dt, qm, stream);
 }

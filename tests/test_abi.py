@@ -161,3 +161,28 @@ def test_residual_rmsnorm_nvfp4_host_validation(kw, want):
 ])
 def test_gate_act_nvfp4_host_validation(kw, want):
     assert c4_call(**kw) == want
+
+
+def ln_call(M=4, D=256, x=A, r=A, ro=A, w=None, b=None, q=A, ss=A, bs=None, dt=1, qm=0):
+    return frt.load().frt_residual_layernorm_fp8(x, r, ro, w, b, q, ss, bs, M, D, 1e-6, dt, qm, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(D=12), INV), (dict(b=A + 4), INV), (dict(w=A + 2), INV), (dict(ss=None), INV), (dict(qm=1), INV),
+    (dict(q=A + 4), INV), (dict(D=32776), UNSUP), (dict(M=0), OK), (dict(M=0, ss=None, q=None), OK),
+])
+def test_residual_layernorm_host_validation(kw, want):
+    assert ln_call(**kw) == want
+
+
+def qln_call(M=4, Hq=8, Hkv=2, hd=128, qkv=A, qw=None, qb=None, kw=None, kb=None, dt=1):
+    return frt.load().frt_qkv_layernorm_rope_kvcache(qkv, qw, qb, kw, kb, A, A, A, A, A, A, None, M, Hq, Hkv, hd, 64,
+                                                     64, 1e-6, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(Hq=6, Hkv=4), INV), (dict(hd=12), UNSUP), (dict(qb=A + 8), INV), (dict(kw=A + 2), INV),
+    (dict(qkv=A + 8), INV), (dict(qkv=None), INV), (dict(M=0), OK), (dict(M=0, qkv=None), OK), (dict(dt=4), INV),
+])
+def test_qkv_layernorm_host_validation(kw, want):
+    assert qln_call(**kw) == want

@@ -535,3 +535,119 @@ def test_nvfp4_large_m_sampled():
     o = oracle.gate_act_nvfp4(hb, wl.act, wl.dt, gs)
     assert_e2m1_codes(q[tc].cpu().numpy(), o["out_fp4"], what="large-M op c e2m1")
     np.testing.assert_array_equal(sf.view(Mc, I // 16)[tc].cpu().numpy(), o["sf"])
+
+
+# ================================================================== NEXT-4 ===
+# LayerNorm variants: residual add + LayerNorm producers (FP8 and NVFP4) and the
+# per-head LayerNorm(Q/K) + RoPE kernel.
+
+def ln_inputs(M, D, dt, seed, weighted=True, biased=True):
+    g = W.generator(seed)
+    x = W.normal16((M, D), dt, g)
+    r = W.normal16((M, D), dt, g, scale=2.0)
+    w = W.norm_weight(D, dt, g) if weighted else None
+    b = W.normal16((D,), dt, g, scale=0.2) if biased else None
+    return x, r, w, b
+
+
+LN_CASES = [(10, 1024, "bf16", "static", True, True), (41, 2048, "bf16", "block128", True, False),
+            (7, 1040, "f16", "block128", False, True), (1176, 1152, "bf16", "static", True, True),
+            (3, 16, "f16", "nvfp4", True, True), (33, 1280, "bf16", "nvfp4", False, False),
+            (5, 8192, "bf16", "nvfp4", True, True), (2, 32768, "bf16", "block128", True, True)]
+
+
+@pytest.mark.parametrize("M,D,dt,quant,weighted,biased", LN_CASES)
+def test_residual_layernorm_parity(M, D, dt, quant, weighted, biased):
+    x, r, w, b = ln_inputs(M, D, dt, M + D, weighted, biased)
+    hx, hr = W.bits16(x), W.bits16(r)
+    hw, hb = (None if t is None else W.bits16(t) for t in (w, b))
+    y = oracle.residual_layernorm(hx, hr, hw, hb, 1e-6, dt, "block128", want_y=True)["y"]
+    xd, rd = x.to(DEV), r.to(DEV).clone()
+    wd, bd = (None if t is None else t.to(DEV) for t in (w, b))
+    if quant == "nvfp4":
+        gs = global_scale_for(y)
+        q = torch.empty((M, D // 2), dtype=torch.uint8, device=DEV)
+        sf = torch.empty((M * D // 16,), dtype=torch.uint8, device=DEV)
+        frt.frt_residual_layernorm_nvfp4(xd, rd, rd, wd, bd, q, sf, torch.tensor([gs], device=DEV))
+        torch.cuda.synchronize()
+        o = oracle.residual_layernorm(hx, hr, hw, hb, 1e-6, dt, "nvfp4", global_scale=gs)
+        assert_e2m1_codes(q.cpu().numpy(), o["out"], max_frac=1e-3, what="LN e2m1")
+        sfs = np.abs(sf.cpu().numpy().astype(int) - o["sf"].ravel().astype(int))
+        assert (sfs <= 1).all() and (sfs > 0).mean() <= 1e-3
+    else:
+        q_raw, q = guarded((M, D), torch.uint8, 0xA5)
+        ss = bs = None
+        scale = None
+        if quant == "static":
+            scale = P.f32(np.abs(y).max() / 448.0)
+            ss = torch.tensor([scale], dtype=torch.float32, device=DEV)
+        else:
+            bs = torch.full((M, (D + 127) // 128), float("nan"), dtype=torch.float32, device=DEV)
+        frt.frt_residual_layernorm_fp8(xd, rd, rd, wd, bd, q, static_scale=ss, block_scales=bs, quant=quant)
+        torch.cuda.synchronize()
+        assert_guard(q_raw, M * D, 0xA5)
+        o = oracle.residual_layernorm(hx, hr, hw, hb, 1e-6, dt, quant, static_scale=scale)
+        P.assert_fp8_codes(q.cpu().numpy(), o["out"], what="LN codes")
+        if quant == "block128":
+            P.assert_scales_close(bs.cpu().numpy(), o["block_scales"])
+    np.testing.assert_array_equal(W.bits16(rd.cpu()), o["residual_out"])
+
+
+def test_residual_layernorm_large_m_sampled():
+    M, D, dt = 65536, 4096, "bf16"
+    g = W.generator(71, DEV)
+    x, r = W.normal16((M, D), dt, g), W.normal16((M, D), dt, g, scale=2.0)
+    w, b = W.norm_weight(D, dt, g), W.normal16((D,), dt, g, scale=0.2)
+    rows = np.unique(np.concatenate([np.random.default_rng(71).choice(M, 192, replace=False), [0, M - 1]]))
+    ti = torch.as_tensor(rows, device=DEV)
+    hx, hr, hw, hb = W.bits16(x[ti].cpu()), W.bits16(r[ti].cpu()), W.bits16(w.cpu()), W.bits16(b.cpu())
+    y = oracle.residual_layernorm(hx, hr, hw, hb, 1e-6, dt, "block128", want_y=True)["y"]
+    scale = P.f32(np.abs(y).max() / 448.0)
+    q = torch.empty((M, D), dtype=torch.uint8, device=DEV)
+    frt.frt_residual_layernorm_fp8(x, r, r, w, b, q, static_scale=torch.tensor([scale], device=DEV))
+    torch.cuda.synchronize()
+    o = oracle.residual_layernorm(hx, hr, hw, hb, 1e-6, dt, "static", static_scale=scale)
+    np.testing.assert_array_equal(W.bits16(r[ti].cpu()), o["residual_out"])
+    P.assert_fp8_codes(q[ti].cpu().numpy(), o["out"], what="large-M LN codes")
+
+
+QLN_CASES = [dict(M=10, Hq=8, Hkv=1, hd=256, dt="bf16"), dict(M=41, Hq=16, Hkv=8, hd=128, dt="bf16"),
+             dict(M=6, Hq=32, Hkv=32, hd=128, dt="bf16"),          # Chameleon-like: 96 heads over two CTAs
+             dict(M=7, Hq=16, Hkv=16, hd=72, dt="f16"), dict(M=700, Hq=32, Hkv=8, hd=128, dt="bf16")]
+
+
+@pytest.mark.parametrize("c", QLN_CASES, ids=lambda c: "M%d-H%d-%d-hd%d-%s" % (c["M"], c["Hq"], c["Hkv"], c["hd"],
+                                                                             c["dt"]))
+@pytest.mark.parametrize("affine", ["both", "q_only", "none"])
+def test_qkv_layernorm_parity(c, affine):
+    M, Hq, Hkv, hd, dt = c["M"], c["Hq"], c["Hkv"], c["hd"], c["dt"]
+    g = W.generator(M * 7 + hd)
+    H = Hq + 2 * Hkv
+    qkv = W.normal16((M, H * hd), dt, g, scale=1.5)
+    qw = W.normal16((Hq, hd), dt, g) if affine != "none" else None
+    qb = W.normal16((Hq, hd), dt, g, scale=0.1) if affine != "none" else None
+    kw = W.normal16((Hkv, hd), dt, g) if affine == "both" else None
+    kb = W.normal16((Hkv, hd), dt, g, scale=0.1) if affine == "both" else None
+    cap = max(64, 2 * M)
+    cos, sin = W.rope_tables(cap, hd, 1e4)
+    pos = torch.randperm(cap, generator=g)[:M].to(torch.int32)
+    kc = torch.full((cap, Hkv, hd), 0x7E7E, dtype=torch.int16).view(W.DTYPES[dt])
+    vc = kc.clone()
+    q_raw, q_out = guarded((M, Hq, hd), qkv.dtype, 0x3C)
+    dev = lambda t: None if t is None else t.to(DEV)
+    kcd, vcd = kc.to(DEV), vc.to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    frt.frt_qkv_layernorm_rope_kvcache(dev(qkv), dev(qw), dev(qb), dev(kw), dev(kb), dev(cos), dev(sin), dev(pos),
+                                       q_out, kcd, vcd, Hq, Hkv, hd, status=status)
+    torch.cuda.synchronize()
+    assert_guard(q_raw, q_out.numel() * 2, 0x3C)
+    hb = lambda t: None if t is None else W.bits16(t)
+    o = oracle.qkv_layernorm_rope_kvcache(W.bits16(qkv), hb(qw), hb(qb), hb(kw), hb(kb), cos.numpy(), sin.numpy(),
+                                          pos.numpy(), Hq, Hkv, hd, cap, 1e-6, dt, v_cache=W.bits16(vc))
+    assert int(status.item()) == o["status"] == 0
+    P.assert_16bit_close(P.decode16(q_out), o["q_out"], what="LN Q", dt=dt)
+    p = pos.long().numpy()
+    P.assert_16bit_close(P.decode16(kcd)[p], o["k_cache"][p], what="LN K", dt=dt)
+    np.testing.assert_array_equal(P.np16(vcd), o["v_cache"])
+    untouched = np.setdiff1d(np.arange(cap), p)
+    assert (P.np16(kcd)[untouched] == 0x7E7E).all()
