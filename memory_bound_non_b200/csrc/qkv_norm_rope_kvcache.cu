@@ -82,6 +82,8 @@ struct Epilogue {
   int q_head_major;
   int M;
   const float* kv_scales;
+  const uint16_t* q_bias;  // LayerNorm level (EPI 3): per-head bias rows, or null
+  const uint16_t* k_bias;
 };
 
 __device__ __forceinline__ int64_t q_row(const Epilogue& ep, int tok, int h, int Hq) {
@@ -259,8 +261,9 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
                                               uint16_t* q_out, int tok, int tid, int H, int NG, int Hq, int Hkv,
                                               int hd, int G, float eps, const Epilogue& ep) {
   using V = typename Vec16<P>::T;
-  constexpr bool QEPI = EPI >= 1;
+  constexpr bool QEPI = EPI == 1 || EPI == 2;
   constexpr bool KV8 = EPI == 2;
+  constexpr bool LN = EPI == 3;
   const int half = hd >> 1;
   const int grp = tid / GP;
   const int li = tid & (GP - 1);
@@ -289,6 +292,72 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
     const uint16_t* nws = is_q ? qwbuf : kwbuf;
     uint16_t* vec = rowbuf + h * hd;
     float a[P], b[P];
+    if (LN) {
+      // per-head LayerNorm: mean, then the centred sum of squares, then the
+      // head's affine rows (global memory, each optional) and RoPE in place
+      float s1 = 0.0f;
+      if (on) {
+        unpack<DT, P>(*reinterpret_cast<const V*>(vec + j0), a);
+        unpack<DT, P>(*reinterpret_cast<const V*>(vec + half + j0), b);
+#pragma unroll
+        for (int e = 0; e < P; ++e) s1 += a[e] + b[e];
+      }
+      const float mean = group_sum<GP>(s1) / (float)hd;
+      float s2 = 0.0f;
+      if (on) {
+#pragma unroll
+        for (int e = 0; e < P; ++e) {
+          a[e] -= mean;
+          b[e] -= mean;
+          s2 = fmaf(a[e], a[e], fmaf(b[e], b[e], s2));
+        }
+      }
+      s2 = group_sum<GP>(s2);
+      if (on) {
+        const float rstd = 1.0f / sqrtf(s2 / (float)hd + eps);
+        const int64_t off = (int64_t)(is_q ? h : h - Hq) * hd;
+        const uint16_t* pw = is_q ? q_norm_w : k_norm_w;
+        const uint16_t* pb = is_q ? ep.q_bias : ep.k_bias;
+        // affine rows kept packed (16-bit pairs), unpacked pair by pair
+        uint32_t wa[P / 2], wb[P / 2], ba[P / 2], bb[P / 2];
+#pragma unroll
+        for (int e = 0; e < P / 2; ++e) {
+          wa[e] = wb[e] = Pack16<DT>::kOnes;
+          ba[e] = bb[e] = 0u;
+        }
+        if (pw != nullptr) {
+          const V t1 = ld_vec<P>(pw + off + j0), t2 = ld_vec<P>(pw + off + half + j0);
+#pragma unroll
+          for (int e = 0; e < P / 2; ++e) {
+            wa[e] = reinterpret_cast<const uint32_t*>(&t1)[e];
+            wb[e] = reinterpret_cast<const uint32_t*>(&t2)[e];
+          }
+        }
+        if (pb != nullptr) {
+          const V t1 = ld_vec<P>(pb + off + j0), t2 = ld_vec<P>(pb + off + half + j0);
+#pragma unroll
+          for (int e = 0; e < P / 2; ++e) {
+            ba[e] = reinterpret_cast<const uint32_t*>(&t1)[e];
+            bb[e] = reinterpret_cast<const uint32_t*>(&t2)[e];
+          }
+        }
+        float o1[P], o2[P];
+#pragma unroll
+        for (int e = 0; e < P; e += 2) {
+          const float2 w1 = Pack16<DT>::to_float2(wa[e / 2]), w2 = Pack16<DT>::to_float2(wb[e / 2]);
+          const float2 b1 = Pack16<DT>::to_float2(ba[e / 2]), b2 = Pack16<DT>::to_float2(bb[e / 2]);
+          const float x1a = fmaf(a[e] * rstd, w1.x, b1.x), x1b = fmaf(a[e + 1] * rstd, w1.y, b1.y);
+          const float x2a = fmaf(b[e] * rstd, w2.x, b2.x), x2b = fmaf(b[e + 1] * rstd, w2.y, b2.y);
+          o1[e] = fmaf(x1a, c[e], -(x2a * s[e]));
+          o2[e] = fmaf(x2a, c[e], x1a * s[e]);
+          o1[e + 1] = fmaf(x1b, c[e + 1], -(x2b * s[e + 1]));
+          o2[e + 1] = fmaf(x2b, c[e + 1], x1b * s[e + 1]);
+        }
+        store_packed<DT, P>(vec + j0, o1);
+        store_packed<DT, P>(vec + half + j0, o2);
+      }
+      continue;
+    }
     float ss = 0.0f;
     if (on) {
       unpack<DT, P>(*reinterpret_cast<const V*>(vec + j0), a);
@@ -353,7 +422,8 @@ template <int EPI>
 __device__ __forceinline__ void store_token(const uint16_t* rowbuf, const uint8_t* k8buf, const uint8_t* v8buf,
                                             uint16_t* q_out, void* k_cache, void* v_cache, int tok, int p, int Hq,
                                             int Hkv, int hd, const Epilogue& ep) {
-  if (!(EPI >= 1 && ep.q_head_major)) bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
+  if (!((EPI == 1 || EPI == 2) && ep.q_head_major))
+    bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
   if (EPI == 2) {
     bulk_store(static_cast<uint8_t*>(k_cache) + (int64_t)p * Hkv * hd, k8buf, (unsigned)(Hkv * hd));
     bulk_store(static_cast<uint8_t*>(v_cache) + (int64_t)p * Hkv * hd, v8buf, (unsigned)(Hkv * hd));
@@ -367,12 +437,14 @@ __device__ __forceinline__ void store_token(const uint16_t* rowbuf, const uint8_
 // NEXT-4: per-head LayerNorm on Q and K + rotate-half RoPE + Q staging + KV
 // write ("FlashRT kernel fusion", §2.2 second bullet: the Chameleon prefill
 // kernel, LayerNorm(Q) + LayerNorm(K) + two rotate_half RoPE in one kernel
-// with each rotation pair kept in one lane).  One lane group per head, the
-// token's heads spread over nhb CTAs; per head the mean and the centred sum
-// of squares are two xor-shuffle reductions inside the group, then
-// y = (v - mean) * rstd * w_h + b_h with per-head affine rows (each optional).
-template <int DT, int P, int GP>
-__global__ void __launch_bounds__(512) qkv_layernorm_rope_kvcache_kernel(
+// with each rotation pair kept in one lane).  Lane groups of GP lanes take up
+// to HPG heads of one token each (slot i of group g is head
+// (hb * HPG + i) * NG + g); all QKV loads and the cos/sin slice are issued
+// first.  Per head the mean and the centred sum of squares are two
+// xor-shuffle reductions inside the group, then y = (v - mean) * rstd * w_h +
+// b_h with per-head affine rows (each optional, read from L2).
+template <int DT, int P, int GP, int HPG>
+__global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcache_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_w, const uint16_t* __restrict__ q_b,
     const uint16_t* __restrict__ k_w, const uint16_t* __restrict__ k_b, const float* __restrict__ cos_tab,
     const float* __restrict__ sin_tab, const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out,
@@ -381,80 +453,94 @@ __global__ void __launch_bounds__(512) qkv_layernorm_rope_kvcache_kernel(
   using V = typename Vec16<P>::T;
   pdl_enter();
   const int tok = blockIdx.x / nhb;
-  const int h = (blockIdx.x - tok * nhb) * NG + (int)(threadIdx.x / GP);
+  const int hb = blockIdx.x - tok * nhb;
+  const int grp = (int)(threadIdx.x / GP);
   const int li = threadIdx.x & (GP - 1);
   const int half = hd >> 1;
   const int j0 = li * P;
-  const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G && h < H;
-  V va, vb;
-  if (lane_ok) {
-    const uint16_t* row = qkv + ((int64_t)tok * H + h) * hd;
-    va = *reinterpret_cast<const V*>(row + j0);
-    vb = *reinterpret_cast<const V*>(row + half + j0);
+  const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G;
+  const uint16_t* row = qkv + (int64_t)tok * H * hd;
+  V va[HPG], vb[HPG];
+#pragma unroll
+  for (int i = 0; i < HPG; ++i) {
+    const int h = (hb * HPG + i) * NG + grp;
+    if (lane_ok && h < H) {
+      va[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + j0);
+      vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
+    }
   }
   const int p = __ldg(positions + tok);
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
-  if (!row_ok && threadIdx.x == 0 && blockIdx.x % nhb == 0 && status != nullptr) atomicOr(status, 1);
-  const bool on = lane_ok && row_ok;
-  const bool is_q = h < Hq;
-  const bool is_v = h >= Hq + Hkv;
-  if (on && is_v) {  // V: bit copy into the cache slot
-    uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
-    *reinterpret_cast<V*>(dst + j0) = va;
-    *reinterpret_cast<V*>(dst + half + j0) = vb;
+  if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
+  const bool active = lane_ok && row_ok;
+  float c[P], sn[P];
+  if (active) {
+    ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
+    ld_f32<P>(sin_tab + (int64_t)p * half + j0, sn);
   }
-  float a[P], b[P];
-  float s1 = 0.0f;
-  if (on && !is_v) {
-    unpack<DT, P>(va, a);
-    unpack<DT, P>(vb, b);
 #pragma unroll
-    for (int e = 0; e < P; ++e) s1 += a[e] + b[e];
-  }
-  const float mean = group_sum<GP>(s1) / (float)hd;  // every lane of the warp takes part
-  float s2 = 0.0f;
-  if (on && !is_v) {
+  for (int i = 0; i < HPG; ++i) {
+    const int h = (hb * HPG + i) * NG + grp;
+    const bool on = active && h < H;
+    const bool is_q = h < Hq;
+    const bool is_v = h >= Hq + Hkv;
+    if (on && is_v) {  // V: bit copy into the cache slot
+      uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
+      *reinterpret_cast<V*>(dst + j0) = va[i];
+      *reinterpret_cast<V*>(dst + half + j0) = vb[i];
+    }
+    const bool qk = on && !is_v;
+    float a[P], b[P];
+    float s1 = 0.0f;
+    if (qk) {
+      unpack<DT, P>(va[i], a);
+      unpack<DT, P>(vb[i], b);
 #pragma unroll
-    for (int e = 0; e < P; ++e) {
-      a[e] -= mean;
-      b[e] -= mean;
-      s2 = fmaf(a[e], a[e], fmaf(b[e], b[e], s2));
+      for (int e = 0; e < P; ++e) s1 += a[e] + b[e];
+    }
+    const float mean = group_sum<GP>(s1) / (float)hd;  // every lane of the warp takes part
+    float s2 = 0.0f;
+    if (qk) {
+#pragma unroll
+      for (int e = 0; e < P; ++e) {
+        a[e] -= mean;
+        b[e] -= mean;
+        s2 = fmaf(a[e], a[e], fmaf(b[e], b[e], s2));
+      }
+    }
+    s2 = group_sum<GP>(s2);
+    if (qk) {
+      const float rstd = 1.0f / sqrtf(s2 / (float)hd + eps);
+      const int hh = is_q ? h : h - Hq;
+      const uint16_t* pw = is_q ? q_w : k_w;
+      const uint16_t* pb = is_q ? q_b : k_b;
+      float fw[2 * P], fb[2 * P];
+#pragma unroll
+      for (int e = 0; e < 2 * P; ++e) {
+        fw[e] = 1.0f;
+        fb[e] = 0.0f;
+      }
+      if (pw != nullptr) {
+        unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + j0), fw);
+        unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + half + j0), fw + P);
+      }
+      if (pb != nullptr) {
+        unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + j0), fb);
+        unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + half + j0), fb + P);
+      }
+      float o1[P], o2[P];
+#pragma unroll
+      for (int e = 0; e < P; ++e) {
+        const float x1 = fmaf(a[e] * rstd, fw[e], fb[e]);
+        const float x2 = fmaf(b[e] * rstd, fw[P + e], fb[P + e]);
+        o1[e] = fmaf(x1, c[e], -(x2 * sn[e]));
+        o2[e] = fmaf(x2, c[e], x1 * sn[e]);
+      }
+      uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + hh) * hd;
+      store_packed<DT, P>(dst + j0, o1);
+      store_packed<DT, P>(dst + half + j0, o2);
     }
   }
-  s2 = group_sum<GP>(s2);
-  if (!(on && !is_v)) return;
-  const float rstd = 1.0f / sqrtf(s2 / (float)hd + eps);
-  const int hh = is_q ? h : h - Hq;
-  const uint16_t* pw = is_q ? q_w : k_w;
-  const uint16_t* pb = is_q ? q_b : k_b;
-  float fw[2 * P], fb[2 * P];
-#pragma unroll
-  for (int e = 0; e < 2 * P; ++e) {
-    fw[e] = 1.0f;
-    fb[e] = 0.0f;
-  }
-  if (pw != nullptr) {
-    unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + j0), fw);
-    unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + half + j0), fw + P);
-  }
-  if (pb != nullptr) {
-    unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + j0), fb);
-    unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + half + j0), fb + P);
-  }
-  float c[P], sn[P];
-  ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
-  ld_f32<P>(sin_tab + (int64_t)p * half + j0, sn);
-  float o1[P], o2[P];
-#pragma unroll
-  for (int e = 0; e < P; ++e) {
-    const float x1 = fmaf(a[e] * rstd, fw[e], fb[e]);
-    const float x2 = fmaf(b[e] * rstd, fw[P + e], fb[P + e]);
-    o1[e] = fmaf(x1, c[e], -(x2 * sn[e]));
-    o2[e] = fmaf(x2, c[e], x1 * sn[e]);
-  }
-  uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + hh) * hd;
-  store_packed<DT, P>(dst + j0, o1);
-  store_packed<DT, P>(dst + half + j0, o2);
 }
 
 // Polls of a bulk-copy barrier before the kernel gives up (each poll may
@@ -470,13 +556,15 @@ constexpr int kMaxPolls = 1 << 22;
 // stores.  A barrier wait that runs out of polls sets bit 1 of *status and the
 // CTA returns without writing.
 // EPI: 0 = op (b) as is (Q token-major, unscaled; 16-bit caches), 1 = Q
-// epilogue (scale, layout), 2 = Q epilogue + e4m3 caches.  At most 128
+// epilogue (scale, layout), 2 = Q epilogue + e4m3 caches, 3 = per-head
+// LayerNorm in place of the RMSNorm (affine rows read from global memory,
+// nothing staged for them).  At most 128
 // threads; the register budget keeps 10 CTAs (tokens) resident per SM (8 for
 // the 16-bit Q epilogue, which would spill at 10): the kernel waits on memory,
 // so resident tokens, not instruction count, set its rate.
 template <int EPI>
 constexpr int tma_min_blocks() {
-  return EPI == 1 ? 8 : 10;
+  return EPI == 1 || EPI == 3 ? 8 : 10;
 }
 
 template <int DT, int P, int GP, int EPI>
@@ -511,11 +599,13 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
   }
   __syncthreads();
   if (tid == 0) {
-    const unsigned first = row_bytes + (q_norm_w ? w_bytes : 0u) + (k_norm_w ? w_bytes : 0u);
+    const bool stage_w = EPI != 3;  // LayerNorm rows are per head: read from global memory instead
+    const unsigned first =
+        row_bytes + (stage_w && q_norm_w ? w_bytes : 0u) + (stage_w && k_norm_w ? w_bytes : 0u);
     mbar_arrive_expect_tx(&bar, first);
     bulk_load(rowbuf, qkv + (int64_t)tok * H * hd, row_bytes, &bar);
-    if (q_norm_w) bulk_load(qwbuf, q_norm_w, w_bytes, &bar);
-    if (k_norm_w) bulk_load(kwbuf, k_norm_w, w_bytes, &bar);
+    if (stage_w && q_norm_w) bulk_load(qwbuf, q_norm_w, w_bytes, &bar);
+    if (stage_w && k_norm_w) bulk_load(kwbuf, k_norm_w, w_bytes, &bar);
     const int p = __ldg(positions + tok);
     const bool ok = p >= 0 && p < max_pos && p < capacity;
     s_pos = ok ? p : -1;
@@ -653,6 +743,36 @@ frt_status launch_dt(int P, int GP, int epi, const Args& a, bool tma, cudaStream
   return P == 8 ? launch_p<DT, 8>(GP, epi, a, tma, st) : launch_p<DT, 4>(GP, epi, a, tma, st);
 }
 
+// The bulk-copy kernel at its LayerNorm level (EPI 3), P = 8 rows.
+template <int DT, int GP>
+frt_status launch_ln_gp(const Args& a, cudaStream_t st) {
+  static std::atomic<int> opted{0};
+  auto kt = qkv_norm_rope_kvcache_tma_kernel<DT, 8, GP, 3>;
+  const size_t smem = tma_smem(a.H, a.Hkv, a.hd, false);
+  const frt_status os = opt_in_smem(kt, smem, opted);
+  if (os != FRT_OK) return os;
+  const int per = a.Hq + a.Hkv;
+  int NG = (per * GP <= 128) ? per : 128 / GP;
+  if (NG < 1) NG = 1;
+  const int threads = ((NG * GP + 31) / 32) * 32;
+  return launch(kt, dim3((unsigned)a.M), dim3(threads), smem, st, static_cast<const uint16_t*>(a.qkv),
+                static_cast<const uint16_t*>(a.qw), static_cast<const uint16_t*>(a.kw), a.cos_tab, a.sin_tab, a.pos,
+                static_cast<uint16_t*>(a.q_out), a.kc, a.vc, a.status, a.H, NG, a.Hq, a.Hkv, a.hd, a.G, a.max_pos,
+                a.capacity, a.eps, a.ep);
+}
+
+template <int DT>
+frt_status launch_ln_tma(int GP, const Args& a, cudaStream_t st) {
+  switch (GP) {
+    case 1: return launch_ln_gp<DT, 1>(a, st);
+    case 2: return launch_ln_gp<DT, 2>(a, st);
+    case 4: return launch_ln_gp<DT, 4>(a, st);
+    case 8: return launch_ln_gp<DT, 8>(a, st);
+    case 16: return launch_ln_gp<DT, 16>(a, st);
+    default: return launch_ln_gp<DT, 32>(a, st);
+  }
+}
+
 // Shared validation and dispatch of both entry points.
 frt_status qkv_op(const void* qkv, const void* q_norm_w, const void* k_norm_w, const float* cos_tab,
                   const float* sin_tab, const int32_t* positions, void* q_out, void* k_cache, void* v_cache,
@@ -683,7 +803,7 @@ frt_status qkv_op(const void* qkv, const void* q_norm_w, const void* k_norm_w, c
   while (GP < G) GP *= 2;
   Args a{qkv, q_norm_w, k_norm_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status,
          M, H, Hq, Hkv, hd, G, max_pos, capacity, eps,
-         Epilogue{q_scale, q_layout == FRT_Q_HEAD_MAJOR ? 1 : 0, M, kv_scales}};
+         Epilogue{q_scale, q_layout == FRT_Q_HEAD_MAJOR ? 1 : 0, M, kv_scales, nullptr, nullptr}};
   if ((int64_t)M * qkv_shape(M, H, GP, kv8).nhb > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
   // Bulk-copy path for large batches when every row it moves is 16-byte
   // aligned (bulk copies need 16-byte addresses and sizes) and fits in
@@ -745,21 +865,45 @@ extern "C" frt_status frt_qkv_layernorm_rope_kvcache(const void* qkv, const void
   const int G = (hd / 2) / P;
   int GP = 1;
   while (GP < G) GP *= 2;
-  const int NG = H * GP <= 512 ? H : 512 / GP;  // up to 512 threads: the affine rows need the registers
-  const int nhb = (H + NG - 1) / NG;
+  // Small batches: one head per lane group, up to 512 threads per token.
+  // Large batches: up to four heads per group (more bytes in flight per
+  // thread), at most 256 threads.
+  const bool large = M >= 4 * 148;
+  int NG, HPG;
+  if (large && H >= 2) {
+    NG = (H + 3) / 4;
+    if (NG * GP > 256) NG = 256 / GP;
+    HPG = 4;
+  } else {
+    NG = H * GP <= 512 ? H : 512 / GP;
+    HPG = 1;
+  }
+  const int nhb = (H + NG * HPG - 1) / (NG * HPG);
   if ((int64_t)M * nhb > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
   const int threads = ((NG * GP + 31) / 32) * 32;
   const dim3 grid((unsigned)((int64_t)M * nhb));
+  // Large batches with 16-byte rows: the bulk-copy kernel at its LayerNorm
+  // level (the token's row staged in shared memory, 10 tokens per SM).
+  if (large && P == 8 && aligned(qkv, 16) && aligned(q_out, 16) && aligned(k_cache, 16) && aligned(v_cache, 16) &&
+      tma_smem(H, Hkv, hd, false) <= kTmaSmemMax) {
+    Args a{qkv, q_w, k_w, cos_tab, sin_tab, positions, q_out, k_cache, v_cache, status, M, H, Hq, Hkv, hd, G,
+           max_pos, capacity, eps,
+           Epilogue{1.0f, 0, M, nullptr, static_cast<const uint16_t*>(q_b), static_cast<const uint16_t*>(k_b)}};
+    return dt == FRT_F16 ? launch_ln_tma<FRT_F16>(GP, a, stream) : launch_ln_tma<FRT_BF16>(GP, a, stream);
+  }
   const uint16_t* qk = static_cast<const uint16_t*>(qkv);
   const uint16_t* w16[4] = {static_cast<const uint16_t*>(q_w), static_cast<const uint16_t*>(q_b),
                             static_cast<const uint16_t*>(k_w), static_cast<const uint16_t*>(k_b)};
   uint16_t* qo = static_cast<uint16_t*>(q_out);
   uint16_t* kc = static_cast<uint16_t*>(k_cache);
   uint16_t* vc = static_cast<uint16_t*>(v_cache);
-#define FRT_LN_LAUNCH(DT_, P_, GP_)                                                                                 \
-  return launch(qkv_layernorm_rope_kvcache_kernel<DT_, P_, GP_>, grid, dim3(threads), 0, stream, qk, w16[0], w16[1], \
-                w16[2], w16[3], cos_tab, sin_tab, positions, qo, kc, vc, status, H, NG, nhb, Hq, Hkv, hd, G, max_pos, \
-                capacity, eps)
+#define FRT_LN_LAUNCH(DT_, P_, GP_)                                                                            \
+  return HPG == 1 ? launch(qkv_layernorm_rope_kvcache_kernel<DT_, P_, GP_, 1>, grid, dim3(threads), 0, stream, qk, \
+                           w16[0], w16[1], w16[2], w16[3], cos_tab, sin_tab, positions, qo, kc, vc, status, H, NG, \
+                           nhb, Hq, Hkv, hd, G, max_pos, capacity, eps)                                            \
+                  : launch(qkv_layernorm_rope_kvcache_kernel<DT_, P_, GP_, 4>, grid, dim3(threads), 0, stream, qk, \
+                           w16[0], w16[1], w16[2], w16[3], cos_tab, sin_tab, positions, qo, kc, vc, status, H, NG, \
+                           nhb, Hq, Hkv, hd, G, max_pos, capacity, eps)
 #define FRT_LN_GP(DT_, P_)          \
   switch (GP) {                     \
     case 1: FRT_LN_LAUNCH(DT_, P_, 1);  \

@@ -32,9 +32,12 @@ constexpr int max_threads() {
 }
 
 // LN (NEXT-4, the ViT "add_layer_norm" producer): LayerNorm instead of
-// RMSNorm, y = (h - mean) * rstd * w + b with mean and the centred sum of
-// squares from two fp64 reductions over the register-held row, and y formed
-// in fp64 and rounded once to fp32 (bias may be null).
+// RMSNorm, y = (h - mean) * rstd * w + b (bias may be null).  The row sum and
+// the centred sum of squares are two reductions over the register-held row
+// (fp32 per thread, fp64 across threads); per element h - mean is formed
+// against the mean split into two floats (error ~1 ulp of the difference, so
+// a large common offset in the row costs no accuracy) and y carries a few
+// fp32 roundings (FP8 codes are 2^-4 apart).
 template <int DT, int K, bool WEIGHTED, int QM, bool LN>
 __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     const uint4* __restrict__ x, const uint4* r_in, uint4* r_out, const uint4* __restrict__ w,
@@ -92,7 +95,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       for (int e = 0; e < 4; ++e) {
         const float2 hf = P16::to_float2(hw[e]);
         if (LN) {  // the row sum first (the centred squares need the mean)
-          ss[k] += (double)hf.x + (double)hf.y;
+          ss[k] += (double)(hf.x + hf.y);
         } else {
           ss[k] = fma((double)hf.x, (double)hf.x, ss[k]);
           ss[k] = fma((double)hf.y, (double)hf.y, ss[k]);
@@ -119,11 +122,13 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   double tot = 0.0;
   const int nw = T >> 5;
   for (int i = 0; i < nw; ++i) tot += red[i];
-  double mean = 0.0;
+  float mean_hi = 0.0f, mean_lo = 0.0f;
   if (LN) {
     // second reduction: the centred sum of squares of the held row
-    mean = tot / (double)D;
-    double sc = 0.0;
+    const double mean = tot / (double)D;
+    mean_hi = (float)mean;
+    mean_lo = (float)(mean - (double)mean_hi);
+    float scf = 0.0f;
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       if (t + k * T < C) {
@@ -131,11 +136,12 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 hf = P16::to_float2(hw[e]);
-          const double d0 = (double)hf.x - mean, d1 = (double)hf.y - mean;
-          sc = fma(d0, d0, fma(d1, d1, sc));
+          const float d0 = (hf.x - mean_hi) - mean_lo, d1 = (hf.y - mean_hi) - mean_lo;
+          scf = fmaf(d0, d0, fmaf(d1, d1, scf));
         }
       }
     }
+    double sc = (double)scf;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, o);
     __syncthreads();  // every thread has read the first partials
@@ -146,6 +152,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   }
   const double rstd64 = rsqrt_f64(tot / (double)D + (double)eps);
   const Split32 rstd(rstd64);
+  const float rstd32 = (float)rstd64;
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
   const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * s_static) : 0.0f;  // NVFP4: RN(1 / RN(6 gs))
 
@@ -167,17 +174,13 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 hf = P16::to_float2(hw[e]);
-        const float2 wf = P16::to_float2(ww[e]);
+        const float2 wf = WEIGHTED ? P16::to_float2(ww[e]) : make_float2(1.0f, 1.0f);
         const float2 bf = P16::to_float2(bw[e]);
-        double y0 = ((double)hf.x - mean) * rstd64, y1 = ((double)hf.y - mean) * rstd64;
-        if (WEIGHTED) {
-          y0 *= (double)wf.x;
-          y1 *= (double)wf.y;
-        }
+        const float d0 = ((hf.x - mean_hi) - mean_lo) * rstd32, d1 = ((hf.y - mean_hi) - mean_lo) * rstd32;
         // bias zeros when absent; lanes past the row end hold 0 (they take
         // part in the block amax)
-        y[2 * e] = valid ? (float)(y0 + (double)bf.x) : 0.0f;
-        y[2 * e + 1] = valid ? (float)(y1 + (double)bf.y) : 0.0f;
+        y[2 * e] = valid ? fmaf(d0, wf.x, bf.x) : 0.0f;
+        y[2 * e + 1] = valid ? fmaf(d1, wf.y, bf.y) : 0.0f;
       }
     } else if (WEIGHTED && valid) {
       const uint4 wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : __ldg(w + c);
