@@ -198,6 +198,55 @@ frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* 
                             cudaStream_t stream);
 
 /*
+ * NEXT-4: the layer chain as one persistent kernel (small batches).
+ * "FlashFormer: Whole-Model Kernels for Efficient Low-Batch Inference" (the
+ * whole sequence in one kernel); the chain is the graphed one: for each of
+ * `steps` steps and each layer l, in order,
+ *   frt_residual_rmsnorm_fp8(x_attn[l], residual, residual, w_attn[l], q8_attn[l], scales[0] / bs_attn[l])
+ *   frt_qkv_norm_rope_kvcache(qkv[l], q_norm_w[l], k_norm_w[l], cos, sin, positions, q_out[l], k_cache[l], v_cache[l])
+ *   frt_residual_rmsnorm_fp8(x_ffn[l], residual, residual, w_ffn[l], q8_ffn[l], scales[1] / bs_ffn[l])
+ *   frt_gate_act_fp8(gate_up[l], act8[l], scales[2] / bs_act[l])
+ * with the same results as those launches (the residual stream carries from
+ * op to op).  Every op of the chain reads only its own row of each buffer, so
+ * one CTA per row runs the row's whole chain in one launch.
+ *
+ *   layers      device array [n_layers] of frt_chain_layer (pointers as in the
+ *               per-op calls; weights may be NULL; bs_* used with BLOCK128).
+ *   residual    device [M, D] 16-bit, updated in place.
+ *   scales      device fp32[3] (attention norm, FFN norm, activation), read
+ *               with STATIC.
+ *   status      as op (b), or NULL.
+ *   Supported: D % 8 == 0 and D <= 8192, hd % 16 == 0 and hd <= 256,
+ *   I % 128 == 0 (else FRT_ERR_UNSUPPORTED); all pointers aligned as the
+ *   per-op calls require (not re-checked per layer on the host).
+ */
+typedef struct frt_chain_layer {
+  const void* x_attn;   /* [M, D] */
+  const void* x_ffn;    /* [M, D] */
+  const void* w_attn;   /* [D] or NULL */
+  const void* w_ffn;    /* [D] or NULL */
+  const void* qkv;      /* [M, (Hq+2Hkv) hd] */
+  const void* q_norm_w; /* [hd] or NULL */
+  const void* k_norm_w; /* [hd] or NULL */
+  const void* gate_up;  /* [M, 2I] interleaved */
+  void* k_cache;        /* [capacity, Hkv, hd] */
+  void* v_cache;        /* [capacity, Hkv, hd] */
+  void* q_out;          /* [M, Hq, hd] */
+  uint8_t* q8_attn;     /* [M, D] */
+  uint8_t* q8_ffn;      /* [M, D] */
+  uint8_t* act8;        /* [M, I] */
+  float* bs_attn;       /* [M, ceil(D/128)] or NULL */
+  float* bs_ffn;        /* [M, ceil(D/128)] or NULL */
+  float* bs_act;        /* [M, I/128] or NULL */
+} frt_chain_layer;
+
+frt_status frt_chain_persistent(const frt_chain_layer* layers, int n_layers, int steps, void* residual,
+                                const float* cos_tab, const float* sin_tab, const int32_t* positions,
+                                const float* scales, int32_t* status, int M, int D, int Hq, int Hkv, int hd, int I,
+                                int max_pos, int capacity, float eps, frt_dtype dt, frt_quant qm, frt_act act,
+                                cudaStream_t stream);
+
+/*
  * NEXT-4: LayerNorm variants.
  *
  * frt_residual_layernorm_fp8 / _nvfp4: the ViT "add_layer_norm" producer (the

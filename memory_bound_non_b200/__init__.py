@@ -28,7 +28,8 @@ ACT = {"gelu_tanh": 0, "silu": 1, "relu2": 2}
 
 # C entry points declared in include/frt.h
 EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_act_fp8",
-           "frt_residual_layernorm_fp8", "frt_residual_layernorm_nvfp4", "frt_qkv_layernorm_rope_kvcache",
+           "frt_chain_persistent", "frt_residual_layernorm_fp8", "frt_residual_layernorm_nvfp4",
+           "frt_qkv_layernorm_rope_kvcache",
            "frt_residual_rmsnorm_nvfp4", "frt_gate_act_nvfp4", "frt_qkv_norm_rope_prepq_kvcache",
            "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_status_string")
 
@@ -58,6 +59,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_qkv_norm_rope_kvcache.restype = i32
     L.frt_qkv_norm_rope_prepq_kvcache.argtypes = [vp] * 10 + [i32] * 6 + [f32, f32, i32, i32, vp, i32, vp]
     L.frt_qkv_norm_rope_prepq_kvcache.restype = i32
+    L.frt_chain_persistent.argtypes = [vp, i32, i32] + [vp] * 6 + [i32] * 8 + [f32, i32, i32, i32, vp]
+    L.frt_chain_persistent.restype = i32
     L.frt_residual_layernorm_fp8.argtypes = [vp] * 8 + [i32, i32, f32, i32, i32, vp]
     L.frt_residual_layernorm_fp8.restype = i32
     L.frt_residual_layernorm_nvfp4.argtypes = [vp] * 8 + [i32, i32, f32, i32, i32, vp]
@@ -196,6 +199,36 @@ def frt_qkv_layernorm_rope_kvcache(qkv, q_w, q_b, k_w, k_b, cos_tab, sin_tab, po
         _ptr(q_out), _ptr(k_cache), _ptr(v_cache), _ptr(status), M, Hq, Hkv, hd, cos_tab.shape[0], k_cache.shape[0],
         float(eps), DTYPE[qkv.dtype], _stream(stream))
     _check("frt_qkv_layernorm_rope_kvcache", st)
+
+
+# field order of frt_chain_layer (include/frt.h)
+CHAIN_LAYER_FIELDS = ("x_attn", "x_ffn", "w_attn", "w_ffn", "qkv", "q_norm_w", "k_norm_w", "gate_up", "k_cache",
+                      "v_cache", "q_out", "q8_attn", "q8_ffn", "act8", "bs_attn", "bs_ffn", "bs_act")
+
+
+def chain_layer_table(layers, device):
+    """Device array of frt_chain_layer structs (17 pointers each) for a list of
+    objects carrying the CHAIN_LAYER_FIELDS tensors (or None)."""
+    import ctypes as c
+    host = (c.c_uint64 * (len(CHAIN_LAYER_FIELDS) * len(layers)))()
+    for i, L in enumerate(layers):
+        for j, name in enumerate(CHAIN_LAYER_FIELDS):
+            t = getattr(L, name)
+            host[i * len(CHAIN_LAYER_FIELDS) + j] = 0 if t is None else t.data_ptr()
+    buf = torch.frombuffer(bytearray(bytes(host)), dtype=torch.uint8)
+    return buf.to(device)
+
+
+def frt_chain_persistent(table, n_layers, steps, residual, cos_tab, sin_tab, positions, scales, status, Hq, Hkv,
+                         hd, I, capacity, eps=1e-6, quant="static", act="gelu_tanh", stream=None):
+    """NEXT-4: steps x layers x (norm, QKV, norm, gate) as one kernel launch;
+    table from chain_layer_table."""
+    M, D = residual.shape
+    st = load().frt_chain_persistent(
+        _ptr(table), n_layers, steps, _ptr(residual), _ptr(cos_tab), _ptr(sin_tab), _ptr(positions), _ptr(scales),
+        _ptr(status), M, D, Hq, Hkv, hd, I, cos_tab.shape[0], capacity, float(eps), DTYPE[residual.dtype],
+        QUANT[quant], ACT[act], _stream(stream))
+    _check("frt_chain_persistent", st)
 
 
 Q_LAYOUT = {"token": 0, "head": 1}

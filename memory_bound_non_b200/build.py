@@ -3,10 +3,13 @@
     python -m memory_bound_non_b200.build        # build if sources changed
     python -m memory_bound_non_b200.build -f     # force
 """
+import concurrent.futures
 import glob
 import os
+import shutil
 import subprocess
 import sys
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -37,16 +40,39 @@ def _stale():
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object in parallel (one nvcc per file),
+    then link the shared library."""
     if not force and not _stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [nvcc] + NVCC_FLAGS + ["-I", INCLUDE, "-I", CSRC, "-o", tmp] + sources()
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    objdir = tempfile.mkdtemp(prefix="frt_build_")
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    jobs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [nvcc] + compile_flags + ["-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        jobs.append((cmd, obj))
+    try:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as pool:
+            results = list(pool.map(lambda j: subprocess.run(j[0], capture_output=True, text=True), jobs))
+        failed = False
+        for (cmd, _), r in zip(jobs, results):
+            if r.stdout or r.stderr:
+                sys.stdout.write(r.stdout)
+                sys.stderr.write(r.stderr)
+            if r.returncode != 0:
+                failed = True
+                sys.stderr.write("failed: %s\n" % " ".join(cmd))
+        if failed:
+            raise subprocess.CalledProcessError(1, "nvcc")
+        tmp = LIB + ".tmp.%d" % os.getpid()
+        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp] +
+                       [o for _, o in jobs], check=True)
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(objdir, ignore_errors=True)
     return LIB
 
 

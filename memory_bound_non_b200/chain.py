@@ -23,7 +23,8 @@ from typing import List, Optional
 
 import torch
 
-from . import frt_gate_act_fp8, frt_qkv_norm_rope_kvcache, frt_residual_rmsnorm_fp8
+from . import (chain_layer_table, frt_chain_persistent, frt_gate_act_fp8, frt_qkv_norm_rope_kvcache,
+               frt_residual_rmsnorm_fp8)
 from .workloads import Inputs, Workload
 
 
@@ -123,6 +124,26 @@ class LayerChain:
         for _ in range(self.wl.steps if steps is None else steps):
             for l in range(len(self.layers)):
                 self.layer(l, stream)
+
+    def run_persistent(self, steps=None, stream=None):
+        """The same chain as one persistent kernel launch (one CTA per row runs
+        the row's steps x layers x 4 ops; see frt_chain_persistent)."""
+        wl = self.wl
+        if getattr(self, "_table", None) is None:
+            self._table = chain_layer_table(self.layers, self.device)
+        frt_chain_persistent(self._table, len(self.layers), wl.steps if steps is None else steps, self.residual,
+                             self.cos, self.sin, self.positions, self.scales, self.status, wl.Hq, wl.Hkv, wl.hd, wl.I,
+                             self.layers[0].k_cache.shape[0], eps=wl.eps, quant=wl.quant, act=wl.act, stream=stream)
+
+    def capture_persistent(self, steps=None):
+        """One-node CUDA graph of the persistent chain (warmed up once first)."""
+        self.run_persistent(steps=1)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run_persistent(steps=steps)
+        self.graph_persistent = g
+        return g
 
     @property
     def launches_per_chain(self) -> int:

@@ -267,6 +267,28 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------------- activations --
+constexpr float kSqrt2OverPi = 0.7978845608028654f;
+constexpr float kGeluCubic = 0.044715f;
+
+// act(g) in fp32.  GELU-tanh uses 0.5 (1 + tanh(z)) = 1 / (1 + exp(-2 z)) and
+// SiLU is g / (1 + exp(-g)); the exponent is capped at 80 so the denominator
+// stays finite (the result is ~0 there either way).
+template <int ACT>
+__device__ __forceinline__ float act_fn(float g) {
+  if (ACT == FRT_ACT_RELU2) {
+    const float r = fmaxf(g, 0.0f);
+    return r * r;
+  } else if (ACT == FRT_ACT_SILU) {
+    const float e = expf(fminf(-g, 80.0f));
+    return __fdividef(g, 1.0f + e);
+  } else {
+    const float z = g * fmaf(kSqrt2OverPi * kGeluCubic, g * g, kSqrt2OverPi);
+    const float e = expf(fminf(-2.0f * z, 80.0f));
+    return __fdividef(g, 1.0f + e);
+  }
+}
+
 // --------------------------------------------------------- reductions --
 template <int WIDTH>
 __device__ __forceinline__ float group_sum(float v) {

@@ -25,27 +25,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kU = 4;  // scale blocks per warp
 
-constexpr float kSqrt2OverPi = 0.7978845608028654f;
-constexpr float kGeluCubic = 0.044715f;
-
-// act(g) in fp32.  GELU-tanh uses 0.5 (1 + tanh(z)) = 1 / (1 + exp(-2 z)) and
-// SiLU is g / (1 + exp(-g)); the exponent is capped at 80 so the denominator
-// stays finite (the result is ~0 there either way).
-template <int ACT>
-__device__ __forceinline__ float act_fn(float g) {
-  if (ACT == FRT_ACT_RELU2) {
-    const float r = fmaxf(g, 0.0f);
-    return r * r;
-  } else if (ACT == FRT_ACT_SILU) {
-    const float e = expf(fminf(-g, 80.0f));
-    return __fdividef(g, 1.0f + e);
-  } else {
-    const float z = g * fmaf(kSqrt2OverPi * kGeluCubic, g * g, kSqrt2OverPi);
-    const float e = expf(fminf(-2.0f * z, 80.0f));
-    return __fdividef(g, 1.0f + e);
-  }
-}
-
 template <int DT, int ACT, int QM, bool FULL>
 __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __restrict__ gu,
                                                                  uint32_t* __restrict__ q,

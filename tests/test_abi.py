@@ -186,3 +186,17 @@ def qln_call(M=4, Hq=8, Hkv=2, hd=128, qkv=A, qw=None, qb=None, kw=None, kb=None
 ])
 def test_qkv_layernorm_host_validation(kw, want):
     assert qln_call(**kw) == want
+
+
+def chain_call(M=4, D=1024, Hq=8, Hkv=1, hd=128, I=4096, layers=A, n=2, steps=3, res=A, qm=0, act=0, dt=1):
+    return frt.load().frt_chain_persistent(layers, n, steps, res, A, A, A, A, None, M, D, Hq, Hkv, hd, I, 64, 64,
+                                           1e-6, dt, qm, act, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(hd=72), UNSUP), (dict(hd=264), UNSUP), (dict(D=8200), UNSUP), (dict(I=4100), UNSUP), (dict(D=12), INV),
+    (dict(Hq=6, Hkv=4), INV), (dict(act=5), INV), (dict(qm=3), INV), (dict(layers=None), INV),
+    (dict(res=A + 8), INV), (dict(M=0), OK), (dict(steps=0), OK), (dict(n=0, layers=None), OK), (dict(M=-1), INV),
+])
+def test_chain_persistent_host_validation(kw, want):
+    assert chain_call(**kw) == want

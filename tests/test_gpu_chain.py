@@ -94,3 +94,45 @@ def test_pdl_on_and_off_give_identical_results():
     finally:
         frt.frt_set_pdl(prev)
     assert all(torch.equal(a, b) for a, b in zip(*results))
+
+
+# ------------------------------------------------- NEXT-4: persistent chain ---
+@pytest.mark.parametrize("name,steps", [("pi05", 10), ("vla_denoise", 10), ("tiny", 3),
+                                        ("qwen3_prefill_S128", 2)])
+def test_persistent_chain_matches_oracle(name, steps):
+    wl = W.get(name, steps=steps, layers=max(W.get(name).layers, 2))
+    inp = W.make_inputs(wl)
+    scales = P.chain_scales(wl, inp)
+    chain = LayerChain(wl, inp, scales=scales)
+    chain.reset()
+    chain.run_persistent()
+    torch.cuda.synchronize()
+    r_ref, outs = P.oracle_chain(wl, inp, scales, steps)
+    compare_chain(wl, inp, chain, r_ref, outs)
+
+
+@pytest.mark.parametrize("name", ["pi05", "vla_denoise", "tiny"])
+def test_persistent_chain_equals_graphed_chain_bitwise(name):
+    """One launch for steps x layers x 4 ops gives the same bits as the
+    graph of per-op launches."""
+    wl = W.get(name, steps=3)
+    inp = W.make_inputs(wl)
+    chain = LayerChain(wl, inp, scales=P.chain_scales(wl, inp))
+    chain.capture()
+    chain.reset()
+    chain.replay()
+    torch.cuda.synchronize()
+    ref = [t.clone() for L in chain.layers for t in (L.q8_attn, L.q8_ffn, L.act8, L.q_out, L.k_cache, L.v_cache)]
+    r_ref = chain.residual.clone()
+    for L in chain.layers:               # clear the outputs so stale values cannot pass
+        for t in (L.q8_attn, L.q8_ffn, L.act8, L.q_out):
+            t.zero_()
+    chain.reset()
+    chain.capture_persistent()
+    chain.reset()
+    chain.graph_persistent.replay()
+    torch.cuda.synchronize()
+    bits = lambda t: t.view(torch.uint8)   # bit patterns: the fp16 cache sentinel 0x7E7E is a NaN
+    assert torch.equal(bits(chain.residual), bits(r_ref))
+    got = [t for L in chain.layers for t in (L.q8_attn, L.q8_ffn, L.act8, L.q_out, L.k_cache, L.v_cache)]
+    assert all(torch.equal(bits(a), bits(b)) for a, b in zip(ref, got))
