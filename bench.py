@@ -21,6 +21,7 @@ Also reported on the same JSON line:
                 (18 layers x 10 steps = 720 nodes) and the VLA denoise loop
                 (32 x 10 = 1280 nodes), each one CUDA graph, L2 flushed
                 between replays; per-node cost against the launch floor;
+                and the same chain as one persistent kernel ("persistent");
   launch_floor  an empty kernel per stream launch and per graph node;
   small_m       per-op microseconds at M <= 41 against the launch floor;
   next_ops      the widened ops timed alone (gated residual + AdaRMSNorm +
@@ -561,7 +562,18 @@ def chain_leg(reps, floor):
                      "hbm_bytes_per_chain": chain_bytes,
                      "hbm_us_at_8TBps": round(chain_bytes / NOMINAL_HBM_GBS / 1e3, 2),
                      "l2": "flushed before each replay (512 MiB write)"}
-        del ch
+        # the same chain as one persistent kernel (one launch per chain)
+        gp = ch.capture_persistent()
+        for _ in range(3):
+            gp.replay()
+        torch.cuda.synchronize()
+        pmed, _ = time_graph(gp, reps, flush, s)
+        out[name]["persistent"] = {"us_per_chain": round(pmed, 2), "launches": 1,
+                                   "us_per_op": round(pmed / nodes, 3),
+                                   "x_graph_node_floor": round(pmed / nodes / floor["graph_node_us"], 3),
+                                   "speedup_vs_graph": round(med / pmed, 2),
+                                   "l2": "flushed before each replay (512 MiB write)"}
+        del ch, gp
     return out
 
 

@@ -216,9 +216,13 @@ frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* 
  *   scales      device fp32[3] (attention norm, FFN norm, activation), read
  *               with STATIC.
  *   status      as op (b), or NULL.
- *   Supported: D % 8 == 0 and D <= 8192, hd % 16 == 0 and hd <= 256,
+ *   Supported: D % 8 == 0 and D <= 8192, hd % 16 == 0 and 64 <= hd <= 256,
  *   I % 128 == 0 (else FRT_ERR_UNSUPPORTED); all pointers aligned as the
  *   per-op calls require (not re-checked per layer on the host).
+ *   Each row is run by a thread-block cluster of up to 8 CTAs, sized so that
+ *   the clusters of all M rows fill the GPU: one runs the row's residual chain
+ *   (the norms), the others split the heads and activation blocks and run
+ *   alongside it.
  */
 typedef struct frt_chain_layer {
   const void* x_attn;   /* [M, D] */

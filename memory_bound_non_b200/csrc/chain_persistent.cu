@@ -7,18 +7,26 @@
 // (FFN norm), op c (gated activation) ("FlashRT kernel fusion", §二 steps 1,
 // 3, 7, 8-10; §三 for the per-step loop).
 //
-// Mapping (B200): one CTA of 256 threads per token row.  The chain's only
-// dependency is the residual stream of each row (a -> a -> next layer's a);
-// the QKV and gate/up buffers that ops b and c read are the fixed per-layer
-// outputs of GEMMs that are not part of the chain, so every op of a row
-// depends on that row alone and the CTA runs the row's whole chain in program
-// order, with the residual row held in registers from the first op to the
-// last (written back once).  No grid-wide barrier is needed; with real GEMMs
-// between the ops it would be (those mix rows).  Each op uses the arithmetic
-// of its per-op kernel (packed 16-bit add, fp64 row sum of squares, correctly
-// rounded FP8 decisions, the same RoPE and activation expressions).
+// Mapping (B200).  The chain's only dependency is the residual stream of each
+// row (a -> a -> next layer's a); the QKV and gate/up buffers that ops b and c
+// read are the fixed per-layer outputs of GEMMs that are not part of the
+// chain, so a row's ops depend on that row alone, and ops b and c do not
+// depend on the residual at all.  Each row is owned by a thread-block cluster
+// of S CTAs (S <= 8, so that rows x S fills the SMs) that runs the row's whole
+// chain in one launch with no grid-wide barrier and no cross-CTA exchange:
+// CTA 0 runs the residual chain (both norms of every layer, the residual row
+// in registers from the first op to the last), while CTAs 1..S-1 split the
+// heads of op b and the 128-output blocks of op c between them and run
+// alongside (with S == 1 one CTA does everything in order).  Each CTA copies
+// the next layer invocation's input slices into a second shared-memory stage
+// (asynchronous copies) while the current one computes.  With real GEMMs
+// between the ops, rows would mix and a grid-wide step would be needed.  Each
+// op uses the arithmetic of its per-op kernel (packed 16-bit add, fp64 row sum
+// of squares, correctly rounded FP8 decisions, the same RoPE and activation
+// expressions), so the results equal the per-op launches bit for bit.
 #include <atomic>
 #include <cmath>
+#include <cooperative_groups.h>
 
 #include "frt_device.cuh"
 #include "frt_host.h"
@@ -26,10 +34,12 @@
 namespace frt {
 namespace {
 
+namespace cg = cooperative_groups;
+
 constexpr int kChainThreads = 256;
 constexpr int kChainWarps = kChainThreads / 32;
 
-// Block-wide fp64 sum (warp butterfly, then the warp partials in order); the
+// CTA-wide fp64 sum (warp butterfly, then the warp partials in order); the
 // trailing barrier lets the next call reuse `red`.
 __device__ __forceinline__ double block_sum(double v, double* red) {
 #pragma unroll
@@ -42,27 +52,34 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
   return tot;
 }
 
-// Op a on this CTA's row: h = x + r (into hv), RMSNorm, FP8 codes.
+// The cluster's slices of one row.
+struct Slice {
+  int c0, nc;  // 16-byte chunks of the D columns
+  int h0, nh;  // heads
+  int b0, nb;  // 128-output activation blocks
+};
+
+// Op a on the row (held by this CTA): h = x + r (into hv), RMSNorm, FP8 codes.
 template <int DT, int K, int QM>
-__device__ __forceinline__ void chain_norm(const uint4* __restrict__ x, const uint4* __restrict__ w, uint2* q,
-                                           float* bs, const Divisor& dv, uint4 (&hv)[K], int64_t row, int C, int NB,
-                                           float D, float eps, double* red) {
+__device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uint2* q, float* bs, const Divisor& dv,
+                                           uint4 (&hv)[K], int64_t row, const Slice& sl, int C, int NB, float D,
+                                           float eps, double* red) {
   using P16 = Pack16<DT>;
   const int t = threadIdx.x;
   uint4 xv[K], wv[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = t + k * kChainThreads;
-    if (c < C) {
-      xv[k] = ld_stream(x + row * C + c);
-      if (w != nullptr) wv[k] = __ldg(w + c);
+    const int j = t + k * kChainThreads;
+    if (j < sl.nc) {
+      xv[k] = xs[j];
+      if (ws != nullptr) wv[k] = ws[j];
     }
   }
   double ss[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     ss[k] = 0.0;
-    if (t + k * kChainThreads < C) {
+    if (t + k * kChainThreads < sl.nc) {
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv[k]);
       uint32_t* hw = reinterpret_cast<uint32_t*>(&hv[k]);
 #pragma unroll
@@ -78,18 +95,20 @@ __device__ __forceinline__ void chain_norm(const uint4* __restrict__ x, const ui
   double sst = ss[0];
 #pragma unroll
   for (int k = 1; k < K; ++k) sst += ss[k];
-  const Split32 rstd(rsqrt_f64(block_sum(sst, red) / (double)D + (double)eps));
+  const double tot = block_sum(sst, red);
+  const Split32 rstd(rsqrt_f64(tot / (double)D + (double)eps));
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = t + k * kChainThreads;
-    const bool valid = c < C;
+    const int j = t + k * kChainThreads;
+    const bool valid = j < sl.nc;
+    const int c = sl.c0 + j;
     const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv[k]);
     const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv[k]);
     float y[8];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 hf = P16::to_float2(hw[e]);
-      if (w != nullptr && valid) {
+      if (ws != nullptr && valid) {
         const float2 wf = P16::to_float2(ww[e]);
         y[2 * e] = rstd.mul(hf.x * wf.x);
         y[2 * e + 1] = rstd.mul(hf.y * wf.y);
@@ -102,7 +121,7 @@ __device__ __forceinline__ void chain_norm(const uint4* __restrict__ x, const ui
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
       am = group_max<16>(am);
       const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
-      if (valid && (t & 15) == 0) bs[row * NB + (c >> 4)] = sb;
+      if (valid && (j & 15) == 0) bs[row * NB + (c >> 4)] = sb;
       if (valid) q[row * C + c] = quant8(y, Divisor(sb));
     } else if (valid) {
       q[row * C + c] = quant8(y, dv);
@@ -110,22 +129,20 @@ __device__ __forceinline__ void chain_norm(const uint4* __restrict__ x, const ui
   }
 }
 
-// Op b on this CTA's token: lane groups of GP lanes per head (P = 8 elements
-// and their rotation partners per lane), T / GP heads per slot.
+// Op b on this CTA's heads: lane groups of GP lanes per head (P = 8 elements
+// and their rotation partners per lane), kChainThreads / GP heads per pass.
 template <int DT, int GP>
-__device__ __forceinline__ void chain_qkv(const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ qw,
-                                          const uint16_t* __restrict__ kw, uint16_t* q_out, uint16_t* k_cache,
-                                          uint16_t* v_cache, const float* c, const float* s, int64_t row, int p,
-                                          bool row_ok, int Hq, int Hkv, int hd, int G, float eps) {
+__device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t* qw, const uint16_t* kw,
+                                          uint16_t* q_out, uint16_t* k_cache, uint16_t* v_cache, const float* c,
+                                          const float* s, int64_t row, int p, bool row_ok, const Slice& sl, int Hq,
+                                          int Hkv, int hd, int G, float eps) {
   constexpr int P = 8;
-  const int H = Hq + 2 * Hkv;
   const int NG = kChainThreads / GP;
   const int grp = threadIdx.x / GP;
   const int li = threadIdx.x & (GP - 1);
   const int half = hd >> 1;
   const int j0 = li * P;
   const bool lane_ok = li < G && row_ok;
-  const uint16_t* rowp = qkv + row * H * hd;
   uint4 qwa = make_uint4(0, 0, 0, 0), qwb = qwa, kwa = qwa, kwb = qwa;
   if (lane_ok) {
     if (qw != nullptr) {
@@ -137,17 +154,18 @@ __device__ __forceinline__ void chain_qkv(const uint16_t* __restrict__ qkv, cons
       kwb = *reinterpret_cast<const uint4*>(kw + half + j0);
     }
   }
-  for (int h0 = 0; h0 < H; h0 += NG) {
-    const int h = h0 + grp;
-    const bool on = lane_ok && h < H;
+  for (int i0 = 0; i0 < sl.nh; i0 += NG) {
+    const int i = i0 + grp;  // head index within the slice
+    const int h = sl.h0 + i;
+    const bool on = lane_ok && i < sl.nh;
     const bool is_q = h < Hq;
     const bool is_v = h >= Hq + Hkv;
     const uint16_t* nw = is_q ? qw : kw;
     const bool do_norm = !is_v && nw != nullptr;
     uint4 va = make_uint4(0, 0, 0, 0), vb = va;
     if (on) {
-      va = *reinterpret_cast<const uint4*>(rowp + (int64_t)h * hd + j0);
-      vb = *reinterpret_cast<const uint4*>(rowp + (int64_t)h * hd + half + j0);
+      va = *reinterpret_cast<const uint4*>(heads + (int64_t)i * hd + j0);
+      vb = *reinterpret_cast<const uint4*>(heads + (int64_t)i * hd + half + j0);
     }
     if (on && is_v) {
       uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
@@ -203,103 +221,182 @@ __device__ __forceinline__ void chain_qkv(const uint16_t* __restrict__ qkv, cons
   }
 }
 
-// Op c on this CTA's row: each warp takes 128-output scale blocks, four at a
-// time with their loads issued first (one 16-byte load = 4 (g, u) pairs).
-template <int DT, int QM>
-__device__ __forceinline__ void chain_act(const uint4* __restrict__ gu, uint32_t* q, float* bs, const Divisor& dv,
-                                          int64_t row, int I4, int NBI, int act) {
+// Op c on this CTA's 128-output blocks: each warp takes blocks four at a time
+// with their loads issued first (one 16-byte load = 4 (g, u) pairs).
+template <int DT, int QM, int ACT>
+__device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* bs, const Divisor& dv, int64_t row,
+                                          const Slice& sl, int I4, int NBI) {
   using P16 = Pack16<DT>;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const uint4* src = gu + row * I4;
   uint32_t* dst = q + row * I4;
-  for (int b0 = warp * 4; b0 < NBI; b0 += kChainWarps * 4) {
+  for (int i0 = warp * 4; i0 < sl.nb; i0 += kChainWarps * 4) {
     uint4 v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      if (b0 + u < NBI) v[u] = ld_stream(src + (b0 + u) * 32 + lane);
+      if (i0 + u < sl.nb) v[u] = gs[(i0 + u) * 32 + lane];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      if (b0 + u >= NBI) break;  // uniform across the warp
+      if (i0 + u >= sl.nb) break;  // uniform across the warp
+      const int b = sl.b0 + i0 + u;
       float a[4];
       const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[u]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 pr = P16::to_float2(w[e]);
-        // the activation is uniform for the launch (a branch, not a template)
-        const float g = act == FRT_ACT_RELU2 ? act_fn<FRT_ACT_RELU2>(pr.x)
-                        : act == FRT_ACT_SILU ? act_fn<FRT_ACT_SILU>(pr.x)
-                                              : act_fn<FRT_ACT_GELU_TANH>(pr.x);
-        a[e] = g * pr.y;
+        a[e] = act_fn<ACT>(pr.x) * pr.y;
       }
       if (QM == FRT_QUANT_BLOCK128) {
         const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
         const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
-        if (lane == 0) bs[row * NBI + b0 + u] = sb;
-        dst[(b0 + u) * 32 + lane] = quant4(a, Divisor(sb));
+        if (lane == 0) bs[row * NBI + b] = sb;
+        dst[b * 32 + lane] = quant4(a, Divisor(sb));
       } else {
-        dst[(b0 + u) * 32 + lane] = quant4(a, dv);
+        dst[b * 32 + lane] = quant4(a, dv);
       }
     }
   }
 }
 
-template <int DT, int K, int QM, int GP>
+// 16-byte asynchronous global -> shared copy (L2 only) and its groups.
+__device__ __forceinline__ void cp_async16(uint4* smem, const void* gmem) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+
+// Offsets (16-byte chunks) of one stage of this CTA's slices: x_attn, x_ffn,
+// the two norm weights, the head slice of the QKV row, the q / k norm
+// weights, the block slice of the gate/up row.
+struct StageMap {
+  int xa, xf, wa, wf, qkv, qw, kw, gu, len;
+  __host__ __device__ StageMap(int cs, int heads16, int hd16, int gu16)
+      : xa(0), xf(cs), wa(2 * cs), wf(3 * cs), qkv(4 * cs), qw(4 * cs + heads16), kw(4 * cs + heads16 + hd16),
+        gu(4 * cs + heads16 + 2 * hd16), len(4 * cs + heads16 + 2 * hd16 + gu16) {}
+};
+
+__device__ __forceinline__ void stage_copy(uint4* dst, const void* src, int64_t off, int n) {
+  if (src == nullptr) return;
+  const uint4* s = static_cast<const uint4*>(src) + off;
+  for (int i = threadIdx.x; i < n; i += kChainThreads) cp_async16(dst + i, s + i);
+}
+
+// Copies every input slice one layer invocation of this CTA reads.
+__device__ __forceinline__ void stage_layer(uint4* st, const StageMap& m, const frt_chain_layer& L, int64_t row,
+                                            const Slice& sl, int C, int qkv16, int hd16, int I4) {
+  stage_copy(st + m.xa, L.x_attn, row * C + sl.c0, sl.nc);
+  stage_copy(st + m.xf, L.x_ffn, row * C + sl.c0, sl.nc);
+  stage_copy(st + m.wa, L.w_attn, sl.c0, sl.nc);
+  stage_copy(st + m.wf, L.w_ffn, sl.c0, sl.nc);
+  stage_copy(st + m.qkv, L.qkv, row * qkv16 + (int64_t)sl.h0 * hd16, sl.nh * hd16);
+  stage_copy(st + m.qw, L.q_norm_w, 0, hd16);
+  stage_copy(st + m.kw, L.k_norm_w, 0, hd16);
+  stage_copy(st + m.gu, L.gate_up, row * I4 + (int64_t)sl.b0 * 32, sl.nb * 32);
+}
+
+template <int DT, int K, int QM, int GP, int ACT>
 __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
     const frt_chain_layer* __restrict__ layers, int n_layers, int steps, uint4* residual,
     const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, const int32_t* __restrict__ positions,
     const float* __restrict__ scales, int32_t* status, int C, int NB, int Hq, int Hkv, int hd, int G, int I4,
-    int NBI, int max_pos, int capacity, float eps, int act) {
+    int NBI, int max_pos, int capacity, float eps) {
   __shared__ double red[kChainWarps];
   pdl_enter();
+  cg::cluster_group cl = cg::this_cluster();
+  const unsigned S = cl.num_blocks();
+  const int r = (int)cl.block_rank();
   const int t = threadIdx.x;
-  const int64_t row = blockIdx.x;
+  const int64_t row = blockIdx.x / S;
+  const int H = Hq + 2 * Hkv;
+  // roles: CTA 0 runs both norms on the whole row (the residual chain); the
+  // heads and activation blocks go to CTAs 1..S-1 (all to CTA 0 when S == 1)
+  const bool norm_cta = r == 0;
+  const int workers = S > 1 ? (int)S - 1 : 1;
+  const int w = S > 1 ? r - 1 : 0;
+  Slice sl;
+  sl.c0 = 0;
+  sl.nc = norm_cta ? C : 0;
+  const int hs = (H + workers - 1) / workers, bsl = (NBI + workers - 1) / workers;
+  const bool bc_cta = S == 1 || r > 0;
+  sl.h0 = bc_cta ? min(H, w * hs) : 0;
+  sl.nh = bc_cta ? min(H, sl.h0 + hs) - sl.h0 : 0;
+  sl.b0 = bc_cta ? min(NBI, w * bsl) : 0;
+  sl.nb = bc_cta ? min(NBI, sl.b0 + bsl) - sl.b0 : 0;
+
   uint4 hv[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = t + k * kChainThreads;
-    hv[k] = c < C ? residual[row * C + c] : make_uint4(0u, 0u, 0u, 0u);
+    const int j = t + k * kChainThreads;
+    hv[k] = j < sl.nc ? residual[row * C + sl.c0 + j] : make_uint4(0u, 0u, 0u, 0u);
   }
   const int p = __ldg(positions + row);
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
-  if (!row_ok && t == 0 && status != nullptr) atomicOr(status, 1);
-  // this lane's cos / sin slice of the token's position (op b)
+  if (!row_ok && t == 0 && r == 0 && status != nullptr) atomicOr(status, 1);
   constexpr int P = 8;
   const int li = t & (GP - 1);
   const int half = hd >> 1;
-  float cs[P], sn[P];
+  float cs8[P], sn8[P];
   if (row_ok && li < G) {
 #pragma unroll
     for (int e = 0; e < P; e += 4) {
       const float4 tc = __ldg(reinterpret_cast<const float4*>(cos_tab + (int64_t)p * half + li * P + e));
       const float4 ts = __ldg(reinterpret_cast<const float4*>(sin_tab + (int64_t)p * half + li * P + e));
-      cs[e] = tc.x, cs[e + 1] = tc.y, cs[e + 2] = tc.z, cs[e + 3] = tc.w;
-      sn[e] = ts.x, sn[e + 1] = ts.y, sn[e + 2] = ts.z, sn[e + 3] = ts.w;
+      cs8[e] = tc.x, cs8[e + 1] = tc.y, cs8[e + 2] = tc.z, cs8[e + 3] = tc.w;
+      sn8[e] = ts.x, sn8[e + 1] = ts.y, sn8[e + 2] = ts.z, sn8[e + 3] = ts.w;
     }
   }
   const Divisor dv_attn(QM == FRT_QUANT_STATIC ? __ldg(scales) : 1.0f);
   const Divisor dv_ffn(QM == FRT_QUANT_STATIC ? __ldg(scales + 1) : 1.0f);
   const Divisor dv_act(QM == FRT_QUANT_STATIC ? __ldg(scales + 2) : 1.0f);
   const float D = (float)(C * 8);
-  for (int step = 0; step < steps; ++step) {
-    for (int l = 0; l < n_layers; ++l) {
-      const frt_chain_layer& L = layers[l];
-      chain_norm<DT, K, QM>(static_cast<const uint4*>(L.x_attn), static_cast<const uint4*>(L.w_attn),
-                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, hv, row, C, NB, D, eps, red);
-      chain_qkv<DT, GP>(static_cast<const uint16_t*>(L.qkv), static_cast<const uint16_t*>(L.q_norm_w),
-                        static_cast<const uint16_t*>(L.k_norm_w), static_cast<uint16_t*>(L.q_out),
-                        static_cast<uint16_t*>(L.k_cache), static_cast<uint16_t*>(L.v_cache), cs, sn, row, p, row_ok,
-                        Hq, Hkv, hd, G, eps);
-      chain_norm<DT, K, QM>(static_cast<const uint4*>(L.x_ffn), static_cast<const uint4*>(L.w_ffn),
-                            reinterpret_cast<uint2*>(L.q8_ffn), L.bs_ffn, dv_ffn, hv, row, C, NB, D, eps, red);
-      chain_act<DT, QM>(static_cast<const uint4*>(L.gate_up), reinterpret_cast<uint32_t*>(L.act8), L.bs_act, dv_act,
-                        row, I4, NBI, act);
-    }
+  const int qkv16 = H * hd / 8, hd16 = hd / 8;
+  // this CTA's stage layout: only the slices of its own roles (the host sizes
+  // shared memory for the larger of the two layouts)
+  const StageMap m(norm_cta ? C : 0, bc_cta ? hs * hd16 : 0, hd16, bc_cta ? bsl * 32 : 0);
+
+  // dynamic shared memory: the layer table (so no iteration waits on a global
+  // load of its pointers), then the two stages
+  extern __shared__ uint4 smem[];
+  frt_chain_layer* tab = reinterpret_cast<frt_chain_layer*>(smem);
+  uint4* stages = smem + (n_layers * (int)sizeof(frt_chain_layer) + 15) / 16;
+  {
+    const uint64_t* src = reinterpret_cast<const uint64_t*>(layers);
+    uint64_t* dst = reinterpret_cast<uint64_t*>(tab);
+    const int words = n_layers * (int)(sizeof(frt_chain_layer) / 8);
+    for (int i = t; i < words; i += kChainThreads) dst[i] = __ldg(src + i);
+    __syncthreads();
+  }
+  const int total = steps * n_layers;
+  if (total > 0) {
+    stage_layer(stages, m, tab[0], row, sl, C, qkv16, hd16, I4);
+    cp_async_commit();
+  }
+  for (int it = 0; it < total; ++it) {
+    const frt_chain_layer& L = tab[it % n_layers];
+    if (it + 1 < total) stage_layer(stages + ((it + 1) & 1) * m.len, m, tab[(it + 1) % n_layers], row, sl, C, qkv16, hd16, I4);
+    cp_async_commit();  // possibly empty: one group per iteration
+    cp_async_wait1();   // this iteration's stage has landed (only the newest group may be pending)
+    __syncthreads();    // ... for every thread's copies
+    const uint4* st = stages + (it & 1) * m.len;
+    if (norm_cta)
+      chain_norm<DT, K, QM>(st + m.xa, L.w_attn != nullptr ? st + m.wa : nullptr,
+                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, hv, row, sl, C, NB, D, eps, red);
+    chain_qkv<DT, GP>(reinterpret_cast<const uint16_t*>(st + m.qkv),
+                      L.q_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.qw) : nullptr,
+                      L.k_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.kw) : nullptr,
+                      static_cast<uint16_t*>(L.q_out), static_cast<uint16_t*>(L.k_cache),
+                      static_cast<uint16_t*>(L.v_cache), cs8, sn8, row, p, row_ok, sl, Hq, Hkv, hd, G, eps);
+    if (norm_cta)
+      chain_norm<DT, K, QM>(st + m.xf, L.w_ffn != nullptr ? st + m.wf : nullptr, reinterpret_cast<uint2*>(L.q8_ffn),
+                            L.bs_ffn, dv_ffn, hv, row, sl, C, NB, D, eps, red);
+    chain_act<DT, QM, ACT>(st + m.gu, reinterpret_cast<uint32_t*>(L.act8), L.bs_act, dv_act, row, sl, I4, NBI);
+    __syncthreads();  // the stage read here is refilled at iteration it + 2
   }
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = t + k * kChainThreads;
-    if (c < C) residual[row * C + c] = hv[k];
+    const int j = t + k * kChainThreads;
+    if (j < sl.nc) residual[row * C + sl.c0 + j] = hv[k];
   }
 }
 
@@ -311,44 +408,60 @@ struct ChainArgs {
   const int32_t* positions;
   const float* scales;
   int32_t* status;
-  int M, C, NB, Hq, Hkv, hd, G, I4, NBI, max_pos, capacity;
+  int M, C, NB, Hq, Hkv, hd, G, I4, NBI, S, max_pos, capacity;
   float eps;
-  int act;
 };
 
+template <int DT, int K, int QM, int GP, int ACT>
+frt_status launch_chain(const ChainArgs& a, size_t smem, cudaStream_t st) {
+  static std::atomic<int> opted{0};
+  auto kern = chain_persistent_kernel<DT, K, QM, GP, ACT>;
+  const frt_status os = opt_in_smem(kern, smem, opted);
+  if (os != FRT_OK) return os;
+  return launch_cluster(kern, dim3((unsigned)(a.M * a.S)), dim3(kChainThreads), smem, st, (unsigned)a.S, a.layers,
+                        a.n_layers, a.steps, static_cast<uint4*>(a.residual), a.cos_tab, a.sin_tab, a.positions,
+                        a.scales, a.status, a.C, a.NB, a.Hq, a.Hkv, a.hd, a.G, a.I4, a.NBI, a.max_pos, a.capacity,
+                        a.eps);
+}
+
 template <int DT, int K, int QM, int GP>
-frt_status launch_chain(const ChainArgs& a, cudaStream_t st) {
-  return launch(chain_persistent_kernel<DT, K, QM, GP>, dim3(a.M), dim3(kChainThreads), 0, st, a.layers, a.n_layers,
-                a.steps, static_cast<uint4*>(a.residual), a.cos_tab, a.sin_tab, a.positions, a.scales, a.status, a.C,
-                a.NB, a.Hq, a.Hkv, a.hd, a.G, a.I4, a.NBI, a.max_pos, a.capacity, a.eps, a.act);
+frt_status chain_act_dispatch(frt_act act, const ChainArgs& a, size_t smem, cudaStream_t st) {
+  switch (act) {
+    case FRT_ACT_GELU_TANH: return launch_chain<DT, K, QM, GP, FRT_ACT_GELU_TANH>(a, smem, st);
+    case FRT_ACT_SILU: return launch_chain<DT, K, QM, GP, FRT_ACT_SILU>(a, smem, st);
+    default: return launch_chain<DT, K, QM, GP, FRT_ACT_RELU2>(a, smem, st);
+  }
 }
 
 template <int DT, int K, int QM>
-frt_status chain_gp_dispatch(int GP, const ChainArgs& a, cudaStream_t st) {
+frt_status chain_gp_dispatch(int GP, frt_act act, const ChainArgs& a, size_t smem, cudaStream_t st) {
   switch (GP) {
-    case 1: return launch_chain<DT, K, QM, 1>(a, st);
-    case 2: return launch_chain<DT, K, QM, 2>(a, st);
-    case 4: return launch_chain<DT, K, QM, 4>(a, st);
-    case 8: return launch_chain<DT, K, QM, 8>(a, st);
-    default: return launch_chain<DT, K, QM, 16>(a, st);
+    case 4: return chain_act_dispatch<DT, K, QM, 4>(act, a, smem, st);
+    case 8: return chain_act_dispatch<DT, K, QM, 8>(act, a, smem, st);
+    default: return chain_act_dispatch<DT, K, QM, 16>(act, a, smem, st);
   }
 }
 
 template <int DT>
-frt_status chain_dispatch(int K, frt_quant qm, int GP, const ChainArgs& a, cudaStream_t st) {
+frt_status chain_dispatch(int K, frt_quant qm, int GP, frt_act act, const ChainArgs& a, size_t smem,
+                          cudaStream_t st) {
   const bool blk = qm == FRT_QUANT_BLOCK128;
   switch (K) {
     case 1:
-      return blk ? chain_gp_dispatch<DT, 1, FRT_QUANT_BLOCK128>(GP, a, st)
-                 : chain_gp_dispatch<DT, 1, FRT_QUANT_STATIC>(GP, a, st);
+      return blk ? chain_gp_dispatch<DT, 1, FRT_QUANT_BLOCK128>(GP, act, a, smem, st)
+                 : chain_gp_dispatch<DT, 1, FRT_QUANT_STATIC>(GP, act, a, smem, st);
     case 2:
-      return blk ? chain_gp_dispatch<DT, 2, FRT_QUANT_BLOCK128>(GP, a, st)
-                 : chain_gp_dispatch<DT, 2, FRT_QUANT_STATIC>(GP, a, st);
+      return blk ? chain_gp_dispatch<DT, 2, FRT_QUANT_BLOCK128>(GP, act, a, smem, st)
+                 : chain_gp_dispatch<DT, 2, FRT_QUANT_STATIC>(GP, act, a, smem, st);
     default:
-      return blk ? chain_gp_dispatch<DT, 4, FRT_QUANT_BLOCK128>(GP, a, st)
-                 : chain_gp_dispatch<DT, 4, FRT_QUANT_STATIC>(GP, a, st);
+      return blk ? chain_gp_dispatch<DT, 4, FRT_QUANT_BLOCK128>(GP, act, a, smem, st)
+                 : chain_gp_dispatch<DT, 4, FRT_QUANT_STATIC>(GP, act, a, smem, st);
   }
 }
+
+// Largest dynamic shared memory the chain uses (one CTA per SM).
+constexpr size_t kChainSmemMax = 200 * 1024;
+
 
 }  // namespace
 }  // namespace frt
@@ -364,20 +477,49 @@ extern "C" frt_status frt_chain_persistent(const frt_chain_layer* layers, int n_
     return FRT_ERR_INVALID_ARG;
   if (!valid_dtype(dt) || !valid_quant(qm)) return FRT_ERR_INVALID_ARG;
   if (act != FRT_ACT_GELU_TANH && act != FRT_ACT_SILU && act != FRT_ACT_RELU2) return FRT_ERR_INVALID_ARG;
-  // supported shapes: D <= 4 * 256 * 8, 16-byte head halves (hd % 16 == 0, hd <= 256),
-  // whole 128-output blocks in the activation
-  if (D > 8192 || hd % 16 != 0 || hd > 256 || I % 128 != 0) return FRT_ERR_UNSUPPORTED;
+  // supported shapes: D <= 4 * 256 * 8, 16-byte head halves with 4..16 lanes
+  // per head (hd % 16 == 0, 64 <= hd <= 256), whole 128-output activation blocks
+  if (D > 8192 || hd % 16 != 0 || hd < 64 || hd > 256 || I % 128 != 0) return FRT_ERR_UNSUPPORTED;
   if (M == 0 || n_layers == 0 || steps == 0) return FRT_OK;
   if (!layers || !residual || !cos_tab || !sin_tab || !positions || !scales) return FRT_ERR_INVALID_ARG;
   if (!aligned(layers, 8) || !aligned(residual, 16) || !aligned(cos_tab, 16) || !aligned(sin_tab, 16) ||
       !aligned(positions, 4) || !aligned(scales, 4) || (status && !aligned(status, 4)))
     return FRT_ERR_INVALID_ARG;
+  if ((int64_t)M * 8 > 0x7FFFFFFF) return FRT_ERR_UNSUPPORTED;
   const int C = D / 8;
-  const int K = C <= 256 ? 1 : C <= 512 ? 2 : 4;
+  const int H = Hq + 2 * Hkv;
+  const int NBI = I / 128;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                cudaSuccess) {
+    (void)cudaGetLastError();
+    sms = 148;
+  }
+  // Cluster size: as many CTAs per row as fill the SMs (at most 8): one runs
+  // the norms, the rest share the heads and activation blocks.
+  int S = sms / M;
+  S = S < 1 ? 1 : S > 8 ? 8 : S;
+  const int hd16 = hd / 8;
+  if (C > 4 * kChainThreads) return FRT_ERR_UNSUPPORTED;
+  const int K = C <= kChainThreads ? 1 : C <= 2 * kChainThreads ? 2 : 4;
   const int G = (hd / 2) / 8;
   int GP = 1;
   while (GP < G) GP *= 2;
-  const ChainArgs a{layers, n_layers, steps, residual, cos_tab, sin_tab, positions, scales, status, M, C,
-                    (D + 127) / 128, Hq, Hkv, hd, G, I / 4, I / 128, max_pos, capacity, eps, (int)act};
-  return dt == FRT_F16 ? chain_dispatch<FRT_F16>(K, qm, GP, a, stream) : chain_dispatch<FRT_BF16>(K, qm, GP, a, stream);
+  const size_t table = ((size_t)n_layers * sizeof(frt_chain_layer) + 15) / 16 * 16;
+  for (;; --S) {
+    const int workers = S > 1 ? S - 1 : 1;
+    const int hs = (H + workers - 1) / workers;
+    const int bsl = (NBI + workers - 1) / workers;
+    // the larger of the two roles' stages sizes the shared memory of every CTA
+    const StageMap mn(C, S > 1 ? 0 : hs * hd16, hd16, S > 1 ? 0 : bsl * 32);
+    const StageMap mw(0, hs * hd16, hd16, bsl * 32);
+    const size_t smem = table + (size_t)2 * (mn.len > mw.len ? mn.len : mw.len) * sizeof(uint4);
+    if (smem <= kChainSmemMax || S == 1) {
+      if (smem > kChainSmemMax) return FRT_ERR_UNSUPPORTED;
+      const ChainArgs a{layers, n_layers, steps, residual, cos_tab, sin_tab, positions, scales, status, M, C,
+                        (D + 127) / 128, Hq, Hkv, hd, G, I / 4, NBI, S, max_pos, capacity, eps};
+      return dt == FRT_F16 ? chain_dispatch<FRT_F16>(K, qm, GP, act, a, smem, stream)
+                           : chain_dispatch<FRT_BF16>(K, qm, GP, act, a, smem, stream);
+    }
+  }
 }

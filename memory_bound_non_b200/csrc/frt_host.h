@@ -48,6 +48,33 @@ inline frt_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
   return launch_status();
 }
 
+// As launch(), with the grid grouped into thread-block clusters of
+// `cluster_x` CTAs along x (co-scheduled; they share distributed shared memory).
+template <typename... KArgs, typename... Args>
+inline frt_status launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                 unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FRT_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // Output modes of the quantising kernels beyond the ABI's FP8 modes: NVFP4
 // with row-major or 128x4-swizzled scale factors (internal template values).
 constexpr int kQuantNvfp4Rows = 2;

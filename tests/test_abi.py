@@ -194,7 +194,8 @@ def chain_call(M=4, D=1024, Hq=8, Hkv=1, hd=128, I=4096, layers=A, n=2, steps=3,
 
 
 @pytest.mark.parametrize("kw,want", [
-    (dict(hd=72), UNSUP), (dict(hd=264), UNSUP), (dict(D=8200), UNSUP), (dict(I=4100), UNSUP), (dict(D=12), INV),
+    (dict(hd=72), UNSUP), (dict(hd=264), UNSUP), (dict(hd=32), UNSUP), (dict(D=8200), UNSUP), (dict(I=4100), UNSUP),
+    (dict(D=12), INV),
     (dict(Hq=6, Hkv=4), INV), (dict(act=5), INV), (dict(qm=3), INV), (dict(layers=None), INV),
     (dict(res=A + 8), INV), (dict(M=0), OK), (dict(steps=0), OK), (dict(n=0, layers=None), OK), (dict(M=-1), INV),
 ])
