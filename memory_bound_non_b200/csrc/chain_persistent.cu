@@ -120,7 +120,7 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
     if (QM == FRT_QUANT_BLOCK128) {
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
       am = group_max<16>(am);
-      const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
+      const float sb = block_scale_448(am);
       if (valid && (j & 15) == 0) bs[row * NB + (c >> 4)] = sb;
       if (valid) q[row * C + c] = quant8(y, Divisor(sb));
     } else if (valid) {
@@ -248,7 +248,7 @@ __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* b
       }
       if (QM == FRT_QUANT_BLOCK128) {
         const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
-        const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
+        const float sb = block_scale_448(am);
         if (lane == 0) bs[row * NBI + b] = sb;
         dst[b * 32 + lane] = quant4(a, Divisor(sb));
       } else {

@@ -119,6 +119,19 @@ struct Divisor {
   __device__ __forceinline__ float div_slow(float y) const { return __fdiv_rn(y, s); }
 };
 
+// Block scale RN(amax / 448) of the block-128 FP8 mode (1 for an all-zero
+// block): Markstein's correction with the correctly rounded reciprocal of 448,
+// q = RN(amax RN(1/448)), r = amax - 448 q (exact), RN(q + r RN(1/448)), which
+// is the IEEE quotient for amax >= 2^-100 (tiny blocks take the IEEE division).
+constexpr float kInv448 = 1.0f / 448.0f;
+__device__ __forceinline__ float block_scale_448(float amax) {
+  if (!(amax > 0.0f)) return 1.0f;
+  if (amax < 0x1p-100f) return __fdiv_rn(amax, 448.0f);
+  const float q = amax * kInv448;
+  const float r = fmaf(-q, 448.0f, amax);
+  return fmaf(r, kInv448, q);
+}
+
 // Eight values -> eight e4m3 codes of y / s (low byte first).
 __device__ __forceinline__ uint2 quant8(const float* y, const Divisor& dv);
 // Four values -> four e4m3 codes of y / s.

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
     // code = e4m3(a / s) with the quotient correctly rounded in fp32
     if (QM == FRT_QUANT_BLOCK128) {
       const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
-      const float sb = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
+      const float sb = block_scale_448(am);
       const int64_t gb = gb0 + u;
       if (lane == 0 && gb < total_blocks) block_scales[gb] = sb;  // [M, NB] row-major == flat block index
       if (valid[u]) q[idx[u]] = quant4(a, Divisor(sb));

@@ -68,3 +68,37 @@ def test_products_of_16bit_values_are_exact_in_fp32():
         ok = np.isfinite(p64) & (np.abs(p64) > 2.0 ** -126) & (np.abs(p64) < 3e38)
         np.testing.assert_array_equal(p32[ok].astype(np.float64), p64[ok])
 
+
+
+def _rn32(x):
+    """Round an exact rational to the nearest fp32 (ties to even)."""
+    from fractions import Fraction
+    f = np.float32(float(x))            # within one ulp (the float() step may double-round)
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    best = min(cands, key=lambda c: (abs(Fraction(float(c)) - x), int(np.array(c).view(np.uint32)) & 1))
+    return best
+
+
+def test_markstein_block_scale_is_the_correctly_rounded_quotient():
+    """The block-128 scale RN(amax / 448) formed as q = RN(amax * RN(1/448)),
+    r = amax - 448 q (exact), RN(q + r * RN(1/448)) -- Markstein's correction
+    with the correctly rounded reciprocal -- equals the IEEE fp32 quotient, on
+    random values, values next to quotient rounding midpoints and every binade."""
+    from fractions import Fraction
+    rng = np.random.default_rng(9)
+    inv = np.float32(1.0) / np.float32(448.0)
+    vals = [np.float32(v) for v in rng.uniform(1.0, 2.0, 3000) * 2.0 ** rng.integers(-90, 100, 3000)]
+    # amax just beside 448 * (a quotient rounding midpoint)
+    for k in rng.integers(1 << 23, 1 << 24, 600):
+        mid = Fraction(int(k) * 2 + 1, 2) * Fraction(448) * Fraction(2) ** -23
+        for d in (-1, 0, 1):
+            v = np.float32(float(mid))
+            vals.append(v if d == 0 else np.nextafter(v, np.float32(d * np.inf)))
+    vals += [np.float32(2.0 ** e) for e in range(-99, 127)]
+    for a in vals:
+        q = np.float32(a * inv)
+        r = Fraction(float(a)) - 448 * Fraction(float(q))
+        assert Fraction(float(np.float32(float(r)))) == r          # the residual is an fp32 number
+        got = _rn32(Fraction(float(q)) + r * Fraction(float(inv)))   # one FMA: exact value rounded once
+        want = np.float32(a) / np.float32(448.0)                     # IEEE fp32 division
+        assert got == want, (a, got, want)
