@@ -75,6 +75,8 @@ def parse_args(argv=None):
                    help="time only the widened ops (gated residual + AdaRMSNorm + FP8) and print their JSON")
     p.add_argument("--next-m", type=int, default=65536, help="rows of the large widened-op case")
     p.add_argument("--next-reps", type=int, default=50)
+    p.add_argument("--persistent-chain", default=None, metavar="WORKLOAD",
+                   help="only run the named chain (e.g. pi05) as one persistent kernel, --chain-reps times")
     return p.parse_args(argv)
 
 
@@ -789,6 +791,26 @@ def main(argv=None):
 
     wl = W.get(args.workload)
     peak, peak_kind = measured_peak()
+    if args.persistent_chain:
+        if rank == 0:
+            from memory_bound_non_b200.chain import LayerChain
+            cw = W.get(args.persistent_chain)
+            ch = LayerChain(cw, W.make_inputs(cw))
+            ch.calibrate_static_scales()
+            st = torch.cuda.current_stream()
+            ts = []
+            for _ in range(args.chain_reps):
+                ch.reset()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                ch.run_persistent()
+                e1.record(st)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            print(json.dumps({"persistent_chain": cw.name, "launches": len(ts),
+                              "us_median": round(statistics.median(ts), 2)}), flush=True)
+        dist.close()
+        return 0
     if args.next_only:
         if rank == 0:
             floor = launch_floor()
