@@ -133,10 +133,12 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
 // and their rotation partners per lane), kChainThreads / GP heads per pass.
 template <int DT, int GP>
 __device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t* qw, const uint16_t* kw,
-                                          uint16_t* q_out, uint16_t* k_cache, uint16_t* v_cache, const float* c,
-                                          const float* s, int64_t row, int p, bool row_ok, const Slice& sl, int Hq,
-                                          int Hkv, int hd, int G, float eps) {
+                                          uint16_t* q_out, uint16_t* k_cache, uint16_t* v_cache, const float2* cs,
+                                          const float2* sn, const float2* nsn, int64_t row, int p, bool row_ok,
+                                          const Slice& sl, int Hq, int Hkv, int hd, int G, float eps) {
   constexpr int P = 8;
+  constexpr int NP = P / 2;
+  const float inv_hd = 1.0f / (float)hd;
   const int NG = kChainThreads / GP;
   const int grp = threadIdx.x / GP;
   const int li = threadIdx.x & (GP - 1);
@@ -172,48 +174,29 @@ __device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t*
       *reinterpret_cast<uint4*>(dst + j0) = va;
       *reinterpret_cast<uint4*>(dst + half + j0) = vb;
     }
-    float a[P], b[P];
+    float2 a[NP], b[NP];
     float ss = 0.0f;
     if (on && !is_v) {
-#pragma unroll
-      for (int e = 0; e < P / 2; ++e) {
-        const float2 ta = Pack16<DT>::to_float2(reinterpret_cast<const uint32_t*>(&va)[e]);
-        const float2 tb = Pack16<DT>::to_float2(reinterpret_cast<const uint32_t*>(&vb)[e]);
-        a[2 * e] = ta.x;
-        a[2 * e + 1] = ta.y;
-        b[2 * e] = tb.x;
-        b[2 * e + 1] = tb.y;
-      }
-      if (do_norm) {
-#pragma unroll
-        for (int e = 0; e < P; ++e) ss = fmaf(b[e], b[e], fmaf(a[e], a[e], ss));
-      }
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&va), a);
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&vb), b);
+      if (do_norm) ss = sum_squares_pairs<NP>(a, b);
     }
     ss = group_sum<GP>(ss);  // every lane of the warp takes part
     if (on && !is_v) {
       if (do_norm) {
-        const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
+        const float rstd = head_rstd(ss, inv_hd, eps);
         const uint4 wa = is_q ? qwa : kwa, wb = is_q ? qwb : kwb;
-#pragma unroll
-        for (int e = 0; e < P / 2; ++e) {
-          const float2 fa = Pack16<DT>::to_float2(reinterpret_cast<const uint32_t*>(&wa)[e]);
-          const float2 fb = Pack16<DT>::to_float2(reinterpret_cast<const uint32_t*>(&wb)[e]);
-          a[2 * e] = a[2 * e] * rstd * fa.x;
-          a[2 * e + 1] = a[2 * e + 1] * rstd * fa.y;
-          b[2 * e] = b[2 * e] * rstd * fb.x;
-          b[2 * e + 1] = b[2 * e + 1] * rstd * fb.y;
-        }
+        float2 fa[NP], fb[NP];
+        unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wa), fa);
+        unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wb), fb);
+        scale_pairs<NP>(a, rstd, fa);
+        scale_pairs<NP>(b, rstd, fb);
       }
+      float2 x[NP], y[NP];
+      rope_pairs<NP>(a, b, cs, sn, nsn, x, y);
       uint4 o1, o2;
-#pragma unroll
-      for (int e = 0; e < P / 2; ++e) {
-        const float x0 = fmaf(a[2 * e], c[2 * e], -(b[2 * e] * s[2 * e]));
-        const float x1 = fmaf(a[2 * e + 1], c[2 * e + 1], -(b[2 * e + 1] * s[2 * e + 1]));
-        const float y0 = fmaf(b[2 * e], c[2 * e], a[2 * e] * s[2 * e]);
-        const float y1 = fmaf(b[2 * e + 1], c[2 * e + 1], a[2 * e + 1] * s[2 * e + 1]);
-        reinterpret_cast<uint32_t*>(&o1)[e] = Pack16<DT>::from_float2(x0, x1);
-        reinterpret_cast<uint32_t*>(&o2)[e] = Pack16<DT>::from_float2(y0, y1);
-      }
+      pack_pairs<DT, NP>(x, reinterpret_cast<uint32_t*>(&o1));
+      pack_pairs<DT, NP>(y, reinterpret_cast<uint32_t*>(&o2));
       uint16_t* dst = is_q ? q_out + (row * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + (h - Hq)) * hd;
       *reinterpret_cast<uint4*>(dst + j0) = o1;
       *reinterpret_cast<uint4*>(dst + half + j0) = o2;
@@ -336,16 +319,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
   constexpr int P = 8;
   const int li = t & (GP - 1);
   const int half = hd >> 1;
-  float cs8[P], sn8[P];
-  if (row_ok && li < G) {
-#pragma unroll
-    for (int e = 0; e < P; e += 4) {
-      const float4 tc = __ldg(reinterpret_cast<const float4*>(cos_tab + (int64_t)p * half + li * P + e));
-      const float4 ts = __ldg(reinterpret_cast<const float4*>(sin_tab + (int64_t)p * half + li * P + e));
-      cs8[e] = tc.x, cs8[e + 1] = tc.y, cs8[e + 2] = tc.z, cs8[e + 3] = tc.w;
-      sn8[e] = ts.x, sn8[e + 1] = ts.y, sn8[e + 2] = ts.z, sn8[e + 3] = ts.w;
-    }
-  }
+  float2 cs8[P / 2], sn8[P / 2], nsn8[P / 2];
+  if (row_ok && li < G)
+    load_rope_pairs<P / 2>(cos_tab + (int64_t)p * half + li * P, sin_tab + (int64_t)p * half + li * P, cs8, sn8,
+                           nsn8);
   const Divisor dv_attn(QM == FRT_QUANT_STATIC ? __ldg(scales) : 1.0f);
   const Divisor dv_ffn(QM == FRT_QUANT_STATIC ? __ldg(scales + 1) : 1.0f);
   const Divisor dv_act(QM == FRT_QUANT_STATIC ? __ldg(scales + 2) : 1.0f);
@@ -386,7 +363,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
                       L.q_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.qw) : nullptr,
                       L.k_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.kw) : nullptr,
                       static_cast<uint16_t*>(L.q_out), static_cast<uint16_t*>(L.k_cache),
-                      static_cast<uint16_t*>(L.v_cache), cs8, sn8, row, p, row_ok, sl, Hq, Hkv, hd, G, eps);
+                      static_cast<uint16_t*>(L.v_cache), cs8, sn8, nsn8, row, p, row_ok, sl, Hq, Hkv, hd, G, eps);
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xf, L.w_ffn != nullptr ? st + m.wf : nullptr, reinterpret_cast<uint2*>(L.q8_ffn),
                             L.bs_ffn, dv_ffn, hv, row, sl, C, NB, D, eps, red);

@@ -109,6 +109,10 @@ struct Divisor {
     inv = __frcp_rn(s_);
     fast = s_ >= 0x1p-100f && s_ <= 0x1p+100f;
   }
+  // from a reciprocal formed once elsewhere (inv_ must be RN(1/s_))
+  __device__ __forceinline__ Divisor(float s_, float inv_) : s(s_), inv(inv_) {
+    fast = s_ >= 0x1p-100f && s_ <= 0x1p+100f;
+  }
   __device__ __forceinline__ float div(float y) const {
     const float q = y * inv;
     const float r = fmaf(-q, s, y);
@@ -318,6 +322,96 @@ __device__ __forceinline__ float group_max(float v) {
 
 __device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
+}
+
+// ------------------------------------------------- q/k head arithmetic --
+// One lane's share of a head: NP packed fp32 pairs of the first half (a,
+// elements j0 .. j0 + 2NP - 1) and of the second half (b, the rotate-half
+// partners j0 + hd/2 ...).  Blackwell issues two fp32 multiplies or FMAs per
+// instruction (mul/fma .f32x2); each half of a pair is rounded to nearest
+// exactly as the scalar operation, so only the order of the sum of squares
+// (two interleaved partial sums) depends on the packing.
+template <int DT, int NP>
+__device__ __forceinline__ void unpack_pairs(const uint32_t* w, float2* f) {
+#pragma unroll
+  for (int e = 0; e < NP; ++e) f[e] = Pack16<DT>::to_float2(w[e]);
+}
+
+template <int DT, int NP>
+__device__ __forceinline__ void pack_pairs(const float2* f, uint32_t* w) {
+#pragma unroll
+  for (int e = 0; e < NP; ++e) w[e] = Pack16<DT>::from_float2(f[e].x, f[e].y);
+}
+
+template <int NP>
+__device__ __forceinline__ float sum_squares_pairs(const float2* a, const float2* b) {
+  float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int e = 0; e < NP; ++e) {
+    acc = __ffma2_rn(a[e], a[e], acc);
+    acc = __ffma2_rn(b[e], b[e], acc);
+  }
+  return acc.x + acc.y;
+}
+
+// RMSNorm scale of a head, 1 / sqrt(ss * inv_n + eps) with inv_n = RN(1/n)
+// (exact for power-of-two n): the hardware reciprocal square root, relative
+// error about 2^-22, far below the half-ulp of the 16-bit outputs.
+__device__ __forceinline__ float head_rstd(float ss, float inv_n, float eps) {
+  return rsqrtf(fmaf(ss, inv_n, eps));
+}
+
+// x <- (x * r) * w per element (the product with r rounded first).
+template <int NP>
+__device__ __forceinline__ void scale_pairs(float2* x, float r, const float2* w) {
+  const float2 rr = make_float2(r, r);
+#pragma unroll
+  for (int e = 0; e < NP; ++e) x[e] = __fmul2_rn(__fmul2_rn(x[e], rr), w[e]);
+}
+
+// x <- (x * r) * w per element, w given as packed 16-bit pairs.
+template <int DT, int NP>
+__device__ __forceinline__ void scale_pairs_w16(float2* x, float r, const uint32_t* w) {
+  const float2 rr = make_float2(r, r);
+#pragma unroll
+  for (int e = 0; e < NP; ++e) x[e] = __fmul2_rn(__fmul2_rn(x[e], rr), Pack16<DT>::to_float2(w[e]));
+}
+
+// Rotate-half RoPE: o1 = a cos - b sin, o2 = b cos + a sin, each one FMA on
+// the rounded sine product; nsn holds -sin so that no operand needs negating.
+template <int NP>
+__device__ __forceinline__ void rope_pairs(const float2* a, const float2* b, const float2* cs, const float2* sn,
+                                           const float2* nsn, float2* o1, float2* o2) {
+#pragma unroll
+  for (int e = 0; e < NP; ++e) {
+    o1[e] = __ffma2_rn(a[e], cs[e], __fmul2_rn(b[e], nsn[e]));
+    o2[e] = __ffma2_rn(b[e], cs[e], __fmul2_rn(a[e], sn[e]));
+  }
+}
+
+template <int NP>
+__device__ __forceinline__ void mul_pairs(float2* x, float r) {
+  const float2 rr = make_float2(r, r);
+#pragma unroll
+  for (int e = 0; e < NP; ++e) x[e] = __fmul2_rn(x[e], rr);
+}
+
+// A lane's cos/sin slice (2 NP fp32 each, 16-byte aligned) as packed pairs,
+// with the negated sine.
+template <int NP>
+__device__ __forceinline__ void load_rope_pairs(const float* c, const float* s, float2* cs, float2* sn,
+                                                float2* nsn) {
+#pragma unroll
+  for (int e = 0; e < NP; e += 2) {
+    const float4 tc = *reinterpret_cast<const float4*>(c + 2 * e);
+    const float4 ts = *reinterpret_cast<const float4*>(s + 2 * e);
+    cs[e] = make_float2(tc.x, tc.y);
+    cs[e + 1] = make_float2(tc.z, tc.w);
+    sn[e] = make_float2(ts.x, ts.y);
+    sn[e + 1] = make_float2(ts.z, ts.w);
+    nsn[e] = make_float2(-ts.x, -ts.y);
+    nsn[e + 1] = make_float2(-ts.z, -ts.w);
+  }
 }
 
 }  // namespace frt

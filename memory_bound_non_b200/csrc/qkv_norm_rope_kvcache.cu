@@ -52,23 +52,19 @@ __device__ __forceinline__ void unpack(const typename Vec16<P>::T& v, float* f) 
 }
 
 template <int DT, int P>
-__device__ __forceinline__ void store_packed(uint16_t* dst, const float* f) {
+__device__ __forceinline__ void store_pairs(uint16_t* dst, const float2* f) {
   typename Vec16<P>::T v;
-  uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-  for (int e = 0; e < P / 2; ++e) w[e] = Pack16<DT>::from_float2(f[2 * e], f[2 * e + 1]);
+  pack_pairs<DT, P / 2>(f, reinterpret_cast<uint32_t*>(&v));
   *reinterpret_cast<typename Vec16<P>::T*>(dst) = v;
 }
 
-template <int P>
-__device__ __forceinline__ void ld_f32(const float* p, float* f) {
+template <int NP>
+__device__ __forceinline__ void ld_pairs_smem(const float* p, float2* f) {
 #pragma unroll
-  for (int e = 0; e < P; e += 4) {
-    const float4 t = __ldg(reinterpret_cast<const float4*>(p + e));
-    f[e] = t.x;
-    f[e + 1] = t.y;
-    f[e + 2] = t.z;
-    f[e + 3] = t.w;
+  for (int e = 0; e < NP; e += 2) {
+    const float4 t = *reinterpret_cast<const float4*>(p + 2 * e);
+    f[e] = make_float2(t.x, t.y);
+    f[e + 1] = make_float2(t.z, t.w);
   }
 }
 
@@ -97,6 +93,46 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const float* v, const 
     *reinterpret_cast<uint2*>(dst) = quant8(v, dv);
   else
     *reinterpret_cast<uint32_t*>(dst) = quant4(v, dv);
+}
+
+// One head's LayerNorm on a lane's packed pairs (NEXT-4): the mean, then the
+// centred sum of squares (each an xor shuffle over the GP lanes of the group;
+// every lane of the warp takes part), then x = (x - mean) * rstd * w + bias in
+// place, the head's affine rows given as packed 16-bit words (null:
+// identity).  `on` gates the lane's arithmetic, not the shuffles.
+template <int DT, int NP, int GP>
+__device__ __forceinline__ void ln_head(float2* a, float2* b, bool on, float inv_hd, float eps,
+                                        const uint32_t* wa, const uint32_t* wb, const uint32_t* ba,
+                                        const uint32_t* bb) {
+  float2 acc = make_float2(0.0f, 0.0f);
+  if (on) {
+#pragma unroll
+    for (int e = 0; e < NP; ++e) acc = __fadd2_rn(__fadd2_rn(acc, a[e]), b[e]);
+  }
+  const float mean = group_sum<GP>(acc.x + acc.y) * inv_hd;
+  float2 acc2 = make_float2(0.0f, 0.0f);
+  if (on) {
+    const float2 nm = make_float2(-mean, -mean);
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+      a[e] = __fadd2_rn(a[e], nm);
+      b[e] = __fadd2_rn(b[e], nm);
+      acc2 = __ffma2_rn(b[e], b[e], __ffma2_rn(a[e], a[e], acc2));
+    }
+  }
+  const float s2 = group_sum<GP>(acc2.x + acc2.y);
+  if (!on) return;
+  const float r = head_rstd(s2, inv_hd, eps);
+  const float2 rr = make_float2(r, r);
+#pragma unroll
+  for (int e = 0; e < NP; ++e) {
+    const float2 w1 = wa ? Pack16<DT>::to_float2(wa[e]) : make_float2(1.0f, 1.0f);
+    const float2 w2 = wb ? Pack16<DT>::to_float2(wb[e]) : make_float2(1.0f, 1.0f);
+    const float2 b1 = ba ? Pack16<DT>::to_float2(ba[e]) : make_float2(0.0f, 0.0f);
+    const float2 b2 = bb ? Pack16<DT>::to_float2(bb[e]) : make_float2(0.0f, 0.0f);
+    a[e] = __ffma2_rn(__fmul2_rn(a[e], rr), w1, b1);
+    b[e] = __ffma2_rn(__fmul2_rn(b[e], rr), w2, b2);
+  }
 }
 
 // Register kernel (small batches, or pointers below 16-byte alignment).  One
@@ -156,11 +192,10 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
   if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
   const bool active = lane_ok && row_ok;
-  float c[P], s[P];
-  if (active) {
-    ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
-    ld_f32<P>(sin_tab + (int64_t)p * half + j0, s);
-  }
+  constexpr int NP = P / 2;
+  float2 cs[NP], sn[NP], nsn[NP];
+  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
+  const float inv_hd = 1.0f / (float)hd;
   const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
   const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
 #pragma unroll
@@ -188,62 +223,51 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
         *reinterpret_cast<V*>(dst + half + j0) = vb[i];
       }
     }
-    float a[P], b[P];
+    float2 a[NP], b[NP];
     float ss = 0.0f;
     if (on && !is_v) {
-      unpack<DT, P>(va[i], a);
-      unpack<DT, P>(vb[i], b);
-      if (do_norm) {
-#pragma unroll
-        for (int e = 0; e < P; ++e) ss = fmaf(b[e], b[e], fmaf(a[e], a[e], ss));
-      }
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&va[i]), a);
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&vb[i]), b);
+      if (do_norm) ss = sum_squares_pairs<NP>(a, b);
     }
     ss = group_sum<GP>(ss);  // every lane of the warp takes part
     if (on && !is_v) {
       if (do_norm) {
-        const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
-        float fa[P], fb[P];
+        const float rstd = head_rstd(ss, inv_hd, eps);
+        float2 fa[NP], fb[NP];
         if (HPG == 1) {  // weights already in registers
-          unpack<DT, P>(is_q ? qwa : kwa, fa);
-          unpack<DT, P>(is_q ? qwb : kwb, fb);
+          const V wa = is_q ? qwa : kwa, wb = is_q ? qwb : kwb;
+          unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wa), fa);
+          unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wb), fb);
         } else {
-          unpack<DT, P>(ld_vec<P>(nw + j0), fa);
-          unpack<DT, P>(ld_vec<P>(nw + half + j0), fb);
+          const V wa = ld_vec<P>(nw + j0), wb = ld_vec<P>(nw + half + j0);
+          unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wa), fa);
+          unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wb), fb);
         }
-#pragma unroll
-        for (int e = 0; e < P; ++e) {
-          a[e] = a[e] * rstd * fa[e];
-          b[e] = b[e] * rstd * fb[e];
-        }
+        scale_pairs<NP>(a, rstd, fa);
+        scale_pairs<NP>(b, rstd, fb);
       }
-      float o1[P], o2[P];
-#pragma unroll
-      for (int e = 0; e < P; ++e) {
-        o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
-        o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
-      }
+      float2 o1[NP], o2[NP];
+      rope_pairs<NP>(a, b, cs, sn, nsn, o1, o2);
       if (is_q) {
         if (QEPI) {
-#pragma unroll
-          for (int e = 0; e < P; ++e) {
-            o1[e] *= ep.q_scale;
-            o2[e] *= ep.q_scale;
-          }
+          mul_pairs<NP>(o1, ep.q_scale);
+          mul_pairs<NP>(o2, ep.q_scale);
         }
         uint16_t* dst = q_out + (QEPI ? q_row(ep, tok, h, Hq) : (int64_t)tok * Hq + h) * hd;
-        store_packed<DT, P>(dst + j0, o1);
-        store_packed<DT, P>(dst + half + j0, o2);
+        store_pairs<DT, P>(dst + j0, o1);
+        store_pairs<DT, P>(dst + half + j0, o2);
       } else {
         const int64_t off = ((int64_t)p * Hkv + (h - Hq)) * hd;
         if (KV8) {
           uint8_t* dst = static_cast<uint8_t*>(k_cache) + off;
           const Divisor dk(k_scale);
-          store_codes<P>(dst + j0, o1, dk);
-          store_codes<P>(dst + half + j0, o2, dk);
+          store_codes<P>(dst + j0, reinterpret_cast<const float*>(o1), dk);
+          store_codes<P>(dst + half + j0, reinterpret_cast<const float*>(o2), dk);
         } else {
           uint16_t* dst = static_cast<uint16_t*>(k_cache) + off;
-          store_packed<DT, P>(dst + j0, o1);
-          store_packed<DT, P>(dst + half + j0, o2);
+          store_pairs<DT, P>(dst + j0, o1);
+          store_pairs<DT, P>(dst + half + j0, o2);
         }
       }
     }
@@ -256,7 +280,7 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
 // EPI 2).  The caller orders these writes before its bulk stores.
 template <int DT, int P, int GP, int EPI>
 __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbuf, const float* sbuf,
-                                              const uint16_t* qwbuf, const uint16_t* kwbuf, uint8_t* k8buf,
+                                              const float* nsbuf, const float* kvs, const uint16_t* qwbuf, const uint16_t* kwbuf, uint8_t* k8buf,
                                               uint8_t* v8buf, const uint16_t* q_norm_w, const uint16_t* k_norm_w,
                                               uint16_t* q_out, int tok, int tid, int H, int NG, int Hq, int Hkv,
                                               int hd, int G, float eps, const Epilogue& ep) {
@@ -269,16 +293,8 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
   const int li = tid & (GP - 1);
   const bool lane_ok = grp < NG && li < G;
   const int j0 = li * P;
-  float c[P], s[P];
-  if (lane_ok) {
-#pragma unroll
-    for (int e = 0; e < P; ++e) {
-      c[e] = cbuf[j0 + e];
-      s[e] = sbuf[j0 + e];
-    }
-  }
-  const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
-  const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
+  constexpr int NP = P / 2;
+  const float inv_hd = 1.0f / (float)hd;
   const bool q_direct = QEPI && ep.q_head_major;  // head-major Q leaves from registers
   // Q and K heads; V heads too with KV8 (their codes), else V leaves untouched.
   const int nheads = KV8 ? H : Hq + Hkv;
@@ -291,125 +307,93 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
     const uint16_t* nwg = is_v ? nullptr : is_q ? q_norm_w : k_norm_w;
     const uint16_t* nws = is_q ? qwbuf : kwbuf;
     uint16_t* vec = rowbuf + h * hd;
-    float a[P], b[P];
     if (LN) {
-      // per-head LayerNorm: mean, then the centred sum of squares, then the
-      // head's affine rows (global memory, each optional) and RoPE in place
-      float s1 = 0.0f;
+      // per-head LayerNorm with the head's affine rows (global memory, each
+      // optional), then RoPE in place
+      float2 x1[NP], x2[NP];
       if (on) {
-        unpack<DT, P>(*reinterpret_cast<const V*>(vec + j0), a);
-        unpack<DT, P>(*reinterpret_cast<const V*>(vec + half + j0), b);
-#pragma unroll
-        for (int e = 0; e < P; ++e) s1 += a[e] + b[e];
+        const V va = *reinterpret_cast<const V*>(vec + j0), vb = *reinterpret_cast<const V*>(vec + half + j0);
+        unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&va), x1);
+        unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&vb), x2);
       }
-      const float mean = group_sum<GP>(s1) / (float)hd;
-      float s2 = 0.0f;
-      if (on) {
-#pragma unroll
-        for (int e = 0; e < P; ++e) {
-          a[e] -= mean;
-          b[e] -= mean;
-          s2 = fmaf(a[e], a[e], fmaf(b[e], b[e], s2));
-        }
+      const int64_t off = (int64_t)(is_q ? h : h - Hq) * hd;
+      const uint16_t* pw = is_q ? q_norm_w : k_norm_w;
+      const uint16_t* pb = is_q ? ep.q_bias : ep.k_bias;
+      V wa, wb, ba, bb;
+      if (on && pw != nullptr) {
+        wa = ld_vec<P>(pw + off + j0);
+        wb = ld_vec<P>(pw + off + half + j0);
       }
-      s2 = group_sum<GP>(s2);
+      if (on && pb != nullptr) {
+        ba = ld_vec<P>(pb + off + j0);
+        bb = ld_vec<P>(pb + off + half + j0);
+      }
+      ln_head<DT, NP, GP>(x1, x2, on, inv_hd, eps, pw ? reinterpret_cast<const uint32_t*>(&wa) : nullptr,
+                          pw ? reinterpret_cast<const uint32_t*>(&wb) : nullptr,
+                          pb ? reinterpret_cast<const uint32_t*>(&ba) : nullptr,
+                          pb ? reinterpret_cast<const uint32_t*>(&bb) : nullptr);
       if (on) {
-        const float rstd = 1.0f / sqrtf(s2 / (float)hd + eps);
-        const int64_t off = (int64_t)(is_q ? h : h - Hq) * hd;
-        const uint16_t* pw = is_q ? q_norm_w : k_norm_w;
-        const uint16_t* pb = is_q ? ep.q_bias : ep.k_bias;
-        // affine rows kept packed (16-bit pairs), unpacked pair by pair
-        uint32_t wa[P / 2], wb[P / 2], ba[P / 2], bb[P / 2];
+        float2 o1[NP], o2[NP];
 #pragma unroll
-        for (int e = 0; e < P / 2; ++e) {
-          wa[e] = wb[e] = Pack16<DT>::kOnes;
-          ba[e] = bb[e] = 0u;
+        for (int e = 0; e < NP; e += 2) {
+          float2 cs[2], sn[2], nsn[2];
+          ld_pairs_smem<2>(cbuf + j0 + 2 * e, cs);
+          ld_pairs_smem<2>(sbuf + j0 + 2 * e, sn);
+          ld_pairs_smem<2>(nsbuf + j0 + 2 * e, nsn);
+          rope_pairs<2>(x1 + e, x2 + e, cs, sn, nsn, o1 + e, o2 + e);
         }
-        if (pw != nullptr) {
-          const V t1 = ld_vec<P>(pw + off + j0), t2 = ld_vec<P>(pw + off + half + j0);
-#pragma unroll
-          for (int e = 0; e < P / 2; ++e) {
-            wa[e] = reinterpret_cast<const uint32_t*>(&t1)[e];
-            wb[e] = reinterpret_cast<const uint32_t*>(&t2)[e];
-          }
-        }
-        if (pb != nullptr) {
-          const V t1 = ld_vec<P>(pb + off + j0), t2 = ld_vec<P>(pb + off + half + j0);
-#pragma unroll
-          for (int e = 0; e < P / 2; ++e) {
-            ba[e] = reinterpret_cast<const uint32_t*>(&t1)[e];
-            bb[e] = reinterpret_cast<const uint32_t*>(&t2)[e];
-          }
-        }
-        float o1[P], o2[P];
-#pragma unroll
-        for (int e = 0; e < P; e += 2) {
-          const float2 w1 = Pack16<DT>::to_float2(wa[e / 2]), w2 = Pack16<DT>::to_float2(wb[e / 2]);
-          const float2 b1 = Pack16<DT>::to_float2(ba[e / 2]), b2 = Pack16<DT>::to_float2(bb[e / 2]);
-          const float x1a = fmaf(a[e] * rstd, w1.x, b1.x), x1b = fmaf(a[e + 1] * rstd, w1.y, b1.y);
-          const float x2a = fmaf(b[e] * rstd, w2.x, b2.x), x2b = fmaf(b[e + 1] * rstd, w2.y, b2.y);
-          o1[e] = fmaf(x1a, c[e], -(x2a * s[e]));
-          o2[e] = fmaf(x2a, c[e], x1a * s[e]);
-          o1[e + 1] = fmaf(x1b, c[e + 1], -(x2b * s[e + 1]));
-          o2[e + 1] = fmaf(x2b, c[e + 1], x1b * s[e + 1]);
-        }
-        store_packed<DT, P>(vec + j0, o1);
-        store_packed<DT, P>(vec + half + j0, o2);
+        store_pairs<DT, P>(vec + j0, o1);
+        store_pairs<DT, P>(vec + half + j0, o2);
       }
       continue;
     }
+    float2 x1[NP], x2[NP];
     float ss = 0.0f;
     if (on) {
-      unpack<DT, P>(*reinterpret_cast<const V*>(vec + j0), a);
-      unpack<DT, P>(*reinterpret_cast<const V*>(vec + half + j0), b);
-      if (nwg != nullptr) {
-#pragma unroll
-        for (int e = 0; e < P; ++e) ss = fmaf(b[e], b[e], fmaf(a[e], a[e], ss));
-      }
+      const V va = *reinterpret_cast<const V*>(vec + j0), vb = *reinterpret_cast<const V*>(vec + half + j0);
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&va), x1);
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&vb), x2);
+      if (nwg != nullptr) ss = sum_squares_pairs<NP>(x1, x2);
     }
     ss = group_sum<GP>(ss);  // every lane of the warp takes part
     if (on && KV8 && is_v) {
       uint8_t* dst = v8buf + (h - Hq - Hkv) * hd;
-      const Divisor dvs(v_scale);
-      store_codes<P>(dst + j0, a, dvs);
-      store_codes<P>(dst + half + j0, b, dvs);
+      const Divisor dvs(kvs[2], kvs[3]);
+      store_codes<P>(dst + j0, reinterpret_cast<const float*>(x1), dvs);
+      store_codes<P>(dst + half + j0, reinterpret_cast<const float*>(x2), dvs);
     } else if (on) {
       if (nwg != nullptr) {
-        const float rstd = 1.0f / sqrtf(ss / (float)hd + eps);
-        float fa[P], fb[P];
-        unpack<DT, P>(*reinterpret_cast<const V*>(nws + j0), fa);
-        unpack<DT, P>(*reinterpret_cast<const V*>(nws + half + j0), fb);
-#pragma unroll
-        for (int e = 0; e < P; ++e) {
-          a[e] = a[e] * rstd * fa[e];
-          b[e] = b[e] * rstd * fb[e];
-        }
+        const float rstd = head_rstd(ss, inv_hd, eps);
+        const V wa = *reinterpret_cast<const V*>(nws + j0), wb = *reinterpret_cast<const V*>(nws + half + j0);
+        float2 fa[NP], fb[NP];
+        unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wa), fa);
+        unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wb), fb);
+        scale_pairs<NP>(x1, rstd, fa);
+        scale_pairs<NP>(x2, rstd, fb);
       }
-      float o1[P], o2[P];
-#pragma unroll
-      for (int e = 0; e < P; ++e) {
-        o1[e] = fmaf(a[e], c[e], -(b[e] * s[e]));
-        o2[e] = fmaf(b[e], c[e], a[e] * s[e]);
-      }
+      // this slot's cos, sin and -sin slices from shared memory
+      float2 cs[NP], sn[NP], nsn[NP];
+      ld_pairs_smem<NP>(cbuf + j0, cs);
+      ld_pairs_smem<NP>(sbuf + j0, sn);
+      ld_pairs_smem<NP>(nsbuf + j0, nsn);
+      float2 o1[NP], o2[NP];
+      rope_pairs<NP>(x1, x2, cs, sn, nsn, o1, o2);
       if (QEPI && is_q) {
-#pragma unroll
-        for (int e = 0; e < P; ++e) {
-          o1[e] *= ep.q_scale;
-          o2[e] *= ep.q_scale;
-        }
+        mul_pairs<NP>(o1, ep.q_scale);
+        mul_pairs<NP>(o2, ep.q_scale);
       }
       if (KV8 && !is_q) {
         uint8_t* dst = k8buf + (h - Hq) * hd;
-        const Divisor dk(k_scale);
-        store_codes<P>(dst + j0, o1, dk);
-        store_codes<P>(dst + half + j0, o2, dk);
+        const Divisor dk(kvs[0], kvs[1]);
+        store_codes<P>(dst + j0, reinterpret_cast<const float*>(o1), dk);
+        store_codes<P>(dst + half + j0, reinterpret_cast<const float*>(o2), dk);
       } else if (q_direct && is_q) {
         uint16_t* dst = q_out + ((int64_t)h * ep.M + tok) * hd;
-        store_packed<DT, P>(dst + j0, o1);
-        store_packed<DT, P>(dst + half + j0, o2);
+        store_pairs<DT, P>(dst + j0, o1);
+        store_pairs<DT, P>(dst + half + j0, o2);
       } else {
-        store_packed<DT, P>(vec + j0, o1);
-        store_packed<DT, P>(vec + half + j0, o2);
+        store_pairs<DT, P>(vec + j0, o1);
+        store_pairs<DT, P>(vec + half + j0, o2);
       }
     }
   }
@@ -473,11 +457,10 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
   if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
   const bool active = lane_ok && row_ok;
-  float c[P], sn[P];
-  if (active) {
-    ld_f32<P>(cos_tab + (int64_t)p * half + j0, c);
-    ld_f32<P>(sin_tab + (int64_t)p * half + j0, sn);
-  }
+  constexpr int NP = P / 2;
+  float2 cs[NP], sn[NP], nsn[NP];
+  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
+  const float inv_hd = 1.0f / (float)hd;
 #pragma unroll
   for (int i = 0; i < HPG; ++i) {
     const int h = (hb * HPG + i) * NG + grp;
@@ -490,55 +473,33 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
       *reinterpret_cast<V*>(dst + half + j0) = vb[i];
     }
     const bool qk = on && !is_v;
-    float a[P], b[P];
-    float s1 = 0.0f;
+    float2 a[NP], b[NP];
     if (qk) {
-      unpack<DT, P>(va[i], a);
-      unpack<DT, P>(vb[i], b);
-#pragma unroll
-      for (int e = 0; e < P; ++e) s1 += a[e] + b[e];
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&va[i]), a);
+      unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&vb[i]), b);
     }
-    const float mean = group_sum<GP>(s1) / (float)hd;  // every lane of the warp takes part
-    float s2 = 0.0f;
-    if (qk) {
-#pragma unroll
-      for (int e = 0; e < P; ++e) {
-        a[e] -= mean;
-        b[e] -= mean;
-        s2 = fmaf(a[e], a[e], fmaf(b[e], b[e], s2));
-      }
+    const int hh = is_q ? h : h - Hq;
+    const uint16_t* pw = is_q ? q_w : k_w;
+    const uint16_t* pb = is_q ? q_b : k_b;
+    V wa, wb, ba, bb;
+    if (qk && pw != nullptr) {
+      wa = ld_vec<P>(pw + (int64_t)hh * hd + j0);
+      wb = ld_vec<P>(pw + (int64_t)hh * hd + half + j0);
     }
-    s2 = group_sum<GP>(s2);
+    if (qk && pb != nullptr) {
+      ba = ld_vec<P>(pb + (int64_t)hh * hd + j0);
+      bb = ld_vec<P>(pb + (int64_t)hh * hd + half + j0);
+    }
+    ln_head<DT, NP, GP>(a, b, qk, inv_hd, eps, pw ? reinterpret_cast<const uint32_t*>(&wa) : nullptr,
+                        pw ? reinterpret_cast<const uint32_t*>(&wb) : nullptr,
+                        pb ? reinterpret_cast<const uint32_t*>(&ba) : nullptr,
+                        pb ? reinterpret_cast<const uint32_t*>(&bb) : nullptr);
     if (qk) {
-      const float rstd = 1.0f / sqrtf(s2 / (float)hd + eps);
-      const int hh = is_q ? h : h - Hq;
-      const uint16_t* pw = is_q ? q_w : k_w;
-      const uint16_t* pb = is_q ? q_b : k_b;
-      float fw[2 * P], fb[2 * P];
-#pragma unroll
-      for (int e = 0; e < 2 * P; ++e) {
-        fw[e] = 1.0f;
-        fb[e] = 0.0f;
-      }
-      if (pw != nullptr) {
-        unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + j0), fw);
-        unpack<DT, P>(ld_vec<P>(pw + (int64_t)hh * hd + half + j0), fw + P);
-      }
-      if (pb != nullptr) {
-        unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + j0), fb);
-        unpack<DT, P>(ld_vec<P>(pb + (int64_t)hh * hd + half + j0), fb + P);
-      }
-      float o1[P], o2[P];
-#pragma unroll
-      for (int e = 0; e < P; ++e) {
-        const float x1 = fmaf(a[e] * rstd, fw[e], fb[e]);
-        const float x2 = fmaf(b[e] * rstd, fw[P + e], fb[P + e]);
-        o1[e] = fmaf(x1, c[e], -(x2 * sn[e]));
-        o2[e] = fmaf(x2, c[e], x1 * sn[e]);
-      }
+      float2 o1[NP], o2[NP];
+      rope_pairs<NP>(a, b, cs, sn, nsn, o1, o2);
       uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + hh) * hd;
-      store_packed<DT, P>(dst + j0, o1);
-      store_packed<DT, P>(dst + half + j0, o2);
+      store_pairs<DT, P>(dst + j0, o1);
+      store_pairs<DT, P>(dst + half + j0, o2);
     }
   }
 }
@@ -558,13 +519,15 @@ constexpr int kMaxPolls = 1 << 22;
 // EPI: 0 = op (b) as is (Q token-major, unscaled; 16-bit caches), 1 = Q
 // epilogue (scale, layout), 2 = Q epilogue + e4m3 caches, 3 = per-head
 // LayerNorm in place of the RMSNorm (affine rows read from global memory,
-// nothing staged for them).  At most 128
-// threads; the register budget keeps 10 CTAs (tokens) resident per SM (8 for
-// the 16-bit Q epilogue, which would spill at 10): the kernel waits on memory,
-// so resident tokens, not instruction count, set its rate.
+// nothing staged for them).  At most 128 threads (launched with 96, or 64 at
+// the LayerNorm level); the register budget (48 registers at level 0, 55-56
+// at levels 1 and 2, 64 at level 3) keeps 12-16 CTAs (tokens) resident per SM:
+// the kernel waits on memory, so resident tokens set its rate.  The head
+// arithmetic runs on packed fp32 pairs, and the rotation reads cos, sin and
+// -sin from shared memory slot by slot rather than holding them.
 template <int EPI>
 constexpr int tma_min_blocks() {
-  return EPI == 1 || EPI == 3 ? 8 : 10;
+  return EPI == 1 || EPI == 3 ? 8 : EPI == 2 ? 9 : 10;
 }
 
 template <int DT, int P, int GP, int EPI>
@@ -575,10 +538,11 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
     void* __restrict__ v_cache, int32_t* status, int H, int NG, int Hq, int Hkv, int hd, int G, int max_pos,
     int capacity, float eps, Epilogue ep) {
   pdl_enter();
-  // [QKV row][cos][sin][q weight][k weight] (+ [K codes][V codes] with EPI 2)
+  // [QKV row][cos][sin][q weight][k weight][-sin] (+ [K codes][V codes] with EPI 2)
   extern __shared__ __align__(128) uint8_t dsmem[];
   __shared__ uint64_t bar;
   __shared__ int s_pos;
+  __shared__ float s_kv[4];  // e4m3 cache scales and their rounded reciprocals (EPI 2)
   const int tok = blockIdx.x;
   const int tid = threadIdx.x;
   const int half = hd >> 1;
@@ -590,7 +554,8 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
   float* sbuf = cbuf + half;
   uint16_t* qwbuf = reinterpret_cast<uint16_t*>(sbuf + half);
   uint16_t* kwbuf = qwbuf + hd;
-  uint8_t* k8buf = reinterpret_cast<uint8_t*>(kwbuf + hd);
+  float* nsbuf = reinterpret_cast<float*>(kwbuf + hd);
+  uint8_t* k8buf = reinterpret_cast<uint8_t*>(nsbuf + half);
   uint8_t* v8buf = k8buf + Hkv * hd;
 
   if (tid == 0) {
@@ -609,6 +574,13 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
     const int p = __ldg(positions + tok);
     const bool ok = p >= 0 && p < max_pos && p < capacity;
     s_pos = ok ? p : -1;
+    if (EPI == 2) {
+      const float ks = __ldg(ep.kv_scales), vs = __ldg(ep.kv_scales + 1);
+      s_kv[0] = ks;
+      s_kv[1] = __frcp_rn(ks);
+      s_kv[2] = vs;
+      s_kv[3] = __frcp_rn(vs);
+    }
     if (ok) {
       mbar_arrive_expect_tx(&bar, 2 * tab_bytes);
       bulk_load(cbuf, cos_tab + (int64_t)p * half, tab_bytes, &bar);
@@ -626,7 +598,10 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
   }
   const int p = s_pos;
   if (p < 0) return;  // position out of range: nothing is written
-  process_token<DT, P, GP, EPI>(rowbuf, cbuf, sbuf, qwbuf, kwbuf, k8buf, v8buf, q_norm_w, k_norm_w, q_out, tok, tid,
+  // -sin beside sin, so the rotation needs no negated operand
+  for (int j = tid; j < half; j += blockDim.x) nsbuf[j] = -sbuf[j];
+  __syncthreads();
+  process_token<DT, P, GP, EPI>(rowbuf, cbuf, sbuf, nsbuf, s_kv, qwbuf, kwbuf, k8buf, v8buf, q_norm_w, k_norm_w, q_out, tok, tid,
                                 H, NG, Hq, Hkv, hd, G, eps, ep);
   fence_proxy_async_smem();  // this thread's writes -> the bulk stores below
   __syncthreads();
@@ -680,11 +655,22 @@ inline Shape qkv_shape(int M, int H, int GP, bool kv8) {
 }
 
 // Shared memory of the bulk-copy kernel: the QKV row, cos and sin rows, two
-// norm weights, and with an e4m3 cache the K and V code rows.
+// norm weights, the negated sin row, and with an e4m3 cache the K and V code
+// rows.
 inline size_t tma_smem(int H, int Hkv, int hd, bool kv8) {
-  return (size_t)H * hd * 2 + (size_t)hd * 4 + (size_t)hd * 4 + (kv8 ? (size_t)2 * Hkv * hd : 0);
+  return (size_t)H * hd * 2 + (size_t)hd * 2 * 2 + (size_t)hd * 2 * 2 + (size_t)hd * 2 +
+         (kv8 ? (size_t)2 * Hkv * hd : 0);
 }
 constexpr size_t kTmaSmemMax = 200 * 1024;
+
+// Threads of the bulk-copy kernel: a token's heads are taken a few slots at a
+// time by fewer lane groups, so more tokens (CTAs) fit on an SM and more
+// bytes are in flight; the kernel's rate follows resident tokens.  Measured
+// at 65536 tokens of 32/8 heads of 128: 96 threads run op (b) 5 % faster
+// than 128 (14 resident tokens instead of 10), and 64 threads suit the
+// LayerNorm level (64 registers a thread).
+constexpr int kTmaThreads = 96;
+constexpr int kTmaThreadsLn = 64;
 
 template <int DT, int P, int GP, int EPI>
 frt_status launch_gp(const Args& a, bool tma, cudaStream_t st) {
@@ -700,7 +686,7 @@ frt_status launch_gp(const Args& a, bool tma, cudaStream_t st) {
     const frt_status os = opt_in_smem(kt, smem, opted);
     if (os != FRT_OK) return os;
     const int per = KV8 ? a.H : a.Hq + a.Hkv;  // lane groups needed for one slot of every processed head
-    int NG = (per * GP <= 128) ? per : 128 / GP;
+    int NG = (per * GP <= kTmaThreads) ? per : kTmaThreads / GP;
     if (NG < 1) NG = 1;
     const int threads = ((NG * GP + 31) / 32) * 32;
     return launch(kt, dim3((unsigned)a.M), dim3(threads), smem, st, qkv, qw, kw, a.cos_tab, a.sin_tab, a.pos, qo,
@@ -752,7 +738,7 @@ frt_status launch_ln_gp(const Args& a, cudaStream_t st) {
   const frt_status os = opt_in_smem(kt, smem, opted);
   if (os != FRT_OK) return os;
   const int per = a.Hq + a.Hkv;
-  int NG = (per * GP <= 128) ? per : 128 / GP;
+  int NG = (per * GP <= kTmaThreadsLn) ? per : kTmaThreadsLn / GP;
   if (NG < 1) NG = 1;
   const int threads = ((NG * GP + 31) / 32) * 32;
   return launch(kt, dim3((unsigned)a.M), dim3(threads), smem, st, static_cast<const uint16_t*>(a.qkv),
