@@ -209,7 +209,6 @@ __device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t*
 template <int DT, int QM, int ACT>
 __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* bs, const Divisor& dv, int64_t row,
                                           const Slice& sl, int I4, int NBI) {
-  using P16 = Pack16<DT>;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   uint32_t* dst = q + row * I4;
@@ -224,11 +223,11 @@ __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* b
       const int b = sl.b0 + i0 + u;
       float a[4];
       const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[u]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 pr = P16::to_float2(w[e]);
-        a[e] = act_fn<ACT>(pr.x) * pr.y;
-      }
+      const float2 a01 = act_mul2<DT, ACT>(w[0], w[1]), a23 = act_mul2<DT, ACT>(w[2], w[3]);
+      a[0] = a01.x;
+      a[1] = a01.y;
+      a[2] = a23.x;
+      a[3] = a23.y;
       if (QM == FRT_QUANT_BLOCK128) {
         const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
         const float sb = block_scale_448(am);

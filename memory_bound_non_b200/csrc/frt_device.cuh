@@ -285,25 +285,57 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ------------------------------------------------------- activations --
-constexpr float kSqrt2OverPi = 0.7978845608028654f;
-constexpr float kGeluCubic = 0.044715f;
+// act(g) in fp32 on packed pairs of gates.  GELU-tanh uses
+// 0.5 (1 + tanh(z)) = 1 / (1 + exp(-2 z)), z = sqrt(2/pi) (g + 0.044715 g^3),
+// and SiLU is g / (1 + exp(-g)).  exp(x) is formed as 2^(x log2 e): the
+// product with log2 e is folded into the polynomial's constants and 2^t is
+// the special-function unit's ex2 (relative error about 2^-22), the quotient
+// g / (1 + e) a multiply by its rcp (about one ulp); both far below the
+// half-step of an FP8 or e2m1 code.  t is capped at 115 (2^115 ~ e^80) so the
+// denominator stays finite; the result is ~0 there either way.  The other
+// steps are fp32 multiplies / FMAs two at a time (mul/fma .f32x2), each half
+// rounded as the scalar operation.
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kGeluC0 = (float)(-2.0 * 0.7978845608028654 * 1.4426950408889634);
+constexpr float kGeluC1 = (float)(-2.0 * 0.7978845608028654 * 0.044715 * 1.4426950408889634);
+constexpr float kExp2Cap = 115.0f;
 
-// act(g) in fp32.  GELU-tanh uses 0.5 (1 + tanh(z)) = 1 / (1 + exp(-2 z)) and
-// SiLU is g / (1 + exp(-g)); the exponent is capped at 80 so the denominator
-// stays finite (the result is ~0 there either way).
+__device__ __forceinline__ float ex2_approx(float t) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(t));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// g / (1 + 2^t) per half, t capped
+__device__ __forceinline__ float2 div_one_plus_exp2(float2 g, float2 t) {
+  const float2 e = make_float2(ex2_approx(fminf(t.x, kExp2Cap)), ex2_approx(fminf(t.y, kExp2Cap)));
+  const float2 d = __fadd2_rn(e, make_float2(1.0f, 1.0f));
+  return __fmul2_rn(g, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
 template <int ACT>
-__device__ __forceinline__ float act_fn(float g) {
+__device__ __forceinline__ float2 act2(float2 g) {
   if (ACT == FRT_ACT_RELU2) {
-    const float r = fmaxf(g, 0.0f);
-    return r * r;
+    const float2 r = make_float2(fmaxf(g.x, 0.0f), fmaxf(g.y, 0.0f));
+    return __fmul2_rn(r, r);
   } else if (ACT == FRT_ACT_SILU) {
-    const float e = expf(fminf(-g, 80.0f));
-    return __fdividef(g, 1.0f + e);
+    return div_one_plus_exp2(g, __fmul2_rn(g, make_float2(-kLog2e, -kLog2e)));
   } else {
-    const float z = g * fmaf(kSqrt2OverPi * kGeluCubic, g * g, kSqrt2OverPi);
-    const float e = expf(fminf(-2.0f * z, 80.0f));
-    return __fdividef(g, 1.0f + e);
+    const float2 p = __ffma2_rn(__fmul2_rn(g, g), make_float2(kGeluC1, kGeluC1), make_float2(kGeluC0, kGeluC0));
+    return div_one_plus_exp2(g, __fmul2_rn(g, p));
   }
+}
+
+// act(g) * u for the (gate, up) pairs held in two packed 16-bit words.
+template <int DT, int ACT>
+__device__ __forceinline__ float2 act_mul2(uint32_t w0, uint32_t w1) {
+  const float2 p0 = Pack16<DT>::to_float2(w0), p1 = Pack16<DT>::to_float2(w1);
+  return __fmul2_rn(act2<ACT>(make_float2(p0.x, p1.x)), make_float2(p0.y, p1.y));
 }
 
 // --------------------------------------------------------- reductions --

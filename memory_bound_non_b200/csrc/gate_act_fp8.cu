@@ -25,13 +25,19 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kU = 4;  // scale blocks per warp
 
+// Six CTAs (48 warps) per SM need at most 40 registers a thread; the
+// block-128 form would take 43 unasked and drop to five.
+template <int QM, bool FULL>
+constexpr int gate_min_blocks() {
+  return QM == FRT_QUANT_BLOCK128 && FULL ? 6 : 1;
+}
+
 template <int DT, int ACT, int QM, bool FULL>
-__global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __restrict__ gu,
+__global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_act_fp8_kernel(const uint4* __restrict__ gu,
                                                                  uint32_t* __restrict__ q,
                                                                  const float* __restrict__ static_scale,
                                                                  float* __restrict__ block_scales,
                                                                  int64_t total_blocks, int NB, int C4) {
-  using P16 = Pack16<DT>;
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -77,12 +83,12 @@ __global__ void __launch_bounds__(kThreads) gate_act_fp8_kernel(const uint4* __r
   for (int u = 0; u < kU; ++u) {
     float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (valid[u]) {
-      const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[u]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 p = P16::to_float2(w[e]);  // (gate, up)
-        a[e] = act_fn<ACT>(p.x) * p.y;
-      }
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[u]);  // (gate, up) pairs
+      const float2 a01 = act_mul2<DT, ACT>(w[0], w[1]), a23 = act_mul2<DT, ACT>(w[2], w[3]);
+      a[0] = a01.x;
+      a[1] = a01.y;
+      a[2] = a23.x;
+      a[3] = a23.y;
     }
     // code = e4m3(a / s) with the quotient correctly rounded in fp32
     if (QM == FRT_QUANT_BLOCK128) {
