@@ -229,7 +229,7 @@ __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* b
       a[2] = a23.x;
       a[3] = a23.y;
       if (QM == FRT_QUANT_BLOCK128) {
-        const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
+        const float am = warp_max_abs(absmax4(a[0], a[1], a[2], a[3]));
         const float sb = block_scale_448(am);
         if (lane == 0) bs[row * NBI + b] = sb;
         dst[b * 32 + lane] = quant4(a, Divisor(sb));

@@ -352,6 +352,14 @@ __device__ __forceinline__ float group_max(float v) {
   return v;
 }
 
+// max |v| over the 32 lanes of the warp in one instruction (sm_100's f32
+// redux; NaN inputs are ignored, as fmaxf does).  Every lane must call it.
+__device__ __forceinline__ float warp_max_abs(float v) {
+  float r;
+  asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 __device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
 }

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
     }
     // code = e4m3(a / s) with the quotient correctly rounded in fp32
     if (QM == FRT_QUANT_BLOCK128) {
-      const float am = group_max<32>(absmax4(a[0], a[1], a[2], a[3]));
+      const float am = warp_max_abs(absmax4(a[0], a[1], a[2], a[3]));
       const float sb = block_scale_448(am);
       const int64_t gb = gb0 + u;
       if (lane == 0 && gb < total_blocks) block_scales[gb] = sb;  // [M, NB] row-major == flat block index
