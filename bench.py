@@ -30,7 +30,9 @@ Also reported on the same JSON line:
                 buffers: host->device copy of the step's inputs, the four ops,
                 device->host copy of the step's outputs;
   clocks        nvidia-smi SM clock and throttle reasons sampled while timing;
-  cpu_baseline  the CPU oracle (single thread) on a bounded row sample.
+  cpu_baseline  the CPU oracle (single thread) on a bounded row sample;
+                cpu_baseline_all_cores the same oracle in one spawned process
+                per host core, each on its own row block.
 
 Multi-GPU (torchrun): each rank runs its own row shard (weak scaling, no
 collective on the data path); timing is max over ranks.
@@ -733,7 +735,34 @@ def cpu_baseline(wl, host, budget_s=12.0):
     b = sum(op_bytes(dataclasses.replace(wl, M=rows)).values())
     return {"value": round(b / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": "first %d of %d token rows of every op of the step (%.1f s, single thread)"
-                      % (rows, wl.M, secs)}
+                      % (rows, wl.M, secs)}, rows / secs
+
+
+def _oracle_worker(task):
+    """One process of the all-cores oracle leg: its own seeded inputs for a
+    row block, then the oracle on them; returns seconds."""
+    import dataclasses
+    from memory_bound_non_b200 import workloads as W
+    wl, rows = task
+    small = dataclasses.replace(wl, M=rows)
+    host = W.make_inputs(small, n_layers=1)
+    return oracle_sample(small, host, rows)
+
+
+def cpu_baseline_all_cores(wl, rows_per_s, budget_s=4.0, max_cores=32, max_rows=1024):
+    """The same oracle, as it stands, in one process per host core (spawned,
+    never forked from this CUDA process), each on its own block of rows;
+    throughput = all rows' bytes / the slowest process's time."""
+    import dataclasses
+    import multiprocessing as mp
+    cores = max(1, min(os.cpu_count() or 1, max_cores))
+    rows = int(max(16, min(max_rows, rows_per_s * budget_s)))  # bounds each process's host memory
+    with mp.get_context("spawn").Pool(cores) as pool:
+        secs = pool.map(_oracle_worker, [(wl, rows)] * cores)
+    b = cores * sum(op_bytes(dataclasses.replace(wl, M=rows)).values())
+    return {"value": round(b / max(secs) / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": "%d processes x %d token rows of every op of the step (slowest %.1f s)"
+                      % (cores, rows, max(secs))}
 
 
 def host_inputs_only(wl):
@@ -838,8 +867,9 @@ def main(argv=None):
     for name, ts in per_op_us.items():
         mean_us = sum(ts) / len(ts)
         gbs = bytes_op[name] / (mean_us * 1e-6) / 1e9
+        q = statistics.quantiles(ts, n=10) if len(ts) >= 2 else [mean_us] * 9
         per_op[name] = {"us_mean": round(mean_us, 2), "us_median": round(statistics.median(ts), 2),
-                        "bytes": bytes_op[name], "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                        "us_p10": round(q[0], 2), "us_p90": round(q[8], 2), "bytes": bytes_op[name], "GBps": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
                         "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4)}
     dom = max(per_op, key=lambda k: per_op[k]["us_mean"])
     traffic = measured_traffic(wl.name, dom)
@@ -869,9 +899,10 @@ def main(argv=None):
         e2e_ms = max_over_ranks(e2e_ms)
         e2e = {"value": round(job_throughput(step_bytes, world, e2e_ms), 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
-    cpu = None
+    cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(step.wl, step.host)
+        cpu, rows_per_s = cpu_baseline(step.wl, step.host)
+        cpu_all = cpu_baseline_all_cores(step.wl, rows_per_s)
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -884,7 +915,8 @@ def main(argv=None):
                            "l2": "inputs larger than L2 (%.1f GB per step)" % (step_bytes / 1e9),
                            "parallelism": "row shards, no collective" if world > 1 else "single GPU"},
                 "roofline": roofline, "per_op": per_op, "gpu_launches": 4 * args.steps, "clocks": clk,
-                "e2e": e2e, "cpu_baseline": cpu, "input_gen_s": round(step.gen_s, 1)}
+                "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_all,
+                "input_gen_s": round(step.gen_s, 1)}
         line.update(extra)
         s = json.dumps(line)
         print(s, flush=True)
