@@ -119,7 +119,7 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
     }
     if (QM == FRT_QUANT_BLOCK128) {
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
-      am = group_max<16>(am);
+      am = half_warp_max_abs(am);
       const float sb = block_scale_448(am);
       if (valid && (j & 15) == 0) bs[row * NB + (c >> 4)] = sb;
       if (valid) q[row * C + c] = quant8(y, Divisor(sb));

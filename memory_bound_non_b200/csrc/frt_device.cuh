@@ -360,6 +360,16 @@ __device__ __forceinline__ float warp_max_abs(float v) {
   return r;
 }
 
+// max |v| over each 16-lane half of the warp: two warp-wide f32 reductions,
+// each seeing only one half's values (the other half contributes 0).
+// Every lane must call it.
+__device__ __forceinline__ float half_warp_max_abs(float v) {
+  const bool upper = (threadIdx.x & 16) != 0;
+  const float lo = warp_max_abs(upper ? 0.0f : v);
+  const float hi = warp_max_abs(upper ? v : 0.0f);
+  return upper ? hi : lo;
+}
+
 __device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
 }

@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     }
     if (QM == FRT_QUANT_BLOCK128) {
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
-      am = group_max<16>(am);  // 16 lanes = the 16 chunks of one 128-column block
+      am = half_warp_max_abs(am);  // 16 lanes = the 16 chunks of one 128-column block
       const float sb = block_scale_448(am);
       if (valid && (t & 15) == 0) block_scales[row * NB + (c >> 4)] = sb;
       if (valid) q[base + c] = quant8(y, Divisor(sb));
