@@ -70,3 +70,15 @@ def test_op_bytes_are_the_algorithmic_bytes():
     assert b["qkv"] == 65536 * 6144 * 4 + 65536 * 128 * 4 + 4 * 65536 + 4 * 128
     # c: gate/up read (4 B per output) + fp8 out, static scale
     assert b["gate"] == 65536 * 16384 * 5 + 4
+
+
+def test_all_cores_oracle_leg_counts_every_process_rows():
+    """The all-cores CPU leg: spawned processes, each on its own row block;
+    the reported throughput counts every process's rows over the slowest
+    process's time, and the rows per process are bounded."""
+    wl = W.get("tiny")
+    out = bench.cpu_baseline_all_cores(wl, rows_per_s=1e6, budget_s=1.0, max_cores=2, max_rows=32)
+    assert out["kind"] == "oracle" and out["unit"] == "GB/s"
+    assert out["cores"] == min(2, os.cpu_count() or 1)
+    assert "%d processes x 32 token rows" % out["cores"] in out["sample"]
+    assert out["value"] > 0
