@@ -184,6 +184,17 @@ __device__ __forceinline__ uint32_t nvfp4_scale(float amax, float rden, float gs
   *reff = eff > 0.0f ? __frcp_rn(eff) : 0.0f;
   return sf;
 }
+// The same with RN(1 / eff) looked up per sf code: reff_of[sf] for all 256
+// codes, filled once per CTA by nvfp4_reff_entry.
+__device__ __forceinline__ float nvfp4_reff_entry(uint32_t sf, float gs) {
+  const float eff = e4m3_value(sf) * gs;
+  return eff > 0.0f ? __frcp_rn(eff) : 0.0f;
+}
+__device__ __forceinline__ uint32_t nvfp4_scale_lookup(float amax, float rden, const float* reff_of, float* reff) {
+  const uint32_t sf = e4m3x2(amax * rden, 0.0f) & 0xFFu;
+  *reff = reff_of[sf];
+  return sf;
+}
 // N (4 or 8) values -> N e2m1 codes of y * reff, element 0 in the low nibble.
 template <int N>
 __device__ __forceinline__ uint32_t nvfp4_codes(const float* y, float reff) {
@@ -345,12 +356,6 @@ __device__ __forceinline__ float group_sum(float v) {
   for (int o = WIDTH / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
   return v;
 }
-template <int WIDTH>
-__device__ __forceinline__ float group_max(float v) {
-#pragma unroll
-  for (int o = WIDTH / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
 
 // max |v| over the 32 lanes of the warp in one instruction (sm_100's f32
 // redux; NaN inputs are ignored, as fmaxf does).  Every lane must call it.
@@ -417,14 +422,6 @@ __device__ __forceinline__ void scale_pairs(float2* x, float r, const float2* w)
   const float2 rr = make_float2(r, r);
 #pragma unroll
   for (int e = 0; e < NP; ++e) x[e] = __fmul2_rn(__fmul2_rn(x[e], rr), w[e]);
-}
-
-// x <- (x * r) * w per element, w given as packed 16-bit pairs.
-template <int DT, int NP>
-__device__ __forceinline__ void scale_pairs_w16(float2* x, float r, const uint32_t* w) {
-  const float2 rr = make_float2(r, r);
-#pragma unroll
-  for (int e = 0; e < NP; ++e) x[e] = __fmul2_rn(__fmul2_rn(x[e], rr), Pack16<DT>::to_float2(w[e]));
 }
 
 // Rotate-half RoPE: o1 = a cos - b sin, o2 = b cos + a sin, each one FMA on

@@ -24,12 +24,14 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kU = 4;  // scale blocks per warp
+static_assert(kThreads == 256, "the NVFP4 reciprocal table takes one sf code per thread");
 
 // Six CTAs (48 warps) per SM need at most 40 registers a thread; the
-// block-128 form would take 43 unasked and drop to five.
+// block-128 and row-major NVFP4 forms would take 43-44 unasked and drop to
+// five (the swizzled NVFP4 form would spill at 40 and keeps five).
 template <int QM, bool FULL>
 constexpr int gate_min_blocks() {
-  return QM == FRT_QUANT_BLOCK128 && FULL ? 6 : 1;
+  return (QM == FRT_QUANT_BLOCK128 || QM == kQuantNvfp4Rows) && FULL ? 6 : 1;
 }
 
 template <int DT, int ACT, int QM, bool FULL>
@@ -78,6 +80,13 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
   const float gs = QM >= kQuantNvfp4Rows ? __ldg(static_scale) : 0.0f;
   const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * gs) : 0.0f;
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? __ldg(static_scale) : 1.0f);
+  // NVFP4: RN(1 / RN(sf * gs)) for each of the 256 sf codes, one per thread,
+  // formed while the loads above are in flight
+  __shared__ float reff_of[QM >= kQuantNvfp4Rows ? kThreads : 1];
+  if (QM >= kQuantNvfp4Rows) {
+    reff_of[threadIdx.x] = nvfp4_reff_entry(threadIdx.x, gs);
+    __syncthreads();
+  }
 
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
@@ -105,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
       am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
       am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
       float reff;
-      const uint32_t sf = nvfp4_scale(am, rden, gs, &reff);
+      const uint32_t sf = nvfp4_scale_lookup(am, rden, reff_of, &reff);
       if (valid[u]) {
         reinterpret_cast<uint16_t*>(q)[idx[u]] = (uint16_t)nvfp4_codes<4>(a, reff);
         if ((lane & 3) == 0) {
