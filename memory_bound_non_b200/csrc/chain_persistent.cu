@@ -96,7 +96,11 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
 #pragma unroll
   for (int k = 1; k < K; ++k) sst += ss[k];
   const double tot = block_sum(sst, red);
-  const Split32 rstd(rsqrt_f64(tot / (double)D + (double)eps));
+  // static FP8: one product with rstd / s, as op a does
+  const double rstd64 = rsqrt_f64(tot / (double)D + (double)eps);
+  const double rs64 = QM == FRT_QUANT_STATIC ? rstd64 / (double)dv.s : 0.0;
+  const bool fold = QM == FRT_QUANT_STATIC && rs64 >= 0x1p-100 && rs64 <= 0x1p+100;
+  const Split32 rstd(fold ? rs64 : rstd64);
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int j = t + k * kChainThreads;
@@ -124,7 +128,7 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
       if (valid && (j & 15) == 0) bs[row * NB + (c >> 4)] = sb;
       if (valid) q[row * C + c] = quant8(y, Divisor(sb));
     } else if (valid) {
-      q[row * C + c] = quant8(y, dv);
+      q[row * C + c] = fold ? e4m3x8(y) : quant8(y, dv);
     }
   }
 }

@@ -158,6 +158,10 @@ __device__ __forceinline__ uint32_t quant4(const float* y, const Divisor& dv) {
 __device__ __forceinline__ uint2 quant8(const float* y, const Divisor& dv) {
   return make_uint2(quant4(y, dv), quant4(y + 4, dv));
 }
+// Eight values already divided by the scale -> eight e4m3 codes.
+__device__ __forceinline__ uint2 e4m3x8(const float* v) {
+  return make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
+}
 
 // ----------------------------------------------------------------- NVFP4 --
 // e2m1 elements in 16-element blocks, each block scaled by an unsigned e4m3

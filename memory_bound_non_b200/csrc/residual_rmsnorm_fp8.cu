@@ -151,7 +151,13 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     for (int i = 0; i < nw; ++i) tot += red[i];
   }
   const double rstd64 = rsqrt_f64(tot / (double)D + (double)eps);
-  const Split32 rstd(rstd64);
+  // Static FP8 on the RMS path: y / s as one product with rstd / s (fp64,
+  // held as an fp32 pair), so each code is decided on one fp32 rounding of
+  // h w rstd / s rather than on RN(RN(h w rstd) / s).  A ratio outside
+  // [2^-100, 2^100] keeps y and the division.
+  const double rs64 = QM == FRT_QUANT_STATIC && !LN ? rstd64 / (double)s_static : 0.0;
+  const bool fold = QM == FRT_QUANT_STATIC && !LN && rs64 >= 0x1p-100 && rs64 <= 0x1p+100;
+  const Split32 rstd(fold ? rs64 : rstd64);
   const float rstd32 = (float)rstd64;
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
   const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * s_static) : 0.0f;  // NVFP4: RN(1 / RN(6 gs))
@@ -223,7 +229,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
         }
       }
     } else if (valid) {
-      q[base + c] = quant8(y, dv_static);
+      q[base + c] = fold ? e4m3x8(y) : quant8(y, dv_static);
     }
   }
 }
