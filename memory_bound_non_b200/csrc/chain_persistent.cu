@@ -62,8 +62,8 @@ struct Slice {
 // Op a on the row (held by this CTA): h = x + r (into hv), RMSNorm, FP8 codes.
 template <int DT, int K, int QM>
 __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uint2* q, float* bs, const Divisor& dv,
-                                           uint4 (&hv)[K], int64_t row, const Slice& sl, int C, int NB, float D,
-                                           float eps, double* red) {
+                                           double inv_s64, uint4 (&hv)[K], int64_t row, const Slice& sl, int C,
+                                           int NB, float D, float eps, double* red) {
   using P16 = Pack16<DT>;
   const int t = threadIdx.x;
   uint4 xv[K], wv[K];
@@ -98,7 +98,7 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
   const double tot = block_sum(sst, red);
   // static FP8: one product with rstd / s, as op a does
   const double rstd64 = rsqrt_f64(tot / (double)D + (double)eps);
-  const double rs64 = QM == FRT_QUANT_STATIC ? rstd64 / (double)dv.s : 0.0;
+  const double rs64 = rstd64 * inv_s64;
   const bool fold = QM == FRT_QUANT_STATIC && rs64 >= 0x1p-100 && rs64 <= 0x1p+100;
   const Split32 rstd(fold ? rs64 : rstd64);
 #pragma unroll
@@ -328,6 +328,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
                            nsn8);
   const Divisor dv_attn(QM == FRT_QUANT_STATIC ? __ldg(scales) : 1.0f);
   const Divisor dv_ffn(QM == FRT_QUANT_STATIC ? __ldg(scales + 1) : 1.0f);
+  // static FP8: 1 / s in fp64 for the norms' folded product (0 otherwise)
+  const double inv_attn = QM == FRT_QUANT_STATIC ? 1.0 / (double)dv_attn.s : 0.0;
+  const double inv_ffn = QM == FRT_QUANT_STATIC ? 1.0 / (double)dv_ffn.s : 0.0;
   const Divisor dv_act(QM == FRT_QUANT_STATIC ? __ldg(scales + 2) : 1.0f);
   const float D = (float)(C * 8);
   const int qkv16 = H * hd / 8, hd16 = hd / 8;
@@ -361,7 +364,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
     const uint4* st = stages + (it & 1) * m.len;
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xa, L.w_attn != nullptr ? st + m.wa : nullptr,
-                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, hv, row, sl, C, NB, D, eps, red);
+                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, inv_attn, hv, row, sl, C, NB, D, eps, red);
     chain_qkv<DT, GP>(reinterpret_cast<const uint16_t*>(st + m.qkv),
                       L.q_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.qw) : nullptr,
                       L.k_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.kw) : nullptr,
@@ -369,7 +372,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
                       static_cast<uint16_t*>(L.v_cache), cs8, sn8, nsn8, row, p, row_ok, sl, Hq, Hkv, hd, G, eps);
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xf, L.w_ffn != nullptr ? st + m.wf : nullptr, reinterpret_cast<uint2*>(L.q8_ffn),
-                            L.bs_ffn, dv_ffn, hv, row, sl, C, NB, D, eps, red);
+                            L.bs_ffn, dv_ffn, inv_ffn, hv, row, sl, C, NB, D, eps, red);
     chain_act<DT, QM, ACT>(st + m.gu, reinterpret_cast<uint32_t*>(L.act8), L.bs_act, dv_act, row, sl, I4, NBI);
     __syncthreads();  // the stage read here is refilled at iteration it + 2
   }

@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   }
   float s_static = 0.0f;
   if (QM == FRT_QUANT_STATIC || QM >= kQuantNvfp4Rows) s_static = __ldg(static_scale);
+  // 1 / s in fp64, formed while the row's loads are in flight
+  const double inv_s64 = QM == FRT_QUANT_STATIC && !LN ? 1.0 / (double)s_static : 0.0;
   // Narrow rows (small-batch, latency-bound calls) load the weight with the
   // row instead of after the reduction: one memory round trip less on the
   // critical path.  Wide rows keep the registers for occupancy.
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   // held as an fp32 pair), so each code is decided on one fp32 rounding of
   // h w rstd / s rather than on RN(RN(h w rstd) / s).  A ratio outside
   // [2^-100, 2^100] keeps y and the division.
-  const double rs64 = QM == FRT_QUANT_STATIC && !LN ? rstd64 / (double)s_static : 0.0;
+  const double rs64 = rstd64 * inv_s64;
   const bool fold = QM == FRT_QUANT_STATIC && !LN && rs64 >= 0x1p-100 && rs64 <= 0x1p+100;
   const Split32 rstd(fold ? rs64 : rstd64);
   const float rstd32 = (float)rstd64;
