@@ -133,6 +133,22 @@ def test_residual_rmsnorm_saturates_and_is_deterministic():
     P.assert_fp8_codes(q1.cpu().numpy(), o["out_fp8"])
 
 
+@pytest.mark.parametrize("s", [2.0 ** -110, 2.0 ** -99, 2.0 ** 99, 2.0 ** 110])
+def test_residual_rmsnorm_static_scale_far_from_one(s):
+    """A static scale whose ratio to rstd leaves (or nears the edge of) the
+    range where the kernel folds 1/s into its fp32-pair product: the codes
+    still follow e4m3(y / s) (all saturated for the tiny scales, all +-0 or
+    subnormal for the huge ones)."""
+    wl = W.get("tiny", quant="static")
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False)
+    L = inp.layers[0]
+    x, r = W.bits16(L.x_attn), W.bits16(inp.residual)
+    w = None if L.w_attn is None else W.bits16(L.w_attn)
+    _, q, _ = run_a_gpu(wl, inp, s)
+    o = oracle.residual_rmsnorm_fp8(x, r, w, wl.eps, wl.dt, "static", static_scale=s)
+    P.assert_fp8_codes(q.cpu().numpy(), o["out_fp8"], what="op a codes, scale %g" % s)
+
+
 # ================================================================ op (b) ===
 B_CASES = [
     ("tiny", {}), ("pi05", {}), ("vla_denoise", {}), ("vit", {}), ("qwen3_prefill_S128", {}),
