@@ -22,7 +22,7 @@
 // (asynchronous copies) while the current one computes.  With real GEMMs
 // between the ops, rows would mix and a grid-wide step would be needed.  Each
 // op uses the arithmetic of its per-op kernel (packed 16-bit add, fp64 row sum
-// of squares, correctly rounded FP8 decisions, the same RoPE and activation
+// of squares, the same FP8 decision arithmetic, RoPE and activation
 // expressions), so the results equal the per-op launches bit for bit.
 #include <atomic>
 #include <cmath>

@@ -10,7 +10,7 @@
 // Mapping (B200): a 16-byte load holds 4 (g, u) pairs -> 4 outputs -> one
 // 32-bit store of 4 codes, so one warp-wide load covers exactly one 128-column
 // scale block (512 contiguous input bytes, 128 output bytes) and the block's
-// amax is a 5-step xor shuffle.  Each warp owns U consecutive blocks of the
+// amax is one warp-wide f32 redux.  Each warp owns U consecutive blocks of the
 // flattened (row, block) index space and issues all U loads before computing,
 // which keeps enough bytes in flight per SM to saturate HBM.
 #include <cmath>

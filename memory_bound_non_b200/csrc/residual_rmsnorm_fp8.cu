@@ -13,8 +13,10 @@
 // of squares is reduced warp-shuffle -> shared memory -> every thread, in a
 // fixed order (bitwise deterministic), in fp64 so the normalised values come
 // out correctly rounded in fp32.  For block-128 scales a 128-column block
-// is 16 chunks owned by 16 consecutive lanes, so its amax is a 4-step xor
-// shuffle inside the warp; no shared memory and no second pass.
+// is 16 chunks owned by 16 consecutive lanes (a half-warp), so its amax comes
+// from two warp-wide f32 reduxes; no shared memory and no second pass.  With
+// a static scale, rstd / s is folded into the product, so no per-element
+// division remains.
 #include <cmath>
 
 #include "frt_device.cuh"
