@@ -108,9 +108,13 @@ typedef enum { FRT_KV_16BIT = 0, FRT_KV_E4M3 = 1 } frt_kv_format;
  *              16-bit type (RNE); written to residual_out (the new residual
  *              stream).
  *   rstd_i   = 1 / sqrt(mean_j(h[i,j]^2) + eps), computed from the rounded h
- *              with fp32 accumulation in a fixed order.
+ *              with fp64 accumulation (the squares are exact) in a fixed
+ *              order.
  *   y[i,j]   = h[i,j] * rstd_i * weight[j]   (weight == NULL: no weight).
  *   out_fp8  = e4m3 of y / s (quant mode as above; block scales over D).
+ *              The value converted is y / s rounded to fp32: with a static
+ *              scale one rounding of h * w * (rstd / s), with block-128
+ *              scales the correctly rounded quotient of the fp32 y.
  *
  *   x, residual_in, residual_out  device, [M, D] 16-bit, 16-byte aligned;
  *                                 residual_out may equal residual_in.
