@@ -143,7 +143,8 @@ frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residual_in, void
  *   v      = one Q or K head, in fp32;
  *   norm   v = v * (1/sqrt(mean(v^2) + eps)) * w   with w = q_norm_w for Q
  *            heads, k_norm_w for K heads; skipped for a side whose weight is
- *            NULL;
+ *            NULL (fp32; 1/sqrt by the hardware reciprocal square root,
+ *            relative error about 2^-22);
  *   rope   for j < half, c = cos_tab[p, j], s = sin_tab[p, j]:
  *            o[j] = v[j] c - v[j+half] s,  o[j+half] = v[j+half] c + v[j] s;
  *   q_out[i, h, :]          = o (Q head h), rounded once to 16 bits;
@@ -188,7 +189,9 @@ frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_norm_w, cons
  * "sm89 prefill FFN megakernel", Phase 2 (silu * mul + per-token block-128 FP8).
  *
  *   a[i,j]   = act(g) * u with g = gate_up[i, 2j], u = gate_up[i, 2j+1],
- *              in fp32, one rounding at the FP8 store.
+ *              in fp32 (GELU-tanh and SiLU through exp(x) = 2^(x log2 e) and
+ *              1 / (1 + e) on the special-function unit's approximations,
+ *              relative error about 2^-21).
  *   out_fp8  = e4m3 of a / s (quant mode as above; block scales over I).
  *
  *   gate_up       device [M, 2I] 16-bit, 16-byte aligned.
