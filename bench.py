@@ -30,6 +30,10 @@ Also reported on the same JSON line:
                 buffers: host->device copy of the step's inputs, the four ops,
                 device->host copy of the step's outputs;
   clocks        nvidia-smi SM clock and throttle reasons sampled while timing;
+  parity        the step's four ops on the GPU for the CPU leg's row sample
+                against the oracle outputs of the same rows (residual and V
+                bit-exact, Q/K within the 16-bit tolerance, FP8 codes at most
+                one step off on at most 0.1 %);
   cpu_baseline  the CPU oracle (single thread) on a bounded row sample;
                 cpu_baseline_all_cores the same oracle in one spawned process
                 per host core, each on its own row block.
@@ -70,6 +74,8 @@ def parse_args(argv=None):
     p.add_argument("--no-chain", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-parity", action="store_true",
+                   help="skip comparing the GPU step on the CPU leg's row sample with the oracle outputs")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--chain-reps", type=int, default=30)
     p.add_argument("--json-out", default=None)
@@ -701,9 +707,9 @@ def e2e_leg(step, K, W_, chunks=8):
 
 
 # -------------------------------------------------------------- CPU legs --
-def oracle_sample(wl, host, rows):
+def oracle_sample(wl, host, rows, keep=None):
     """Run the oracle on the first `rows` rows of every op of the step.
-    Returns seconds."""
+    Returns seconds; with `keep` (a dict) the outputs are stored in it."""
     import oracle
     from memory_bound_non_b200 import workloads as W
     hl = host.layers[0]
@@ -719,23 +725,98 @@ def oracle_sample(wl, host, rows):
     cos, sin = host.cos.cpu().numpy(), host.sin.cpu().numpy()
     t0 = time.perf_counter()
     o = oracle.residual_rmsnorm_fp8(x_a, r, wa, wl.eps, wl.dt, wl.quant, static_scale=0.01)
-    oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, wl.Hq, wl.Hkv, wl.hd, rows, wl.eps, wl.dt,
-                                 slots=np.arange(rows))
-    oracle.residual_rmsnorm_fp8(x_f, o["residual_out"], wf, wl.eps, wl.dt, wl.quant, static_scale=0.01)
-    oracle.gate_act_fp8(gu, wl.act, wl.dt, wl.quant, static_scale=0.01)
-    return time.perf_counter() - t0
+    ob = oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, wl.Hq, wl.Hkv, wl.hd, rows, wl.eps, wl.dt,
+                                      slots=np.arange(rows))
+    of = oracle.residual_rmsnorm_fp8(x_f, o["residual_out"], wf, wl.eps, wl.dt, wl.quant, static_scale=0.01)
+    oc = oracle.gate_act_fp8(gu, wl.act, wl.dt, wl.quant, static_scale=0.01)
+    secs = time.perf_counter() - t0
+    if keep is not None:
+        keep.update(a=o, b=ob, f=of, c=oc)
+    return secs
 
 
-def cpu_baseline(wl, host, budget_s=12.0):
+def _code_steps(got, want):
+    """FP8 e4m3 codes: how many differ, and the largest difference in steps
+    (codes of one sign are ordered like their magnitudes)."""
+    g, w = got.astype(np.int32).ravel(), want.astype(np.int32).ravel()
+    same_sign = (g & 0x80) == (w & 0x80)
+    steps = np.where(same_sign, np.abs((g & 0x7F) - (w & 0x7F)), (g & 0x7F) + (w & 0x7F))
+    return int((g != w).sum()), int(steps.max()) if steps.size else 0
+
+
+def _rel_16bit_ok(got16, want64, dt):
+    """16-bit outputs against fp64 values: |g - o| <= 2e-3 max(|o|, 2^-6) +
+    half an ulp of the 16-bit type."""
+    g = got16.astype(np.float64)
+    ulp = 2.0 ** (-7 if dt == "bf16" else -10)
+    tol = 2e-3 * np.maximum(np.abs(want64), 2.0 ** -6) + 0.5 * ulp * np.abs(want64)
+    return bool(np.all(np.abs(g - want64) <= tol + 1e-30))
+
+
+def step_parity(wl, host, rows, keep):
+    """The step's four ops on the GPU for the first `rows` rows of the bench's
+    inputs (the same kernels, static scale 0.01 as the CPU leg), compared with
+    the oracle outputs the CPU leg kept for the same rows."""
+    import memory_bound_non_b200 as frt
+    from memory_bound_non_b200 import workloads as W
+    dev = torch.device("cuda")
+    hl = host.layers[0]
+    D, I, hd = wl.D, wl.I, wl.hd
+    s = torch.tensor([0.01], dtype=torch.float32, device=dev)
+    x_a, x_f = hl.x_attn[:rows].to(dev), hl.x_ffn[:rows].to(dev)
+    r = host.residual[:rows].to(dev).clone()
+    wa = None if hl.w_attn is None else hl.w_attn.to(dev)
+    wf = None if hl.w_ffn is None else hl.w_ffn.to(dev)
+    qa = torch.empty((rows, D), dtype=torch.uint8, device=dev)
+    qf = torch.empty_like(qa)
+    frt.frt_residual_rmsnorm_fp8(x_a, r, r, wa, qa, static_scale=s, eps=wl.eps, quant="static")
+    r_a = r.clone()
+    frt.frt_residual_rmsnorm_fp8(x_f, r, r, wf, qf, static_scale=s, eps=wl.eps, quant="static")
+    # op b with the RoPE position as the slot: the rows' caches are read back
+    # at their positions (the oracle wrote slot i for row i)
+    pos = host.positions[:rows].to(dev)
+    cap = int(host.positions[:rows].max()) + 1
+    q_out = torch.empty((rows, wl.Hq, hd), dtype=x_a.dtype, device=dev)
+    kc = torch.zeros((cap, wl.Hkv, hd), dtype=x_a.dtype, device=dev)
+    vc = torch.zeros_like(kc)
+    qw = None if hl.q_norm_w is None else hl.q_norm_w.to(dev)
+    kw = None if hl.k_norm_w is None else hl.k_norm_w.to(dev)
+    frt.frt_qkv_norm_rope_kvcache(hl.qkv[:rows].to(dev), qw, kw, host.cos.to(dev), host.sin.to(dev), pos, q_out,
+                                  kc, vc, wl.Hq, wl.Hkv, hd, eps=wl.eps)
+    qc = torch.empty((rows, I), dtype=torch.uint8, device=dev)
+    frt.frt_gate_act_fp8(hl.gate_up[:rows].to(dev), qc, static_scale=s, act=wl.act, quant="static")
+    torch.cuda.synchronize()
+    p = pos.long()
+    out = {"rows": rows}
+    out["residual_bit_exact"] = bool(np.array_equal(W.bits16(r_a.cpu()), keep["a"]["residual_out"])
+                                     and np.array_equal(W.bits16(r.cpu()), keep["f"]["residual_out"]))
+    na, sa = _code_steps(qa.cpu().numpy(), keep["a"]["out_fp8"])
+    nf, sf = _code_steps(qf.cpu().numpy(), keep["f"]["out_fp8"])
+    nc, sc = _code_steps(qc.cpu().numpy(), keep["c"]["out_fp8"])
+    out["fp8_codes_differing"] = {"attn_norm": na, "ffn_norm": nf, "gate": nc}
+    out["fp8_max_step"] = max(sa, sf, sc)
+    q_ok = _rel_16bit_ok(q_out.float().cpu().numpy(), keep["b"]["q_out"], wl.dt)
+    k_ok = _rel_16bit_ok(kc[p].float().cpu().numpy(), keep["b"]["k_cache"][:rows], wl.dt)
+    v_ok = bool(np.array_equal(W.bits16(vc[p].cpu()).reshape(rows, -1),
+                               W.bits16(hl.qkv[:rows])[:, (wl.Hq + wl.Hkv) * hd:]))
+    out["qkv_within_tolerance"] = bool(q_ok and k_ok)
+    out["v_bit_exact"] = v_ok
+    n_codes = rows * (2 * D + I)
+    out["ok"] = bool(out["residual_bit_exact"] and q_ok and k_ok and v_ok and out["fp8_max_step"] <= 1
+                     and (na + nf + nc) <= 0.001 * n_codes)
+    return out
+
+
+def cpu_baseline(wl, host, budget_s=12.0, keep=None):
     import dataclasses
     rows = 16
     secs = oracle_sample(wl, host, rows)
     rows = int(max(16, min(wl.M, rows * budget_s / max(secs, 1e-6))))
-    secs = oracle_sample(wl, host, rows)
+    secs = oracle_sample(wl, host, rows, keep=keep)
     b = sum(op_bytes(dataclasses.replace(wl, M=rows)).values())
     return {"value": round(b / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": "first %d of %d token rows of every op of the step (%.1f s, single thread)"
-                      % (rows, wl.M, secs)}, rows / secs
+                      % (rows, wl.M, secs)}, rows / secs, rows
 
 
 def _oracle_worker(task):
@@ -899,10 +980,19 @@ def main(argv=None):
         e2e_ms = max_over_ranks(e2e_ms)
         e2e = {"value": round(job_throughput(step_bytes, world, e2e_ms), 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
-    cpu = cpu_all = None
+    cpu = cpu_all = parity = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu, rows_per_s = cpu_baseline(step.wl, step.host)
+        want_parity = not args.no_parity
+        keep = {} if want_parity else None
+        cpu, rows_per_s, rows = cpu_baseline(step.wl, step.host, keep=keep)
         cpu_all = cpu_baseline_all_cores(step.wl, rows_per_s)
+        if want_parity and step.wl.quant != "static":
+            parity = {"ok": None, "skipped": "the CPU leg's sample uses a static scale"}
+        elif want_parity:
+            try:
+                parity = step_parity(step.wl, step.host, rows, keep)
+            except Exception as exc:  # reported, never fatal to the timing line
+                parity = {"ok": False, "error": "%s: %s" % (type(exc).__name__, exc)}
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -915,7 +1005,7 @@ def main(argv=None):
                            "l2": "inputs larger than L2 (%.1f GB per step)" % (step_bytes / 1e9),
                            "parallelism": "row shards, no collective" if world > 1 else "single GPU"},
                 "roofline": roofline, "per_op": per_op, "gpu_launches": 4 * args.steps, "clocks": clk,
-                "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_all,
+                "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_all, "parity": parity,
                 "input_gen_s": round(step.gen_s, 1)}
         line.update(extra)
         s = json.dumps(line)

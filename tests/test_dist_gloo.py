@@ -82,3 +82,19 @@ def test_all_cores_oracle_leg_counts_every_process_rows():
     assert out["cores"] == min(2, os.cpu_count() or 1)
     assert "%d processes x 32 token rows" % out["cores"] in out["sample"]
     assert out["value"] > 0
+
+
+def test_parity_helpers_count_code_steps_and_16bit_tolerance():
+    """The bench's parity summary: FP8 codes compared by count and by steps
+    (one sign's codes are ordered like their magnitudes; across signs the
+    steps go through zero), 16-bit outputs against fp64 values."""
+    import numpy as np
+    want = np.array([0x00, 0x38, 0x38, 0xB8, 0x7E], dtype=np.uint8)
+    got = np.array([0x00, 0x39, 0x38, 0x38, 0x7E], dtype=np.uint8)
+    n, steps = bench._code_steps(got, want)
+    assert n == 2 and steps == 2 * 0x38
+    n, steps = bench._code_steps(want, want)
+    assert n == 0 and steps == 0
+    o = np.array([1.0, -3.0, 1e-3])
+    assert bench._rel_16bit_ok(o.astype(np.float32), o, "bf16")
+    assert not bench._rel_16bit_ok((o * 1.02).astype(np.float32), o, "bf16")
