@@ -846,11 +846,6 @@ def cpu_baseline_all_cores(wl, rows_per_s, budget_s=4.0, max_cores=32, max_rows=
                       % (cores, rows, max(secs))}
 
 
-def host_inputs_only(wl):
-    from memory_bound_non_b200 import workloads as W
-    return W.make_inputs(wl, n_layers=1)
-
-
 def reference_arm(args):
     """The oracle, as it stands, timed on host cores on the same workload."""
     import dataclasses
