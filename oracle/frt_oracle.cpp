@@ -212,14 +212,17 @@ void quant_block128(const double* y, int64_t n, uint8_t* q, double* scales) {
 //   block    16 consecutive elements of a row share one unsigned e4m3 scale
 //            factor sf; with the per-tensor fp32 global scale gs,
 //            y ~ e2m1 * decode(sf) * gs.
-//   decision in fp32 (as every FP8 decision here), scaling by correctly
-//            rounded reciprocals as NVFP4 quantisers do: with y32 the fp32
-//            values and amax32 = max |y32| over the block,
-//              rden = fp32(1 / fp32(6 * gs)),
-//              sf   = e4m3(fp32(amax32 * rden))   (RNE, saturating to 448),
-//              eff  = fp32(decode(sf) * gs),  reff = fp32(1 / eff),
-//              code = e2m1(fp32(y32 * reff));
-//            sf == 0 (an all-zero or negligible block) gives all-zero codes.
+//   decision the nearest code to an exact quotient, taken on that quotient
+//            rounded once to fp32 (the precision every FP8 decision here is
+//            taken in): with y32 the fp32 values and amax32 = max |y32| over
+//            the block,
+//              sf   = e4m3(fp32(amax32 / (6 gs)))          (RNE, saturating to 448),
+//              code = e2m1(fp32(y32 / (decode(sf) gs)))  (RNE, saturating to 6);
+//            6 gs and decode(sf) gs are exact in fp64 (at most 28 significant
+//            bits), and an fp64 quotient of fp32 operands rounded to fp32 is
+//            the correctly rounded fp32 quotient (double rounding is
+//            innocuous for division when 53 >= 2 * 24 + 2).  sf == 0 (an
+//            all-zero or negligible block) gives all-zero codes.
 uint8_t e2m1_encode(double v) {
   const uint8_t s = std::signbit(v) ? 0x8 : 0x0;
   const double a = std::fabs(v);
@@ -242,7 +245,7 @@ double e2m1_decode(uint8_t c) {
 // One row of n (a multiple of 16) values -> n/2 packed bytes and n/16 scale
 // factors (row-major).
 void quant_nvfp4_row(const double* y, int64_t n, float gs, uint8_t* packed, uint8_t* sf) {
-  const float rden = 1.0f / (6.0f * gs);
+  const double den = 6.0 * (double)gs;  // exact
   for (int64_t b = 0; b < n / 16; ++b) {
     float y32[16];
     float amax = 0.0f;
@@ -250,12 +253,11 @@ void quant_nvfp4_row(const double* y, int64_t n, float gs, uint8_t* packed, uint
       y32[j] = (float)y[16 * b + j];
       amax = std::fmax(amax, std::fabs(y32[j]));
     }
-    const uint8_t code_sf = e4m3_encode((double)(amax * rden));
+    const uint8_t code_sf = e4m3_encode((double)(float)((double)amax / den));
     sf[b] = code_sf;
-    const float eff = (float)e4m3_decode(code_sf) * gs;
-    const float reff = (eff > 0.0f) ? 1.0f / eff : 0.0f;
+    const double eff = e4m3_decode(code_sf) * (double)gs;  // exact
     uint8_t q[16];
-    for (int j = 0; j < 16; ++j) q[j] = (eff > 0.0f) ? e2m1_encode((double)(y32[j] * reff)) : 0;
+    for (int j = 0; j < 16; ++j) q[j] = (eff > 0.0) ? e2m1_encode((double)(float)((double)y32[j] / eff)) : 0;
     for (int j = 0; j < 8; ++j) packed[8 * b + j] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
   }
 }

@@ -5,6 +5,8 @@ fusion", §三, gate_res_adarms_fp8_static): reduction to op (a) when the gate i
 one and the modulation zero, a zero gate, a closed form on constant rows, the
 condition-row mapping, and the brute-force rational restatement on 4 x 8."""
 import math
+import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -225,29 +227,46 @@ def test_e2m1_ties_to_even_and_saturation():
     assert oracle.e2m1_encode(6.0) == 7 and oracle.e2m1_encode(1e30) == 7 and oracle.e2m1_encode(-7.5) == 15
 
 
+def _round_f32(q):
+    """The fp32 value nearest the rational q (ties to the even significand),
+    by brute force over the fp32 neighbours of a first guess, with exact
+    rational distances."""
+    f = np.float32(float(q))
+    cands = {f, np.nextafter(f, np.float32(np.inf)), np.nextafter(f, np.float32(-np.inf))}
+    cands = [c for c in cands if np.isfinite(c)]
+    best = min(abs(Fraction(float(c)) - q) for c in cands)
+    near = [c for c in cands if abs(Fraction(float(c)) - q) == best]
+    if len(near) > 1:
+        near = [c for c in near if (int(np.array(c, dtype=np.float32).view(np.uint32)) & 1) == 0]
+    return float(near[0])
+
+
 def _nvfp4_brute(y, gs):
-    """The NVFP4 reading restated with numpy fp32 scalars (scaling by correctly
-    rounded reciprocals) and brute-force nearest-code searches (e4m3 via the
-    whole code table, e2m1 over its 8 magnitudes, ties to the even code)."""
+    """The NVFP4 reading restated with exact rational quotients: the block
+    scale is the e4m3 code nearest fp32(amax / (6 gs)) and each element the
+    e2m1 code nearest fp32(y / (sf gs)), every quotient exact and then rounded
+    once to fp32 (found by brute force), nearest codes found by searching the
+    whole e4m3 table and the 8 e2m1 magnitudes (ties to the even code)."""
     y32 = np.asarray(y, dtype=np.float32)
+    g = Fraction(float(np.float32(gs)))
     packed, sfs = [], []
     for b in range(len(y32) // 16):
         blk = y32[16 * b:16 * b + 16]
-        amax = np.float32(np.max(np.abs(blk)))
-        rden = np.float32(np.float32(1.0) / (np.float32(6.0) * np.float32(gs)))
-        sf = int(_nearest_e4m3(np.array([float(np.float32(amax * rden))]))[0])
-        eff = np.float32(np.float32(oracle.e4m3_decode(sf)) * np.float32(gs))
+        amax = Fraction(float(np.max(np.abs(blk))))
+        sf = int(_nearest_e4m3(np.array([_round_f32(amax / (6 * g))]))[0])
+        eff = Fraction(oracle.e4m3_decode(sf)) * g
         codes = []
         for v in blk:
             if eff == 0:
                 codes.append(0)
                 continue
-            t = float(np.float32(v * np.float32(np.float32(1.0) / eff)))
+            t = _round_f32(Fraction(float(v)) / eff)
             a = min(abs(t), 6.0)
             d = [abs(m - a) for m in E2M1]
             best = [k for k in range(8) if d[k] == min(d)]
             k = [k for k in best if k % 2 == 0][0] if len(best) > 1 else best[0]
-            codes.append(k | (8 if math.copysign(1.0, t) < 0 else 0))
+            codes.append(k | (8 if math.copysign(1.0, t) < 0 or (t == 0 and math.copysign(1.0, float(v)) < 0)
+                              else 0))
         sfs.append(sf)
         packed += [codes[2 * j] | (codes[2 * j + 1] << 4) for j in range(8)]
     return np.array(packed, dtype=np.uint8), np.array(sfs, dtype=np.uint8)
@@ -264,6 +283,70 @@ def test_nvfp4_row_matches_brute_force(gs):
     np.testing.assert_array_equal(sf, bsf)
     np.testing.assert_array_equal(packed, bp)
     assert sf[2] == 0 and (packed[16:24] == 0).all()
+
+
+def _e2m1_nearest(t):
+    a = min(abs(t), 6.0)
+    d = [abs(m - a) for m in E2M1]
+    best = [k for k in range(8) if d[k] == min(d)]
+    return [k for k in best if k % 2 == 0][0] if len(best) > 1 else best[0]
+
+
+def _reciprocal_form_codes(blk, gs):
+    """Scaling by rounded reciprocals instead of quotients (a plausible
+    alternative the oracle must not be): sf = e4m3(RN(amax RN(1/RN(6 gs)))),
+    code = e2m1(RN(y RN(1/RN(sf gs)))), in numpy fp32."""
+    gs = np.float32(gs)
+    blk = np.asarray(blk, dtype=np.float32)
+    rden = np.float32(np.float32(1.0) / (np.float32(6.0) * gs))
+    sf = int(oracle.e4m3_encode(float(np.float32(np.max(np.abs(blk)) * rden))))
+    eff = np.float32(np.float32(oracle.e4m3_decode(sf)) * gs)
+    reff = np.float32(np.float32(1.0) / eff)
+    return sf, [_e2m1_nearest(float(np.float32(v * reff))) for v in blk]
+
+
+def _neighbours(v, n):
+    out, a, b = [np.float32(v)], np.float32(v), np.float32(v)
+    for _ in range(n):
+        a, b = np.nextafter(a, np.float32(np.inf)), np.nextafter(b, np.float32(-np.inf))
+        out += [a, b]
+    return out
+
+
+@pytest.mark.parametrize("gs", [1.0 / 3.0, 0.0123])
+def test_nvfp4_decisions_are_quotients_not_reciprocal_products(gs):
+    """Blocks built so that scaling by rounded reciprocals decides a different
+    scale factor or element code than the quotient definition: the oracle must
+    follow the definition (the exact-rational brute force) on every one."""
+    g32 = Fraction(float(np.float32(gs)))
+    blocks = []
+    # element codes: amax fixes sf; the other values sit next to e2m1 midpoints
+    for sf_code in (0x38, 0x3B, 0x45):
+        eff = Fraction(oracle.e4m3_decode(sf_code)) * g32
+        amax = np.float32(float(6 * eff))
+        for m in (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0):
+            for v in _neighbours(float(m * eff), 12):
+                blk = np.zeros(16, dtype=np.float32)
+                blk[0], blk[1], blk[2] = amax, v, -v
+                sf_r, codes_r = _reciprocal_form_codes(blk, gs)
+                t = _round_f32(Fraction(float(v)) / (Fraction(oracle.e4m3_decode(sf_r)) * g32))
+                if sf_r == sf_code and codes_r[1] != _e2m1_nearest(t):
+                    blocks.append(blk)
+    # scale factors: amax next to (e4m3 midpoint) * 6 gs
+    for c in range(0x10, 0x70, 5):
+        mid = (Fraction(oracle.e4m3_decode(c)) + Fraction(oracle.e4m3_decode(c + 1))) / 2
+        for a in _neighbours(float(mid * 6 * g32), 6):
+            want = int(_nearest_e4m3(np.array([_round_f32(Fraction(float(a)) / (6 * g32))]))[0])
+            blk = np.zeros(16, dtype=np.float32)
+            blk[0] = a
+            if _reciprocal_form_codes(blk, gs)[0] != want:
+                blocks.append(blk)
+    assert len(blocks) >= 8, "too few discriminating blocks (%d)" % len(blocks)
+    y = np.concatenate(blocks).astype(np.float64)
+    packed, sf = oracle.quant_nvfp4_row(y, gs)
+    bp, bsf = _nvfp4_brute(y, gs)
+    np.testing.assert_array_equal(sf, bsf)
+    np.testing.assert_array_equal(packed, bp)
 
 
 def test_nvfp4_exact_block_closed_form_and_nibble_order():
@@ -316,6 +399,52 @@ def test_nvfp4_ops_reuse_op_a_and_op_c():
     for i in range(2):
         p, s = oracle.quant_nvfp4_row(c["a"][i], 0.003)
         np.testing.assert_array_equal(c["out_fp4"][i], p)
+
+
+def _torch_to_blocked():
+    """PyTorch's to_blocked (and its ceil_div) taken from the installed
+    torch/testing/_internal/common_quantized.py source: the module itself
+    imports test-only packages this image lacks, so the two functions are
+    compiled alone from their source text, unchanged."""
+    import ast
+    import importlib.util
+    path = os.path.join(os.path.dirname(importlib.util.find_spec("torch").origin), "testing", "_internal",
+                        "common_quantized.py")
+    with open(path) as f:
+        tree = ast.parse(f.read())
+    fns = [n for n in tree.body if isinstance(n, ast.FunctionDef) and n.name in ("ceil_div", "to_blocked")]
+    assert sorted(n.name for n in fns) == ["ceil_div", "to_blocked"]
+    ns = {"torch": torch}
+    exec(compile(ast.Module(body=fns, type_ignores=[]), path, "exec"), ns)
+    return ns["to_blocked"]
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 1), (128, 4), (130, 10), (300, 7), (256, 64), (77, 256)])
+def test_sf_swizzle_matches_torch_to_blocked(rows, cols):
+    """The swizzled scale-factor layout pinned to an implementation outside
+    this repository: PyTorch's own test helper for block-scaled matmul,
+    torch.testing._internal.common_quantized.to_blocked, which rearranges an
+    [rows, cols] scale matrix into the cuBLAS 1-D block-scaling-factor layout
+    (128 x 4 tiles of 512 bytes).  Position p of its flattened output holds
+    element (r, c) exactly when the oracle's offset of (r, c) is p; a
+    transposed reading (4 k + 16 i) or a column-major tile order fails."""
+    to_blocked = _torch_to_blocked()
+    idx = torch.arange(1, rows * cols + 1, dtype=torch.int64).reshape(rows, cols)
+    flat = to_blocked(idx).numpy()
+    n_cols = cols
+    assert flat.size == ((rows + 127) // 128) * 128 * ((cols + 3) // 4) * 4
+    seen = 0
+    for p in np.flatnonzero(flat):
+        r, c = divmod(int(flat[p]) - 1, cols)
+        assert oracle.sf_swizzle_offset(r, c, n_cols) == p, (r, c, p)
+        seen += 1
+    assert seen == rows * cols
+    # and the oracle's whole-matrix helper places every element the same way
+    sf = (np.arange(rows * cols, dtype=np.int64) % 251 + 1).astype(np.uint8).reshape(rows, cols)
+    want = to_blocked(torch.from_numpy(sf.astype(np.int64))).numpy().astype(np.uint8)
+    got = oracle.sf_swizzle(sf)
+    written = want != 0
+    np.testing.assert_array_equal(got[written], want[written])
 
 
 def test_sf_swizzle_layout():
