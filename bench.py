@@ -871,6 +871,8 @@ def reference_arm(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "io_dtypes": {"in": wl.dt, "out": "e4m3", "residual": wl.dt,
+                          "arithmetic": "fp64 (FP8 decisions on fp32 quotients)"},
             "data": "synthetic (seeded torch.Generator('cpu'))",
             "config": {"workload": wl.name, "M": wl.M, "D": wl.D, "Hq": wl.Hq, "Hkv": wl.Hkv, "hd": wl.hd,
                        "I": wl.I, "act": wl.act, "quant": wl.quant, "sample_rows_per_step": rows},
@@ -993,6 +995,8 @@ def main(argv=None):
         line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "io_dtypes": {"in": wl.dt, "out": "e4m3", "residual": wl.dt,
+                              "arithmetic": "fp32, fp64 row sums of squares"},
                 "data": "synthetic: seeded torch.Generator('cpu'), N(0,1) activations, 1+0.1N norm weights",
                 "config": {"workload": wl.name, "M": wl.M, "D": wl.D, "Hq": wl.Hq, "Hkv": wl.Hkv, "hd": wl.hd,
                            "I": wl.I, "act": wl.act, "quant": wl.quant, "io": "bf16 in, e4m3 out",

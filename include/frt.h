@@ -166,13 +166,16 @@ frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residual_in, void
  *                              >= capacity; that row is skipped entirely (no
  *                              Q, K or V write);
  *                       bit 1  a kernel gave up waiting for its own bulk copy
- *                              (a bounded wait ran out; only a failing device
- *                              can cause it); that token's outputs are not
+ *                              (a bounded wait ran out: only a failing device,
+ *                              or a bound lowered by frt_set_wait_polls, can
+ *                              cause it); that token's outputs are not
  *                              written.
- *   16-bit pointers must be 16-byte aligned when hd % 16 == 0 and 8-byte
- *   aligned otherwise.
+ *   16-bit pointers must be 16-byte aligned when hd % 16 == 0, 8-byte aligned
+ *   when hd % 8 == 0, and 2-byte aligned otherwise (a head dim that no vector
+ *   width divides, e.g. 66 or 100, runs an element-wise kernel); cos_tab and
+ *   sin_tab 16-byte aligned when hd % 8 == 0, else 4-byte.
  *   Layout rule: Hq, Hkv > 0, Hq % Hkv == 0, hd > 0 and even, max_pos > 0,
- *   capacity > 0.  Unsupported: hd % 8 != 0 or hd > 256.
+ *   capacity > 0.  Unsupported: hd > 256.
  */
 frt_status frt_qkv_norm_rope_kvcache(const void* qkv, const void* q_norm_w, const void* k_norm_w,
                                      const float* cos_tab, const float* sin_tab, const int32_t* positions,
@@ -345,7 +348,7 @@ frt_status frt_gate_act_nvfp4(const void* gate_up, uint8_t* out_fp4, uint8_t* ou
  *   q_layout     FRT_Q_TOKEN_MAJOR or FRT_Q_HEAD_MAJOR.
  *   kv_format    FRT_KV_16BIT (caches as op (b)) or FRT_KV_E4M3 (caches
  *                [capacity, Hkv, hd] uint8, 8-byte aligned when hd % 16 == 0,
- *                4-byte aligned otherwise).
+ *                4-byte aligned when hd % 8 == 0, unaligned otherwise).
  *   kv_scales    device fp32[2] = {k_scale, v_scale}, read with E4M3 only
  *                (may be NULL with 16BIT).
  *   Errors: as op (b); also FRT_ERR_INVALID_ARG for an unknown layout or
@@ -402,12 +405,35 @@ frt_status frt_noop(int grid, int block, cudaStream_t stream);
  * the GPU may schedule it while the previous kernel of the same stream is
  * still running (hiding launch latency, e.g. between the nodes of a CUDA
  * graph), and the kernel waits for that previous kernel to complete, with its
- * writes visible, before it touches memory (griddepcontrol.wait).  Results are
- * identical either way.  The switch is process-wide and read at each launch;
- * changing it while another thread launches affects only later launches.
+ * writes visible (griddepcontrol.wait), before it reads its data inputs (x,
+ * residual, qkv, gate_up, the AdaRMSNorm condition rows) or writes anything.
+ * Its constant inputs -- norm weights, RoPE tables, positions and the scale
+ * inputs (static_scale, kv_scales, global_scale) -- are read before that
+ * wait, so they must not be written by the kernel launched just before it on
+ * the same stream (no kernel of this library writes them; a host copy or a
+ * kernel further back is fine: a kernel is scheduled early only once every
+ * CTA of its predecessor has passed its own wait).  Results are identical
+ * either way.  The switch is process-wide and read at each launch; changing
+ * it while another thread launches affects only later launches.
  */
 void frt_set_pdl(int enable);
 int frt_get_pdl(void);
+
+/*
+ * Bound on the polls of the bulk-copy barrier wait of the QKV ops' large-batch
+ * kernel (frt_qkv_norm_rope_kvcache and its NEXT-2 / LayerNorm forms, M >=
+ * 592 with 16-byte rows).  That kernel's CTA waits for its token's row to land
+ * in shared memory; a wait that runs out of polls sets bit 1 of the op's
+ * status word, writes none of the token's outputs, waits once more (with the
+ * default bound, whatever this setting) for the copies it issued to land, and
+ * returns.  Only a failing device makes the default bound run out; a bound of
+ * 0 gives up at once on every token, which lets a test check that path.
+ * Process-wide, read at each launch, like frt_set_pdl.
+ * Returns FRT_ERR_INVALID_ARG for polls < 0.
+ */
+#define FRT_DEFAULT_WAIT_POLLS (1 << 22)
+frt_status frt_set_wait_polls(int polls);
+int frt_get_wait_polls(void);
 
 /* Static, NUL-terminated description of a status value; never NULL. */
 const char* frt_status_string(frt_status status);

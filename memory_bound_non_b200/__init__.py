@@ -31,7 +31,8 @@ EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_ac
            "frt_chain_persistent", "frt_residual_layernorm_fp8", "frt_residual_layernorm_nvfp4",
            "frt_qkv_layernorm_rope_kvcache",
            "frt_residual_rmsnorm_nvfp4", "frt_gate_act_nvfp4", "frt_qkv_norm_rope_prepq_kvcache",
-           "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_status_string")
+           "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_set_wait_polls",
+           "frt_get_wait_polls", "frt_status_string")
 
 
 class FrtError(RuntimeError):
@@ -81,6 +82,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_set_pdl.restype = None
     L.frt_get_pdl.argtypes = []
     L.frt_get_pdl.restype = i32
+    L.frt_set_wait_polls.argtypes = [i32]
+    L.frt_set_wait_polls.restype = i32
+    L.frt_get_wait_polls.argtypes = []
+    L.frt_get_wait_polls.restype = i32
     L.frt_status_string.argtypes = [i32]
     L.frt_status_string.restype = c.c_char_p
     _lib = L
@@ -281,6 +286,19 @@ def frt_set_pdl(enable: bool):
 
 def frt_get_pdl() -> bool:
     return bool(load().frt_get_pdl())
+
+
+FRT_DEFAULT_WAIT_POLLS = 1 << 22
+
+
+def frt_set_wait_polls(polls: int):
+    """Bound on the polls of the QKV ops' bulk-copy barrier wait (process-wide;
+    FRT_DEFAULT_WAIT_POLLS restores the default; 0 gives up at once)."""
+    _check("frt_set_wait_polls", load().frt_set_wait_polls(int(polls)))
+
+
+def frt_get_wait_polls() -> int:
+    return int(load().frt_get_wait_polls())
 
 
 def frt_noop(grid=1, block=32, stream=None):

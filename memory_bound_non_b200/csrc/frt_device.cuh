@@ -13,9 +13,14 @@
 namespace frt {
 
 // ------------------------------------------------------------------ PDL --
-// Every kernel starts with these two: wait until the grid this launch depends
-// on has completed and its writes are visible (a no-op without a programmatic
+// Every kernel calls this before it touches any memory that the previous
+// kernel of the stream may write: wait until the grid this launch depends on
+// has completed and its writes are visible (a no-op without a programmatic
 // dependency), then let the next launch of the stream be scheduled early.
+// Loads of constant inputs (norm weights, RoPE tables, positions, scales)
+// may come before it: the next kernel is launched only once every CTA of this
+// one has passed the wait, so those early loads overlap the previous kernel
+// alone, which never writes them.
 __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" :::);

@@ -23,6 +23,10 @@ inline frt_status launch_status() { return cudaGetLastError() == cudaSuccess ? F
 // Process-wide switch for programmatic dependent launch (frt_set_pdl).
 bool pdl_enabled();
 
+// Process-wide bound on the polls of a kernel's bulk-copy barrier wait
+// (frt_set_wait_polls).
+int wait_polls();
+
 // Launch `kernel` on `stream`, with programmatic stream serialisation when
 // PDL is on: the kernel may then be scheduled while the previous kernel of the
 // stream still runs, and waits for it (griddepcontrol.wait) before its first

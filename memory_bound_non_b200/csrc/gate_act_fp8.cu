@@ -40,6 +40,14 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
                                                                  const float* __restrict__ static_scale,
                                                                  float* __restrict__ block_scales,
                                                                  int64_t total_blocks, int NB, int C4) {
+  // Constant inputs before the wait for the previous kernel: static FP8 the
+  // scale; NVFP4 the global scale gs, RN(1 / RN(6 gs)) and RN(1 / RN(sf * gs))
+  // for each of the 256 sf codes (one per thread).
+  const float gs = QM >= kQuantNvfp4Rows ? __ldg(static_scale) : 0.0f;
+  const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * gs) : 0.0f;
+  const Divisor dv_static(QM == FRT_QUANT_STATIC ? __ldg(static_scale) : 1.0f);
+  __shared__ float reff_of[QM >= kQuantNvfp4Rows ? kThreads : 1];
+  if (QM >= kQuantNvfp4Rows) reff_of[threadIdx.x] = nvfp4_reff_entry(threadIdx.x, gs);
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -76,17 +84,7 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
     }
   }
 
-  // static FP8: the scale; NVFP4: the global scale gs and RN(1 / RN(6 gs))
-  const float gs = QM >= kQuantNvfp4Rows ? __ldg(static_scale) : 0.0f;
-  const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * gs) : 0.0f;
-  const Divisor dv_static(QM == FRT_QUANT_STATIC ? __ldg(static_scale) : 1.0f);
-  // NVFP4: RN(1 / RN(sf * gs)) for each of the 256 sf codes, one per thread,
-  // formed while the loads above are in flight
-  __shared__ float reff_of[QM >= kQuantNvfp4Rows ? kThreads : 1];
-  if (QM >= kQuantNvfp4Rows) {
-    reff_of[threadIdx.x] = nvfp4_reff_entry(threadIdx.x, gs);
-    __syncthreads();
-  }
+  if (QM >= kQuantNvfp4Rows) __syncthreads();  // the reciprocal table is complete
 
 #pragma unroll
   for (int u = 0; u < kU; ++u) {

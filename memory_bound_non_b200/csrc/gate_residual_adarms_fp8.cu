@@ -61,6 +61,11 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
   // The gate rides in registers with x and the residual; at the widest rows
   // (K = 8) registers run out and it is staged in shared memory instead.
   constexpr bool kGateSmem = K >= 8;
+  // the static scale is a constant input: read before the wait for the
+  // previous kernel (the gate, scale and shift rows are computed per step by
+  // a preceding kernel, so they wait)
+  float s_static = 0.0f;
+  if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
   pdl_enter();
   const int t = threadIdx.x;
   const int T = blockDim.x;
@@ -102,8 +107,6 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
     }
     cp_async_commit();
   }
-  float s_static = 0.0f;
-  if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
   if (GATED && kGateSmem) {
     if (MOD) cp_async_wait<1>();  // the gate group; scale / shift may still be in flight
     else cp_async_wait<0>();

@@ -157,7 +157,6 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
   using V = typename Vec16<P>::T;
   constexpr bool QEPI = EPI >= 1;
   constexpr bool KV8 = EPI == 2;
-  pdl_enter();
   const int tok = blockIdx.x / nhb;
   const int hb = blockIdx.x - tok * nhb;
   const int grp = (int)(threadIdx.x / GP);
@@ -165,18 +164,15 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
   const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G;
   const int half = hd >> 1;
   const int j0 = li * P;
-  const uint16_t* row = qkv + (int64_t)tok * H * hd;
-  // The QKV vectors and the norm weights do not depend on the position: load
-  // them alongside it, so only the cos/sin rows wait for the position.
-  V va[HPG], vb[HPG];
-#pragma unroll
-  for (int i = 0; i < HPG; ++i) {
-    const int h = (hb * hpg + i) * NG + grp;
-    if (lane_ok && i < hpg && h < H) {
-      va[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + j0);
-      vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
-    }
-  }
+  // Constant inputs before the wait for the previous kernel: the position,
+  // the lane's cos/sin slice at that position (two dependent loads, off the
+  // critical path this way), the norm weights and the e4m3 cache scales.
+  const int p = __ldg(positions + tok);
+  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
+  const bool active = lane_ok && row_ok;
+  constexpr int NP = P / 2;
+  float2 cs[NP], sn[NP], nsn[NP];
+  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
   V qwa, qwb, kwa, kwb;
   if (HPG == 1 && lane_ok) {
     if (q_norm_w != nullptr) {
@@ -188,16 +184,21 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
       kwb = ld_vec<P>(k_norm_w + half + j0);
     }
   }
-  const int p = __ldg(positions + tok);
-  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
-  if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
-  const bool active = lane_ok && row_ok;
-  constexpr int NP = P / 2;
-  float2 cs[NP], sn[NP], nsn[NP];
-  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
-  const float inv_hd = 1.0f / (float)hd;
   const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
   const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
+  pdl_enter();
+  const uint16_t* row = qkv + (int64_t)tok * H * hd;
+  V va[HPG], vb[HPG];
+#pragma unroll
+  for (int i = 0; i < HPG; ++i) {
+    const int h = (hb * hpg + i) * NG + grp;
+    if (lane_ok && i < hpg && h < H) {
+      va[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + j0);
+      vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
+    }
+  }
+  if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
+  const float inv_hd = 1.0f / (float)hd;
 #pragma unroll
   for (int i = 0; i < HPG; ++i) {
     if (i >= hpg) break;  // uniform across the CTA
@@ -435,7 +436,6 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
     uint16_t* __restrict__ k_cache, uint16_t* __restrict__ v_cache, int32_t* status, int H, int NG, int nhb, int Hq,
     int Hkv, int hd, int G, int max_pos, int capacity, float eps) {
   using V = typename Vec16<P>::T;
-  pdl_enter();
   const int tok = blockIdx.x / nhb;
   const int hb = blockIdx.x - tok * nhb;
   const int grp = (int)(threadIdx.x / GP);
@@ -443,6 +443,15 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
   const int half = hd >> 1;
   const int j0 = li * P;
   const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G;
+  // the position and the lane's cos/sin slice are constant inputs: read
+  // before the wait for the previous kernel
+  const int p = __ldg(positions + tok);
+  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
+  const bool active = lane_ok && row_ok;
+  constexpr int NP = P / 2;
+  float2 cs[NP], sn[NP], nsn[NP];
+  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
+  pdl_enter();
   const uint16_t* row = qkv + (int64_t)tok * H * hd;
   V va[HPG], vb[HPG];
 #pragma unroll
@@ -453,13 +462,7 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
       vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
     }
   }
-  const int p = __ldg(positions + tok);
-  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
   if (!row_ok && threadIdx.x == 0 && hb == 0 && status != nullptr) atomicOr(status, 1);
-  const bool active = lane_ok && row_ok;
-  constexpr int NP = P / 2;
-  float2 cs[NP], sn[NP], nsn[NP];
-  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
   const float inv_hd = 1.0f / (float)hd;
 #pragma unroll
   for (int i = 0; i < HPG; ++i) {
@@ -504,9 +507,187 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
   }
 }
 
-// Polls of a bulk-copy barrier before the kernel gives up (each poll may
-// suspend the thread for a while; the bound is far beyond any real copy).
-constexpr int kMaxPolls = 1 << 22;
+// Any even head_dim (hd % 8 != 0, e.g. 66 or 100, where no vector width fits
+// both halves of a head): one warp per (token, head) slot, lane l holding the
+// elements j = l, l + 32, ... (< hd/2) and their rotate-half partners
+// j + hd/2, read and written as single 16-bit elements (a 64-byte run per
+// warp access).  The arithmetic is the vector kernels', element by element:
+// the head's sum of squares (or mean and centred squares for LayerNorm) is a
+// warp reduction, then norm, RoPE, the Q epilogue and the cache stores.
+// EPI as the bulk-copy kernel (0 op (b), 1 Q epilogue, 2 + e4m3 caches, 3
+// per-head LayerNorm with affine rows [H, hd] and biases in ep).
+constexpr int kGenericMaxK = 4;  // hd / 2 <= 128 = 32 lanes x 4
+
+template <int DT>
+__device__ __forceinline__ float ld16(const uint16_t* p) {
+  const uint32_t u = *p;
+  return DT == FRT_BF16 ? __uint_as_float(u << 16) : __half2float(__ushort_as_half((unsigned short)u));
+}
+template <int DT>
+__device__ __forceinline__ void st16(uint16_t* p, float v) {
+  if (DT == FRT_BF16)
+    *p = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  else
+    *p = __half_as_ushort(__float2half_rn(v));
+}
+
+template <int DT, int EPI>
+__global__ void __launch_bounds__(512) qkv_generic_kernel(
+    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ q_w, const uint16_t* __restrict__ k_w,
+    const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, const int32_t* __restrict__ positions,
+    uint16_t* __restrict__ q_out, void* __restrict__ k_cache, void* __restrict__ v_cache, int32_t* status, int H,
+    int Hq, int Hkv, int hd, int max_pos, int capacity, float eps, Epilogue ep) {
+  constexpr bool QEPI = EPI == 1 || EPI == 2;
+  constexpr bool KV8 = EPI == 2;
+  constexpr bool LN = EPI == 3;
+  const int tok = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int half = hd >> 1;
+  // constant inputs before the wait for the previous kernel
+  const int p = __ldg(positions + tok);
+  const bool row_ok = p >= 0 && p < max_pos && p < capacity;
+  float cs[kGenericMaxK], sn[kGenericMaxK];
+#pragma unroll
+  for (int k = 0; k < kGenericMaxK; ++k) {
+    const int j = lane + 32 * k;
+    cs[k] = sn[k] = 0.0f;
+    if (row_ok && j < half) {
+      cs[k] = __ldg(cos_tab + (int64_t)p * half + j);
+      sn[k] = __ldg(sin_tab + (int64_t)p * half + j);
+    }
+  }
+  const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
+  const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
+  pdl_enter();
+  if (!row_ok) {
+    if (threadIdx.x == 0 && status != nullptr) atomicOr(status, 1);
+    return;
+  }
+  const float inv_hd = 1.0f / (float)hd;
+  const Divisor dk(k_scale), dv(v_scale);
+  const uint16_t* row = qkv + (int64_t)tok * H * hd;
+  for (int h = threadIdx.x >> 5; h < H; h += blockDim.x >> 5) {  // uniform per warp
+    const bool is_q = h < Hq;
+    const bool is_v = h >= Hq + Hkv;
+    const int hh = is_q ? h : is_v ? h - Hq - Hkv : h - Hq;  // head index within its section
+    float a[kGenericMaxK], b[kGenericMaxK];
+#pragma unroll
+    for (int k = 0; k < kGenericMaxK; ++k) {
+      const int j = lane + 32 * k;
+      a[k] = b[k] = 0.0f;
+      if (j < half) {
+        a[k] = ld16<DT>(row + (int64_t)h * hd + j);
+        b[k] = ld16<DT>(row + (int64_t)h * hd + half + j);
+      }
+    }
+    const int64_t cache_off = ((int64_t)p * Hkv + hh) * hd;
+    if (is_v) {
+#pragma unroll
+      for (int k = 0; k < kGenericMaxK; ++k) {
+        const int j = lane + 32 * k;
+        if (j >= half) continue;
+        if (KV8) {
+          uint8_t* dst = static_cast<uint8_t*>(v_cache) + cache_off;
+          dst[j] = (uint8_t)(e4m3x2(dv.fast ? dv.div(a[k]) : dv.div_slow(a[k]), 0.0f) & 0xFFu);
+          dst[half + j] = (uint8_t)(e4m3x2(dv.fast ? dv.div(b[k]) : dv.div_slow(b[k]), 0.0f) & 0xFFu);
+        } else {  // bit copy
+          uint16_t* dst = static_cast<uint16_t*>(v_cache) + cache_off;
+          dst[j] = row[(int64_t)h * hd + j];
+          dst[half + j] = row[(int64_t)h * hd + half + j];
+        }
+      }
+      continue;
+    }
+    const uint16_t* w = is_q ? q_w : k_w;
+    if (LN) {
+      const uint16_t* bias = is_q ? ep.q_bias : ep.k_bias;
+      float acc = 0.0f;
+#pragma unroll
+      for (int k = 0; k < kGenericMaxK; ++k) acc += a[k] + b[k];
+      const float mean = group_sum<32>(acc) * inv_hd;
+      float acc2 = 0.0f;
+#pragma unroll
+      for (int k = 0; k < kGenericMaxK; ++k) {
+        if (lane + 32 * k < half) {
+          a[k] -= mean;
+          b[k] -= mean;
+          acc2 = fmaf(b[k], b[k], fmaf(a[k], a[k], acc2));
+        }
+      }
+      const float r = head_rstd(group_sum<32>(acc2), inv_hd, eps);
+#pragma unroll
+      for (int k = 0; k < kGenericMaxK; ++k) {
+        const int j = lane + 32 * k;
+        if (j >= half) continue;
+        const int64_t o = (int64_t)hh * hd;
+        const float w1 = w ? ld16<DT>(w + o + j) : 1.0f, w2 = w ? ld16<DT>(w + o + half + j) : 1.0f;
+        const float b1 = bias ? ld16<DT>(bias + o + j) : 0.0f, b2 = bias ? ld16<DT>(bias + o + half + j) : 0.0f;
+        a[k] = fmaf(a[k] * r, w1, b1);
+        b[k] = fmaf(b[k] * r, w2, b2);
+      }
+    } else if (w != nullptr) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int k = 0; k < kGenericMaxK; ++k) acc = fmaf(b[k], b[k], fmaf(a[k], a[k], acc));
+      const float r = head_rstd(group_sum<32>(acc), inv_hd, eps);
+#pragma unroll
+      for (int k = 0; k < kGenericMaxK; ++k) {
+        const int j = lane + 32 * k;
+        if (j >= half) continue;
+        a[k] = (a[k] * r) * ld16<DT>(w + j);
+        b[k] = (b[k] * r) * ld16<DT>(w + half + j);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kGenericMaxK; ++k) {
+      const int j = lane + 32 * k;
+      if (j >= half) continue;
+      float o1 = fmaf(a[k], cs[k], b[k] * -sn[k]);
+      float o2 = fmaf(b[k], cs[k], a[k] * sn[k]);
+      if (is_q) {
+        if (QEPI) {
+          o1 *= ep.q_scale;
+          o2 *= ep.q_scale;
+        }
+        uint16_t* dst = q_out + (QEPI ? q_row(ep, tok, h, Hq) : (int64_t)tok * Hq + h) * hd;
+        st16<DT>(dst + j, o1);
+        st16<DT>(dst + half + j, o2);
+      } else if (KV8) {
+        uint8_t* dst = static_cast<uint8_t*>(k_cache) + cache_off;
+        dst[j] = (uint8_t)(e4m3x2(dk.fast ? dk.div(o1) : dk.div_slow(o1), 0.0f) & 0xFFu);
+        dst[half + j] = (uint8_t)(e4m3x2(dk.fast ? dk.div(o2) : dk.div_slow(o2), 0.0f) & 0xFFu);
+      } else {
+        uint16_t* dst = static_cast<uint16_t*>(k_cache) + cache_off;
+        st16<DT>(dst + j, o1);
+        st16<DT>(dst + half + j, o2);
+      }
+    }
+  }
+}
+
+template <int DT>
+frt_status launch_generic(int epi, const uint16_t* qkv, const uint16_t* qw, const uint16_t* kw, const float* c,
+                          const float* sn, const int32_t* pos, uint16_t* qo, void* kc, void* vc, int32_t* status,
+                          int M, int H, int Hq, int Hkv, int hd, int max_pos, int capacity, float eps,
+                          const Epilogue& ep, cudaStream_t st) {
+  const int warps = H < 16 ? H : 16;
+  const dim3 grid((unsigned)M), block((unsigned)(32 * warps));
+  switch (epi) {
+    case 0: return launch(qkv_generic_kernel<DT, 0>, grid, block, 0, st, qkv, qw, kw, c, sn, pos, qo, kc, vc, status,
+                          H, Hq, Hkv, hd, max_pos, capacity, eps, ep);
+    case 1: return launch(qkv_generic_kernel<DT, 1>, grid, block, 0, st, qkv, qw, kw, c, sn, pos, qo, kc, vc, status,
+                          H, Hq, Hkv, hd, max_pos, capacity, eps, ep);
+    case 2: return launch(qkv_generic_kernel<DT, 2>, grid, block, 0, st, qkv, qw, kw, c, sn, pos, qo, kc, vc, status,
+                          H, Hq, Hkv, hd, max_pos, capacity, eps, ep);
+    default: return launch(qkv_generic_kernel<DT, 3>, grid, block, 0, st, qkv, qw, kw, c, sn, pos, qo, kc, vc,
+                           status, H, Hq, Hkv, hd, max_pos, capacity, eps, ep);
+  }
+}
+
+// Polls of the drain wait that follows a give-up (each poll may suspend the
+// thread for a while; the bound is far beyond any real copy).  The first
+// wait's bound is the process-wide limit of frt_set_wait_polls.
+constexpr int kDrainPolls = 1 << 22;
 
 // Bulk-copy kernel (large batches).  One CTA per token.  One thread moves the
 // token's whole QKV row, its cos/sin rows and both norm weights into shared
@@ -514,8 +695,10 @@ constexpr int kMaxPolls = 1 << 22;
 // holds in-flight data and a small CTA keeps 12+ KB per token in flight.  Lane
 // groups (GP lanes per head) normalise and rotate the Q and K heads in place;
 // then the Q row, the K row and the untouched V row leave as three bulk
-// stores.  A barrier wait that runs out of polls sets bit 1 of *status and the
-// CTA returns without writing.
+// stores.  A barrier wait that runs out of polls (max_polls) sets bit 1 of
+// *status; the CTA then writes nothing, waits again (kDrainPolls) for the
+// copies it issued to land, so that none is still writing into its shared
+// memory when it exits, and returns.
 // EPI: 0 = op (b) as is (Q token-major, unscaled; 16-bit caches), 1 = Q
 // epilogue (scale, layout), 2 = Q epilogue + e4m3 caches, 3 = per-head
 // LayerNorm in place of the RMSNorm (affine rows read from global memory,
@@ -536,7 +719,7 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
     const uint16_t* __restrict__ k_norm_w, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
     const int32_t* __restrict__ positions, uint16_t* __restrict__ q_out, void* __restrict__ k_cache,
     void* __restrict__ v_cache, int32_t* status, int H, int NG, int Hq, int Hkv, int hd, int G, int max_pos,
-    int capacity, float eps, Epilogue ep) {
+    int capacity, float eps, Epilogue ep, int max_polls) {
   pdl_enter();
   // [QKV row][cos][sin][q weight][k weight][-sin] (+ [K codes][V codes] with EPI 2)
   extern __shared__ __align__(128) uint8_t dsmem[];
@@ -590,10 +773,14 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
       mbar_arrive_expect_tx(&bar, 0u);
     }
   }
-  const bool landed = mbar_wait_bounded(&bar, 0, kMaxPolls);
+  const bool landed = mbar_wait_bounded(&bar, 0, max_polls);
   if (!__syncthreads_and(landed)) {
     if (tid == 0 && status != nullptr) atomicOr(status, 2);
-    mbar_wait_bounded(&bar, 0, kMaxPolls);  // give copies still in flight a last chance to land
+    // Write nothing; drain: every copy above was issued with a byte count the
+    // barrier expects, so its phase completes once they have landed.  Only a
+    // device whose copies never complete runs this wait out too, and then
+    // the CTA exits with them outstanding.
+    mbar_wait_bounded(&bar, 0, kDrainPolls);
     return;
   }
   const int p = s_pos;
@@ -690,7 +877,8 @@ frt_status launch_gp(const Args& a, bool tma, cudaStream_t st) {
     if (NG < 1) NG = 1;
     const int threads = ((NG * GP + 31) / 32) * 32;
     return launch(kt, dim3((unsigned)a.M), dim3(threads), smem, st, qkv, qw, kw, a.cos_tab, a.sin_tab, a.pos, qo,
-                  a.kc, a.vc, a.status, a.H, NG, a.Hq, a.Hkv, a.hd, a.G, a.max_pos, a.capacity, a.eps, a.ep);
+                  a.kc, a.vc, a.status, a.H, NG, a.Hq, a.Hkv, a.hd, a.G, a.max_pos, a.capacity, a.eps, a.ep,
+                  wait_polls());
   }
   const Shape sh = qkv_shape(a.M, a.H, GP, KV8);
   const dim3 grid((unsigned)((int64_t)a.M * sh.nhb));
@@ -744,7 +932,7 @@ frt_status launch_ln_gp(const Args& a, cudaStream_t st) {
   return launch(kt, dim3((unsigned)a.M), dim3(threads), smem, st, static_cast<const uint16_t*>(a.qkv),
                 static_cast<const uint16_t*>(a.qw), static_cast<const uint16_t*>(a.kw), a.cos_tab, a.sin_tab, a.pos,
                 static_cast<uint16_t*>(a.q_out), a.kc, a.vc, a.status, a.H, NG, a.Hq, a.Hkv, a.hd, a.G, a.max_pos,
-                a.capacity, a.eps, a.ep);
+                a.capacity, a.eps, a.ep, wait_polls());
 }
 
 template <int DT>
@@ -770,11 +958,29 @@ frt_status qkv_op(const void* qkv, const void* q_norm_w, const void* k_norm_w, c
   if (q_layout != FRT_Q_TOKEN_MAJOR && q_layout != FRT_Q_HEAD_MAJOR) return FRT_ERR_INVALID_ARG;
   if (kv_format != FRT_KV_16BIT && kv_format != FRT_KV_E4M3) return FRT_ERR_INVALID_ARG;
   if (!std::isfinite(q_scale)) return FRT_ERR_INVALID_ARG;
-  if (hd % 8 != 0 || hd > 256) return FRT_ERR_UNSUPPORTED;
+  if (hd > 256) return FRT_ERR_UNSUPPORTED;
   if (M == 0) return FRT_OK;
   if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
   const bool kv8 = kv_format == FRT_KV_E4M3;
   if (kv8 && (!kv_scales || !aligned(kv_scales, 4))) return FRT_ERR_INVALID_ARG;
+  const int epi = kv8 ? 2 : (q_scale != 1.0f || q_layout != FRT_Q_TOKEN_MAJOR) ? 1 : 0;
+  if (hd % 8 != 0) {  // element-wise kernel: 16-bit pointers 2-byte aligned
+    if (!aligned(qkv, 2) || !aligned(q_out, 2) || (!kv8 && (!aligned(k_cache, 2) || !aligned(v_cache, 2))) ||
+        (q_norm_w && !aligned(q_norm_w, 2)) || (k_norm_w && !aligned(k_norm_w, 2)) || !aligned(cos_tab, 4) ||
+        !aligned(sin_tab, 4) || !aligned(positions, 4) || (status && !aligned(status, 4)))
+      return FRT_ERR_INVALID_ARG;
+    const Epilogue ep{q_scale, q_layout == FRT_Q_HEAD_MAJOR ? 1 : 0, M, kv_scales, nullptr, nullptr};
+    const int H = Hq + 2 * Hkv;
+    const auto* qk = static_cast<const uint16_t*>(qkv);
+    const auto* qw = static_cast<const uint16_t*>(q_norm_w);
+    const auto* kw = static_cast<const uint16_t*>(k_norm_w);
+    auto* qo = static_cast<uint16_t*>(q_out);
+    return dt == FRT_F16 ? launch_generic<FRT_F16>(epi, qk, qw, kw, cos_tab, sin_tab, positions, qo, k_cache, v_cache,
+                                                   status, M, H, Hq, Hkv, hd, max_pos, capacity, eps, ep, stream)
+                         : launch_generic<FRT_BF16>(epi, qk, qw, kw, cos_tab, sin_tab, positions, qo, k_cache,
+                                                    v_cache, status, M, H, Hq, Hkv, hd, max_pos, capacity, eps, ep,
+                                                    stream);
+  }
   const int P = (hd % 16 == 0) ? 8 : 4;
   const uintptr_t al = (P == 8) ? 16 : 8;
   const uintptr_t al_kv = kv8 ? (uintptr_t)P : al;  // e4m3 rows: P codes per lane store
@@ -798,7 +1004,6 @@ frt_status qkv_op(const void* qkv, const void* q_norm_w, const void* k_norm_w, c
                    aligned(v_cache, 16) && (!q_norm_w || aligned(q_norm_w, 16)) &&
                    (!k_norm_w || aligned(k_norm_w, 16)) && (!kv8 || (Hkv * hd) % 16 == 0) &&
                    tma_smem(H, Hkv, hd, kv8) <= kTmaSmemMax;
-  const int epi = kv8 ? 2 : (q_scale != 1.0f || q_layout != FRT_Q_TOKEN_MAJOR) ? 1 : 0;
   return dt == FRT_F16 ? launch_dt<FRT_F16>(P, GP, epi, a, tma, stream)
                        : launch_dt<FRT_BF16>(P, GP, epi, a, tma, stream);
 }
@@ -836,9 +1041,26 @@ extern "C" frt_status frt_qkv_layernorm_rope_kvcache(const void* qkv, const void
   using namespace frt;
   if (M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || hd <= 0 || hd % 2 != 0) return FRT_ERR_INVALID_ARG;
   if (max_pos <= 0 || capacity <= 0 || !valid_dtype(dt)) return FRT_ERR_INVALID_ARG;
-  if (hd % 8 != 0 || hd > 256) return FRT_ERR_UNSUPPORTED;
+  if (hd > 256) return FRT_ERR_UNSUPPORTED;
   if (M == 0) return FRT_OK;
   if (!qkv || !cos_tab || !sin_tab || !positions || !q_out || !k_cache || !v_cache) return FRT_ERR_INVALID_ARG;
+  const int H = Hq + 2 * Hkv;
+  if (hd % 8 != 0) {  // element-wise kernel (see frt_qkv_norm_rope_kvcache)
+    if (!aligned(qkv, 2) || !aligned(q_out, 2) || !aligned(k_cache, 2) || !aligned(v_cache, 2) ||
+        !aligned(cos_tab, 4) || !aligned(sin_tab, 4) || !aligned(positions, 4) || (status && !aligned(status, 4)))
+      return FRT_ERR_INVALID_ARG;
+    for (const void* w : {q_w, q_b, k_w, k_b})
+      if (w && !aligned(w, 2)) return FRT_ERR_INVALID_ARG;
+    const Epilogue ep{1.0f, 0, M, nullptr, static_cast<const uint16_t*>(q_b), static_cast<const uint16_t*>(k_b)};
+    const auto* qk = static_cast<const uint16_t*>(qkv);
+    const auto* qw = static_cast<const uint16_t*>(q_w);
+    const auto* kw = static_cast<const uint16_t*>(k_w);
+    auto* qo = static_cast<uint16_t*>(q_out);
+    return dt == FRT_F16 ? launch_generic<FRT_F16>(3, qk, qw, kw, cos_tab, sin_tab, positions, qo, k_cache, v_cache,
+                                                   status, M, H, Hq, Hkv, hd, max_pos, capacity, eps, ep, stream)
+                         : launch_generic<FRT_BF16>(3, qk, qw, kw, cos_tab, sin_tab, positions, qo, k_cache, v_cache,
+                                                    status, M, H, Hq, Hkv, hd, max_pos, capacity, eps, ep, stream);
+  }
   const int P = (hd % 16 == 0) ? 8 : 4;
   const uintptr_t al = (P == 8) ? 16 : 8;
   if (!aligned(qkv, al) || !aligned(q_out, al) || !aligned(k_cache, al) || !aligned(v_cache, al))
@@ -847,7 +1069,6 @@ extern "C" frt_status frt_qkv_layernorm_rope_kvcache(const void* qkv, const void
     if (w && !aligned(w, al)) return FRT_ERR_INVALID_ARG;
   if (!aligned(cos_tab, 16) || !aligned(sin_tab, 16) || !aligned(positions, 4)) return FRT_ERR_INVALID_ARG;
   if (status && !aligned(status, 4)) return FRT_ERR_INVALID_ARG;
-  const int H = Hq + 2 * Hkv;
   const int G = (hd / 2) / P;
   int GP = 1;
   while (GP < G) GP *= 2;

@@ -46,12 +46,28 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     const uint4* __restrict__ bias, uint2* __restrict__ q, const float* __restrict__ static_scale,
     float* __restrict__ block_scales, int C, int NB, float D, float eps) {
   using P16 = Pack16<DT>;
-  pdl_enter();
   const int t = threadIdx.x;
   const int T = blockDim.x;
   const int64_t row = blockIdx.x;
   const int64_t base = row * (int64_t)C;
   __shared__ double red[32];
+
+  // Constant inputs first, before the wait for the previous kernel: the
+  // scale (and 1 / s in fp64) and, on narrow rows (small-batch,
+  // latency-bound calls), the weight, so neither is on the critical path.
+  // Wide rows load the weight after the reduction and keep the registers
+  // for occupancy.
+  float s_static = 0.0f;
+  if (QM == FRT_QUANT_STATIC || QM >= kQuantNvfp4Rows) s_static = __ldg(static_scale);
+  const double inv_s64 = QM == FRT_QUANT_STATIC && !LN ? 1.0 / (double)s_static : 0.0;
+  constexpr bool kEarlyWeight = WEIGHTED && K <= 2;
+  uint4 wv_early[kEarlyWeight ? K : 1];
+  if (kEarlyWeight) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (t + k * T < C) wv_early[k] = __ldg(w + t + k * T);
+  }
+  pdl_enter();
 
   // Issue every load of the row before any store (r_out may alias r_in).
   uint4 xv[K], rv[K];
@@ -62,20 +78,6 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       xv[k] = ld_stream(x + base + c);
       rv[k] = ld_plain(r_in + base + c);
     }
-  }
-  float s_static = 0.0f;
-  if (QM == FRT_QUANT_STATIC || QM >= kQuantNvfp4Rows) s_static = __ldg(static_scale);
-  // 1 / s in fp64, formed while the row's loads are in flight
-  const double inv_s64 = QM == FRT_QUANT_STATIC && !LN ? 1.0 / (double)s_static : 0.0;
-  // Narrow rows (small-batch, latency-bound calls) load the weight with the
-  // row instead of after the reduction: one memory round trip less on the
-  // critical path.  Wide rows keep the registers for occupancy.
-  constexpr bool kEarlyWeight = WEIGHTED && K <= 2;
-  uint4 wv_early[kEarlyWeight ? K : 1];
-  if (kEarlyWeight) {
-#pragma unroll
-    for (int k = 0; k < K; ++k)
-      if (t + k * T < C) wv_early[k] = __ldg(w + t + k * T);
   }
 
   // Pass 1: h = x + r rounded once to 16 bits (the correctly rounded exact

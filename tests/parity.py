@@ -11,7 +11,11 @@ Tolerances (element by element):
     elements must be the correctly rounded value itself (|g - o| <= ulp/2);
   * FP8 codes: equal (+0 == -0), else one code step apart with the same sign,
     on at most 0.1% of the elements;
-  * block scales: relative error <= 1e-6 against the fp64 amax / 448.
+  * block scales: relative error <= 1e-6 against the fp64 amax / 448;
+  * NVFP4 (the same rule for 4-bit codes): e4m3 scale factors equal or one
+    code step apart on at most 0.1% of the blocks; e2m1 codes equal (+0 ==
+    -0) or one step apart with the same sign, on at most 0.1% of the elements
+    plus the 16 elements of each block whose scale factor differs.
 """
 import numpy as np
 import torch
@@ -52,6 +56,36 @@ def assert_fp8_codes(gpu, ref, max_frac=FP8_MAX_FRAC, what="fp8"):
             what, int(bad.sum()), int(np.flatnonzero(diff)[np.argmax(bad)]), g[diff][bad][0], o[diff][bad][0])
     assert n <= max_frac * g.size, "%s: %d of %d codes one step off (> %.2g%%)" % (what, n, g.size, 100 * max_frac)
     return n
+
+
+def unpack_e2m1(packed):
+    """[..., n] bytes -> [..., 2n] e2m1 codes, element 2j from the low nibble."""
+    p = np.asarray(packed, dtype=np.uint8)
+    return np.stack([p & 0xF, p >> 4], axis=-1).reshape(*p.shape[:-1], p.shape[-1] * 2)
+
+
+def assert_nvfp4(gpu_codes, gpu_sf, ref_codes, ref_sf, what="nvfp4"):
+    """NVFP4 agreement: gpu_codes / ref_codes packed e2m1 bytes [rows, n/2],
+    gpu_sf / ref_sf row-major e4m3 scale factors [rows, n/16].  Returns the
+    number of differing scale factors and codes."""
+    sg = np.asarray(gpu_sf, dtype=np.int32).reshape(np.shape(ref_sf))
+    so = np.asarray(ref_sf, dtype=np.int32)
+    sdiff = sg != so
+    n_sf = int(sdiff.sum())
+    assert (np.abs(sg - so) <= 1).all(), "%s: a scale factor differs by more than one code step" % what
+    assert n_sf <= FP8_MAX_FRAC * so.size, "%s: %d of %d scale factors one step off" % (what, n_sf, so.size)
+    g = unpack_e2m1(np.asarray(gpu_codes).reshape(np.shape(ref_codes))).astype(np.int32)
+    o = unpack_e2m1(ref_codes).astype(np.int32)
+    gm, om = g & 7, o & 7
+    diff = ~((g == o) | ((gm == 0) & (om == 0)))
+    n = int(diff.sum())
+    if n:
+        bad = (np.abs(gm[diff] - om[diff]) != 1) | ((((g[diff] ^ o[diff]) & 8) != 0) & (gm[diff] != 0) &
+                                                  (om[diff] != 0))
+        assert not bad.any(), "%s: %d codes differ by more than one step" % (what, int(bad.sum()))
+    allow = FP8_MAX_FRAC * g.size + 16 * n_sf
+    assert n <= allow, "%s: %d of %d codes one step off (allowance %.1f)" % (what, n, g.size, allow)
+    return n_sf, n
 
 
 # significand bits and smallest normal exponent of the 16-bit formats

@@ -56,12 +56,15 @@ def b_call(M=4, Hq=8, Hkv=2, hd=128, qkv=A, cos=A, sin=A, pos=A, qo=A, kc=A, vc=
 
 @pytest.mark.parametrize("kw,want", [
     (dict(M=-3), INV), (dict(Hq=0), INV), (dict(Hkv=0), INV), (dict(Hq=6, Hkv=4), INV), (dict(hd=7), INV),
-    (dict(hd=0), INV), (dict(hd=6), UNSUP), (dict(hd=12), UNSUP), (dict(hd=264), UNSUP),
+    (dict(hd=0), INV), (dict(hd=264), UNSUP),
     (dict(max_pos=0), INV), (dict(cap=0), INV), (dict(qkv=None), INV), (dict(cos=None), INV),
     (dict(pos=None), INV), (dict(kc=None), INV), (dict(qkv=A + 8), INV), (dict(hd=72, qkv=A + 8, M=0), OK),
     (dict(hd=72, qkv=A + 4), INV), (dict(cos=A + 8), INV), (dict(pos=A + 2), INV), (dict(status=A + 1), INV),
     (dict(qw=A + 8), INV), (dict(dt=9), INV), (dict(M=0), OK), (dict(M=0, qkv=None, kc=None), OK),
-    (dict(M=0, hd=12), UNSUP), (dict(M=0, Hq=6, Hkv=4), INV),
+    (dict(M=0, hd=264), UNSUP), (dict(M=0, Hq=6, Hkv=4), INV),
+    # any even hd (element-wise kernel): 2-byte 16-bit pointers, 4-byte tables
+    (dict(hd=66, qkv=A + 1), INV), (dict(hd=66, kc=A + 3), INV), (dict(hd=100, cos=A + 2), INV),
+    (dict(hd=66, qw=A + 1), INV), (dict(M=0, hd=66), OK), (dict(M=0, hd=2), OK),
 ])
 def test_qkv_host_validation(kw, want):
     assert b_call(**kw) == want
@@ -107,6 +110,19 @@ def test_pdl_switch():
         frt.frt_set_pdl(prev)
 
 
+def test_wait_polls_setting():
+    prev = frt.frt_get_wait_polls()
+    assert prev == frt.FRT_DEFAULT_WAIT_POLLS
+    try:
+        frt.frt_set_wait_polls(0)
+        assert frt.frt_get_wait_polls() == 0
+        assert frt.load().frt_set_wait_polls(-1) == INV
+        assert frt.frt_get_wait_polls() == 0
+    finally:
+        frt.frt_set_wait_polls(prev)
+    assert frt.frt_get_wait_polls() == frt.FRT_DEFAULT_WAIT_POLLS
+
+
 def ada_call(M=4, D=256, x=A, g=A, r=A, ro=A, sc=A, sh=A, q=A, ss=A, bs=None, rpc=4, dt=1, qm=0):
     return frt.load().frt_gate_residual_adarms_fp8(x, g, r, ro, sc, sh, q, ss, bs, M, D, rpc, 1e-6, dt, qm, None)
 
@@ -131,8 +147,9 @@ def b8_call(M=4, Hq=8, Hkv=2, hd=128, kc=A, vc=A, qs=0.125, layout=1, kv=1, scal
 @pytest.mark.parametrize("kw,want", [
     (dict(layout=2), INV), (dict(layout=-1), INV), (dict(kv=2), INV), (dict(qs=float("inf")), INV),
     (dict(qs=float("nan")), INV), (dict(scales=None), INV), (dict(scales=A + 2), INV), (dict(kc=A + 4), INV),
-    (dict(hd=72, vc=A + 2), INV), (dict(kc=None), INV), (dict(hd=12), UNSUP), (dict(M=-1), INV),
+    (dict(hd=72, vc=A + 2), INV), (dict(kc=None), INV), (dict(hd=264), UNSUP), (dict(M=-1), INV),
     (dict(M=0), OK), (dict(M=0, scales=None), OK), (dict(M=0, layout=3), INV), (dict(M=0, kv=0, scales=None), OK),
+    (dict(hd=66, scales=A + 2), INV), (dict(hd=66, scales=None), INV), (dict(M=0, hd=66), OK),
 ])
 def test_qkv_prepq_host_validation(kw, want):
     assert b8_call(**kw) == want
@@ -181,8 +198,9 @@ def qln_call(M=4, Hq=8, Hkv=2, hd=128, qkv=A, qw=None, qb=None, kw=None, kb=None
 
 
 @pytest.mark.parametrize("kw,want", [
-    (dict(Hq=6, Hkv=4), INV), (dict(hd=12), UNSUP), (dict(qb=A + 8), INV), (dict(kw=A + 2), INV),
+    (dict(Hq=6, Hkv=4), INV), (dict(hd=264), UNSUP), (dict(qb=A + 8), INV), (dict(kw=A + 2), INV),
     (dict(qkv=A + 8), INV), (dict(qkv=None), INV), (dict(M=0), OK), (dict(M=0, qkv=None), OK), (dict(dt=4), INV),
+    (dict(hd=66, qkv=A + 1), INV), (dict(hd=66, qb=A + 1), INV), (dict(M=0, hd=66), OK),
 ])
 def test_qkv_layernorm_host_validation(kw, want):
     assert qln_call(**kw) == want

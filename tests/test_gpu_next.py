@@ -278,6 +278,23 @@ def run_prepq_gpu(wl, inp, q_layout, kv, q_scale, kv_scales=(0.02, 0.015), posit
     return q_out, kc, vc, int(status.item())
 
 
+@pytest.mark.parametrize("q_layout", ["token", "head"])
+def test_prepq_bulk_copy_wait_give_up(q_layout):
+    """Levels 1-2 of the bulk-copy kernel with its barrier wait forced to give
+    up (0 polls): status bit 1 and no output written (Q keeps its fill, the
+    e4m3 caches their 0x7E sentinel)."""
+    wl = W.get("large_m_M4096", M=640, capacity=2048)
+    inp = W.make_inputs(wl, n_layers=1, with_caches=False)
+    frt.frt_set_wait_polls(0)
+    try:
+        q_out, kc, vc, status = run_prepq_gpu(wl, inp, q_layout, "e4m3", softmax_scale(wl.hd))
+    finally:
+        frt.frt_set_wait_polls(frt.FRT_DEFAULT_WAIT_POLLS)
+    assert status == 2
+    assert (P.np16(q_out) == 0x3C3C).all()
+    assert bool((kc == 0x7E).all()) and bool((vc == 0x7E).all())
+
+
 def oracle_prepq(wl, inp, q_layout, kv, q_scale, kv_scales=(0.02, 0.015), rows=None, positions=None):
     L = inp.layers[0]
     pos_t = inp.positions if positions is None else positions
@@ -315,7 +332,8 @@ def check_prepq(wl, inp, q_layout, kv, q_scale):
 PREPQ_CASES = [("tiny", {}), ("pi05", {}), ("vla_denoise", {}), ("qwen3_prefill_S512", {}), ("vit", {"M": 40}),
                ("tiny", {"M": 3, "hd": 24, "Hq": 4, "Hkv": 4}), ("tiny", {"M": 2, "hd": 256, "dt": "bf16"}),
                ("large_m_M4096", {"M": 640, "capacity": 2048}),
-               ("large_m_M4096", {"M": 700, "hd": 72, "Hq": 16, "Hkv": 16, "capacity": 2048})]
+               ("large_m_M4096", {"M": 700, "hd": 72, "Hq": 16, "Hkv": 16, "capacity": 2048}),
+               ("tiny", {"M": 5, "hd": 66}), ("vit", {"M": 9, "hd": 100, "qk_norm": True})]
 
 
 @pytest.mark.parametrize("name,ov", PREPQ_CASES, ids=["%s%s" % (n, "".join("-%s%s" % kv for kv in o.items()))
@@ -383,22 +401,29 @@ def test_prepq_large_m_sampled(M):
 # scale factors and a global fp32 scale, scale factors row-major or in the
 # 128x4-swizzled layout of block-scaled GEMMs.
 
-def unpack_e2m1(packed):
-    p = np.asarray(packed, dtype=np.uint8)
-    return np.stack([p & 0xF, p >> 4], axis=-1).reshape(*p.shape[:-1], p.shape[-1] * 2)
+def unswizzle(swz, rows, cols):
+    """Row-major [rows, cols] view of a 128x4-swizzled scale-factor array,
+    gathered through the oracle's offsets."""
+    idx = np.array([[oracle.sf_swizzle_offset(r, c, cols) for c in range(cols)] for r in range(rows)])
+    return np.asarray(swz)[idx]
 
 
-def assert_e2m1_codes(gpu, ref, max_frac=0.0, what="e2m1"):
-    g, o = unpack_e2m1(gpu).ravel().astype(np.int32), unpack_e2m1(ref).ravel().astype(np.int32)
-    gm, om = g & 7, o & 7
-    same = (g == o) | ((gm == 0) & (om == 0))
-    diff = ~same
-    n = int(diff.sum())
-    if n:
-        bad = (np.abs(gm[diff] - om[diff]) != 1) | (((g[diff] ^ o[diff]) & 8) != 0) & (gm[diff] != 0) & (om[diff] != 0)
-        assert not bad.any(), "%s: %d codes differ by more than one step" % (what, int(bad.sum()))
-    assert n <= max_frac * g.size, "%s: %d of %d codes one step off" % (what, n, g.size)
-    return n
+def check_nvfp4(q, sf, o_codes, o_sf, sf_layout, what):
+    """GPU NVFP4 output against the oracle (parity.assert_nvfp4); the
+    swizzled layout is read back through the oracle's offsets.  Prints the
+    mismatch counts."""
+    rows, nsf = o_sf.shape
+    got_sf = sf.cpu().numpy()
+    if sf_layout == "rows":
+        got_sf = got_sf.reshape(rows, nsf)
+    else:
+        pad = oracle.sf_swizzle(np.ones((rows, nsf), dtype=np.uint8)) == 0
+        assert (got_sf[pad] == 0).all(), what + ": a padding byte of the swizzled layout was written"
+        got_sf = unswizzle(got_sf, rows, nsf)
+    n_sf, n = P.assert_nvfp4(q.cpu().numpy(), got_sf, o_codes, o_sf, what=what)
+    print("%s: %d of %d scale factors, %d of %d codes one step off" % (what, n_sf, o_sf.size, n,
+                                                                       2 * np.asarray(o_codes).size))
+    return n_sf, n
 
 
 def global_scale_for(vals):
@@ -440,9 +465,7 @@ def test_residual_rmsnorm_nvfp4_parity(name, ov, sf_layout):
     ro, q, sf = run_a_nvfp4(L.x_attn, inp.residual, L.w_attn, gs, sf_layout)
     o = oracle.residual_rmsnorm_nvfp4(x, r, w, wl.eps, wl.dt, gs)
     np.testing.assert_array_equal(W.bits16(ro.cpu()), o["residual_out"])
-    assert_e2m1_codes(q.cpu().numpy(), o["out_fp4"], what="op a e2m1")
-    want_sf = o["sf"].ravel() if sf_layout == "rows" else oracle.sf_swizzle(o["sf"])
-    np.testing.assert_array_equal(sf.cpu().numpy(), want_sf)
+    check_nvfp4(q, sf, o["out_fp4"], o["sf"], sf_layout, "op a nvfp4")
 
 
 @pytest.mark.parametrize("gs", [1e-6, 1e4])
@@ -455,8 +478,7 @@ def test_residual_rmsnorm_nvfp4_scale_saturation_and_underflow(gs):
     x, r, w = W.bits16(L.x_attn), W.bits16(inp.residual), W.bits16(L.w_attn)
     ro, q, sf = run_a_nvfp4(L.x_attn, inp.residual, L.w_attn, gs)
     o = oracle.residual_rmsnorm_nvfp4(x, r, w, wl.eps, wl.dt, gs)
-    np.testing.assert_array_equal(sf.cpu().numpy(), o["sf"].ravel())
-    assert_e2m1_codes(q.cpu().numpy(), o["out_fp4"], what="op a e2m1")
+    check_nvfp4(q, sf, o["out_fp4"], o["sf"], "rows", "op a nvfp4")
     assert (o["sf"] == 0x7E).all() if gs < 1 else (o["sf"] == 0).all()
 
 
@@ -489,15 +511,7 @@ def test_gate_act_nvfp4_parity(name, ov, sf_layout):
     gs = global_scale_for(a)
     q, sf = run_c_nvfp4(gu, gs, wl.act, sf_layout)
     o = oracle.gate_act_nvfp4(hb, wl.act, wl.dt, gs)
-    exact = wl.act == "relu2"
-    assert_e2m1_codes(q.cpu().numpy(), o["out_fp4"], max_frac=0.0 if exact else 1e-3, what="op c e2m1")
-    want_sf = o["sf"].ravel() if sf_layout == "rows" else oracle.sf_swizzle(o["sf"])
-    got_sf = sf.cpu().numpy()
-    if exact:
-        np.testing.assert_array_equal(got_sf, want_sf)
-    else:
-        step = np.abs(got_sf.astype(int) - want_sf.astype(int))   # positive e4m3 codes: adjacent = 1 apart
-        assert (step <= 1).all() and (step > 0).mean() <= 1e-3
+    check_nvfp4(q, sf, o["out_fp4"], o["sf"], sf_layout, "op c nvfp4")
 
 
 def test_nvfp4_large_m_sampled():
@@ -519,8 +533,7 @@ def test_nvfp4_large_m_sampled():
     torch.cuda.synchronize()
     o = oracle.residual_rmsnorm_nvfp4(x, r, w, wl.eps, wl.dt, gs)
     np.testing.assert_array_equal(W.bits16(rr[ti].cpu()), o["residual_out"])
-    assert_e2m1_codes(q[ti].cpu().numpy(), o["out_fp4"], what="large-M op a e2m1")
-    np.testing.assert_array_equal(sf.view(M, D // 16)[ti].cpu().numpy(), o["sf"])
+    check_nvfp4(q[ti], sf.view(M, D // 16)[ti], o["out_fp4"], o["sf"], "rows", "large-M op a nvfp4")
     # op c on the first 16384 rows of the large-M gate/up buffer
     Mc, I = 16384, wl.I
     gu = L.gate_up[:Mc]
@@ -533,8 +546,7 @@ def test_nvfp4_large_m_sampled():
     frt.frt_gate_act_nvfp4(gu, q, sf, torch.tensor([gs], dtype=torch.float32, device=DEV), act=wl.act)
     torch.cuda.synchronize()
     o = oracle.gate_act_nvfp4(hb, wl.act, wl.dt, gs)
-    assert_e2m1_codes(q[tc].cpu().numpy(), o["out_fp4"], what="large-M op c e2m1")
-    np.testing.assert_array_equal(sf.view(Mc, I // 16)[tc].cpu().numpy(), o["sf"])
+    check_nvfp4(q[tc], sf.view(Mc, I // 16)[tc], o["out_fp4"], o["sf"], "rows", "large-M op c nvfp4")
 
 
 # ================================================================== NEXT-4 ===
@@ -571,9 +583,7 @@ def test_residual_layernorm_parity(M, D, dt, quant, weighted, biased):
         frt.frt_residual_layernorm_nvfp4(xd, rd, rd, wd, bd, q, sf, torch.tensor([gs], device=DEV))
         torch.cuda.synchronize()
         o = oracle.residual_layernorm(hx, hr, hw, hb, 1e-6, dt, "nvfp4", global_scale=gs)
-        assert_e2m1_codes(q.cpu().numpy(), o["out"], max_frac=1e-3, what="LN e2m1")
-        sfs = np.abs(sf.cpu().numpy().astype(int) - o["sf"].ravel().astype(int))
-        assert (sfs <= 1).all() and (sfs > 0).mean() <= 1e-3
+        check_nvfp4(q, sf, o["out"], o["sf"], "rows", "LN nvfp4")
     else:
         q_raw, q = guarded((M, D), torch.uint8, 0xA5)
         ss = bs = None
@@ -611,9 +621,34 @@ def test_residual_layernorm_large_m_sampled():
     P.assert_fp8_codes(q[ti].cpu().numpy(), o["out"], what="large-M LN codes")
 
 
+def test_qkv_layernorm_bulk_copy_wait_give_up():
+    """The LayerNorm level of the bulk-copy kernel with its wait forced to
+    give up: status bit 1, nothing written."""
+    M, Hq, Hkv, hd, dt = 700, 32, 8, 128, "bf16"
+    g = W.generator(5)
+    qkv = W.normal16((M, (Hq + 2 * Hkv) * hd), dt, g)
+    cos, sin = W.rope_tables(1024, hd, 1e4)
+    pos = torch.randperm(1024, generator=g)[:M].to(torch.int32)
+    kc = torch.full((1024, Hkv, hd), 0x7E7E, dtype=torch.int16).view(W.DTYPES[dt]).to(DEV)
+    vc = kc.clone()
+    q_raw, q_out = guarded((M, Hq, hd), qkv.dtype, 0x3C)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    frt.frt_set_wait_polls(0)
+    try:
+        frt.frt_qkv_layernorm_rope_kvcache(qkv.to(DEV), None, None, None, None, cos.to(DEV), sin.to(DEV),
+                                           pos.to(DEV), q_out, kc, vc, Hq, Hkv, hd, status=status)
+        torch.cuda.synchronize()
+    finally:
+        frt.frt_set_wait_polls(frt.FRT_DEFAULT_WAIT_POLLS)
+    assert int(status.item()) == 2
+    assert (P.np16(q_out) == 0x3C3C).all()
+    assert (P.np16(kc) == 0x7E7E).all() and (P.np16(vc) == 0x7E7E).all()
+
+
 QLN_CASES = [dict(M=10, Hq=8, Hkv=1, hd=256, dt="bf16"), dict(M=41, Hq=16, Hkv=8, hd=128, dt="bf16"),
              dict(M=6, Hq=32, Hkv=32, hd=128, dt="bf16"),          # Chameleon-like: 96 heads over two CTAs
-             dict(M=7, Hq=16, Hkv=16, hd=72, dt="f16"), dict(M=700, Hq=32, Hkv=8, hd=128, dt="bf16")]
+             dict(M=7, Hq=16, Hkv=16, hd=72, dt="f16"), dict(M=700, Hq=32, Hkv=8, hd=128, dt="bf16"),
+             dict(M=5, Hq=4, Hkv=2, hd=66, dt="bf16"), dict(M=9, Hq=8, Hkv=8, hd=100, dt="f16")]
 
 
 @pytest.mark.parametrize("c", QLN_CASES, ids=lambda c: "M%d-H%d-%d-hd%d-%s" % (c["M"], c["Hq"], c["Hkv"], c["hd"],

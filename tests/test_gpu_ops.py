@@ -158,6 +158,10 @@ B_CASES = [
     ("tiny", {"M": 5, "hd": 40, "Hq": 6, "Hkv": 3}), ("tiny", {"M": 4, "hd": 64}),
     ("vit", {"M": 7, "qk_norm": True}), ("tiny", {"M": 2, "hd": 248, "Hq": 2, "Hkv": 1}),
     ("tiny", {"M": 2, "hd": 256, "dt": "bf16"}), ("tiny", {"M": 1}),
+    # hd % 8 != 0: the element-wise kernel (odd hd / 2 for 66 and 2)
+    ("tiny", {"M": 5, "hd": 66}), ("vit", {"M": 9, "hd": 100, "qk_norm": True}),
+    ("tiny", {"M": 4, "hd": 2, "Hq": 4, "Hkv": 2}), ("tiny", {"M": 3, "hd": 250, "Hq": 2, "Hkv": 1, "dt": "bf16"}),
+    ("large_m_M4096", {"M": 700, "hd": 100, "Hq": 20, "Hkv": 4, "capacity": 2048}),
 ]
 
 
@@ -298,6 +302,27 @@ def test_qkv_bulk_copy_path_bad_positions():
     assert written.sum() == wl.M - 3
     np.testing.assert_array_equal(P.np16(kc)[~written], W.bits16(inp.layers[0].k_cache)[~written])
     np.testing.assert_array_equal(P.np16(vc), o["v_cache"])
+
+
+def test_qkv_bulk_copy_wait_give_up_sets_bit1_and_writes_nothing():
+    """The bulk-copy kernel's bounded barrier wait, forced to give up (a bound
+    of 0 polls): every token sets status bit 1 and writes none of its
+    outputs (Q staging keeps its fill, both caches their contents); the
+    kernel drains its copies before exiting, and the next call with the
+    default bound is correct."""
+    wl = W.get("large_m_M4096", M=640, capacity=2048)
+    inp = b_inputs(wl)
+    L = inp.layers[0]
+    frt.frt_set_wait_polls(0)
+    try:
+        q_out, kc, vc, status = run_b_gpu(wl, inp)
+    finally:
+        frt.frt_set_wait_polls(frt.FRT_DEFAULT_WAIT_POLLS)
+    assert status == 2
+    assert (P.np16(q_out) == 0x3C3C).all()
+    np.testing.assert_array_equal(P.np16(kc), W.bits16(L.k_cache))
+    np.testing.assert_array_equal(P.np16(vc), W.bits16(L.v_cache))
+    check_b_full(wl, inp)
 
 
 @pytest.mark.parametrize("qn,kn", [(True, False), (False, True), (False, False)])
