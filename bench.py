@@ -83,6 +83,8 @@ def parse_args(argv=None):
                    help="time only the widened ops (gated residual + AdaRMSNorm + FP8) and print their JSON")
     p.add_argument("--next-m", type=int, default=65536, help="rows of the large widened-op case")
     p.add_argument("--next-reps", type=int, default=50)
+    p.add_argument("--table", action="store_true",
+                   help="per-op GPU and CPU-oracle microseconds on every named workload (one JSON object per row)")
     p.add_argument("--persistent-chain", default=None, metavar="WORKLOAD",
                    help="only run the named chain (e.g. pi05) as one persistent kernel, --chain-reps times")
     return p.parse_args(argv)
@@ -315,7 +317,12 @@ def launch_floor(reps=2000):
 
 
 def small_m_ops(floor, reps=400):
-    """Per-op us at M <= 41: back-to-back stream launches and graph nodes."""
+    """Per-op us at M <= 41: back-to-back stream launches and graph nodes,
+    against the empty-kernel floor and against the dependent-copy floor (a
+    graph of in-place row copies of the residual, [M, D] 16-bit: one
+    dependent load and store per node, what any op whose input is its
+    predecessor's output pays at least)."""
+    import memory_bound_non_b200 as frt
     from memory_bound_non_b200 import workloads as W
     from memory_bound_non_b200.chain import LayerChain
     out = {}
@@ -325,8 +332,9 @@ def small_m_ops(floor, reps=400):
         ch = LayerChain(wl, W.make_inputs(wl, n_layers=1))
         ch.calibrate_static_scales()
         res = {}
-        for op in ("attn_norm", "qkv", "gate"):
-            fn = getattr(ch, op)
+        buf = ch.residual.clone()
+        for op in ("dep_copy", "attn_norm", "qkv", "gate"):
+            fn = (lambda _l: frt.frt_copy_rows(buf, buf)) if op == "dep_copy" else getattr(ch, op)
             for _ in range(20):
                 fn(0)
             torch.cuda.synchronize()
@@ -355,6 +363,8 @@ def small_m_ops(floor, reps=400):
             res[op] = {"stream_us": round(stream_us, 3), "graph_node_us": round(node_us, 3),
                        "x_stream_floor": round(stream_us / floor["stream_launch_us"], 3),
                        "x_graph_floor": round(node_us / floor["graph_node_us"], 3)}
+            if op != "dep_copy":
+                res[op]["x_dep_copy_floor"] = round(node_us / res["dep_copy"]["graph_node_us"], 3)
         out[name] = res
     return out
 
@@ -846,6 +856,147 @@ def cpu_baseline_all_cores(wl, rows_per_s, budget_s=4.0, max_cores=32, max_rows=
                       % (cores, rows, max(secs))}
 
 
+# ------------------------------------------------------- per-op table --
+TABLE_WORKLOADS = ("tiny", "pi05", "qwen3_prefill_S128", "qwen3_prefill_S192", "qwen3_prefill_S512",
+                   "qwen3_prefill_S1024", "vla_denoise", "vit", "large_m_M4096", "large_m_M16384", "large_m_M65536")
+
+
+def _oracle_op(wl, host, op, rows):
+    """Seconds the oracle takes for one op on the first `rows` rows."""
+    import oracle
+    from memory_bound_non_b200 import workloads as W
+    hl = host.layers[0]
+    if op in ("attn_norm", "ffn_norm"):
+        x = W.bits16((hl.x_attn if op == "attn_norm" else hl.x_ffn)[:rows])
+        r = W.bits16(host.residual[:rows])
+        w = hl.w_attn if op == "attn_norm" else hl.w_ffn
+        w = None if w is None else W.bits16(w)
+        t0 = time.perf_counter()
+        oracle.residual_rmsnorm_fp8(x, r, w, wl.eps, wl.dt, wl.quant, static_scale=0.01)
+    elif op == "qkv":
+        qkv = W.bits16(hl.qkv[:rows])
+        qw = None if hl.q_norm_w is None else W.bits16(hl.q_norm_w)
+        kw = None if hl.k_norm_w is None else W.bits16(hl.k_norm_w)
+        pos = host.positions[:rows].cpu().numpy()
+        cos, sin = host.cos.cpu().numpy(), host.sin.cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.qkv_norm_rope_kvcache(qkv, qw, kw, cos, sin, pos, wl.Hq, wl.Hkv, wl.hd, rows, wl.eps, wl.dt,
+                                     slots=np.arange(rows))
+    else:
+        gu = W.bits16(hl.gate_up[:rows])
+        t0 = time.perf_counter()
+        oracle.gate_act_fp8(gu, wl.act, wl.dt, wl.quant, static_scale=0.01)
+    return time.perf_counter() - t0
+
+
+def _oracle_op_worker(task):
+    """One process of the all-cores column: its own seeded rows, one op."""
+    import dataclasses
+    from memory_bound_non_b200 import workloads as W
+    wl, op, rows = task
+    small = dataclasses.replace(wl, M=rows)
+    return _oracle_op(small, W.make_inputs(small, n_layers=1), op, rows)
+
+
+def baseline_table(peak, reps=20, max_cores=32, sample_s=1.0):
+    """Per op and workload: GPU microseconds (CUDA events around each launch,
+    L2 flushed before it; at M <= 41 also per graph node), GB/s and roofline
+    fractions, and the CPU oracle's microseconds for the whole batch on one
+    host thread (timed on a row sample, scaled to all rows) and on all host
+    cores (one spawned process per core, each on its share of the rows)."""
+    import dataclasses
+    import multiprocessing as mp
+    from memory_bound_non_b200 import workloads as W
+    from memory_bound_non_b200.chain import LayerChain
+    cores = max(1, min(os.cpu_count() or 1, max_cores))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream()
+    rows_out = []
+    pool = mp.get_context("spawn").Pool(cores)
+    try:
+        for name in TABLE_WORKLOADS:
+            wl = W.get(name, layers=1, steps=1)
+            big = wl.M >= 4096
+            inp = W.make_inputs(wl, n_layers=1, device="cuda" if big else "cpu")
+            ch = LayerChain(wl, inp)
+            ch.calibrate_static_scales()
+            nbytes = op_bytes(wl)
+            for op in ("attn_norm", "qkv", "ffn_norm", "gate"):
+                fn = getattr(ch, op)
+                for _ in range(3):
+                    fn(0)
+                ts = []
+                for _ in range(reps):
+                    flush_l2(flush)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(s)
+                    fn(0)
+                    e1.record(s)
+                    e1.synchronize()
+                    ts.append(e0.elapsed_time(e1) * 1e3)
+                us = statistics.median(ts)
+                gbs = nbytes[op] / (us * 1e-6) / 1e9
+                row = {"workload": name, "op": op, "M": wl.M, "bytes": nbytes[op], "gpu_us": round(us, 2),
+                       "GBps": round(gbs, 1), "frac_of_8TBps": round(gbs / NOMINAL_HBM_GBS, 4),
+                       "frac_of_measured": round(gbs / peak, 4)}
+                if wl.M <= 41:
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        for _ in range(100):
+                            fn(0)
+                    g.replay()
+                    torch.cuda.synchronize()
+                    gt = []
+                    for _ in range(5):
+                        e0.record(s)
+                        g.replay()
+                        e1.record(s)
+                        e1.synchronize()
+                        gt.append(e0.elapsed_time(e1) * 1e3 / 100)
+                    del g
+                    row["gpu_us_graph_node"] = round(statistics.median(gt), 3)
+                # CPU oracle: one thread on a sample of rows, scaled to M
+                host = inp if not big else None
+                n = min(wl.M, 16)
+                if big:
+                    sub = dataclasses.replace(wl, M=n)
+                    host = W.make_inputs(sub, n_layers=1)
+                t1 = _oracle_op(wl if not big else sub, host, op, n)
+                n2 = int(max(n, min(wl.M, n * sample_s / max(t1, 1e-6))))
+                if n2 > n:
+                    if big:
+                        sub = dataclasses.replace(wl, M=n2)
+                        host = W.make_inputs(sub, n_layers=1)
+                    t1 = _oracle_op(wl if not big else sub, host, op, n2)
+                    n = n2
+                row["cpu_1thread_us"] = round(t1 / n * wl.M * 1e6, 1)
+                row["cpu_1thread_sample_rows"] = n
+                per = max(1, -(-wl.M // cores))
+                per_run = min(per, max(1, int(n * 2)))  # bounded: each process times at most ~2 s
+                secs = pool.map(_oracle_op_worker, [(wl, op, per_run)] * min(cores, wl.M))
+                row["cpu_all_cores_us"] = round(max(secs) / per_run * per * 1e6, 1)
+                row["cpu_all_cores_rows_per_process"] = per_run
+                rows_out.append(row)
+                print(json.dumps(row), flush=True)
+            del ch, inp
+            torch.cuda.empty_cache()
+    finally:
+        pool.close()
+        pool.join()
+    return {"cores": cores, "cpu": _cpu_model(), "rows": rows_out}
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def reference_arm(args):
     """The oracle, as it stands, timed on host cores on the same workload."""
     import dataclasses
@@ -916,6 +1067,17 @@ def main(argv=None):
                 ts.append(e0.elapsed_time(e1) * 1e3)
             print(json.dumps({"persistent_chain": cw.name, "launches": len(ts),
                               "us_median": round(statistics.median(ts), 2)}), flush=True)
+        dist.close()
+        return 0
+    if args.table:
+        if rank == 0:
+            t = baseline_table(peak)
+            t.update(peak=peak, peak_kind=peak_kind)
+            s = json.dumps(t)
+            print(s, flush=True)
+            if args.json_out:
+                with open(args.json_out, "w") as f:
+                    f.write(s + "\n")
         dist.close()
         return 0
     if args.next_only:

@@ -268,8 +268,10 @@ frt_status frt_chain_persistent(const frt_chain_layer* layers, int n_layers, int
  * with LayerNorm in place of RMSNorm:
  *   h = x + residual (rounded once, written back);
  *   y = (h - mean) / sqrt(var + eps) * weight + bias, mean and (biased) var
- *       over the row, y rounded once to fp32;
- *   then FP8 (static / block-128) or NVFP4 exactly as the RMSNorm ops.
+ *       over the row (one fp64 pass: var = E[h^2] - mean^2), y in fp32 with a
+ *       few roundings (static FP8: 1 / s folded into the norm factor and the
+ *       bias);
+ *   then FP8 (static / block-128) or NVFP4 as the RMSNorm ops.
  *   weight, bias: device [D] 16-bit, 16-byte aligned, each optional (NULL:
  *   1 / 0).  Other arguments and rules as frt_residual_rmsnorm_fp8 /
  *   frt_residual_rmsnorm_nvfp4.
@@ -337,12 +339,17 @@ frt_status frt_gate_act_nvfp4(const void* gate_up, uint8_t* out_fp4, uint8_t* ou
  *
  * Everything as frt_qkv_norm_rope_kvcache, except:
  *   q_out[i, h, :] (token-major) or q_out[h, i, :] (head-major)
- *          = o * q_scale, the product in fp32, rounded once to 16 bits;
+ *          = o * q_scale in fp32 (q_scale multiplies the head's norm factor,
+ *            or the head before RoPE without a q norm), rounded once to 16
+ *            bits;
  *   kv_format E4M3:
  *     k_cache[p, g, :] = e4m3(o / k_scale)  (uint8; o the K head after norm
- *                                           and RoPE, in fp32),
- *     v_cache[p, g, :] = e4m3(v / v_scale)  (uint8),
- *     each quotient correctly rounded in fp32, RNE, saturating to +-448.
+ *                                           and RoPE, in fp32; the division
+ *                                           is a product with RN(1 / k_scale)
+ *                                           folded in like q_scale),
+ *     v_cache[p, g, :] = e4m3(v / v_scale)  (uint8; the quotient correctly
+ *                                           rounded in fp32),
+ *     RNE, saturating to +-448.
  *
  *   q_scale      host fp32, finite (1 = no scaling).
  *   q_layout     FRT_Q_TOKEN_MAJOR or FRT_Q_HEAD_MAJOR.
@@ -398,6 +405,19 @@ frt_status frt_gate_residual_adarms_fp8(const void* x, const void* gate, const v
  * Returns FRT_ERR_INVALID_ARG for grid < 1 or block outside [1, 1024].
  */
 frt_status frt_noop(int grid, int block, cudaStream_t stream);
+
+/*
+ * Dependent-copy probe, the companion of frt_noop: the smallest op that reads
+ * what the kernel before it wrote.  `rows` CTAs each copy one row of
+ * `row_bytes` bytes from src to dst (device, 16-byte aligned; src == dst is
+ * allowed: each 16-byte chunk is read, then written back).  Its time per
+ * graph node is the empty-kernel floor plus one dependent load and one store:
+ * the floor of any op whose input is its predecessor's output.
+ * Returns FRT_ERR_INVALID_ARG for rows < 0, row_bytes <= 0 or not a multiple
+ * of 16 (or above 2^30), NULL or misaligned pointers (rows == 0: FRT_OK,
+ * nothing launched, pointers not inspected).
+ */
+frt_status frt_copy_rows(const void* src, void* dst, int rows, int row_bytes, cudaStream_t stream);
 
 /*
  * Programmatic dependent launch (PDL), on by default.  With it on, every

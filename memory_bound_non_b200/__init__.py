@@ -13,6 +13,7 @@ Functions carry the C names of ``include/frt.h``:
     frt_gate_residual_adarms_fp8(...)      (NEXT-1)
     frt_noop(grid, block)
 """
+import contextlib
 import ctypes
 import os
 
@@ -20,6 +21,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfrt.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libfrt_debug.so")
 
 FRT_OK, FRT_ERR_INVALID_ARG, FRT_ERR_UNSUPPORTED, FRT_ERR_CUDA = 0, 1, 2, 3
 DTYPE = {torch.float16: 0, torch.bfloat16: 1}
@@ -31,7 +33,7 @@ EXPORTS = ("frt_residual_rmsnorm_fp8", "frt_qkv_norm_rope_kvcache", "frt_gate_ac
            "frt_chain_persistent", "frt_residual_layernorm_fp8", "frt_residual_layernorm_nvfp4",
            "frt_qkv_layernorm_rope_kvcache",
            "frt_residual_rmsnorm_nvfp4", "frt_gate_act_nvfp4", "frt_qkv_norm_rope_prepq_kvcache",
-           "frt_gate_residual_adarms_fp8", "frt_noop", "frt_set_pdl", "frt_get_pdl", "frt_set_wait_polls",
+           "frt_gate_residual_adarms_fp8", "frt_noop", "frt_copy_rows", "frt_set_pdl", "frt_get_pdl", "frt_set_wait_polls",
            "frt_get_wait_polls", "frt_status_string")
 
 
@@ -49,6 +51,48 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     global _lib
     if _lib is not None:
         return _lib
+    _lib = _open(path)
+    return _lib
+
+
+_debug_lib = None
+
+
+def load_debug(path: str = DEBUG_LIB_PATH) -> ctypes.CDLL:
+    """Load the bounds-checked build libfrt_debug.so (once): the same entry
+    points plus frt_debug_bounds_violations (include/frt_debug.h).  Use it
+    through ``using_library``."""
+    global _debug_lib
+    if _debug_lib is None:
+        L = _open(path)
+        L.frt_debug_bounds_violations.argtypes = [ctypes.c_void_p]
+        L.frt_debug_bounds_violations.restype = ctypes.c_int
+        _debug_lib = L
+    return _debug_lib
+
+
+def bounds_violations() -> int:
+    """Out-of-range accesses the bounds-checked build skipped since the last
+    call (synchronises the device; resets the count)."""
+    n = ctypes.c_uint(0)
+    _check("frt_debug_bounds_violations", load_debug().frt_debug_bounds_violations(ctypes.byref(n)))
+    return int(n.value)
+
+
+@contextlib.contextmanager
+def using_library(L):
+    """Route this module's calls through the library handle L (e.g. the
+    bounds-checked build) inside the block."""
+    global _lib
+    prev = load()
+    _lib = L
+    try:
+        yield L
+    finally:
+        _lib = prev
+
+
+def _open(path):
     if not os.path.exists(path):
         raise FrtError("load", -1, "%s is missing; build it with `python -m memory_bound_non_b200.build`" % path)
     L = ctypes.CDLL(path)
@@ -78,6 +122,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_gate_residual_adarms_fp8.restype = i32
     L.frt_noop.argtypes = [i32, i32, vp]
     L.frt_noop.restype = i32
+    L.frt_copy_rows.argtypes = [vp, vp, i32, i32, vp]
+    L.frt_copy_rows.restype = i32
     L.frt_set_pdl.argtypes = [i32]
     L.frt_set_pdl.restype = None
     L.frt_get_pdl.argtypes = []
@@ -88,7 +134,6 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.frt_get_wait_polls.restype = i32
     L.frt_status_string.argtypes = [i32]
     L.frt_status_string.restype = c.c_char_p
-    _lib = L
     return L
 
 
@@ -304,3 +349,11 @@ def frt_get_wait_polls() -> int:
 def frt_noop(grid=1, block=32, stream=None):
     """Empty kernel: the launch floor."""
     _check("frt_noop", load().frt_noop(int(grid), int(block), _stream(stream)))
+
+
+def frt_copy_rows(src, dst, stream=None):
+    """Dependent-copy probe: each row of src ([rows, n] contiguous, n * itemsize
+    a multiple of 16 bytes) copied to dst (may be src)."""
+    rows = src.shape[0]
+    row_bytes = src[0].numel() * src.element_size() if rows else 16
+    _check("frt_copy_rows", load().frt_copy_rows(_ptr(src), _ptr(dst), rows, row_bytes, _stream(stream)))

@@ -1,6 +1,8 @@
-"""Build libfrt.so (the CUDA library) in-tree for sm_100a with nvcc.
+"""Build libfrt.so (the CUDA library) in-tree for sm_100a with nvcc, and its
+bounds-checked variant libfrt_debug.so (FRT_DEBUG_BOUNDS, relocatable device
+code so that every source shares one device-side violation counter).
 
-    python -m memory_bound_non_b200.build        # build if sources changed
+    python -m memory_bound_non_b200.build        # build both if sources changed
     python -m memory_bound_non_b200.build -f     # force
 """
 import concurrent.futures
@@ -16,6 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfrt.so")
+DEBUG_LIB = os.path.join(PKG, "libfrt_debug.so")
+DEBUG_FLAGS = ["-rdc=true", "-DFRT_DEBUG_BOUNDS"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -30,23 +34,26 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale():
-    if not os.path.exists(LIB):
+def _stale(lib=LIB):
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False) -> str:
     """Compile every source to an object in parallel (one nvcc per file),
-    then link the shared library."""
-    if not force and not _stale():
-        return LIB
+    then link the shared library (the bounds-checked one with
+    debug_bounds)."""
+    lib = DEBUG_LIB if debug_bounds else LIB
+    extra = DEBUG_FLAGS if debug_bounds else []
+    if not force and not _stale(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
     objdir = tempfile.mkdtemp(prefix="frt_build_")
-    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"] + extra
     jobs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
@@ -67,14 +74,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
                 sys.stderr.write("failed: %s\n" % " ".join(cmd))
         if failed:
             raise subprocess.CalledProcessError(1, "nvcc")
-        tmp = LIB + ".tmp.%d" % os.getpid()
-        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp] +
+        tmp = lib + ".tmp.%d" % os.getpid()
+        subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared"] + extra[:1] + ["-o", tmp] +
                        [o for _, o in jobs], check=True)
-        os.replace(tmp, LIB)
+        os.replace(tmp, lib)
     finally:
         shutil.rmtree(objdir, ignore_errors=True)
-    return LIB
+    return lib
+
+
+def build_all(force: bool = False, verbose: bool = False):
+    return build(force, verbose), build(force, verbose, debug_bounds=True)
 
 
 if __name__ == "__main__":
-    print(build(force="-f" in sys.argv, verbose="-v" in sys.argv))
+    for path in build_all(force="-f" in sys.argv, verbose="-v" in sys.argv):
+        print(path)

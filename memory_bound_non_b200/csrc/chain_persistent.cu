@@ -63,7 +63,7 @@ struct Slice {
 template <int DT, int K, int QM>
 __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uint2* q, float* bs, const Divisor& dv,
                                            double inv_s64, uint4 (&hv)[K], int64_t row, const Slice& sl, int C,
-                                           int NB, float D, float eps, double* red) {
+                                           int NB, float D, float eps, double* red, int64_t n_rows) {
   using P16 = Pack16<DT>;
   const int t = threadIdx.x;
   uint4 xv[K], wv[K];
@@ -125,9 +125,9 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
       am = half_warp_max_abs(am);
       const float sb = block_scale_448(am);
-      if (valid && (j & 15) == 0) bs[row * NB + (c >> 4)] = sb;
-      if (valid) q[row * C + c] = quant8(y, Divisor(sb));
-    } else if (valid) {
+      if (valid && (j & 15) == 0 && FRT_IDX_OK(row * NB + (c >> 4), n_rows * NB)) bs[row * NB + (c >> 4)] = sb;
+      if (valid && FRT_IDX_OK(row * C + c, n_rows * C)) q[row * C + c] = quant8(y, Divisor(sb));
+    } else if (valid && FRT_IDX_OK(row * C + c, n_rows * C)) {
       q[row * C + c] = fold ? e4m3x8(y) : quant8(y, dv);
     }
   }
@@ -139,7 +139,8 @@ template <int DT, int GP>
 __device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t* qw, const uint16_t* kw,
                                           uint16_t* q_out, uint16_t* k_cache, uint16_t* v_cache, const float2* cs,
                                           const float2* sn, const float2* nsn, int64_t row, int p, bool row_ok,
-                                          const Slice& sl, int Hq, int Hkv, int hd, int G, float eps) {
+                                          const Slice& sl, int Hq, int Hkv, int hd, int G, float eps,
+                                          int64_t n_rows, int capacity) {
   constexpr int P = 8;
   constexpr int NP = P / 2;
   const float inv_hd = 1.0f / (float)hd;
@@ -173,7 +174,8 @@ __device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t*
       va = *reinterpret_cast<const uint4*>(heads + (int64_t)i * hd + j0);
       vb = *reinterpret_cast<const uint4*>(heads + (int64_t)i * hd + half + j0);
     }
-    if (on && is_v) {
+    const int64_t n_kv = (int64_t)capacity * Hkv * hd;
+    if (on && is_v && FRT_SPAN_OK(((int64_t)p * Hkv + (h - Hq - Hkv)) * hd + j0, half + P, n_kv)) {
       uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
       *reinterpret_cast<uint4*>(dst + j0) = va;
       *reinterpret_cast<uint4*>(dst + half + j0) = vb;
@@ -201,9 +203,12 @@ __device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t*
       uint4 o1, o2;
       pack_pairs<DT, NP>(x, reinterpret_cast<uint32_t*>(&o1));
       pack_pairs<DT, NP>(y, reinterpret_cast<uint32_t*>(&o2));
-      uint16_t* dst = is_q ? q_out + (row * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + (h - Hq)) * hd;
-      *reinterpret_cast<uint4*>(dst + j0) = o1;
-      *reinterpret_cast<uint4*>(dst + half + j0) = o2;
+      const int64_t o = is_q ? (row * Hq + h) * hd : ((int64_t)p * Hkv + (h - Hq)) * hd;
+      uint16_t* dst = (is_q ? q_out : k_cache) + o;
+      if (FRT_SPAN_OK(o + j0, half + P, is_q ? n_rows * Hq * hd : n_kv)) {
+        *reinterpret_cast<uint4*>(dst + j0) = o1;
+        *reinterpret_cast<uint4*>(dst + half + j0) = o2;
+      }
     }
   }
 }
@@ -212,7 +217,7 @@ __device__ __forceinline__ void chain_qkv(const uint16_t* heads, const uint16_t*
 // with their loads issued first (one 16-byte load = 4 (g, u) pairs).
 template <int DT, int QM, int ACT>
 __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* bs, const Divisor& dv, int64_t row,
-                                          const Slice& sl, int I4, int NBI) {
+                                          const Slice& sl, int I4, int NBI, int64_t n_rows) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   uint32_t* dst = q + row * I4;
@@ -235,9 +240,9 @@ __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* b
       if (QM == FRT_QUANT_BLOCK128) {
         const float am = warp_max_abs(absmax4(a[0], a[1], a[2], a[3]));
         const float sb = block_scale_448(am);
-        if (lane == 0) bs[row * NBI + b] = sb;
-        dst[b * 32 + lane] = quant4(a, Divisor(sb));
-      } else {
+        if (lane == 0 && FRT_IDX_OK(row * NBI + b, n_rows * NBI)) bs[row * NBI + b] = sb;
+        if (FRT_IDX_OK(row * I4 + b * 32 + lane, n_rows * I4)) dst[b * 32 + lane] = quant4(a, Divisor(sb));
+      } else if (FRT_IDX_OK(row * I4 + b * 32 + lane, n_rows * I4)) {
         dst[b * 32 + lane] = quant4(a, dv);
       }
     }
@@ -262,23 +267,25 @@ struct StageMap {
         gu(4 * cs + heads16 + 2 * hd16), len(4 * cs + heads16 + 2 * hd16 + gu16) {}
 };
 
-__device__ __forceinline__ void stage_copy(uint4* dst, const void* src, int64_t off, int n) {
+// (n_src: the source buffer's 16-byte chunks, checked in the bounds-checked build)
+__device__ __forceinline__ void stage_copy(uint4* dst, const void* src, int64_t off, int n, int64_t n_src) {
   if (src == nullptr) return;
   const uint4* s = static_cast<const uint4*>(src) + off;
-  for (int i = threadIdx.x; i < n; i += kChainThreads) cp_async16(dst + i, s + i);
+  for (int i = threadIdx.x; i < n; i += kChainThreads)
+    if (FRT_IDX_OK(off + i, n_src)) cp_async16(dst + i, s + i);
 }
 
 // Copies every input slice one layer invocation of this CTA reads.
 __device__ __forceinline__ void stage_layer(uint4* st, const StageMap& m, const frt_chain_layer& L, int64_t row,
-                                            const Slice& sl, int C, int qkv16, int hd16, int I4) {
-  stage_copy(st + m.xa, L.x_attn, row * C + sl.c0, sl.nc);
-  stage_copy(st + m.xf, L.x_ffn, row * C + sl.c0, sl.nc);
-  stage_copy(st + m.wa, L.w_attn, sl.c0, sl.nc);
-  stage_copy(st + m.wf, L.w_ffn, sl.c0, sl.nc);
-  stage_copy(st + m.qkv, L.qkv, row * qkv16 + (int64_t)sl.h0 * hd16, sl.nh * hd16);
-  stage_copy(st + m.qw, L.q_norm_w, 0, hd16);
-  stage_copy(st + m.kw, L.k_norm_w, 0, hd16);
-  stage_copy(st + m.gu, L.gate_up, row * I4 + (int64_t)sl.b0 * 32, sl.nb * 32);
+                                            const Slice& sl, int C, int qkv16, int hd16, int I4, int64_t n_rows) {
+  stage_copy(st + m.xa, L.x_attn, row * C + sl.c0, sl.nc, n_rows * C);
+  stage_copy(st + m.xf, L.x_ffn, row * C + sl.c0, sl.nc, n_rows * C);
+  stage_copy(st + m.wa, L.w_attn, sl.c0, sl.nc, C);
+  stage_copy(st + m.wf, L.w_ffn, sl.c0, sl.nc, C);
+  stage_copy(st + m.qkv, L.qkv, row * qkv16 + (int64_t)sl.h0 * hd16, sl.nh * hd16, n_rows * qkv16);
+  stage_copy(st + m.qw, L.q_norm_w, 0, hd16, hd16);
+  stage_copy(st + m.kw, L.k_norm_w, 0, hd16, hd16);
+  stage_copy(st + m.gu, L.gate_up, row * I4 + (int64_t)sl.b0 * 32, sl.nb * 32, n_rows * I4);
 }
 
 template <int DT, int K, int QM, int GP, int ACT>
@@ -310,28 +317,31 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
   sl.b0 = bc_cta ? min(NBI, w * bsl) : 0;
   sl.nb = bc_cta ? min(NBI, sl.b0 + bsl) - sl.b0 : 0;
 
+  const int64_t n_rows = gridDim.x / S;  // extents for the bounds-checked build
   uint4 hv[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int j = t + k * kChainThreads;
-    hv[k] = j < sl.nc ? residual[row * C + sl.c0 + j] : make_uint4(0u, 0u, 0u, 0u);
+    hv[k] = j < sl.nc && FRT_IDX_OK(row * C + sl.c0 + j, n_rows * C) ? residual[row * C + sl.c0 + j]
+                                                                   : make_uint4(0u, 0u, 0u, 0u);
   }
-  const int p = __ldg(positions + row);
+  const int p = FRT_IDX_OK(row, n_rows) ? __ldg(positions + row) : -1;
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
   if (!row_ok && t == 0 && r == 0 && status != nullptr) atomicOr(status, 1);
   constexpr int P = 8;
   const int li = t & (GP - 1);
   const int half = hd >> 1;
   float2 cs8[P / 2], sn8[P / 2], nsn8[P / 2];
-  if (row_ok && li < G)
+  if (row_ok && li < G && FRT_SPAN_OK((int64_t)p * half + li * P, P, (int64_t)max_pos * half))
     load_rope_pairs<P / 2>(cos_tab + (int64_t)p * half + li * P, sin_tab + (int64_t)p * half + li * P, cs8, sn8,
                            nsn8);
-  const Divisor dv_attn(QM == FRT_QUANT_STATIC ? __ldg(scales) : 1.0f);
-  const Divisor dv_ffn(QM == FRT_QUANT_STATIC ? __ldg(scales + 1) : 1.0f);
+  const bool scales_ok = FRT_SPAN_OK(0, 3, 3);
+  const Divisor dv_attn(QM == FRT_QUANT_STATIC && scales_ok ? __ldg(scales) : 1.0f);
+  const Divisor dv_ffn(QM == FRT_QUANT_STATIC && scales_ok ? __ldg(scales + 1) : 1.0f);
   // static FP8: 1 / s in fp64 for the norms' folded product (0 otherwise)
   const double inv_attn = QM == FRT_QUANT_STATIC ? 1.0 / (double)dv_attn.s : 0.0;
   const double inv_ffn = QM == FRT_QUANT_STATIC ? 1.0 / (double)dv_ffn.s : 0.0;
-  const Divisor dv_act(QM == FRT_QUANT_STATIC ? __ldg(scales + 2) : 1.0f);
+  const Divisor dv_act(QM == FRT_QUANT_STATIC && scales_ok ? __ldg(scales + 2) : 1.0f);
   const float D = (float)(C * 8);
   const int qkv16 = H * hd / 8, hd16 = hd / 8;
   // this CTA's stage layout: only the slices of its own roles (the host sizes
@@ -347,39 +357,44 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
     const uint64_t* src = reinterpret_cast<const uint64_t*>(layers);
     uint64_t* dst = reinterpret_cast<uint64_t*>(tab);
     const int words = n_layers * (int)(sizeof(frt_chain_layer) / 8);
-    for (int i = t; i < words; i += kChainThreads) dst[i] = __ldg(src + i);
+    for (int i = t; i < words; i += kChainThreads)
+      if (FRT_IDX_OK(i, words)) dst[i] = __ldg(src + i);
     __syncthreads();
   }
   const int total = steps * n_layers;
   if (total > 0) {
-    stage_layer(stages, m, tab[0], row, sl, C, qkv16, hd16, I4);
+    stage_layer(stages, m, tab[0], row, sl, C, qkv16, hd16, I4, n_rows);
     cp_async_commit();
   }
   for (int it = 0; it < total; ++it) {
     const frt_chain_layer& L = tab[it % n_layers];
-    if (it + 1 < total) stage_layer(stages + ((it + 1) & 1) * m.len, m, tab[(it + 1) % n_layers], row, sl, C, qkv16, hd16, I4);
+    if (it + 1 < total)
+      stage_layer(stages + ((it + 1) & 1) * m.len, m, tab[(it + 1) % n_layers], row, sl, C, qkv16, hd16, I4, n_rows);
     cp_async_commit();  // possibly empty: one group per iteration
     cp_async_wait1();   // this iteration's stage has landed (only the newest group may be pending)
     __syncthreads();    // ... for every thread's copies
     const uint4* st = stages + (it & 1) * m.len;
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xa, L.w_attn != nullptr ? st + m.wa : nullptr,
-                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, inv_attn, hv, row, sl, C, NB, D, eps, red);
+                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, inv_attn, hv, row, sl, C, NB, D, eps, red,
+                            n_rows);
     chain_qkv<DT, GP>(reinterpret_cast<const uint16_t*>(st + m.qkv),
                       L.q_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.qw) : nullptr,
                       L.k_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.kw) : nullptr,
                       static_cast<uint16_t*>(L.q_out), static_cast<uint16_t*>(L.k_cache),
-                      static_cast<uint16_t*>(L.v_cache), cs8, sn8, nsn8, row, p, row_ok, sl, Hq, Hkv, hd, G, eps);
+                      static_cast<uint16_t*>(L.v_cache), cs8, sn8, nsn8, row, p, row_ok, sl, Hq, Hkv, hd, G, eps,
+                      n_rows, capacity);
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xf, L.w_ffn != nullptr ? st + m.wf : nullptr, reinterpret_cast<uint2*>(L.q8_ffn),
-                            L.bs_ffn, dv_ffn, inv_ffn, hv, row, sl, C, NB, D, eps, red);
-    chain_act<DT, QM, ACT>(st + m.gu, reinterpret_cast<uint32_t*>(L.act8), L.bs_act, dv_act, row, sl, I4, NBI);
+                            L.bs_ffn, dv_ffn, inv_ffn, hv, row, sl, C, NB, D, eps, red, n_rows);
+    chain_act<DT, QM, ACT>(st + m.gu, reinterpret_cast<uint32_t*>(L.act8), L.bs_act, dv_act, row, sl, I4, NBI,
+                           n_rows);
     __syncthreads();  // the stage read here is refilled at iteration it + 2
   }
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int j = t + k * kChainThreads;
-    if (j < sl.nc) residual[row * C + sl.c0 + j] = hv[k];
+    if (j < sl.nc && FRT_IDX_OK(row * C + sl.c0 + j, n_rows * C)) residual[row * C + sl.c0 + j] = hv[k];
   }
 }
 

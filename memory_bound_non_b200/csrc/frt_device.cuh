@@ -12,6 +12,31 @@
 
 namespace frt {
 
+// ---------------------------------------------------- bounds-checked build --
+// Built with FRT_DEBUG_BOUNDS (the separate libfrt_debug.so, relocatable
+// device code), every global access of the kernels is preceded by a check of
+// its element index against the extent the kernel's own arguments and grid
+// give that buffer; an index out of range skips the access and counts one
+// violation in frt_bounds_violations (read and cleared on the host with
+// frt_debug_bounds_violations).  In the product library the checks are the
+// constant true and compile to nothing.
+#ifdef FRT_DEBUG_BOUNDS
+extern __device__ unsigned int frt_bounds_violations;
+__device__ __forceinline__ bool in_range(int64_t i, int64_t n) {
+  if (i >= 0 && i < n) return true;
+  atomicAdd(&frt_bounds_violations, 1u);
+  return false;
+}
+// index i of an n-element buffer
+#define FRT_IDX_OK(i, n) ::frt::in_range((int64_t)(i), (int64_t)(n))
+// elements [i, i + len) of an n-element buffer
+#define FRT_SPAN_OK(i, len, n) \
+  (::frt::in_range((int64_t)(i), (int64_t)(n)) && ::frt::in_range((int64_t)(i) + (int64_t)(len) - 1, (int64_t)(n)))
+#else
+#define FRT_IDX_OK(i, n) ((void)(i), (void)(n), true)
+#define FRT_SPAN_OK(i, len, n) ((void)(i), (void)(len), (void)(n), true)
+#endif
+
 // ------------------------------------------------------------------ PDL --
 // Every kernel calls this before it touches any memory that the previous
 // kernel of the stream may write: wait until the grid this launch depends on

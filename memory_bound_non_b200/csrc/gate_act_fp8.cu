@@ -23,7 +23,10 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kU = 4;  // scale blocks per warp
+// Scale blocks per warp: 4 on large batches (each warp keeps four loads in
+// flight), 1 on small ones (latency-bound: as many warps as blocks).
+constexpr int kU = 4;
+constexpr int64_t kSmallBlocks = 148 * kWarps * 4;  // at most 4 CTAs per SM with one block per warp
 static_assert(kThreads == 256, "the NVFP4 reciprocal table takes one sf code per thread");
 
 // Six CTAs (48 warps) per SM need at most 40 registers a thread; the
@@ -34,7 +37,7 @@ constexpr int gate_min_blocks() {
   return (QM == FRT_QUANT_BLOCK128 || QM == kQuantNvfp4Rows) && FULL ? 6 : 1;
 }
 
-template <int DT, int ACT, int QM, bool FULL>
+template <int DT, int ACT, int QM, bool FULL, int U>
 __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_act_fp8_kernel(const uint4* __restrict__ gu,
                                                                  uint32_t* __restrict__ q,
                                                                  const float* __restrict__ static_scale,
@@ -43,40 +46,43 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
   // Constant inputs before the wait for the previous kernel: static FP8 the
   // scale; NVFP4 the global scale gs, RN(1 / RN(6 gs)) and RN(1 / RN(sf * gs))
   // for each of the 256 sf codes (one per thread).
-  const float gs = QM >= kQuantNvfp4Rows ? __ldg(static_scale) : 0.0f;
+  const float gs = QM >= kQuantNvfp4Rows && FRT_IDX_OK(0, 1) ? __ldg(static_scale) : 0.0f;
   const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * gs) : 0.0f;
-  const Divisor dv_static(QM == FRT_QUANT_STATIC ? __ldg(static_scale) : 1.0f);
+  const Divisor dv_static(QM == FRT_QUANT_STATIC && FRT_IDX_OK(0, 1) ? __ldg(static_scale) : 1.0f);
   __shared__ float reff_of[QM >= kQuantNvfp4Rows ? kThreads : 1];
   if (QM >= kQuantNvfp4Rows) reff_of[threadIdx.x] = nvfp4_reff_entry(threadIdx.x, gs);
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int64_t gb0 = warp * kU;
+  const int64_t gb0 = warp * U;
+  // extents: M = total_blocks / NB rows of C4 16-byte input chunks (and as
+  // many 4-byte output words); block scales [M, NB]
+  const int64_t n_chunks = total_blocks / NB * C4;
 
   // Load phase: chunk `lane` of each of the U blocks (4 outputs = 16 bytes).
   // FULL (I % 128 == 0): every block is 32 whole chunks, so the flat chunk
   // index is just 32 * block + lane; otherwise rows end in a partial block
   // and the (row, block) position is tracked.
-  uint4 v[kU];
-  int64_t idx[kU];
-  bool valid[kU];
+  uint4 v[U];
+  int64_t idx[U];
+  bool valid[U];
   if (FULL) {
     const int64_t i0 = gb0 * 32 + lane;
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
+    for (int u = 0; u < U; ++u) {
       valid[u] = gb0 + u < total_blocks;
       idx[u] = i0 + 32 * u;  // same index for the input (uint4) and output (uint32) views
-      if (valid[u]) v[u] = ld_stream(gu + idx[u]);
+      if (valid[u] && FRT_IDX_OK(idx[u], n_chunks)) v[u] = ld_stream(gu + idx[u]);
     }
   } else {
     int64_t row = gb0 / NB;
     int b = (int)(gb0 - row * NB);
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int chunk = b * 32 + lane;  // chunk index within the row (4 outputs each)
       valid[u] = gb0 + u < total_blocks && chunk < C4;
       idx[u] = row * C4 + chunk;
-      if (valid[u]) v[u] = ld_stream(gu + idx[u]);
+      if (valid[u] && FRT_IDX_OK(idx[u], n_chunks)) v[u] = ld_stream(gu + idx[u]);
       if (++b == NB) {
         b = 0;
         ++row;
@@ -87,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
   if (QM >= kQuantNvfp4Rows) __syncthreads();  // the reciprocal table is complete
 
 #pragma unroll
-  for (int u = 0; u < kU; ++u) {
+  for (int u = 0; u < U; ++u) {
     float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (valid[u]) {
       const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[u]);  // (gate, up) pairs
@@ -102,8 +108,9 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
       const float am = warp_max_abs(absmax4(a[0], a[1], a[2], a[3]));
       const float sb = block_scale_448(am);
       const int64_t gb = gb0 + u;
-      if (lane == 0 && gb < total_blocks) block_scales[gb] = sb;  // [M, NB] row-major == flat block index
-      if (valid[u]) q[idx[u]] = quant4(a, Divisor(sb));
+      if (lane == 0 && gb < total_blocks && FRT_IDX_OK(gb, total_blocks))
+        block_scales[gb] = sb;  // [M, NB] row-major == flat block index
+      if (valid[u] && FRT_IDX_OK(idx[u], n_chunks)) q[idx[u]] = quant4(a, Divisor(sb));
     } else if (QM >= kQuantNvfp4Rows) {
       // NVFP4: a 16-output block is 4 consecutive lanes; codes leave as 16 bits
       // per lane, the scale factor from the block's first lane.  q /
@@ -114,46 +121,54 @@ __global__ void __launch_bounds__(kThreads, gate_min_blocks<QM, FULL>()) gate_ac
       float reff;
       const uint32_t sf = nvfp4_scale_lookup(am, rden, reff_of, &reff);
       if (valid[u]) {
-        reinterpret_cast<uint16_t*>(q)[idx[u]] = (uint16_t)nvfp4_codes<4>(a, reff);
+        if (FRT_IDX_OK(idx[u], n_chunks)) reinterpret_cast<uint16_t*>(q)[idx[u]] = (uint16_t)nvfp4_codes<4>(a, reff);
         if ((lane & 3) == 0) {
           uint8_t* sfo = reinterpret_cast<uint8_t*>(block_scales);
           if (QM == kQuantNvfp4Rows) {
-            sfo[idx[u] >> 2] = (uint8_t)sf;  // flat output index / 16 == row * (I/16) + column block
+            // flat output index / 16 == row * (I/16) + column block
+            if (FRT_IDX_OK(idx[u] >> 2, n_chunks >> 2)) sfo[idx[u] >> 2] = (uint8_t)sf;
           } else {
             const int64_t row = idx[u] / C4;
-            sfo[sf_offset_swizzled(row, (int)((idx[u] - row * C4) >> 2), C4 >> 2)] = (uint8_t)sf;
+            const int64_t o = sf_offset_swizzled(row, (int)((idx[u] - row * C4) >> 2), C4 >> 2);
+            if (FRT_IDX_OK(o, (total_blocks / NB + 127) / 128 * 128 * (((C4 >> 2) + 3) / 4) * 4)) sfo[o] = (uint8_t)sf;
           }
         }
       }
-    } else if (valid[u]) {
+    } else if (valid[u] && FRT_IDX_OK(idx[u], n_chunks)) {
       q[idx[u]] = quant4(a, dv_static);
     }
   }
 }
 
+template <int DT, int ACT, int QM, int U>
+frt_status launch_u(bool full, const uint4* in, uint32_t* out, const float* ss, float* bs, int64_t total, int NB,
+                    int C4, cudaStream_t st) {
+  const int64_t warps = (total + U - 1) / U;
+  const dim3 grid((unsigned)((warps + kWarps - 1) / kWarps));
+  return full ? launch(gate_act_fp8_kernel<DT, ACT, QM, true, U>, grid, dim3(kThreads), 0, st, in, out, ss, bs,
+                       total, NB, C4)
+              : launch(gate_act_fp8_kernel<DT, ACT, QM, false, U>, grid, dim3(kThreads), 0, st, in, out, ss, bs,
+                       total, NB, C4);
+}
+
 template <int DT, int ACT, int QM>
-frt_status launch_q(bool full, dim3 grid, const uint4* in, uint32_t* out, const float* ss, float* bs, int64_t total,
-                    int NB, int C4, cudaStream_t st) {
-  return full ? launch(gate_act_fp8_kernel<DT, ACT, QM, true>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
-                       NB, C4)
-              : launch(gate_act_fp8_kernel<DT, ACT, QM, false>, grid, dim3(kThreads), 0, st, in, out, ss, bs, total,
-                       NB, C4);
+frt_status launch_q(bool full, const uint4* in, uint32_t* out, const float* ss, float* bs, int64_t total, int NB,
+                    int C4, cudaStream_t st) {
+  return total <= kSmallBlocks ? launch_u<DT, ACT, QM, 1>(full, in, out, ss, bs, total, NB, C4, st)
+                               : launch_u<DT, ACT, QM, kU>(full, in, out, ss, bs, total, NB, C4, st);
 }
 
 template <int DT, int ACT>
 frt_status launch_act(int qm, const void* gu, uint8_t* q, const float* ss, float* bs, int64_t total, int NB, int C4,
                       cudaStream_t st) {
-  const int64_t warps = (total + kU - 1) / kU;
-  const dim3 grid((unsigned)((warps + kWarps - 1) / kWarps));
   const uint4* in = static_cast<const uint4*>(gu);
   uint32_t* out = reinterpret_cast<uint32_t*>(q);
   const bool full = C4 == NB * 32;
   switch (qm) {
-    case FRT_QUANT_STATIC: return launch_q<DT, ACT, FRT_QUANT_STATIC>(full, grid, in, out, ss, bs, total, NB, C4, st);
-    case FRT_QUANT_BLOCK128:
-      return launch_q<DT, ACT, FRT_QUANT_BLOCK128>(full, grid, in, out, ss, bs, total, NB, C4, st);
-    case kQuantNvfp4Rows: return launch_q<DT, ACT, kQuantNvfp4Rows>(full, grid, in, out, ss, bs, total, NB, C4, st);
-    default: return launch_q<DT, ACT, kQuantNvfp4Swizzled>(full, grid, in, out, ss, bs, total, NB, C4, st);
+    case FRT_QUANT_STATIC: return launch_q<DT, ACT, FRT_QUANT_STATIC>(full, in, out, ss, bs, total, NB, C4, st);
+    case FRT_QUANT_BLOCK128: return launch_q<DT, ACT, FRT_QUANT_BLOCK128>(full, in, out, ss, bs, total, NB, C4, st);
+    case kQuantNvfp4Rows: return launch_q<DT, ACT, kQuantNvfp4Rows>(full, in, out, ss, bs, total, NB, C4, st);
+    default: return launch_q<DT, ACT, kQuantNvfp4Swizzled>(full, in, out, ss, bs, total, NB, C4, st);
   }
 }
 

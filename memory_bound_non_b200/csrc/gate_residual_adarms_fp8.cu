@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
   // previous kernel (the gate, scale and shift rows are computed per step by
   // a preceding kernel, so they wait)
   float s_static = 0.0f;
-  if (QM == FRT_QUANT_STATIC) s_static = __ldg(static_scale);
+  if (QM == FRT_QUANT_STATIC && FRT_IDX_OK(0, 1)) s_static = __ldg(static_scale);
   pdl_enter();
   const int t = threadIdx.x;
   const int T = blockDim.x;
@@ -78,20 +78,24 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
   uint4* s_scale = cond + (GATED && kGateSmem ? C : 0);
   uint4* s_shift = s_scale + C;
 
+  // extents: [M, C] 16-byte chunks of x / r / q, [ceil(M / rows_per_cond), C] of the condition rows
+  const int64_t n_rc = (int64_t)gridDim.x * C;
+  const int64_t n_cond = ((int64_t)gridDim.x + rows_per_cond - 1) / rows_per_cond * C;
   uint4 xv[K], rv[K], gv[GATED && !kGateSmem ? K : 1];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = t + k * T;
-    if (c < C) {
+    if (c < C && FRT_IDX_OK(base + c, n_rc)) {
       xv[k] = ld_stream(x + base + c);
       rv[k] = ld_plain(r_in + base + c);
-      if (GATED && !kGateSmem) gv[k] = __ldg(gate + cbase + c);
+      if (GATED && !kGateSmem && FRT_IDX_OK(cbase + c, n_cond)) gv[k] = __ldg(gate + cbase + c);
     }
   }
   if (GATED && kGateSmem) {
 #pragma unroll
     for (int k = 0; k < K; ++k)
-      if (t + k * T < C) cp_async16(s_gate + t + k * T, gate + cbase + t + k * T);
+      if (t + k * T < C && FRT_IDX_OK(cbase + t + k * T, n_cond))
+        cp_async16(s_gate + t + k * T, gate + cbase + t + k * T);
     cp_async_commit();
   }
   if (MOD) {
@@ -99,9 +103,9 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
     for (int k = 0; k < K; ++k) {
       const int c = t + k * T;
       if (c < C) {
-        if (scale != nullptr) cp_async16(s_scale + c, scale + cbase + c);
+        if (scale != nullptr && FRT_IDX_OK(cbase + c, n_cond)) cp_async16(s_scale + c, scale + cbase + c);
         else s_scale[c] = make_uint4(0u, 0u, 0u, 0u);  // 16-bit zeros
-        if (shift != nullptr) cp_async16(s_shift + c, shift + cbase + c);
+        if (shift != nullptr && FRT_IDX_OK(cbase + c, n_cond)) cp_async16(s_shift + c, shift + cbase + c);
         else s_shift[c] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
@@ -138,7 +142,7 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
         sk = fma((Acc)hf.y, (Acc)hf.y, sk);
       }
       ss += sk;
-      r_out[base + c] = hv[k];
+      if (FRT_IDX_OK(base + c, n_rc)) r_out[base + c] = hv[k];
     }
   }
 
@@ -191,9 +195,10 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
       am = half_warp_max_abs(am);
       const float sb = block_scale_448(am);
-      if (valid && (t & 15) == 0) block_scales[row * NB + (c >> 4)] = sb;
-      if (valid) q[base + c] = quant8(y, Divisor(sb));
-    } else if (valid) {
+      if (valid && (t & 15) == 0 && FRT_IDX_OK(row * NB + (c >> 4), (int64_t)gridDim.x * NB))
+        block_scales[row * NB + (c >> 4)] = sb;
+      if (valid && FRT_IDX_OK(base + c, n_rc)) q[base + c] = quant8(y, Divisor(sb));
+    } else if (valid && FRT_IDX_OK(base + c, n_rc)) {
       q[base + c] = quant8(y, dv_static);
     }
   }

@@ -95,6 +95,16 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const float* v, const 
     *reinterpret_cast<uint32_t*>(dst) = quant4(v, dv);
 }
 
+// P fp32 values already divided by the scale -> P e4m3 codes at dst.
+template <int P>
+__device__ __forceinline__ void store_codes_raw(uint8_t* dst, const float2* v) {
+  const float* f = reinterpret_cast<const float*>(v);
+  if (P == 8)
+    *reinterpret_cast<uint2*>(dst) = e4m3x8(f);
+  else
+    *reinterpret_cast<uint32_t*>(dst) = e4m3x4(f[0], f[1], f[2], f[3]);
+}
+
 // One head's LayerNorm on a lane's packed pairs (NEXT-4): the mean, then the
 // centred sum of squares (each an xor shuffle over the GP lanes of the group;
 // every lane of the warp takes part), then x = (x - mean) * rstd * w + bias in
@@ -167,14 +177,16 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
   // Constant inputs before the wait for the previous kernel: the position,
   // the lane's cos/sin slice at that position (two dependent loads, off the
   // critical path this way), the norm weights and the e4m3 cache scales.
-  const int p = __ldg(positions + tok);
+  const int64_t M = gridDim.x / nhb;  // extents for the bounds-checked build
+  const int p = FRT_IDX_OK(tok, M) ? __ldg(positions + tok) : -1;
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
   const bool active = lane_ok && row_ok;
   constexpr int NP = P / 2;
   float2 cs[NP], sn[NP], nsn[NP];
-  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
+  if (active && FRT_SPAN_OK((int64_t)p * half + j0, P, (int64_t)max_pos * half))
+    load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
   V qwa, qwb, kwa, kwb;
-  if (HPG == 1 && lane_ok) {
+  if (HPG == 1 && lane_ok && FRT_SPAN_OK(j0, half + P, hd)) {
     if (q_norm_w != nullptr) {
       qwa = ld_vec<P>(q_norm_w + j0);
       qwb = ld_vec<P>(q_norm_w + half + j0);
@@ -184,15 +196,16 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
       kwb = ld_vec<P>(k_norm_w + half + j0);
     }
   }
-  const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
-  const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
+  const float k_inv = KV8 && FRT_IDX_OK(0, 2) ? __frcp_rn(__ldg(ep.kv_scales)) : 1.0f;  // RN(1 / k_scale)
+  const float v_scale = KV8 && FRT_IDX_OK(1, 2) ? __ldg(ep.kv_scales + 1) : 1.0f;
   pdl_enter();
   const uint16_t* row = qkv + (int64_t)tok * H * hd;
+  const int64_t n_qkv = M * H * hd, n_q = M * Hq * hd, n_kv = (int64_t)capacity * Hkv * hd;
   V va[HPG], vb[HPG];
 #pragma unroll
   for (int i = 0; i < HPG; ++i) {
     const int h = (hb * hpg + i) * NG + grp;
-    if (lane_ok && i < hpg && h < H) {
+    if (lane_ok && i < hpg && h < H && FRT_SPAN_OK((int64_t)tok * H * hd + (int64_t)h * hd + j0, half + P, n_qkv)) {
       va[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + j0);
       vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
     }
@@ -208,7 +221,8 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
     const bool is_v = h >= Hq + Hkv;
     const uint16_t* nw = is_q ? q_norm_w : k_norm_w;
     const bool do_norm = !is_v && nw != nullptr;
-    if (on && is_v) {  // V: bit copy into the cache slot (or its e4m3 codes)
+    if (on && is_v && FRT_SPAN_OK(((int64_t)p * Hkv + (h - Hq - Hkv)) * hd + j0, half + P, n_kv)) {
+      // V: bit copy into the cache slot (or its e4m3 codes)
       const int64_t off = ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
       if (KV8) {
         float a[P], b[P];
@@ -233,15 +247,26 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
     }
     ss = group_sum<GP>(ss);  // every lane of the warp takes part
     if (on && !is_v) {
+      // the Q epilogue's scale and, with e4m3 caches, RN(1 / k_scale) ride on
+      // the head's norm factor (a product per element otherwise)
+      const float post = (QEPI && is_q) ? ep.q_scale : (KV8 && !is_q) ? k_inv : 1.0f;
+      if (!do_norm && ((QEPI && is_q) || (KV8 && !is_q))) {
+        mul_pairs<NP>(a, post);
+        mul_pairs<NP>(b, post);
+      }
       if (do_norm) {
-        const float rstd = head_rstd(ss, inv_hd, eps);
+        const float rstd = head_rstd(ss, inv_hd, eps) * post;
         float2 fa[NP], fb[NP];
         if (HPG == 1) {  // weights already in registers
           const V wa = is_q ? qwa : kwa, wb = is_q ? qwb : kwb;
           unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wa), fa);
           unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wb), fb);
         } else {
-          const V wa = ld_vec<P>(nw + j0), wb = ld_vec<P>(nw + half + j0);
+          V wa, wb;
+          if (FRT_SPAN_OK(j0, half + P, hd)) {
+            wa = ld_vec<P>(nw + j0);
+            wb = ld_vec<P>(nw + half + j0);
+          }
           unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wa), fa);
           unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wb), fb);
         }
@@ -251,20 +276,18 @@ __global__ void __launch_bounds__(reg_kernel_threads<HPG, EPI>()) qkv_norm_rope_
       float2 o1[NP], o2[NP];
       rope_pairs<NP>(a, b, cs, sn, nsn, o1, o2);
       if (is_q) {
-        if (QEPI) {
-          mul_pairs<NP>(o1, ep.q_scale);
-          mul_pairs<NP>(o2, ep.q_scale);
+        const int64_t qo = (QEPI ? q_row(ep, tok, h, Hq) : (int64_t)tok * Hq + h) * hd;
+        uint16_t* dst = q_out + qo;
+        if (FRT_SPAN_OK(qo + j0, half + P, n_q)) {
+          store_pairs<DT, P>(dst + j0, o1);
+          store_pairs<DT, P>(dst + half + j0, o2);
         }
-        uint16_t* dst = q_out + (QEPI ? q_row(ep, tok, h, Hq) : (int64_t)tok * Hq + h) * hd;
-        store_pairs<DT, P>(dst + j0, o1);
-        store_pairs<DT, P>(dst + half + j0, o2);
-      } else {
+      } else if (FRT_SPAN_OK(((int64_t)p * Hkv + (h - Hq)) * hd + j0, half + P, n_kv)) {
         const int64_t off = ((int64_t)p * Hkv + (h - Hq)) * hd;
-        if (KV8) {
+        if (KV8) {  // already divided by k_scale
           uint8_t* dst = static_cast<uint8_t*>(k_cache) + off;
-          const Divisor dk(k_scale);
-          store_codes<P>(dst + j0, reinterpret_cast<const float*>(o1), dk);
-          store_codes<P>(dst + half + j0, reinterpret_cast<const float*>(o2), dk);
+          store_codes_raw<P>(dst + j0, o1);
+          store_codes_raw<P>(dst + half + j0, o2);
         } else {
           uint16_t* dst = static_cast<uint16_t*>(k_cache) + off;
           store_pairs<DT, P>(dst + j0, o1);
@@ -321,11 +344,12 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
       const uint16_t* pw = is_q ? q_norm_w : k_norm_w;
       const uint16_t* pb = is_q ? ep.q_bias : ep.k_bias;
       V wa, wb, ba, bb;
-      if (on && pw != nullptr) {
+      const int64_t n_aff = (int64_t)(is_q ? Hq : Hkv) * hd;  // per-head affine rows [Hq | Hkv, hd]
+      if (on && pw != nullptr && FRT_SPAN_OK(off + j0, half + P, n_aff)) {
         wa = ld_vec<P>(pw + off + j0);
         wb = ld_vec<P>(pw + off + half + j0);
       }
-      if (on && pb != nullptr) {
+      if (on && pb != nullptr && FRT_SPAN_OK(off + j0, half + P, n_aff)) {
         ba = ld_vec<P>(pb + off + j0);
         bb = ld_vec<P>(pb + off + half + j0);
       }
@@ -363,14 +387,20 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
       store_codes<P>(dst + j0, reinterpret_cast<const float*>(x1), dvs);
       store_codes<P>(dst + half + j0, reinterpret_cast<const float*>(x2), dvs);
     } else if (on) {
+      // the Q epilogue's scale and, with e4m3 caches, RN(1 / k_scale) ride on
+      // the head's norm factor (a product per element otherwise)
+      const float post = (QEPI && is_q) ? ep.q_scale : (KV8 && !is_q) ? kvs[1] : 1.0f;
       if (nwg != nullptr) {
-        const float rstd = head_rstd(ss, inv_hd, eps);
+        const float rstd = head_rstd(ss, inv_hd, eps) * post;
         const V wa = *reinterpret_cast<const V*>(nws + j0), wb = *reinterpret_cast<const V*>(nws + half + j0);
         float2 fa[NP], fb[NP];
         unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wa), fa);
         unpack_pairs<DT, NP>(reinterpret_cast<const uint32_t*>(&wb), fb);
         scale_pairs<NP>(x1, rstd, fa);
         scale_pairs<NP>(x2, rstd, fb);
+      } else if ((QEPI && is_q) || (KV8 && !is_q)) {
+        mul_pairs<NP>(x1, post);
+        mul_pairs<NP>(x2, post);
       }
       // this slot's cos, sin and -sin slices from shared memory
       float2 cs[NP], sn[NP], nsn[NP];
@@ -379,19 +409,16 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
       ld_pairs_smem<NP>(nsbuf + j0, nsn);
       float2 o1[NP], o2[NP];
       rope_pairs<NP>(x1, x2, cs, sn, nsn, o1, o2);
-      if (QEPI && is_q) {
-        mul_pairs<NP>(o1, ep.q_scale);
-        mul_pairs<NP>(o2, ep.q_scale);
-      }
-      if (KV8 && !is_q) {
+      if (KV8 && !is_q) {  // already divided by k_scale
         uint8_t* dst = k8buf + (h - Hq) * hd;
-        const Divisor dk(kvs[0], kvs[1]);
-        store_codes<P>(dst + j0, reinterpret_cast<const float*>(o1), dk);
-        store_codes<P>(dst + half + j0, reinterpret_cast<const float*>(o2), dk);
+        store_codes_raw<P>(dst + j0, o1);
+        store_codes_raw<P>(dst + half + j0, o2);
       } else if (q_direct && is_q) {
         uint16_t* dst = q_out + ((int64_t)h * ep.M + tok) * hd;
-        store_pairs<DT, P>(dst + j0, o1);
-        store_pairs<DT, P>(dst + half + j0, o2);
+        if (FRT_SPAN_OK(((int64_t)h * ep.M + tok) * hd + j0, half + P, (int64_t)Hq * ep.M * hd)) {
+          store_pairs<DT, P>(dst + j0, o1);
+          store_pairs<DT, P>(dst + half + j0, o2);
+        }
       } else {
         store_pairs<DT, P>(vec + j0, o1);
         store_pairs<DT, P>(vec + half + j0, o2);
@@ -406,9 +433,12 @@ __device__ __forceinline__ void process_token(uint16_t* rowbuf, const float* cbu
 template <int EPI>
 __device__ __forceinline__ void store_token(const uint16_t* rowbuf, const uint8_t* k8buf, const uint8_t* v8buf,
                                             uint16_t* q_out, void* k_cache, void* v_cache, int tok, int p, int Hq,
-                                            int Hkv, int hd, const Epilogue& ep) {
-  if (!((EPI == 1 || EPI == 2) && ep.q_head_major))
+                                            int Hkv, int hd, int capacity, const Epilogue& ep) {
+  const int64_t n_kv = (int64_t)capacity * Hkv * hd;
+  if (!((EPI == 1 || EPI == 2) && ep.q_head_major) &&
+      FRT_SPAN_OK((int64_t)tok * Hq * hd, Hq * hd, (int64_t)ep.M * Hq * hd))
     bulk_store(q_out + (int64_t)tok * Hq * hd, rowbuf, (unsigned)(Hq * hd * 2));
+  if (!FRT_SPAN_OK((int64_t)p * Hkv * hd, Hkv * hd, n_kv)) return;
   if (EPI == 2) {
     bulk_store(static_cast<uint8_t*>(k_cache) + (int64_t)p * Hkv * hd, k8buf, (unsigned)(Hkv * hd));
     bulk_store(static_cast<uint8_t*>(v_cache) + (int64_t)p * Hkv * hd, v8buf, (unsigned)(Hkv * hd));
@@ -445,19 +475,22 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
   const bool lane_ok = threadIdx.x < (unsigned)(NG * GP) && li < G;
   // the position and the lane's cos/sin slice are constant inputs: read
   // before the wait for the previous kernel
-  const int p = __ldg(positions + tok);
+  const int64_t M = gridDim.x / nhb;  // extents for the bounds-checked build
+  const int p = FRT_IDX_OK(tok, M) ? __ldg(positions + tok) : -1;
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
   const bool active = lane_ok && row_ok;
   constexpr int NP = P / 2;
   float2 cs[NP], sn[NP], nsn[NP];
-  if (active) load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
+  if (active && FRT_SPAN_OK((int64_t)p * half + j0, P, (int64_t)max_pos * half))
+    load_rope_pairs<NP>(cos_tab + (int64_t)p * half + j0, sin_tab + (int64_t)p * half + j0, cs, sn, nsn);
   pdl_enter();
   const uint16_t* row = qkv + (int64_t)tok * H * hd;
+  const int64_t n_kv = (int64_t)capacity * Hkv * hd;
   V va[HPG], vb[HPG];
 #pragma unroll
   for (int i = 0; i < HPG; ++i) {
     const int h = (hb * HPG + i) * NG + grp;
-    if (lane_ok && h < H) {
+    if (lane_ok && h < H && FRT_SPAN_OK((int64_t)tok * H * hd + (int64_t)h * hd + j0, half + P, M * H * hd)) {
       va[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + j0);
       vb[i] = *reinterpret_cast<const V*>(row + (int64_t)h * hd + half + j0);
     }
@@ -470,7 +503,8 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
     const bool on = active && h < H;
     const bool is_q = h < Hq;
     const bool is_v = h >= Hq + Hkv;
-    if (on && is_v) {  // V: bit copy into the cache slot
+    if (on && is_v && FRT_SPAN_OK(((int64_t)p * Hkv + (h - Hq - Hkv)) * hd + j0, half + P, n_kv)) {
+      // V: bit copy into the cache slot
       uint16_t* dst = v_cache + ((int64_t)p * Hkv + (h - Hq - Hkv)) * hd;
       *reinterpret_cast<V*>(dst + j0) = va[i];
       *reinterpret_cast<V*>(dst + half + j0) = vb[i];
@@ -485,11 +519,12 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
     const uint16_t* pw = is_q ? q_w : k_w;
     const uint16_t* pb = is_q ? q_b : k_b;
     V wa, wb, ba, bb;
-    if (qk && pw != nullptr) {
+    const int64_t n_aff = (int64_t)(is_q ? Hq : Hkv) * hd;  // per-head affine rows
+    if (qk && pw != nullptr && FRT_SPAN_OK((int64_t)hh * hd + j0, half + P, n_aff)) {
       wa = ld_vec<P>(pw + (int64_t)hh * hd + j0);
       wb = ld_vec<P>(pw + (int64_t)hh * hd + half + j0);
     }
-    if (qk && pb != nullptr) {
+    if (qk && pb != nullptr && FRT_SPAN_OK((int64_t)hh * hd + j0, half + P, n_aff)) {
       ba = ld_vec<P>(pb + (int64_t)hh * hd + j0);
       bb = ld_vec<P>(pb + (int64_t)hh * hd + half + j0);
     }
@@ -500,9 +535,12 @@ __global__ void __launch_bounds__(HPG == 1 ? 512 : 256) qkv_layernorm_rope_kvcac
     if (qk) {
       float2 o1[NP], o2[NP];
       rope_pairs<NP>(a, b, cs, sn, nsn, o1, o2);
-      uint16_t* dst = is_q ? q_out + ((int64_t)tok * Hq + h) * hd : k_cache + ((int64_t)p * Hkv + hh) * hd;
-      store_pairs<DT, P>(dst + j0, o1);
-      store_pairs<DT, P>(dst + half + j0, o2);
+      const int64_t o = is_q ? ((int64_t)tok * Hq + h) * hd : ((int64_t)p * Hkv + hh) * hd;
+      uint16_t* dst = (is_q ? q_out : k_cache) + o;
+      if (FRT_SPAN_OK(o + j0, half + P, is_q ? M * Hq * hd : n_kv)) {
+        store_pairs<DT, P>(dst + j0, o1);
+        store_pairs<DT, P>(dst + half + j0, o2);
+      }
     }
   }
 }
@@ -544,21 +582,23 @@ __global__ void __launch_bounds__(512) qkv_generic_kernel(
   const int lane = threadIdx.x & 31;
   const int half = hd >> 1;
   // constant inputs before the wait for the previous kernel
-  const int p = __ldg(positions + tok);
+  const int64_t M = gridDim.x;  // extents for the bounds-checked build
+  const int p = FRT_IDX_OK(tok, M) ? __ldg(positions + tok) : -1;
   const bool row_ok = p >= 0 && p < max_pos && p < capacity;
   float cs[kGenericMaxK], sn[kGenericMaxK];
 #pragma unroll
   for (int k = 0; k < kGenericMaxK; ++k) {
     const int j = lane + 32 * k;
     cs[k] = sn[k] = 0.0f;
-    if (row_ok && j < half) {
+    if (row_ok && j < half && FRT_IDX_OK((int64_t)p * half + j, (int64_t)max_pos * half)) {
       cs[k] = __ldg(cos_tab + (int64_t)p * half + j);
       sn[k] = __ldg(sin_tab + (int64_t)p * half + j);
     }
   }
-  const float k_scale = KV8 ? __ldg(ep.kv_scales) : 1.0f;
-  const float v_scale = KV8 ? __ldg(ep.kv_scales + 1) : 1.0f;
+  const float k_scale = KV8 && FRT_IDX_OK(0, 2) ? __ldg(ep.kv_scales) : 1.0f;
+  const float v_scale = KV8 && FRT_IDX_OK(1, 2) ? __ldg(ep.kv_scales + 1) : 1.0f;
   pdl_enter();
+  const int64_t n_qkv = M * H * hd, n_q = M * Hq * hd, n_kv = (int64_t)capacity * Hkv * hd;
   if (!row_ok) {
     if (threadIdx.x == 0 && status != nullptr) atomicOr(status, 1);
     return;
@@ -575,7 +615,7 @@ __global__ void __launch_bounds__(512) qkv_generic_kernel(
     for (int k = 0; k < kGenericMaxK; ++k) {
       const int j = lane + 32 * k;
       a[k] = b[k] = 0.0f;
-      if (j < half) {
+      if (j < half && FRT_SPAN_OK((int64_t)tok * H * hd + (int64_t)h * hd + j, half + 1, n_qkv)) {
         a[k] = ld16<DT>(row + (int64_t)h * hd + j);
         b[k] = ld16<DT>(row + (int64_t)h * hd + half + j);
       }
@@ -585,7 +625,7 @@ __global__ void __launch_bounds__(512) qkv_generic_kernel(
 #pragma unroll
       for (int k = 0; k < kGenericMaxK; ++k) {
         const int j = lane + 32 * k;
-        if (j >= half) continue;
+        if (j >= half || !FRT_SPAN_OK(cache_off + j, half + 1, n_kv)) continue;
         if (KV8) {
           uint8_t* dst = static_cast<uint8_t*>(v_cache) + cache_off;
           dst[j] = (uint8_t)(e4m3x2(dv.fast ? dv.div(a[k]) : dv.div_slow(a[k]), 0.0f) & 0xFFu);
@@ -620,8 +660,10 @@ __global__ void __launch_bounds__(512) qkv_generic_kernel(
         const int j = lane + 32 * k;
         if (j >= half) continue;
         const int64_t o = (int64_t)hh * hd;
-        const float w1 = w ? ld16<DT>(w + o + j) : 1.0f, w2 = w ? ld16<DT>(w + o + half + j) : 1.0f;
-        const float b1 = bias ? ld16<DT>(bias + o + j) : 0.0f, b2 = bias ? ld16<DT>(bias + o + half + j) : 0.0f;
+        const bool aff_ok = FRT_SPAN_OK(o + j, half + 1, (int64_t)(is_q ? Hq : Hkv) * hd);  // rows [Hq | Hkv, hd]
+        const float w1 = w && aff_ok ? ld16<DT>(w + o + j) : 1.0f, w2 = w && aff_ok ? ld16<DT>(w + o + half + j) : 1.0f;
+        const float b1 = bias && aff_ok ? ld16<DT>(bias + o + j) : 0.0f;
+        const float b2 = bias && aff_ok ? ld16<DT>(bias + o + half + j) : 0.0f;
         a[k] = fmaf(a[k] * r, w1, b1);
         b[k] = fmaf(b[k] * r, w2, b2);
       }
@@ -633,7 +675,7 @@ __global__ void __launch_bounds__(512) qkv_generic_kernel(
 #pragma unroll
       for (int k = 0; k < kGenericMaxK; ++k) {
         const int j = lane + 32 * k;
-        if (j >= half) continue;
+        if (j >= half || !FRT_SPAN_OK(j, half + 1, hd)) continue;
         a[k] = (a[k] * r) * ld16<DT>(w + j);
         b[k] = (b[k] * r) * ld16<DT>(w + half + j);
       }
@@ -649,9 +691,12 @@ __global__ void __launch_bounds__(512) qkv_generic_kernel(
           o1 *= ep.q_scale;
           o2 *= ep.q_scale;
         }
-        uint16_t* dst = q_out + (QEPI ? q_row(ep, tok, h, Hq) : (int64_t)tok * Hq + h) * hd;
-        st16<DT>(dst + j, o1);
-        st16<DT>(dst + half + j, o2);
+        const int64_t qo = (QEPI ? q_row(ep, tok, h, Hq) : (int64_t)tok * Hq + h) * hd;
+        if (!FRT_SPAN_OK(qo + j, half + 1, n_q)) continue;
+        st16<DT>(q_out + qo + j, o1);
+        st16<DT>(q_out + qo + half + j, o2);
+      } else if (!FRT_SPAN_OK(cache_off + j, half + 1, n_kv)) {
+        continue;
       } else if (KV8) {
         uint8_t* dst = static_cast<uint8_t*>(k_cache) + cache_off;
         dst[j] = (uint8_t)(e4m3x2(dk.fast ? dk.div(o1) : dk.div_slow(o1), 0.0f) & 0xFFu);
@@ -748,16 +793,22 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
   __syncthreads();
   if (tid == 0) {
     const bool stage_w = EPI != 3;  // LayerNorm rows are per head: read from global memory instead
+    // (bounds-checked build: a row outside the QKV buffer is not copied and
+    // the token is skipped like a bad position, without the status bit)
+    const bool in_b = FRT_SPAN_OK((int64_t)tok * H * hd, H * hd, (int64_t)gridDim.x * H * hd);
     const unsigned first =
-        row_bytes + (stage_w && q_norm_w ? w_bytes : 0u) + (stage_w && k_norm_w ? w_bytes : 0u);
+        in_b ? row_bytes + (stage_w && q_norm_w ? w_bytes : 0u) + (stage_w && k_norm_w ? w_bytes : 0u) : 0u;
     mbar_arrive_expect_tx(&bar, first);
-    bulk_load(rowbuf, qkv + (int64_t)tok * H * hd, row_bytes, &bar);
-    if (stage_w && q_norm_w) bulk_load(qwbuf, q_norm_w, w_bytes, &bar);
-    if (stage_w && k_norm_w) bulk_load(kwbuf, k_norm_w, w_bytes, &bar);
-    const int p = __ldg(positions + tok);
-    const bool ok = p >= 0 && p < max_pos && p < capacity;
+    if (in_b) {
+      bulk_load(rowbuf, qkv + (int64_t)tok * H * hd, row_bytes, &bar);
+      if (stage_w && q_norm_w) bulk_load(qwbuf, q_norm_w, w_bytes, &bar);
+      if (stage_w && k_norm_w) bulk_load(kwbuf, k_norm_w, w_bytes, &bar);
+    }
+    const int p = in_b ? __ldg(positions + tok) : -1;
+    const bool ok = p >= 0 && p < max_pos && p < capacity &&
+                    FRT_SPAN_OK((int64_t)p * half, half, (int64_t)max_pos * half);
     s_pos = ok ? p : -1;
-    if (EPI == 2) {
+    if (EPI == 2 && FRT_SPAN_OK(0, 2, 2)) {
       const float ks = __ldg(ep.kv_scales), vs = __ldg(ep.kv_scales + 1);
       s_kv[0] = ks;
       s_kv[1] = __frcp_rn(ks);
@@ -769,7 +820,7 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
       bulk_load(cbuf, cos_tab + (int64_t)p * half, tab_bytes, &bar);
       bulk_load(sbuf, sin_tab + (int64_t)p * half, tab_bytes, &bar);
     } else {
-      if (status != nullptr) atomicOr(status, 1);
+      if (status != nullptr && in_b) atomicOr(status, 1);
       mbar_arrive_expect_tx(&bar, 0u);
     }
   }
@@ -793,7 +844,7 @@ __global__ void __launch_bounds__(128, tma_min_blocks<EPI>()) qkv_norm_rope_kvca
   fence_proxy_async_smem();  // this thread's writes -> the bulk stores below
   __syncthreads();
   if (tid == 0) {
-    store_token<EPI>(rowbuf, k8buf, v8buf, q_out, k_cache, v_cache, tok, p, Hq, Hkv, hd, ep);
+    store_token<EPI>(rowbuf, k8buf, v8buf, q_out, k_cache, v_cache, tok, p, Hq, Hkv, hd, capacity, ep);
     bulk_commit();
     bulk_wait_read();  // shared memory must outlive the stores' reads
   }

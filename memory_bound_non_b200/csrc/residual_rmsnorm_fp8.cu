@@ -25,21 +25,26 @@
 namespace frt {
 namespace {
 
-// Threads per CTA: at most 128 for K <= 2, 512 for K >= 4 (128 at D = 4096).
-// Small CTAs keep many rows in flight per SM, which is what hides each row's
-// load -> reduce -> quantise latency.
+// Threads per CTA: at most 128 for K = 2, 512 for K >= 4 (128 at D = 4096)
+// and for K = 1 (one chunk per thread: the small-batch shape, up to D =
+// 4096).  Small CTAs keep many rows in flight per SM, which is what hides
+// each row's load -> reduce -> quantise latency on large batches.
 template <int K>
 constexpr int max_threads() {
-  return K >= 4 ? 512 : 128;
+  return K == 2 ? 128 : 512;
 }
 
 // LN (NEXT-4, the ViT "add_layer_norm" producer): LayerNorm instead of
-// RMSNorm, y = (h - mean) * rstd * w + b (bias may be null).  The row sum and
-// the centred sum of squares are two reductions over the register-held row
-// (fp32 per thread, fp64 across threads); per element h - mean is formed
-// against the mean split into two floats (error ~1 ulp of the difference, so
-// a large common offset in the row costs no accuracy) and y carries a few
-// fp32 roundings (FP8 codes are 2^-4 apart).
+// RMSNorm, y = (h - mean) * rstd * w + b (bias may be null).  One pass over
+// the register-held row sums h and h^2 in fp64 (every square of a 16-bit
+// value is exact in fp64, and so are the sums short of an extreme exponent
+// spread); var = E[h^2] - mean^2 in fp64 then loses at most a few fp64 ulps of
+// the mean^2 / var ratio, far below the fp32 the output carries.  Per element
+// h - mean is formed against the mean split into two floats (error ~1 ulp of
+// the difference, so a large common offset costs no accuracy) on packed fp32
+// pairs, and y carries a few fp32 roundings (FP8 codes are 2^-4 apart); with
+// a static scale 1 / s is folded into rstd and the bias, as the RMS path
+// folds it into rstd.
 template <int DT, int K, bool WEIGHTED, int QM, bool LN>
 __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     const uint4* __restrict__ x, const uint4* r_in, uint4* r_out, const uint4* __restrict__ w,
@@ -57,15 +62,16 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   // latency-bound calls), the weight, so neither is on the critical path.
   // Wide rows load the weight after the reduction and keep the registers
   // for occupancy.
+  const int64_t n_rc = (int64_t)gridDim.x * C;  // 16-byte chunks of x, r_in, r_out (and 8-byte ones of q)
   float s_static = 0.0f;
-  if (QM == FRT_QUANT_STATIC || QM >= kQuantNvfp4Rows) s_static = __ldg(static_scale);
-  const double inv_s64 = QM == FRT_QUANT_STATIC && !LN ? 1.0 / (double)s_static : 0.0;
+  if ((QM == FRT_QUANT_STATIC || QM >= kQuantNvfp4Rows) && FRT_IDX_OK(0, 1)) s_static = __ldg(static_scale);
+  const double inv_s64 = QM == FRT_QUANT_STATIC ? 1.0 / (double)s_static : 0.0;
   constexpr bool kEarlyWeight = WEIGHTED && K <= 2;
   uint4 wv_early[kEarlyWeight ? K : 1];
   if (kEarlyWeight) {
 #pragma unroll
     for (int k = 0; k < K; ++k)
-      if (t + k * T < C) wv_early[k] = __ldg(w + t + k * T);
+      if (t + k * T < C && FRT_IDX_OK(t + k * T, C)) wv_early[k] = __ldg(w + t + k * T);
   }
   pdl_enter();
 
@@ -74,7 +80,7 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = t + k * T;
-    if (c < C) {
+    if (c < C && FRT_IDX_OK(base + c, n_rc)) {
       xv[k] = ld_stream(x + base + c);
       rv[k] = ld_plain(r_in + base + c);
     }
@@ -84,10 +90,11 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   // sum), kept packed; fp64 sum of squares (squares of 16-bit values are
   // exact, so the sum is exact to ~2^-40), one accumulator per chunk.
   uint4 hv[K];
-  double ss[K];
+  double ss[K], sm[LN ? K : 1];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     ss[k] = 0.0;
+    if (LN) sm[LN ? k : 0] = 0.0;
     const int c = t + k * T;
     if (c < C) {
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv[k]);
@@ -100,21 +107,22 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 hf = P16::to_float2(hw[e]);
-        if (LN) {  // the row sum first (the centred squares need the mean)
-          ss[k] += (double)(hf.x + hf.y);
-        } else {
-          ss[k] = fma((double)hf.x, (double)hf.x, ss[k]);
-          ss[k] = fma((double)hf.y, (double)hf.y, ss[k]);
-        }
+        const double h0 = (double)hf.x, h1 = (double)hf.y;
+        ss[k] = fma(h0, h0, ss[k]);
+        ss[k] = fma(h1, h1, ss[k]);
+        if (LN) sm[LN ? k : 0] += h0 + h1;  // exact: two 16-bit values
       }
-      r_out[base + c] = hv[k];
+      if (FRT_IDX_OK(base + c, n_rc)) r_out[base + c] = hv[k];
     } else {
       hv[k] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  double sst = ss[0];
+  double sst = ss[0], smt = LN ? sm[0] : 0.0;
 #pragma unroll
-  for (int k = 1; k < K; ++k) sst += ss[k];
+  for (int k = 1; k < K; ++k) {
+    sst += ss[k];
+    if (LN) smt += sm[LN ? k : 0];
+  }
 
   // Row total: warp butterfly, then every thread adds the warp partials in
   // the same order and forms rstd in fp64.  y = h * w * rstd is rounded once
@@ -122,49 +130,41 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
   // rounded fp32 value of the exact normalised element and the FP8 codes are
   // decided on the value an exact computation would give.
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sst += __shfl_xor_sync(0xFFFFFFFFu, sst, o);
-  if ((t & 31) == 0) red[t >> 5] = sst;
+  for (int o = 16; o > 0; o >>= 1) {
+    sst += __shfl_xor_sync(0xFFFFFFFFu, sst, o);
+    if (LN) smt += __shfl_xor_sync(0xFFFFFFFFu, smt, o);
+  }
+  if ((t & 31) == 0) {
+    red[t >> 5] = sst;
+    if (LN) red[16 + (t >> 5)] = smt;
+  }
   __syncthreads();
-  double tot = 0.0;
+  double tot = 0.0, tsum = 0.0;
   const int nw = T >> 5;
-  for (int i = 0; i < nw; ++i) tot += red[i];
+  for (int i = 0; i < nw; ++i) {
+    tot += red[i];
+    if (LN) tsum += red[16 + i];
+  }
   float mean_hi = 0.0f, mean_lo = 0.0f;
+  double var = tot / (double)D;  // RMSNorm: the mean square
   if (LN) {
-    // second reduction: the centred sum of squares of the held row
-    const double mean = tot / (double)D;
+    const double mean = tsum / (double)D;
+    var = fmax(var - mean * mean, 0.0);
     mean_hi = (float)mean;
     mean_lo = (float)(mean - (double)mean_hi);
-    float scf = 0.0f;
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      if (t + k * T < C) {
-        const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv[k]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 hf = P16::to_float2(hw[e]);
-          const float d0 = (hf.x - mean_hi) - mean_lo, d1 = (hf.y - mean_hi) - mean_lo;
-          scf = fmaf(d0, d0, fmaf(d1, d1, scf));
-        }
-      }
-    }
-    double sc = (double)scf;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, o);
-    __syncthreads();  // every thread has read the first partials
-    if ((t & 31) == 0) red[t >> 5] = sc;
-    __syncthreads();
-    tot = 0.0;
-    for (int i = 0; i < nw; ++i) tot += red[i];
   }
-  const double rstd64 = rsqrt_f64(tot / (double)D + (double)eps);
+  const double rstd64 = rsqrt_f64(var + (double)eps);
   // Static FP8 on the RMS path: y / s as one product with rstd / s (fp64,
   // held as an fp32 pair), so each code is decided on one fp32 rounding of
   // h w rstd / s rather than on RN(RN(h w rstd) / s).  A ratio outside
   // [2^-100, 2^100] keeps y and the division.
   const double rs64 = rstd64 * inv_s64;
-  const bool fold = QM == FRT_QUANT_STATIC && !LN && rs64 >= 0x1p-100 && rs64 <= 0x1p+100;
+  const bool fold = QM == FRT_QUANT_STATIC && rs64 >= 0x1p-100 && rs64 <= 0x1p+100;
   const Split32 rstd(fold ? rs64 : rstd64);
-  const float rstd32 = (float)rstd64;
+  // LayerNorm: rstd (/ s when folded) and the bias factor (1 / s when folded)
+  const float2 rstd2 = make_float2((float)(fold ? rs64 : rstd64), (float)(fold ? rs64 : rstd64));
+  const float2 bfac2 = make_float2(fold ? (float)inv_s64 : 1.0f, fold ? (float)inv_s64 : 1.0f);
+  const float2 nmhi2 = make_float2(-mean_hi, -mean_hi), nmlo2 = make_float2(-mean_lo, -mean_lo);
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
   const float rden = QM >= kQuantNvfp4Rows ? __frcp_rn(6.0f * s_static) : 0.0f;  // NVFP4: RN(1 / RN(6 gs))
 
@@ -178,8 +178,8 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
     if (LN) {
       uint4 wv = make_uint4(0u, 0u, 0u, 0u), bv = make_uint4(0u, 0u, 0u, 0u);
       if (valid) {
-        if (WEIGHTED) wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : __ldg(w + c);
-        if (bias != nullptr) bv = __ldg(bias + c);
+        if (WEIGHTED && FRT_IDX_OK(c, C)) wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : __ldg(w + c);
+        if (bias != nullptr && FRT_IDX_OK(c, C)) bv = __ldg(bias + c);
       }
       const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv);
       const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv);
@@ -187,15 +187,16 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       for (int e = 0; e < 4; ++e) {
         const float2 hf = P16::to_float2(hw[e]);
         const float2 wf = WEIGHTED ? P16::to_float2(ww[e]) : make_float2(1.0f, 1.0f);
-        const float2 bf = P16::to_float2(bw[e]);
-        const float d0 = ((hf.x - mean_hi) - mean_lo) * rstd32, d1 = ((hf.y - mean_hi) - mean_lo) * rstd32;
-        // bias zeros when absent; lanes past the row end hold 0 (they take
-        // part in the block amax)
-        y[2 * e] = valid ? fmaf(d0, wf.x, bf.x) : 0.0f;
-        y[2 * e + 1] = valid ? fmaf(d1, wf.y, bf.y) : 0.0f;
+        // (h - mean) rstd w + b, on packed pairs; bias zeros when absent
+        const float2 d = __fmul2_rn(__fadd2_rn(__fadd2_rn(hf, nmhi2), nmlo2), rstd2);
+        const float2 yy = __ffma2_rn(d, wf, __fmul2_rn(P16::to_float2(bw[e]), bfac2));
+        // lanes past the row end hold 0 (they take part in the block amax)
+        y[2 * e] = valid ? yy.x : 0.0f;
+        y[2 * e + 1] = valid ? yy.y : 0.0f;
       }
     } else if (WEIGHTED && valid) {
-      const uint4 wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : __ldg(w + c);
+      const uint4 wv = kEarlyWeight ? wv_early[kEarlyWeight ? k : 0] : FRT_IDX_OK(c, C) ? __ldg(w + c)
+                                                                                        : make_uint4(0u, 0u, 0u, 0u);
       const uint32_t* ww = reinterpret_cast<const uint32_t*>(&wv);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -216,8 +217,9 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       float am = fmaxf(absmax4(y[0], y[1], y[2], y[3]), absmax4(y[4], y[5], y[6], y[7]));
       am = half_warp_max_abs(am);  // 16 lanes = the 16 chunks of one 128-column block
       const float sb = block_scale_448(am);
-      if (valid && (t & 15) == 0) block_scales[row * NB + (c >> 4)] = sb;
-      if (valid) q[base + c] = quant8(y, Divisor(sb));
+      if (valid && (t & 15) == 0 && FRT_IDX_OK(row * NB + (c >> 4), (int64_t)gridDim.x * NB))
+        block_scales[row * NB + (c >> 4)] = sb;
+      if (valid && FRT_IDX_OK(base + c, n_rc)) q[base + c] = quant8(y, Divisor(sb));
     } else if (QM >= kQuantNvfp4Rows) {
       // NVFP4: a 16-element block is chunks 2b and 2b+1, held by lanes t and
       // t ^ 1; codes leave as one 32-bit word per chunk, the scale factor from
@@ -227,14 +229,18 @@ __global__ void __launch_bounds__(max_threads<K>()) residual_rmsnorm_fp8_kernel(
       float reff;
       const uint32_t sf = nvfp4_scale(am, rden, s_static, &reff);
       if (valid) {
-        reinterpret_cast<uint32_t*>(q)[base + c] = nvfp4_codes<8>(y, reff);
+        if (FRT_IDX_OK(base + c, n_rc)) reinterpret_cast<uint32_t*>(q)[base + c] = nvfp4_codes<8>(y, reff);
         if ((c & 1) == 0) {
           uint8_t* sfo = reinterpret_cast<uint8_t*>(block_scales);
           const int nsf = C >> 1;
-          sfo[QM == kQuantNvfp4Rows ? row * nsf + (c >> 1) : sf_offset_swizzled(row, c >> 1, nsf)] = (uint8_t)sf;
+          const int64_t o = QM == kQuantNvfp4Rows ? row * nsf + (c >> 1) : sf_offset_swizzled(row, c >> 1, nsf);
+          // row-major [M, nsf]; swizzled: 128-row x 4-column atoms
+          const int64_t n_sf = QM == kQuantNvfp4Rows ? (int64_t)gridDim.x * nsf
+                                                     : (((int64_t)gridDim.x + 127) / 128) * 128 * ((nsf + 3) / 4) * 4;
+          if (FRT_IDX_OK(o, n_sf)) sfo[o] = (uint8_t)sf;
         }
       }
-    } else if (valid) {
+    } else if (valid && FRT_IDX_OK(base + c, n_rc)) {
       q[base + c] = fold ? e4m3x8(y) : quant8(y, dv_static);
     }
   }
@@ -288,11 +294,15 @@ frt_status launch_dt(int K, bool weighted, bool ln, int qm, const NormArgs& a, c
 
 }  // namespace
 
-// Chunks per thread (K) and threads per row (T) for a row of C 16-byte
-// chunks (D = 8C): K = 1 up to D = 1024, 2 up to 2048, 4 up to 16384 (128 to
-// 512 threads), 8 up to 32768.
-static void rmsnorm_shape(int C, int* K, int* T) {
-  const int k = C <= 128 ? 1 : C <= 256 ? 2 : C <= 2048 ? 4 : 8;
+// Chunks per thread (K) and threads per row (T) for M rows of C 16-byte
+// chunks (D = 8C).  Large batches (bandwidth-bound, many rows per SM): K = 1
+// up to D = 1024, 2 up to 2048, 4 up to 16384 (128 to 512 threads), 8 up to
+// 32768.  Small batches (fewer rows than 4 per SM: latency-bound), up to D =
+// 4096: one chunk per thread, which shortens each thread's serial part of the
+// row reduction.
+static void rmsnorm_shape(int M, int C, int* K, int* T) {
+  int k = C <= 128 ? 1 : C <= 256 ? 2 : C <= 2048 ? 4 : 8;
+  if (M < 4 * 148 && C <= 512) k = 1;
   const int per = (C + k - 1) / k;
   *K = k;
   *T = ((per + 31) / 32) * 32;
@@ -317,7 +327,7 @@ extern "C" frt_status frt_residual_rmsnorm_fp8(const void* x, const void* residu
   const int C = D / 8;
   const int NB = (D + 127) / 128;
   int K, T;
-  rmsnorm_shape(C, &K, &T);
+  rmsnorm_shape(M, C, &K, &T);
   const NormArgs a{x, residual_in, residual_out, weight, nullptr, out_fp8, static_scale, block_scales, M, C, NB, T,
                    eps};
   return dt == FRT_F16 ? launch_dt<FRT_F16>(K, weight != nullptr, false, qm, a, stream)
@@ -339,7 +349,7 @@ extern "C" frt_status frt_residual_rmsnorm_nvfp4(const void* x, const void* resi
   if (!nvfp4_args_ok(sf_layout, global_scale, out_fp4, out_sf, 4)) return FRT_ERR_INVALID_ARG;
   const int C = D / 8;
   int K, T;
-  rmsnorm_shape(C, &K, &T);
+  rmsnorm_shape(M, C, &K, &T);
   const int qm = sf_layout == FRT_SF_ROW_MAJOR ? kQuantNvfp4Rows : kQuantNvfp4Swizzled;
   float* sf = reinterpret_cast<float*>(out_sf);  // the kernel's scale pointer carries the sf bytes
   const NormArgs a{x, residual_in, residual_out, weight, nullptr, out_fp4, global_scale, sf, M, C, 0, T, eps};
@@ -359,7 +369,7 @@ frt_status layernorm_op(const void* x, const void* residual_in, void* residual_o
   if ((weight && !aligned(weight, 16)) || (bias && !aligned(bias, 16))) return FRT_ERR_INVALID_ARG;
   const int C = D / 8;
   int K, T;
-  rmsnorm_shape(C, &K, &T);
+  rmsnorm_shape(M, C, &K, &T);
   const NormArgs a{x, residual_in, residual_out, weight, bias, out, scale, scales_out, M, C, (D + 127) / 128, T,
                    eps};
   return dt == FRT_F16 ? launch_dt<FRT_F16>(K, weight != nullptr, true, qm, a, stream)

@@ -28,6 +28,20 @@ def test_library_loads_and_exports_every_declared_symbol():
         assert hasattr(L, n), n
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """libfrt_debug.so (the bounds-checked build) exports frt.h's entry points
+    and the one include/frt_debug.h adds, which rejects a NULL count on the
+    host."""
+    src = open(os.path.join(ROOT, "include", "frt_debug.h")).read()
+    extra = sorted(set(re.findall(r"\b(frt_[a-z0-9_]+)\s*\(", re.sub(r"/\*.*?\*/", "", src, flags=re.S))))
+    assert extra == ["frt_debug_bounds_violations"]
+    D = frt.load_debug()
+    for n in declared_functions() + extra:
+        assert hasattr(D, n), n
+    assert not hasattr(frt.load(), "frt_debug_bounds_violations")
+    assert D.frt_debug_bounds_violations(None) == INV
+
+
 def test_status_strings():
     for s in (OK, INV, UNSUP, frt.FRT_ERR_CUDA, 99):
         assert isinstance(frt.status_string(s), str) and frt.status_string(s)
@@ -108,6 +122,12 @@ def test_pdl_switch():
         assert frt.frt_get_pdl() is True
     finally:
         frt.frt_set_pdl(prev)
+
+
+@pytest.mark.parametrize("args,want", [((A, A, -1, 32), INV), ((A, A, 2, 0), INV), ((A, A, 2, 24), INV),
+                                       ((A + 8, A, 2, 32), INV), ((None, A, 2, 32), INV), ((None, None, 0, 32), OK)])
+def test_copy_rows_host_validation(args, want):
+    assert frt.load().frt_copy_rows(*args, None) == want
 
 
 def test_wait_polls_setting():
