@@ -890,12 +890,15 @@ def _oracle_op(wl, host, op, rows):
 
 
 def _oracle_op_worker(task):
-    """One process of the all-cores column: its own seeded rows, one op."""
+    """One process of the all-cores column: its own seeded rows, one op (a
+    first untimed call on one row loads the oracle library)."""
     import dataclasses
     from memory_bound_non_b200 import workloads as W
     wl, op, rows = task
     small = dataclasses.replace(wl, M=rows)
-    return _oracle_op(small, W.make_inputs(small, n_layers=1), op, rows)
+    host = W.make_inputs(small, n_layers=1)
+    _oracle_op(small, host, op, 1)
+    return _oracle_op(small, host, op, rows)
 
 
 def baseline_table(peak, reps=20, max_cores=32, sample_s=1.0):
