@@ -382,6 +382,10 @@ frt_status frt_qkv_norm_rope_prepq_kvcache(const void* qkv, const void* q_norm_w
  *   y[i,j]  = h[i,j] * rstd_i * (1 + scale[c,j]) + shift[c,j],
  *             rstd_i = 1 / sqrt(mean_j(h[i,j]^2) + eps).
  *   out_fp8 = e4m3 of y / s (quant mode as in op (a); block scales over D).
+ *             Without scale and shift the arithmetic is op (a)'s (y and the
+ *             quotient correctly rounded in fp32); with them y carries a few
+ *             fp32 roundings and y / s is a product with 1 / s (folded into
+ *             rstd and the shift for a static scale).
  *
  *   x, residual_in, residual_out  device [M, D] 16-bit, 16-byte aligned;
  *                                 residual_out may equal residual_in.

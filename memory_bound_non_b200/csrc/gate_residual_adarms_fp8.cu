@@ -22,7 +22,10 @@
 // definition itself.  Without modulation the sum of squares is fp64 and
 // y = h * rstd is the correctly rounded fp32 value, as in op (a); with
 // modulation y carries three fp32 roundings anyway and an fp32 sum of squares
-// suffices.  FP8 codes are those of the correctly rounded quotient y / s.
+// suffices.  Without modulation the FP8 codes are those of the correctly
+// rounded quotient y / s; with it the division is a product (a static scale
+// folded into rstd and the shift, block-128 scales through RN(1 / s_b)), one
+// more fp32 rounding on top of y's.
 #include <atomic>
 #include <cmath>
 #include <type_traits>
@@ -158,6 +161,12 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
   const Split32 rstd(MOD ? 0.0 : rsqrt_f64(tot / (double)D + (double)eps));
   const float rstd32 = MOD ? rsqrtf((float)tot / D + eps) : 0.0f;
   const Divisor dv_static(QM == FRT_QUANT_STATIC ? s_static : 1.0f);
+  // Modulated rows carry a few fp32 roundings anyway, so a static scale is
+  // folded in (rstd / s and shift / s: y / s in one pass, no divide) when s
+  // lies in [2^-100, 2^100]; block-128 scales divide through RN(1 / s_b).
+  const bool mfold = MOD && QM == FRT_QUANT_STATIC && dv_static.fast;
+  const float mrs = mfold ? rstd32 * dv_static.inv : rstd32;
+  const float msh = mfold ? dv_static.inv : 1.0f;
   if (MOD) cp_async_wait<0>();
 
   // Pass 2: y and its FP8 codes.
@@ -180,8 +189,8 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
         const float2 hf = P16::to_float2(hw[e]);
         const float2 sc = P16::to_float2(scw[e]);
         const float2 sh = P16::to_float2(shw[e]);
-        y[2 * e] = fmaf(hf.x * rstd32, 1.0f + sc.x, sh.x);
-        y[2 * e + 1] = fmaf(hf.y * rstd32, 1.0f + sc.y, sh.y);
+        y[2 * e] = fmaf(hf.x * mrs, 1.0f + sc.x, sh.x * msh);
+        y[2 * e + 1] = fmaf(hf.y * mrs, 1.0f + sc.y, sh.y * msh);
       }
     } else {
 #pragma unroll
@@ -197,9 +206,19 @@ __global__ void __launch_bounds__(max_threads<K>()) gate_residual_adarms_fp8_ker
       const float sb = block_scale_448(am);
       if (valid && (t & 15) == 0 && FRT_IDX_OK(row * NB + (c >> 4), (int64_t)gridDim.x * NB))
         block_scales[row * NB + (c >> 4)] = sb;
-      if (valid && FRT_IDX_OK(base + c, n_rc)) q[base + c] = quant8(y, Divisor(sb));
+      if (valid && FRT_IDX_OK(base + c, n_rc)) {
+        if (MOD && sb >= 0x1p-100f && sb <= 0x1p+100f) {
+          const float r = __frcp_rn(sb);
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = y[e] * r;
+          q[base + c] = e4m3x8(v);
+        } else {
+          q[base + c] = quant8(y, Divisor(sb));
+        }
+      }
     } else if (valid && FRT_IDX_OK(base + c, n_rc)) {
-      q[base + c] = quant8(y, dv_static);
+      q[base + c] = mfold ? e4m3x8(y) : quant8(y, dv_static);
     }
   }
 }
