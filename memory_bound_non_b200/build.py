@@ -84,7 +84,11 @@ def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False
 
 
 def build_all(force: bool = False, verbose: bool = False):
-    return build(force, verbose), build(force, verbose, debug_bounds=True)
+    """Both libraries, built side by side (their objects are independent)."""
+    with concurrent.futures.ThreadPoolExecutor(max_workers=2) as pool:
+        release = pool.submit(build, force, verbose)
+        debug = pool.submit(build, force, verbose, True)
+        return release.result(), debug.result()
 
 
 if __name__ == "__main__":
