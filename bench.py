@@ -231,30 +231,54 @@ class ClockSampler:
                 "power_w_max": max((num(r[3]) or 0) for r in rows)}
 
 
-def kernel_source_hash():
-    """sha256 over the CUDA sources: ties a recorded ncu traffic figure to the
-    kernels it was measured on."""
+# Sources a traffic record depends on: the kernel's own file and the shared
+# device and host headers.
+SHARED_SOURCES = ("frt_device.cuh", "frt_host.h")
+KERNEL_SOURCE = {"attn_norm": "residual_rmsnorm_fp8.cu", "ffn_norm": "residual_rmsnorm_fp8.cu",
+                 "qkv": "qkv_norm_rope_kvcache.cu", "gate": "gate_act_fp8.cu",
+                 "gate_residual_adarms": "gate_residual_adarms_fp8.cu", "qkv_prepq": "qkv_norm_rope_kvcache.cu",
+                 "residual_rmsnorm_nvfp4": "residual_rmsnorm_fp8.cu", "gate_act_nvfp4": "gate_act_fp8.cu",
+                 "residual_layernorm": "residual_rmsnorm_fp8.cu", "qkv_layernorm": "qkv_norm_rope_kvcache.cu"}
+
+
+def source_hashes():
+    """sha256 of each CUDA source file: ties a recorded ncu traffic figure to
+    the kernel it was measured on."""
     import glob
     import hashlib
-    h = hashlib.sha256()
+    out = {}
     csrc = os.path.join(ROOT, "memory_bound_non_b200", "csrc")
     for path in sorted(glob.glob(os.path.join(csrc, "*"))):
         if path.endswith((".cu", ".cuh", ".h")):
             with open(path, "rb") as f:
-                h.update(os.path.basename(path).encode() + b"\0" + f.read())
-    return h.hexdigest()
+                out[os.path.basename(path)] = hashlib.sha256(f.read()).hexdigest()
+    return out
+
+
+def _traffic_sources(workload, op):
+    """The source files behind one traffic record: `op` names the kernel for
+    the step's ops, the workload key does for the widened ops."""
+    kernel = KERNEL_SOURCE.get(op)
+    for prefix in ("gate_residual_adarms", "qkv_prepq", "residual_rmsnorm_nvfp4", "gate_act_nvfp4",
+                   "residual_layernorm", "qkv_layernorm"):
+        if workload.startswith(prefix):
+            kernel = KERNEL_SOURCE[prefix]
+    return (kernel,) + SHARED_SOURCES if kernel else None
 
 
 def measured_traffic(workload, op):
     """DRAM bytes per launch (read + write) of `op` on `workload` from the
-    committed ncu record, or None when the kernels changed since."""
+    committed ncu record, or None when its kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    if rec.get("kernel_source_sha256") != kernel_source_hash():
+    files = _traffic_sources(workload, op)
+    recorded = rec.get("source_sha256", {})
+    now = source_hashes()
+    if files is None or any(recorded.get(f) is None or recorded.get(f) != now.get(f) for f in files):
         return None
     v = rec.get("per_launch_bytes", {}).get(workload, {}).get(op)
     return int(v) if v is not None else None
