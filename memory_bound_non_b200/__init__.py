@@ -11,7 +11,12 @@ Functions carry the C names of ``include/frt.h``:
     frt_gate_act_fp8(gate_up, out_fp8, ...)
     frt_qkv_norm_rope_prepq_kvcache(...)   (NEXT-2)
     frt_gate_residual_adarms_fp8(...)      (NEXT-1)
-    frt_noop(grid, block)
+    frt_noop(grid, block), frt_copy_rows(src, dst)      (launch-floor probes)
+    frt_set_pdl / frt_get_pdl, frt_set_wait_polls / frt_get_wait_polls
+
+``load_debug()`` opens the bounds-checked build (libfrt_debug.so,
+include/frt_debug.h); ``using_library(load_debug())`` routes these functions
+through it and ``bounds_violations()`` reads and clears its counter.
 """
 import contextlib
 import ctypes
