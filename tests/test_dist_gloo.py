@@ -98,3 +98,33 @@ def test_parity_helpers_count_code_steps_and_16bit_tolerance():
     o = np.array([1.0, -3.0, 1e-3])
     assert bench._rel_16bit_ok(o.astype(np.float32), o, "bf16")
     assert not bench._rel_16bit_ok((o * 1.02).astype(np.float32), o, "bf16")
+
+
+def test_traffic_records_follow_their_own_kernel_source(tmp_path, monkeypatch):
+    """A DRAM-traffic record is used only while its kernel's source file and
+    the shared headers keep the sha256 recorded with it: editing another
+    kernel's file leaves it valid, editing its own voids it."""
+    import json
+    import bench
+    now = bench.source_hashes()
+    rec = {"source_sha256": dict(now),
+           "per_launch_bytes": {"large_m_M65536": {"gate": 123, "attn_norm": 456},
+                                "qkv_prepq_e4m3_M65536": {"qkv_prepq": 789}}}
+    root = tmp_path
+    (root / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    monkeypatch.setattr(bench, "source_hashes", lambda: now)
+
+    def write(r):
+        (root / "profiles" / "traffic.json").write_text(json.dumps(r))
+    write(rec)
+    assert bench.measured_traffic("large_m_M65536", "gate") == 123
+    assert bench.measured_traffic("qkv_prepq_e4m3_M65536", "qkv_prepq") == 789
+    assert bench.measured_traffic("large_m_M65536", "qkv") is None          # no record
+    changed = dict(rec, source_sha256=dict(now, **{"residual_rmsnorm_fp8.cu": "0" * 64}))
+    write(changed)
+    assert bench.measured_traffic("large_m_M65536", "attn_norm") is None    # its own file changed
+    assert bench.measured_traffic("large_m_M65536", "gate") == 123         # another kernel's file
+    shared = dict(rec, source_sha256=dict(now, **{"frt_device.cuh": "0" * 64}))
+    write(shared)
+    assert bench.measured_traffic("large_m_M65536", "gate") is None        # a shared header changed
