@@ -47,6 +47,8 @@ A_CASES = [
     ("pi05", {"M": 5, "D": 1032, "quant": "block128"}), ("tiny", {"M": 2, "D": 8192, "dt": "bf16"}),
     ("vit", {"M": 3, "D": 16384, "quant": "block128"}), ("vit", {"M": 2, "D": 32768, "quant": "block128"}),
     ("pi05", {"M": 7, "D": 2056}), ("tiny", {"M": 9, "D": 4104, "quant": "block128", "weighted": False}),
+    # small batches run one chunk per thread up to D = 4096 (512 threads a row)
+    ("large_m_M4096", {"M": 100}), ("large_m_M4096", {"M": 591, "quant": "block128"}),
 ]
 
 
