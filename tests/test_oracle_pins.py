@@ -406,9 +406,10 @@ def test_bruteforce_op_a(dt, weighted, quant):
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 @pytest.mark.parametrize("qk_norm", [True, False])
-def test_bruteforce_op_b(dt, qk_norm):
-    g = W.generator(22)
-    Hq, Hkv, hd, M = 2, 1, 8, 4
+@pytest.mark.parametrize("hd", [8, 6, 2])   # hd / 2 odd for 6 and 2: the rotation pairs j, j + hd/2 straddle
+def test_bruteforce_op_b(dt, qk_norm, hd):
+    g = W.generator(22 + hd)
+    Hq, Hkv, M = 2, 1, 4
     qkv = W.bits16(W.normal16((M, (Hq + 2 * Hkv) * hd), dt, g))
     qw = W.bits16(W.norm_weight(hd, dt, g)) if qk_norm else None
     kw = W.bits16(W.norm_weight(hd, dt, g)) if qk_norm else None
