@@ -225,10 +225,16 @@ frt_status frt_gate_act_fp8(const void* gate_up, uint8_t* out_fp8, const float* 
  *   residual    device [M, D] 16-bit, updated in place.
  *   scales      device fp32[3] (attention norm, FFN norm, activation), read
  *               with STATIC.
- *   status      as op (b), or NULL.
+ *   status      device int32[1] or NULL; bits set with an atomic OR, never
+ *               cleared: bit 0 as op (b) (a row's position out of range:
+ *               that row's QKV outputs are skipped); bit 2 a layer record
+ *               holds a pointer below its field's alignment (16 bytes for the
+ *               eight inputs, k_cache, v_cache and q_out, 8 for q8_attn and
+ *               q8_ffn, 4 for act8 and bs_*), checked in the kernel before
+ *               anything is read or written: the launch then writes nothing.
  *   Supported: D % 8 == 0 and D <= 8192, hd % 16 == 0 and 64 <= hd <= 256,
- *   I % 128 == 0 (else FRT_ERR_UNSUPPORTED); all pointers aligned as the
- *   per-op calls require (not re-checked per layer on the host).
+ *   I % 128 == 0 (else FRT_ERR_UNSUPPORTED).  residual, cos_tab and sin_tab
+ *   16-byte aligned, positions and scales 4-byte (checked on the host).
  *   Each row is run by a thread-block cluster of up to 8 CTAs, sized so that
  *   the clusters of all M rows fill the GPU: one runs the row's residual chain
  *   (the norms), the others split the heads and activation blocks and run

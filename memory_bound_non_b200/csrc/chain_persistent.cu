@@ -19,13 +19,23 @@
 // heads of op b and the 128-output blocks of op c between them and run
 // alongside (with S == 1 one CTA does everything in order).  Each CTA copies
 // the next layer invocation's input slices into a second shared-memory stage
-// (asynchronous copies) while the current one computes.  With real GEMMs
-// between the ops, rows would mix and a grid-wide step would be needed.  Each
-// op uses the arithmetic of its per-op kernel (packed 16-bit add, fp64 row sum
-// of squares, the same FP8 decision arithmetic, RoPE and activation
-// expressions), so the results equal the per-op launches bit for bit.
+// (16-byte asynchronous copies, spread evenly over all its threads) while the
+// current one computes.  With real GEMMs between the ops, rows would mix and a
+// grid-wide step would be needed.  Each op uses the arithmetic of its per-op
+// kernel (packed 16-bit add, fp64 row sum of squares, the same FP8 decision
+// arithmetic, RoPE and activation expressions), so the results equal the
+// per-op launches bit for bit.  A table pointer below its field's alignment
+// sets status bit 2 before anything is read or written.
+//
+// Staging forms measured at 10 and 41 tokens and not kept: the eight slices
+// as 1-D bulk copies (TMA) issued by one thread on an mbarrier (7-9 % slower:
+// one thread's eight issues sit on the critical path at the next barrier,
+// wherever they are placed), and the copies issued after the barrier so they
+// overlap the arithmetic (8-10 % slower: they queue beside the norms' shared
+// loads and shuffles).
 #include <atomic>
 #include <cmath>
+#include <cstddef>
 #include <cooperative_groups.h>
 
 #include "frt_device.cuh"
@@ -39,16 +49,18 @@ namespace cg = cooperative_groups;
 constexpr int kChainThreads = 256;
 constexpr int kChainWarps = kChainThreads / 32;
 
-// CTA-wide fp64 sum (warp butterfly, then the warp partials in order); the
-// trailing barrier lets the next call reuse `red`.
+// CTA-wide fp64 sum (warp butterfly, then the warp partials in order).  The
+// two norms of a layer use the two halves of a 2 * kChainWarps buffer, so a
+// call needs no trailing barrier: the next call on the same half comes after
+// the loop's barriers.
 __device__ __forceinline__ double block_sum(double v, double* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
   __syncthreads();
   double tot = 0.0;
+#pragma unroll
   for (int i = 0; i < kChainWarps; ++i) tot += red[i];
-  __syncthreads();
   return tot;
 }
 
@@ -63,7 +75,7 @@ struct Slice {
 template <int DT, int K, int QM>
 __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uint2* q, float* bs, const Divisor& dv,
                                            double inv_s64, uint4 (&hv)[K], int64_t row, const Slice& sl, int C,
-                                           int NB, float D, float eps, double* red, int64_t n_rows) {
+                                           int NB, float D, double invD, float eps, double* red, int64_t n_rows) {
   using P16 = Pack16<DT>;
   const int t = threadIdx.x;
   uint4 xv[K], wv[K];
@@ -96,8 +108,10 @@ __device__ __forceinline__ void chain_norm(const uint4* xs, const uint4* ws, uin
 #pragma unroll
   for (int k = 1; k < K; ++k) sst += ss[k];
   const double tot = block_sum(sst, red);
+  // the mean square (for a power-of-two D the product with 1 / D is exact)
+  const double ms = invD > 0.0 ? tot * invD : tot / (double)D;
   // static FP8: one product with rstd / s, as op a does
-  const double rstd64 = rsqrt_f64(tot / (double)D + (double)eps);
+  const double rstd64 = rsqrt_f64(ms + (double)eps);
   const double rs64 = rstd64 * inv_s64;
   const bool fold = QM == FRT_QUANT_STATIC && rs64 >= 0x1p-100 && rs64 <= 0x1p+100;
   const Split32 rstd(fold ? rs64 : rstd64);
@@ -219,7 +233,9 @@ template <int DT, int QM, int ACT>
 __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* bs, const Divisor& dv, int64_t row,
                                           const Slice& sl, int I4, int NBI, int64_t n_rows) {
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
+  // blocks go to the warps from the last one down and heads (chain_qkv) to
+  // the threads from the first one up, so small slices of both overlap
+  const int warp = kChainWarps - 1 - (threadIdx.x >> 5);
   uint32_t* dst = q + row * I4;
   for (int i0 = warp * 4; i0 < sl.nb; i0 += kChainWarps * 4) {
     uint4 v[4];
@@ -252,7 +268,9 @@ __device__ __forceinline__ void chain_act(const uint4* gs, uint32_t* q, float* b
 // 16-byte asynchronous global -> shared copy (L2 only) and its groups.
 __device__ __forceinline__ void cp_async16(uint4* smem, const void* gmem) {
   const uint32_t a = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(gmem) : "memory");
+  // no memory clobber: nothing reads the stage before cp_async_wait1 and the
+  // barrier after it, which order the copies for the compiler
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(gmem));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
@@ -267,25 +285,44 @@ struct StageMap {
         gu(4 * cs + heads16 + 2 * hd16), len(4 * cs + heads16 + 2 * hd16 + gu16) {}
 };
 
-// (n_src: the source buffer's 16-byte chunks, checked in the bounds-checked build)
-__device__ __forceinline__ void stage_copy(uint4* dst, const void* src, int64_t off, int n, int64_t n_src) {
-  if (src == nullptr) return;
-  const uint4* s = static_cast<const uint4*>(src) + off;
-  for (int i = threadIdx.x; i < n; i += kChainThreads)
-    if (FRT_IDX_OK(off + i, n_src)) cp_async16(dst + i, s + i);
+// A layer's eight stage sources are the first eight pointers of its table
+// entry, in StageMap order.
+static_assert(offsetof(frt_chain_layer, x_attn) == 0 && offsetof(frt_chain_layer, x_ffn) == 8 &&
+                  offsetof(frt_chain_layer, w_attn) == 16 && offsetof(frt_chain_layer, w_ffn) == 24 &&
+                  offsetof(frt_chain_layer, qkv) == 32 && offsetof(frt_chain_layer, q_norm_w) == 40 &&
+                  offsetof(frt_chain_layer, k_norm_w) == 48 && offsetof(frt_chain_layer, gate_up) == 56,
+              "stage sources lead the layer record");
+
+// Words of one frt_chain_layer record, and the alignment each pointer needs:
+// the eight staged inputs and the 16-byte stores (q_out, the caches) 16
+// bytes, the 8-byte code stores 8, the activation codes and the scales 4.
+constexpr int kLayerWords = (int)(sizeof(frt_chain_layer) / 8);
+static_assert(kLayerWords == 17, "frt_chain_layer holds 17 pointers");
+static_assert(offsetof(frt_chain_layer, k_cache) == 64 && offsetof(frt_chain_layer, q_out) == 80 &&
+                  offsetof(frt_chain_layer, q8_attn) == 88 && offsetof(frt_chain_layer, act8) == 104,
+              "frt_chain_layer field order");
+__device__ __forceinline__ uint64_t layer_field_align(int field) {
+  return field < 11 ? 16u : field < 13 ? 8u : 4u;
 }
 
-// Copies every input slice one layer invocation of this CTA reads.
-__device__ __forceinline__ void stage_layer(uint4* st, const StageMap& m, const frt_chain_layer& L, int64_t row,
-                                            const Slice& sl, int C, int qkv16, int hd16, int I4, int64_t n_rows) {
-  stage_copy(st + m.xa, L.x_attn, row * C + sl.c0, sl.nc, n_rows * C);
-  stage_copy(st + m.xf, L.x_ffn, row * C + sl.c0, sl.nc, n_rows * C);
-  stage_copy(st + m.wa, L.w_attn, sl.c0, sl.nc, C);
-  stage_copy(st + m.wf, L.w_ffn, sl.c0, sl.nc, C);
-  stage_copy(st + m.qkv, L.qkv, row * qkv16 + (int64_t)sl.h0 * hd16, sl.nh * hd16, n_rows * qkv16);
-  stage_copy(st + m.qw, L.q_norm_w, 0, hd16, hd16);
-  stage_copy(st + m.kw, L.k_norm_w, 0, hd16, hd16);
-  stage_copy(st + m.gu, L.gate_up, row * I4 + (int64_t)sl.b0 * 32, sl.nb * 32, n_rows * I4);
+// Where the chunks of one stage slice come from: stage chunk i of slice s is
+// chunk delta + i of that slice's source buffer (lim chunks long).
+struct SliceSrc {
+  int64_t delta, lim;
+};
+
+// Copies every input slice one layer invocation of this CTA reads.  The stage
+// is one run of m.len chunks (slices in StageMap order); each thread takes
+// every kChainThreads-th chunk, finds its slice by comparing against the slice
+// starts, and copies it from that layer's source pointer (src: the layer's
+// eight source pointers, null for an absent weight).
+__device__ __forceinline__ void stage_layer(uint4* st, const StageMap& m, const uint64_t* src, const SliceSrc* ss) {
+  for (int i = threadIdx.x; i < m.len; i += kChainThreads) {
+    const int s = (i >= m.xf) + (i >= m.wa) + (i >= m.wf) + (i >= m.qkv) + (i >= m.qw) + (i >= m.kw) + (i >= m.gu);
+    const uint64_t p = src[s];
+    const int64_t j = ss[s].delta + i;
+    if (p != 0 && FRT_IDX_OK(j, ss[s].lim)) cp_async16(st + i, reinterpret_cast<const uint4*>(p) + j);
+  }
 }
 
 template <int DT, int K, int QM, int GP, int ACT>
@@ -294,7 +331,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
     const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, const int32_t* __restrict__ positions,
     const float* __restrict__ scales, int32_t* status, int C, int NB, int Hq, int Hkv, int hd, int G, int I4,
     int NBI, int max_pos, int capacity, float eps) {
-  __shared__ double red[kChainWarps];
+  __shared__ double red[2 * kChainWarps];
   pdl_enter();
   cg::cluster_group cl = cg::this_cluster();
   const unsigned S = cl.num_blocks();
@@ -343,40 +380,70 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
   const double inv_ffn = QM == FRT_QUANT_STATIC ? 1.0 / (double)dv_ffn.s : 0.0;
   const Divisor dv_act(QM == FRT_QUANT_STATIC && scales_ok ? __ldg(scales + 2) : 1.0f);
   const float D = (float)(C * 8);
+  const double invD = (C * 8 & (C * 8 - 1)) == 0 ? 1.0 / (double)(C * 8) : 0.0;  // exact for powers of two
   const int qkv16 = H * hd / 8, hd16 = hd / 8;
-  // this CTA's stage layout: only the slices of its own roles (the host sizes
-  // shared memory for the larger of the two layouts)
-  const StageMap m(norm_cta ? C : 0, bc_cta ? hs * hd16 : 0, hd16, bc_cta ? bsl * 32 : 0);
+  // this CTA's stage layout: exactly the slices of its own roles (the last
+  // worker's head and block slices can be shorter than hs and bsl; the host
+  // sizes shared memory for the largest layout, so this one always fits).
+  // Every chunk of the layout is copied, so it must not reach past a slice.
+  const StageMap m(sl.nc, sl.nh * hd16, hd16, sl.nb * 32);
 
   // dynamic shared memory: the layer table (so no iteration waits on a global
   // load of its pointers), then the two stages
   extern __shared__ uint4 smem[];
+  __shared__ SliceSrc ssrc[8];
   frt_chain_layer* tab = reinterpret_cast<frt_chain_layer*>(smem);
   uint4* stages = smem + (n_layers * (int)sizeof(frt_chain_layer) + 15) / 16;
   {
     const uint64_t* src = reinterpret_cast<const uint64_t*>(layers);
     uint64_t* dst = reinterpret_cast<uint64_t*>(tab);
     const int words = n_layers * (int)(sizeof(frt_chain_layer) / 8);
+    bool misaligned = false;
     for (int i = t; i < words; i += kChainThreads)
-      if (FRT_IDX_OK(i, words)) dst[i] = __ldg(src + i);
-    __syncthreads();
+      if (FRT_IDX_OK(i, words)) {
+        const uint64_t w = __ldg(src + i);
+        dst[i] = w;
+        misaligned |= (w & (layer_field_align(i % kLayerWords) - 1)) != 0;
+      }
+    if (t < 8) {  // slice t of this CTA's stage: where its chunks come from
+      int b;
+      int64_t o, l;
+      switch (t) {
+        case 0: b = m.xa; o = row * C + sl.c0; l = n_rows * C; break;
+        case 1: b = m.xf; o = row * C + sl.c0; l = n_rows * C; break;
+        case 2: b = m.wa; o = sl.c0; l = C; break;
+        case 3: b = m.wf; o = sl.c0; l = C; break;
+        case 4: b = m.qkv; o = row * qkv16 + (int64_t)sl.h0 * hd16; l = n_rows * qkv16; break;
+        case 5: b = m.qw; o = 0; l = hd16; break;
+        case 6: b = m.kw; o = 0; l = hd16; break;
+        default: b = m.gu; o = row * I4 + (int64_t)sl.b0 * 32; l = n_rows * I4; break;
+      }
+      ssrc[t].delta = o - b;
+      ssrc[t].lim = l;
+    }
+    // a table pointer below its field's alignment: report it and touch none
+    if (__syncthreads_or(misaligned)) {
+      if (t == 0 && r == 0 && status != nullptr) atomicOr(status, 4);
+      return;
+    }
   }
   const int total = steps * n_layers;
   if (total > 0) {
-    stage_layer(stages, m, tab[0], row, sl, C, qkv16, hd16, I4, n_rows);
+    stage_layer(stages, m, reinterpret_cast<const uint64_t*>(tab), ssrc);
     cp_async_commit();
   }
   for (int it = 0; it < total; ++it) {
     const frt_chain_layer& L = tab[it % n_layers];
     if (it + 1 < total)
-      stage_layer(stages + ((it + 1) & 1) * m.len, m, tab[(it + 1) % n_layers], row, sl, C, qkv16, hd16, I4, n_rows);
+      stage_layer(stages + ((it + 1) & 1) * m.len, m, reinterpret_cast<const uint64_t*>(tab + (it + 1) % n_layers),
+                  ssrc);
     cp_async_commit();  // possibly empty: one group per iteration
     cp_async_wait1();   // this iteration's stage has landed (only the newest group may be pending)
     __syncthreads();    // ... for every thread's copies
     const uint4* st = stages + (it & 1) * m.len;
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xa, L.w_attn != nullptr ? st + m.wa : nullptr,
-                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, inv_attn, hv, row, sl, C, NB, D, eps, red,
+                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, inv_attn, hv, row, sl, C, NB, D, invD, eps, red,
                             n_rows);
     chain_qkv<DT, GP>(reinterpret_cast<const uint16_t*>(st + m.qkv),
                       L.q_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.qw) : nullptr,
@@ -386,7 +453,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
                       n_rows, capacity);
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xf, L.w_ffn != nullptr ? st + m.wf : nullptr, reinterpret_cast<uint2*>(L.q8_ffn),
-                            L.bs_ffn, dv_ffn, inv_ffn, hv, row, sl, C, NB, D, eps, red, n_rows);
+                            L.bs_ffn, dv_ffn, inv_ffn, hv, row, sl, C, NB, D, invD, eps, red + kChainWarps, n_rows);
     chain_act<DT, QM, ACT>(st + m.gu, reinterpret_cast<uint32_t*>(L.act8), L.bs_act, dv_act, row, sl, I4, NBI,
                            n_rows);
     __syncthreads();  // the stage read here is refilled at iteration it + 2

@@ -136,3 +136,32 @@ def test_persistent_chain_equals_graphed_chain_bitwise(name):
     assert torch.equal(bits(chain.residual), bits(r_ref))
     got = [t for L in chain.layers for t in (L.q8_attn, L.q8_ffn, L.act8, L.q_out, L.k_cache, L.v_cache)]
     assert all(torch.equal(bits(a), bits(b)) for a, b in zip(ref, got))
+
+
+@pytest.mark.parametrize("field,offset", [("x_attn", 2), ("q8_attn", 4), ("act8", 2), ("k_cache", 8)])
+def test_persistent_chain_misaligned_table_pointer_sets_bit2_and_writes_nothing(field, offset):
+    """A layer record whose pointer sits below its field's alignment (16 bytes
+    for the staged inputs and the caches, 8 for the norm codes, 4 for the
+    activation codes) is caught in the kernel before anything is read through
+    the table: status bit 2, and every output keeps its contents."""
+    wl = W.get("pi05", layers=3, steps=1)
+    inp = W.make_inputs(wl)
+    chain = LayerChain(wl, inp, scales=P.chain_scales(wl, inp))
+    chain.reset()
+    L = chain.layers[1]
+    t = getattr(L, field)
+    nbytes = t.numel() * t.element_size()
+    raw = torch.zeros(nbytes + 16, dtype=torch.uint8, device=t.device)
+    raw[offset:offset + nbytes].copy_(t.reshape(-1).view(torch.uint8))
+    setattr(L, field, raw[offset:offset + nbytes].view(t.dtype).view(t.shape))
+    assert getattr(L, field).data_ptr() % 16 == offset
+    before = [x.clone() for x in [chain.residual] + [getattr(Y, n) for Y in chain.layers
+                                                     for n in ("q8_attn", "q8_ffn", "act8", "q_out", "k_cache",
+                                                               "v_cache")]]
+    chain.run_persistent()
+    torch.cuda.synchronize()
+    assert int(chain.status.item()) == 4
+    after = [chain.residual] + [getattr(Y, n) for Y in chain.layers
+                                for n in ("q8_attn", "q8_ffn", "act8", "q_out", "k_cache", "v_cache")]
+    bits = lambda x: x.view(torch.uint8)
+    assert all(torch.equal(bits(a), bits(b)) for a, b in zip(before, after))
