@@ -401,9 +401,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
     bool misaligned = false;
     for (int i = t; i < words; i += kChainThreads)
       if (FRT_IDX_OK(i, words)) {
-        const uint64_t w = __ldg(src + i);
-        dst[i] = w;
-        misaligned |= (w & (layer_field_align(i % kLayerWords) - 1)) != 0;
+        const uint64_t word = __ldg(src + i);
+        dst[i] = word;
+        misaligned |= (word & (layer_field_align(i % kLayerWords) - 1)) != 0;
       }
     if (t < 8) {  // slice t of this CTA's stage: where its chunks come from
       int b;
@@ -443,8 +443,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
     const uint4* st = stages + (it & 1) * m.len;
     if (norm_cta)
       chain_norm<DT, K, QM>(st + m.xa, L.w_attn != nullptr ? st + m.wa : nullptr,
-                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, inv_attn, hv, row, sl, C, NB, D, invD, eps, red,
-                            n_rows);
+                            reinterpret_cast<uint2*>(L.q8_attn), L.bs_attn, dv_attn, inv_attn, hv, row, sl, C, NB, D,
+                            invD, eps, red, n_rows);
     chain_qkv<DT, GP>(reinterpret_cast<const uint16_t*>(st + m.qkv),
                       L.q_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.qw) : nullptr,
                       L.k_norm_w != nullptr ? reinterpret_cast<const uint16_t*>(st + m.kw) : nullptr,
@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_persistent_kernel(
                             L.bs_ffn, dv_ffn, inv_ffn, hv, row, sl, C, NB, D, invD, eps, red + kChainWarps, n_rows);
     chain_act<DT, QM, ACT>(st + m.gu, reinterpret_cast<uint32_t*>(L.act8), L.bs_act, dv_act, row, sl, I4, NBI,
                            n_rows);
-    __syncthreads();  // the stage read here is refilled at iteration it + 2
+    __syncthreads();  // the slot read here is refilled (for it + 2) at the top of it + 1
   }
 #pragma unroll
   for (int k = 0; k < K; ++k) {
