@@ -277,7 +277,9 @@ def chain_layer_table(layers, device):
 def frt_chain_persistent(table, n_layers, steps, residual, cos_tab, sin_tab, positions, scales, status, Hq, Hkv,
                          hd, I, capacity, eps=1e-6, quant="static", act="gelu_tanh", stream=None):
     """NEXT-4: steps x layers x (norm, QKV, norm, gate) as one kernel launch;
-    table from chain_layer_table."""
+    table from chain_layer_table.  status (int32[1]) gets bit 0 for a row
+    whose position is out of range and bit 2 when a layer record holds a
+    pointer below its field's alignment (then nothing is written)."""
     M, D = residual.shape
     st = load().frt_chain_persistent(
         _ptr(table), n_layers, steps, _ptr(residual), _ptr(cos_tab), _ptr(sin_tab), _ptr(positions), _ptr(scales),
